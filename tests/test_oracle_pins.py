@@ -1,0 +1,417 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Nothing here compares the oracle with itself: each check uses a value the
+pages print, a closed form, brute force, an independent library routine or
+an invariant.  ``test_planted_mistakes_are_caught`` plants plausible bugs in
+the oracle (on the CPU) and shows that one of these pins fails for each.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import moe_oracle as om
+from mixture_experts_routing_02_b200 import synthetic as syn
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_golden(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, val = line.split(":", 1)
+            out[key.strip()] = val.split()
+    return out
+
+
+# --------------------------------------------------------------------------- pins as functions
+# (returning True when the pin holds, so the planted-mistake test can reuse them)
+
+def pin_worked_example():
+    g = _read_golden("worked_top2.txt")
+    logits = np.array([[float(v) for v in g["logits"]]])
+    k = int(g["k"][0])
+    ids = oracle.topk_ids(logits, k)
+    w = oracle.topk_weights(logits, ids)
+    ok = list(ids[0]) == [int(v) for v in g["ids"]]
+    ok &= np.allclose(np.round(w[0], 3), [float(v) for v in g["weights_3dp"]], atol=0, rtol=0)
+    closed = math.exp(0.4) / (1 + math.exp(0.4))
+    ok &= abs(w[0, 0] - closed) < 1e-12 and abs(w[0, 1] - (1 - closed)) < 1e-12
+    return bool(ok)
+
+
+def pin_topk_brute_force(seed=0, T=40, E=7):
+    rng = np.random.default_rng(seed)
+    logits = rng.normal(size=(T, E))
+    for k in range(1, E + 1):
+        ids = oracle.topk_ids(logits, k)
+        for t in range(T):
+            l32 = logits[t].astype(np.float32).astype(np.float64)
+            best = max(itertools.combinations(range(E), k), key=lambda s: sum(l32[list(s)]))
+            want = sorted(best, key=lambda e: -l32[e])
+            if list(ids[t]) != want:
+                return False
+    return True
+
+
+def pin_weights_full_softmax(seed=1, T=50, E=16, k=4):
+    rng = np.random.default_rng(seed)
+    logits = rng.normal(scale=3.0, size=(T, E))
+    ids = oracle.topk_ids(logits, k)
+    w = oracle.topk_weights(logits, ids)
+    p = torch.softmax(torch.from_numpy(logits), dim=1).numpy()
+    sel = np.take_along_axis(p, ids, axis=1)
+    ref = sel / sel.sum(axis=1, keepdims=True)
+    return bool(np.allclose(w, ref, rtol=1e-12, atol=1e-15)
+                and np.allclose(w.sum(1), 1.0, atol=1e-14)
+                and (np.diff(w, axis=1) <= 0).all())
+
+
+def pin_router_logits_library(seed=2):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(37, 96, generator=g).to(torch.bfloat16)
+    wr = (torch.randn(11, 96, generator=g) * 0.02).to(torch.bfloat16)
+    b = torch.randn(11, generator=g)
+    ref = torch.nn.functional.linear(x.double(), wr.double(), b.double()).numpy()
+    return bool(np.allclose(oracle.router_logits(x, wr, b), ref, rtol=1e-13, atol=1e-13))
+
+
+def pin_histogram_bincount(seed=3, T=300, E=13, k=3):
+    ids = syn.lognormal_topk_ids(E, T, k, 1.0, seed=seed).numpy()
+    c = oracle.histogram(ids, E)
+    return bool(c.sum() == T * k and (c == np.bincount(ids.ravel(), minlength=E)).all())
+
+
+def pin_rank_stable_sort(seed=4, T=200, E=9, k=3):
+    ids = syn.lognormal_topk_ids(E, T, k, 1.5, seed=seed).numpy()
+    flat = ids.ravel()
+    rank = oracle.expert_rank(ids, E)
+    order = np.argsort(flat, kind="stable")
+    first = np.searchsorted(flat[order], np.arange(E))
+    want = np.empty_like(rank)
+    want[order] = np.arange(flat.size) - first[flat[order]]
+    return bool((rank == want).all())
+
+
+def _small_layer(seed, T=24, d=64, E=6, k=2, F=64, zipf=0.0):
+    w = syn.Workload("pin", T=T, d=d, E=E, k=k, F=F, zipf_s=zipf)
+    x, wr, b = syn.router_inputs(w, seed)
+    oracle.enforce_margin(x, wr, b, k, lambda t, a: syn.x_row_redraw(w, seed, t, a))
+    wg, wu, wd = syn.expert_weights(w, seed)
+    return x, wr, b, wg, wu, wd
+
+
+def pin_layer_equals_eager(seed=5, capacity=0):
+    """The dispatched layer equals a per-token, per-expert loop (the 'eager' backend)."""
+    T, E, k = 24, 6, 2
+    x, wr, b, wg, wu, wd = _small_layer(seed, T=T, E=E, k=k, zipf=1.2)
+    res = oracle.layer_forward(x, wr, b, wg, wu, wd, k, capacity=capacity)
+    x64 = oracle.f64(x)
+    logits = oracle.router_logits(x, wr, b)
+    seen = {}
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-np.float32(logits[t, e]), e))[:k]
+        sel = logits[t, order]
+        w = np.exp(sel - sel.max()); w /= w.sum()
+        keep = []
+        for e in order:
+            seen[e] = seen.get(e, 0) + 1
+            keep.append(capacity == 0 or seen[e] <= capacity)
+        want = oracle.token_output(x64[t], order, w, wg, wu, wd, keep=keep)
+        if not np.allclose(res.out[t], want, rtol=1e-11, atol=1e-13):
+            return False
+    return True
+
+
+def pin_dense_ffn_e1k1(seed=6):
+    """E = 1, k = 1 reduces to one dense SwiGLU FFN applied to every token."""
+    x, wr, b, wg, wu, wd = _small_layer(seed, T=17, E=1, k=1)
+    res = oracle.layer_forward(x, wr, b, wg, wu, wd, 1)
+    F_ = torch.nn.functional
+    xd = x.double()
+    ref = F_.linear(F_.silu(F_.linear(xd, wg[0].double())) * F_.linear(xd, wu[0].double()),
+                    wd[0].double()).numpy()
+    return bool(np.allclose(res.out, ref, rtol=1e-11, atol=1e-13))
+
+
+def pin_silu_library():
+    z = np.linspace(-30, 30, 2001)
+    ref = torch.nn.functional.silu(torch.from_numpy(z)).numpy()
+    return bool(np.allclose(oracle.silu(z), ref, rtol=1e-14, atol=1e-300) and oracle.silu(np.zeros(1))[0] == 0)
+
+
+def pin_dispatch_invariants(seed=7, capacity=0):
+    T, E, k = 50, 5, 2
+    ids = syn.lognormal_topk_ids(E, T, k, 1.0, seed=seed).numpy()
+    counts = oracle.histogram(ids, E)
+    segs = oracle.plain_segments(counts, capacity)
+    dest, src = oracle.dispatch_positions(ids, segs, E)
+    flat = ids.ravel()
+    kept = dest >= 0
+    rows = int(segs.offsets[-1])
+    ok = sorted(dest[kept].tolist()) == list(range(rows))
+    ok &= all(src[dest[q]] == q for q in np.nonzero(kept)[0])
+    off = segs.offsets
+    for e in range(E):
+        seg_src = src[off[e]:off[e + 1]]
+        ok &= bool((flat[seg_src] == e).all()) and bool((np.diff(seg_src) > 0).all())
+        want = min(counts[e], capacity) if capacity else counts[e]
+        ok &= (off[e + 1] - off[e]) == want
+    if capacity:
+        ok &= int((~kept).sum()) == int(np.maximum(counts - capacity, 0).sum())
+    else:
+        ok &= bool(kept.all())
+    return bool(ok)
+
+
+def _plan_check(ids, E, R, S, k, B):
+    counts = oracle.histogram(ids, E)
+    segs, stats = oracle.balanced_plan(counts, R, S, k, B)
+    dest, src = oracle.dispatch_positions(ids, segs, E)
+    flat = ids.ravel()
+    CAP = S * k
+    n_per_group = E // R + B
+    off = segs.offsets
+    ok = bool((dest >= 0).all()) and sorted(dest.tolist()) == list(range(R * CAP))
+    for g in range(R):
+        ok &= int(off[(g + 1) * n_per_group] - off[g * n_per_group]) == CAP
+    for s, e in enumerate(segs.expert):
+        rows = src[off[s]:off[s + 1]]
+        if e < 0:
+            ok &= len(rows) == 0
+        else:
+            ok &= bool((flat[rows] == e).all())
+    epg = E // R
+    seg_group = np.repeat(np.arange(R), n_per_group)
+    row_group = np.empty(R * CAP, dtype=np.int64)
+    for s in range(len(segs.expert)):
+        row_group[off[s]:off[s + 1]] = seg_group[s]
+    moved = int((row_group[dest] != flat // epg).sum())
+    loads = np.array([counts[g * epg:(g + 1) * epg].sum() for g in range(R)])
+    lower_bound = int(np.maximum(loads - CAP, 0).sum())
+    ok &= moved == lower_bound == stats.migrated_rows
+    return ok, stats, loads
+
+
+def pin_plan_moonep_table(sigmas=(0.5, 1.0, 2.0, 5.0)):
+    """E=256, R=8, S=2048, k=8 (the MoonEP page's experiment): every group gets exactly S*k."""
+    E, R, S, k, B = 256, 8, 2048, 8, 32
+    for sigma in sigmas:
+        ids = syn.lognormal_topk_ids(E, R * S, k, sigma, seed=11).numpy()
+        ok, stats, loads = _plan_check(ids, E, R, S, k, B)
+        if not ok:
+            return False
+    return True
+
+
+def pin_plan_uniform():
+    """Perfectly even routing needs no migration and no replica (sigma = 0 row)."""
+    E, R, S, k, B = 256, 8, 2048, 8, 32
+    ids = syn.uniform_roundrobin_ids(E, R * S, k).numpy()
+    ok, stats, loads = _plan_check(ids, E, R, S, k, B)
+    return ok and stats.migrated_rows == 0 and stats.replicas_used == 0 and (loads == S * k).all()
+
+
+def pin_plan_toy_skew():
+    """8 experts on 4 groups, top-1, 100 tokens, 70 on group 0's two experts, 10 on each other group.
+
+    Busiest group: 70 tokens = 7x the others and 2.8x the mean of 25; the
+    plan gives every group 25 rows and moves 45 of 100 rows.
+    """
+    ids = np.array([0] * 35 + [1] * 35 + [2] * 5 + [3] * 5 + [4] * 5 + [5] * 5 + [6] * 5 + [7] * 5)
+    ids = ids.reshape(100, 1)
+    ok, stats, loads = _plan_check(ids, E=8, R=4, S=25, k=1, B=4)
+    ok &= list(loads) == [70, 10, 10, 10] and loads.max() / loads.mean() == 2.8
+    ok &= loads.max() == 7 * loads[1:].max() and stats.migrated_rows == 45
+    return bool(ok)
+
+
+# --------------------------------------------------------------------------- the tests
+
+def test_worked_top2_example():
+    assert pin_worked_example()
+
+
+def test_topk_brute_force():
+    assert pin_topk_brute_force()
+
+
+def test_topk_ties_go_to_lower_id():
+    logits = np.array([[1.0, 3.0, 3.0, 2.0, 3.0]])
+    assert list(oracle.topk_ids(logits, 3)[0]) == [1, 2, 4]
+
+
+def test_topk_fp32_decision():
+    # 1e-9 apart in fp64 but equal in fp32: the decision is taken in fp32, so the lower id wins
+    logits = np.array([[1.0, 1.0 + 1e-9]])
+    assert list(oracle.topk_ids(logits, 1)[0]) == [0]
+
+
+def test_weights_equal_full_softmax_then_renorm():
+    assert pin_weights_full_softmax()
+
+
+def test_k1_weight_is_one():
+    logits = np.random.default_rng(0).normal(size=(20, 8))
+    w = oracle.topk_weights(logits, oracle.topk_ids(logits, 1))
+    assert (w == 1.0).all()
+
+
+def test_router_logits_match_library_linear():
+    assert pin_router_logits_library()
+
+
+def test_histogram():
+    assert pin_histogram_bincount()
+
+
+def test_rank_is_stable_sort_position():
+    assert pin_rank_stable_sort()
+
+
+def test_dispatch_invariants_no_capacity():
+    assert pin_dispatch_invariants(capacity=0)
+
+
+def test_dispatch_invariants_capacity():
+    assert pin_dispatch_invariants(capacity=14)
+
+
+def test_capacity_closed_form_skewed():
+    w = syn.SKEWED
+    assert oracle.capacity_rows(w.capacity_factor, w.T, w.k, w.E) == 320
+    assert oracle.capacity_rows(0.0, 10, 2, 4) == 0
+    assert oracle.capacity_rows(1.0, 10, 2, 4) == 5
+    assert oracle.capacity_rows(1.0, 10, 2, 3) == 7
+
+
+def test_silu():
+    assert pin_silu_library()
+
+
+def test_layer_equals_eager_loop():
+    assert pin_layer_equals_eager(capacity=0)
+
+
+def test_layer_equals_eager_loop_with_capacity():
+    assert pin_layer_equals_eager(capacity=5)
+
+
+def test_dense_ffn_e1_k1():
+    assert pin_dense_ffn_e1k1()
+
+
+def test_plan_moonep_experiment_invariants():
+    assert pin_plan_moonep_table()
+
+
+def test_plan_uniform_routing_moves_nothing():
+    assert pin_plan_uniform()
+
+
+def test_plan_toy_skew_example():
+    assert pin_plan_toy_skew()
+
+
+def test_plan_infeasible_raises():
+    ids = np.array([0] * 70 + [2] * 10 + [4] * 10 + [6] * 10).reshape(100, 1)
+    with pytest.raises(oracle.PlanInfeasible):
+        oracle.balanced_plan(oracle.histogram(ids, 8), 4, 25, 1, 0)
+
+
+def test_plan_segment_count():
+    assert oracle.num_segments(256, 8, 32) == 512
+    assert oracle.num_segments(64, 0, 0) == 64
+
+
+def test_margin_enforcement():
+    w = syn.Workload("m", T=400, d=64, E=16, k=4, F=64)
+    x, wr, b = syn.router_inputs(w, 3)
+    before = oracle.margin_violations(oracle.router_logits(x, wr, b), w.k, 1e-3).sum()
+    n = oracle.enforce_margin(x, wr, b, w.k, lambda t, a: syn.x_row_redraw(w, 3, t, a))
+    after = oracle.margin_violations(oracle.router_logits(x, wr, b), w.k, 1e-3).sum()
+    assert n == before and after == 0
+
+
+# --------------------------------------------------------------------------- planted mistakes
+
+def _mut_silu_sign(z):
+    return z / (1.0 + np.exp(z))
+
+
+def _mut_weights_no_renorm(logits64, ids):
+    p = np.exp(logits64 - logits64.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    return np.take_along_axis(p, ids, axis=1)
+
+
+def _mut_topk_ascending(logits64, k):
+    return np.argsort(np.asarray(logits64).astype(np.float32), axis=1, kind="stable")[:, :k]
+
+
+def _mut_histogram_offby1(ids, E):
+    c = np.bincount(np.asarray(ids).ravel(), minlength=E)
+    c[0] += 1
+    return c
+
+
+def _mut_rank_unstable(ids, E):
+    flat = np.asarray(ids).ravel()
+    rank = np.empty(flat.size, dtype=np.int64)
+    seen = np.zeros(E, dtype=np.int64)
+    for q in range(flat.size - 1, -1, -1):
+        rank[q] = seen[flat[q]]
+        seen[flat[q]] += 1
+    return rank
+
+
+_orig_expert_ffn = om.expert_ffn
+
+
+def _mut_down_transposed(x_rows64, w_gate_e, w_up_e, w_down_e):
+    wg, wu, wd = om.f64(w_gate_e), om.f64(w_up_e), om.f64(w_down_e)
+    h = om.silu(x_rows64 @ wg.T) * (x_rows64 @ wu.T)
+    return h, h @ wd   # wrong: W_down used untransposed
+
+
+def _mut_logits_no_bias(x, w_router, bias=None):
+    return om.f64(x) @ om.f64(w_router).T
+
+
+_orig_combine = om.combine
+
+
+def _mut_combine_unweighted(yp64, dest, weights64, T, k):
+    return _orig_combine(yp64, dest, np.ones_like(weights64), T, k)
+
+MUTATIONS = [
+    ("silu", _mut_silu_sign, [pin_silu_library, pin_dense_ffn_e1k1]),
+    ("topk_weights", _mut_weights_no_renorm, [pin_worked_example, pin_weights_full_softmax]),
+    ("topk_ids", _mut_topk_ascending, [pin_worked_example, pin_topk_brute_force]),
+    ("histogram", _mut_histogram_offby1, [pin_histogram_bincount]),
+    ("expert_rank", _mut_rank_unstable, [pin_rank_stable_sort, pin_dispatch_invariants]),
+    ("expert_ffn", _mut_down_transposed, [pin_dense_ffn_e1k1]),
+    ("router_logits", _mut_logits_no_bias, [pin_router_logits_library]),
+    ("combine", _mut_combine_unweighted, [pin_layer_equals_eager]),
+]
+
+
+@pytest.mark.parametrize("name,mutant,pins", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistakes_are_caught(monkeypatch, name, mutant, pins):
+    monkeypatch.setattr(om, name, mutant)
+    monkeypatch.setattr(oracle, name, mutant)
+    results = []
+    for pin in pins:
+        try:
+            results.append(pin())
+        except Exception:
+            results.append(False)
+    assert not all(results), f"planted mistake in {name} went unnoticed"
