@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the single-GPU top-k MoE FFN layer forward (B200).
+
+One step = one whole layer forward over one batch of T tokens through the C
+ABI: moe_route -> moe_dispatch -> moe_expert_gate_up -> moe_expert_down ->
+moe_combine (the calls moe_layer_fwd makes), with CUDA events between the
+calls so every kernel's duration is measured inside the timed region.  The
+default workload is the Mixtral-like layer (T=4096, d=4096, E=8, top-2,
+F=14336), random-init weights and seeded synthetic inputs.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an
+independent replica on its own GPU (the layer does not shard: replicas
+only); the value is all ranks' tokens over the slowest rank's device time.
+The reference arm (--impl reference) times the CPU fp64 oracle on a bounded
+sample of the same workload on the host cores (rank 0 only).
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd tokens/s; grouped-GEMM TFLOPS and permute GB/s vs roofline"
+FLUSH_BYTES = 256 << 20
+KERNELS = ("route", "dispatch", "gate_up", "down", "combine")
+LAUNCHES_PER_STEP = 7  # route, histogram, segments|plan, permute, gate_up, down, combine
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            entries = json.load(f)
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for fn in ("umma_gemm.cu", "common.cuh", "dispatch.cu", "combine.cu"):
+        with open(os.path.join(ROOT, "mixture_experts_routing_02_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    for e in entries:
+        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("source_sha256") == h.hexdigest():
+            return e.get("dram_bytes_per_launch")
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons of one GPU through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_device: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            props = torch.cuda.get_device_properties(torch_device)
+            handle = None
+            try:
+                bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+                handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = int(vis.split(",")[torch_device]) if vis and vis.split(",")[0].isdigit() else torch_device
+                handle = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._nv, self._h = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _reasons(self):
+        nv = self._nv
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(nv, fn):
+                return getattr(nv, fn)(self._h)
+        return 0
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                bits = self._reasons()
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.1)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _config(w, capacity):
+    return {"workload": w.name, "T": w.T, "d_model": w.d, "n_experts": w.E, "top_k": w.k, "d_ff": w.F,
+            "capacity": capacity, "n_groups": w.n_groups, "replica_slots": w.replica_slots,
+            "zipf_bias_s": w.zipf_s, "l2": "flushed between steps (256 MiB write outside the timed events)",
+            "parallelism": "replicas (no exchange between GPUs)"}
+
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+
+def _oracle_sample(w, seed: int, n_route: int, n_ffn: int, wg, wu, wd):
+    """Time the oracle on a bounded sample of the workload; returns (tokens/s, description)."""
+    import numpy as np
+    import torch
+    import oracle
+    from mixture_experts_routing_02_b200 import synthetic as syn
+
+    x, w_r, bias = syn.router_inputs(w.scaled(T=n_route), seed)
+    t0 = time.perf_counter()
+    logits, ids, wts = oracle.route(x, w_r, bias, w.k)
+    t1 = time.perf_counter()
+    counts = oracle.histogram(ids, w.E)
+    segs = oracle.plain_segments(counts, 0)
+    dest, src = oracle.dispatch_positions(ids, segs, w.E)
+    xp = oracle.permute_rows(x, src, w.k)
+    t2 = time.perf_counter()
+    _, y = oracle.expert_ffn(xp[:n_ffn], wg[0], wu[0], wd[0])
+    t3 = time.perf_counter()
+    yfull = np.zeros((xp.shape[0], w.d))
+    yfull[:n_ffn] = y
+    oracle.combine(yfull, dest, wts, n_route, w.k)
+    t4 = time.perf_counter()
+    per_token = (t1 - t0) / n_route + (t2 - t1) / n_route + w.k * (t3 - t2) / n_ffn + (t4 - t3) / n_route
+    desc = (f"routing, histogram, segments, dispatch positions and combine of {n_route} tokens; expert FFN "
+            f"(gate/up/down, fp64) of {n_ffn} rows of one expert; per-token cost = per-token routing+dispatch"
+            f"+combine + k x per-row FFN, extrapolated to tokens/s")
+    return 1.0 / per_token, desc, t4 - t0
+
+
+def _threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    capacity = _capacity(w)
+    n_route, n_ffn = 256, 8
+    from mixture_experts_routing_02_b200 import synthetic as syn
+    wg, wu, wd = syn.expert_weights(w, args.seed, experts=range(1))
+    for _ in range(args.warmup):
+        _oracle_sample(w, args.seed, n_route, n_ffn, wg, wu, wd)
+    vals, secs = [], []
+    desc = ""
+    for _ in range(args.steps):
+        v, desc, s = _oracle_sample(w, args.seed, n_route, n_ffn, wg, wu, wd)
+        vals.append(v)
+        secs.append(s)
+    value = statistics.mean(vals)
+    cores = _threads_used()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(secs),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; random-init weights)", "config": _config(w, capacity),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _capacity(w):
+    if w.capacity_factor <= 0:
+        return 0
+    return int(-(-(w.capacity_factor * w.T * w.k) // w.E))
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_routing_02_b200 as moe
+    from mixture_experts_routing_02_b200 import synthetic as syn
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    moe.load_library()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    capacity = _capacity(w)
+    s = moe.shape(w.T, w.d, w.E, w.k, w.F, capacity=capacity, n_groups=w.n_groups,
+                  replica_slots=w.replica_slots)
+    n_seg, rows_alloc = moe.moe_layout(s)
+    _, layer_bytes = moe.moe_workspace_size(s)
+
+    seed = args.seed + rank
+    x_cpu, w_r, bias = syn.router_inputs(w, seed)
+    x_host = x_cpu.pin_memory()
+    x = x_cpu.to(dev)
+    w_r = w_r.to(dev)
+    bias = bias.to(dev) if bias is not None else None
+    wg, wu, wd = syn.expert_weights(w, seed, device=dev)
+    ws = torch.empty(layer_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty(w.T, w.d, dtype=torch.bfloat16, device=dev)
+    out_host = torch.empty(w.T, w.d, dtype=torch.bfloat16).pin_memory()
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    v = moe.moe_layer_views(s, ws)
+
+    def view(addr, n, dtype):
+        off = addr - ws.data_ptr()
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return ws[off:off + nbytes].view(dtype)
+
+    ids = view(v.topk_ids, w.T * w.k, torch.int32)
+    wts = view(v.topk_w, w.T * w.k, torch.float32)
+    counts = view(v.counts, w.E, torch.int32)
+    seg_e = view(v.seg_expert, n_seg, torch.int32)
+    seg_o = view(v.seg_offsets, n_seg + 1, torch.int32)
+    seg_f = view(v.seg_first_rank, n_seg, torch.int32)
+    dest = view(v.dest, w.T * w.k, torch.int32)
+    src = view(v.src, rows_alloc, torch.int32)
+    xp = view(v.xp, rows_alloc * w.d, torch.bfloat16)
+    hp = view(v.hp, rows_alloc * w.F, torch.bfloat16)
+    yp = view(v.yp, rows_alloc * w.d, torch.bfloat16)
+    dws = view(v.dispatch_ws, v.dispatch_ws_bytes, torch.uint8)
+
+    def step(ev):
+        ev[0].record(stream)
+        moe.moe_route(s, x, w_r, bias, None, ids, wts, status, stream)
+        ev[1].record(stream)
+        moe.moe_dispatch(s, x, ids, 0, counts, seg_e, seg_o, seg_f, dest, src, xp, status, dws, stream)
+        ev[2].record(stream)
+        moe.moe_expert_gate_up(s, xp, seg_e, seg_o, wg, wu, hp, status, stream)
+        ev[3].record(stream)
+        moe.moe_expert_down(s, hp, seg_e, seg_o, wd, yp, status, stream)
+        ev[4].record(stream)
+        moe.moe_combine(s, yp, dest, wts, out, stream)
+        ev[5].record(stream)
+
+    def e2e_step(ev):
+        ev[0].record(stream)
+        x.copy_(x_host, non_blocking=True)
+        moe.moe_layer_fwd(s, x, w_r, bias, wg, wu, wd, out, status, ws, stream)
+        out_host.copy_(out, non_blocking=True)
+        ev[1].record(stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step([torch.cuda.Event(enable_timing=True) for _ in range(6)])
+    for _ in range(max(1, min(args.warmup, 3))):
+        flush.zero_()
+        e2e_step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    torch.cuda.synchronize()
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()} after warm-up")
+    rows_used = int(seg_o[-1].item())
+    active_experts = int((torch.bincount(seg_e[seg_o[1:] > seg_o[:-1]].long().clamp_min(0),
+                                         minlength=w.E) > 0).sum().item())
+
+    # timed region: K steps, events between every call
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            step(events[i])
+        barrier()
+    per_kernel = {k: [] for k in KERNELS}
+    step_ms = []
+    for ev in events:
+        step_ms.append(ev[0].elapsed_time(ev[5]))
+        for j, k in enumerate(KERNELS):
+            per_kernel[k].append(ev[j].elapsed_time(ev[j + 1]))
+    total_ms = sum(step_ms)
+
+    # end to end through moe_layer_fwd with host buffers
+    e2e_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_step(e2e_events[i])
+    barrier()
+    e2e_ms = sum(ev[0].elapsed_time(ev[1]) for ev in e2e_events)
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()}")
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    hbm, bf16, bf16_sus, peak_kind = _peaks()
+    avg = {k: statistics.mean(v) for k, v in per_kernel.items()}
+    T, d, E, k, F = w.T, w.d, w.E, w.k, w.F
+    breakdown = {}
+    breakdown["route"] = dict(ms=avg["route"], bytes=T * d * 2 + E * d * 2 + T * k * 8, flops=2 * T * d * E)
+    breakdown["dispatch"] = dict(ms=avg["dispatch"], bytes=T * d * 2 + rows_used * d * 2 + T * k * 4 * 3 + rows_used * 4)
+    breakdown["gate_up"] = dict(ms=avg["gate_up"], flops=4 * rows_used * d * F,
+                                bytes=2 * active_experts * F * d * 2 + rows_used * d * 2 + rows_used * F * 2)
+    breakdown["down"] = dict(ms=avg["down"], flops=2 * rows_used * d * F,
+                             bytes=active_experts * d * F * 2 + rows_used * F * 2 + rows_used * d * 2)
+    breakdown["combine"] = dict(ms=avg["combine"], bytes=rows_used * d * 2 + T * d * 2 + T * k * 8)
+    for name, b in breakdown.items():
+        sec = b["ms"] / 1e3
+        if "flops" in b and name in ("gate_up", "down"):
+            b["tflops"] = b["flops"] / sec / 1e12
+            b["frac_bf16_peak"] = b["tflops"] / bf16
+        b["gbs"] = b["bytes"] / sec / 1e9
+        b["frac_hbm_peak"] = b["gbs"] / hbm
+    dom = max(breakdown, key=lambda n: breakdown[n]["ms"])
+    db = breakdown[dom]
+    if dom in ("gate_up", "down"):
+        roof = {"bound": "tensor", "achieved": db["tflops"], "peak": bf16, "unit": "TFLOP/s",
+                "frac": db["tflops"] / bf16, "kernel": dom,
+                "peak_source": f"{peak_kind} bf16_tflops (burst); sustained {bf16_sus}"}
+    else:
+        roof = {"bound": "hbm", "achieved": db["gbs"], "peak": hbm, "unit": "GB/s", "frac": db["gbs"] / hbm,
+                "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs"}
+    traffic = _traffic(dom, w.name)
+    roof["traffic"] = traffic
+
+    tokens = T * args.steps * world
+    value = tokens / (total_ms / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init weights)", "config": _config(w, capacity),
+        "rows_dispatched": rows_used, "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "roofline": roof,
+        "breakdown": {n: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in b.items()}
+                      for n, b in breakdown.items()},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
+                "d2h_bytes_per_step": T * d * 2, "api": "moe_layer_fwd with pinned host X/out copies"},
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wg0, wu0, wd0 = wg[:1].cpu(), wu[:1].cpu(), wd[:1].cpu()
+        cv, desc, _ = _oracle_sample(w, seed, 512, 32, wg0, wu0, wd0)
+        line["cpu_baseline"] = {"value": cv, "unit": "tokens/s", "cores": _threads_used(), "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    from mixture_experts_routing_02_b200 import synthetic as syn
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=syn.MIXTRAL_LIKE.name, choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = syn.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,296 @@
+/*
+ * moe_routing.h -- C ABI of the single-GPU top-k Mixture-of-Experts FFN
+ * layer forward for NVIDIA B200 (sm_100a).
+ *
+ * The layer (forward pipeline of "Sparsely-Gated MoE 구현 관점에서 살펴보기:
+ * Router, Top-k, 부하 분산", section "순전파 과정(forward pass)은 디스패치와
+ * 결합(combine)을 포함"):
+ *
+ *   logits = X W_r^T (+ b)                        moe_route
+ *   ids, w = top-k of logits, softmax over them     moe_route / moe_route_from_logits
+ *   counts = per-expert histogram of ids            moe_histogram
+ *   segments (expert-contiguous layout), either
+ *     one per expert, capped at C rows            moe_segments
+ *     or the balanced plan over R groups          moe_plan_balanced
+ *   Xp = rows of X written to their final slots     moe_dispatch
+ *   Hp = silu(Xp W_g^T) * (Xp W_u^T)  per segment  moe_expert_gate_up
+ *   Yp = Hp W_d^T                     per segment  moe_expert_down
+ *   out[t] = sum_j w[t,j] Yp[dest[t*k+j]]           moe_combine
+ *   all of the above in one call                    moe_layer_fwd
+ *
+ * Conventions for every call:
+ *  - Tensor arguments are DEVICE pointers owned by the caller; the library
+ *    allocates and frees nothing, keeps no per-call state and never
+ *    synchronises the host.  All work is enqueued on `stream` (a
+ *    cudaStream_t; NULL is the legacy default stream) and is asynchronous.
+ *  - bf16 tensors are passed as `moe_bf16_t` (raw IEEE bfloat16 bits).
+ *  - All matrices are row-major and dense.  Weights use the nn.Linear
+ *    [out, in] layout: W_r [E, d], W_g and W_u [E, F, d], W_d [E, d, F].
+ *  - The return value reports errors that the host can see before anything
+ *    is enqueued (bad arguments, unsupported sizes, launch failures).  In
+ *    that case nothing, or only a prefix of a composite call, was enqueued.
+ *  - Errors only the device can see (an infeasible balanced plan, a bounded
+ *    wait that ran out) are OR-ed into the caller's `int32_t *status` device
+ *    word (MOE_DEV_ERR_* bits; 0 = fine).  The caller clears it and reads it
+ *    whenever it next synchronises.  `status` may be NULL to ignore them.
+ *  - Every wait inside a kernel is bounded (about two seconds); a wait that
+ *    runs out sets MOE_DEV_ERR_TIMEOUT and the kernel returns.
+ *
+ * Supported sizes: 0 <= T, T*k < 2^30; 1 <= E <= 256; 1 <= k <= min(E, 8);
+ * d_model and d_ff multiples of 64 (>= 64); at most 2048 segments.
+ */
+#ifndef MOE_ROUTING_H
+#define MOE_ROUTING_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef uint16_t moe_bf16_t;
+typedef void *moe_stream_t; /* cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, negative size, k > E, bad group split */
+    MOE_ERR_UNSUPPORTED = 2, /* sizes outside the supported range above */
+    MOE_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
+    MOE_ERR_CUDA = 4         /* a CUDA runtime call or launch failed */
+} moe_status_t;
+
+/* bits of the device status word */
+#define MOE_DEV_ERR_PLAN 0x1    /* balanced plan needs more than B replica slots */
+#define MOE_DEV_ERR_TIMEOUT 0x2 /* a bounded wait inside a kernel ran out */
+
+/*
+ * Layer shape.
+ *   T              tokens (rows of X)
+ *   d_model        hidden size d
+ *   n_experts      E
+ *   top_k          k
+ *   d_ff           expert FFN inner size F
+ *   capacity       0 = no limit; else C, the most rows one expert keeps.
+ *                  A (t, j) pair whose stable rank inside its expert (pairs
+ *                  ordered by q = t*k + j) is >= C is dropped: dest = -1, it
+ *                  contributes nothing, and the kept weights of that token
+ *                  are not renormalised.  ("로드 밸런싱 손실(load-balancing
+ *                  loss)과 용량(capacity)은 별개": overflow skips the expert
+ *                  and leaves only the residual path.)  The caller computes C,
+ *                  e.g. ceil(cf * T * k / E).
+ *   n_groups       R; 0 = no balanced plan.  With R > 0 the E experts are
+ *                  homed in R contiguous groups of E/R, the T tokens form R
+ *                  groups of S = T/R, and every group receives exactly S*k
+ *                  rows ("가장 바쁜 랭크가 속도를 정합니다: MoonEP의 계획 코드를 직접
+ *                  돌려봤습니다", sections "개요" and "이 기술은 무엇인가").
+ *                  Requires E % R == 0, T % R == 0 and capacity == 0.
+ *   replica_slots  B, replica slots per group (the page's [E, E+B) slots).
+ */
+typedef struct {
+    int32_t T;
+    int32_t d_model;
+    int32_t n_experts;
+    int32_t top_k;
+    int32_t d_ff;
+    int32_t capacity;
+    int32_t n_groups;
+    int32_t replica_slots;
+} moe_shape_t;
+
+/*
+ * Segment tables.  The dispatched rows Xp / Hp / Yp are laid out as n_seg
+ * consecutive segments; segment s holds rows [seg_offsets[s],
+ * seg_offsets[s+1]) of expert seg_expert[s] (-1 = unused slot, 0 rows), and
+ * its first row is the pair of within-expert rank seg_first_rank[s].  This is
+ * the device-side cu_seqlens of the MoonEP page ("설치 및 통합").
+ *   no plan:  n_seg = E, segment e = expert e, min(count_e, C) rows.
+ *   plan:     n_seg = R * (E/R + B); group g owns segments
+ *             [g*(E/R+B), (g+1)*(E/R+B)): its E/R home experts in ascending
+ *             id, then its B replica slots in creation order; it spans rows
+ *             [g*S*k, (g+1)*S*k).
+ */
+
+/* Human-readable name of a moe_status_t. */
+MOE_API const char *moe_status_string(moe_status_t s);
+
+/*
+ * Sizes implied by a shape: *n_segments (as above) and *rows_alloc, the rows
+ * Xp, Hp and Yp must have: T*k without capacity, min(T*k, C*E) with it.
+ * Host only; enqueues nothing.  Either output pointer may be NULL.
+ */
+MOE_API moe_status_t moe_layout(const moe_shape_t *shape, int32_t *n_segments, int32_t *rows_alloc);
+
+/*
+ * Workspace bytes for moe_dispatch (*dispatch_bytes) and for moe_layer_fwd
+ * (*layer_bytes, which also holds every intermediate of the layer).  Host
+ * only.  Either output pointer may be NULL.
+ */
+MOE_API moe_status_t moe_workspace_size(const moe_shape_t *shape, size_t *dispatch_bytes, size_t *layer_bytes);
+
+/*
+ * Router projection fused with top-k and the renormalised softmax
+ * ("Sparsely-Gated MoE 구현 관점에서 살펴보기", sections "Router를 텐서 형태에서
+ * 추적하기", "Top-2 라우팅의 수치 예시", "pure Python으로 Top-k Router 확인하기").
+ *   x        [T, d] bf16            w_router [E, d] bf16
+ *   bias     [E] fp32 or NULL; added to the logits before selection
+ *   logits   [T, E] fp32 out, or NULL to skip writing it
+ *   topk_ids [T, k] int32 out: the k largest logits, descending; equal
+ *            values go to the lower expert id
+ *   topk_w   [T, k] fp32 out: w_j = exp(l_j - l_max) / sum_sel exp(l - l_max)
+ * The projection runs on the tensor cores (bf16 in, fp32 accumulate); the
+ * selection is made on the fp32 logits.
+ */
+MOE_API moe_status_t moe_route(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *w_router,
+                       const float *bias, float *logits, int32_t *topk_ids, float *topk_w,
+                       int32_t *status, moe_stream_t stream);
+
+/* Top-k selection and weights alone, on given fp32 logits [T, E] (same selection and weights as moe_route). */
+MOE_API moe_status_t moe_route_from_logits(const moe_shape_t *shape, const float *logits, int32_t *topk_ids,
+                                   float *topk_w, moe_stream_t stream);
+
+/*
+ * Histogram: counts[e] = number of (t, j) with topk_ids[t, j] == e, raw (before any
+ * capacity).  ("5.3 Expert Parallelism", section "2. 디스패처 엔지니어링":
+ * the per-destination bincount; MoonEP page "설치 및 통합": tokens_per_expert.)
+ *   topk_ids [T, k] int32 in, values in [0, E)     counts [E] int32 out
+ */
+MOE_API moe_status_t moe_histogram(const moe_shape_t *shape, const int32_t *topk_ids, int32_t *counts,
+                           moe_stream_t stream);
+
+/*
+ * Plain segment layout: one segment per expert holding min(counts[e], C)
+ * rows (all of them when capacity == 0); seg_offsets is the exclusive scan.
+ *   counts [E] in; seg_expert [E], seg_offsets [E+1], seg_first_rank [E] out.
+ * Requires n_groups == 0.
+ */
+MOE_API moe_status_t moe_segments(const moe_shape_t *shape, const int32_t *counts, int32_t *seg_expert,
+                          int32_t *seg_offsets, int32_t *seg_first_rank, moe_stream_t stream);
+
+/*
+ * Balanced plan (MoonEP page, sections "개요", "이 기술은 무엇인가",
+ * "설치 및 통합", "실제 실험 결과").  Every one of the R groups receives
+ * exactly S*k rows; overloaded groups give rows of their most loaded experts
+ * (descending count, ties to the lower id) to underloaded groups, which hold
+ * them in replica slots.  Deterministic; the algorithm, which the page does
+ * not give, is: groups above S*k in ascending order queue their excess as
+ * (expert, rows) chunks; groups below S*k in ascending order take their
+ * deficit from the front of that queue, one replica slot per (expert, group)
+ * piece; an expert's rows in stable order fill its home segment first, then
+ * its pieces in creation order.
+ *   counts [E] in (Σ counts must be T*k); seg tables [n_seg] / [n_seg+1] out.
+ * If some group would need more than B slots the plan is infeasible (the
+ * page's `alloc.sum(dim=0) > CAP` error): MOE_DEV_ERR_PLAN is set in *status
+ * and every segment is written empty, so later calls move and compute nothing.
+ */
+MOE_API moe_status_t moe_plan_balanced(const moe_shape_t *shape, const int32_t *counts, int32_t *seg_expert,
+                               int32_t *seg_offsets, int32_t *seg_first_rank, int32_t *status,
+                               moe_stream_t stream);
+
+/*
+ * Dispatch.  When plan_ready == 0 this computes counts
+ * and the segment tables first (moe_histogram, then moe_plan_balanced if
+ * n_groups > 0 else moe_segments), writing them to the given buffers; when
+ * plan_ready != 0 they are inputs from earlier calls.  Then, in one pass with
+ * a decoupled look-back over tiles of (t, j) pairs, each pair gets its
+ * stable rank r inside its expert and its final row
+ *   dest[t*k+j] = seg_offsets[s] + r - seg_first_rank[s]
+ * for the segment s of that expert covering rank r (-1 if none: dropped), and
+ * the token's row is copied straight to that slot ("MoonEP", section "이 기술은
+ * 무엇인가": writing each row to its final position makes the separate sort
+ * and copy disappear):
+ *   Xp[dest[t*k+j]] = X[t],  src[dest[q]] = q.
+ *   x [T, d] bf16 in; dest [T*k] int32 out; src [rows_alloc] int32 out;
+ *   xp [rows_alloc, d] bf16 out (rows past seg_offsets[n_seg] untouched).
+ *   ws, ws_bytes: at least moe_workspace_size()'s dispatch_bytes of device
+ *   memory; its contents need not be initialised and are clobbered.
+ */
+MOE_API moe_status_t moe_dispatch(const moe_shape_t *shape, const moe_bf16_t *x, const int32_t *topk_ids,
+                          int32_t plan_ready, int32_t *counts, int32_t *seg_expert,
+                          int32_t *seg_offsets, int32_t *seg_first_rank, int32_t *dest,
+                          int32_t *src, moe_bf16_t *xp, int32_t *status, void *ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/*
+ * Grouped GEMM of the gate and up projections fused with SwiGLU
+ * ("5.3 Expert Parallelism", section "3. 고도화된 최적화: 오버래핑(Overlapping) 및
+ * GroupGEMM": all experts' GEMMs in one launch):
+ *   Hp[r, :] = silu(Xp[r] W_g[e]^T) * (Xp[r] W_u[e]^T),  e = expert of r's segment,
+ * silu(z) = z / (1 + exp(-z)); fp32 accumulation in tensor memory, Hp
+ * rounded to bf16.  Segment sizes are read on the device (no host sync).
+ *   xp [rows_alloc, d]; w_gate, w_up [E, F, d]; hp [rows_alloc, F] out.
+ */
+MOE_API moe_status_t moe_expert_gate_up(const moe_shape_t *shape, const moe_bf16_t *xp,
+                                const int32_t *seg_expert, const int32_t *seg_offsets,
+                                const moe_bf16_t *w_gate, const moe_bf16_t *w_up, moe_bf16_t *hp,
+                                int32_t *status, moe_stream_t stream);
+
+/*
+ * Grouped down projection Yp[r, :] = Hp[r] W_d[e]^T (fp32 accumulate,
+ * bf16 out).   hp [rows_alloc, F]; w_down [E, d, F]; yp [rows_alloc, d] out.
+ */
+MOE_API moe_status_t moe_expert_down(const moe_shape_t *shape, const moe_bf16_t *hp,
+                             const int32_t *seg_expert, const int32_t *seg_offsets,
+                             const moe_bf16_t *w_down, moe_bf16_t *yp, int32_t *status,
+                             moe_stream_t stream);
+
+/* moe_expert_gate_up then moe_expert_down. */
+MOE_API moe_status_t moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *xp, const int32_t *seg_expert,
+                            const int32_t *seg_offsets, const moe_bf16_t *w_gate,
+                            const moe_bf16_t *w_up, const moe_bf16_t *w_down, moe_bf16_t *hp,
+                            moe_bf16_t *yp, int32_t *status, moe_stream_t stream);
+
+/*
+ * Combine ("Sparsely-Gated MoE 구현 관점에서 살펴보기", section "순전파 과정
+ * ...", last step: un-permute and weight by the router; MoonEP page
+ * "설치 및 통합": combine):
+ *   out[t] = sum over j with dest[t*k+j] >= 0 of topk_w[t, j] * Yp[dest[t*k+j]]
+ * accumulated in fp32 in ascending j, rounded to bf16.  A token whose pairs
+ * were all dropped gets 0.
+ *   yp [rows_alloc, d]; dest [T*k]; topk_w [T, k]; out [T, d] bf16.
+ */
+MOE_API moe_status_t moe_combine(const moe_shape_t *shape, const moe_bf16_t *yp, const int32_t *dest,
+                         const float *topk_w, moe_bf16_t *out, moe_stream_t stream);
+
+/*
+ * The whole layer: moe_route (logits not stored) -> moe_dispatch ->
+ * moe_expert_gate_up -> moe_expert_down -> moe_combine, all on `stream`.
+ * The intermediates live in `ws` (moe_workspace_size()'s layer_bytes); their
+ * addresses are given by moe_layer_views.
+ */
+MOE_API moe_status_t moe_layer_fwd(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *w_router,
+                           const float *bias, const moe_bf16_t *w_gate, const moe_bf16_t *w_up,
+                           const moe_bf16_t *w_down, moe_bf16_t *out, int32_t *status, void *ws,
+                           size_t ws_bytes, moe_stream_t stream);
+
+/* Device addresses of the intermediates moe_layer_fwd keeps in its workspace. */
+typedef struct {
+    int32_t *topk_ids;       /* [T, k] */
+    float *topk_w;           /* [T, k] */
+    int32_t *counts;         /* [E] */
+    int32_t *seg_expert;     /* [n_seg] */
+    int32_t *seg_offsets;    /* [n_seg + 1] */
+    int32_t *seg_first_rank; /* [n_seg] */
+    int32_t *dest;           /* [T * k] */
+    int32_t *src;            /* [rows_alloc] */
+    moe_bf16_t *xp;          /* [rows_alloc, d] */
+    moe_bf16_t *hp;          /* [rows_alloc, F] */
+    moe_bf16_t *yp;          /* [rows_alloc, d] */
+    void *dispatch_ws;       /* moe_dispatch's own workspace */
+    size_t dispatch_ws_bytes;
+} moe_layer_views_t;
+
+/* Fill *views with the addresses inside a layer workspace `ws`. Host only. */
+MOE_API moe_status_t moe_layer_views(const moe_shape_t *shape, void *ws, moe_layer_views_t *views);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_ROUTING_H */

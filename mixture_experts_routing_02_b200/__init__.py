@@ -1,0 +1,196 @@
+"""Python binding of the C ABI in ``include/moe_routing.h`` (libmoe_b200.so).
+
+Argument marshalling only: every function takes torch CUDA tensors (or None
+for a nullable pointer), passes their device addresses and the current CUDA
+stream to the C call of the same name, and raises ``MoeError`` when the call
+returns a status other than MOE_OK.  All computation happens in the library's
+CUDA kernels; there is no fallback of any kind.  If the library has not been
+built, the first call raises ``RuntimeError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "MoeError", "MoeShape", "MoeLayerViews", "LIB_PATH", "SYMBOLS", "load_library", "shape",
+    "moe_status_string", "moe_layout", "moe_workspace_size", "moe_route", "moe_route_from_logits",
+    "moe_histogram", "moe_segments", "moe_plan_balanced", "moe_dispatch", "moe_expert_gate_up",
+    "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_layer_fwd", "moe_layer_views",
+    "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+
+DEV_ERR_PLAN = 0x1
+DEV_ERR_TIMEOUT = 0x2
+
+
+class MoeError(RuntimeError):
+    pass
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("T", "d_model", "n_experts", "top_k", "d_ff", "capacity", "n_groups", "replica_slots")]
+
+
+class MoeLayerViews(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("topk_ids", "topk_w", "counts", "seg_expert", "seg_offsets", "seg_first_rank", "dest",
+                 "src", "xp", "hp", "yp", "dispatch_ws")] + [("dispatch_ws_bytes", ctypes.c_size_t)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_S = ctypes.POINTER(MoeShape)
+
+# name -> argument types (return type is moe_status_t = int, except moe_status_string)
+SYMBOLS = {
+    "moe_status_string": [ctypes.c_int],
+    "moe_layout": [_S, _P, _P],
+    "moe_workspace_size": [_S, _P, _P],
+    "moe_route": [_S, _P, _P, _P, _P, _P, _P, _P, _P],
+    "moe_route_from_logits": [_S, _P, _P, _P, _P],
+    "moe_histogram": [_S, _P, _P, _P],
+    "moe_segments": [_S, _P, _P, _P, _P, _P],
+    "moe_plan_balanced": [_S, _P, _P, _P, _P, _P, _P],
+    "moe_dispatch": [_S, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "moe_expert_gate_up": [_S, _P, _P, _P, _P, _P, _P, _P, _P],
+    "moe_expert_down": [_S, _P, _P, _P, _P, _P, _P, _P],
+    "moe_expert_ffn": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "moe_combine": [_S, _P, _P, _P, _P, _P],
+    "moe_layer_fwd": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "moe_layer_views": [_S, _P, ctypes.POINTER(MoeLayerViews)],
+}
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmoe_b200.so and declare every exported call (raises if it is missing)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built; run `python -m mixture_experts_routing_02_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, args in SYMBOLS.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_char_p if name == "moe_status_string" else ctypes.c_int
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def shape(T, d_model, n_experts, top_k, d_ff, capacity=0, n_groups=0, replica_slots=0) -> MoeShape:
+    return MoeShape(T, d_model, n_experts, top_k, d_ff, capacity, n_groups, replica_slots)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor arguments must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _check(name: str, st: int):
+    if st != 0:
+        raise MoeError(f"{name}: {load_library().moe_status_string(st).decode()}")
+
+
+def moe_status_string(st: int) -> str:
+    return load_library().moe_status_string(st).decode()
+
+
+def moe_layout(s: MoeShape):
+    n_seg, rows = ctypes.c_int32(), ctypes.c_int32()
+    _check("moe_layout", load_library().moe_layout(ctypes.byref(s), ctypes.byref(n_seg), ctypes.byref(rows)))
+    return n_seg.value, rows.value
+
+
+def moe_workspace_size(s: MoeShape):
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check("moe_workspace_size", load_library().moe_workspace_size(ctypes.byref(s), ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
+
+
+def moe_route(s, x, w_router, bias, logits, topk_ids, topk_w, status=None, stream=None):
+    _check("moe_route", load_library().moe_route(
+        ctypes.byref(s), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logits), _ptr(topk_ids), _ptr(topk_w),
+        _ptr(status), _stream(stream)))
+
+
+def moe_route_from_logits(s, logits, topk_ids, topk_w, stream=None):
+    _check("moe_route_from_logits", load_library().moe_route_from_logits(
+        ctypes.byref(s), _ptr(logits), _ptr(topk_ids), _ptr(topk_w), _stream(stream)))
+
+
+def moe_histogram(s, topk_ids, counts, stream=None):
+    _check("moe_histogram", load_library().moe_histogram(ctypes.byref(s), _ptr(topk_ids), _ptr(counts),
+                                                          _stream(stream)))
+
+
+def moe_segments(s, counts, seg_expert, seg_offsets, seg_first_rank, stream=None):
+    _check("moe_segments", load_library().moe_segments(
+        ctypes.byref(s), _ptr(counts), _ptr(seg_expert), _ptr(seg_offsets), _ptr(seg_first_rank), _stream(stream)))
+
+
+def moe_plan_balanced(s, counts, seg_expert, seg_offsets, seg_first_rank, status=None, stream=None):
+    _check("moe_plan_balanced", load_library().moe_plan_balanced(
+        ctypes.byref(s), _ptr(counts), _ptr(seg_expert), _ptr(seg_offsets), _ptr(seg_first_rank), _ptr(status),
+        _stream(stream)))
+
+
+def moe_dispatch(s, x, topk_ids, plan_ready, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp,
+                 status, ws, stream=None):
+    _check("moe_dispatch", load_library().moe_dispatch(
+        ctypes.byref(s), _ptr(x), _ptr(topk_ids), int(plan_ready), _ptr(counts), _ptr(seg_expert),
+        _ptr(seg_offsets), _ptr(seg_first_rank), _ptr(dest), _ptr(src), _ptr(xp), _ptr(status), _ptr(ws),
+        ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def moe_expert_gate_up(s, xp, seg_expert, seg_offsets, w_gate, w_up, hp, status=None, stream=None):
+    _check("moe_expert_gate_up", load_library().moe_expert_gate_up(
+        ctypes.byref(s), _ptr(xp), _ptr(seg_expert), _ptr(seg_offsets), _ptr(w_gate), _ptr(w_up), _ptr(hp),
+        _ptr(status), _stream(stream)))
+
+
+def moe_expert_down(s, hp, seg_expert, seg_offsets, w_down, yp, status=None, stream=None):
+    _check("moe_expert_down", load_library().moe_expert_down(
+        ctypes.byref(s), _ptr(hp), _ptr(seg_expert), _ptr(seg_offsets), _ptr(w_down), _ptr(yp), _ptr(status),
+        _stream(stream)))
+
+
+def moe_expert_ffn(s, xp, seg_expert, seg_offsets, w_gate, w_up, w_down, hp, yp, status=None, stream=None):
+    _check("moe_expert_ffn", load_library().moe_expert_ffn(
+        ctypes.byref(s), _ptr(xp), _ptr(seg_expert), _ptr(seg_offsets), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+        _ptr(hp), _ptr(yp), _ptr(status), _stream(stream)))
+
+
+def moe_combine(s, yp, dest, topk_w, out, stream=None):
+    _check("moe_combine", load_library().moe_combine(
+        ctypes.byref(s), _ptr(yp), _ptr(dest), _ptr(topk_w), _ptr(out), _stream(stream)))
+
+
+def moe_layer_fwd(s, x, w_router, bias, w_gate, w_up, w_down, out, status, ws, stream=None):
+    _check("moe_layer_fwd", load_library().moe_layer_fwd(
+        ctypes.byref(s), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(out),
+        _ptr(status), _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def moe_layer_views(s, ws) -> MoeLayerViews:
+    v = MoeLayerViews()
+    _check("moe_layer_views", load_library().moe_layer_views(ctypes.byref(s), _ptr(ws), ctypes.byref(v)))
+    return v

@@ -1,0 +1,410 @@
+// C ABI of the library: argument validation, TMA descriptor encoding and the
+// launch sequence of every call.  Nothing here allocates device memory,
+// synchronises the host, or keeps per-call state; the only process-wide state
+// is the driver entry point of cuTensorMapEncodeTiled and a per-device cache
+// of the SM count.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool have_encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+int sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev >= 0 && dev < 64) cache[dev] = n;
+    return n;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Dims {
+    int T, d, E, k, F, C, R, B, S;
+    int n_seg;
+    int rows;  // rows_alloc
+};
+
+moe_status_t check_shape(const moe_shape_t* s, Dims* out) {
+    if (s == nullptr) return MOE_ERR_INVALID_ARG;
+    Dims v;
+    v.T = s->T; v.d = s->d_model; v.E = s->n_experts; v.k = s->top_k; v.F = s->d_ff;
+    v.C = s->capacity; v.R = s->n_groups; v.B = s->replica_slots;
+    if (v.T < 0 || v.d < 1 || v.E < 1 || v.k < 1 || v.k > v.E || v.F < 1 || v.C < 0 || v.R < 0 || v.B < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (v.R > 0 && (v.E % v.R != 0 || v.T % v.R != 0 || v.C > 0)) return MOE_ERR_INVALID_ARG;
+    if (v.E > kMaxExperts || v.k > kMaxTopK || v.d % 64 != 0 || v.F % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(v.T) * v.k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+    const int64_t n_seg = v.R > 0 ? static_cast<int64_t>(v.R) * (v.E / v.R + v.B) : v.E;
+    if (n_seg > kMaxSegments) return MOE_ERR_UNSUPPORTED;
+    v.n_seg = static_cast<int>(n_seg);
+    v.S = v.R > 0 ? v.T / v.R : v.T;
+    int64_t rows = static_cast<int64_t>(v.T) * v.k;
+    if (v.C > 0) rows = std::min<int64_t>(rows, static_cast<int64_t>(v.C) * v.E);
+    v.rows = static_cast<int>(rows);
+    if (out) *out = v;
+    return MOE_OK;
+}
+
+bool encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+            const cuuint32_t* box) {
+    const cuuint32_t es[3] = {1, 1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, K] row-major bf16, tiles of 128 rows x 64 columns
+bool tmap_rows(CUtensorMap* m, const void* p, int rows, int K) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    return encode(m, p, 2, dims, strides, box);
+}
+
+// [E, N, K] row-major bf16 (one [N, K] weight per expert), tiles of box_n rows x 64 columns of one expert
+bool tmap_experts(CUtensorMap* m, const void* p, int E, int N, int K, int box_n) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(E)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, static_cast<cuuint64_t>(K) * N * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_n), 1};
+    return encode(m, p, 3, dims, strides, box);
+}
+
+inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// ------------------------------------------------------------------------------ implementations
+
+moe_status_t route_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
+                        float* logits, int32_t* ids, float* w, int32_t* status, cudaStream_t st) {
+    if (!x || !w_router || !ids || !w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+    if (v.T == 0) return MOE_OK;
+    if (!have_encoder()) return MOE_ERR_CUDA;
+    const int epad = std::max(16, (v.E + 15) / 16 * 16);
+    CUtensorMap ta, tb;
+    if (!tmap_rows(&ta, x, v.T, v.d)) return MOE_ERR_CUDA;
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(v.d), static_cast<cuuint64_t>(v.E)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(v.d) * 2};
+        const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(v.E)};
+        if (!encode(&tb, w_router, 2, dims, strides, box)) return MOE_ERR_CUDA;
+    }
+    GemmArgs g{};
+    g.seg_offsets = nullptr; g.seg_expert = nullptr; g.n_seg = 1; g.M = v.T; g.K = v.d; g.N = v.E;
+    g.BN = epad; g.n_tiles_n = 1; g.mma_n = epad; g.stages = gemm_pick_stages(epad);
+    g.bias = bias; g.logits = logits; g.topk_ids = ids; g.topk_w = w; g.k = v.k; g.status = status;
+    const int grid = std::min(sm_count(), (v.T + 127) / 128);
+    return cuda_status(launch_umma_gemm(kEpiRoute, ta, tb, tb, g, grid, st));
+}
+
+moe_status_t gate_up_impl(const Dims& v, const moe_bf16_t* xp, const int32_t* seg_expert, const int32_t* seg_offsets,
+                          const moe_bf16_t* wg, const moe_bf16_t* wu, moe_bf16_t* hp, int32_t* status,
+                          cudaStream_t st) {
+    if (!xp || !seg_expert || !seg_offsets || !wg || !wu || !hp) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(xp) || !aligned16(wg) || !aligned16(wu) || !aligned16(hp)) return MOE_ERR_INVALID_ARG;
+    if (v.T == 0 || v.rows == 0) return MOE_OK;
+    if (!have_encoder()) return MOE_ERR_CUDA;
+    const int bn = v.F >= 128 ? 128 : v.F;
+    CUtensorMap ta, tg, tu;
+    if (!tmap_rows(&ta, xp, v.rows, v.d) || !tmap_experts(&tg, wg, v.E, v.F, v.d, bn) ||
+        !tmap_experts(&tu, wu, v.E, v.F, v.d, bn))
+        return MOE_ERR_CUDA;
+    GemmArgs g{};
+    g.seg_offsets = seg_offsets; g.seg_expert = seg_expert; g.n_seg = v.n_seg; g.M = v.rows; g.K = v.d; g.N = v.F;
+    g.BN = bn; g.n_tiles_n = (v.F + bn - 1) / bn; g.mma_n = 2 * bn; g.stages = gemm_pick_stages(2 * bn);
+    g.out = reinterpret_cast<__nv_bfloat16*>(hp); g.ldo = v.F; g.k = v.k; g.status = status;
+    const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 128 + v.n_seg) * g.n_tiles_n;
+    const int grid = static_cast<int>(std::min<int64_t>(sm_count(), max_tiles));
+    return cuda_status(launch_umma_gemm(kEpiSwiglu, ta, tg, tu, g, grid, st));
+}
+
+moe_status_t down_impl(const Dims& v, const moe_bf16_t* hp, const int32_t* seg_expert, const int32_t* seg_offsets,
+                       const moe_bf16_t* wd, moe_bf16_t* yp, int32_t* status, cudaStream_t st) {
+    if (!hp || !seg_expert || !seg_offsets || !wd || !yp) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(hp) || !aligned16(wd) || !aligned16(yp)) return MOE_ERR_INVALID_ARG;
+    if (v.T == 0 || v.rows == 0) return MOE_OK;
+    if (!have_encoder()) return MOE_ERR_CUDA;
+    const int bn = v.d >= 256 ? 256 : v.d;
+    CUtensorMap ta, tb;
+    if (!tmap_rows(&ta, hp, v.rows, v.F) || !tmap_experts(&tb, wd, v.E, v.d, v.F, bn)) return MOE_ERR_CUDA;
+    GemmArgs g{};
+    g.seg_offsets = seg_offsets; g.seg_expert = seg_expert; g.n_seg = v.n_seg; g.M = v.rows; g.K = v.F; g.N = v.d;
+    g.BN = bn; g.n_tiles_n = (v.d + bn - 1) / bn; g.mma_n = bn; g.stages = gemm_pick_stages(bn);
+    g.out = reinterpret_cast<__nv_bfloat16*>(yp); g.ldo = v.d; g.k = v.k; g.status = status;
+    const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 128 + v.n_seg) * g.n_tiles_n;
+    const int grid = static_cast<int>(std::min<int64_t>(sm_count(), max_tiles));
+    return cuda_status(launch_umma_gemm(kEpiStore, ta, tb, tb, g, grid, st));
+}
+
+moe_status_t segments_or_plan(const Dims& v, const int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets,
+                              int32_t* seg_first_rank, int32_t* status, cudaStream_t st) {
+    if (v.R > 0)
+        return cuda_status(launch_plan(counts, v.E, v.R, v.S, v.k, v.B, seg_expert, seg_offsets, seg_first_rank,
+                                       status, st));
+    return cuda_status(launch_segments(counts, v.E, v.C, seg_expert, seg_offsets, seg_first_rank, st));
+}
+
+moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* ids, int32_t plan_ready,
+                           int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank,
+                           int32_t* dest, int32_t* src, moe_bf16_t* xp, int32_t* status, void* ws,
+                           size_t ws_bytes, cudaStream_t st) {
+    if (!x || !ids || !counts || !seg_expert || !seg_offsets || !seg_first_rank || !dest || !src || !xp)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+    const size_t need = permute_ws_bytes(v.T, v.k, v.E);
+    if (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (!plan_ready) {
+        moe_status_t s = cuda_status(launch_histogram(ids, v.T * v.k, v.E, counts, sm_count(), st));
+        if (s != MOE_OK) return s;
+        s = segments_or_plan(v, counts, seg_expert, seg_offsets, seg_first_rank, status, st);
+        if (s != MOE_OK) return s;
+    }
+    PermuteArgs a{};
+    a.ids = ids; a.x = reinterpret_cast<const __nv_bfloat16*>(x); a.xp = reinterpret_cast<__nv_bfloat16*>(xp);
+    a.seg_expert = seg_expert; a.seg_offsets = seg_offsets; a.seg_first_rank = seg_first_rank;
+    a.dest = dest; a.src = src;
+    a.ticket = static_cast<uint32_t*>(ws);
+    a.tile_state = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 256);
+    a.status = status;
+    a.T = v.T; a.k = v.k; a.E = v.E; a.d = v.d; a.n_seg = v.n_seg;
+    a.tokens_per_tile = permute_tokens_per_tile(v.k);
+    a.n_tiles = permute_n_tiles(v.T, v.k);
+    return cuda_status(launch_permute(a, sm_count(), st));
+}
+
+struct LayerLayout {
+    size_t ids, w, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, dispatch_ws, xp, hp, yp, total;
+    size_t dispatch_ws_bytes;
+};
+
+LayerLayout layer_layout(const Dims& v) {
+    LayerLayout L{};
+    size_t o = 0;
+    const size_t tk = static_cast<size_t>(v.T) * v.k;
+    L.ids = o; o = align256(o + tk * 4);
+    L.w = o; o = align256(o + tk * 4);
+    L.counts = o; o = align256(o + static_cast<size_t>(v.E) * 4);
+    L.seg_expert = o; o = align256(o + static_cast<size_t>(v.n_seg) * 4);
+    L.seg_offsets = o; o = align256(o + static_cast<size_t>(v.n_seg + 1) * 4);
+    L.seg_first_rank = o; o = align256(o + static_cast<size_t>(v.n_seg) * 4);
+    L.dest = o; o = align256(o + tk * 4);
+    L.src = o; o = align256(o + static_cast<size_t>(v.rows) * 4);
+    L.dispatch_ws_bytes = permute_ws_bytes(v.T, v.k, v.E);
+    L.dispatch_ws = o; o = align256(o + L.dispatch_ws_bytes);
+    L.xp = o; o = align256(o + static_cast<size_t>(v.rows) * v.d * 2);
+    L.hp = o; o = align256(o + static_cast<size_t>(v.rows) * v.F * 2);
+    L.yp = o; o = align256(o + static_cast<size_t>(v.rows) * v.d * 2);
+    L.total = o;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: size outside the supported range";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA runtime or launch failure";
+    }
+    return "unknown moe_status_t";
+}
+
+moe_status_t moe_layout(const moe_shape_t* shape, int32_t* n_segments, int32_t* rows_alloc) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (n_segments) *n_segments = v.n_seg;
+    if (rows_alloc) *rows_alloc = v.rows;
+    return MOE_OK;
+}
+
+moe_status_t moe_workspace_size(const moe_shape_t* shape, size_t* dispatch_bytes, size_t* layer_bytes) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (dispatch_bytes) *dispatch_bytes = permute_ws_bytes(v.T, v.k, v.E);
+    if (layer_bytes) *layer_bytes = layer_layout(v).total;
+    return MOE_OK;
+}
+
+moe_status_t moe_route(const moe_shape_t* shape, const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
+                       float* logits, int32_t* topk_ids, float* topk_w, int32_t* status, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    return route_impl(v, x, w_router, bias, logits, topk_ids, topk_w, status, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_route_from_logits(const moe_shape_t* shape, const float* logits, int32_t* topk_ids, float* topk_w,
+                                   moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_route_from_logits(logits, v.T, v.E, v.k, topk_ids, topk_w, sm_count(),
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_histogram(const moe_shape_t* shape, const int32_t* topk_ids, int32_t* counts, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!topk_ids || !counts) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_histogram(topk_ids, v.T * v.k, v.E, counts, sm_count(), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_segments(const moe_shape_t* shape, const int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets,
+                          int32_t* seg_first_rank, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (v.R > 0 || !counts || !seg_expert || !seg_offsets || !seg_first_rank) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_segments(counts, v.E, v.C, seg_expert, seg_offsets, seg_first_rank,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_plan_balanced(const moe_shape_t* shape, const int32_t* counts, int32_t* seg_expert,
+                               int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* status, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (v.R == 0 || !counts || !seg_expert || !seg_offsets || !seg_first_rank) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_plan(counts, v.E, v.R, v.S, v.k, v.B, seg_expert, seg_offsets, seg_first_rank, status,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_ids, int32_t plan_ready,
+                          int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank,
+                          int32_t* dest, int32_t* src, moe_bf16_t* xp, int32_t* status, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    return dispatch_impl(v, x, topk_ids, plan_ready, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp,
+                         status, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* xp, const int32_t* seg_expert,
+                                const int32_t* seg_offsets, const moe_bf16_t* w_gate, const moe_bf16_t* w_up,
+                                moe_bf16_t* hp, int32_t* status, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    return gate_up_impl(v, xp, seg_expert, seg_offsets, w_gate, w_up, hp, status, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_down(const moe_shape_t* shape, const moe_bf16_t* hp, const int32_t* seg_expert,
+                             const int32_t* seg_offsets, const moe_bf16_t* w_down, moe_bf16_t* yp, int32_t* status,
+                             moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    return down_impl(v, hp, seg_expert, seg_offsets, w_down, yp, status, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* xp, const int32_t* seg_expert,
+                            const int32_t* seg_offsets, const moe_bf16_t* w_gate, const moe_bf16_t* w_up,
+                            const moe_bf16_t* w_down, moe_bf16_t* hp, moe_bf16_t* yp, int32_t* status,
+                            moe_stream_t stream) {
+    Dims v;
+    moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = gate_up_impl(v, xp, seg_expert, seg_offsets, w_gate, w_up, hp, status, st);
+    if (s != MOE_OK) return s;
+    return down_impl(v, hp, seg_expert, seg_offsets, w_down, yp, status, st);
+}
+
+moe_status_t moe_combine(const moe_shape_t* shape, const moe_bf16_t* yp, const int32_t* dest, const float* topk_w,
+                         moe_bf16_t* out, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(yp) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_combine(reinterpret_cast<const __nv_bfloat16*>(yp), dest, topk_w, v.T, v.k, v.d,
+                                      reinterpret_cast<__nv_bfloat16*>(out), sm_count(),
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_layer_views(const moe_shape_t* shape, void* ws, moe_layer_views_t* views) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!ws || !views) return MOE_ERR_INVALID_ARG;
+    const LayerLayout L = layer_layout(v);
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    views->topk_ids = reinterpret_cast<int32_t*>(b + L.ids);
+    views->topk_w = reinterpret_cast<float*>(b + L.w);
+    views->counts = reinterpret_cast<int32_t*>(b + L.counts);
+    views->seg_expert = reinterpret_cast<int32_t*>(b + L.seg_expert);
+    views->seg_offsets = reinterpret_cast<int32_t*>(b + L.seg_offsets);
+    views->seg_first_rank = reinterpret_cast<int32_t*>(b + L.seg_first_rank);
+    views->dest = reinterpret_cast<int32_t*>(b + L.dest);
+    views->src = reinterpret_cast<int32_t*>(b + L.src);
+    views->xp = reinterpret_cast<moe_bf16_t*>(b + L.xp);
+    views->hp = reinterpret_cast<moe_bf16_t*>(b + L.hp);
+    views->yp = reinterpret_cast<moe_bf16_t*>(b + L.yp);
+    views->dispatch_ws = b + L.dispatch_ws;
+    views->dispatch_ws_bytes = L.dispatch_ws_bytes;
+    return MOE_OK;
+}
+
+moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const moe_bf16_t* w_router,
+                           const float* bias, const moe_bf16_t* w_gate, const moe_bf16_t* w_up,
+                           const moe_bf16_t* w_down, moe_bf16_t* out, int32_t* status, void* ws, size_t ws_bytes,
+                           moe_stream_t stream) {
+    Dims v;
+    moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!out || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    const LayerLayout L = layer_layout(v);
+    if (ws == nullptr || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (v.T == 0) return MOE_OK;
+    moe_layer_views_t w;
+    moe_layer_views(shape, ws, &w);
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = route_impl(v, x, w_router, bias, nullptr, w.topk_ids, w.topk_w, status, st);
+    if (s != MOE_OK) return s;
+    s = dispatch_impl(v, x, w.topk_ids, 0, w.counts, w.seg_expert, w.seg_offsets, w.seg_first_rank, w.dest, w.src,
+                      w.xp, status, w.dispatch_ws, w.dispatch_ws_bytes, st);
+    if (s != MOE_OK) return s;
+    s = gate_up_impl(v, w.xp, w.seg_expert, w.seg_offsets, w_gate, w_up, w.hp, status, st);
+    if (s != MOE_OK) return s;
+    s = down_impl(v, w.hp, w.seg_expert, w.seg_offsets, w_down, w.yp, status, st);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_combine(reinterpret_cast<const __nv_bfloat16*>(w.yp), w.dest, w.topk_w, v.T, v.k, v.d,
+                                      reinterpret_cast<__nv_bfloat16*>(out), sm_count(), st));
+}
+
+}  // extern "C"

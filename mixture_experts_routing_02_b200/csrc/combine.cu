@@ -1,0 +1,79 @@
+// Combine: out[t] = sum_j w[t, j] * Yp[dest[t*k + j]] over the kept pairs,
+// accumulated in fp32 in ascending j and rounded to bf16 once.
+//
+// Sources: "Sparsely-Gated MoE 구현 관점에서 살펴보기", section "순전파 과정 ..."
+// (un-permute the expert outputs and combine them with the router weights);
+// the MoonEP page, section "설치 및 통합" (combine returns the tokens in their
+// original order).
+//
+// One warp per token: each lane owns 16-byte vectors of the row, issues the k
+// gathers of a vector before using any of them, and writes the result with one
+// 16-byte store.  The kernel is HBM-bound: it reads k rows and writes one row
+// per token.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ yp,
+                                                      const int32_t* __restrict__ dest,
+                                                      const float* __restrict__ w, int T, int k, int d,
+                                                      __nv_bfloat16* __restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int warps_total = gridDim.x * (blockDim.x >> 5);
+    const int vec_per_row = d / 8;
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
+        int mine_d = -1;
+        float mine_w = 0.f;
+        if (lane < k) {
+            mine_d = __ldg(dest + static_cast<size_t>(t) * k + lane);
+            mine_w = __ldg(w + static_cast<size_t>(t) * k + lane);
+        }
+        int dr[kMaxTopK];
+        float wr[kMaxTopK];
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            dr[j] = __shfl_sync(0xffffffffu, mine_d, j);
+            wr[j] = __shfl_sync(0xffffffffu, mine_w, j);
+            if (j >= k) dr[j] = -1;
+        }
+        uint4* orow = reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * d);
+        for (int v = lane; v < vec_per_row; v += 32) {
+            uint4 val[kMaxTopK];
+#pragma unroll
+            for (int j = 0; j < kMaxTopK; ++j)
+                if (dr[j] >= 0) val[j] = __ldg(reinterpret_cast<const uint4*>(yp + static_cast<size_t>(dr[j]) * d) + v);
+            float acc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+            for (int j = 0; j < kMaxTopK; ++j) {
+                if (dr[j] >= 0) {
+                    const uint32_t p[4] = {val[j].x, val[j].y, val[j].z, val[j].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc[2 * i] = fmaf(wr[j], bf16_lo(p[i]), acc[2 * i]);
+                        acc[2 * i + 1] = fmaf(wr[j], bf16_hi(p[i]), acc[2 * i + 1]);
+                    }
+                }
+            }
+            orow[v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                 pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const __nv_bfloat16* yp, const int32_t* dest, const float* w, int T, int k, int d,
+                           __nv_bfloat16* out, int num_sms, cudaStream_t stream) {
+    if (T == 0) return cudaSuccess;
+    int grid = (T + 7) / 8;
+    if (grid > 8 * num_sms) grid = 8 * num_sms;
+    combine_kernel<<<grid, 256, 0, stream>>>(yp, dest, w, T, k, d, out);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

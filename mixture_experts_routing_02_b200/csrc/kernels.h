@@ -1,0 +1,83 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 8;
+constexpr int kMaxSegments = 2048;
+constexpr size_t kGemmSmemBudget = 200 * 1024;  // operand stages of the GEMM
+constexpr size_t kGemmSmemMin = 120 * 1024;     // > half an SM's shared memory: one CTA per SM
+
+enum EpiKind : int { kEpiRoute = 0, kEpiSwiglu = 1, kEpiStore = 2 };
+
+struct GemmArgs {
+    const int32_t* seg_offsets;  // [n_seg+1] or nullptr: a single segment of M rows
+    const int32_t* seg_expert;   // [n_seg] or nullptr: expert 0
+    int n_seg;
+    int M;          // rows when seg_offsets == nullptr
+    int K;          // reduction length, multiple of 64
+    int N;          // valid output columns (route: E)
+    int BN;         // output columns per tile
+    int n_tiles_n;  // column tiles
+    int mma_n;      // UMMA N
+    int stages;     // smem pipeline depth
+    __nv_bfloat16* out;
+    int ldo;
+    const float* bias;
+    float* logits;
+    int32_t* topk_ids;
+    float* topk_w;
+    int k;
+    int32_t* status;
+};
+
+size_t gemm_smem_bytes(int stages, int mma_n);
+int gemm_pick_stages(int mma_n);
+cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                             const GemmArgs& g, int grid, cudaStream_t stream);
+
+// dispatch.cu
+constexpr int kPermuteThreads = 256;
+constexpr int kPermutePairs = 256;  // (t, j) pairs per look-back tile, rounded to whole tokens
+
+struct PermuteArgs {
+    const int32_t* ids;
+    const __nv_bfloat16* x;
+    __nv_bfloat16* xp;
+    const int32_t* seg_expert;
+    const int32_t* seg_offsets;
+    const int32_t* seg_first_rank;
+    int32_t* dest;
+    int32_t* src;
+    uint32_t* tile_state;  // [n_tiles * E], zero on entry
+    uint32_t* ticket;      // zero on entry
+    int32_t* status;
+    int T, k, E, d, n_seg, tokens_per_tile, n_tiles;
+};
+
+int permute_tokens_per_tile(int k);
+int permute_n_tiles(int T, int k);
+size_t permute_ws_bytes(int T, int k, int E);
+
+cudaError_t launch_histogram(const int32_t* ids, int n_pairs, int E, int32_t* counts, int num_sms,
+                             cudaStream_t stream);
+cudaError_t launch_segments(const int32_t* counts, int E, int capacity, int32_t* seg_expert, int32_t* seg_offsets,
+                            int32_t* seg_first_rank, cudaStream_t stream);
+cudaError_t launch_plan(const int32_t* counts, int E, int R, int S, int k, int B, int32_t* seg_expert,
+                        int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* status, cudaStream_t stream);
+cudaError_t launch_permute(const PermuteArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                                     int num_sms, cudaStream_t stream);
+
+// combine.cu
+cudaError_t launch_combine(const __nv_bfloat16* yp, const int32_t* dest, const float* w, int T, int k, int d,
+                           __nv_bfloat16* out, int num_sms, cudaStream_t stream);
+
+}  // namespace moe

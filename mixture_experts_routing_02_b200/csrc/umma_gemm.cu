@@ -1,0 +1,364 @@
+// Grouped GEMM on the 5th-generation tensor cores (tcgen05 / TMEM / TMA).
+//
+// One persistent kernel template serves three contractions of the layer:
+//   * the router projection logits = X W_r^T, with top-k and the softmax over
+//     the selected logits fused into the epilogue ("Sparsely-Gated MoE 구현
+//     관점에서 살펴보기", sections "순전파 과정 ..." and "Top-2 라우팅의 수치 예시");
+//   * the gate and up projections of every expert in one launch, with SwiGLU
+//     fused into the epilogue ("5.3 Expert Parallelism", section "3. 고도화된
+//     최적화: 오버래핑(Overlapping) 및 GroupGEMM"; MoonEP page "설치 및 통합":
+//     the grouped GEMM selects each expert's rows through cu_seqlens);
+//   * the down projection of every expert.
+//
+// Rows come in segments (rows [off[s], off[s+1]) use expert seg_expert[s]);
+// the segment table is read on the device, so token counts never go back to
+// the host.  The work unit is a 128-row x BN-column output tile; tiles are
+// ordered segment-major, then by column tile, then by row tile, so the CTAs
+// running at the same moment share the same expert weight tile through L2
+// and each expert's weights cross HBM about once.
+//
+// CTA layout (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A tile [128 x 64] and B tile [N x 64] per stage
+//   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
+//               (M=128, N=mma_n, K=16, bf16 x bf16 -> fp32) and commits
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one row per thread),
+//               fused math, direct 16-byte stores of the valid rows
+// Two accumulator buffers (columns [0,256) and [256,512)) let the epilogue of
+// one tile overlap the main loop of the next.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kUmmaK = 16;
+constexpr int kMaxStages = 8;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccStride = 256;
+constexpr uint32_t kABytes = kBM * kBK * 2;
+
+struct TileCoord {
+    int seg, m, n, row0, row_end, expert;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(int tile, const int* prefix, int n_seg, int n_tiles_n,
+                                                 const GemmArgs& g) {
+    const int key = tile / n_tiles_n;
+    int lo = 0, hi = n_seg;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= key) lo = mid; else hi = mid;
+    }
+    TileCoord c;
+    c.seg = lo;
+    const int mt = prefix[lo + 1] - prefix[lo];
+    const int local = tile - prefix[lo] * n_tiles_n;
+    c.n = local / mt;
+    c.m = local - c.n * mt;
+    const int start = g.seg_offsets ? __ldg(g.seg_offsets + lo) : 0;
+    c.row_end = g.seg_offsets ? __ldg(g.seg_offsets + lo + 1) : g.M;
+    c.row0 = start + c.m * kBM;
+    c.expert = g.seg_expert ? __ldg(g.seg_expert + lo) : 0;
+    return c;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                     const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
+    __shared__ __align__(8) uint64_t full_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+    __shared__ int tile_prefix[kMaxSegments + 1];
+    extern __shared__ uint8_t dsmem[];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int stages = g.stages;
+    const uint32_t b_stage_bytes = static_cast<uint32_t>(g.mma_n) * 128u;
+
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + stages * kABytes;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull_bar[b], 1);
+            mbar_init(&tempty_bar[b], 4);
+        }
+        mbar_init(&drain_bar, 1);
+        abort_sh = 0;
+        mbar_fence_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB0);
+        if (EPI == kEpiSwiglu) tma_prefetch_desc(&tmB1);
+    }
+    if (warp == 1) tmem_alloc(&tmem_base_sh, kTmemCols);
+    if (warp == 2) {
+        // cumulative row-tile count of the segments (empty / unused segments have none)
+        int carry = 0;
+        for (int b = 0; b < g.n_seg; b += 32) {
+            const int s = b + lane;
+            int mt = 0;
+            if (s < g.n_seg) {
+                const int a = g.seg_offsets ? __ldg(g.seg_offsets + s) : 0;
+                const int e = g.seg_offsets ? __ldg(g.seg_offsets + s + 1) : g.M;
+                const bool live = (g.seg_expert == nullptr) || __ldg(g.seg_expert + s) >= 0;
+                mt = (live && e > a) ? (e - a + kBM - 1) / kBM : 0;
+            }
+            int v = mt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += t;
+            }
+            if (s < g.n_seg) tile_prefix[s] = carry + v - mt;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (lane == 0) tile_prefix[g.n_seg] = carry;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = tmem_base_sh;
+    const int total = tile_prefix[g.n_seg] * g.n_tiles_n;
+    const int nkb = g.K / kBK;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0, issued = 0;
+            uint32_t phase = 0;
+            const uint32_t tx = kABytes + (EPI == kEpiRoute ? static_cast<uint32_t>(g.N) * 128u : b_stage_bytes);
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g);
+                const int n0 = c.n * g.BN;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, g.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full_bar[stage], tx);
+                    uint8_t* a_dst = sA + stage * kABytes;
+                    uint8_t* b_dst = sB + stage * b_stage_bytes;
+                    tma_load_2d(a_dst, &tmA, kb * kBK, c.row0, &full_bar[stage]);
+                    if (EPI == kEpiRoute) {
+                        tma_load_2d(b_dst, &tmB0, kb * kBK, 0, &full_bar[stage]);
+                    } else if (EPI == kEpiSwiglu) {
+                        tma_load_3d(b_dst, &tmB0, kb * kBK, n0, c.expert, &full_bar[stage]);
+                        tma_load_3d(b_dst + g.BN * 128, &tmB1, kb * kBK, n0, c.expert, &full_bar[stage]);
+                    } else {
+                        tma_load_3d(b_dst, &tmB0, kb * kBK, n0, c.expert, &full_bar[stage]);
+                    }
+                    ++issued;
+                    if (++stage == stages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok) {
+                // give every copy still in flight a bounded chance to land before the CTA exits
+                const int first = issued > stages ? issued - stages : 0;
+                for (int i = first; i < issued; ++i)
+                    mbar_wait(&full_bar[i % stages], static_cast<uint32_t>((i / stages) & 1), nullptr, nullptr);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            const uint32_t idesc = umma_idesc_bf16(kBM, g.mma_n);
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_sh, g.status)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kAccStride;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&full_bar[stage], phase, &abort_sh, g.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * kABytes));
+                    const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * b_stage_bytes));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                        // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4)
+                        umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&empty_bar[stage]);
+                    if (++stage == stages) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                umma_commit(&tfull_bar[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            // every MMA issued by this thread completes before tensor memory is released
+            umma_commit(&drain_bar);
+            mbar_wait(&drain_bar, 0, nullptr, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;  // a warp may only touch TMEM lanes [32*(warp%4), +32)
+        const int r_in_tile = quarter * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g);
+            const bool got = mbar_wait(&tfull_bar[acc], acc_phase, &abort_sh, g.status);
+            if (!__all_sync(0xffffffffu, got)) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(acc) * kAccStride;
+            const int row = c.row0 + r_in_tile;
+            const bool valid = row < c.row_end;
+            const int n0 = c.n * g.BN;
+
+            if (EPI == kEpiSwiglu) {
+                for (int cc = 0; cc < g.BN; cc += 32) {
+                    uint32_t gr[32], ur[32];
+                    tmem_ld32(t_row + cc, gr);
+                    tmem_ld32(t_row + g.BN + cc, ur);
+                    tmem_ld_wait();
+                    if (valid && n0 + cc < g.N) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float g0 = __uint_as_float(gr[2 * i]), g1 = __uint_as_float(gr[2 * i + 1]);
+                            const float u0 = __uint_as_float(ur[2 * i]), u1 = __uint_as_float(ur[2 * i + 1]);
+                            const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                            const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                            pk[i] = pack_bf16x2(h0, h1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(g.out + static_cast<size_t>(row) * g.ldo + n0 + cc);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    }
+                }
+            } else if (EPI == kEpiStore) {
+                for (int cc = 0; cc < g.BN; cc += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(t_row + cc, r);
+                    tmem_ld_wait();
+                    if (valid && n0 + cc < g.N) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        uint4* dst = reinterpret_cast<uint4*>(g.out + static_cast<size_t>(row) * g.ldo + n0 + cc);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    }
+                }
+            } else {
+                // router: top-k over the E logits of this row, softmax over the selected ones
+                float tv[kMaxTopK];
+                int ti[kMaxTopK];
+#pragma unroll
+                for (int j = 0; j < kMaxTopK; ++j) { tv[j] = -INFINITY; ti[j] = 0x7fffffff; }
+                for (int cc = 0; cc < g.N; cc += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(t_row + cc, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int e = cc + i;
+                        if (e < g.N) {
+                            float v = __uint_as_float(r[i]);
+                            if (g.bias != nullptr) v += __ldg(g.bias + e);
+                            if (valid && g.logits != nullptr) g.logits[static_cast<size_t>(row) * g.N + e] = v;
+                            // insertion into the sorted list; strict '>' keeps the lower id on ties
+                            float cv = v;
+                            int ci = e;
+#pragma unroll
+                            for (int j = 0; j < kMaxTopK; ++j) {
+                                const bool gt = cv > tv[j];
+                                const float ov = tv[j];
+                                const int oi = ti[j];
+                                tv[j] = gt ? cv : ov;
+                                ti[j] = gt ? ci : oi;
+                                cv = gt ? ov : cv;
+                                ci = gt ? oi : ci;
+                            }
+                        }
+                    }
+                }
+                if (valid) {
+                    float ex[kMaxTopK];
+                    float sum = 0.f;
+#pragma unroll
+                    for (int j = 0; j < kMaxTopK; ++j) {
+                        ex[j] = (j < g.k) ? expf(tv[j] - tv[0]) : 0.f;
+                        sum += ex[j];
+                    }
+                    const float inv = 1.0f / sum;
+#pragma unroll
+                    for (int j = 0; j < kMaxTopK; ++j) {
+                        if (j < g.k) {
+                            g.topk_ids[static_cast<size_t>(row) * g.k + j] = ti[j];
+                            g.topk_w[static_cast<size_t>(row) * g.k + j] = ex[j] * inv;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace
+
+size_t gemm_smem_bytes(int stages, int mma_n) {
+    return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(mma_n) * 128u);
+}
+
+int gemm_pick_stages(int mma_n) {
+    const size_t per = kABytes + static_cast<size_t>(mma_n) * 128u;
+    int s = static_cast<int>((kGemmSmemBudget - 1024) / per);
+    if (s > kMaxStages) s = kMaxStages;
+    return s;
+}
+
+template <int EPI>
+static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmArgs& g,
+                              int grid, cudaStream_t stream) {
+    auto kern = umma_gemm_kernel<EPI>;
+    size_t smem = gemm_smem_bytes(g.stages, g.mma_n);
+    if (smem < kGemmSmemMin) smem = kGemmSmemMin;  // keeps one CTA per SM (all TMEM columns are taken)
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    kern<<<grid, kThreads, smem, stream>>>(a, b0, b1, g);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                             const GemmArgs& g, int grid, cudaStream_t stream) {
+    switch (epi) {
+        case kEpiRoute: return launch_one<kEpiRoute>(a, b0, b1, g, grid, stream);
+        case kEpiSwiglu: return launch_one<kEpiSwiglu>(a, b0, b1, g, grid, stream);
+        default: return launch_one<kEpiStore>(a, b0, b1, g, grid, stream);
+    }
+}
+
+}  // namespace moe

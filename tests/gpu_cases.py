@@ -1,0 +1,126 @@
+"""Helpers of the GPU parity tests: seeded inputs (with the top-k margin rule),
+device buffers, the tolerance of floating-point outputs, and the oracle side
+of each comparison.  Imported only by tests."""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+import torch
+
+import oracle
+import mixture_experts_routing_02_b200 as moe
+from mixture_experts_routing_02_b200 import synthetic as syn
+
+# Floating-point outputs (bf16 in, fp32 accumulate, bf16 out) against the fp64 oracle:
+# max-abs error <= 2e-2 * RMS(reference) and mean relative error (sum|err| / sum|ref|) <= 5e-3.
+MAX_ABS_OF_RMS = 2e-2
+MEAN_REL = 5e-3
+
+
+def check_close(got, ref, what="", max_abs_of_rms=MAX_ABS_OF_RMS, mean_rel=MEAN_REL):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    if ref.size == 0:
+        return
+    err = np.abs(got - ref)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    denom = float(np.abs(ref).sum())
+    max_abs = float(err.max())
+    rel = float(err.sum()) / denom if denom > 0 else float(err.sum())
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    assert max_abs <= max_abs_of_rms * max(rms, 1e-30), f"{what}: max-abs {max_abs:.3e} > {max_abs_of_rms} * rms {rms:.3e}"
+    assert rel <= mean_rel, f"{what}: mean-rel {rel:.3e} > {mean_rel}"
+
+
+def capacity_rows(w: syn.Workload) -> int:
+    return oracle.capacity_rows(w.capacity_factor, w.T, w.k, w.E)
+
+
+def moe_shape(w: syn.Workload, capacity: Optional[int] = None):
+    C = capacity_rows(w) if capacity is None else capacity
+    return moe.shape(w.T, w.d, w.E, w.k, w.F, capacity=C, n_groups=w.n_groups, replica_slots=w.replica_slots)
+
+
+@dataclasses.dataclass
+class Case:
+    w: syn.Workload
+    x: torch.Tensor        # CPU bf16, margin-enforced
+    w_r: torch.Tensor      # CPU bf16
+    bias: Optional[torch.Tensor]
+    wg: torch.Tensor       # bf16 on `weights_device`
+    wu: torch.Tensor
+    wd: torch.Tensor
+
+
+def make_case(w: syn.Workload, seed: int = 0, weights_device="cpu", margin=True) -> Case:
+    x, w_r, bias = syn.router_inputs(w, seed)
+    if margin and w.E > 1:
+        oracle.enforce_margin(x, w_r, bias, w.k, lambda t, a: syn.x_row_redraw(w, seed, t, a))
+    wg, wu, wd = syn.expert_weights(w, seed, device=weights_device)
+    return Case(w, x, w_r, bias, wg, wu, wd)
+
+
+def dev(t, device="cuda"):
+    return None if t is None else t.to(device).contiguous()
+
+
+def i32(n, device="cuda"):
+    return torch.zeros(max(int(n), 1), dtype=torch.int32, device=device)
+
+
+def to_np(t):
+    if t.dtype == torch.bfloat16:
+        t = t.float()
+    return t.detach().cpu().numpy()
+
+
+def run_layer(case: Case, capacity=None, stream=None):
+    """moe_layer_fwd through the C ABI; returns the output and every intermediate (CPU)."""
+    w = case.w
+    s = moe_shape(w, capacity)
+    n_seg, rows = moe.moe_layout(s)
+    _, layer_bytes = moe.moe_workspace_size(s)
+    ws = torch.empty(layer_bytes, dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full((w.T, w.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    x, w_r, bias = dev(case.x), dev(case.w_r), dev(case.bias)
+    wg, wu, wd = dev(case.wg), dev(case.wu), dev(case.wd)
+    moe.moe_layer_fwd(s, x, w_r, bias, wg, wu, wd, out, status, ws, stream=stream)
+    torch.cuda.synchronize()
+    v = moe.moe_layer_views(s, ws)
+
+    def view(addr, n, dtype, shape=None):
+        base = ws.data_ptr()
+        off = addr - base
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        t = ws[off:off + nbytes].view(dtype)
+        return t.view(*shape) if shape else t
+
+    T, k = w.T, w.k
+    res = dict(
+        out=out, status=int(status.item()), n_seg=n_seg, rows=rows, ws=ws, x_dev=x,
+        ids=view(v.topk_ids, T * k, torch.int32, (T, k)).cpu(),
+        w=view(v.topk_w, T * k, torch.float32, (T, k)).cpu(),
+        counts=view(v.counts, w.E, torch.int32).cpu(),
+        seg_expert=view(v.seg_expert, n_seg, torch.int32).cpu(),
+        seg_offsets=view(v.seg_offsets, n_seg + 1, torch.int32).cpu(),
+        seg_first_rank=view(v.seg_first_rank, n_seg, torch.int32).cpu(),
+        dest=view(v.dest, T * k, torch.int32).cpu(),
+        src=view(v.src, rows, torch.int32).cpu(),
+        xp=view(v.xp, rows * w.d, torch.bfloat16, (rows, w.d)),
+        hp=view(v.hp, rows * w.F, torch.bfloat16, (rows, w.F)),
+        yp=view(v.yp, rows * w.d, torch.bfloat16, (rows, w.d)),
+    )
+    return res
+
+
+def oracle_segments(case: Case, counts, capacity=None):
+    w = case.w
+    if w.n_groups:
+        segs, _ = oracle.balanced_plan(counts, w.n_groups, w.T // w.n_groups, w.k, w.replica_slots)
+    else:
+        segs = oracle.plain_segments(counts, capacity_rows(w) if capacity is None else capacity)
+    return segs

@@ -1,0 +1,131 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+call the header declares, validates its arguments before touching CUDA, and
+sizes its buffers as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_routing_02_b200 as moe
+from mixture_experts_routing_02_b200 import synthetic as syn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+INCLUDE = os.path.join(ROOT, "include")
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(INCLUDE):
+        if fn.endswith(".h"):
+            with open(os.path.join(INCLUDE, fn)) as f:
+                names |= set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", f.read()))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(moe.LIB_PATH):
+        from mixture_experts_routing_02_b200 import build
+        build.build()
+    return moe.load_library()
+
+
+def test_header_declares_the_boundary_calls():
+    names = _declared_symbols()
+    for required in ("moe_route", "moe_plan_balanced", "moe_dispatch", "moe_expert_ffn", "moe_combine",
+                     "moe_layer_fwd"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_symbols()
+    assert names, "no MOE_API declarations found"
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(moe.SYMBOLS) <= names | {"moe_status_string"}
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert moe.moe_status_string(code).startswith("MOE_")
+
+
+def _shape(**kw):
+    base = dict(T=64, d_model=128, n_experts=8, top_k=2, d_ff=256)
+    base.update(kw)
+    return moe.shape(**base)
+
+
+def test_layout_plain_and_capacity(lib):
+    assert moe.moe_layout(_shape()) == (8, 128)
+    w = syn.SKEWED
+    C = 320  # ceil(1.25 * 8192 * 2 / 64)
+    s = moe.shape(w.T, w.d, w.E, w.k, w.F, capacity=C)
+    assert moe.moe_layout(s) == (64, min(w.T * w.k, C * w.E))
+    s = moe.shape(10, 64, 4, 2, 64, capacity=1)
+    assert moe.moe_layout(s) == (4, 4)
+
+
+def test_layout_balanced_plan(lib):
+    w = syn.BALANCED
+    s = moe.shape(w.T, w.d, w.E, w.k, w.F, n_groups=w.n_groups, replica_slots=w.replica_slots)
+    assert moe.moe_layout(s) == (8 * (256 // 8 + 32), w.T * w.k)
+
+
+def test_dispatch_buffer_matches_moonep_memory_table(lib):
+    """MoonEP page, "실제 실험 결과" memory table: the dispatch buffer of one rank
+    with S=4096, H=7168, K=8 is 0.44 GiB (S*K rows of H bf16 = 0.4375 GiB)."""
+    s = moe.shape(4096, 7168, 256, 8, 2048)
+    _, rows = moe.moe_layout(s)
+    assert rows * 7168 * 2 == 0.4375 * (1 << 30)
+    assert round(rows * 7168 * 2 / (1 << 30), 2) == 0.44
+
+
+def test_workspace_sizes_grow_with_the_layer(lib):
+    small = moe.moe_workspace_size(_shape())
+    big = moe.moe_workspace_size(_shape(T=4096))
+    assert 0 < small[0] < big[0] and 0 < small[1] < big[1]
+    # the layer workspace holds at least Xp, Hp and Yp
+    T, d, k, F = 4096, 128, 2, 256
+    assert big[1] >= T * k * (2 * d + F) * 2
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=-1), 1), (dict(top_k=9, n_experts=8), 1), (dict(top_k=0), 1), (dict(n_experts=0), 1),
+    (dict(n_groups=3), 1), (dict(n_groups=2, capacity=4), 1), (dict(capacity=-2), 1),
+    (dict(n_experts=300, top_k=2), 2), (dict(d_model=100), 2), (dict(d_ff=96), 2),
+    (dict(n_experts=16, top_k=9), 2), (dict(T=1 << 29, top_k=2), 2),
+    (dict(n_experts=256, n_groups=2, replica_slots=1000, T=64), 2),
+])
+def test_shape_validation(lib, kw, code):
+    s = _shape(**kw)
+    n_seg, rows = ctypes.c_int32(), ctypes.c_int32()
+    assert lib.moe_layout(ctypes.byref(s), ctypes.byref(n_seg), ctypes.byref(rows)) == code
+
+
+def test_null_pointers_rejected_before_any_cuda_call(lib):
+    s = _shape()
+    assert lib.moe_route(ctypes.byref(s), None, None, None, None, None, None, None, None) == 1
+    assert lib.moe_combine(ctypes.byref(s), None, None, None, None, None) == 1
+    assert lib.moe_expert_ffn(ctypes.byref(s), *([None] * 10)) == 1
+    assert lib.moe_plan_balanced(ctypes.byref(s), None, None, None, None, None, None) == 1  # no groups
+
+
+def test_small_workspace_rejected(lib):
+    s = _shape()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check comes first
+    args = [fake] * 9
+    rc = lib.moe_dispatch(ctypes.byref(s), fake, fake, 0, *args[:7], fake, fake, 16, None)
+    assert rc == 3
+    rc = lib.moe_layer_fwd(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, None, fake, 16, None)
+    assert rc == 3
+
+
+def test_misaligned_workspace_rejected(lib):
+    s = _shape()
+    fake = ctypes.c_void_p(1 << 20)
+    need = moe.moe_workspace_size(s)[1]
+    rc = lib.moe_layer_fwd(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, None,
+                           ctypes.c_void_p((1 << 20) + 64), need, None)
+    assert rc == 3

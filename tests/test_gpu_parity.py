@@ -1,0 +1,238 @@
+"""GPU-vs-oracle parity of every C-ABI call on small, ragged and degenerate
+cases (the oracle finishes each in seconds; the cases span several tiles and
+leave ragged tails).  Integer and index outputs must match bit for bit;
+floating-point outputs must meet the tolerance in ``gpu_cases.check_close``.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import mixture_experts_routing_02_b200 as moe
+from mixture_experts_routing_02_b200 import synthetic as syn
+
+from gpu_cases import (Case, check_close, dev, i32, make_case, moe_shape, oracle_segments, run_layer,
+                       to_np)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    syn.TINY,
+    syn.Workload("ragged", T=300, d=192, E=6, k=2, F=320, zipf_s=1.2),
+    syn.Workload("many-experts", T=333, d=256, E=64, k=8, F=128),
+    syn.Workload("capacity", T=500, d=128, E=16, k=2, F=192, zipf_s=1.2, capacity_factor=1.0),
+    syn.Workload("capacity-1", T=40, d=64, E=4, k=2, F=64, capacity_factor=0.05),
+    syn.Workload("plan", T=512, d=128, E=16, k=4, F=128, zipf_s=1.2, n_groups=4, replica_slots=8),
+    syn.Workload("dense-e1k1", T=130, d=64, E=1, k=1, F=64),
+    syn.Workload("k-equals-e", T=77, d=128, E=8, k=8, F=128),
+    syn.Workload("one-token", T=1, d=64, E=4, k=2, F=64),
+    syn.Workload("multi-tile", T=1000, d=512, E=4, k=2, F=512, zipf_s=0.5),
+    syn.Workload("wide-router", T=260, d=128, E=256, k=6, F=64),
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_ok):
+    moe.load_library()
+
+
+def _oracle_layer(case: Case):
+    w = case.w
+    C = oracle.capacity_rows(w.capacity_factor, w.T, w.k, w.E)
+    return oracle.layer_forward(case.x, case.w_r, case.bias, case.wg, case.wu, case.wd, w.k,
+                                capacity=C, n_groups=w.n_groups, replica_slots=w.replica_slots)
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_layer_matches_oracle(w):
+    case = make_case(w, seed=1)
+    ref = _oracle_layer(case)
+    got = run_layer(case)
+    assert got["status"] == 0
+    # routing: ids bit-exact, weights to fp32 accuracy
+    assert (got["ids"].numpy() == ref.ids).all(), "top-k ids differ"
+    assert np.abs(got["w"].numpy() - ref.weights).max() < 1e-4
+    # dispatch: counts, segment tables, positions bit-exact
+    assert (got["counts"].numpy() == ref.counts).all()
+    assert (got["seg_expert"].numpy() == ref.segs.expert).all()
+    assert (got["seg_offsets"].numpy() == ref.segs.offsets).all()
+    assert (got["seg_first_rank"].numpy() == ref.segs.first_rank).all()
+    assert (got["dest"].numpy() == ref.dest).all()
+    used = int(ref.segs.offsets[-1])
+    assert (got["src"].numpy()[:used] == ref.src).all()
+    # permuted rows are exact copies
+    assert (to_np(got["xp"][:used]) == ref.xp).all()
+    # expert FFN and combine within tolerance of the fp64 oracle
+    check_close(to_np(got["hp"][:used]), ref.hp, "Hp")
+    check_close(to_np(got["yp"][:used]), ref.yp, "Yp")
+    check_close(to_np(got["out"]), ref.out, "out")
+
+
+def test_route_logits_and_bias():
+    w = syn.Workload("route", T=333, d=320, E=40, k=5, F=64, zipf_s=1.2)
+    case = make_case(w, seed=2)
+    s = moe_shape(w)
+    logits = torch.empty(w.T, w.E, device="cuda")
+    ids = i32(w.T * w.k).view(w.T, w.k)
+    wt = torch.empty(w.T, w.k, device="cuda")
+    st = i32(1)
+    moe.moe_route(s, dev(case.x), dev(case.w_r), dev(case.bias), logits, ids, wt, st)
+    torch.cuda.synchronize()
+    l64, rid, rw = oracle.route(case.x, case.w_r, case.bias, w.k)
+    check_close(to_np(logits), l64, "logits", max_abs_of_rms=1e-4, mean_rel=1e-5)
+    assert (ids.cpu().numpy() == rid).all()
+    assert np.abs(wt.cpu().numpy() - rw).max() < 1e-4
+    assert st.item() == 0
+
+
+def test_route_from_logits_ties_and_exact_decision():
+    T, E, k = 97, 37, 6
+    rng = np.random.default_rng(5)
+    l = rng.normal(size=(T, E)).astype(np.float32)
+    l[:, 7] = l[:, 3]            # exact ties: the lower id must come first
+    l[:10, :] = 1.0              # rows of all-equal logits
+    l[10, :] = np.float32(-3.0)
+    l[10, 20] = 2.0
+    s = moe.shape(T, 64, E, k, 64)
+    ids = i32(T * k).view(T, k)
+    wt = torch.empty(T, k, device="cuda")
+    moe.moe_route_from_logits(s, torch.from_numpy(l).cuda(), ids, wt)
+    torch.cuda.synchronize()
+    l64 = l.astype(np.float64)
+    rid = oracle.topk_ids(l64, k)
+    assert (ids.cpu().numpy() == rid).all()
+    assert np.abs(wt.cpu().numpy() - oracle.topk_weights(l64, rid)).max() < 1e-6
+    assert list(ids.cpu().numpy()[0]) == list(range(k))
+
+
+def test_worked_example_on_the_gpu():
+    """The worked top-2 example (E4 = 2.0, E6 = 1.6 -> ids 3, 5, weights 0.599 / 0.401)."""
+    l = np.array([[0.3, -1.2, 1.5, 2.0, -0.4, 1.6, 0.9, -2.1]], dtype=np.float32)
+    s = moe.shape(1, 64, 8, 2, 64)
+    ids = i32(2).view(1, 2)
+    wt = torch.empty(1, 2, device="cuda")
+    moe.moe_route_from_logits(s, torch.from_numpy(l).cuda(), ids, wt)
+    torch.cuda.synchronize()
+    assert ids.cpu().tolist() == [[3, 5]]
+    assert np.round(wt.cpu().numpy()[0], 3).tolist() == [0.599, 0.401]
+
+
+@pytest.mark.parametrize("sigma", [0.0, 1.0, 5.0])
+def test_histogram_segments_and_plan_on_given_ids(sigma):
+    E, R, S, k, B = 64, 4, 300, 4, 16
+    T = R * S
+    ids = syn.lognormal_topk_ids(E, T, k, sigma, seed=3)
+    counts_ref = oracle.histogram(ids.numpy(), E)
+    s = moe.shape(T, 64, E, k, 64, n_groups=R, replica_slots=B)
+    counts = i32(E)
+    moe.moe_histogram(s, ids.cuda(), counts)
+    n_seg, rows = moe.moe_layout(s)
+    se, so, sf = i32(n_seg), i32(n_seg + 1), i32(n_seg)
+    st = i32(1)
+    moe.moe_plan_balanced(s, counts, se, so, sf, st)
+    torch.cuda.synchronize()
+    assert (counts.cpu().numpy() == counts_ref).all()
+    segs, _ = oracle.balanced_plan(counts_ref, R, S, k, B)
+    assert st.item() == 0
+    assert (se.cpu().numpy() == segs.expert).all()
+    assert (so.cpu().numpy() == segs.offsets).all()
+    assert (sf.cpu().numpy() == segs.first_rank).all()
+    # plain segments with a capacity
+    s2 = moe.shape(T, 64, E, k, 64, capacity=40)
+    se2, so2, sf2 = i32(E), i32(E + 1), i32(E)
+    moe.moe_segments(s2, counts, se2, so2, sf2)
+    torch.cuda.synchronize()
+    ref2 = oracle.plain_segments(counts_ref, 40)
+    assert (so2.cpu().numpy() == ref2.offsets).all() and (se2.cpu().numpy() == ref2.expert).all()
+
+
+def test_dispatch_with_given_plan_tables():
+    """plan_ready = 1: the permutation alone, on counts and tables from the oracle."""
+    E, R, S, k, B, d = 32, 4, 200, 4, 8, 128
+    T = R * S
+    ids = syn.lognormal_topk_ids(E, T, k, 2.0, seed=4)
+    counts_ref = oracle.histogram(ids.numpy(), E)
+    segs, _ = oracle.balanced_plan(counts_ref, R, S, k, B)
+    dest_ref, src_ref = oracle.dispatch_positions(ids.numpy(), segs, E)
+    x = torch.randn(T, d).to(torch.bfloat16)
+    s = moe.shape(T, d, E, k, 64, n_groups=R, replica_slots=B)
+    n_seg, rows = moe.moe_layout(s)
+    ws = torch.empty(moe.moe_workspace_size(s)[0], dtype=torch.uint8, device="cuda")
+    dest, src = i32(T * k), i32(rows)
+    xp = torch.zeros(rows, d, dtype=torch.bfloat16, device="cuda")
+    to_i32 = lambda a: torch.from_numpy(np.asarray(a, dtype=np.int32)).cuda()
+    st = i32(1)
+    moe.moe_dispatch(s, x.cuda(), ids.cuda(), 1, to_i32(counts_ref), to_i32(segs.expert), to_i32(segs.offsets),
+                     to_i32(segs.first_rank), dest, src, xp, st, ws)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert (dest.cpu().numpy() == dest_ref).all()
+    assert (src.cpu().numpy() == src_ref).all()
+    assert (to_np(xp) == oracle.permute_rows(x, src_ref, k)).all()
+
+
+def test_expert_ffn_on_given_rows():
+    w = syn.Workload("ffn", T=400, d=256, E=5, k=2, F=384, zipf_s=1.0)
+    case = make_case(w, seed=6)
+    ref = oracle.layer_forward(case.x, case.w_r, case.bias, case.wg, case.wu, case.wd, w.k)
+    s = moe_shape(w)
+    n_seg, rows = moe.moe_layout(s)
+    xp = torch.from_numpy(ref.xp.astype(np.float32)).to(torch.bfloat16).cuda()
+    to_i32 = lambda a: torch.from_numpy(np.asarray(a, dtype=np.int32)).cuda()
+    hp = torch.empty(rows, w.F, dtype=torch.bfloat16, device="cuda")
+    yp = torch.empty(rows, w.d, dtype=torch.bfloat16, device="cuda")
+    st = i32(1)
+    moe.moe_expert_ffn(s, xp, to_i32(ref.segs.expert), to_i32(ref.segs.offsets), dev(case.wg), dev(case.wu),
+                       dev(case.wd), hp, yp, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    check_close(to_np(hp), ref.hp, "Hp")
+    check_close(to_np(yp), ref.yp, "Yp")
+
+
+def test_combine_on_given_rows():
+    T, k, d, E = 300, 4, 192, 8
+    ids = syn.lognormal_topk_ids(E, T, k, 1.0, seed=7).numpy()
+    counts = oracle.histogram(ids, E)
+    segs = oracle.plain_segments(counts, 120)     # drops some pairs
+    dest, src = oracle.dispatch_positions(ids, segs, E)
+    rows = int(segs.offsets[-1])
+    yp = torch.randn(rows, d).to(torch.bfloat16)
+    wts = torch.rand(T, k)
+    ref = oracle.combine(oracle.f64(yp), dest, oracle.f64(wts), T, k)
+    s = moe.shape(T, d, E, k, 64, capacity=120)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(s, yp.cuda(), torch.from_numpy(dest.astype(np.int32)).cuda(), wts.cuda(), out)
+    torch.cuda.synchronize()
+    # only fp32 accumulation and one bf16 rounding separate the two
+    check_close(to_np(out), ref, "out", max_abs_of_rms=2e-2, mean_rel=3e-3)
+    dropped_all = (dest.reshape(T, k) < 0).all(axis=1)
+    assert (to_np(out)[dropped_all] == 0).all()
+
+
+def test_infeasible_plan_reports_and_moves_nothing():
+    w = syn.Workload("infeasible", T=256, d=64, E=8, k=1, F=64, zipf_s=3.0, n_groups=4, replica_slots=0)
+    case = make_case(w, seed=8)
+    got = run_layer(case)
+    assert got["status"] & moe.DEV_ERR_PLAN
+    assert (got["dest"].numpy() == -1).all()
+    assert (got["seg_offsets"].numpy() == 0).all()
+    assert (to_np(got["out"]) == 0).all()
+    with pytest.raises(oracle.PlanInfeasible):
+        oracle.balanced_plan(oracle.histogram(got["ids"].numpy(), 8), 4, 64, 1, 0)
+
+
+def test_zero_tokens_is_a_no_op():
+    s = moe.shape(0, 128, 8, 2, 256)
+    ws = torch.empty(max(moe.moe_workspace_size(s)[1], 256), dtype=torch.uint8, device="cuda")
+    dummy = torch.zeros(256, dtype=torch.bfloat16, device="cuda")
+    moe.moe_layer_fwd(s, dummy, dummy, None, dummy, dummy, dummy, dummy, None, ws)
+    torch.cuda.synchronize()
+
+
+def test_repeated_calls_are_deterministic():
+    case = make_case(SMALL[1], seed=9)
+    a = run_layer(case)
+    b = run_layer(case)
+    assert torch.equal(a["out"], b["out"]) and torch.equal(a["dest"], b["dest"])
+    assert torch.equal(a["hp"], b["hp"])
