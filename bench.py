@@ -255,8 +255,8 @@ def run_ours(args, w):
     bias = bias.to(dev) if bias is not None else None
     wg, wu, wd = syn.expert_weights(w, seed, device=dev)
     ws = torch.empty(layer_bytes, dtype=torch.uint8, device=dev)
-    out = torch.empty(w.T, w.d, dtype=torch.bfloat16, device=dev)
-    out_host = torch.empty(w.T, w.d, dtype=torch.bfloat16).pin_memory()
+    out = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
+    out_host = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     v = moe.moe_layer_views(s, ws)
@@ -276,7 +276,7 @@ def run_ours(args, w):
     src = view(v.src, rows_alloc, torch.int32)
     xp = view(v.xp, rows_alloc * w.d, torch.bfloat16)
     hp = view(v.hp, rows_alloc * w.F, torch.bfloat16)
-    yp = view(v.yp, rows_alloc * w.d, torch.bfloat16)
+    yp = view(v.yp, rows_alloc * w.d, torch.float32)
     dws = view(v.dispatch_ws, v.dispatch_ws_bytes, torch.uint8)
 
     def step(ev):
@@ -360,8 +360,8 @@ def run_ours(args, w):
     breakdown["gate_up"] = dict(ms=avg["gate_up"], flops=4 * rows_used * d * F,
                                 bytes=2 * active_experts * F * d * 2 + rows_used * d * 2 + rows_used * F * 2)
     breakdown["down"] = dict(ms=avg["down"], flops=2 * rows_used * d * F,
-                             bytes=active_experts * d * F * 2 + rows_used * F * 2 + rows_used * d * 2)
-    breakdown["combine"] = dict(ms=avg["combine"], bytes=rows_used * d * 2 + T * d * 2 + T * k * 8)
+                             bytes=active_experts * d * F * 2 + rows_used * F * 2 + rows_used * d * 4)
+    breakdown["combine"] = dict(ms=avg["combine"], bytes=rows_used * d * 4 + T * d * 4 + T * k * 8)
     for name, b in breakdown.items():
         sec = b["ms"] / 1e3
         if "flops" in b and name in ("gate_up", "down"):
@@ -393,7 +393,7 @@ def run_ours(args, w):
         "breakdown": {n: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in b.items()}
                       for n, b in breakdown.items()},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
-                "d2h_bytes_per_step": T * d * 2, "api": "moe_layer_fwd with pinned host X/out copies"},
+                "d2h_bytes_per_step": T * d * 4, "api": "moe_layer_fwd with pinned host X (bf16) / out (fp32) copies"},
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

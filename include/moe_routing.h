@@ -232,41 +232,44 @@ MOE_API moe_status_t moe_expert_gate_up(const moe_shape_t *shape, const moe_bf16
                                 int32_t *status, moe_stream_t stream);
 
 /*
- * Grouped down projection Yp[r, :] = Hp[r] W_d[e]^T (fp32 accumulate,
- * bf16 out).   hp [rows_alloc, F]; w_down [E, d, F]; yp [rows_alloc, d] out.
+ * Grouped down projection Yp[r, :] = Hp[r] W_d[e]^T, accumulated in fp32 and
+ * stored in fp32 (Yp is only read by the combine; keeping it in fp32 leaves
+ * one rounding, the bf16 Hp operand, between the expert and the output).
+ *   hp [rows_alloc, F] bf16; w_down [E, d, F] bf16; yp [rows_alloc, d] fp32 out.
  */
 MOE_API moe_status_t moe_expert_down(const moe_shape_t *shape, const moe_bf16_t *hp,
                              const int32_t *seg_expert, const int32_t *seg_offsets,
-                             const moe_bf16_t *w_down, moe_bf16_t *yp, int32_t *status,
+                             const moe_bf16_t *w_down, float *yp, int32_t *status,
                              moe_stream_t stream);
 
 /* moe_expert_gate_up then moe_expert_down. */
 MOE_API moe_status_t moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *xp, const int32_t *seg_expert,
                             const int32_t *seg_offsets, const moe_bf16_t *w_gate,
                             const moe_bf16_t *w_up, const moe_bf16_t *w_down, moe_bf16_t *hp,
-                            moe_bf16_t *yp, int32_t *status, moe_stream_t stream);
+                            float *yp, int32_t *status, moe_stream_t stream);
 
 /*
  * Combine ("Sparsely-Gated MoE 구현 관점에서 살펴보기", section "순전파 과정
  * ...", last step: un-permute and weight by the router; MoonEP page
  * "설치 및 통합": combine):
  *   out[t] = sum over j with dest[t*k+j] >= 0 of topk_w[t, j] * Yp[dest[t*k+j]]
- * accumulated in fp32 in ascending j, rounded to bf16.  A token whose pairs
- * were all dropped gets 0.
- *   yp [rows_alloc, d]; dest [T*k]; topk_w [T, k]; out [T, d] bf16.
+ * accumulated in fp32 in ascending j and stored in fp32 (the layer output is
+ * the combine's fp32 accumulator; rounding it to bf16 is left to the caller).
+ * A token whose pairs were all dropped gets 0.
+ *   yp [rows_alloc, d] fp32; dest [T*k]; topk_w [T, k]; out [T, d] fp32.
  */
-MOE_API moe_status_t moe_combine(const moe_shape_t *shape, const moe_bf16_t *yp, const int32_t *dest,
-                         const float *topk_w, moe_bf16_t *out, moe_stream_t stream);
+MOE_API moe_status_t moe_combine(const moe_shape_t *shape, const float *yp, const int32_t *dest,
+                         const float *topk_w, float *out, moe_stream_t stream);
 
 /*
  * The whole layer: moe_route (logits not stored) -> moe_dispatch ->
  * moe_expert_gate_up -> moe_expert_down -> moe_combine, all on `stream`.
- * The intermediates live in `ws` (moe_workspace_size()'s layer_bytes); their
- * addresses are given by moe_layer_views.
+ * out [T, d] fp32.  The intermediates live in `ws` (moe_workspace_size()'s
+ * layer_bytes); their addresses are given by moe_layer_views.
  */
 MOE_API moe_status_t moe_layer_fwd(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *w_router,
                            const float *bias, const moe_bf16_t *w_gate, const moe_bf16_t *w_up,
-                           const moe_bf16_t *w_down, moe_bf16_t *out, int32_t *status, void *ws,
+                           const moe_bf16_t *w_down, float *out, int32_t *status, void *ws,
                            size_t ws_bytes, moe_stream_t stream);
 
 /* Device addresses of the intermediates moe_layer_fwd keeps in its workspace. */
@@ -281,7 +284,7 @@ typedef struct {
     int32_t *src;            /* [rows_alloc] */
     moe_bf16_t *xp;          /* [rows_alloc, d] */
     moe_bf16_t *hp;          /* [rows_alloc, F] */
-    moe_bf16_t *yp;          /* [rows_alloc, d] */
+    float *yp;               /* [rows_alloc, d] fp32 */
     void *dispatch_ws;       /* moe_dispatch's own workspace */
     size_t dispatch_ws_bytes;
 } moe_layer_views_t;

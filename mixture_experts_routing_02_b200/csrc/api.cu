@@ -138,14 +138,14 @@ moe_status_t gate_up_impl(const Dims& v, const moe_bf16_t* xp, const int32_t* se
     GemmArgs g{};
     g.seg_offsets = seg_offsets; g.seg_expert = seg_expert; g.n_seg = v.n_seg; g.M = v.rows; g.K = v.d; g.N = v.F;
     g.BN = bn; g.n_tiles_n = (v.F + bn - 1) / bn; g.mma_n = 2 * bn; g.stages = gemm_pick_stages(2 * bn);
-    g.out = reinterpret_cast<__nv_bfloat16*>(hp); g.ldo = v.F; g.k = v.k; g.status = status;
+    g.out = hp; g.ldo = v.F; g.k = v.k; g.status = status;
     const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 128 + v.n_seg) * g.n_tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(sm_count(), max_tiles));
     return cuda_status(launch_umma_gemm(kEpiSwiglu, ta, tg, tu, g, grid, st));
 }
 
 moe_status_t down_impl(const Dims& v, const moe_bf16_t* hp, const int32_t* seg_expert, const int32_t* seg_offsets,
-                       const moe_bf16_t* wd, moe_bf16_t* yp, int32_t* status, cudaStream_t st) {
+                       const moe_bf16_t* wd, float* yp, int32_t* status, cudaStream_t st) {
     if (!hp || !seg_expert || !seg_offsets || !wd || !yp) return MOE_ERR_INVALID_ARG;
     if (!aligned16(hp) || !aligned16(wd) || !aligned16(yp)) return MOE_ERR_INVALID_ARG;
     if (v.T == 0 || v.rows == 0) return MOE_OK;
@@ -156,7 +156,7 @@ moe_status_t down_impl(const Dims& v, const moe_bf16_t* hp, const int32_t* seg_e
     GemmArgs g{};
     g.seg_offsets = seg_offsets; g.seg_expert = seg_expert; g.n_seg = v.n_seg; g.M = v.rows; g.K = v.F; g.N = v.d;
     g.BN = bn; g.n_tiles_n = (v.d + bn - 1) / bn; g.mma_n = bn; g.stages = gemm_pick_stages(bn);
-    g.out = reinterpret_cast<__nv_bfloat16*>(yp); g.ldo = v.d; g.k = v.k; g.status = status;
+    g.out = yp; g.ldo = v.d; g.k = v.k; g.status = status;
     const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 128 + v.n_seg) * g.n_tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(sm_count(), max_tiles));
     return cuda_status(launch_umma_gemm(kEpiStore, ta, tb, tb, g, grid, st));
@@ -219,7 +219,7 @@ LayerLayout layer_layout(const Dims& v) {
     L.dispatch_ws = o; o = align256(o + L.dispatch_ws_bytes);
     L.xp = o; o = align256(o + static_cast<size_t>(v.rows) * v.d * 2);
     L.hp = o; o = align256(o + static_cast<size_t>(v.rows) * v.F * 2);
-    L.yp = o; o = align256(o + static_cast<size_t>(v.rows) * v.d * 2);
+    L.yp = o; o = align256(o + static_cast<size_t>(v.rows) * v.d * 4);
     L.total = o;
     return L;
 }
@@ -324,7 +324,7 @@ moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* xp, 
 }
 
 moe_status_t moe_expert_down(const moe_shape_t* shape, const moe_bf16_t* hp, const int32_t* seg_expert,
-                             const int32_t* seg_offsets, const moe_bf16_t* w_down, moe_bf16_t* yp, int32_t* status,
+                             const int32_t* seg_offsets, const moe_bf16_t* w_down, float* yp, int32_t* status,
                              moe_stream_t stream) {
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
@@ -334,7 +334,7 @@ moe_status_t moe_expert_down(const moe_shape_t* shape, const moe_bf16_t* hp, con
 
 moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* xp, const int32_t* seg_expert,
                             const int32_t* seg_offsets, const moe_bf16_t* w_gate, const moe_bf16_t* w_up,
-                            const moe_bf16_t* w_down, moe_bf16_t* hp, moe_bf16_t* yp, int32_t* status,
+                            const moe_bf16_t* w_down, moe_bf16_t* hp, float* yp, int32_t* status,
                             moe_stream_t stream) {
     Dims v;
     moe_status_t s = check_shape(shape, &v);
@@ -345,15 +345,14 @@ moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* xp, cons
     return down_impl(v, hp, seg_expert, seg_offsets, w_down, yp, status, st);
 }
 
-moe_status_t moe_combine(const moe_shape_t* shape, const moe_bf16_t* yp, const int32_t* dest, const float* topk_w,
-                         moe_bf16_t* out, moe_stream_t stream) {
+moe_status_t moe_combine(const moe_shape_t* shape, const float* yp, const int32_t* dest, const float* topk_w,
+                         float* out, moe_stream_t stream) {
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(yp) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_combine(reinterpret_cast<const __nv_bfloat16*>(yp), dest, topk_w, v.T, v.k, v.d,
-                                      reinterpret_cast<__nv_bfloat16*>(out), sm_count(),
+    return cuda_status(launch_combine(yp, dest, topk_w, v.T, v.k, v.d, out, sm_count(),
                                       static_cast<cudaStream_t>(stream)));
 }
 
@@ -374,7 +373,7 @@ moe_status_t moe_layer_views(const moe_shape_t* shape, void* ws, moe_layer_views
     views->src = reinterpret_cast<int32_t*>(b + L.src);
     views->xp = reinterpret_cast<moe_bf16_t*>(b + L.xp);
     views->hp = reinterpret_cast<moe_bf16_t*>(b + L.hp);
-    views->yp = reinterpret_cast<moe_bf16_t*>(b + L.yp);
+    views->yp = reinterpret_cast<float*>(b + L.yp);
     views->dispatch_ws = b + L.dispatch_ws;
     views->dispatch_ws_bytes = L.dispatch_ws_bytes;
     return MOE_OK;
@@ -382,7 +381,7 @@ moe_status_t moe_layer_views(const moe_shape_t* shape, void* ws, moe_layer_views
 
 moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const moe_bf16_t* w_router,
                            const float* bias, const moe_bf16_t* w_gate, const moe_bf16_t* w_up,
-                           const moe_bf16_t* w_down, moe_bf16_t* out, int32_t* status, void* ws, size_t ws_bytes,
+                           const moe_bf16_t* w_down, float* out, int32_t* status, void* ws, size_t ws_bytes,
                            moe_stream_t stream) {
     Dims v;
     moe_status_t s = check_shape(shape, &v);
@@ -403,8 +402,7 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
     if (s != MOE_OK) return s;
     s = down_impl(v, w.hp, w.seg_expert, w.seg_offsets, w_down, w.yp, status, st);
     if (s != MOE_OK) return s;
-    return cuda_status(launch_combine(reinterpret_cast<const __nv_bfloat16*>(w.yp), w.dest, w.topk_w, v.T, v.k, v.d,
-                                      reinterpret_cast<__nv_bfloat16*>(out), sm_count(), st));
+    return cuda_status(launch_combine(w.yp, w.dest, w.topk_w, v.T, v.k, v.d, out, sm_count(), st));
 }
 
 }  // extern "C"

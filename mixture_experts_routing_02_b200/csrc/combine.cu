@@ -1,15 +1,15 @@
 // Combine: out[t] = sum_j w[t, j] * Yp[dest[t*k + j]] over the kept pairs,
-// accumulated in fp32 in ascending j and rounded to bf16 once.
+// accumulated in fp32 in ascending j; Yp and out are fp32.
 //
 // Sources: "Sparsely-Gated MoE 구현 관점에서 살펴보기", section "순전파 과정 ..."
 // (un-permute the expert outputs and combine them with the router weights);
 // the MoonEP page, section "설치 및 통합" (combine returns the tokens in their
 // original order).
 //
-// One warp per token: each lane owns 16-byte vectors of the row, issues the k
-// gathers of a vector before using any of them, and writes the result with one
-// 16-byte store.  The kernel is HBM-bound: it reads k rows and writes one row
-// per token.
+// One warp per token: each lane owns 16-byte vectors (4 floats) of the row,
+// issues the k gathers of a vector before using any of them, and writes the
+// result with one 16-byte store.  The kernel is HBM-bound: it reads k rows and
+// writes one row per token.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -17,13 +17,12 @@ namespace moe {
 
 namespace {
 
-__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ yp,
-                                                      const int32_t* __restrict__ dest,
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ dest,
                                                       const float* __restrict__ w, int T, int k, int d,
-                                                      __nv_bfloat16* __restrict__ out) {
+                                                      float* __restrict__ out) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
-    const int vec_per_row = d / 8;
+    const int vec_per_row = d / 4;  // float4 vectors
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
         int mine_d = -1;
         float mine_w = 0.f;
@@ -39,36 +38,31 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
             wr[j] = __shfl_sync(0xffffffffu, mine_w, j);
             if (j >= k) dr[j] = -1;
         }
-        uint4* orow = reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * d);
+        float4* orow = reinterpret_cast<float4*>(out + static_cast<size_t>(t) * d);
         for (int v = lane; v < vec_per_row; v += 32) {
-            uint4 val[kMaxTopK];
+            float4 val[kMaxTopK];
 #pragma unroll
             for (int j = 0; j < kMaxTopK; ++j)
-                if (dr[j] >= 0) val[j] = __ldg(reinterpret_cast<const uint4*>(yp + static_cast<size_t>(dr[j]) * d) + v);
-            float acc[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+                if (dr[j] >= 0) val[j] = __ldg(reinterpret_cast<const float4*>(yp + static_cast<size_t>(dr[j]) * d) + v);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int j = 0; j < kMaxTopK; ++j) {
                 if (dr[j] >= 0) {
-                    const uint32_t p[4] = {val[j].x, val[j].y, val[j].z, val[j].w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        acc[2 * i] = fmaf(wr[j], bf16_lo(p[i]), acc[2 * i]);
-                        acc[2 * i + 1] = fmaf(wr[j], bf16_hi(p[i]), acc[2 * i + 1]);
-                    }
+                    acc.x = fmaf(wr[j], val[j].x, acc.x);
+                    acc.y = fmaf(wr[j], val[j].y, acc.y);
+                    acc.z = fmaf(wr[j], val[j].z, acc.z);
+                    acc.w = fmaf(wr[j], val[j].w, acc.w);
                 }
             }
-            orow[v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                                 pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+            orow[v] = acc;
         }
     }
 }
 
 }  // namespace
 
-cudaError_t launch_combine(const __nv_bfloat16* yp, const int32_t* dest, const float* w, int T, int k, int d,
-                           __nv_bfloat16* out, int num_sms, cudaStream_t stream) {
+cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, int T, int k, int d, float* out,
+                           int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     int grid = (T + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;

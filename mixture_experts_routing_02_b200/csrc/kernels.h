@@ -28,7 +28,7 @@ struct GemmArgs {
     int n_tiles_n;  // column tiles
     int mma_n;      // UMMA N
     int stages;     // smem pipeline depth
-    __nv_bfloat16* out;
+    void* out;      // bf16 Hp (SwiGLU epilogue) or fp32 Yp (store epilogue)
     int ldo;
     const float* bias;
     float* logits;
@@ -77,7 +77,7 @@ cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, i
                                      int num_sms, cudaStream_t stream);
 
 // combine.cu
-cudaError_t launch_combine(const __nv_bfloat16* yp, const int32_t* dest, const float* w, int T, int k, int d,
-                           __nv_bfloat16* out, int num_sms, cudaStream_t stream);
+cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, int T, int k, int d, float* out,
+                           int num_sms, cudaStream_t stream);
 
 }  // namespace moe

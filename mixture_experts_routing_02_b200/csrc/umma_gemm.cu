@@ -240,24 +240,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
                             pk[i] = pack_bf16x2(h0, h1);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(g.out + static_cast<size_t>(row) * g.ldo + n0 + cc);
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
+                                                              static_cast<size_t>(row) * g.ldo + n0 + cc);
 #pragma unroll
                         for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                     }
                 }
             } else if (EPI == kEpiStore) {
+                // fp32 rows: the accumulator is stored as is
                 for (int cc = 0; cc < g.BN; cc += 32) {
                     uint32_t r[32];
                     tmem_ld32(t_row + cc, r);
                     tmem_ld_wait();
                     if (valid && n0 + cc < g.N) {
-                        uint32_t pk[16];
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(g.out) +
+                                                              static_cast<size_t>(row) * g.ldo + n0 + cc);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                        uint4* dst = reinterpret_cast<uint4*>(g.out + static_cast<size_t>(row) * g.ldo + n0 + cc);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        for (int v = 0; v < 8; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
                     }
                 }
             } else {

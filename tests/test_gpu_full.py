@@ -1,0 +1,93 @@
+"""Full-size parity: the four large workloads at their real sizes, run through
+moe_layer_fwd (the launch configuration the benchmark times).
+
+Every index output (top-k ids, counts, segment tables, dest, src) is compared
+with the oracle in full, bit for bit; every permuted row is checked to be an
+exact copy of its token; floating-point outputs are compared on sampled rows
+and tokens that the oracle evaluates one by one in fp64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_routing_02_b200 import synthetic as syn
+
+from gpu_cases import check_bf16_storage, check_close, make_case, oracle_segments, run_layer, to_np
+
+pytestmark = pytest.mark.gpu
+
+FULL = [syn.MIXTRAL_LIKE, syn.DEEPSEEK_LIKE, syn.SKEWED, syn.BALANCED]
+
+
+def _expert_rows(pairs, wg, wu, wd):
+    """{key: (h, y)} for (key, x_row64, expert) pairs, one expert's weights in fp64 at a time."""
+    by_e = {}
+    for key, xrow, e in pairs:
+        by_e.setdefault(int(e), []).append((key, xrow))
+    out = {}
+    for e, items in by_e.items():
+        g64, u64, d64 = (oracle.f64(t[e].cpu()) for t in (wg, wu, wd))
+        xs = np.stack([x for _, x in items])
+        h = oracle.silu(xs @ g64.T) * (xs @ u64.T)
+        y = h @ d64.T
+        for i, (key, _) in enumerate(items):
+            out[key] = (h[i], y[i])
+    return out
+
+
+@pytest.mark.parametrize("w", FULL, ids=[w.name for w in FULL])
+def test_full_size_layer(cuda_ok, w):
+    case = make_case(w, seed=0, weights_device="cuda")
+    got = run_layer(case)
+    assert got["status"] == 0
+
+    # routing of all T tokens
+    logits, ids, wts = oracle.route(case.x, case.w_r, case.bias, w.k)
+    assert (got["ids"].numpy() == ids).all(), "top-k ids differ"
+    assert np.abs(got["w"].numpy() - wts).max() < 1e-4
+
+    # dispatch tables and positions of all T*k pairs
+    counts = oracle.histogram(ids, w.E)
+    assert (got["counts"].numpy() == counts).all()
+    segs = oracle_segments(case, counts)
+    assert (got["seg_expert"].numpy() == segs.expert).all()
+    assert (got["seg_offsets"].numpy() == segs.offsets).all()
+    assert (got["seg_first_rank"].numpy() == segs.first_rank).all()
+    dest, src = oracle.dispatch_positions(ids, segs, w.E)
+    assert (got["dest"].numpy() == dest).all()
+    used = int(segs.offsets[-1])
+    assert (got["src"].numpy()[:used] == src).all()
+    if w.n_groups:
+        cap = w.tokens_per_group * w.k
+        assert (np.diff(segs.offsets[:: w.E // w.n_groups + w.replica_slots]) == cap).all()
+
+    # every dispatched row is an exact copy of its token's row (checked on the device)
+    src_dev = torch.from_numpy(src.astype(np.int64)).cuda()
+    assert torch.equal(got["xp"][:used], got["x_dev"][src_dev // w.k])
+
+    # expert FFN on sampled rows: first, last and a middle row of a spread of segments
+    rng = np.random.default_rng(0)
+    live = [s for s in range(len(segs.expert)) if segs.length[s] > 0]
+    pick = sorted(set(rng.choice(live, size=min(24, len(live)), replace=False).tolist()))
+    rows = []
+    for s in pick:
+        a, b = int(segs.offsets[s]), int(segs.offsets[s + 1])
+        rows += sorted({a, b - 1, (a + b) // 2})
+    x64 = oracle.f64(case.x)
+    row_expert = {r: int(segs.expert[np.searchsorted(segs.offsets, r, side="right") - 1]) for r in rows}
+    ref_rows = _expert_rows([(r, x64[src[r] // w.k], row_expert[r]) for r in rows], case.wg, case.wu, case.wd)
+    rsel = torch.tensor(rows, device="cuda")
+    check_bf16_storage(to_np(got["hp"][rsel]), np.stack([ref_rows[r][0] for r in rows]), "Hp (sampled rows)")
+    check_close(to_np(got["yp"][rsel]), np.stack([ref_rows[r][1] for r in rows]), "Yp (sampled rows)")
+
+    # layer output on sampled tokens, evaluated token by token (no dispatch)
+    toks = sorted(set(rng.choice(w.T, size=12, replace=False).tolist()) | {0, w.T - 1})
+    pairs = [((t, j), x64[t], ids[t, j]) for t in toks for j in range(w.k) if dest[t * w.k + j] >= 0]
+    ref_pairs = _expert_rows(pairs, case.wg, case.wu, case.wd)
+    ref_out = np.zeros((len(toks), w.d))
+    for i, t in enumerate(toks):
+        for j in range(w.k):
+            if (t, j) in ref_pairs:
+                ref_out[i] += wts[t, j] * ref_pairs[(t, j)][1]
+    check_close(to_np(got["out"][torch.tensor(toks, device="cuda")]), ref_out, "out (sampled tokens)")
