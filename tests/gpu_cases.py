@@ -37,19 +37,32 @@ def check_close(got, ref, what="", max_abs_of_rms=MAX_ABS_OF_RMS, mean_rel=MEAN_
 
 def check_bf16_storage(got, ref, what=""):
     """An intermediate stored in bf16 (Hp): one round-to-nearest to bf16 of an fp32 value that
-    differs from the fp64 reference only by fp32 accumulation error, i.e.
-    |got - ref| <= 2^-8 |ref| (half an ulp of 8 significant bits) + a tiny absolute term."""
+    differs from the fp64 reference by fp32 accumulation error.  Bound per element:
+    2^-7 |ref| (one bf16 ulp: half an ulp for the rounding, and the fp32 value may sit across a
+    rounding boundary from the fp64 one) + 2^-12 RMS(ref) for the accumulation error of values
+    near zero (about 30x the typical sqrt(K) * 2^-24 accumulation error at K <= 16384)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     if ref.size == 0:
         return
     rms = float(np.sqrt(np.mean(ref * ref)))
-    bound = 2.0 ** -8 * np.abs(ref) * (1 + 1e-3) + 1e-5 * rms
+    bound = 2.0 ** -7 * np.abs(ref) + 2.0 ** -12 * rms
     bad = np.abs(got - ref) > bound
     assert np.isfinite(got).all(), f"{what}: non-finite values"
     assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond one bf16 rounding, worst " \
                           f"{float((np.abs(got - ref) / np.maximum(bound, 1e-300)).max()):.3f}x the bound"
+
+
+def check_layer_output(got, ref, dest, T, k, what="out"):
+    """Layer output against the oracle.  Rows of tokens whose k pairs were all dropped (capacity)
+    must be exactly 0; the tolerance of check_close applies to the other rows, whose RMS is the
+    scale of the computed values (a tensor of mostly structural zeros would otherwise shrink it)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    dropped = (np.asarray(dest).reshape(T, k) < 0).all(axis=1)
+    assert (got[dropped] == 0).all(), f"{what}: rows of fully dropped tokens are not zero"
+    check_close(got[~dropped], ref[~dropped], what)
 
 
 def capacity_rows(w: syn.Workload) -> int:

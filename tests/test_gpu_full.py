@@ -13,7 +13,7 @@ import torch
 import oracle
 from mixture_experts_routing_02_b200 import synthetic as syn
 
-from gpu_cases import check_bf16_storage, check_close, make_case, oracle_segments, run_layer, to_np
+from gpu_cases import check_bf16_storage, check_close, check_layer_output, make_case, oracle_segments, run_layer, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -90,4 +90,6 @@ def test_full_size_layer(cuda_ok, w):
         for j in range(w.k):
             if (t, j) in ref_pairs:
                 ref_out[i] += wts[t, j] * ref_pairs[(t, j)][1]
-    check_close(to_np(got["out"][torch.tensor(toks, device="cuda")]), ref_out, "out (sampled tokens)")
+    sel_dest = np.concatenate([dest[t * w.k:(t + 1) * w.k] for t in toks])
+    check_layer_output(to_np(got["out"][torch.tensor(toks, device="cuda")]), ref_out, sel_dest, len(toks), w.k,
+                       "out (sampled tokens)")

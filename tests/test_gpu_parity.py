@@ -11,8 +11,8 @@ import oracle
 import mixture_experts_routing_02_b200 as moe
 from mixture_experts_routing_02_b200 import synthetic as syn
 
-from gpu_cases import (Case, check_bf16_storage, check_close, dev, i32, make_case, moe_shape, oracle_segments,
-                       run_layer, to_np)
+from gpu_cases import (Case, check_bf16_storage, check_close, check_layer_output, dev, i32, make_case, moe_shape,
+                       oracle_segments, run_layer, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -65,7 +65,7 @@ def test_layer_matches_oracle(w):
     # expert FFN and combine within tolerance of the fp64 oracle
     check_bf16_storage(to_np(got["hp"][:used]), ref.hp, "Hp")
     check_close(to_np(got["yp"][:used]), ref.yp, "Yp")
-    check_close(to_np(got["out"]), ref.out, "out")
+    check_layer_output(to_np(got["out"]), ref.out, ref.dest, w.T, w.k)
 
 
 def test_route_logits_and_bias():
