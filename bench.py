@@ -139,6 +139,22 @@ def _dist():
     return world, rank, local
 
 
+def max_over_ranks(values, device, world: int):
+    """Element-wise max of a list of floats over all ranks (identity with one rank)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's device time."""
+    return tokens_per_rank_step * steps * world / (max_ms / 1e3)
+
+
 def _config(w, capacity):
     return {"workload": w.name, "T": w.T, "d_model": w.d, "n_experts": w.E, "top_k": w.k, "d_ff": w.F,
             "capacity": capacity, "n_groups": w.n_groups, "replica_slots": w.replica_slots,
@@ -346,10 +362,7 @@ def run_ours(args, w):
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()}")
 
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, world)
 
     hbm, bf16, bf16_sus, peak_kind = _peaks()
     avg = {k: statistics.mean(v) for k, v in per_kernel.items()}
@@ -381,8 +394,7 @@ def run_ours(args, w):
     traffic = _traffic(dom, w.name)
     roof["traffic"] = traffic
 
-    tokens = T * args.steps * world
-    value = tokens / (total_ms / 1e3)
+    value = job_throughput(T, args.steps, world, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -392,7 +404,7 @@ def run_ours(args, w):
         "roofline": roof,
         "breakdown": {n: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in b.items()}
                       for n, b in breakdown.items()},
-        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
+        "e2e": {"value": job_throughput(T, args.steps, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                 "d2h_bytes_per_step": T * d * 4, "api": "moe_layer_fwd with pinned host X (bf16) / out (fp32) copies"},
         "clocks": clocks.summary(),
     }

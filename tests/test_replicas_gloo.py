@@ -1,0 +1,63 @@
+"""The multi-GPU form of the benchmark is replicas only: no collective on the data
+path, only the max over ranks of the device time.  This checks that reduction
+and the whole-job throughput with two gloo ranks on the CPU."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # rank r "measured" (10 + r) ms for the step loop and (20 - r) ms end to end
+        got = bench.max_over_ranks([10.0 + rank, 20.0 - rank], "cpu", world)
+        value = bench.job_throughput(4096, 5, world, got[0])
+        q.put((rank, got, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_job_value_two_ranks():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, got, value in results:
+        assert got == [11.0, 20.0]            # every rank sees the slowest rank's times
+        assert value == pytest.approx(4096 * 5 * 2 / 0.011)
+
+
+def test_single_rank_is_identity():
+    assert bench.max_over_ranks([1.5, 2.5], "cpu", 1) == [1.5, 2.5]
+    assert bench.job_throughput(100, 2, 1, 1000.0) == 200.0
+
+
+def test_reference_arm_runs_on_rank0_only(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+
+    class A:
+        steps, warmup, seed, gpus = 1, 0, 0, 2
+
+    from mixture_experts_routing_02_b200 import synthetic as syn
+    assert bench.run_reference(A, syn.TINY) == 0      # returns at once, no work, no output
