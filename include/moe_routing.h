@@ -218,6 +218,35 @@ MOE_API moe_status_t moe_dispatch(const moe_shape_t *shape, const moe_bf16_t *x,
                           moe_stream_t stream);
 
 /*
+ * moe_dispatch without a workspace argument, for callers that cannot allocate
+ * device memory: code that runs while a stream is being captured into a CUDA
+ * graph (where cudaMalloc is not allowed), plug-in hooks of runtimes that hand
+ * over only input and output buffers, and processes whose device memory is
+ * already fully reserved by a pool they do not own.  The pages have no
+ * counterpart of this call; it is a convenience of this library.
+ *
+ * Arguments and results are those of moe_dispatch.  The look-back scratch
+ * (ticket + per-tile words) is taken from one 4 MiB array in the library's
+ * device image instead of `ws`; every GPU on which the library is loaded holds
+ * those 4 MiB until the process exits.  Shapes whose scratch would exceed
+ * 4 MiB (256 + ceil(T / tokens_per_tile) * E * 4 bytes, tokens_per_tile =
+ * max(1, 256 / k)) are rejected with MOE_ERR_UNSUPPORTED before anything is
+ * enqueued.  No call allocates: the first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current) and
+ * caches it, so make that first call before any stream capture begins.
+ *
+ * All calls share the one array.  Each call clears the part it needs on
+ * `stream` before using it, but two calls whose work can overlap on the same
+ * GPU (different streams without ordering between them, or different host
+ * threads) race on the array and give wrong results: order them.
+ */
+MOE_API moe_status_t moe_dispatch_static(const moe_shape_t *shape, const moe_bf16_t *x,
+                                 const int32_t *topk_ids, int32_t plan_ready, int32_t *counts,
+                                 int32_t *seg_expert, int32_t *seg_offsets,
+                                 int32_t *seg_first_rank, int32_t *dest, int32_t *src,
+                                 moe_bf16_t *xp, int32_t *status, moe_stream_t stream);
+
+/*
  * Grouped GEMM of the gate and up projections fused with SwiGLU
  * ("5.3 Expert Parallelism", section "3. 고도화된 최적화: 오버래핑(Overlapping) 및
  * GroupGEMM": all experts' GEMMs in one launch):

@@ -16,7 +16,7 @@ from typing import Optional
 __all__ = [
     "MoeError", "MoeShape", "MoeLayerViews", "LIB_PATH", "SYMBOLS", "load_library", "shape",
     "moe_status_string", "moe_layout", "moe_workspace_size", "moe_route", "moe_route_from_logits",
-    "moe_histogram", "moe_segments", "moe_plan_balanced", "moe_dispatch", "moe_expert_gate_up",
+    "moe_histogram", "moe_segments", "moe_plan_balanced", "moe_dispatch", "moe_dispatch_static", "moe_expert_gate_up",
     "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_layer_fwd", "moe_layer_views",
     "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT",
 ]
@@ -57,6 +57,7 @@ SYMBOLS = {
     "moe_segments": [_S, _P, _P, _P, _P, _P],
     "moe_plan_balanced": [_S, _P, _P, _P, _P, _P, _P],
     "moe_dispatch": [_S, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "moe_dispatch_static": [_S, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_expert_gate_up": [_S, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_expert_down": [_S, _P, _P, _P, _P, _P, _P, _P],
     "moe_expert_ffn": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
@@ -159,6 +160,14 @@ def moe_dispatch(s, x, topk_ids, plan_ready, counts, seg_expert, seg_offsets, se
         ctypes.byref(s), _ptr(x), _ptr(topk_ids), int(plan_ready), _ptr(counts), _ptr(seg_expert),
         _ptr(seg_offsets), _ptr(seg_first_rank), _ptr(dest), _ptr(src), _ptr(xp), _ptr(status), _ptr(ws),
         ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def moe_dispatch_static(s, x, topk_ids, plan_ready, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp,
+                        status, stream=None):
+    """moe_dispatch with the library's own static scratch instead of a workspace (see the header)."""
+    _check("moe_dispatch_static", load_library().moe_dispatch_static(
+        ctypes.byref(s), _ptr(x), _ptr(topk_ids), int(plan_ready), _ptr(counts), _ptr(seg_expert),
+        _ptr(seg_offsets), _ptr(seg_first_rank), _ptr(dest), _ptr(src), _ptr(xp), _ptr(status), _stream(stream)))
 
 
 def moe_expert_gate_up(s, xp, seg_expert, seg_offsets, w_gate, w_up, hp, status=None, stream=None):

@@ -198,6 +198,29 @@ moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* id
     return cuda_status(launch_permute(a, sm_count(), st));
 }
 
+// Scratch of moe_dispatch_static: one array in the library's device image.  Host code
+// may not use the symbol itself as a device address; its address is looked up once
+// per device with cudaGetSymbolAddress (with that device current) and cached.
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_dispatch_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of the scratch array on the current device (nullptr on failure).
+void* static_scratch_address() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_dispatch_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        g_scratch_addr[dev] = p;
+    }
+    return g_scratch_addr[dev];
+}
+
 struct LayerLayout {
     size_t ids, w, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, dispatch_ws, xp, hp, yp, total;
     size_t dispatch_ws_bytes;
@@ -312,6 +335,20 @@ moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const i
     if (s != MOE_OK) return s;
     return dispatch_impl(v, x, topk_ids, plan_ready, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp,
                          status, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_dispatch_static(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_ids,
+                                 int32_t plan_ready, int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets,
+                                 int32_t* seg_first_rank, int32_t* dest, int32_t* src, moe_bf16_t* xp,
+                                 int32_t* status, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (permute_ws_bytes(v.T, v.k, v.E) > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED;
+    void* scratch = static_scratch_address();
+    if (scratch == nullptr) return MOE_ERR_CUDA;
+    return dispatch_impl(v, x, topk_ids, plan_ready, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp,
+                         status, scratch, kStaticScratchBytes, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* xp, const int32_t* seg_expert,
