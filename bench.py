@@ -57,12 +57,17 @@ def _traffic(kernel: str, workload: str):
             entries = json.load(f)
     except Exception:
         return None
-    h = hashlib.sha256()
-    for fn in ("umma_gemm.cu", "common.cuh", "dispatch.cu", "combine.cu"):
-        with open(os.path.join(ROOT, "mixture_experts_routing_02_b200", "csrc", fn), "rb") as f:
-            h.update(f.read())
     for e in entries:
-        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("source_sha256") == h.hexdigest():
+        if e.get("kernel") != kernel or e.get("workload") != workload:
+            continue
+        h = hashlib.sha256()
+        try:
+            for fn in e["source_files"]:
+                with open(os.path.join(ROOT, fn), "rb") as f:
+                    h.update(f.read())
+        except Exception:
+            return None
+        if e.get("source_sha256") == h.hexdigest():
             return e.get("dram_bytes_per_launch")
     return None
 
