@@ -193,7 +193,7 @@ moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* id
     a.tile_state = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 256);
     a.status = status;
     a.T = v.T; a.k = v.k; a.E = v.E; a.d = v.d; a.n_seg = v.n_seg;
-    a.tokens_per_tile = permute_tokens_per_tile(v.k);
+    a.tokens_per_tile = permute_tokens_per_tile(v.T, v.k);
     a.n_tiles = permute_n_tiles(v.T, v.k);
     return cuda_status(launch_permute(a, sm_count(), st));
 }

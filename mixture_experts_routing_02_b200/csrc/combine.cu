@@ -17,6 +17,9 @@ namespace moe {
 
 namespace {
 
+// KMAX: the largest k this instance handles (registers scale with KMAX * UNROLL);
+// UNROLL: row vectors per lane whose gathers are all in flight together.
+template <int KMAX, int UNROLL>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ dest,
                                                       const float* __restrict__ w, int T, int k, int d,
                                                       float* __restrict__ out) {
@@ -30,31 +33,42 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
             mine_d = __ldg(dest + static_cast<size_t>(t) * k + lane);
             mine_w = __ldg(w + static_cast<size_t>(t) * k + lane);
         }
-        int dr[kMaxTopK];
-        float wr[kMaxTopK];
+        int dr[KMAX];
+        float wr[KMAX];
 #pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) {
+        for (int j = 0; j < KMAX; ++j) {
             dr[j] = __shfl_sync(0xffffffffu, mine_d, j);
             wr[j] = __shfl_sync(0xffffffffu, mine_w, j);
             if (j >= k) dr[j] = -1;
         }
         float4* orow = reinterpret_cast<float4*>(out + static_cast<size_t>(t) * d);
-        for (int v = lane; v < vec_per_row; v += 32) {
-            float4 val[kMaxTopK];
+        for (int v0 = lane; v0 < vec_per_row; v0 += 32 * UNROLL) {
+            // all gathers of UNROLL vectors issued before any is used
+            float4 val[UNROLL][KMAX];
 #pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j)
-                if (dr[j] >= 0) val[j] = __ldg(reinterpret_cast<const float4*>(yp + static_cast<size_t>(dr[j]) * d) + v);
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int u = 0; u < UNROLL; ++u) {
+                const int v = v0 + 32 * u;
 #pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j) {
-                if (dr[j] >= 0) {
-                    acc.x = fmaf(wr[j], val[j].x, acc.x);
-                    acc.y = fmaf(wr[j], val[j].y, acc.y);
-                    acc.z = fmaf(wr[j], val[j].z, acc.z);
-                    acc.w = fmaf(wr[j], val[j].w, acc.w);
-                }
+                for (int j = 0; j < KMAX; ++j)
+                    if (dr[j] >= 0 && v < vec_per_row)
+                        val[u][j] = __ldg(reinterpret_cast<const float4*>(yp + static_cast<size_t>(dr[j]) * d) + v);
             }
-            orow[v] = acc;
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int v = v0 + 32 * u;
+                if (v >= vec_per_row) break;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) {
+                    if (dr[j] >= 0) {
+                        acc.x = fmaf(wr[j], val[u][j].x, acc.x);
+                        acc.y = fmaf(wr[j], val[u][j].y, acc.y);
+                        acc.z = fmaf(wr[j], val[u][j].z, acc.z);
+                        acc.w = fmaf(wr[j], val[u][j].w, acc.w);
+                    }
+                }
+                orow[v] = acc;
+            }
         }
     }
 }
@@ -66,7 +80,12 @@ cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w,
     if (T == 0) return cudaSuccess;
     int grid = (T + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
-    combine_kernel<<<grid, 256, 0, stream>>>(yp, dest, w, T, k, d, out);
+    if (k <= 2)
+        combine_kernel<2, 4><<<grid, 256, 0, stream>>>(yp, dest, w, T, k, d, out);
+    else if (k <= 4)
+        combine_kernel<4, 2><<<grid, 256, 0, stream>>>(yp, dest, w, T, k, d, out);
+    else
+        combine_kernel<kMaxTopK, 1><<<grid, 256, 0, stream>>>(yp, dest, w, T, k, d, out);
     return cudaGetLastError();
 }
 

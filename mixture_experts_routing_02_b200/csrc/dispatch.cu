@@ -30,6 +30,7 @@ constexpr uint32_t kFlagAggregate = 1u << 30;
 constexpr uint32_t kFlagPrefix = 2u << 30;
 constexpr uint32_t kValueMask = (1u << 30) - 1;
 constexpr int kPermuteWarps = kPermuteThreads / 32;
+constexpr int kCopyUnroll = 8;
 
 // Exclusive scan over the 256 threads of a block; *total receives the sum.
 __device__ __forceinline__ int block_exclusive_scan_256(int v, int* warp_sums, int* total) {
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(256) plan_kernel(const int32_t* __restrict__ c
 
 // ------------------------------------------------------------------------------ stable rank + permute
 
-__global__ void __launch_bounds__(kPermuteThreads) permute_kernel(const PermuteArgs a) {
+__global__ void __launch_bounds__(kPermuteThreads, 4) permute_kernel(const PermuteArgs a) {
     __shared__ int s_dest[kPermutePairs];
     __shared__ int s_wcnt[kPermuteWarps][kMaxExperts];
     __shared__ int s_excl[kMaxExperts];
@@ -339,24 +340,25 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(const PermuteA
         }
         __syncthreads();
 
-        // 4. copy each token row once from X into its k slots (16-byte vectors, coalesced)
+        // 4. copy each token row once from X into its k slots (16-byte vectors, coalesced);
+        //    8 loads in flight per lane before the stores
         for (int tl = warp; tl < t1 - t0; tl += kPermuteWarps) {
             const uint4* xs = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + tl) * a.d);
             int dj[kMaxTopK];
 #pragma unroll
             for (int j = 0; j < kMaxTopK; ++j) dj[j] = (j < k) ? s_dest[tl * k + j] : -1;
-            for (int v = lane; v < vec_per_row; v += 128) {
-                uint4 val[4];
+            for (int v = lane; v < vec_per_row; v += 32 * kCopyUnroll) {
+                uint4 val[kCopyUnroll];
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
+                for (int u = 0; u < kCopyUnroll; ++u)
                     if (v + 32 * u < vec_per_row) val[u] = __ldg(xs + v + 32 * u);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (v + 32 * u < vec_per_row) {
+                for (int j = 0; j < kMaxTopK; ++j) {
+                    if (dj[j] >= 0) {
+                        uint4* dst = reinterpret_cast<uint4*>(a.xp + static_cast<size_t>(dj[j]) * a.d);
 #pragma unroll
-                        for (int j = 0; j < kMaxTopK; ++j)
-                            if (dj[j] >= 0)
-                                reinterpret_cast<uint4*>(a.xp + static_cast<size_t>(dj[j]) * a.d)[v + 32 * u] = val[u];
+                        for (int u = 0; u < kCopyUnroll; ++u)
+                            if (v + 32 * u < vec_per_row) dst[v + 32 * u] = val[u];
                     }
                 }
             }
@@ -426,12 +428,19 @@ __global__ void __launch_bounds__(256) route_from_logits_kernel(const float* __r
 
 }  // namespace
 
-int permute_tokens_per_tile(int k) {
-    const int t = kPermutePairs / k;
+int permute_tokens_per_tile(int T, int k) {
+    // about kPermuteTargetTiles tiles (enough CTAs to fill the GPU with row copies), at most
+    // kPermutePairs pairs per tile (one pair per thread), at least one token
+    int t = (T + kPermuteTargetTiles - 1) / kPermuteTargetTiles;
+    const int cap = kPermutePairs / k;
+    if (t > cap) t = cap;
     return t < 1 ? 1 : t;
 }
 
-int permute_n_tiles(int T, int k) { return (T + permute_tokens_per_tile(k) - 1) / permute_tokens_per_tile(k); }
+int permute_n_tiles(int T, int k) {
+    const int tpt = permute_tokens_per_tile(T, k);
+    return (T + tpt - 1) / tpt;
+}
 
 size_t permute_ws_bytes(int T, int k, int E) {
     return 256 + static_cast<size_t>(permute_n_tiles(T, k)) * static_cast<size_t>(E) * sizeof(uint32_t);
@@ -464,7 +473,7 @@ cudaError_t launch_permute(const PermuteArgs& a, int num_sms, cudaStream_t strea
     cudaError_t err = cudaMemsetAsync(a.ticket, 0, permute_ws_bytes(a.T, a.k, a.E), stream);
     if (err != cudaSuccess) return err;
     if (a.n_tiles == 0) return cudaSuccess;
-    int grid = a.n_tiles < 4 * num_sms ? a.n_tiles : 4 * num_sms;
+    int grid = a.n_tiles < 8 * num_sms ? a.n_tiles : 8 * num_sms;
     permute_kernel<<<grid, kPermuteThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }

@@ -45,7 +45,8 @@ cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b
 
 // dispatch.cu
 constexpr int kPermuteThreads = 256;
-constexpr int kPermutePairs = 256;  // (t, j) pairs per look-back tile, rounded to whole tokens
+constexpr int kPermutePairs = 256;          // most (t, j) pairs per look-back tile (one per thread)
+constexpr int kPermuteTargetTiles = 1024;   // tiles aimed for, so the row copies fill the GPU
 
 struct PermuteArgs {
     const int32_t* ids;
@@ -62,7 +63,7 @@ struct PermuteArgs {
     int T, k, E, d, n_seg, tokens_per_tile, n_tiles;
 };
 
-int permute_tokens_per_tile(int k);
+int permute_tokens_per_tile(int T, int k);
 int permute_n_tiles(int T, int k);
 size_t permute_ws_bytes(int T, int k, int E);
 
