@@ -22,7 +22,8 @@
 //   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
 //               (M=128, N=mma_n, K=16, bf16 x bf16 -> fp32) and commits
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (one row per thread),
-//               fused math, direct 16-byte stores of the valid rows
+//               fused math, a shared-memory transpose, then row-contiguous 16-byte
+//               stores of the valid rows
 // Two accumulator buffers (columns [0,256) and [256,512)) let the epilogue of
 // one tile overlap the main loop of the next.
 #include "common.cuh"
@@ -40,6 +41,7 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 256;
 constexpr uint32_t kABytes = kBM * kBK * 2;
+constexpr int kStageWords = 32 * 33;  // one epilogue warp's transpose buffer (32 rows x 33 words)
 
 struct TileCoord {
     int seg, m, n, row0, row_end, expert;
@@ -88,6 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + stages * kABytes;
+    uint32_t* epi_stage = reinterpret_cast<uint32_t*>(sB + stages * b_stage_bytes);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -224,27 +227,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool valid = row < c.row_end;
             const int n0 = c.n * g.BN;
 
+            // Stores go through a per-warp shared-memory transpose: each thread owns one row of
+            // the accumulator, but the global stores are issued row-contiguous (whole 128-byte
+            // lines per group of lanes) with the ragged rows of a segment masked.
+            uint32_t* stg = epi_stage + (warp - 2) * kStageWords;
             if (EPI == kEpiSwiglu) {
                 for (int cc = 0; cc < g.BN; cc += 32) {
                     uint32_t gr[32], ur[32];
                     tmem_ld32(t_row + cc, gr);
                     tmem_ld32(t_row + g.BN + cc, ur);
                     tmem_ld_wait();
-                    if (valid && n0 + cc < g.N) {
-                        uint32_t pk[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float g0 = __uint_as_float(gr[2 * i]), g1 = __uint_as_float(gr[2 * i + 1]);
-                            const float u0 = __uint_as_float(ur[2 * i]), u1 = __uint_as_float(ur[2 * i + 1]);
-                            const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-                            const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
-                            pk[i] = pack_bf16x2(h0, h1);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
-                                                              static_cast<size_t>(row) * g.ldo + n0 + cc);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    for (int i = 0; i < 16; ++i) {
+                        const float g0 = __uint_as_float(gr[2 * i]), g1 = __uint_as_float(gr[2 * i + 1]);
+                        const float u0 = __uint_as_float(ur[2 * i]), u1 = __uint_as_float(ur[2 * i + 1]);
+                        const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                        const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                        stg[lane * 17 + i] = pack_bf16x2(h0, h1);
                     }
+                    __syncwarp();
+                    if (n0 + cc < g.N) {
+                        // 32 rows x 64 bytes: 4 lanes per row, 8 rows per pass
+                        const int rr = lane >> 2, q = lane & 3;
+#pragma unroll
+                        for (int pass = 0; pass < 4; ++pass) {
+                            const int rl = pass * 8 + rr;
+                            const int grow = c.row0 + quarter * 32 + rl;
+                            if (grow < c.row_end) {
+                                const uint32_t* src = stg + rl * 17 + q * 4;
+                                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
+                                                                      static_cast<size_t>(grow) * g.ldo + n0 + cc + q * 8);
+                                *dst = make_uint4(src[0], src[1], src[2], src[3]);
+                            }
+                        }
+                    }
+                    __syncwarp();
                 }
             } else if (EPI == kEpiStore) {
                 // fp32 rows: the accumulator is stored as is
@@ -252,12 +269,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t r[32];
                     tmem_ld32(t_row + cc, r);
                     tmem_ld_wait();
-                    if (valid && n0 + cc < g.N) {
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(g.out) +
-                                                              static_cast<size_t>(row) * g.ldo + n0 + cc);
 #pragma unroll
-                        for (int v = 0; v < 8; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+                    for (int i = 0; i < 32; ++i) stg[lane * 33 + i] = r[i];
+                    __syncwarp();
+                    if (n0 + cc < g.N) {
+                        // 32 rows x 128 bytes: 8 lanes per row, 4 rows per pass
+                        const int rr = lane >> 3, q = lane & 7;
+#pragma unroll
+                        for (int pass = 0; pass < 8; ++pass) {
+                            const int rl = pass * 4 + rr;
+                            const int grow = c.row0 + quarter * 32 + rl;
+                            if (grow < c.row_end) {
+                                const uint32_t* src = stg + rl * 33 + q * 4;
+                                uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(g.out) +
+                                                                      static_cast<size_t>(grow) * g.ldo + n0 + cc + q * 4);
+                                *dst = make_uint4(src[0], src[1], src[2], src[3]);
+                            }
+                        }
                     }
+                    __syncwarp();
                 }
             } else {
                 // router: top-k over the E logits of this row, softmax over the selected ones
@@ -329,7 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 size_t gemm_smem_bytes(int stages, int mma_n) {
-    return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(mma_n) * 128u);
+    return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(mma_n) * 128u) +
+           4 * kStageWords * sizeof(uint32_t);
 }
 
 int gemm_pick_stages(int mma_n) {
