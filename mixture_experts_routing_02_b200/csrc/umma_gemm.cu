@@ -48,7 +48,7 @@ struct TileCoord {
 };
 
 __device__ __forceinline__ TileCoord decode_tile(int tile, const int* prefix, int n_seg, int n_tiles_n,
-                                                 const GemmArgs& g) {
+                                                 const GemmArgs& g, int bm = kBM) {
     const int key = tile / n_tiles_n;
     int lo = 0, hi = n_seg;
     while (hi - lo > 1) {
@@ -63,9 +63,100 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const int* prefix, in
     c.m = local - c.n * mt;
     const int start = g.seg_offsets ? __ldg(g.seg_offsets + lo) : 0;
     c.row_end = g.seg_offsets ? __ldg(g.seg_offsets + lo + 1) : g.M;
-    c.row0 = start + c.m * kBM;
+    c.row0 = start + c.m * bm;
     c.expert = g.seg_expert ? __ldg(g.seg_expert + lo) : 0;
     return c;
+}
+
+// One warp: cumulative count of bm-row tiles over the segments (empty / unused segments have none).
+__device__ __forceinline__ void build_tile_prefix(int* prefix, const GemmArgs& g, int bm, int lane) {
+    int carry = 0;
+    for (int b = 0; b < g.n_seg; b += 32) {
+        const int s = b + lane;
+        int mt = 0;
+        if (s < g.n_seg) {
+            const int a = g.seg_offsets ? __ldg(g.seg_offsets + s) : 0;
+            const int e = g.seg_offsets ? __ldg(g.seg_offsets + s + 1) : g.M;
+            const bool live = (g.seg_expert == nullptr) || __ldg(g.seg_expert + s) >= 0;
+            mt = (live && e > a) ? (e - a + bm - 1) / bm : 0;
+        }
+        int v = mt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += t;
+        }
+        if (s < g.n_seg) prefix[s] = carry + v - mt;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) prefix[g.n_seg] = carry;
+}
+
+// Epilogue of one warp's 32 accumulator rows (rows row_base.. of the output, columns n0..n0+BN)
+// for the SwiGLU (bf16 Hp) and plain (fp32 Yp) contractions.  Each thread owns one row of the
+// accumulator; the rows go through a per-warp shared-memory transpose so that the global stores
+// are row-contiguous (whole 128-byte lines per group of lanes), with rows >= row_end masked.
+template <int EPI>
+__device__ __forceinline__ void epilogue_rows(const GemmArgs& g, uint32_t t_row, int row_base, int row_end, int n0,
+                                              int lane, uint32_t* stg) {
+    if (EPI == kEpiSwiglu) {
+        for (int cc = 0; cc < g.BN; cc += 32) {
+            uint32_t gr[32], ur[32];
+            tmem_ld32(t_row + cc, gr);
+            tmem_ld32(t_row + g.BN + cc, ur);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float g0 = __uint_as_float(gr[2 * i]), g1 = __uint_as_float(gr[2 * i + 1]);
+                const float u0 = __uint_as_float(ur[2 * i]), u1 = __uint_as_float(ur[2 * i + 1]);
+                const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                stg[lane * 17 + i] = pack_bf16x2(h0, h1);
+            }
+            __syncwarp();
+            if (n0 + cc < g.N) {
+                // 32 rows x 64 bytes: 4 lanes per row, 8 rows per pass
+                const int rr = lane >> 2, q = lane & 3;
+#pragma unroll
+                for (int pass = 0; pass < 4; ++pass) {
+                    const int rl = pass * 8 + rr;
+                    const int grow = row_base + rl;
+                    if (grow < row_end) {
+                        const uint32_t* src = stg + rl * 17 + q * 4;
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
+                                                              static_cast<size_t>(grow) * g.ldo + n0 + cc + q * 8);
+                        *dst = make_uint4(src[0], src[1], src[2], src[3]);
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    } else {
+        for (int cc = 0; cc < g.BN; cc += 32) {
+            uint32_t r[32];
+            tmem_ld32(t_row + cc, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) stg[lane * 33 + i] = r[i];
+            __syncwarp();
+            if (n0 + cc < g.N) {
+                // 32 rows x 128 bytes: 8 lanes per row, 4 rows per pass
+                const int rr = lane >> 3, q = lane & 7;
+#pragma unroll
+                for (int pass = 0; pass < 8; ++pass) {
+                    const int rl = pass * 4 + rr;
+                    const int grow = row_base + rl;
+                    if (grow < row_end) {
+                        const uint32_t* src = stg + rl * 33 + q * 4;
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(g.out) +
+                                                              static_cast<size_t>(grow) * g.ldo + n0 + cc + q * 4);
+                        *dst = make_uint4(src[0], src[1], src[2], src[3]);
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
 }
 
 template <int EPI>
@@ -109,29 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (EPI == kEpiSwiglu) tma_prefetch_desc(&tmB1);
     }
     if (warp == 1) tmem_alloc(&tmem_base_sh, kTmemCols);
-    if (warp == 2) {
-        // cumulative row-tile count of the segments (empty / unused segments have none)
-        int carry = 0;
-        for (int b = 0; b < g.n_seg; b += 32) {
-            const int s = b + lane;
-            int mt = 0;
-            if (s < g.n_seg) {
-                const int a = g.seg_offsets ? __ldg(g.seg_offsets + s) : 0;
-                const int e = g.seg_offsets ? __ldg(g.seg_offsets + s + 1) : g.M;
-                const bool live = (g.seg_expert == nullptr) || __ldg(g.seg_expert + s) >= 0;
-                mt = (live && e > a) ? (e - a + kBM - 1) / kBM : 0;
-            }
-            int v = mt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int t = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += t;
-            }
-            if (s < g.n_seg) tile_prefix[s] = carry + v - mt;
-            carry += __shfl_sync(0xffffffffu, v, 31);
-        }
-        if (lane == 0) tile_prefix[g.n_seg] = carry;
-    }
+    if (warp == 2) build_tile_prefix(tile_prefix, g, kBM, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -227,68 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool valid = row < c.row_end;
             const int n0 = c.n * g.BN;
 
-            // Stores go through a per-warp shared-memory transpose: each thread owns one row of
-            // the accumulator, but the global stores are issued row-contiguous (whole 128-byte
-            // lines per group of lanes) with the ragged rows of a segment masked.
-            uint32_t* stg = epi_stage + (warp - 2) * kStageWords;
-            if (EPI == kEpiSwiglu) {
-                for (int cc = 0; cc < g.BN; cc += 32) {
-                    uint32_t gr[32], ur[32];
-                    tmem_ld32(t_row + cc, gr);
-                    tmem_ld32(t_row + g.BN + cc, ur);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float g0 = __uint_as_float(gr[2 * i]), g1 = __uint_as_float(gr[2 * i + 1]);
-                        const float u0 = __uint_as_float(ur[2 * i]), u1 = __uint_as_float(ur[2 * i + 1]);
-                        const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-                        const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
-                        stg[lane * 17 + i] = pack_bf16x2(h0, h1);
-                    }
-                    __syncwarp();
-                    if (n0 + cc < g.N) {
-                        // 32 rows x 64 bytes: 4 lanes per row, 8 rows per pass
-                        const int rr = lane >> 2, q = lane & 3;
-#pragma unroll
-                        for (int pass = 0; pass < 4; ++pass) {
-                            const int rl = pass * 8 + rr;
-                            const int grow = c.row0 + quarter * 32 + rl;
-                            if (grow < c.row_end) {
-                                const uint32_t* src = stg + rl * 17 + q * 4;
-                                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) +
-                                                                      static_cast<size_t>(grow) * g.ldo + n0 + cc + q * 8);
-                                *dst = make_uint4(src[0], src[1], src[2], src[3]);
-                            }
-                        }
-                    }
-                    __syncwarp();
-                }
-            } else if (EPI == kEpiStore) {
-                // fp32 rows: the accumulator is stored as is
-                for (int cc = 0; cc < g.BN; cc += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(t_row + cc, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) stg[lane * 33 + i] = r[i];
-                    __syncwarp();
-                    if (n0 + cc < g.N) {
-                        // 32 rows x 128 bytes: 8 lanes per row, 4 rows per pass
-                        const int rr = lane >> 3, q = lane & 7;
-#pragma unroll
-                        for (int pass = 0; pass < 8; ++pass) {
-                            const int rl = pass * 4 + rr;
-                            const int grow = c.row0 + quarter * 32 + rl;
-                            if (grow < c.row_end) {
-                                const uint32_t* src = stg + rl * 33 + q * 4;
-                                uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(g.out) +
-                                                                      static_cast<size_t>(grow) * g.ldo + n0 + cc + q * 4);
-                                *dst = make_uint4(src[0], src[1], src[2], src[3]);
-                            }
-                        }
-                    }
-                    __syncwarp();
-                }
+            if (EPI == kEpiSwiglu || EPI == kEpiStore) {
+                epilogue_rows<EPI>(g, t_row, c.row0 + quarter * 32, c.row_end, n0, lane,
+                                   epi_stage + (warp - 2) * kStageWords);
             } else {
                 // router: top-k over the E logits of this row, softmax over the selected ones
                 float tv[kMaxTopK];
@@ -356,6 +366,172 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+
+// ------------------------------------------------------------------------------------------
+// The same contraction on a CTA pair (cluster of 2, tcgen05 cta_group::2): a 256-row tile whose
+// rows [0,128) live in CTA 0 and [128,256) in CTA 1.  Each CTA loads its own 128 rows of A and
+// its half of the B tile (SwiGLU: CTA 0 the gate rows, CTA 1 the up rows; plain: the two halves
+// of the output columns), so every SM moves half the B bytes of the single-CTA kernel and a stage
+// is 32 KB (6 stages).  The leader (rank 0) expects the bytes of both CTAs' loads on its full
+// barrier and issues M=256 MMAs; its commits arrive on the barriers of both CTAs; the epilogue
+// warps of both CTAs read their own tensor memory and release the accumulator buffer on the
+// leader's barrier.
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                          const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
+    __shared__ __align__(8) uint64_t full_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+    __shared__ int tile_prefix[kMaxSegments + 1];
+    extern __shared__ uint8_t dsmem[];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1;
+    const int n_pairs = gridDim.x >> 1;
+    const int stages = g.stages;
+    const int b_half_rows = g.mma_n / 2;
+    const uint32_t b_half_bytes = static_cast<uint32_t>(b_half_rows) * 128u;
+
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + stages * kABytes;
+    uint32_t* epi_stage = reinterpret_cast<uint32_t*>(sB + stages * b_half_bytes);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull_bar[b], 1);
+            mbar_init(&tempty_bar[b], 8);  // 4 epilogue warps of each CTA (used in the leader)
+        }
+        mbar_init(&drain_bar, 1);
+        abort_sh = 0;
+        mbar_fence_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(EPI == kEpiSwiglu && rank == 1 ? &tmB1 : &tmB0);
+    }
+    if (warp == 1) tmem_alloc_pair(&tmem_base_sh, kTmemCols);
+    if (warp == 2) build_tile_prefix(tile_prefix, g, 2 * kBM, lane);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrive
+    tc_fence_after();
+
+    const uint32_t tmem_base = tmem_base_sh;
+    const int total = tile_prefix[g.n_seg] * g.n_tiles_n;
+    const int nkb = g.K / kBK;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0, issued = 0;
+            uint32_t phase = 0;
+            const uint32_t tx = 2u * (kABytes + b_half_bytes);
+            const CUtensorMap* tb = (EPI == kEpiSwiglu && rank == 1) ? &tmB1 : &tmB0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < total; tile += n_pairs) {
+                const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g, 2 * kBM);
+                const int n0 = c.n * g.BN;
+                const int b_row = (EPI == kEpiSwiglu) ? n0 : n0 + static_cast<int>(rank) * b_half_rows;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, g.status)) { ok = false; break; }
+                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], tx);
+                    const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+                    tma_load_2d_pair(sA + stage * kABytes, &tmA, kb * kBK, c.row0 + static_cast<int>(rank) * kBM, fb);
+                    tma_load_3d_pair(sB + stage * b_half_bytes, tb, kb * kBK, b_row, c.expert, fb);
+                    ++issued;
+                    if (++stage == stages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok) {
+                // let copies in flight land before the CTA pair exits (bounded)
+                if (rank == 0) {
+                    const int first = issued > stages ? issued - stages : 0;
+                    for (int i = first; i < issued; ++i)
+                        mbar_wait(&full_bar[i % stages], static_cast<uint32_t>((i / stages) & 1), nullptr, nullptr);
+                } else {
+                    for (int i = 0; i < 1000; ++i) sleep_ns(1000);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer (leader only)
+        if (lane == 0 && rank == 0) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            const uint32_t idesc = umma_idesc_bf16(2 * kBM, g.mma_n);
+            bool ok = true;
+            for (int tile = pair; ok && tile < total; tile += n_pairs) {
+                if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_sh, g.status)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kAccStride;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&full_bar[stage], phase, &abort_sh, g.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * kABytes));
+                    const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * b_half_bytes));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+                        umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    const uint32_t eb = smem_u32(&empty_bar[stage]);
+                    umma_commit_pair(eb);
+                    umma_commit_pair(mapa_shared(eb, 1));
+                    if (++stage == stages) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                const uint32_t fb = smem_u32(&tfull_bar[acc]);
+                umma_commit_pair(fb);
+                umma_commit_pair(mapa_shared(fb, 1));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            umma_commit_pair(smem_u32(&drain_bar));
+            mbar_wait(&drain_bar, 0, nullptr, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ epilogue (both CTAs)
+        const int quarter = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+        const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty_bar[1]), 0);
+        for (int tile = pair; tile < total; tile += n_pairs) {
+            const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g, 2 * kBM);
+            const bool got = mbar_wait(&tfull_bar[acc], acc_phase, &abort_sh, g.status);
+            if (!__all_sync(0xffffffffu, got)) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(acc) * kAccStride;
+            epilogue_rows<EPI>(g, t_row, c.row0 + static_cast<int>(rank) * kBM + quarter * 32, c.row_end,
+                               c.n * g.BN, lane, epi_stage + (warp - 2) * kStageWords);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while its pair may still read its shared or tensor memory
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+}
+
 }  // namespace
 
 size_t gemm_smem_bytes(int stages, int mma_n) {
@@ -380,6 +556,50 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     if (err != cudaSuccess) return err;
     kern<<<grid, kThreads, smem, stream>>>(a, b0, b1, g);
     return cudaGetLastError();
+}
+
+size_t gemm_pair_smem_bytes(int stages, int mma_n) {
+    return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(mma_n / 2) * 128u) +
+           4 * kStageWords * sizeof(uint32_t);
+}
+
+int gemm_pair_pick_stages(int mma_n) {
+    const size_t per = kABytes + static_cast<size_t>(mma_n / 2) * 128u;
+    int s = static_cast<int>((kGemmSmemBudget - 1024) / per);
+    if (s > kMaxStages) s = kMaxStages;
+    return s;
+}
+
+template <int EPI>
+static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmArgs& g,
+                               int n_pairs, cudaStream_t stream) {
+    auto kern = umma_gemm_pair_kernel<EPI>;
+    size_t smem = gemm_pair_smem_bytes(g.stages, g.mma_n);
+    if (smem < kGemmSmemMin) smem = kGemmSmemMin;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * n_pairs, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, g);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_umma_gemm_pair(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                                  const GemmArgs& g, int n_pairs, cudaStream_t stream) {
+    if (epi == kEpiSwiglu) return launch_pair<kEpiSwiglu>(a, b0, b1, g, n_pairs, stream);
+    if (epi == kEpiStore) return launch_pair<kEpiStore>(a, b0, b1, g, n_pairs, stream);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
