@@ -229,9 +229,9 @@ MOE_API moe_status_t moe_dispatch(const moe_shape_t *shape, const moe_bf16_t *x,
  * (ticket + per-tile words) is taken from one 4 MiB array in the library's
  * device image instead of `ws`; every GPU on which the library is loaded holds
  * those 4 MiB until the process exits.  Shapes whose scratch would exceed
- * 4 MiB (256 + n_tiles * E * 4 bytes, n_tiles = ceil(T / tokens_per_tile),
- * tokens_per_tile = clamp(ceil(T / 1024), 1, max(1, 256 / k))) are rejected
- * with MOE_ERR_UNSUPPORTED before anything is enqueued.  No call allocates: the first call on each device looks up the
+ * 4 MiB (256 + n_tiles * E * 4 + 64 * E * 4 bytes, n_tiles = ceil(T /
+ * tokens_per_tile), tokens_per_tile = clamp(ceil(T / 1024), 1, max(1, 256 / k)))
+ * are rejected with MOE_ERR_UNSUPPORTED before anything is enqueued.  No call allocates: the first call on each device looks up the
  * array's device address (cudaGetSymbolAddress, with that device current) and
  * caches it, so make that first call before any stream capture begins.
  *

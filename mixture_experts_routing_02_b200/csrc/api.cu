@@ -98,10 +98,14 @@ bool tmap_experts(CUtensorMap* m, const void* p, int E, int N, int K, int box_n)
 
 inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// Grouped GEMMs run on CTA pairs (256-row tiles) when segments are long enough on average that
-// the second 128 rows of a tile are mostly real rows; otherwise on single CTAs (128-row tiles).
-bool use_pairs(const Dims& v) {
-    return v.n_seg > 0 && static_cast<int64_t>(v.rows) >= static_cast<int64_t>(kPairMinRowsPerSegment) * v.n_seg;
+// The down projection runs on CTA pairs (256-row tiles) when segments are long enough on average
+// that the second 128 rows of a tile are mostly real rows and its reduction (F) is short, so the
+// fp32 epilogue is a large share of each tile; measured on B200 the pair kernel is then ~8 % faster.
+// Everything else (and the gate/up projection always) runs on single CTAs with 128-row tiles,
+// which measured as fast or faster: the contraction is power-limited, not operand-bandwidth-limited.
+bool use_pairs_for_down(const Dims& v) {
+    return v.n_seg > 0 && v.F <= kPairMaxReduction &&
+           static_cast<int64_t>(v.rows) >= static_cast<int64_t>(kPairMinRowsPerSegment) * v.n_seg;
 }
 
 // ------------------------------------------------------------------------------ implementations
@@ -145,13 +149,6 @@ moe_status_t gate_up_impl(const Dims& v, const moe_bf16_t* xp, const int32_t* se
     g.seg_offsets = seg_offsets; g.seg_expert = seg_expert; g.n_seg = v.n_seg; g.M = v.rows; g.K = v.d; g.N = v.F;
     g.BN = bn; g.n_tiles_n = (v.F + bn - 1) / bn; g.mma_n = 2 * bn;
     g.out = hp; g.ldo = v.F; g.k = v.k; g.status = status;
-    if (use_pairs(v)) {
-        // CTA 0 of a pair loads the gate rows, CTA 1 the up rows: the same boxes as below
-        g.stages = gemm_pair_pick_stages(g.mma_n);
-        const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 256 + v.n_seg) * g.n_tiles_n;
-        const int n_pairs = static_cast<int>(std::min<int64_t>(sm_count() / 2, max_tiles));
-        return cuda_status(launch_umma_gemm_pair(kEpiSwiglu, ta, tg, tu, g, n_pairs, st));
-    }
     g.stages = gemm_pick_stages(2 * bn);
     const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 128 + v.n_seg) * g.n_tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(sm_count(), max_tiles));
@@ -165,7 +162,7 @@ moe_status_t down_impl(const Dims& v, const moe_bf16_t* hp, const int32_t* seg_e
     if (v.T == 0 || v.rows == 0) return MOE_OK;
     if (!have_encoder()) return MOE_ERR_CUDA;
     const int bn = v.d >= 256 ? 256 : v.d;
-    const bool pairs = use_pairs(v);
+    const bool pairs = use_pairs_for_down(v);
     CUtensorMap ta, tb;
     // a CTA of a pair loads half of the B tile's rows
     if (!tmap_rows(&ta, hp, v.rows, v.F) || !tmap_experts(&tb, wd, v.E, v.d, v.F, pairs ? bn / 2 : bn))
@@ -186,12 +183,14 @@ moe_status_t down_impl(const Dims& v, const moe_bf16_t* hp, const int32_t* seg_e
     return cuda_status(launch_umma_gemm(kEpiStore, ta, tb, tb, g, grid, st));
 }
 
-moe_status_t segments_or_plan(const Dims& v, const int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets,
-                              int32_t* seg_first_rank, int32_t* status, cudaStream_t st) {
+moe_status_t segments_or_plan(const Dims& v, int32_t* counts, const int32_t* partials, int n_partials,
+                              int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* status,
+                              cudaStream_t st) {
     if (v.R > 0)
-        return cuda_status(launch_plan(counts, v.E, v.R, v.S, v.k, v.B, seg_expert, seg_offsets, seg_first_rank,
-                                       status, st));
-    return cuda_status(launch_segments(counts, v.E, v.C, seg_expert, seg_offsets, seg_first_rank, st));
+        return cuda_status(launch_plan(counts, partials, n_partials, v.E, v.R, v.S, v.k, v.B, seg_expert, seg_offsets,
+                                       seg_first_rank, status, st));
+    return cuda_status(
+        launch_segments(counts, partials, n_partials, v.E, v.C, seg_expert, seg_offsets, seg_first_rank, st));
 }
 
 moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* ids, int32_t plan_ready,
@@ -203,10 +202,15 @@ moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* id
     if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
     const size_t need = permute_ws_bytes(v.T, v.k, v.E);
     if (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    const size_t scratch = permute_scratch_bytes(v.T, v.k, v.E);
     if (!plan_ready) {
-        moe_status_t s = cuda_status(launch_histogram(ids, v.T * v.k, v.E, counts, sm_count(), st));
+        // histogram partials + clearing of the look-back scratch in one launch, then the tables
+        int32_t* partials = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + scratch);
+        moe_status_t s = cuda_status(launch_histogram_partials(ids, v.T * v.k, v.E, partials,
+                                                               static_cast<uint32_t*>(ws), scratch, st));
         if (s != MOE_OK) return s;
-        s = segments_or_plan(v, counts, seg_expert, seg_offsets, seg_first_rank, status, st);
+        s = segments_or_plan(v, counts, partials, histogram_partial_ctas(v.T * v.k), seg_expert, seg_offsets,
+                             seg_first_rank, status, st);
         if (s != MOE_OK) return s;
     }
     PermuteArgs a{};
@@ -219,7 +223,7 @@ moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* id
     a.T = v.T; a.k = v.k; a.E = v.E; a.d = v.d; a.n_seg = v.n_seg;
     a.tokens_per_tile = permute_tokens_per_tile(v.T, v.k);
     a.n_tiles = permute_n_tiles(v.T, v.k);
-    return cuda_status(launch_permute(a, sm_count(), st));
+    return cuda_status(launch_permute(a, !plan_ready, sm_count(), st));
 }
 
 // Scratch of moe_dispatch_static: one array in the library's device image.  Host code
@@ -336,8 +340,8 @@ moe_status_t moe_segments(const moe_shape_t* shape, const int32_t* counts, int32
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (v.R > 0 || !counts || !seg_expert || !seg_offsets || !seg_first_rank) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_segments(counts, v.E, v.C, seg_expert, seg_offsets, seg_first_rank,
-                                       static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_segments(const_cast<int32_t*>(counts), nullptr, 0, v.E, v.C, seg_expert, seg_offsets,
+                                       seg_first_rank, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_plan_balanced(const moe_shape_t* shape, const int32_t* counts, int32_t* seg_expert,
@@ -346,8 +350,8 @@ moe_status_t moe_plan_balanced(const moe_shape_t* shape, const int32_t* counts, 
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (v.R == 0 || !counts || !seg_expert || !seg_offsets || !seg_first_rank) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_plan(counts, v.E, v.R, v.S, v.k, v.B, seg_expert, seg_offsets, seg_first_rank, status,
-                                   static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_plan(const_cast<int32_t*>(counts), nullptr, 0, v.E, v.R, v.S, v.k, v.B, seg_expert,
+                                   seg_offsets, seg_first_rank, status, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_ids, int32_t plan_ready,

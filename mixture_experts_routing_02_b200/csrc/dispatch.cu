@@ -75,16 +75,46 @@ __global__ void __launch_bounds__(256) histogram_kernel(const int32_t* __restric
         if (h[e] != 0) atomicAdd(counts + e, h[e]);
 }
 
+// Per-CTA histograms written to partials[cta][E] (every entry, zeros included), so nothing needs
+// clearing first and no global atomics are used; the segment / plan kernel sums them.  The same
+// launch clears the permutation's look-back words (zero_ptr), which the permutation reads next.
+__global__ void __launch_bounds__(256) histogram_partial_kernel(const int32_t* __restrict__ ids, int n, int E,
+                                                                int32_t* __restrict__ partials,
+                                                                uint32_t* __restrict__ zero_ptr, size_t zero_words) {
+    __shared__ int h[kMaxExperts];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    __syncthreads();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const int e = __ldg(ids + i);
+        if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(&h[e], 1);
+    }
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < zero_words;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x)
+        zero_ptr[i] = 0u;
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) partials[blockIdx.x * E + e] = h[e];
+}
+
+// counts[e] from the per-CTA partials (and written out), or read from counts when partials is null
+__device__ __forceinline__ int expert_count(const int32_t* counts_in, const int32_t* partials, int n_partials, int E,
+                                            int e, int32_t* counts_out) {
+    if (partials == nullptr) return counts_in[e];
+    int c = 0;
+    for (int g = 0; g < n_partials; ++g) c += partials[g * E + e];
+    counts_out[e] = c;
+    return c;
+}
+
 // ------------------------------------------------------------------------------ plain segments
 
-__global__ void __launch_bounds__(256) segments_kernel(const int32_t* __restrict__ counts, int E, int capacity,
-                                                       int32_t* seg_expert, int32_t* seg_offsets,
+__global__ void __launch_bounds__(256) segments_kernel(int32_t* counts, const int32_t* partials, int n_partials,
+                                                       int E, int capacity, int32_t* seg_expert, int32_t* seg_offsets,
                                                        int32_t* seg_first_rank) {
     __shared__ int warp_sums[8];
     const int e = threadIdx.x;
     int v = 0;
     if (e < E) {
-        const int c = counts[e];
+        const int c = expert_count(counts, partials, n_partials, E, e, counts);
         v = (capacity > 0 && c > capacity) ? capacity : c;
     }
     int total;
@@ -101,9 +131,9 @@ __global__ void __launch_bounds__(256) segments_kernel(const int32_t* __restrict
 
 constexpr int kMaxGroups = 256;
 
-__global__ void __launch_bounds__(256) plan_kernel(const int32_t* __restrict__ counts, int E, int R, int S, int k,
-                                                   int B, int32_t* seg_expert, int32_t* seg_offsets,
-                                                   int32_t* seg_first_rank, int32_t* status) {
+__global__ void __launch_bounds__(256) plan_kernel(int32_t* counts, const int32_t* partials, int n_partials, int E,
+                                                   int R, int S, int k, int B, int32_t* seg_expert,
+                                                   int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* status) {
     __shared__ int c[kMaxExperts];
     __shared__ int order[kMaxExperts];  // experts of each group by (count desc, id asc)
     __shared__ int given[kMaxExperts];  // rows an expert hands to other groups
@@ -122,7 +152,10 @@ __global__ void __launch_bounds__(256) plan_kernel(const int32_t* __restrict__ c
     const int n_seg = R * per_group;
     const int cap = S * k;
 
-    for (int e = tid; e < E; e += blockDim.x) { c[e] = counts[e]; given[e] = 0; }
+    for (int e = tid; e < E; e += blockDim.x) {
+        c[e] = expert_count(counts, partials, n_partials, E, e, counts);
+        given[e] = 0;
+    }
     __syncthreads();
     for (int g = tid; g < R; g += blockDim.x) {
         int s = 0;
@@ -442,8 +475,13 @@ int permute_n_tiles(int T, int k) {
     return (T + tpt - 1) / tpt;
 }
 
-size_t permute_ws_bytes(int T, int k, int E) {
+size_t permute_scratch_bytes(int T, int k, int E) {
     return 256 + static_cast<size_t>(permute_n_tiles(T, k)) * static_cast<size_t>(E) * sizeof(uint32_t);
+}
+
+size_t permute_ws_bytes(int T, int k, int E) {
+    return permute_scratch_bytes(T, k, E) +
+           static_cast<size_t>(kMaxHistogramPartials) * static_cast<size_t>(E) * sizeof(int32_t);
 }
 
 cudaError_t launch_histogram(const int32_t* ids, int n_pairs, int E, int32_t* counts, int num_sms,
@@ -457,21 +495,39 @@ cudaError_t launch_histogram(const int32_t* ids, int n_pairs, int E, int32_t* co
     return cudaGetLastError();
 }
 
-cudaError_t launch_segments(const int32_t* counts, int E, int capacity, int32_t* seg_expert, int32_t* seg_offsets,
-                            int32_t* seg_first_rank, cudaStream_t stream) {
-    segments_kernel<<<1, 256, 0, stream>>>(counts, E, capacity, seg_expert, seg_offsets, seg_first_rank);
+int histogram_partial_ctas(int n_pairs) {
+    int g = (n_pairs + 4095) / 4096;
+    if (g > kMaxHistogramPartials) g = kMaxHistogramPartials;
+    return g < 1 ? 1 : g;
+}
+
+cudaError_t launch_histogram_partials(const int32_t* ids, int n_pairs, int E, int32_t* partials, uint32_t* zero_ptr,
+                                      size_t zero_bytes, cudaStream_t stream) {
+    histogram_partial_kernel<<<histogram_partial_ctas(n_pairs), 256, 0, stream>>>(ids, n_pairs, E, partials, zero_ptr,
+                                                                                   zero_bytes / 4);
     return cudaGetLastError();
 }
 
-cudaError_t launch_plan(const int32_t* counts, int E, int R, int S, int k, int B, int32_t* seg_expert,
-                        int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* status, cudaStream_t stream) {
-    plan_kernel<<<1, 256, 0, stream>>>(counts, E, R, S, k, B, seg_expert, seg_offsets, seg_first_rank, status);
+cudaError_t launch_segments(int32_t* counts, const int32_t* partials, int n_partials, int E, int capacity,
+                            int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank, cudaStream_t stream) {
+    segments_kernel<<<1, 256, 0, stream>>>(counts, partials, n_partials, E, capacity, seg_expert, seg_offsets,
+                                           seg_first_rank);
     return cudaGetLastError();
 }
 
-cudaError_t launch_permute(const PermuteArgs& a, int num_sms, cudaStream_t stream) {
-    cudaError_t err = cudaMemsetAsync(a.ticket, 0, permute_ws_bytes(a.T, a.k, a.E), stream);
-    if (err != cudaSuccess) return err;
+cudaError_t launch_plan(int32_t* counts, const int32_t* partials, int n_partials, int E, int R, int S, int k, int B,
+                        int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* status,
+                        cudaStream_t stream) {
+    plan_kernel<<<1, 256, 0, stream>>>(counts, partials, n_partials, E, R, S, k, B, seg_expert, seg_offsets,
+                                       seg_first_rank, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, cudaStream_t stream) {
+    if (!ws_cleared) {
+        cudaError_t err = cudaMemsetAsync(a.ticket, 0, permute_scratch_bytes(a.T, a.k, a.E), stream);
+        if (err != cudaSuccess) return err;
+    }
     if (a.n_tiles == 0) return cudaSuccess;
     int grid = a.n_tiles < 8 * num_sms ? a.n_tiles : 8 * num_sms;
     permute_kernel<<<grid, kPermuteThreads, 0, stream>>>(a);

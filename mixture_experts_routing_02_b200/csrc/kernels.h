@@ -42,12 +42,14 @@ size_t gemm_smem_bytes(int stages, int mma_n);
 int gemm_pick_stages(int mma_n);
 cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                              const GemmArgs& g, int grid, cudaStream_t stream);
-// CTA-pair version (SwiGLU and plain epilogues only): 256-row tiles; B tiles of mma_n/2 rows per CTA.
+// CTA-pair version (plain fp32 epilogue, i.e. the down projection): 256-row tiles; B tiles of
+// mma_n/2 rows per CTA.
 size_t gemm_pair_smem_bytes(int stages, int mma_n);
 int gemm_pair_pick_stages(int mma_n);
 cudaError_t launch_umma_gemm_pair(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                                   const GemmArgs& g, int n_pairs, cudaStream_t stream);
 constexpr int kPairMinRowsPerSegment = 192;  // average rows per segment from which pairs pay off
+constexpr int kPairMaxReduction = 4096;      // the down projection uses pairs up to this d_ff
 
 // dispatch.cu
 constexpr int kPermuteThreads = 256;
@@ -69,17 +71,29 @@ struct PermuteArgs {
     int T, k, E, d, n_seg, tokens_per_tile, n_tiles;
 };
 
+constexpr int kMaxHistogramPartials = 64;   // CTAs of the fused histogram (one partial count row each)
+
 int permute_tokens_per_tile(int T, int k);
 int permute_n_tiles(int T, int k);
+// Dispatch workspace: [ticket, 256 B][look-back words, n_tiles * E * 4 B] = the permutation's
+// scratch, then [histogram partials, kMaxHistogramPartials * E * 4 B].
+size_t permute_scratch_bytes(int T, int k, int E);
 size_t permute_ws_bytes(int T, int k, int E);
+int histogram_partial_ctas(int n_pairs);
 
 cudaError_t launch_histogram(const int32_t* ids, int n_pairs, int E, int32_t* counts, int num_sms,
                              cudaStream_t stream);
-cudaError_t launch_segments(const int32_t* counts, int E, int capacity, int32_t* seg_expert, int32_t* seg_offsets,
-                            int32_t* seg_first_rank, cudaStream_t stream);
-cudaError_t launch_plan(const int32_t* counts, int E, int R, int S, int k, int B, int32_t* seg_expert,
-                        int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* status, cudaStream_t stream);
-cudaError_t launch_permute(const PermuteArgs& a, int num_sms, cudaStream_t stream);
+// partial histograms (partials[histogram_partial_ctas(n)][E]) + clearing zero_bytes at zero_ptr
+cudaError_t launch_histogram_partials(const int32_t* ids, int n_pairs, int E, int32_t* partials, uint32_t* zero_ptr,
+                                      size_t zero_bytes, cudaStream_t stream);
+// partials == nullptr: counts is the input; else counts is written as the sum of the partials
+cudaError_t launch_segments(int32_t* counts, const int32_t* partials, int n_partials, int E, int capacity,
+                            int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank, cudaStream_t stream);
+cudaError_t launch_plan(int32_t* counts, const int32_t* partials, int n_partials, int E, int R, int S, int k, int B,
+                        int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* status,
+                        cudaStream_t stream);
+// ws_cleared: the ticket and look-back words are already zero (cleared by the fused histogram)
+cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, cudaStream_t stream);
 cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                                      int num_sms, cudaStream_t stream);
 

@@ -597,7 +597,7 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, cons
 
 cudaError_t launch_umma_gemm_pair(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                                   const GemmArgs& g, int n_pairs, cudaStream_t stream) {
-    if (epi == kEpiSwiglu) return launch_pair<kEpiSwiglu>(a, b0, b1, g, n_pairs, stream);
+    // only the plain (down-projection) epilogue runs on pairs; see use_pairs_for_down in api.cu
     if (epi == kEpiStore) return launch_pair<kEpiStore>(a, b0, b1, g, n_pairs, stream);
     return cudaErrorInvalidValue;
 }
