@@ -197,9 +197,9 @@ MOE_API moe_status_t moe_plan_balanced(const moe_shape_t *shape, const int32_t *
  * Dispatch.  When plan_ready == 0 this computes counts
  * and the segment tables first (moe_histogram, then moe_plan_balanced if
  * n_groups > 0 else moe_segments), writing them to the given buffers; when
- * plan_ready != 0 they are inputs from earlier calls.  Then, in one pass with
- * a decoupled look-back over tiles of (t, j) pairs, each pair gets its
- * stable rank r inside its expert and its final row
+ * plan_ready != 0 they are inputs from earlier calls.  Then, with a decoupled
+ * look-back over tiles of (t, j) pairs, each pair gets its stable rank r
+ * inside its expert and its final row
  *   dest[t*k+j] = seg_offsets[s] + r - seg_first_rank[s]
  * for the segment s of that expert covering rank r (-1 if none: dropped), and
  * the token's row is copied straight to that slot ("MoonEP", section "이 기술은
@@ -230,8 +230,8 @@ MOE_API moe_status_t moe_dispatch(const moe_shape_t *shape, const moe_bf16_t *x,
  * device image instead of `ws`; every GPU on which the library is loaded holds
  * those 4 MiB until the process exits.  Shapes whose scratch would exceed
  * 4 MiB (256 + n_tiles * E * 4 + 64 * E * 4 bytes, n_tiles = ceil(T /
- * tokens_per_tile), tokens_per_tile = clamp(ceil(T / 1024), 1, max(1, 256 / k)))
- * are rejected with MOE_ERR_UNSUPPORTED before anything is enqueued.  No call allocates: the first call on each device looks up the
+ * max(1, 256 / k))) are rejected with MOE_ERR_UNSUPPORTED before anything is
+ * enqueued.  No call allocates: the first call on each device looks up the
  * array's device address (cudaGetSymbolAddress, with that device current) and
  * caches it, so make that first call before any stream capture begins.
  *

@@ -1,6 +1,6 @@
-// Dispatch kernels: histogram, segment tables (plain or balanced plan), and the
-// one-pass stable permutation that writes each (token, k) row straight into its
-// final expert-contiguous slot.
+// Dispatch kernels: histogram, segment tables (plain or balanced plan), the stable
+// rank of every (token, k) pair inside its expert, and the scatter that writes each
+// token row straight into its k final expert-contiguous slots.
 //
 // The permutation is a counting sort on the expert id with one digit pass: the
 // global histogram is known beforehand (histogram_kernel), and the rank of a
@@ -84,9 +84,15 @@ __global__ void __launch_bounds__(256) histogram_partial_kernel(const int32_t* _
     __shared__ int h[kMaxExperts];
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
     __syncthreads();
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
-        const int e = __ldg(ids + i);
-        if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(&h[e], 1);
+    // warp-aggregated: one shared atomic per distinct expert in a warp
+    const int lane = threadIdx.x & 31;
+    const int stride = gridDim.x * blockDim.x;
+    for (int base = blockIdx.x * blockDim.x; base < n; base += stride) {
+        const int i = base + threadIdx.x;
+        int e = i < n ? __ldg(ids + i) : -1;
+        if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) e = -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(same) - 1) atomicAdd(&h[e], __popc(same));
     }
     for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < zero_words;
          i += static_cast<size_t>(gridDim.x) * blockDim.x)
@@ -248,8 +254,7 @@ __global__ void __launch_bounds__(256) plan_kernel(int32_t* counts, const int32_
 
 // ------------------------------------------------------------------------------ stable rank + permute
 
-__global__ void __launch_bounds__(kPermuteThreads, 4) permute_kernel(const PermuteArgs a) {
-    __shared__ int s_dest[kPermutePairs];
+__global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs a) {
     __shared__ int s_wcnt[kPermuteWarps][kMaxExperts];
     __shared__ int s_excl[kMaxExperts];
     __shared__ int s_cbeg[kMaxExperts + 1];
@@ -287,7 +292,6 @@ __global__ void __launch_bounds__(kPermuteThreads, 4) permute_kernel(const Permu
     }
     __syncthreads();
 
-    const int vec_per_row = a.d / 8;  // 16-byte vectors of 8 bf16
     const unsigned lanemask_lt = (1u << lane) - 1u;
 
     for (;;) {
@@ -368,35 +372,45 @@ __global__ void __launch_bounds__(kPermuteThreads, 4) permute_kernel(const Permu
                 }
             }
             a.dest[q0 + tid] = dst;
-            s_dest[tid] = dst;
             if (dst >= 0) a.src[dst] = q0 + tid;
         }
         __syncthreads();
 
-        // 4. copy each token row once from X into its k slots (16-byte vectors, coalesced);
-        //    8 loads in flight per lane before the stores
-        for (int tl = warp; tl < t1 - t0; tl += kPermuteWarps) {
-            const uint4* xs = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + tl) * a.d);
-            int dj[kMaxTopK];
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------------------ row scatter
+
+// One warp per token: read the token's row of X once (16-byte vectors, 8 in flight per lane)
+// and write it to each of its k final slots.  Pure streaming: no shared memory, no barriers.
+__global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                           const int32_t* __restrict__ dest, int T, int k, int d,
+                                                           __nv_bfloat16* __restrict__ xp) {
+    const int lane = threadIdx.x & 31;
+    const int warps_total = gridDim.x * (blockDim.x >> 5);
+    const int vec_per_row = d / 8;
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
+        const int mine = lane < k ? __ldg(dest + static_cast<size_t>(t) * k + lane) : -1;
+        int dj[kMaxTopK];
 #pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j) dj[j] = (j < k) ? s_dest[tl * k + j] : -1;
-            for (int v = lane; v < vec_per_row; v += 32 * kCopyUnroll) {
-                uint4 val[kCopyUnroll];
+        for (int j = 0; j < kMaxTopK; ++j) dj[j] = __shfl_sync(0xffffffffu, mine, j);
+        const uint4* xs = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
+        for (int v = lane; v < vec_per_row; v += 32 * kCopyUnroll) {
+            uint4 val[kCopyUnroll];
 #pragma unroll
-                for (int u = 0; u < kCopyUnroll; ++u)
-                    if (v + 32 * u < vec_per_row) val[u] = __ldg(xs + v + 32 * u);
+            for (int u = 0; u < kCopyUnroll; ++u)
+                if (v + 32 * u < vec_per_row) val[u] = __ldg(xs + v + 32 * u);
 #pragma unroll
-                for (int j = 0; j < kMaxTopK; ++j) {
-                    if (dj[j] >= 0) {
-                        uint4* dst = reinterpret_cast<uint4*>(a.xp + static_cast<size_t>(dj[j]) * a.d);
+            for (int j = 0; j < kMaxTopK; ++j) {
+                if (j < k && dj[j] >= 0) {
+                    uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(dj[j]) * d);
 #pragma unroll
-                        for (int u = 0; u < kCopyUnroll; ++u)
-                            if (v + 32 * u < vec_per_row) dst[v + 32 * u] = val[u];
-                    }
+                    for (int u = 0; u < kCopyUnroll; ++u)
+                        if (v + 32 * u < vec_per_row) dst[v + 32 * u] = val[u];
                 }
             }
         }
-        __syncthreads();
     }
 }
 
@@ -462,11 +476,9 @@ __global__ void __launch_bounds__(256) route_from_logits_kernel(const float* __r
 }  // namespace
 
 int permute_tokens_per_tile(int T, int k) {
-    // about kPermuteTargetTiles tiles (enough CTAs to fill the GPU with row copies), at most
-    // kPermutePairs pairs per tile (one pair per thread), at least one token
-    int t = (T + kPermuteTargetTiles - 1) / kPermuteTargetTiles;
-    const int cap = kPermutePairs / k;
-    if (t > cap) t = cap;
+    // as many whole tokens as fit in kPermutePairs pairs (one pair per thread)
+    (void)T;
+    const int t = kPermutePairs / k;
     return t < 1 ? 1 : t;
 }
 
@@ -496,7 +508,7 @@ cudaError_t launch_histogram(const int32_t* ids, int n_pairs, int E, int32_t* co
 }
 
 int histogram_partial_ctas(int n_pairs) {
-    int g = (n_pairs + 4095) / 4096;
+    int g = (n_pairs + 1023) / 1024;
     if (g > kMaxHistogramPartials) g = kMaxHistogramPartials;
     return g < 1 ? 1 : g;
 }
@@ -530,7 +542,12 @@ cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, c
     }
     if (a.n_tiles == 0) return cudaSuccess;
     int grid = a.n_tiles < 8 * num_sms ? a.n_tiles : 8 * num_sms;
-    permute_kernel<<<grid, kPermuteThreads, 0, stream>>>(a);
+    rank_kernel<<<grid, kPermuteThreads, 0, stream>>>(a);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    int sgrid = (a.T + 7) / 8;
+    if (sgrid > 16 * num_sms) sgrid = 16 * num_sms;
+    scatter_rows_kernel<<<sgrid, 256, 0, stream>>>(a.x, a.dest, a.T, a.k, a.d, a.xp);
     return cudaGetLastError();
 }
 

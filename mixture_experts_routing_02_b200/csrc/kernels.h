@@ -54,7 +54,6 @@ constexpr int kPairMaxReduction = 4096;      // the down projection uses pairs u
 // dispatch.cu
 constexpr int kPermuteThreads = 256;
 constexpr int kPermutePairs = 256;          // most (t, j) pairs per look-back tile (one per thread)
-constexpr int kPermuteTargetTiles = 1024;   // tiles aimed for, so the row copies fill the GPU
 
 struct PermuteArgs {
     const int32_t* ids;
