@@ -73,8 +73,10 @@ def test_layer_matches_oracle(w):
     check_layer_output(to_np(got["out"]), ref.out, ref.dest, w.T, w.k)
 
 
-def test_route_logits_and_bias():
-    w = syn.Workload("route", T=333, d=320, E=40, k=5, F=64, zipf_s=1.2)
+@pytest.mark.parametrize("E", [5, 24, 32, 33, 40, 256])
+def test_route_logits_and_bias(E):
+    """Both routers: CUDA cores for E <= 32, tensor cores above."""
+    w = syn.Workload("route", T=333, d=320, E=E, k=min(5, E), F=64, zipf_s=1.2)
     case = make_case(w, seed=2)
     s = moe_shape(w)
     logits = torch.empty(w.T, w.E, device="cuda")
