@@ -115,12 +115,6 @@ moe_status_t route_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_
     if (!x || !w_router || !ids || !w) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
     if (v.T == 0) return MOE_OK;
-    if (v.E <= kRouteSimtMaxExperts) {
-        // few experts: a thin pass over X, on the CUDA cores over every SM
-        return cuda_status(launch_route_simt(reinterpret_cast<const __nv_bfloat16*>(x),
-                                             reinterpret_cast<const __nv_bfloat16*>(w_router), bias, v.T, v.d, v.E,
-                                             v.k, logits, ids, w, sm_count(), st));
-    }
     if (!have_encoder()) return MOE_ERR_CUDA;
     const int epad = std::max(16, (v.E + 15) / 16 * 16);
     CUtensorMap ta, tb;

@@ -96,11 +96,6 @@ cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, c
 cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                                      int num_sms, cudaStream_t stream);
 
-// route.cu: CUDA-core router for small expert counts
-constexpr int kRouteSimtMaxExperts = 32;
-cudaError_t launch_route_simt(const __nv_bfloat16* x, const __nv_bfloat16* w_router, const float* bias, int T, int d,
-                              int E, int k, float* logits, int32_t* ids, float* w, int num_sms, cudaStream_t stream);
-
 // combine.cu
 cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, int T, int k, int d, float* out,
                            int num_sms, cudaStream_t stream);

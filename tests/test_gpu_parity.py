@@ -75,7 +75,7 @@ def test_layer_matches_oracle(w):
 
 @pytest.mark.parametrize("E", [5, 24, 32, 33, 40, 256])
 def test_route_logits_and_bias(E):
-    """Both routers: CUDA cores for E <= 32, tensor cores above."""
+    """The tensor-core router with N = E padded to a multiple of 16 (E = 5 ... 256)."""
     w = syn.Workload("route", T=333, d=320, E=E, k=min(5, E), F=64, zipf_s=1.2)
     case = make_case(w, seed=2)
     s = moe_shape(w)
