@@ -117,7 +117,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            self._stop.wait(0.1)
+            self._stop.wait(0.005)
 
     def __enter__(self):
         if self._nv is not None:
