@@ -300,8 +300,25 @@ def run_ours(args, w):
     yp = view(v.yp, rows_alloc * w.d, torch.float32)
     dws = view(v.dispatch_ws, v.dispatch_ws_bytes, torch.uint8)
 
+    Fs = args.shared_expert
+    if Fs:
+        gs, us, dsw = (t.to(dev) for t in syn.shared_expert_weights(w, Fs, seed))
+        h_s = torch.empty(w.T, Fs, dtype=torch.bfloat16, device=dev)
+        y_s = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
+        side = torch.cuda.Stream(device=dev)
+        shared_ms = []
+
     def step(ev):
         ev[0].record(stream)
+        if Fs:
+            # the shared expert runs on a side stream while the routed tokens are routed,
+            # dispatched and computed; the combine waits for it
+            side.wait_event(ev[0])
+            se0, se1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            se0.record(side)
+            moe.moe_shared_expert(s, Fs, x, gs, us, dsw, h_s, y_s, status, side)
+            se1.record(side)
+            shared_ms.append((se0, se1))
         moe.moe_route(s, x, w_r, bias, None, ids, wts, status, stream)
         ev[1].record(stream)
         moe.moe_dispatch(s, x, ids, 0, counts, seg_e, seg_o, seg_f, dest, src, xp, status, dws, stream)
@@ -310,7 +327,11 @@ def run_ours(args, w):
         ev[3].record(stream)
         moe.moe_expert_down(s, hp, seg_e, seg_o, wd, yp, status, stream)
         ev[4].record(stream)
-        moe.moe_combine(s, yp, dest, wts, out, stream)
+        if Fs:
+            stream.wait_event(shared_ms[-1][1])
+            moe.moe_combine_add(s, yp, dest, wts, y_s, out, stream)
+        else:
+            moe.moe_combine(s, yp, dest, wts, out, stream)
         ev[5].record(stream)
 
     # End to end through moe_layer_fwd: each step copies its X from pinned host memory to the
@@ -392,6 +413,12 @@ def run_ours(args, w):
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, world)
 
+    shared_info = None
+    if Fs:
+        sm = [a.elapsed_time(b) for a, b in shared_ms[-args.steps:]]
+        shared_info = {"d_ff_shared": Fs, "ms_alone_on_side_stream": statistics.mean(sm),
+                       "flops": 6 * w.T * w.d * Fs,
+                       "note": "runs concurrently with route/dispatch/gate_up/down; the combine waits for it"}
     hbm, bf16, bf16_sus, peak_kind = _peaks()
     avg = {k: statistics.mean(v) for k, v in per_kernel.items()}
     T, d, E, k, F = w.T, w.d, w.E, w.k, w.F
@@ -436,6 +463,10 @@ def run_ours(args, w):
                 "d2h_bytes_per_step": T * d * 4, "api": "moe_layer_fwd; per step X (bf16) copied in from pinned host memory and out (fp32) copied back; steps pipelined over copy-in / compute / copy-out streams with double-buffered device buffers"},
         "clocks": clocks.summary(),
     }
+    if shared_info:
+        line["shared_expert"] = shared_info
+        line["config"]["shared_expert_d_ff"] = Fs
+        line["gpu_launches"] = (LAUNCHES_PER_STEP + 2) * args.steps
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         wg0, wu0, wd0 = wg[:1].cpu(), wu[:1].cpu(), wd[:1].cpu()
         cv, desc, _ = _oracle_sample(w, seed, 512, 32, wg0, wu0, wd0)
@@ -459,6 +490,8 @@ def main():
     ap.add_argument("--workload", default=syn.MIXTRAL_LIKE.name, choices=sorted(syn.WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shared-expert", type=int, default=0, metavar="F_S",
+                    help="add one shared expert of inner size F_S, overlapped on a second stream")
     args = ap.parse_args()
     w = syn.WORKLOADS[args.workload]
     if args.impl == "reference":

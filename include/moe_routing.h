@@ -92,7 +92,16 @@ typedef enum {
  *                  돌려봤습니다", sections "개요" and "이 기술은 무엇인가").
  *                  Requires E % R == 0, T % R == 0 and capacity == 0.
  *   replica_slots  B, replica slots per group (the page's [E, E+B) slots).
+ *   route_flags    0: weights = softmax over the k selected logits (default);
+ *                  MOE_ROUTE_SOFTMAX_ALL: weights = softmax over all E logits,
+ *                  taken at the k selected experts and not renormalised (they
+ *                  sum to less than 1).  "Sparsely-Gated MoE 구현 관점에서
+ *                  살펴보기", section "Top-2 라우팅의 수치 예시": whether the
+ *                  softmax comes before or after the top-k differs between
+ *                  implementations; with renormalisation both orders agree.
  */
+#define MOE_ROUTE_SOFTMAX_ALL 0x1
+
 typedef struct {
     int32_t T;
     int32_t d_model;
@@ -102,6 +111,7 @@ typedef struct {
     int32_t capacity;
     int32_t n_groups;
     int32_t replica_slots;
+    int32_t route_flags;
 } moe_shape_t;
 
 /*
@@ -144,6 +154,7 @@ MOE_API moe_status_t moe_workspace_size(const moe_shape_t *shape, size_t *dispat
  *   topk_ids [T, k] int32 out: the k largest logits, descending; equal
  *            values go to the lower expert id
  *   topk_w   [T, k] fp32 out: w_j = exp(l_j - l_max) / sum_sel exp(l - l_max)
+ *            (with MOE_ROUTE_SOFTMAX_ALL the sum runs over all E logits)
  * The projection runs on the tensor cores (bf16 in, fp32 accumulate); the
  * selection is made on the fp32 logits.
  */
@@ -289,6 +300,34 @@ MOE_API moe_status_t moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *
  */
 MOE_API moe_status_t moe_combine(const moe_shape_t *shape, const float *yp, const int32_t *dest,
                          const float *topk_w, float *out, moe_stream_t stream);
+
+/*
+ * Combine with a base term: out[t] = base[t] + the combine above (base [T, d]
+ * fp32, nullable: then identical to moe_combine).  With base = the shared
+ * expert's output (moe_shared_expert) this finishes a layer with a shared
+ * expert.  out may alias base.
+ */
+MOE_API moe_status_t moe_combine_add(const moe_shape_t *shape, const float *yp, const int32_t *dest,
+                             const float *topk_w, const float *base, float *out,
+                             moe_stream_t stream);
+
+/*
+ * Shared expert: a dense SwiGLU FFN applied to every token, y_s = silu(X W_gs^T) *
+ * (X W_us^T) W_ds^T ("5.3 Expert Parallelism", section "3. 고도화된 최적화:
+ * 오버래핑(Overlapping) 및 GroupGEMM", first optimisation: the shared expert is
+ * local to every device, so its GEMMs can run on a second stream while the
+ * routed tokens are being routed and dispatched).  Same tensor-core kernels as
+ * the routed experts, as one segment of T rows.
+ *   d_ff_shared  F_s, multiple of 64
+ *   x [T, d] bf16; w_gate_s, w_up_s [F_s, d] bf16; w_down_s [d, F_s] bf16
+ *   h_s [T, F_s] bf16 (scratch, written); y_s [T, d] fp32 out.
+ * Enqueued on `stream`; to overlap, use a stream other than the routed path's
+ * and make moe_combine_add wait for it.
+ */
+MOE_API moe_status_t moe_shared_expert(const moe_shape_t *shape, int32_t d_ff_shared, const moe_bf16_t *x,
+                               const moe_bf16_t *w_gate_s, const moe_bf16_t *w_up_s,
+                               const moe_bf16_t *w_down_s, moe_bf16_t *h_s, float *y_s,
+                               int32_t *status, moe_stream_t stream);
 
 /*
  * The whole layer: moe_route (logits not stored) -> moe_dispatch ->

@@ -17,8 +17,9 @@ __all__ = [
     "MoeError", "MoeShape", "MoeLayerViews", "LIB_PATH", "SYMBOLS", "load_library", "shape",
     "moe_status_string", "moe_layout", "moe_workspace_size", "moe_route", "moe_route_from_logits",
     "moe_histogram", "moe_segments", "moe_plan_balanced", "moe_dispatch", "moe_dispatch_static", "moe_expert_gate_up",
-    "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_layer_fwd", "moe_layer_views",
-    "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT",
+    "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_combine_add", "moe_shared_expert", "moe_layer_fwd",
+    "moe_layer_views",
+    "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT", "ROUTE_SOFTMAX_ALL",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -33,7 +34,8 @@ class MoeError(RuntimeError):
 
 class MoeShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("T", "d_model", "n_experts", "top_k", "d_ff", "capacity", "n_groups", "replica_slots")]
+                ("T", "d_model", "n_experts", "top_k", "d_ff", "capacity", "n_groups", "replica_slots",
+                 "route_flags")]
 
 
 class MoeLayerViews(ctypes.Structure):
@@ -62,6 +64,8 @@ SYMBOLS = {
     "moe_expert_down": [_S, _P, _P, _P, _P, _P, _P, _P],
     "moe_expert_ffn": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_combine": [_S, _P, _P, _P, _P, _P],
+    "moe_combine_add": [_S, _P, _P, _P, _P, _P, _P],
+    "moe_shared_expert": [_S, _I, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_layer_fwd": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_layer_views": [_S, _P, ctypes.POINTER(MoeLayerViews)],
 }
@@ -86,8 +90,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     return lib
 
 
-def shape(T, d_model, n_experts, top_k, d_ff, capacity=0, n_groups=0, replica_slots=0) -> MoeShape:
-    return MoeShape(T, d_model, n_experts, top_k, d_ff, capacity, n_groups, replica_slots)
+ROUTE_SOFTMAX_ALL = 0x1
+
+
+def shape(T, d_model, n_experts, top_k, d_ff, capacity=0, n_groups=0, replica_slots=0, route_flags=0) -> MoeShape:
+    return MoeShape(T, d_model, n_experts, top_k, d_ff, capacity, n_groups, replica_slots, route_flags)
 
 
 def _ptr(t) -> Optional[int]:
@@ -191,6 +198,17 @@ def moe_expert_ffn(s, xp, seg_expert, seg_offsets, w_gate, w_up, w_down, hp, yp,
 def moe_combine(s, yp, dest, topk_w, out, stream=None):
     _check("moe_combine", load_library().moe_combine(
         ctypes.byref(s), _ptr(yp), _ptr(dest), _ptr(topk_w), _ptr(out), _stream(stream)))
+
+
+def moe_combine_add(s, yp, dest, topk_w, base, out, stream=None):
+    _check("moe_combine_add", load_library().moe_combine_add(
+        ctypes.byref(s), _ptr(yp), _ptr(dest), _ptr(topk_w), _ptr(base), _ptr(out), _stream(stream)))
+
+
+def moe_shared_expert(s, d_ff_shared, x, w_gate_s, w_up_s, w_down_s, h_s, y_s, status=None, stream=None):
+    _check("moe_shared_expert", load_library().moe_shared_expert(
+        ctypes.byref(s), int(d_ff_shared), _ptr(x), _ptr(w_gate_s), _ptr(w_up_s), _ptr(w_down_s), _ptr(h_s),
+        _ptr(y_s), _ptr(status), _stream(stream)))
 
 
 def moe_layer_fwd(s, x, w_router, bias, w_gate, w_up, w_down, out, status, ws, stream=None):

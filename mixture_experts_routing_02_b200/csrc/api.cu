@@ -46,7 +46,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Dims {
-    int T, d, E, k, F, C, R, B, S;
+    int T, d, E, k, F, C, R, B, S, flags;
     int n_seg;
     int rows;  // rows_alloc
 };
@@ -55,7 +55,8 @@ moe_status_t check_shape(const moe_shape_t* s, Dims* out) {
     if (s == nullptr) return MOE_ERR_INVALID_ARG;
     Dims v;
     v.T = s->T; v.d = s->d_model; v.E = s->n_experts; v.k = s->top_k; v.F = s->d_ff;
-    v.C = s->capacity; v.R = s->n_groups; v.B = s->replica_slots;
+    v.C = s->capacity; v.R = s->n_groups; v.B = s->replica_slots; v.flags = s->route_flags;
+    if (v.flags & ~MOE_ROUTE_SOFTMAX_ALL) return MOE_ERR_INVALID_ARG;
     if (v.T < 0 || v.d < 1 || v.E < 1 || v.k < 1 || v.k > v.E || v.F < 1 || v.C < 0 || v.R < 0 || v.B < 0)
         return MOE_ERR_INVALID_ARG;
     if (v.R > 0 && (v.E % v.R != 0 || v.T % v.R != 0 || v.C > 0)) return MOE_ERR_INVALID_ARG;
@@ -129,6 +130,7 @@ moe_status_t route_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_
     g.seg_offsets = nullptr; g.seg_expert = nullptr; g.n_seg = 1; g.M = v.T; g.K = v.d; g.N = v.E;
     g.BN = epad; g.n_tiles_n = 1; g.mma_n = epad; g.stages = gemm_pick_stages(epad);
     g.bias = bias; g.logits = logits; g.topk_ids = ids; g.topk_w = w; g.k = v.k; g.status = status;
+    g.route_flags = v.flags;
     const int grid = std::min(sm_count(), (v.T + 127) / 128);
     return cuda_status(launch_umma_gemm(kEpiRoute, ta, tb, tb, g, grid, st));
 }
@@ -322,7 +324,7 @@ moe_status_t moe_route_from_logits(const moe_shape_t* shape, const float* logits
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_route_from_logits(logits, v.T, v.E, v.k, topk_ids, topk_w, sm_count(),
+    return cuda_status(launch_route_from_logits(logits, v.T, v.E, v.k, v.flags, topk_ids, topk_w, sm_count(),
                                                 static_cast<cudaStream_t>(stream)));
 }
 
@@ -417,8 +419,65 @@ moe_status_t moe_combine(const moe_shape_t* shape, const float* yp, const int32_
     if (s != MOE_OK) return s;
     if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(yp) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_combine(yp, dest, topk_w, v.T, v.k, v.d, out, sm_count(),
+    return cuda_status(launch_combine(yp, dest, topk_w, nullptr, v.T, v.k, v.d, out, sm_count(),
                                       static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_combine_add(const moe_shape_t* shape, const float* yp, const int32_t* dest, const float* topk_w,
+                             const float* base, float* out, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(yp) || !aligned16(out) || (base && !aligned16(base))) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_combine(yp, dest, topk_w, base, v.T, v.k, v.d, out, sm_count(),
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_shared_expert(const moe_shape_t* shape, int32_t d_ff_shared, const moe_bf16_t* x,
+                               const moe_bf16_t* w_gate_s, const moe_bf16_t* w_up_s, const moe_bf16_t* w_down_s,
+                               moe_bf16_t* h_s, float* y_s, int32_t* status, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    const int Fs = d_ff_shared;
+    if (Fs < 1) return MOE_ERR_INVALID_ARG;
+    if (Fs % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if (!x || !w_gate_s || !w_up_s || !w_down_s || !h_s || !y_s) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_gate_s) || !aligned16(w_up_s) || !aligned16(w_down_s) || !aligned16(h_s) ||
+        !aligned16(y_s))
+        return MOE_ERR_INVALID_ARG;
+    if (v.T == 0) return MOE_OK;
+    if (!have_encoder()) return MOE_ERR_CUDA;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // one segment of all T rows and a single "expert": the same kernels as the routed FFN
+    {
+        const int bn = Fs >= 128 ? 128 : Fs;
+        CUtensorMap ta, tg, tu;
+        if (!tmap_rows(&ta, x, v.T, v.d) || !tmap_experts(&tg, w_gate_s, 1, Fs, v.d, bn) ||
+            !tmap_experts(&tu, w_up_s, 1, Fs, v.d, bn))
+            return MOE_ERR_CUDA;
+        GemmArgs g{};
+        g.seg_offsets = nullptr; g.seg_expert = nullptr; g.n_seg = 1; g.M = v.T; g.K = v.d; g.N = Fs;
+        g.BN = bn; g.n_tiles_n = (Fs + bn - 1) / bn; g.mma_n = 2 * bn; g.stages = gemm_pick_stages(2 * bn);
+        g.out = h_s; g.ldo = Fs; g.status = status;
+        const int64_t tiles = static_cast<int64_t>((v.T + 127) / 128) * g.n_tiles_n;
+        const int grid = static_cast<int>(std::min<int64_t>(sm_count(), tiles));
+        const moe_status_t r = cuda_status(launch_umma_gemm(kEpiSwiglu, ta, tg, tu, g, grid, st));
+        if (r != MOE_OK) return r;
+    }
+    {
+        const int bn = v.d >= 256 ? 256 : v.d;
+        CUtensorMap ta, tb;
+        if (!tmap_rows(&ta, h_s, v.T, Fs) || !tmap_experts(&tb, w_down_s, 1, v.d, Fs, bn)) return MOE_ERR_CUDA;
+        GemmArgs g{};
+        g.seg_offsets = nullptr; g.seg_expert = nullptr; g.n_seg = 1; g.M = v.T; g.K = Fs; g.N = v.d;
+        g.BN = bn; g.n_tiles_n = (v.d + bn - 1) / bn; g.mma_n = bn; g.stages = gemm_pick_stages(bn);
+        g.out = y_s; g.ldo = v.d; g.status = status;
+        const int64_t tiles = static_cast<int64_t>((v.T + 127) / 128) * g.n_tiles_n;
+        const int grid = static_cast<int>(std::min<int64_t>(sm_count(), tiles));
+        return cuda_status(launch_umma_gemm(kEpiStore, ta, tb, tb, g, grid, st));
+    }
 }
 
 moe_status_t moe_layer_views(const moe_shape_t* shape, void* ws, moe_layer_views_t* views) {
@@ -467,7 +526,7 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
     if (s != MOE_OK) return s;
     s = down_impl(v, w.hp, w.seg_expert, w.seg_offsets, w_down, w.yp, status, st);
     if (s != MOE_OK) return s;
-    return cuda_status(launch_combine(w.yp, w.dest, w.topk_w, v.T, v.k, v.d, out, sm_count(), st));
+    return cuda_status(launch_combine(w.yp, w.dest, w.topk_w, nullptr, v.T, v.k, v.d, out, sm_count(), st));
 }
 
 }  // extern "C"

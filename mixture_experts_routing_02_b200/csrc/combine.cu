@@ -1,5 +1,6 @@
-// Combine: out[t] = sum_j w[t, j] * Yp[dest[t*k + j]] over the kept pairs,
-// accumulated in fp32 in ascending j; Yp and out are fp32.
+// Combine: out[t] = base[t] + sum_j w[t, j] * Yp[dest[t*k + j]] over the kept pairs,
+// accumulated in fp32 in ascending j; Yp, base (optional, e.g. the shared expert's
+// output) and out are fp32.
 //
 // Sources: "Sparsely-Gated MoE 구현 관점에서 살펴보기", section "순전파 과정 ..."
 // (un-permute the expert outputs and combine them with the router weights);
@@ -21,8 +22,8 @@ namespace {
 // UNROLL: row vectors per lane whose gathers are all in flight together.
 template <int KMAX, int UNROLL>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ dest,
-                                                      const float* __restrict__ w, int T, int k, int d,
-                                                      float* __restrict__ out) {
+                                                      const float* __restrict__ w, const float* __restrict__ base,
+                                                      int T, int k, int d, float* __restrict__ out) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     const int vec_per_row = d / 4;  // float4 vectors
@@ -42,6 +43,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
             if (j >= k) dr[j] = -1;
         }
         float4* orow = reinterpret_cast<float4*>(out + static_cast<size_t>(t) * d);
+        const float4* brow = base ? reinterpret_cast<const float4*>(base + static_cast<size_t>(t) * d) : nullptr;
         for (int v0 = lane; v0 < vec_per_row; v0 += 32 * UNROLL) {
             // all gathers of UNROLL vectors issued before any is used
             float4 val[UNROLL][KMAX];
@@ -57,7 +59,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
             for (int u = 0; u < UNROLL; ++u) {
                 const int v = v0 + 32 * u;
                 if (v >= vec_per_row) break;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                float4 acc = brow ? __ldg(brow + v) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j) {
                     if (dr[j] >= 0) {
@@ -75,17 +77,17 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 }  // namespace
 
-cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, int T, int k, int d, float* out,
-                           int num_sms, cudaStream_t stream) {
+cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
+                           int d, float* out, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     int grid = (T + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
     if (k <= 2)
-        combine_kernel<2, 4><<<grid, 256, 0, stream>>>(yp, dest, w, T, k, d, out);
+        combine_kernel<2, 4><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, out);
     else if (k <= 4)
-        combine_kernel<4, 2><<<grid, 256, 0, stream>>>(yp, dest, w, T, k, d, out);
+        combine_kernel<4, 2><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, out);
     else
-        combine_kernel<kMaxTopK, 1><<<grid, 256, 0, stream>>>(yp, dest, w, T, k, d, out);
+        combine_kernel<kMaxTopK, 1><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, out);
     return cudaGetLastError();
 }
 

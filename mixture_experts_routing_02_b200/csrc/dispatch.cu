@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* 
 // ------------------------------------------------------------------------------ top-k from given logits
 
 __global__ void __launch_bounds__(256) route_from_logits_kernel(const float* __restrict__ logits, int T, int E,
-                                                                int k, int32_t* __restrict__ ids,
+                                                                int k, int route_flags, int32_t* __restrict__ ids,
                                                                 float* __restrict__ w) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
@@ -455,6 +455,15 @@ __global__ void __launch_bounds__(256) route_from_logits_kernel(const float* __r
                 si[j] = bi;
             }
         }
+        // denominator over all E logits (softmax-all mode), shifted by the largest (sv[0])
+        float all = 0.f;
+        if (route_flags & MOE_ROUTE_SOFTMAX_ALL) {
+#pragma unroll
+            for (int u = 0; u < kMaxExperts / 32; ++u)
+                if (lane + 32 * u < E) all += expf(v[u] - sv[0]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) all += __shfl_xor_sync(0xffffffffu, all, o);
+        }
         if (lane == 0) {
             float ex[kMaxTopK], sum = 0.f;
 #pragma unroll
@@ -462,7 +471,7 @@ __global__ void __launch_bounds__(256) route_from_logits_kernel(const float* __r
                 ex[j] = j < k ? expf(sv[j] - sv[0]) : 0.f;
                 sum += ex[j];
             }
-            const float inv = 1.0f / sum;
+            const float inv = 1.0f / ((route_flags & MOE_ROUTE_SOFTMAX_ALL) ? all : sum);
 #pragma unroll
             for (int j = 0; j < kMaxTopK; ++j)
                 if (j < k) {
@@ -551,12 +560,12 @@ cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, c
     return cudaGetLastError();
 }
 
-cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int32_t* ids, float* w,
-                                     int num_sms, cudaStream_t stream) {
+cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int route_flags, int32_t* ids,
+                                     float* w, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     int grid = (T + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
-    route_from_logits_kernel<<<grid, 256, 0, stream>>>(logits, T, E, k, ids, w);
+    route_from_logits_kernel<<<grid, 256, 0, stream>>>(logits, T, E, k, route_flags, ids, w);
     return cudaGetLastError();
 }
 

@@ -35,6 +35,7 @@ struct GemmArgs {
     int32_t* topk_ids;
     float* topk_w;
     int k;
+    int route_flags;  // MOE_ROUTE_SOFTMAX_ALL: weights from a softmax over all N logits
     int32_t* status;
 };
 
@@ -93,11 +94,11 @@ cudaError_t launch_plan(int32_t* counts, const int32_t* partials, int n_partials
                         cudaStream_t stream);
 // ws_cleared: the ticket and look-back words are already zero (cleared by the fused histogram)
 cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, cudaStream_t stream);
-cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int32_t* ids, float* w,
-                                     int num_sms, cudaStream_t stream);
+cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int route_flags, int32_t* ids,
+                                     float* w, int num_sms, cudaStream_t stream);
 
 // combine.cu
-cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, int T, int k, int d, float* out,
-                           int num_sms, cudaStream_t stream);
+cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
+                           int d, float* out, int num_sms, cudaStream_t stream);
 
 }  // namespace moe

@@ -305,6 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int ti[kMaxTopK];
 #pragma unroll
                 for (int j = 0; j < kMaxTopK; ++j) { tv[j] = -INFINITY; ti[j] = 0x7fffffff; }
+                const bool softmax_all = (g.route_flags & MOE_ROUTE_SOFTMAX_ALL) != 0;
+                float run_max = -INFINITY, run_sum = 0.f;  // online softmax denominator over all logits
                 for (int cc = 0; cc < g.N; cc += 32) {
                     uint32_t r[32];
                     tmem_ld32(t_row + cc, r);
@@ -316,6 +318,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             float v = __uint_as_float(r[i]);
                             if (g.bias != nullptr) v += __ldg(g.bias + e);
                             if (valid && g.logits != nullptr) g.logits[static_cast<size_t>(row) * g.N + e] = v;
+                            if (softmax_all) {
+                                if (v > run_max) {
+                                    run_sum = run_sum * expf(run_max - v) + 1.0f;
+                                    run_max = v;
+                                } else {
+                                    run_sum += expf(v - run_max);
+                                }
+                            }
                             // insertion into the sorted list; strict '>' keeps the lower id on ties
                             float cv = v;
                             int ci = e;
@@ -340,7 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ex[j] = (j < g.k) ? expf(tv[j] - tv[0]) : 0.f;
                         sum += ex[j];
                     }
-                    const float inv = 1.0f / sum;
+                    // run_max == tv[0]: the largest logit is the first selected one
+                    const float inv = 1.0f / (softmax_all ? run_sum : sum);
 #pragma unroll
                     for (int j = 0; j < kMaxTopK; ++j) {
                         if (j < g.k) {

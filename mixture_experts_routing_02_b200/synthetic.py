@@ -121,6 +121,15 @@ def expert_weights(w: Workload, seed: int = 0, device="cpu", experts: Optional[r
     return wg, wu, wd
 
 
+def shared_expert_weights(w: Workload, d_ff_shared: int, seed: int = 0, device="cpu"):
+    """The shared expert's W_gate, W_up [F_s, d] and W_down [d, F_s] (bf16)."""
+    out = []
+    for name, shape in (("ws_gate", (d_ff_shared, w.d)), ("ws_up", (d_ff_shared, w.d)), ("ws_down", (w.d, d_ff_shared))):
+        g = _gen(device, sub_seed(seed, name))
+        out.append((torch.randn(shape, generator=g, device=device) * WEIGHT_STD).to(torch.bfloat16))
+    return tuple(out)
+
+
 def lognormal_topk_ids(E: int, T: int, k: int, sigma: float, seed: int = 0) -> torch.Tensor:
     """Skewed routing ids [T, k] int32 drawn directly, without a router.
 
@@ -152,6 +161,6 @@ def ceil_div(a: int, b: int) -> int:
 
 __all__ = [
     "Workload", "TINY", "MIXTRAL_LIKE", "DEEPSEEK_LIKE", "SKEWED", "BALANCED", "WORKLOADS",
-    "sub_seed", "zipf_bias", "router_inputs", "x_row_redraw", "expert_weights",
+    "sub_seed", "zipf_bias", "router_inputs", "x_row_redraw", "expert_weights", "shared_expert_weights",
     "lognormal_topk_ids", "uniform_roundrobin_ids", "gib", "ceil_div",
 ]

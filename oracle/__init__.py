@@ -8,5 +8,6 @@ from .moe_oracle import (  # noqa: F401
     LayerResult, PlanInfeasible, PlanStats, Segments, balanced_plan, capacity_rows, combine,
     dispatch_positions, enforce_margin, expert_ffn, expert_rank, f64, grouped_expert_ffn,
     histogram, i64, layer_forward, margin_violations, num_segments, permute_rows,
-    plain_segments, route, router_logits, silu, token_output, topk_ids, topk_weights,
+    plain_segments, route, router_logits, shared_expert, silu, token_output, topk_ids, topk_weights,
+    topk_weights_softmax_all,
 )

@@ -120,11 +120,21 @@ def topk_weights(logits64: np.ndarray, ids: np.ndarray) -> np.ndarray:
     return e / e.sum(axis=1, keepdims=True)
 
 
-def route(x, w_router, bias, k: int):
+def topk_weights_softmax_all(logits64: np.ndarray, ids: np.ndarray) -> np.ndarray:
+    """The other order the page mentions, without renormalisation: a softmax over all E
+    logits, read at the selected experts (the k weights sum to less than 1)."""
+    l = np.asarray(logits64, dtype=np.float64)
+    e = np.exp(l - l.max(axis=1, keepdims=True))
+    p = e / e.sum(axis=1, keepdims=True)
+    return np.take_along_axis(p, ids, axis=1)
+
+
+def route(x, w_router, bias, k: int, softmax_all: bool = False):
     """(logits fp64 [T,E], ids int64 [T,k], weights fp64 [T,k])."""
     logits = router_logits(x, w_router, bias)
     ids = topk_ids(logits, k)
-    return logits, ids, topk_weights(logits, ids)
+    w = topk_weights_softmax_all(logits, ids) if softmax_all else topk_weights(logits, ids)
+    return logits, ids, w
 
 
 # ----------------------------------------------------------------------------
@@ -406,12 +416,24 @@ class LayerResult:
     plan: Optional[PlanStats] = None
 
 
+def shared_expert(x, w_gate_s, w_up_s, w_down_s) -> np.ndarray:
+    """The shared expert: one dense SwiGLU FFN applied to every token (fp64).
+
+    [EP-textbook] "3. 고도화된 최적화: 오버래핑(Overlapping) 및 GroupGEMM", first optimisation:
+    alongside the routed experts, one shared expert processes every token; its output is
+    added to the routed combine.
+    """
+    return expert_ffn(f64(x), w_gate_s, w_up_s, w_down_s)[1]
+
+
 def layer_forward(x, w_router, bias, w_gate, w_up, w_down, k: int,
-                  capacity: int = 0, n_groups: int = 0, replica_slots: int = 0) -> LayerResult:
-    """Router -> top-k -> (capacity | balanced plan) -> dispatch -> expert FFN -> combine."""
+                  capacity: int = 0, n_groups: int = 0, replica_slots: int = 0, shared=None,
+                  softmax_all: bool = False) -> LayerResult:
+    """Router -> top-k -> (capacity | balanced plan) -> dispatch -> expert FFN -> combine
+    (+ the shared expert's output when ``shared`` = (W_gate_s, W_up_s, W_down_s))."""
     T = x.shape[0]
     E = w_router.shape[0]
-    logits, ids, w = route(x, w_router, bias, k)
+    logits, ids, w = route(x, w_router, bias, k, softmax_all)
     counts = histogram(ids, E)
     plan = None
     if n_groups > 0:
@@ -424,6 +446,8 @@ def layer_forward(x, w_router, bias, w_gate, w_up, w_down, k: int,
     xp = permute_rows(x, src, k)
     hp, yp = grouped_expert_ffn(xp, segs, w_gate, w_up, w_down)
     out = combine(yp, dest, w, T, k)
+    if shared is not None:
+        out = out + shared_expert(x, *shared)
     return LayerResult(logits, ids, w, counts, segs, dest, src, xp, hp, yp, out, plan)
 
 

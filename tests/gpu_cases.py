@@ -107,10 +107,11 @@ def to_np(t):
     return t.detach().cpu().numpy()
 
 
-def run_layer(case: Case, capacity=None, stream=None):
+def run_layer(case: Case, capacity=None, stream=None, route_flags=0):
     """moe_layer_fwd through the C ABI; returns the output and every intermediate (CPU)."""
     w = case.w
     s = moe_shape(w, capacity)
+    s.route_flags = route_flags
     n_seg, rows = moe.moe_layout(s)
     _, layer_bytes = moe.moe_workspace_size(s)
     ws = torch.empty(layer_bytes, dtype=torch.uint8, device="cuda")

@@ -97,6 +97,7 @@ def test_workspace_sizes_grow_with_the_layer(lib):
     (dict(n_experts=300, top_k=2), 2), (dict(d_model=100), 2), (dict(d_ff=96), 2),
     (dict(n_experts=16, top_k=9), 2), (dict(T=1 << 29, top_k=2), 2),
     (dict(n_experts=256, n_groups=2, replica_slots=1000, T=64), 2),
+    (dict(route_flags=2), 1), (dict(route_flags=-1), 1),
 ])
 def test_shape_validation(lib, kw, code):
     s = _shape(**kw)

@@ -93,3 +93,23 @@ def test_full_size_layer(cuda_ok, w):
     sel_dest = np.concatenate([dest[t * w.k:(t + 1) * w.k] for t in toks])
     check_layer_output(to_np(got["out"][torch.tensor(toks, device="cuda")]), ref_out, sel_dest, len(toks), w.k,
                        "out (sampled tokens)")
+
+
+def test_full_size_shared_expert(cuda_ok):
+    """DeepSeek-like shape with one shared expert (F_s = 2048): sampled rows against the oracle."""
+    import mixture_experts_routing_02_b200 as moe
+    w = syn.DEEPSEEK_LIKE
+    Fs = 2048
+    x, _, _ = syn.router_inputs(w, 0)
+    gs, us, ds = syn.shared_expert_weights(w, Fs, 0)
+    s = moe.shape(w.T, w.d, w.E, w.k, w.F)
+    h_s = torch.empty(w.T, Fs, dtype=torch.bfloat16, device="cuda")
+    y_s = torch.empty(w.T, w.d, dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.moe_shared_expert(s, Fs, x.cuda(), gs.cuda(), us.cuda(), ds.cuda(), h_s, y_s, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    rng = np.random.default_rng(1)
+    toks = sorted(set(rng.choice(w.T, size=16, replace=False).tolist()) | {0, w.T - 1})
+    ref = oracle.shared_expert(x[toks], gs, us, ds)
+    check_close(to_np(y_s[torch.tensor(toks, device="cuda")]), ref, "shared expert (sampled tokens)")

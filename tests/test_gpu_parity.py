@@ -73,26 +73,42 @@ def test_layer_matches_oracle(w):
     check_layer_output(to_np(got["out"]), ref.out, ref.dest, w.T, w.k)
 
 
-@pytest.mark.parametrize("E", [5, 24, 32, 33, 40, 256])
-def test_route_logits_and_bias(E):
-    """The tensor-core router with N = E padded to a multiple of 16 (E = 5 ... 256)."""
+@pytest.mark.parametrize("E,flags", [(5, 0), (24, 0), (32, 0), (33, 0), (40, 0), (256, 0), (8, 1), (256, 1)])
+def test_layer_softmax_all_variant():
+    """The whole layer with weights from a softmax over all experts (no renormalisation)."""
+    w = syn.Workload("softmax-all", T=300, d=192, E=16, k=4, F=128, zipf_s=0.8)
+    case = make_case(w, seed=13)
+    ref = oracle.layer_forward(case.x, case.w_r, case.bias, case.wg, case.wu, case.wd, w.k, softmax_all=True)
+    got = run_layer(case, route_flags=moe.ROUTE_SOFTMAX_ALL)
+    assert got["status"] == 0
+    assert (got["ids"].numpy() == ref.ids).all()
+    assert np.abs(got["w"].numpy() - ref.weights).max() < 1e-5
+    assert (got["w"].numpy().sum(1) < 1).all()
+    check_layer_output(to_np(got["out"]), ref.out, ref.dest, w.T, w.k)
+
+
+def test_route_logits_and_bias(E, flags):
+    """The tensor-core router with N = E padded to a multiple of 16 (E = 5 ... 256); flags = 1 is
+    the softmax over all E without renormalisation."""
     w = syn.Workload("route", T=333, d=320, E=E, k=min(5, E), F=64, zipf_s=1.2)
     case = make_case(w, seed=2)
     s = moe_shape(w)
+    s.route_flags = flags
     logits = torch.empty(w.T, w.E, device="cuda")
     ids = i32(w.T * w.k).view(w.T, w.k)
     wt = torch.empty(w.T, w.k, device="cuda")
     st = i32(1)
     moe.moe_route(s, dev(case.x), dev(case.w_r), dev(case.bias), logits, ids, wt, st)
     torch.cuda.synchronize()
-    l64, rid, rw = oracle.route(case.x, case.w_r, case.bias, w.k)
+    l64, rid, rw = oracle.route(case.x, case.w_r, case.bias, w.k, softmax_all=bool(flags))
     check_close(to_np(logits), l64, "logits", max_abs_of_rms=1e-4, mean_rel=1e-5)
     assert (ids.cpu().numpy() == rid).all()
     assert np.abs(wt.cpu().numpy() - rw).max() < 1e-4
     assert st.item() == 0
 
 
-def test_route_from_logits_ties_and_exact_decision():
+@pytest.mark.parametrize("flags", [0, 1])
+def test_route_from_logits_ties_and_exact_decision(flags):
     T, E, k = 97, 37, 6
     rng = np.random.default_rng(5)
     l = rng.normal(size=(T, E)).astype(np.float32)
@@ -100,7 +116,7 @@ def test_route_from_logits_ties_and_exact_decision():
     l[:10, :] = 1.0              # rows of all-equal logits
     l[10, :] = np.float32(-3.0)
     l[10, 20] = 2.0
-    s = moe.shape(T, 64, E, k, 64)
+    s = moe.shape(T, 64, E, k, 64, route_flags=flags)
     ids = i32(T * k).view(T, k)
     wt = torch.empty(T, k, device="cuda")
     moe.moe_route_from_logits(s, torch.from_numpy(l).cuda(), ids, wt)
@@ -108,7 +124,8 @@ def test_route_from_logits_ties_and_exact_decision():
     l64 = l.astype(np.float64)
     rid = oracle.topk_ids(l64, k)
     assert (ids.cpu().numpy() == rid).all()
-    assert np.abs(wt.cpu().numpy() - oracle.topk_weights(l64, rid)).max() < 1e-6
+    ref_w = oracle.topk_weights_softmax_all(l64, rid) if flags else oracle.topk_weights(l64, rid)
+    assert np.abs(wt.cpu().numpy() - ref_w).max() < 1e-6
     assert list(ids.cpu().numpy()[0]) == list(range(k))
 
 
@@ -244,3 +261,65 @@ def test_repeated_calls_are_deterministic():
     b = run_layer(case)
     assert torch.equal(a["out"], b["out"]) and torch.equal(a["dest"], b["dest"])
     assert torch.equal(a["hp"], b["hp"])
+
+
+def _shared_case(seed=10):
+    w = syn.Workload("shared", T=333, d=192, E=6, k=2, F=128, zipf_s=1.0)
+    case = make_case(w, seed=seed)
+    Fs = 320
+    gs, us, ds = syn.shared_expert_weights(w, Fs, seed)
+    return w, case, Fs, (gs, us, ds)
+
+
+def test_shared_expert_and_combine_add():
+    """Shared expert (dense SwiGLU on every token) and the combine with a base term."""
+    w, case, Fs, sh = _shared_case()
+    ref = oracle.layer_forward(case.x, case.w_r, case.bias, case.wg, case.wu, case.wd, w.k, shared=sh)
+    s = moe_shape(w)
+    h_s = torch.empty(w.T, Fs, dtype=torch.bfloat16, device="cuda")
+    y_s = torch.empty(w.T, w.d, dtype=torch.float32, device="cuda")
+    st = i32(1)
+    moe.moe_shared_expert(s, Fs, dev(case.x), *(dev(t) for t in sh), h_s, y_s, st)
+    got = run_layer(case)
+    out = torch.empty(w.T, w.d, dtype=torch.float32, device="cuda")
+    v = moe.moe_layer_views(s, got["ws"])
+    base = got["ws"].data_ptr()
+    n_seg, rows = moe.moe_layout(s)
+    yp = got["yp"]
+    dest = got["ws"][v.dest - base:][: w.T * w.k * 4].view(torch.int32)
+    tw = got["ws"][v.topk_w - base:][: w.T * w.k * 4].view(torch.float32)
+    moe.moe_combine_add(s, yp, dest, tw, y_s, out)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    check_close(to_np(y_s), oracle.shared_expert(case.x, *sh), "shared expert")
+    check_close(to_np(out), ref.out, "routed + shared")
+    # base = None is exactly moe_combine
+    out2 = torch.empty_like(out)
+    moe.moe_combine_add(s, yp, dest, tw, None, out2)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, got["out"])
+
+
+def test_shared_expert_overlapped_on_a_second_stream():
+    """Run on a side stream while the routed path runs; joined by an event, the result is bit-identical."""
+    w, case, Fs, sh = _shared_case(seed=11)
+    s = moe_shape(w)
+    x = dev(case.x)
+    shd = [dev(t) for t in sh]
+    h1 = torch.empty(w.T, Fs, dtype=torch.bfloat16, device="cuda")
+    y1 = torch.empty(w.T, w.d, dtype=torch.float32, device="cuda")
+    moe.moe_shared_expert(s, Fs, x, *shd, h1, y1)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    start = torch.cuda.Event()
+    start.record()
+    side.wait_event(start)
+    h2 = torch.empty_like(h1)
+    y2 = torch.full_like(y1, float("nan"))
+    moe.moe_shared_expert(s, Fs, x, *shd, h2, y2, stream=side)
+    got = run_layer(case)                       # the routed path on the default stream meanwhile
+    done = torch.cuda.Event()
+    done.record(side)
+    torch.cuda.current_stream().wait_event(done)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)

@@ -75,6 +75,18 @@ def pin_weights_full_softmax(seed=1, T=50, E=16, k=4):
                 and (np.diff(w, axis=1) <= 0).all())
 
 
+def pin_weights_softmax_all(seed=12, T=40, E=12, k=3):
+    """Softmax over all E (library softmax), read at the selected experts, no renormalisation."""
+    rng = np.random.default_rng(seed)
+    logits = rng.normal(scale=2.0, size=(T, E))
+    ids = oracle.topk_ids(logits, k)
+    w = oracle.topk_weights_softmax_all(logits, ids)
+    p = torch.softmax(torch.from_numpy(logits), dim=1).numpy()
+    ref = np.take_along_axis(p, ids, axis=1)
+    return bool(np.allclose(w, ref, rtol=1e-12, atol=1e-15) and (w.sum(1) < 1).all()
+                and np.allclose(w / w.sum(1, keepdims=True), oracle.topk_weights(logits, ids), rtol=1e-12))
+
+
 def pin_router_logits_library(seed=2):
     g = torch.Generator().manual_seed(seed)
     x = torch.randn(37, 96, generator=g).to(torch.bfloat16)
@@ -140,6 +152,20 @@ def pin_dense_ffn_e1k1(seed=6):
     ref = F_.linear(F_.silu(F_.linear(xd, wg[0].double())) * F_.linear(xd, wu[0].double()),
                     wd[0].double()).numpy()
     return bool(np.allclose(res.out, ref, rtol=1e-11, atol=1e-13))
+
+
+def pin_shared_expert_additive(seed=8):
+    """With a shared expert the output is the routed output plus a dense SwiGLU FFN (library linear/silu)."""
+    T, E, k, Fs = 20, 6, 2, 96
+    x, wr, b, wg, wu, wd = _small_layer(seed, T=T, E=E, k=k)
+    w = syn.Workload("pin", T=T, d=64, E=E, k=k, F=64)
+    gs, us, ds = syn.shared_expert_weights(w, Fs, seed)
+    routed = oracle.layer_forward(x, wr, b, wg, wu, wd, k).out
+    both = oracle.layer_forward(x, wr, b, wg, wu, wd, k, shared=(gs, us, ds)).out
+    F_ = torch.nn.functional
+    xd = x.double()
+    dense = F_.linear(F_.silu(F_.linear(xd, gs.double())) * F_.linear(xd, us.double()), ds.double()).numpy()
+    return bool(np.allclose(both - routed, dense, rtol=1e-10, atol=1e-13))
 
 
 def pin_silu_library():
@@ -259,6 +285,10 @@ def test_weights_equal_full_softmax_then_renorm():
     assert pin_weights_full_softmax()
 
 
+def test_weights_softmax_all_variant():
+    assert pin_weights_softmax_all()
+
+
 def test_k1_weight_is_one():
     logits = np.random.default_rng(0).normal(size=(20, 8))
     w = oracle.topk_weights(logits, oracle.topk_ids(logits, 1))
@@ -295,6 +325,10 @@ def test_capacity_closed_form_skewed():
 
 def test_silu():
     assert pin_silu_library()
+
+
+def test_shared_expert_adds_a_dense_ffn():
+    assert pin_shared_expert_additive()
 
 
 def test_layer_equals_eager_loop():
@@ -387,10 +421,15 @@ def _mut_logits_no_bias(x, w_router, bias=None):
 
 
 _orig_combine = om.combine
+_orig_weights = om.topk_weights
 
 
 def _mut_combine_unweighted(yp64, dest, weights64, T, k):
     return _orig_combine(yp64, dest, np.ones_like(weights64), T, k)
+
+def _mut_shared_transposed(x, w_gate_s, w_up_s, w_down_s):
+    return om.expert_ffn(om.f64(x), w_up_s, w_gate_s, w_down_s)[1]   # gate and up swapped
+
 
 MUTATIONS = [
     ("silu", _mut_silu_sign, [pin_silu_library, pin_dense_ffn_e1k1]),
@@ -401,6 +440,8 @@ MUTATIONS = [
     ("expert_ffn", _mut_down_transposed, [pin_dense_ffn_e1k1]),
     ("router_logits", _mut_logits_no_bias, [pin_router_logits_library]),
     ("combine", _mut_combine_unweighted, [pin_layer_equals_eager]),
+    ("shared_expert", _mut_shared_transposed, [pin_shared_expert_additive]),
+    ("topk_weights_softmax_all", lambda l, i: _orig_weights(l, i), [pin_weights_softmax_all]),
 ]
 
 
