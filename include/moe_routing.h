@@ -340,6 +340,23 @@ MOE_API moe_status_t moe_layer_fwd(const moe_shape_t *shape, const moe_bf16_t *x
                            const moe_bf16_t *w_down, float *out, int32_t *status, void *ws,
                            size_t ws_bytes, moe_stream_t stream);
 
+/*
+ * Testing only: moe_dispatch (plan_ready = 0) with tile 0 of the stable-rank pass
+ * never taken, so every other tile's look-back waits on a flag that nothing sets.
+ * Each such wait gives up after its bound (about 2 s), sets MOE_DEV_ERR_TIMEOUT in
+ * *status and returns; dest / src / xp are then incomplete (pairs whose dest was
+ * not written keep the caller's values; values outside [0, rows_alloc) are never
+ * written through).  It shows that a wait that cannot end returns an error
+ * instead of hanging, and that the context stays usable.  Needs T large enough
+ * for at least two tiles (T * k > 256).
+ */
+MOE_API moe_status_t moe_testing_dispatch_stalled(const moe_shape_t *shape, const moe_bf16_t *x,
+                                          const int32_t *topk_ids, int32_t *counts,
+                                          int32_t *seg_expert, int32_t *seg_offsets,
+                                          int32_t *seg_first_rank, int32_t *dest, int32_t *src,
+                                          moe_bf16_t *xp, int32_t *status, void *ws, size_t ws_bytes,
+                                          moe_stream_t stream);
+
 /* Device addresses of the intermediates moe_layer_fwd keeps in its workspace. */
 typedef struct {
     int32_t *topk_ids;       /* [T, k] */

@@ -60,6 +60,7 @@ SYMBOLS = {
     "moe_plan_balanced": [_S, _P, _P, _P, _P, _P, _P],
     "moe_dispatch": [_S, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_dispatch_static": [_S, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "moe_testing_dispatch_stalled": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_expert_gate_up": [_S, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_expert_down": [_S, _P, _P, _P, _P, _P, _P, _P],
     "moe_expert_ffn": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
@@ -175,6 +176,15 @@ def moe_dispatch_static(s, x, topk_ids, plan_ready, counts, seg_expert, seg_offs
     _check("moe_dispatch_static", load_library().moe_dispatch_static(
         ctypes.byref(s), _ptr(x), _ptr(topk_ids), int(plan_ready), _ptr(counts), _ptr(seg_expert),
         _ptr(seg_offsets), _ptr(seg_first_rank), _ptr(dest), _ptr(src), _ptr(xp), _ptr(status), _stream(stream)))
+
+
+def moe_testing_dispatch_stalled(s, x, topk_ids, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp,
+                                 status, ws, stream=None):
+    """Testing only: a dispatch whose look-back waits cannot end; they time out (see the header)."""
+    _check("moe_testing_dispatch_stalled", load_library().moe_testing_dispatch_stalled(
+        ctypes.byref(s), _ptr(x), _ptr(topk_ids), _ptr(counts), _ptr(seg_expert), _ptr(seg_offsets),
+        _ptr(seg_first_rank), _ptr(dest), _ptr(src), _ptr(xp), _ptr(status), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_expert_gate_up(s, xp, seg_expert, seg_offsets, w_gate, w_up, hp, status=None, stream=None):

@@ -198,7 +198,7 @@ moe_status_t segments_or_plan(const Dims& v, int32_t* counts, const int32_t* par
 moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* ids, int32_t plan_ready,
                            int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank,
                            int32_t* dest, int32_t* src, moe_bf16_t* xp, int32_t* status, void* ws,
-                           size_t ws_bytes, cudaStream_t st) {
+                           size_t ws_bytes, cudaStream_t st, int first_tile = 0) {
     if (!x || !ids || !counts || !seg_expert || !seg_offsets || !seg_first_rank || !dest || !src || !xp)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
@@ -224,6 +224,8 @@ moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* id
     a.status = status;
     a.T = v.T; a.k = v.k; a.E = v.E; a.d = v.d; a.n_seg = v.n_seg;
     a.tokens_per_tile = permute_tokens_per_tile(v.T, v.k);
+    a.rows = v.rows;
+    a.first_tile = first_tile;
     a.n_tiles = permute_n_tiles(v.T, v.k);
     return cuda_status(launch_permute(a, !plan_ready, sm_count(), st));
 }
@@ -419,8 +421,20 @@ moe_status_t moe_combine(const moe_shape_t* shape, const float* yp, const int32_
     if (s != MOE_OK) return s;
     if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(yp) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_combine(yp, dest, topk_w, nullptr, v.T, v.k, v.d, out, sm_count(),
+    return cuda_status(launch_combine(yp, dest, topk_w, nullptr, v.T, v.k, v.d, v.rows, out, sm_count(),
                                       static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_testing_dispatch_stalled(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_ids,
+                                          int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets,
+                                          int32_t* seg_first_rank, int32_t* dest, int32_t* src, moe_bf16_t* xp,
+                                          int32_t* status, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (permute_n_tiles(v.T, v.k) < 2) return MOE_ERR_INVALID_ARG;  // needs a tile that waits on tile 0
+    return dispatch_impl(v, x, topk_ids, 0, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp, status,
+                         ws, ws_bytes, static_cast<cudaStream_t>(stream), 1);
 }
 
 moe_status_t moe_combine_add(const moe_shape_t* shape, const float* yp, const int32_t* dest, const float* topk_w,
@@ -430,7 +444,7 @@ moe_status_t moe_combine_add(const moe_shape_t* shape, const float* yp, const in
     if (s != MOE_OK) return s;
     if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(yp) || !aligned16(out) || (base && !aligned16(base))) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_combine(yp, dest, topk_w, base, v.T, v.k, v.d, out, sm_count(),
+    return cuda_status(launch_combine(yp, dest, topk_w, base, v.T, v.k, v.d, v.rows, out, sm_count(),
                                       static_cast<cudaStream_t>(stream)));
 }
 
@@ -526,7 +540,7 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
     if (s != MOE_OK) return s;
     s = down_impl(v, w.hp, w.seg_expert, w.seg_offsets, w_down, w.yp, status, st);
     if (s != MOE_OK) return s;
-    return cuda_status(launch_combine(w.yp, w.dest, w.topk_w, nullptr, v.T, v.k, v.d, out, sm_count(), st));
+    return cuda_status(launch_combine(w.yp, w.dest, w.topk_w, nullptr, v.T, v.k, v.d, v.rows, out, sm_count(), st));
 }
 
 }  // extern "C"

@@ -23,7 +23,7 @@ namespace {
 template <int KMAX, int UNROLL>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ dest,
                                                       const float* __restrict__ w, const float* __restrict__ base,
-                                                      int T, int k, int d, float* __restrict__ out) {
+                                                      int T, int k, int d, int rows, float* __restrict__ out) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     const int vec_per_row = d / 4;  // float4 vectors
@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
         for (int j = 0; j < KMAX; ++j) {
             dr[j] = __shfl_sync(0xffffffffu, mine_d, j);
             wr[j] = __shfl_sync(0xffffffffu, mine_w, j);
-            if (j >= k) dr[j] = -1;
+            if (j >= k || dr[j] >= rows) dr[j] = -1;  // dropped, or outside Yp: contributes nothing
         }
         float4* orow = reinterpret_cast<float4*>(out + static_cast<size_t>(t) * d);
         const float4* brow = base ? reinterpret_cast<const float4*>(base + static_cast<size_t>(t) * d) : nullptr;
@@ -78,16 +78,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 }  // namespace
 
 cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
-                           int d, float* out, int num_sms, cudaStream_t stream) {
+                           int d, int rows, float* out, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     int grid = (T + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
     if (k <= 2)
-        combine_kernel<2, 4><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, out);
+        combine_kernel<2, 4><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
     else if (k <= 4)
-        combine_kernel<4, 2><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, out);
+        combine_kernel<4, 2><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
     else
-        combine_kernel<kMaxTopK, 1><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, out);
+        combine_kernel<kMaxTopK, 1><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
     return cudaGetLastError();
 }
 

@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs
     const unsigned lanemask_lt = (1u << lane) - 1u;
 
     for (;;) {
-        if (tid == 0) s_tile = static_cast<int>(atomicAdd(a.ticket, 1u));
+        if (tid == 0) s_tile = static_cast<int>(atomicAdd(a.ticket, 1u)) + a.first_tile;
         for (int i = tid; i < kPermuteWarps * kMaxExperts; i += blockDim.x) (&s_wcnt[0][0])[i] = 0;
         __syncthreads();
         const int tile = s_tile;
@@ -331,6 +331,7 @@ __global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs
                 int j = tile - 1;
                 uint64_t t_start = 0;
                 uint32_t spins = 0;
+                bool gave_up = false;
                 while (j >= 0) {
                     const uint32_t w = ld_relaxed_u32(a.tile_state + static_cast<size_t>(j) * E + tid);
                     const uint32_t flag = w & ~kValueMask;
@@ -341,6 +342,7 @@ __global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs
                             else if (now - t_start > kWaitLimitNs) {
                                 report(a.status, MOE_DEV_ERR_TIMEOUT);
                                 s_abort = 1;
+                                gave_up = true;
                                 break;
                             }
                         }
@@ -350,7 +352,8 @@ __global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs
                     if (flag == kFlagPrefix) break;
                     --j;
                 }
-                st_relaxed_u32(mine, kFlagPrefix | static_cast<uint32_t>(excl + h));
+                // a tile that gave up publishes no prefix, so the tiles after it give up too
+                if (!gave_up) st_relaxed_u32(mine, kFlagPrefix | static_cast<uint32_t>(excl + h));
             }
             s_excl[tid] = excl;
         }
@@ -386,7 +389,7 @@ __global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs
 // and write it to each of its k final slots.  Pure streaming: no shared memory, no barriers.
 __global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* __restrict__ x,
                                                            const int32_t* __restrict__ dest, int T, int k, int d,
-                                                           __nv_bfloat16* __restrict__ xp) {
+                                                           int rows, __nv_bfloat16* __restrict__ xp) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     const int vec_per_row = d / 8;
@@ -403,7 +406,7 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* 
                 if (v + 32 * u < vec_per_row) val[u] = __ldg(xs + v + 32 * u);
 #pragma unroll
             for (int j = 0; j < kMaxTopK; ++j) {
-                if (j < k && dj[j] >= 0) {
+                if (j < k && dj[j] >= 0 && dj[j] < rows) {
                     uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(dj[j]) * d);
 #pragma unroll
                     for (int u = 0; u < kCopyUnroll; ++u)
@@ -556,7 +559,7 @@ cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, c
     if (err != cudaSuccess) return err;
     int sgrid = (a.T + 7) / 8;
     if (sgrid > 16 * num_sms) sgrid = 16 * num_sms;
-    scatter_rows_kernel<<<sgrid, 256, 0, stream>>>(a.x, a.dest, a.T, a.k, a.d, a.xp);
+    scatter_rows_kernel<<<sgrid, 256, 0, stream>>>(a.x, a.dest, a.T, a.k, a.d, a.rows, a.xp);
     return cudaGetLastError();
 }
 

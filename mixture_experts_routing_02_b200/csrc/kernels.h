@@ -69,6 +69,8 @@ struct PermuteArgs {
     uint32_t* ticket;      // zero on entry
     int32_t* status;
     int T, k, E, d, n_seg, tokens_per_tile, n_tiles;
+    int rows;        // rows of xp: dest values outside [0, rows) are never written through
+    int first_tile;  // 0; 1 only in moe_testing_dispatch_stalled (tile 0 is never taken)
 };
 
 constexpr int kMaxHistogramPartials = 64;   // CTAs of the fused histogram (one partial count row each)
@@ -99,6 +101,6 @@ cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, i
 
 // combine.cu
 cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
-                           int d, float* out, int num_sms, cudaStream_t stream);
+                           int d, int rows, float* out, int num_sms, cudaStream_t stream);
 
 }  // namespace moe

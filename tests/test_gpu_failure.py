@@ -1,0 +1,63 @@
+"""Failure detection on the GPU without a fault: every spin-wait in the library is
+bounded, so a wait that can never end (a flag that nothing sets) gives up after
+about two seconds, reports MOE_DEV_ERR_TIMEOUT in the status word, and leaves the
+CUDA context usable.  The infeasible balanced plan (MOE_DEV_ERR_PLAN) is checked
+in test_gpu_parity.py."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import mixture_experts_routing_02_b200 as moe
+from mixture_experts_routing_02_b200 import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+
+def _buffers(s, T, k, d, E):
+    n_seg, rows = moe.moe_layout(s)
+    mk = lambda n, fill: torch.full((max(n, 1),), fill, dtype=torch.int32, device="cuda")
+    return dict(counts=mk(E, 0), seg_expert=mk(n_seg, 0), seg_offsets=mk(n_seg + 1, 0), seg_first_rank=mk(n_seg, 0),
+                dest=mk(T * k, -1), src=mk(rows, -1), xp=torch.zeros(rows, d, dtype=torch.bfloat16, device="cuda"),
+                status=torch.zeros(1, dtype=torch.int32, device="cuda"))
+
+
+def test_lookback_wait_that_cannot_end_times_out(cuda_ok):
+    T, d, E, k = 1000, 64, 16, 2               # 2000 pairs: 8 look-back tiles
+    s = moe.shape(T, d, E, k, 64)
+    ids = syn.lognormal_topk_ids(E, T, k, 1.0, seed=30).cuda()
+    x = torch.randn(T, d, generator=torch.Generator().manual_seed(31)).to(torch.bfloat16).cuda()
+    ws = torch.empty(moe.moe_workspace_size(s)[0], dtype=torch.uint8, device="cuda")
+
+    b = _buffers(s, T, k, d, E)
+    t0 = time.time()
+    moe.moe_testing_dispatch_stalled(s, x, ids, b["counts"], b["seg_expert"], b["seg_offsets"], b["seg_first_rank"],
+                                     b["dest"], b["src"], b["xp"], b["status"], ws)
+    torch.cuda.synchronize()
+    elapsed = time.time() - t0
+    assert b["status"].item() & moe.DEV_ERR_TIMEOUT
+    assert 1.0 < elapsed < 60.0
+    assert (b["dest"].cpu().numpy() == -1).all()   # no tile could finish its look-back
+
+    # the context is still usable: the same dispatch now gives the oracle's positions
+    g = _buffers(s, T, k, d, E)
+    moe.moe_dispatch(s, x, ids, 0, g["counts"], g["seg_expert"], g["seg_offsets"], g["seg_first_rank"], g["dest"],
+                     g["src"], g["xp"], g["status"], ws)
+    torch.cuda.synchronize()
+    assert g["status"].item() == 0
+    ids_np = ids.cpu().numpy()
+    segs = oracle.plain_segments(oracle.histogram(ids_np, E))
+    dest, _ = oracle.dispatch_positions(ids_np, segs, E)
+    assert (g["dest"].cpu().numpy() == dest).all()
+
+
+def test_stalled_dispatch_needs_two_tiles(cuda_ok):
+    s = moe.shape(10, 64, 4, 2, 64)              # 20 pairs: a single tile, nothing would wait
+    with pytest.raises(moe.MoeError):
+        dummy = torch.zeros(64, dtype=torch.int32, device="cuda")
+        moe.moe_testing_dispatch_stalled(s, torch.zeros(10, 64, dtype=torch.bfloat16, device="cuda"), dummy, dummy,
+                                         dummy, dummy, dummy, dummy, dummy,
+                                         torch.zeros(20, 64, dtype=torch.bfloat16, device="cuda"), None,
+                                         torch.zeros(1 << 16, dtype=torch.uint8, device="cuda"))
