@@ -62,7 +62,14 @@ SKEWED = Workload("skewed", T=8192, d=4096, E=64, k=2, F=1408,
 BALANCED = Workload("balanced-plan", T=32768, d=7168, E=256, k=8, F=2048,
                     zipf_s=1.2, n_groups=8, replica_slots=32)
 
-WORKLOADS = {w.name: w for w in (TINY, MIXTRAL_LIKE, DEEPSEEK_LIKE, SKEWED, BALANCED)}
+# Reduced copies for profiling captures that must stay at a few GB on the device: the same
+# per-expert shapes and rows per expert as the full workloads, with fewer experts.
+DEEPSEEK_LIKE_E32 = Workload("deepseek-like-e32", T=512, d=7168, E=32, k=8, F=2048)
+BALANCED_E32 = Workload("balanced-plan-e32", T=4096, d=7168, E=32, k=8, F=2048,
+                        zipf_s=1.2, n_groups=2, replica_slots=16)
+
+WORKLOADS = {w.name: w for w in (TINY, MIXTRAL_LIKE, DEEPSEEK_LIKE, SKEWED, BALANCED, DEEPSEEK_LIKE_E32,
+                                 BALANCED_E32)}
 
 
 def sub_seed(seed: int, tag: str, *idx: int) -> int:
@@ -160,7 +167,8 @@ def ceil_div(a: int, b: int) -> int:
 
 
 __all__ = [
-    "Workload", "TINY", "MIXTRAL_LIKE", "DEEPSEEK_LIKE", "SKEWED", "BALANCED", "WORKLOADS",
+    "Workload", "TINY", "MIXTRAL_LIKE", "DEEPSEEK_LIKE", "SKEWED", "BALANCED", "DEEPSEEK_LIKE_E32", "BALANCED_E32",
+    "WORKLOADS",
     "sub_seed", "zipf_bias", "router_inputs", "x_row_redraw", "expert_weights", "shared_expert_weights",
     "lognormal_topk_ids", "uniform_roundrobin_ids", "gib", "ceil_div",
 ]
