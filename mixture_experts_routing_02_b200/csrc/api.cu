@@ -104,10 +104,6 @@ inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 // fp32 epilogue is a large share of each tile; measured on B200 the pair kernel is then ~8 % faster.
 // Everything else (and the gate/up projection always) runs on single CTAs with 128-row tiles,
 // which measured as fast or faster: the contraction is power-limited, not operand-bandwidth-limited.
-bool use_two_row_tiles(const Dims& v) {
-    return v.n_seg > 0 && static_cast<int64_t>(v.rows) < static_cast<int64_t>(kPairMinRowsPerSegment) * v.n_seg;
-}
-
 bool use_pairs_for_down(const Dims& v) {
     return v.n_seg > 0 && v.F <= kPairMaxReduction &&
            static_cast<int64_t>(v.rows) >= static_cast<int64_t>(kPairMinRowsPerSegment) * v.n_seg;
@@ -146,11 +142,7 @@ moe_status_t gate_up_impl(const Dims& v, const moe_bf16_t* xp, const int32_t* se
     if (!aligned16(xp) || !aligned16(wg) || !aligned16(wu) || !aligned16(hp)) return MOE_ERR_INVALID_ARG;
     if (v.T == 0 || v.rows == 0) return MOE_OK;
     if (!have_encoder()) return MOE_ERR_CUDA;
-    // Short segments (about one 128-row tile per expert or less): each work unit computes two row
-    // tiles against one B tile of 64 gate + 64 up rows held in shared memory, so an expert whose
-    // rows spill just past 128 does not stream its weights into a second SM.
-    const int mt = use_two_row_tiles(v) ? 2 : 1;
-    const int bn = mt == 2 ? 64 : (v.F >= 128 ? 128 : v.F);
+    const int bn = v.F >= 128 ? 128 : v.F;
     CUtensorMap ta, tg, tu;
     if (!tmap_rows(&ta, xp, v.rows, v.d) || !tmap_experts(&tg, wg, v.E, v.F, v.d, bn) ||
         !tmap_experts(&tu, wu, v.E, v.F, v.d, bn))
@@ -159,10 +151,10 @@ moe_status_t gate_up_impl(const Dims& v, const moe_bf16_t* xp, const int32_t* se
     g.seg_offsets = seg_offsets; g.seg_expert = seg_expert; g.n_seg = v.n_seg; g.M = v.rows; g.K = v.d; g.N = v.F;
     g.BN = bn; g.n_tiles_n = (v.F + bn - 1) / bn; g.mma_n = 2 * bn;
     g.out = hp; g.ldo = v.F; g.k = v.k; g.status = status;
-    g.stages = gemm_pick_stages(2 * bn, mt);
-    const int64_t max_tiles = (static_cast<int64_t>(v.rows) / (128 * mt) + v.n_seg) * g.n_tiles_n;
+    g.stages = gemm_pick_stages(2 * bn);
+    const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 128 + v.n_seg) * g.n_tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(sm_count(), max_tiles));
-    return cuda_status(launch_umma_gemm(kEpiSwiglu, ta, tg, tu, g, grid, st, mt));
+    return cuda_status(launch_umma_gemm(kEpiSwiglu, ta, tg, tu, g, grid, st));
 }
 
 moe_status_t down_impl(const Dims& v, const moe_bf16_t* hp, const int32_t* seg_expert, const int32_t* seg_offsets,

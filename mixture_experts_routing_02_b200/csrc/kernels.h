@@ -39,11 +39,10 @@ struct GemmArgs {
     int32_t* status;
 };
 
-// mt: row tiles of 128 per work unit (2 only with the SwiGLU epilogue; then mma_n <= 128)
-size_t gemm_smem_bytes(int stages, int mma_n, int mt = 1);
-int gemm_pick_stages(int mma_n, int mt = 1);
+size_t gemm_smem_bytes(int stages, int mma_n);
+int gemm_pick_stages(int mma_n);
 cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                             const GemmArgs& g, int grid, cudaStream_t stream, int mt = 1);
+                             const GemmArgs& g, int grid, cudaStream_t stream);
 // CTA-pair version (plain fp32 epilogue, i.e. the down projection): 256-row tiles; B tiles of
 // mma_n/2 rows per CTA.
 size_t gemm_pair_smem_bytes(int stages, int mma_n);

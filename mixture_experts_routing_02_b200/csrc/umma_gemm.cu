@@ -159,10 +159,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& g, uint32_t t_row,
     }
 }
 
-// MT = row tiles per work unit.  MT = 2 (SwiGLU only) computes two 128-row tiles against one B tile
-// held in shared memory (two accumulators of mma_n <= 128 columns), so each weight byte enters one
-// SM once even when a segment is only a little longer than 128 rows.
-template <int EPI, int MT>
+template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
@@ -180,12 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x & 31;
     const int stages = g.stages;
     const uint32_t b_stage_bytes = static_cast<uint32_t>(g.mma_n) * 128u;
-    constexpr uint32_t a_stage_bytes = MT * kABytes;
-    constexpr int bm = MT * kBM;
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + stages * a_stage_bytes;
+    uint8_t* sB = smem + stages * kABytes;
     uint32_t* epi_stage = reinterpret_cast<uint32_t*>(sB + stages * b_stage_bytes);
 
     if (threadIdx.x == 0) {
@@ -205,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (EPI == kEpiSwiglu) tma_prefetch_desc(&tmB1);
     }
     if (warp == 1) tmem_alloc(&tmem_base_sh, kTmemCols);
-    if (warp == 2) build_tile_prefix(tile_prefix, g, bm, lane);
+    if (warp == 2) build_tile_prefix(tile_prefix, g, kBM, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -219,19 +214,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int stage = 0, issued = 0;
             uint32_t phase = 0;
-            const uint32_t tx = a_stage_bytes + (EPI == kEpiRoute ? static_cast<uint32_t>(g.N) * 128u : b_stage_bytes);
+            const uint32_t tx = kABytes + (EPI == kEpiRoute ? static_cast<uint32_t>(g.N) * 128u : b_stage_bytes);
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g, bm);
+                const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g);
                 const int n0 = c.n * g.BN;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, g.status)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full_bar[stage], tx);
-                    uint8_t* a_dst = sA + stage * a_stage_bytes;
+                    uint8_t* a_dst = sA + stage * kABytes;
                     uint8_t* b_dst = sB + stage * b_stage_bytes;
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
-                        tma_load_2d(a_dst + mt * kABytes, &tmA, kb * kBK, c.row0 + mt * kBM, &full_bar[stage]);
+                    tma_load_2d(a_dst, &tmA, kb * kBK, c.row0, &full_bar[stage]);
                     if (EPI == kEpiRoute) {
                         tma_load_2d(b_dst, &tmB0, kb * kBK, 0, &full_bar[stage]);
                     } else if (EPI == kEpiSwiglu) {
@@ -266,16 +259,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, &abort_sh, g.status)) { ok = false; break; }
                     tc_fence_after();
+                    const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * kABytes));
                     const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * b_stage_bytes));
 #pragma unroll
                     for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                         // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4)
-#pragma unroll
-                        for (int mt = 0; mt < MT; ++mt) {
-                            const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * a_stage_bytes + mt * kABytes));
-                            umma_bf16(d_tmem + static_cast<uint32_t>(mt * g.mma_n), adesc + 2 * kk, bdesc + 2 * kk,
-                                      idesc, (kb | kk) != 0 ? 1u : 0u);
-                        }
+                        umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     umma_commit(&empty_bar[stage]);
                     if (++stage == stages) { stage = 0; phase ^= 1u; }
@@ -297,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g, bm);
+            const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g);
             const bool got = mbar_wait(&tfull_bar[acc], acc_phase, &abort_sh, g.status);
             if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
@@ -308,10 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n0 = c.n * g.BN;
 
             if (EPI == kEpiSwiglu || EPI == kEpiStore) {
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-                    epilogue_rows<EPI>(g, t_row + static_cast<uint32_t>(mt * g.mma_n), c.row0 + mt * kBM + quarter * 32,
-                                       c.row_end, n0, lane, epi_stage + (warp - 2) * kStageWords);
+                epilogue_rows<EPI>(g, t_row, c.row0 + quarter * 32, c.row_end, n0, lane,
+                                   epi_stage + (warp - 2) * kStageWords);
             } else {
                 // router: top-k over the E logits of this row, softmax over the selected ones
                 float tv[kMaxTopK];
@@ -558,23 +545,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-size_t gemm_smem_bytes(int stages, int mma_n, int mt) {
-    return 1024 + static_cast<size_t>(stages) * (mt * kABytes + static_cast<size_t>(mma_n) * 128u) +
+size_t gemm_smem_bytes(int stages, int mma_n) {
+    return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(mma_n) * 128u) +
            4 * kStageWords * sizeof(uint32_t);
 }
 
-int gemm_pick_stages(int mma_n, int mt) {
-    const size_t per = mt * kABytes + static_cast<size_t>(mma_n) * 128u;
+int gemm_pick_stages(int mma_n) {
+    const size_t per = kABytes + static_cast<size_t>(mma_n) * 128u;
     int s = static_cast<int>((kGemmSmemBudget - 1024) / per);
     if (s > kMaxStages) s = kMaxStages;
     return s;
 }
 
-template <int EPI, int MT>
+template <int EPI>
 static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmArgs& g,
                               int grid, cudaStream_t stream) {
-    auto kern = umma_gemm_kernel<EPI, MT>;
-    size_t smem = gemm_smem_bytes(g.stages, g.mma_n, MT);
+    auto kern = umma_gemm_kernel<EPI>;
+    size_t smem = gemm_smem_bytes(g.stages, g.mma_n);
     if (smem < kGemmSmemMin) smem = kGemmSmemMin;  // keeps one CTA per SM (all TMEM columns are taken)
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
@@ -627,13 +614,11 @@ cudaError_t launch_umma_gemm_pair(int epi, const CUtensorMap& a, const CUtensorM
 }
 
 cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                             const GemmArgs& g, int grid, cudaStream_t stream, int mt) {
+                             const GemmArgs& g, int grid, cudaStream_t stream) {
     switch (epi) {
-        case kEpiRoute: return launch_one<kEpiRoute, 1>(a, b0, b1, g, grid, stream);
-        case kEpiSwiglu:
-            return mt == 2 ? launch_one<kEpiSwiglu, 2>(a, b0, b1, g, grid, stream)
-                           : launch_one<kEpiSwiglu, 1>(a, b0, b1, g, grid, stream);
-        default: return launch_one<kEpiStore, 1>(a, b0, b1, g, grid, stream);
+        case kEpiRoute: return launch_one<kEpiRoute>(a, b0, b1, g, grid, stream);
+        case kEpiSwiglu: return launch_one<kEpiSwiglu>(a, b0, b1, g, grid, stream);
+        default: return launch_one<kEpiStore>(a, b0, b1, g, grid, stream);
     }
 }
 
