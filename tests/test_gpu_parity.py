@@ -323,3 +323,35 @@ def test_shared_expert_overlapped_on_a_second_stream():
     torch.cuda.current_stream().wait_event(done)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+
+
+def test_layer_fwd_captured_in_a_cuda_graph():
+    """The whole layer allocates nothing and never synchronises, so it can be captured into a
+    CUDA graph and replayed; replays read the same device buffers and match eager calls."""
+    w = SMALL[1]  # ragged
+    case = make_case(w, seed=14)
+    s = moe_shape(w)
+    _, layer_bytes = moe.moe_workspace_size(s)
+    ws = torch.empty(layer_bytes, dtype=torch.uint8, device="cuda")
+    x, w_r, bias = dev(case.x), dev(case.w_r), dev(case.bias)
+    wg, wu, wd = dev(case.wg), dev(case.wu), dev(case.wd)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    eager = torch.empty(w.T, w.d, dtype=torch.float32, device="cuda")
+    moe.moe_layer_fwd(s, x, w_r, bias, wg, wu, wd, eager, status, ws)   # warm-up outside capture
+    torch.cuda.synchronize()
+
+    graphed = torch.zeros_like(eager)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.moe_layer_fwd(s, x, w_r, bias, wg, wu, wd, graphed, status, ws)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(graphed, eager)
+
+    # new input values in the same buffer: the replay follows them
+    x.copy_(dev(syn.router_inputs(w, 99)[0]))
+    g.replay()
+    moe.moe_layer_fwd(s, x, w_r, bias, wg, wu, wd, eager, status, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(graphed, eager)
+    assert status.item() == 0

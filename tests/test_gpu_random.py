@@ -1,0 +1,69 @@
+"""Randomised GPU-vs-oracle checks over many small shapes and seeds (the property
+tests of the parity plan): every combination of capacity / balanced plan / bias /
+routing variant, ragged T, d and F, E from 1 to 64 and k from 1 to min(E, 8).
+Each case runs the whole layer through moe_layer_fwd and compares every output."""
+import numpy as np
+import pytest
+
+import oracle
+import mixture_experts_routing_02_b200 as moe
+from mixture_experts_routing_02_b200 import synthetic as syn
+
+from gpu_cases import check_bf16_storage, check_close, check_layer_output, make_case, run_layer, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _random_workload(seed):
+    rng = np.random.default_rng(1000 + seed)
+    E = int(rng.choice([1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 64]))
+    k = int(rng.integers(1, min(E, 8) + 1))
+    mode = rng.choice(["plain", "capacity", "plan"]) if E > 1 else "plain"
+    R = 0
+    if mode == "plan":
+        divisors = [r for r in (2, 3, 4, 8) if E % r == 0]
+        if not divisors:
+            mode = "plain"
+        else:
+            R = int(rng.choice(divisors))
+    S = int(rng.integers(8, 120))
+    T = R * S if R else int(rng.integers(1, 700))
+    d = 64 * int(rng.integers(1, 6))
+    F = 64 * int(rng.integers(1, 7))
+    return syn.Workload(f"random-{seed}", T=T, d=d, E=E, k=k, F=F,
+                        zipf_s=float(rng.choice([0.0, 0.8, 1.5])),
+                        capacity_factor=float(rng.uniform(0.3, 1.5)) if mode == "capacity" else 0.0,
+                        n_groups=R, replica_slots=int(rng.integers(1, 6)) if R else 0), int(rng.integers(0, 2))
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_random_layer_matches_oracle(cuda_ok, seed):
+    w, flags = _random_workload(seed)
+    case = make_case(w, seed=seed)
+    C = oracle.capacity_rows(w.capacity_factor, w.T, w.k, w.E)
+    try:
+        ref = oracle.layer_forward(case.x, case.w_r, case.bias, case.wg, case.wu, case.wd, w.k, capacity=C,
+                                   n_groups=w.n_groups, replica_slots=w.replica_slots, softmax_all=bool(flags))
+        feasible = True
+    except oracle.PlanInfeasible:
+        feasible = False
+    got = run_layer(case, route_flags=flags)
+    if not feasible:
+        # more replica pieces than slots: reported, nothing dispatched, zero output
+        assert got["status"] & moe.DEV_ERR_PLAN
+        assert (got["dest"].numpy() == -1).all() and (to_np(got["out"]) == 0).all()
+        return
+    assert got["status"] == 0
+    assert (got["ids"].numpy() == ref.ids).all()
+    assert np.abs(got["w"].numpy() - ref.weights).max() < 1e-4
+    assert (got["counts"].numpy() == ref.counts).all()
+    assert (got["seg_offsets"].numpy() == ref.segs.offsets).all()
+    assert (got["seg_expert"].numpy() == ref.segs.expert).all()
+    assert (got["dest"].numpy() == ref.dest).all()
+    used = int(ref.segs.offsets[-1])
+    assert (got["src"].numpy()[:used] == ref.src).all()
+    assert (to_np(got["xp"][:used]) == ref.xp).all()
+    check_bf16_storage(to_np(got["hp"][:used]), ref.hp, "Hp")
+    if used:
+        check_close(to_np(got["yp"][:used]), ref.yp, "Yp")
+    check_layer_output(to_np(got["out"]), ref.out, ref.dest, w.T, w.k)
