@@ -9,5 +9,5 @@ from .moe_oracle import (  # noqa: F401
     dispatch_positions, enforce_margin, expert_ffn, expert_rank, f64, grouped_expert_ffn,
     histogram, i64, layer_forward, margin_violations, num_segments, permute_rows,
     plain_segments, route, router_logits, shared_expert, silu, token_output, topk_ids, topk_weights,
-    topk_weights_softmax_all,
+    topk_weights_softmax_all, ExpertChoice, expert_choice, expert_choice_forward, expert_scores,
 )

@@ -500,3 +500,56 @@ def enforce_margin(x, w_router, bias, k: int, redraw, min_gap: float = 1e-3,
         else:
             raise RuntimeError(f"could not satisfy the top-k margin for token {t}")
     return len(bad)
+
+
+# ----------------------------------------------------------------------------
+# expert-choice routing   [Token-skew] "라우팅 분포와 학습 안정성": instead of tokens
+# choosing experts, experts choose tokens
+# ----------------------------------------------------------------------------
+
+def expert_scores(logits64: np.ndarray) -> np.ndarray:
+    """S[t, e]: softmax of token t's logits over the E experts (fp64)."""
+    l = np.asarray(logits64, dtype=np.float64)
+    e = np.exp(l - l.max(axis=1, keepdims=True))
+    return e / e.sum(axis=1, keepdims=True)
+
+
+@dataclasses.dataclass
+class ExpertChoice:
+    scores: np.ndarray     # [T, E] fp64
+    picks: List[np.ndarray]  # per expert: picked tokens, ascending id
+    segs: Segments         # E segments of min(C, T) rows, expert order
+    src: np.ndarray        # [rows] token of each dispatched row
+    row_w: np.ndarray      # [rows] score S[t, e] of each row
+
+
+def expert_choice(logits64: np.ndarray, capacity: int) -> ExpertChoice:
+    """Each expert e takes the C tokens with the largest S[t, e] (compared in fp32, the
+    kernels' precision; equal scores go to the lower token id); its segment lists them in
+    ascending token order."""
+    S = expert_scores(logits64)
+    T, E = S.shape
+    C = min(capacity, T)
+    s32 = S.astype(np.float32)
+    picks = []
+    for e in range(E):
+        order = np.argsort(-s32[:, e], kind="stable")[:C]
+        picks.append(np.sort(order).astype(np.int64))
+    length = np.full(E, C, dtype=np.int64)
+    segs = Segments(expert=np.arange(E, dtype=np.int64), length=length, first_rank=np.zeros(E, dtype=np.int64))
+    src = np.concatenate(picks) if E else np.zeros(0, dtype=np.int64)
+    row_w = np.concatenate([S[picks[e], e] for e in range(E)]) if E else np.zeros(0)
+    return ExpertChoice(S, picks, segs, src, row_w)
+
+
+def expert_choice_forward(x, w_router, bias, w_gate, w_up, w_down, capacity: int):
+    """out[t] = sum over the experts e that picked t of S[t, e] * FFN_e(x_t)."""
+    logits = router_logits(x, w_router, bias)
+    ec = expert_choice(logits, capacity)
+    xp = f64(x)[ec.src]
+    hp, yp = grouped_expert_ffn(xp, ec.segs, w_gate, w_up, w_down)
+    T, d = f64(x).shape[0], w_down.shape[1]
+    out = np.zeros((T, d))
+    for r in range(len(ec.src)):
+        out[ec.src[r]] += ec.row_w[r] * yp[r]
+    return logits, ec, xp, hp, yp, out

@@ -168,6 +168,39 @@ def pin_shared_expert_additive(seed=8):
     return bool(np.allclose(both - routed, dense, rtol=1e-10, atol=1e-13))
 
 
+def pin_expert_choice_brute_force(seed=20, T=7, E=3, C=3):
+    """Each expert's picks are the C-subset of tokens with the largest summed scores (brute force),
+    listed in ascending id; scores are the library softmax over experts."""
+    rng = np.random.default_rng(seed)
+    logits = rng.normal(size=(T, E))
+    ec = oracle.expert_choice(logits, C)
+    S = torch.softmax(torch.from_numpy(logits), dim=1).numpy()
+    ok = np.allclose(ec.scores, S, rtol=1e-12, atol=1e-15)
+    for e in range(E):
+        s32 = S[:, e].astype(np.float32).astype(np.float64)
+        best = max(itertools.combinations(range(T), C), key=lambda sub: sum(s32[list(sub)]))
+        ok &= list(ec.picks[e]) == sorted(best)
+    ok &= (ec.segs.offsets == np.arange(E + 1) * C).all()
+    return bool(ok)
+
+
+def pin_expert_choice_layer_eager(seed=21):
+    """The expert-choice layer equals a per-expert loop over its picked tokens."""
+    T, E, C = 30, 4, 9
+    x, wr, b, wg, wu, wd = _small_layer(seed, T=T, E=E, k=1)
+    logits, ec, xp, hp, yp, out = oracle.expert_choice_forward(x, wr, b, wg, wu, wd, C)
+    x64 = oracle.f64(x)
+    S = oracle.expert_scores(oracle.router_logits(x, wr, b))
+    want = np.zeros_like(out)
+    for e in range(E):
+        s32 = S[:, e].astype(np.float32)
+        chosen = sorted(range(T), key=lambda t: (-s32[t], t))[:C]
+        for t in chosen:
+            _, y = oracle.expert_ffn(x64[t][None, :], wg[e], wu[e], wd[e])
+            want[t] += S[t, e] * y[0]
+    return bool(np.allclose(out, want, rtol=1e-11, atol=1e-13))
+
+
 def pin_silu_library():
     z = np.linspace(-30, 30, 2001)
     ref = torch.nn.functional.silu(torch.from_numpy(z)).numpy()
@@ -327,6 +360,20 @@ def test_silu():
     assert pin_silu_library()
 
 
+def test_expert_choice_brute_force():
+    assert pin_expert_choice_brute_force()
+
+
+def test_expert_choice_layer_equals_loop():
+    assert pin_expert_choice_layer_eager()
+
+
+def test_expert_choice_capacity_above_tokens():
+    logits = np.random.default_rng(3).normal(size=(5, 3))
+    ec = oracle.expert_choice(logits, 99)
+    assert all(list(p) == [0, 1, 2, 3, 4] for p in ec.picks)
+
+
 def test_shared_expert_adds_a_dense_ffn():
     assert pin_shared_expert_additive()
 
@@ -431,6 +478,13 @@ def _mut_shared_transposed(x, w_gate_s, w_up_s, w_down_s):
     return om.expert_ffn(om.f64(x), w_up_s, w_gate_s, w_down_s)[1]   # gate and up swapped
 
 
+_orig_expert_choice = om.expert_choice
+
+
+def _mut_ec_keeps_weakest(logits64, capacity):
+    return _orig_expert_choice(-np.asarray(logits64, dtype=np.float64), capacity)   # picks the lowest scores
+
+
 MUTATIONS = [
     ("silu", _mut_silu_sign, [pin_silu_library, pin_dense_ffn_e1k1]),
     ("topk_weights", _mut_weights_no_renorm, [pin_worked_example, pin_weights_full_softmax]),
@@ -442,6 +496,9 @@ MUTATIONS = [
     ("combine", _mut_combine_unweighted, [pin_layer_equals_eager]),
     ("shared_expert", _mut_shared_transposed, [pin_shared_expert_additive]),
     ("topk_weights_softmax_all", lambda l, i: _orig_weights(l, i), [pin_weights_softmax_all]),
+    ("expert_scores", lambda l: np.exp(l) / np.exp(l).sum(0, keepdims=True),   # softmax over tokens
+     [pin_expert_choice_brute_force, pin_expert_choice_layer_eager]),
+    ("expert_choice", _mut_ec_keeps_weakest, [pin_expert_choice_brute_force, pin_expert_choice_layer_eager]),
 ]
 
 
