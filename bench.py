@@ -37,6 +37,7 @@ METRIC = "MoE layer fwd tokens/s; grouped-GEMM TFLOPS and permute GB/s vs roofli
 FLUSH_BYTES = 256 << 20
 KERNELS = ("route", "dispatch", "gate_up", "down", "combine")
 LAUNCHES_PER_STEP = 7  # route, histogram, segments|plan, permute, gate_up, down, combine
+LAUNCHES_PER_STEP_EC = 6  # expert choice: route scores, select, gather, gate_up, down, combine
 
 
 def _peaks():
@@ -163,7 +164,8 @@ def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: fl
 def _config(w, capacity):
     return {"workload": w.name, "T": w.T, "d_model": w.d, "n_experts": w.E, "top_k": w.k, "d_ff": w.F,
             "capacity": capacity, "n_groups": w.n_groups, "replica_slots": w.replica_slots,
-            "zipf_bias_s": w.zipf_s, "l2": "flushed between steps (256 MiB write outside the timed events)",
+            "zipf_bias_s": w.zipf_s, "routing": "expert-choice" if w.expert_choice else "top-k",
+            "l2": "flushed between steps (256 MiB write outside the timed events)",
             "parallelism": "replicas (no exchange between GPUs)"}
 
 
@@ -177,6 +179,8 @@ def _oracle_sample(w, seed: int, n_route: int, n_ffn: int, wg, wu, wd):
     from mixture_experts_routing_02_b200 import synthetic as syn
 
     x, w_r, bias = syn.router_inputs(w.scaled(T=n_route), seed)
+    if w.expert_choice:
+        return _oracle_sample_ec(w, x, w_r, bias, n_route, n_ffn, wg, wu, wd)
     t0 = time.perf_counter()
     logits, ids, wts = oracle.route(x, w_r, bias, w.k)
     t1 = time.perf_counter()
@@ -196,6 +200,31 @@ def _oracle_sample(w, seed: int, n_route: int, n_ffn: int, wg, wu, wd):
             f"(gate/up/down, fp64) of {n_ffn} rows of one expert; per-token cost = per-token routing+dispatch"
             f"+combine + k x per-row FFN, extrapolated to tokens/s")
     return 1.0 / per_token, desc, t4 - t0
+
+
+def _oracle_sample_ec(w, x, w_r, bias, n_route: int, n_ffn: int, wg, wu, wd):
+    """The expert-choice layer's oracle on a sample: scores and selection of n_route tokens
+    (C scaled to them), the FFN of n_ffn rows of one expert, the combine."""
+    import numpy as np
+    import oracle
+
+    C = _capacity(w.scaled(T=n_route))
+    t0 = time.perf_counter()
+    ec = oracle.expert_choice(oracle.router_logits(x, w_r, bias), C)
+    xp = oracle.f64(x)[ec.src]
+    t1 = time.perf_counter()
+    _, y = oracle.expert_ffn(xp[:n_ffn], wg[0], wu[0], wd[0])
+    t2 = time.perf_counter()
+    yfull = np.zeros((xp.shape[0], w.d))
+    yfull[:n_ffn] = y
+    oracle.combine_expert_choice(yfull, ec.src, ec.row_w, n_route)
+    t3 = time.perf_counter()
+    rows_per_token = len(ec.src) / n_route
+    per_token = (t1 - t0) / n_route + rows_per_token * (t2 - t1) / n_ffn + (t3 - t2) / n_route
+    desc = (f"expert-choice scores, selection and dispatch of {n_route} tokens (C={C}) and combine; expert FFN "
+            f"(gate/up/down, fp64) of {n_ffn} rows of one expert; per-token cost = per-token routing+dispatch"
+            f"+combine + (rows per token = {rows_per_token:g}) x per-row FFN, extrapolated to tokens/s")
+    return 1.0 / per_token, desc, t3 - t0
 
 
 def _threads_used():
@@ -263,8 +292,9 @@ def run_ours(args, w):
     stream = torch.cuda.current_stream()
 
     capacity = _capacity(w)
+    ec = w.expert_choice
     s = moe.shape(w.T, w.d, w.E, w.k, w.F, capacity=capacity, n_groups=w.n_groups,
-                  replica_slots=w.replica_slots)
+                  replica_slots=w.replica_slots, route_flags=moe.ROUTE_EXPERT_CHOICE if ec else 0)
     n_seg, rows_alloc = moe.moe_layout(s)
     _, layer_bytes = moe.moe_workspace_size(s)
 
@@ -299,6 +329,10 @@ def run_ours(args, w):
     hp = view(v.hp, rows_alloc * w.F, torch.bfloat16)
     yp = view(v.yp, rows_alloc * w.d, torch.float32)
     dws = view(v.dispatch_ws, v.dispatch_ws_bytes, torch.uint8)
+    if ec:
+        scores = view(v.scores, w.E * w.T, torch.float32)
+        emap = view(v.emap, w.T * w.E, torch.int32)
+        row_w = view(v.row_w, rows_alloc, torch.float32)
 
     Fs = args.shared_expert
     if Fs:
@@ -319,9 +353,14 @@ def run_ours(args, w):
             moe.moe_shared_expert(s, Fs, x, gs, us, dsw, h_s, y_s, status, side)
             se1.record(side)
             shared_ms.append((se0, se1))
-        moe.moe_route(s, x, w_r, bias, None, ids, wts, status, stream)
-        ev[1].record(stream)
-        moe.moe_dispatch(s, x, ids, 0, counts, seg_e, seg_o, seg_f, dest, src, xp, status, dws, stream)
+        if ec:
+            moe.moe_route_scores(s, x, w_r, bias, scores, status, stream)
+            ev[1].record(stream)
+            moe.moe_expert_choose(s, scores, x, seg_e, seg_o, src, row_w, emap, xp, stream)
+        else:
+            moe.moe_route(s, x, w_r, bias, None, ids, wts, status, stream)
+            ev[1].record(stream)
+            moe.moe_dispatch(s, x, ids, 0, counts, seg_e, seg_o, seg_f, dest, src, xp, status, dws, stream)
         ev[2].record(stream)
         moe.moe_expert_gate_up(s, xp, seg_e, seg_o, wg, wu, hp, status, stream)
         ev[3].record(stream)
@@ -329,6 +368,9 @@ def run_ours(args, w):
         ev[4].record(stream)
         if Fs:
             stream.wait_event(shared_ms[-1][1])
+        if ec:
+            moe.moe_combine_expert_choice(s, yp, emap, row_w, y_s if Fs else None, out, stream)
+        elif Fs:
             moe.moe_combine_add(s, yp, dest, wts, y_s, out, stream)
         else:
             moe.moe_combine(s, yp, dest, wts, out, stream)
@@ -423,13 +465,23 @@ def run_ours(args, w):
     avg = {k: statistics.mean(v) for k, v in per_kernel.items()}
     T, d, E, k, F = w.T, w.d, w.E, w.k, w.F
     breakdown = {}
-    breakdown["route"] = dict(ms=avg["route"], bytes=T * d * 2 + E * d * 2 + T * k * 8, flops=2 * T * d * E)
-    breakdown["dispatch"] = dict(ms=avg["dispatch"], bytes=T * d * 2 + rows_used * d * 2 + T * k * 4 * 3 + rows_used * 4)
+    if ec:
+        # scores [E, T] fp32 written by the route epilogue, read by the selection; the [T, E] row map
+        breakdown["route"] = dict(ms=avg["route"], bytes=T * d * 2 + E * d * 2 + E * T * 4, flops=2 * T * d * E)
+        breakdown["dispatch"] = dict(ms=avg["dispatch"],
+                                     bytes=E * T * 4 + T * E * 4 + rows_used * 8 + 2 * rows_used * d * 2)
+    else:
+        breakdown["route"] = dict(ms=avg["route"], bytes=T * d * 2 + E * d * 2 + T * k * 8, flops=2 * T * d * E)
+        breakdown["dispatch"] = dict(ms=avg["dispatch"],
+                                     bytes=T * d * 2 + rows_used * d * 2 + T * k * 4 * 3 + rows_used * 4)
     breakdown["gate_up"] = dict(ms=avg["gate_up"], flops=4 * rows_used * d * F,
                                 bytes=2 * active_experts * F * d * 2 + rows_used * d * 2 + rows_used * F * 2)
     breakdown["down"] = dict(ms=avg["down"], flops=2 * rows_used * d * F,
                              bytes=active_experts * d * F * 2 + rows_used * F * 2 + rows_used * d * 4)
-    breakdown["combine"] = dict(ms=avg["combine"], bytes=rows_used * d * 4 + T * d * 4 + T * k * 8)
+    if ec:
+        breakdown["combine"] = dict(ms=avg["combine"], bytes=rows_used * d * 4 + T * d * 4 + T * E * 4 + rows_used * 4)
+    else:
+        breakdown["combine"] = dict(ms=avg["combine"], bytes=rows_used * d * 4 + T * d * 4 + T * k * 8)
     for name, b in breakdown.items():
         sec = b["ms"] / 1e3
         if "flops" in b and name in ("gate_up", "down"):
@@ -455,7 +507,7 @@ def run_ours(args, w):
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init weights)", "config": _config(w, capacity),
-        "rows_dispatched": rows_used, "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "rows_dispatched": rows_used, "gpu_launches": (LAUNCHES_PER_STEP_EC if ec else LAUNCHES_PER_STEP) * args.steps,
         "roofline": roof,
         "breakdown": {n: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in b.items()}
                       for n, b in breakdown.items()},
@@ -466,7 +518,7 @@ def run_ours(args, w):
     if shared_info:
         line["shared_expert"] = shared_info
         line["config"]["shared_expert_d_ff"] = Fs
-        line["gpu_launches"] = (LAUNCHES_PER_STEP + 2) * args.steps
+        line["gpu_launches"] = ((LAUNCHES_PER_STEP_EC if ec else LAUNCHES_PER_STEP) + 2) * args.steps
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         wg0, wu0, wd0 = wg[:1].cpu(), wu[:1].cpu(), wd[:1].cpu()
         cv, desc, _ = _oracle_sample(w, seed, 512, 32, wg0, wu0, wd0)

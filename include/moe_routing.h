@@ -99,8 +99,24 @@ typedef enum {
  *                  살펴보기", section "Top-2 라우팅의 수치 예시": whether the
  *                  softmax comes before or after the top-k differs between
  *                  implementations; with renormalisation both orders agree.
+ *                  MOE_ROUTE_EXPERT_CHOICE: experts choose tokens instead of
+ *                  tokens choosing experts ("Expert를 똑같이 나눴는데도 GPU가
+ *                  대기하는 이유: MoE의 토큰 쏠림", section "라우팅 분포와 학습
+ *                  안정성").  Scores S[t, e] = softmax over the E logits of
+ *                  token t; expert e keeps the C tokens with the largest
+ *                  S[t, e] (equal scores: the lower token id), laid out in
+ *                  ascending token order in segment e, which holds
+ *                  C' = min(C, T) rows; token t's output is the sum of
+ *                  S[t, e] * FFN_e(x_t) over the experts that kept it (0 if
+ *                  none did).  Requires capacity >= 1 (the C above) and
+ *                  n_groups == 0; excludes MOE_ROUTE_SOFTMAX_ALL; top_k is
+ *                  not used by the selection (only validated).  n_seg = E,
+ *                  rows_alloc = E * C'.  Takes moe_route_scores,
+ *                  moe_expert_choose and moe_combine_expert_choice in place of
+ *                  moe_route, moe_dispatch and moe_combine, which reject it.
  */
 #define MOE_ROUTE_SOFTMAX_ALL 0x1
+#define MOE_ROUTE_EXPERT_CHOICE 0x2
 
 typedef struct {
     int32_t T;
@@ -332,6 +348,9 @@ MOE_API moe_status_t moe_shared_expert(const moe_shape_t *shape, int32_t d_ff_sh
 /*
  * The whole layer: moe_route (logits not stored) -> moe_dispatch ->
  * moe_expert_gate_up -> moe_expert_down -> moe_combine, all on `stream`.
+ * With MOE_ROUTE_EXPERT_CHOICE: moe_route_scores -> moe_expert_choose ->
+ * moe_expert_gate_up -> moe_expert_down -> moe_combine_expert_choice; the
+ * views topk_ids, topk_w, dest, seg_first_rank and dispatch_ws are then unused.
  * out [T, d] fp32.  The intermediates live in `ws` (moe_workspace_size()'s
  * layer_bytes); their addresses are given by moe_layer_views.
  */
@@ -357,6 +376,50 @@ MOE_API moe_status_t moe_testing_dispatch_stalled(const moe_shape_t *shape, cons
                                           moe_bf16_t *xp, int32_t *status, void *ws, size_t ws_bytes,
                                           moe_stream_t stream);
 
+/*
+ * Expert-choice routing (shape.route_flags = MOE_ROUTE_EXPERT_CHOICE; see
+ * moe_shape_t).  Router scores, transposed so that each expert's column is
+ * contiguous:
+ *   x        [T, d] bf16            w_router [E, d] bf16
+ *   bias     [E] fp32 or NULL; added to the logits
+ *   scores   [E, T] fp32 out: scores[e * T + t] = exp(l_te - max_e' l_te') /
+ *            sum_e' exp(l_te' - max_e' l_te')
+ * The projection runs on the tensor cores (bf16 in, fp32 accumulate) with
+ * the softmax in its epilogue.  Rejects shapes without the flag.
+ */
+MOE_API moe_status_t moe_route_scores(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *w_router,
+                              const float *bias, float *scores, int32_t *status, moe_stream_t stream);
+
+/*
+ * Expert-choice selection and dispatch: each expert keeps its C' = min(C, T)
+ * highest-scoring tokens (compared as fp32; equal scores go to the lower
+ * token id), and their rows of X are copied into segment e of Xp in
+ * ascending token order.
+ *   scores      [E, T] fp32 (moe_route_scores)
+ *   x           [T, d] bf16
+ *   seg_expert  [E] int32 out: e;  seg_offsets [E + 1] int32 out: e * C'
+ *   src         [E * C'] int32 out: token of each row
+ *   row_w       [E * C'] fp32 out: the score S[src, e] of each row
+ *   emap        [T, E] int32 out: row of (t, e), or -1 if e did not keep t
+ *   xp          [E * C', d] bf16 out
+ * Scores must be finite.  Two launches (selection: one CTA per expert;
+ * row copy).  Rejects shapes without the flag.
+ */
+MOE_API moe_status_t moe_expert_choose(const moe_shape_t *shape, const float *scores, const moe_bf16_t *x,
+                               int32_t *seg_expert, int32_t *seg_offsets, int32_t *src, float *row_w,
+                               int32_t *emap, moe_bf16_t *xp, moe_stream_t stream);
+
+/*
+ * Expert-choice combine: out[t] = base[t] + sum over e ascending with
+ * emap[t, e] >= 0 of row_w[r] * yp[r], r = emap[t, e], accumulated in fp32.
+ *   yp [E * C', d] fp32;  emap [T, E] int32;  row_w [E * C'] fp32
+ *   base [T, d] fp32 or NULL;  out [T, d] fp32 (may alias base)
+ * Rows outside [0, E * C') contribute nothing.  Rejects shapes without the flag.
+ */
+MOE_API moe_status_t moe_combine_expert_choice(const moe_shape_t *shape, const float *yp, const int32_t *emap,
+                                       const float *row_w, const float *base, float *out,
+                                       moe_stream_t stream);
+
 /* Device addresses of the intermediates moe_layer_fwd keeps in its workspace. */
 typedef struct {
     int32_t *topk_ids;       /* [T, k] */
@@ -372,6 +435,9 @@ typedef struct {
     float *yp;               /* [rows_alloc, d] fp32 */
     void *dispatch_ws;       /* moe_dispatch's own workspace */
     size_t dispatch_ws_bytes;
+    float *scores;           /* [E, T] expert-choice scores (NULL without the flag) */
+    int32_t *emap;           /* [T, E] expert-choice row map (NULL without the flag) */
+    float *row_w;            /* [rows_alloc] expert-choice row weights (NULL without the flag) */
 } moe_layer_views_t;
 
 /* Fill *views with the addresses inside a layer workspace `ws`. Host only. */

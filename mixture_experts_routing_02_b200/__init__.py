@@ -18,8 +18,9 @@ __all__ = [
     "moe_status_string", "moe_layout", "moe_workspace_size", "moe_route", "moe_route_from_logits",
     "moe_histogram", "moe_segments", "moe_plan_balanced", "moe_dispatch", "moe_dispatch_static", "moe_expert_gate_up",
     "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_combine_add", "moe_shared_expert", "moe_layer_fwd",
+    "moe_route_scores", "moe_expert_choose", "moe_combine_expert_choice",
     "moe_layer_views",
-    "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT", "ROUTE_SOFTMAX_ALL",
+    "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT", "ROUTE_SOFTMAX_ALL", "ROUTE_EXPERT_CHOICE",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -41,7 +42,8 @@ class MoeShape(ctypes.Structure):
 class MoeLayerViews(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("topk_ids", "topk_w", "counts", "seg_expert", "seg_offsets", "seg_first_rank", "dest",
-                 "src", "xp", "hp", "yp", "dispatch_ws")] + [("dispatch_ws_bytes", ctypes.c_size_t)]
+                 "src", "xp", "hp", "yp", "dispatch_ws")] + [("dispatch_ws_bytes", ctypes.c_size_t)] + \
+        [(n, ctypes.c_void_p) for n in ("scores", "emap", "row_w")]
 
 
 _P = ctypes.c_void_p
@@ -69,6 +71,9 @@ SYMBOLS = {
     "moe_shared_expert": [_S, _I, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_layer_fwd": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_layer_views": [_S, _P, ctypes.POINTER(MoeLayerViews)],
+    "moe_route_scores": [_S, _P, _P, _P, _P, _P, _P],
+    "moe_expert_choose": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "moe_combine_expert_choice": [_S, _P, _P, _P, _P, _P, _P],
 }
 
 _lib = None
@@ -92,6 +97,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 
 ROUTE_SOFTMAX_ALL = 0x1
+ROUTE_EXPERT_CHOICE = 0x2
 
 
 def shape(T, d_model, n_experts, top_k, d_ff, capacity=0, n_groups=0, replica_slots=0, route_flags=0) -> MoeShape:
@@ -231,3 +237,19 @@ def moe_layer_views(s, ws) -> MoeLayerViews:
     v = MoeLayerViews()
     _check("moe_layer_views", load_library().moe_layer_views(ctypes.byref(s), _ptr(ws), ctypes.byref(v)))
     return v
+
+
+def moe_route_scores(s, x, w_router, bias, scores, status=None, stream=None):
+    _check("moe_route_scores", load_library().moe_route_scores(
+        ctypes.byref(s), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(scores), _ptr(status), _stream(stream)))
+
+
+def moe_expert_choose(s, scores, x, seg_expert, seg_offsets, src, row_w, emap, xp, stream=None):
+    _check("moe_expert_choose", load_library().moe_expert_choose(
+        ctypes.byref(s), _ptr(scores), _ptr(x), _ptr(seg_expert), _ptr(seg_offsets), _ptr(src), _ptr(row_w),
+        _ptr(emap), _ptr(xp), _stream(stream)))
+
+
+def moe_combine_expert_choice(s, yp, emap, row_w, base, out, stream=None):
+    _check("moe_combine_expert_choice", load_library().moe_combine_expert_choice(
+        ctypes.byref(s), _ptr(yp), _ptr(emap), _ptr(row_w), _ptr(base), _ptr(out), _stream(stream)))

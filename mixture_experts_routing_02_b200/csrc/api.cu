@@ -47,6 +47,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Dims {
     int T, d, E, k, F, C, R, B, S, flags;
+    bool ec() const { return (flags & MOE_ROUTE_EXPERT_CHOICE) != 0; }
+    int cp() const { return ec() ? std::min(C, T) : 0; }  // expert choice: rows per expert
     int n_seg;
     int rows;  // rows_alloc
 };
@@ -56,7 +58,9 @@ moe_status_t check_shape(const moe_shape_t* s, Dims* out) {
     Dims v;
     v.T = s->T; v.d = s->d_model; v.E = s->n_experts; v.k = s->top_k; v.F = s->d_ff;
     v.C = s->capacity; v.R = s->n_groups; v.B = s->replica_slots; v.flags = s->route_flags;
-    if (v.flags & ~MOE_ROUTE_SOFTMAX_ALL) return MOE_ERR_INVALID_ARG;
+    if (v.flags & ~(MOE_ROUTE_SOFTMAX_ALL | MOE_ROUTE_EXPERT_CHOICE)) return MOE_ERR_INVALID_ARG;
+    const bool ec = (v.flags & MOE_ROUTE_EXPERT_CHOICE) != 0;
+    if (ec && ((v.flags & MOE_ROUTE_SOFTMAX_ALL) || s->capacity < 1 || s->n_groups != 0)) return MOE_ERR_INVALID_ARG;
     if (v.T < 0 || v.d < 1 || v.E < 1 || v.k < 1 || v.k > v.E || v.F < 1 || v.C < 0 || v.R < 0 || v.B < 0)
         return MOE_ERR_INVALID_ARG;
     if (v.R > 0 && (v.E % v.R != 0 || v.T % v.R != 0 || v.C > 0)) return MOE_ERR_INVALID_ARG;
@@ -68,6 +72,11 @@ moe_status_t check_shape(const moe_shape_t* s, Dims* out) {
     v.S = v.R > 0 ? v.T / v.R : v.T;
     int64_t rows = static_cast<int64_t>(v.T) * v.k;
     if (v.C > 0) rows = std::min<int64_t>(rows, static_cast<int64_t>(v.C) * v.E);
+    if (ec) {
+        // segment e holds expert e's C' = min(C, T) chosen tokens
+        rows = static_cast<int64_t>(std::min(v.C, v.T)) * v.E;
+        if (rows >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+    }
     v.rows = static_cast<int>(rows);
     if (out) *out = v;
     return MOE_OK;
@@ -133,6 +142,44 @@ moe_status_t route_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_
     g.route_flags = v.flags;
     const int grid = std::min(sm_count(), (v.T + 127) / 128);
     return cuda_status(launch_umma_gemm(kEpiRoute, ta, tb, tb, g, grid, st));
+}
+
+// Expert-choice scores: the router projection with the softmax over all E logits in the
+// epilogue, written expert-major ([E, T]).
+moe_status_t route_scores_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
+                               float* scores, int32_t* status, cudaStream_t st) {
+    if (!x || !w_router || !scores) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+    if (v.T == 0) return MOE_OK;
+    if (!have_encoder()) return MOE_ERR_CUDA;
+    const int epad = std::max(16, (v.E + 15) / 16 * 16);
+    CUtensorMap ta, tb;
+    if (!tmap_rows(&ta, x, v.T, v.d)) return MOE_ERR_CUDA;
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(v.d), static_cast<cuuint64_t>(v.E)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(v.d) * 2};
+        const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(v.E)};
+        if (!encode(&tb, w_router, 2, dims, strides, box)) return MOE_ERR_CUDA;
+    }
+    GemmArgs g{};
+    g.seg_offsets = nullptr; g.seg_expert = nullptr; g.n_seg = 1; g.M = v.T; g.K = v.d; g.N = v.E;
+    g.BN = epad; g.n_tiles_n = 1; g.mma_n = epad; g.stages = gemm_pick_stages(epad);
+    g.bias = bias; g.scores_t = scores; g.k = v.k; g.status = status;
+    const int grid = std::min(sm_count(), (v.T + 127) / 128);
+    return cuda_status(launch_umma_gemm(kEpiRoute, ta, tb, tb, g, grid, st));
+}
+
+moe_status_t choose_impl(const Dims& v, const float* scores, const moe_bf16_t* x, int32_t* seg_expert,
+                         int32_t* seg_offsets, int32_t* src, float* row_w, int32_t* emap, moe_bf16_t* xp,
+                         cudaStream_t st) {
+    if (!scores || !x || !seg_expert || !seg_offsets || !src || !row_w || !emap || !xp) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+    if (v.T == 0) return MOE_OK;
+    moe_status_t s = cuda_status(launch_ec_select(scores, v.T, v.E, v.cp(), seg_expert, seg_offsets, src, row_w,
+                                                  emap, st));
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_ec_gather(reinterpret_cast<const __nv_bfloat16*>(x), src, v.rows, v.T, v.d,
+                                        reinterpret_cast<__nv_bfloat16*>(xp), sm_count(), st));
 }
 
 moe_status_t gate_up_impl(const Dims& v, const moe_bf16_t* xp, const int32_t* seg_expert, const int32_t* seg_offsets,
@@ -254,14 +301,17 @@ void* static_scratch_address() {
 }
 
 struct LayerLayout {
-    size_t ids, w, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, dispatch_ws, xp, hp, yp, total;
+    size_t ids, w, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, dispatch_ws, xp, hp, yp, scores, emap,
+        row_w, total;
     size_t dispatch_ws_bytes;
 };
 
 LayerLayout layer_layout(const Dims& v) {
     LayerLayout L{};
     size_t o = 0;
-    const size_t tk = static_cast<size_t>(v.T) * v.k;
+    // expert choice keeps no per-pair arrays and no dispatch workspace
+    const size_t tk = v.ec() ? 0 : static_cast<size_t>(v.T) * v.k;
+    const size_t te = v.ec() ? static_cast<size_t>(v.T) * v.E : 0;
     L.ids = o; o = align256(o + tk * 4);
     L.w = o; o = align256(o + tk * 4);
     L.counts = o; o = align256(o + static_cast<size_t>(v.E) * 4);
@@ -270,11 +320,14 @@ LayerLayout layer_layout(const Dims& v) {
     L.seg_first_rank = o; o = align256(o + static_cast<size_t>(v.n_seg) * 4);
     L.dest = o; o = align256(o + tk * 4);
     L.src = o; o = align256(o + static_cast<size_t>(v.rows) * 4);
-    L.dispatch_ws_bytes = permute_ws_bytes(v.T, v.k, v.E);
+    L.dispatch_ws_bytes = v.ec() ? 0 : permute_ws_bytes(v.T, v.k, v.E);
     L.dispatch_ws = o; o = align256(o + L.dispatch_ws_bytes);
     L.xp = o; o = align256(o + static_cast<size_t>(v.rows) * v.d * 2);
     L.hp = o; o = align256(o + static_cast<size_t>(v.rows) * v.F * 2);
     L.yp = o; o = align256(o + static_cast<size_t>(v.rows) * v.d * 4);
+    L.scores = o; o = align256(o + te * 4);
+    L.emap = o; o = align256(o + te * 4);
+    L.row_w = o; o = align256(o + (v.ec() ? static_cast<size_t>(v.rows) * 4 : 0));
     L.total = o;
     return L;
 }
@@ -307,7 +360,7 @@ moe_status_t moe_workspace_size(const moe_shape_t* shape, size_t* dispatch_bytes
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
-    if (dispatch_bytes) *dispatch_bytes = permute_ws_bytes(v.T, v.k, v.E);
+    if (dispatch_bytes) *dispatch_bytes = v.ec() ? 0 : permute_ws_bytes(v.T, v.k, v.E);
     if (layer_bytes) *layer_bytes = layer_layout(v).total;
     return MOE_OK;
 }
@@ -317,6 +370,7 @@ moe_status_t moe_route(const moe_shape_t* shape, const moe_bf16_t* x, const moe_
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     return route_impl(v, x, w_router, bias, logits, topk_ids, topk_w, status, static_cast<cudaStream_t>(stream));
 }
 
@@ -325,6 +379,7 @@ moe_status_t moe_route_from_logits(const moe_shape_t* shape, const float* logits
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_route_from_logits(logits, v.T, v.E, v.k, v.flags, topk_ids, topk_w, sm_count(),
                                                 static_cast<cudaStream_t>(stream)));
@@ -334,6 +389,7 @@ moe_status_t moe_histogram(const moe_shape_t* shape, const int32_t* topk_ids, in
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     if (!topk_ids || !counts) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_histogram(topk_ids, v.T * v.k, v.E, counts, sm_count(), static_cast<cudaStream_t>(stream)));
 }
@@ -343,6 +399,7 @@ moe_status_t moe_segments(const moe_shape_t* shape, const int32_t* counts, int32
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     if (v.R > 0 || !counts || !seg_expert || !seg_offsets || !seg_first_rank) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_segments(const_cast<int32_t*>(counts), nullptr, 0, v.E, v.C, seg_expert, seg_offsets,
                                        seg_first_rank, static_cast<cudaStream_t>(stream)));
@@ -353,6 +410,7 @@ moe_status_t moe_plan_balanced(const moe_shape_t* shape, const int32_t* counts, 
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     if (v.R == 0 || !counts || !seg_expert || !seg_offsets || !seg_first_rank) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_plan(const_cast<int32_t*>(counts), nullptr, 0, v.E, v.R, v.S, v.k, v.B, seg_expert,
                                    seg_offsets, seg_first_rank, status, static_cast<cudaStream_t>(stream)));
@@ -365,6 +423,7 @@ moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const i
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     return dispatch_impl(v, x, topk_ids, plan_ready, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp,
                          status, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
@@ -376,6 +435,7 @@ moe_status_t moe_dispatch_static(const moe_shape_t* shape, const moe_bf16_t* x, 
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     if (permute_ws_bytes(v.T, v.k, v.E) > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED;
     void* scratch = static_scratch_address();
     if (scratch == nullptr) return MOE_ERR_CUDA;
@@ -419,6 +479,7 @@ moe_status_t moe_combine(const moe_shape_t* shape, const float* yp, const int32_
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(yp) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_combine(yp, dest, topk_w, nullptr, v.T, v.k, v.d, v.rows, out, sm_count(),
@@ -432,6 +493,7 @@ moe_status_t moe_testing_dispatch_stalled(const moe_shape_t* shape, const moe_bf
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     if (permute_n_tiles(v.T, v.k) < 2) return MOE_ERR_INVALID_ARG;  // needs a tile that waits on tile 0
     return dispatch_impl(v, x, topk_ids, 0, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp, status,
                          ws, ws_bytes, static_cast<cudaStream_t>(stream), 1);
@@ -442,6 +504,7 @@ moe_status_t moe_combine_add(const moe_shape_t* shape, const float* yp, const in
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(yp) || !aligned16(out) || (base && !aligned16(base))) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_combine(yp, dest, topk_w, base, v.T, v.k, v.d, v.rows, out, sm_count(),
@@ -494,6 +557,37 @@ moe_status_t moe_shared_expert(const moe_shape_t* shape, int32_t d_ff_shared, co
     }
 }
 
+moe_status_t moe_route_scores(const moe_shape_t* shape, const moe_bf16_t* x, const moe_bf16_t* w_router,
+                              const float* bias, float* scores, int32_t* status, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!v.ec()) return MOE_ERR_INVALID_ARG;
+    return route_scores_impl(v, x, w_router, bias, scores, status, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_choose(const moe_shape_t* shape, const float* scores, const moe_bf16_t* x,
+                               int32_t* seg_expert, int32_t* seg_offsets, int32_t* src, float* row_w, int32_t* emap,
+                               moe_bf16_t* xp, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!v.ec()) return MOE_ERR_INVALID_ARG;
+    return choose_impl(v, scores, x, seg_expert, seg_offsets, src, row_w, emap, xp, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_combine_expert_choice(const moe_shape_t* shape, const float* yp, const int32_t* emap,
+                                       const float* row_w, const float* base, float* out, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!v.ec()) return MOE_ERR_INVALID_ARG;
+    if (!yp || !emap || !row_w || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(yp) || !aligned16(out) || (base && !aligned16(base))) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_ec_combine(yp, emap, row_w, base, v.T, v.E, v.d, v.rows, out, sm_count(),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_layer_views(const moe_shape_t* shape, void* ws, moe_layer_views_t* views) {
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
@@ -514,6 +608,9 @@ moe_status_t moe_layer_views(const moe_shape_t* shape, void* ws, moe_layer_views
     views->yp = reinterpret_cast<float*>(b + L.yp);
     views->dispatch_ws = b + L.dispatch_ws;
     views->dispatch_ws_bytes = L.dispatch_ws_bytes;
+    views->scores = v.ec() ? reinterpret_cast<float*>(b + L.scores) : nullptr;
+    views->emap = v.ec() ? reinterpret_cast<int32_t*>(b + L.emap) : nullptr;
+    views->row_w = v.ec() ? reinterpret_cast<float*>(b + L.row_w) : nullptr;
     return MOE_OK;
 }
 
@@ -531,6 +628,18 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
     moe_layer_views_t w;
     moe_layer_views(shape, ws, &w);
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (v.ec()) {
+        s = route_scores_impl(v, x, w_router, bias, w.scores, status, st);
+        if (s != MOE_OK) return s;
+        s = choose_impl(v, w.scores, x, w.seg_expert, w.seg_offsets, w.src, w.row_w, w.emap, w.xp, st);
+        if (s != MOE_OK) return s;
+        s = gate_up_impl(v, w.xp, w.seg_expert, w.seg_offsets, w_gate, w_up, w.hp, status, st);
+        if (s != MOE_OK) return s;
+        s = down_impl(v, w.hp, w.seg_expert, w.seg_offsets, w_down, w.yp, status, st);
+        if (s != MOE_OK) return s;
+        return cuda_status(launch_ec_combine(w.yp, w.emap, w.row_w, nullptr, v.T, v.E, v.d, v.rows, out, sm_count(),
+                                             st));
+    }
     s = route_impl(v, x, w_router, bias, nullptr, w.topk_ids, w.topk_w, status, st);
     if (s != MOE_OK) return s;
     s = dispatch_impl(v, x, w.topk_ids, 0, w.counts, w.seg_expert, w.seg_offsets, w.seg_first_rank, w.dest, w.src,

@@ -1,0 +1,282 @@
+// Expert-choice routing: experts choose tokens instead of tokens choosing experts
+// ("Expert를 똑같이 나눴는데도 GPU가 대기하는 이유: MoE의 토큰 쏠림", section "라우팅 분포와
+// 학습 안정성").  The router scores S[t, e] (softmax over the experts of token t) arrive
+// expert-major from the route GEMM's epilogue; here
+//   * ec_select_kernel: one CTA per expert finds the C'-th largest score of its column by a
+//     three-pass radix select (11 + 11 + 10 bits of an order-preserving key) and then
+//     compacts the kept tokens in ascending token order: the row of a kept token is the
+//     number of kept tokens before it, from one block-wide scan per 1024 tokens.  Equal
+//     scores at the threshold go to the lower token ids.  It also writes the segment table
+//     (segment e = expert e, C' rows) and the [T, E] map from (token, expert) to row.
+//   * ec_gather_kernel: Xp[r] = X[src[r]], one warp per row, 16-byte vectors.
+//   * ec_combine_kernel: out[t] = base[t] + sum of row_w[r] * Yp[r] over the rows r of
+//     token t in ascending expert order, one warp per token.
+// The gather and the combine are HBM-bound; the selection reads the E x T scores four
+// times, from L2.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kSelectWarps = kSelectThreads / 32;
+static_assert(kSelectWarps == 32, "the warp-total scan below uses one lane per warp");
+
+// Order-preserving map of fp32 bits to uint32: larger float -> larger key.
+__device__ __forceinline__ uint32_t order_key(uint32_t u) { return (u & 0x80000000u) ? ~u : (u | 0x80000000u); }
+
+// Exclusive prefix sum of v over the CTA's threads in index order; *total = the CTA's sum.
+// Ends with a barrier, so `warp_sums` ([kSelectWarps + 1]) may be reused right after.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
+    }
+    if (lane == 31) warp_sums[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t w = warp_sums[lane];
+        uint32_t wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += t;
+        }
+        __syncwarp();
+        warp_sums[lane] = wi - w;
+        if (lane == 31) warp_sums[kSelectWarps] = wi;
+    }
+    __syncthreads();
+    const uint32_t r = warp_sums[warp] + inc - v;
+    *total = warp_sums[kSelectWarps];
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kSelectThreads, 1)
+    ec_select_kernel(const float* __restrict__ scores_t, int T, int E, int cp, int32_t* __restrict__ seg_expert,
+                     int32_t* __restrict__ seg_offsets, int32_t* __restrict__ src, float* __restrict__ row_w,
+                     int32_t* __restrict__ emap) {
+    __shared__ uint32_t hist[2048];
+    __shared__ uint32_t warp_sums[kSelectWarps + 1];
+    __shared__ uint32_t sel[2];
+    const int e = blockIdx.x;
+    const int tid = threadIdx.x;
+    if (tid == 0) { sel[0] = 0; sel[1] = 1; }
+    const uint32_t* col = reinterpret_cast<const uint32_t*>(scores_t) + static_cast<size_t>(e) * T;
+    if (tid == 0) {
+        seg_expert[e] = e;
+        seg_offsets[e] = e * cp;
+        if (e == E - 1) seg_offsets[E] = E * cp;
+    }
+
+    // ---- radix select of the cp-th largest key, most significant digit first
+    uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(cp);  // need: rank (from the top) inside the class
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        for (int i = tid; i < nb; i += kSelectThreads) hist[i] = 0;
+        __syncthreads();
+        for (int t = tid; t < T; t += kSelectThreads) {
+            const uint32_t k = order_key(__ldg(col + t));
+            if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & static_cast<uint32_t>(nb - 1)], 1u);
+        }
+        __syncthreads();
+        // thread i owns `per` bins counted down from the top digit; `above` = keys in higher bins
+        const int per = nb / kSelectThreads;
+        uint32_t mine = 0;
+        for (int j = 0; j < per; ++j) mine += hist[nb - 1 - (tid * per + j)];
+        uint32_t tot;
+        const uint32_t above = block_exclusive_scan(mine, warp_sums, &tot);
+        if (above < need && above + mine >= need) {
+            uint32_t a = above;
+            for (int j = 0; j < per; ++j) {
+                const int b = nb - 1 - (tid * per + j);
+                const uint32_t h = hist[b];
+                if (a + h >= need) {
+                    sel[0] = static_cast<uint32_t>(b);
+                    sel[1] = need - a;
+                    break;
+                }
+                a += h;
+            }
+        }
+        __syncthreads();
+        prefix |= sel[0] << shift;
+        mask |= static_cast<uint32_t>(nb - 1) << shift;
+        need = sel[1];
+        __syncthreads();
+    }
+    // prefix = the threshold key; `need` keys equal to it are kept (the lowest token ids),
+    // together with every key above it: cp - need of them
+
+    // ---- compaction in ascending token order
+    uint32_t run_gt = 0, run_eq = 0;
+    const int base_row = e * cp;
+#pragma unroll 1
+    for (int t0 = 0; t0 < T; t0 += kSelectThreads) {
+        const int t = t0 + tid;
+        uint32_t raw = 0;
+        bool gt = false, eq = false;
+        if (t < T) {
+            raw = __ldg(col + t);
+            const uint32_t k = order_key(raw);
+            gt = k > prefix;
+            eq = k == prefix;
+        }
+        uint32_t tot;
+        const uint32_t ex = block_exclusive_scan((gt ? 1u : 0u) | (eq ? 0x10000u : 0u), warp_sums, &tot);
+        const uint32_t gt_before = run_gt + (ex & 0xffffu), eq_before = run_eq + (ex >> 16);
+        if (t < T) {
+            int32_t row = -1;
+            const uint32_t pos = gt_before + min(eq_before, need);
+            if ((gt || (eq && eq_before < need)) && pos < static_cast<uint32_t>(cp)) {  // pos < cp always holds
+                row = base_row + static_cast<int32_t>(pos);
+                src[row] = t;
+                row_w[row] = __uint_as_float(raw);
+            }
+            emap[static_cast<size_t>(t) * E + e] = row;
+        }
+        run_gt += tot & 0xffffu;
+        run_eq += tot >> 16;
+    }
+}
+
+constexpr int kGatherUnroll = 8;
+
+__global__ void __launch_bounds__(256) ec_gather_kernel(const __nv_bfloat16* __restrict__ x,
+                                                        const int32_t* __restrict__ src, int rows, int T, int d,
+                                                        __nv_bfloat16* __restrict__ xp) {
+    const int lane = threadIdx.x & 31;
+    const int warps_total = gridDim.x * (blockDim.x >> 5);
+    const int vec_per_row = d / 8;
+    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps_total) {
+        const int t = __ldg(src + r);
+        if (t < 0 || t >= T) continue;
+        const uint4* xs = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
+        uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(r) * d);
+        for (int v = lane; v < vec_per_row; v += 32 * kGatherUnroll) {
+            uint4 val[kGatherUnroll];
+#pragma unroll
+            for (int u = 0; u < kGatherUnroll; ++u)
+                if (v + 32 * u < vec_per_row) val[u] = __ldg(xs + v + 32 * u);
+#pragma unroll
+            for (int u = 0; u < kGatherUnroll; ++u)
+                if (v + 32 * u < vec_per_row) dst[v + 32 * u] = val[u];
+        }
+    }
+}
+
+constexpr int kCombineWarps = 8;
+constexpr int kCombineUnroll = 4;
+
+__device__ __forceinline__ void fma4(float4& acc, float w, const float4& y) {
+    acc.x = fmaf(w, y.x, acc.x);
+    acc.y = fmaf(w, y.y, acc.y);
+    acc.z = fmaf(w, y.z, acc.z);
+    acc.w = fmaf(w, y.w, acc.w);
+}
+
+__global__ void __launch_bounds__(kCombineWarps * 32)
+    ec_combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ emap, const float* __restrict__ row_w,
+                      const float* __restrict__ base, int T, int E, int d, int rows, float* __restrict__ out) {
+    __shared__ int2 picks[kCombineWarps][kMaxExperts];  // (row, weight bits) of the current token
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int warps_total = gridDim.x * kCombineWarps;
+    const int vec_per_row = d / 4;
+    int2* my = picks[warp];
+    for (int t = blockIdx.x * kCombineWarps + warp; t < T; t += warps_total) {
+        int n = 0;
+        for (int c = 0; c < E; c += 32) {
+            const int e = c + lane;
+            const int r = e < E ? __ldg(emap + static_cast<size_t>(t) * E + e) : -1;
+            const bool ok = r >= 0 && r < rows;
+            const unsigned ball = __ballot_sync(0xffffffffu, ok);
+            if (ok) {
+                const int pos = n + __popc(ball & ((1u << lane) - 1u));
+                my[pos] = make_int2(r, __float_as_int(__ldg(row_w + r)));
+            }
+            n += __popc(ball);
+        }
+        __syncwarp();
+        float4* orow = reinterpret_cast<float4*>(out + static_cast<size_t>(t) * d);
+        const float4* brow = base ? reinterpret_cast<const float4*>(base + static_cast<size_t>(t) * d) : nullptr;
+        for (int v0 = lane; v0 < vec_per_row; v0 += 32 * kCombineUnroll) {
+            float4 acc[kCombineUnroll];
+#pragma unroll
+            for (int u = 0; u < kCombineUnroll; ++u) {
+                const int v = v0 + 32 * u;
+                acc[u] = (brow && v < vec_per_row) ? __ldg(brow + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            int p = 0;
+            // two rows at a time: all 2 x kCombineUnroll gathers in flight before any is used
+            for (; p + 1 < n; p += 2) {
+                const int2 a = my[p], b = my[p + 1];
+                float4 ya[kCombineUnroll], yb[kCombineUnroll];
+#pragma unroll
+                for (int u = 0; u < kCombineUnroll; ++u) {
+                    const int v = v0 + 32 * u;
+                    if (v < vec_per_row) {
+                        ya[u] = __ldg(reinterpret_cast<const float4*>(yp + static_cast<size_t>(a.x) * d) + v);
+                        yb[u] = __ldg(reinterpret_cast<const float4*>(yp + static_cast<size_t>(b.x) * d) + v);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kCombineUnroll; ++u) {
+                    if (v0 + 32 * u < vec_per_row) {
+                        fma4(acc[u], __int_as_float(a.y), ya[u]);
+                        fma4(acc[u], __int_as_float(b.y), yb[u]);
+                    }
+                }
+            }
+            if (p < n) {
+                const int2 a = my[p];
+#pragma unroll
+                for (int u = 0; u < kCombineUnroll; ++u) {
+                    const int v = v0 + 32 * u;
+                    if (v < vec_per_row)
+                        fma4(acc[u], __int_as_float(a.y),
+                             __ldg(reinterpret_cast<const float4*>(yp + static_cast<size_t>(a.x) * d) + v));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kCombineUnroll; ++u)
+                if (v0 + 32 * u < vec_per_row) orow[v0 + 32 * u] = acc[u];
+        }
+        __syncwarp();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_ec_select(const float* scores_t, int T, int E, int cp, int32_t* seg_expert, int32_t* seg_offsets,
+                             int32_t* src, float* row_w, int32_t* emap, cudaStream_t stream) {
+    if (T == 0 || E == 0) return cudaSuccess;
+    ec_select_kernel<<<E, kSelectThreads, 0, stream>>>(scores_t, T, E, cp, seg_expert, seg_offsets, src, row_w, emap);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ec_gather(const __nv_bfloat16* x, const int32_t* src, int rows, int T, int d, __nv_bfloat16* xp,
+                             int num_sms, cudaStream_t stream) {
+    if (rows == 0) return cudaSuccess;
+    int grid = (rows + 7) / 8;
+    if (grid > 8 * num_sms) grid = 8 * num_sms;
+    ec_gather_kernel<<<grid, 256, 0, stream>>>(x, src, rows, T, d, xp);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ec_combine(const float* yp, const int32_t* emap, const float* row_w, const float* base, int T,
+                              int E, int d, int rows, float* out, int num_sms, cudaStream_t stream) {
+    if (T == 0) return cudaSuccess;
+    int grid = (T + kCombineWarps - 1) / kCombineWarps;
+    if (grid > 8 * num_sms) grid = 8 * num_sms;
+    ec_combine_kernel<<<grid, kCombineWarps * 32, 0, stream>>>(yp, emap, row_w, base, T, E, d, rows, out);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -36,6 +36,7 @@ struct GemmArgs {
     float* topk_w;
     int k;
     int route_flags;  // MOE_ROUTE_SOFTMAX_ALL: weights from a softmax over all N logits
+    float* scores_t;  // route only: non-null = write softmax scores [N, M] (expert-major) instead of top-k
     int32_t* status;
 };
 
@@ -102,5 +103,14 @@ cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, i
 // combine.cu
 cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
                            int d, int rows, float* out, int num_sms, cudaStream_t stream);
+
+// expert_choice.cu
+constexpr int kSelectThreads = 1024;  // one CTA per expert
+cudaError_t launch_ec_select(const float* scores_t, int T, int E, int cp, int32_t* seg_expert, int32_t* seg_offsets,
+                             int32_t* src, float* row_w, int32_t* emap, cudaStream_t stream);
+cudaError_t launch_ec_gather(const __nv_bfloat16* x, const int32_t* src, int rows, int T, int d, __nv_bfloat16* xp,
+                             int num_sms, cudaStream_t stream);
+cudaError_t launch_ec_combine(const float* yp, const int32_t* emap, const float* row_w, const float* base, int T,
+                              int E, int d, int rows, float* out, int num_sms, cudaStream_t stream);
 
 }  // namespace moe

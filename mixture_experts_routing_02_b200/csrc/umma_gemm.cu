@@ -3,7 +3,10 @@
 // One persistent kernel template serves three contractions of the layer:
 //   * the router projection logits = X W_r^T, with top-k and the softmax over
 //     the selected logits fused into the epilogue ("Sparsely-Gated MoE 구현
-//     관점에서 살펴보기", sections "순전파 과정 ..." and "Top-2 라우팅의 수치 예시");
+//     관점에서 살펴보기", sections "순전파 과정 ..." and "Top-2 라우팅의 수치 예시"),
+//     or, for expert-choice routing, with the softmax over all E logits stored
+//     expert-major ("Expert를 똑같이 나눴는데도 GPU가 대기하는 이유", section
+//     "라우팅 분포와 학습 안정성");
 //   * the gate and up projections of every expert in one launch, with SwiGLU
 //     fused into the epilogue ("5.3 Expert Parallelism", section "3. 고도화된
 //     최적화: 오버래핑(Overlapping) 및 GroupGEMM"; MoonEP page "설치 및 통합":
@@ -299,6 +302,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (EPI == kEpiSwiglu || EPI == kEpiStore) {
                 epilogue_rows<EPI>(g, t_row, c.row0 + quarter * 32, c.row_end, n0, lane,
                                    epi_stage + (warp - 2) * kStageWords);
+            } else if (g.scores_t != nullptr) {
+                // expert choice: softmax over the E logits of this row, stored expert-major so
+                // that the 32 lanes (consecutive rows) of a warp write 128 contiguous bytes
+                float run_max = -INFINITY, run_sum = 0.f;
+                for (int cc = 0; cc < g.N; cc += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(t_row + cc, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int e = cc + i;
+                        if (e < g.N) {
+                            float v = __uint_as_float(r[i]);
+                            if (g.bias != nullptr) v += __ldg(g.bias + e);
+                            if (valid && g.logits != nullptr) g.logits[static_cast<size_t>(row) * g.N + e] = v;
+                            if (v > run_max) {
+                                run_sum = run_sum * expf(run_max - v) + 1.0f;
+                                run_max = v;
+                            } else {
+                                run_sum += expf(v - run_max);
+                            }
+                        }
+                    }
+                }
+                const float inv = 1.0f / run_sum;
+                for (int cc = 0; cc < g.N; cc += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(t_row + cc, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int e = cc + i;
+                        if (e < g.N && valid) {
+                            float v = __uint_as_float(r[i]);
+                            if (g.bias != nullptr) v += __ldg(g.bias + e);
+                            g.scores_t[static_cast<size_t>(e) * g.M + row] = expf(v - run_max) * inv;
+                        }
+                    }
+                }
             } else {
                 // router: top-k over the E logits of this row, softmax over the selected ones
                 float tv[kMaxTopK];

@@ -10,4 +10,5 @@ from .moe_oracle import (  # noqa: F401
     histogram, i64, layer_forward, margin_violations, num_segments, permute_rows,
     plain_segments, route, router_logits, shared_expert, silu, token_output, topk_ids, topk_weights,
     topk_weights_softmax_all, ExpertChoice, expert_choice, expert_choice_forward, expert_scores,
+    select_tokens, ec_margin_violations, enforce_ec_margin, combine_expert_choice, expert_choice_map,
 )

@@ -527,7 +527,12 @@ def expert_choice(logits64: np.ndarray, capacity: int) -> ExpertChoice:
     """Each expert e takes the C tokens with the largest S[t, e] (compared in fp32, the
     kernels' precision; equal scores go to the lower token id); its segment lists them in
     ascending token order."""
-    S = expert_scores(logits64)
+    return select_tokens(expert_scores(logits64), capacity)
+
+
+def select_tokens(S: np.ndarray, capacity: int) -> ExpertChoice:
+    """The expert-choice selection on given scores S [T, E]."""
+    S = np.asarray(S, dtype=np.float64)
     T, E = S.shape
     C = min(capacity, T)
     s32 = S.astype(np.float32)
@@ -548,8 +553,64 @@ def expert_choice_forward(x, w_router, bias, w_gate, w_up, w_down, capacity: int
     ec = expert_choice(logits, capacity)
     xp = f64(x)[ec.src]
     hp, yp = grouped_expert_ffn(xp, ec.segs, w_gate, w_up, w_down)
-    T, d = f64(x).shape[0], w_down.shape[1]
-    out = np.zeros((T, d))
-    for r in range(len(ec.src)):
-        out[ec.src[r]] += ec.row_w[r] * yp[r]
+    out = combine_expert_choice(yp, ec.src, ec.row_w, f64(x).shape[0])
     return logits, ec, xp, hp, yp, out
+
+
+def combine_expert_choice(yp64, src, row_w, T: int) -> np.ndarray:
+    """out[t] = sum over the rows r with src[r] = t of row_w[r] * Yp[r] (rows in order)."""
+    yp64 = np.asarray(yp64, dtype=np.float64)
+    out = np.zeros((T, yp64.shape[1]))
+    for r in range(len(src)):
+        out[src[r]] += row_w[r] * yp64[r]
+    return out
+
+
+def expert_choice_map(ec: "ExpertChoice", T: int) -> np.ndarray:
+    """[T, E] row of (t, e), or -1 where expert e did not keep token t."""
+    E = len(ec.picks)
+    m = np.full((T, E), -1, dtype=np.int64)
+    for r in range(len(ec.src)):
+        e = int(np.searchsorted(ec.segs.offsets, r, side="right") - 1)
+        m[ec.src[r], e] = r
+    return m
+
+
+def ec_margin_violations(S: np.ndarray, capacity: int, min_rel_gap: float) -> np.ndarray:
+    """Experts whose C-th and (C+1)-th largest scores are closer than min_rel_gap times the
+    C-th, so that a rounding difference in the scores could change which tokens the expert
+    keeps (a score's relative rounding error is about its logit's absolute error)."""
+    S = np.asarray(S, dtype=np.float64)
+    T, E = S.shape
+    if capacity >= T:
+        return np.zeros(E, dtype=bool)
+    srt = -np.sort(-S, axis=0)
+    return (srt[capacity - 1] - srt[capacity]) < min_rel_gap * srt[capacity - 1]
+
+
+def enforce_ec_margin(x, w_router, bias, capacity: int, redraw, min_rel_gap: float = 5e-4,
+                      max_redraws: int = 10000):
+    """Replace rows of X (a bf16 torch tensor, edited in place) until every expert's C-th
+    and (C+1)-th largest scores are at least min_rel_gap (relative) apart (``redraw(t,
+    attempt)`` returns a new bf16 row from the seeded generator).  Returns the number of
+    redraws."""
+    logits = router_logits(x, w_router, bias)
+    w64 = f64(w_router)
+    b64 = f64(bias) if bias is not None else 0.0
+    attempts = {}
+    n = 0
+    while True:
+        S = expert_scores(logits)
+        bad = np.nonzero(ec_margin_violations(S, capacity, min_rel_gap))[0]
+        if len(bad) == 0:
+            return n
+        if n >= max_redraws:
+            raise RuntimeError("could not satisfy the expert-choice margin")
+        e = int(bad[0])
+        t = int(np.argsort(-S[:, e], kind="stable")[capacity - 1])   # the last kept token
+        a = attempts.get(t, 0)
+        attempts[t] = a + 1
+        row = redraw(t, a)
+        x[t] = row
+        logits[t] = f64(row) @ w64.T + b64
+        n += 1

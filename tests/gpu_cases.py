@@ -97,7 +97,8 @@ def capacity_rows(w: syn.Workload) -> int:
 
 def moe_shape(w: syn.Workload, capacity: Optional[int] = None):
     C = capacity_rows(w) if capacity is None else capacity
-    return moe.shape(w.T, w.d, w.E, w.k, w.F, capacity=C, n_groups=w.n_groups, replica_slots=w.replica_slots)
+    return moe.shape(w.T, w.d, w.E, w.k, w.F, capacity=C, n_groups=w.n_groups, replica_slots=w.replica_slots,
+                     route_flags=moe.ROUTE_EXPERT_CHOICE if w.expert_choice else 0)
 
 
 @dataclasses.dataclass
@@ -114,7 +115,11 @@ class Case:
 def make_case(w: syn.Workload, seed: int = 0, weights_device="cpu", margin=True) -> Case:
     x, w_r, bias = syn.router_inputs(w, seed)
     if margin and w.E > 1:
-        oracle.enforce_margin(x, w_r, bias, w.k, lambda t, a: syn.x_row_redraw(w, seed, t, a))
+        redraw = lambda t, a: syn.x_row_redraw(w, seed, t, a)
+        if w.expert_choice:
+            oracle.enforce_ec_margin(x, w_r, bias, capacity_rows(w), redraw)
+        else:
+            oracle.enforce_margin(x, w_r, bias, w.k, redraw)
     wg, wu, wd = syn.expert_weights(w, seed, device=weights_device)
     return Case(w, x, w_r, bias, wg, wu, wd)
 
@@ -137,7 +142,7 @@ def run_layer(case: Case, capacity=None, stream=None, route_flags=0):
     """moe_layer_fwd through the C ABI; returns the output and every intermediate (CPU)."""
     w = case.w
     s = moe_shape(w, capacity)
-    s.route_flags = route_flags
+    s.route_flags |= route_flags
     n_seg, rows = moe.moe_layout(s)
     _, layer_bytes = moe.moe_workspace_size(s)
     ws = torch.empty(layer_bytes, dtype=torch.uint8, device="cuda")
@@ -157,6 +162,20 @@ def run_layer(case: Case, capacity=None, stream=None, route_flags=0):
         return t.view(*shape) if shape else t
 
     T, k = w.T, w.k
+    common = dict(
+        out=out, status=int(status.item()), n_seg=n_seg, rows=rows, ws=ws, x_dev=x,
+        seg_expert=view(v.seg_expert, n_seg, torch.int32).cpu(),
+        seg_offsets=view(v.seg_offsets, n_seg + 1, torch.int32).cpu(),
+        src=view(v.src, rows, torch.int32).cpu(),
+        xp=view(v.xp, rows * w.d, torch.bfloat16, (rows, w.d)),
+        hp=view(v.hp, rows * w.F, torch.bfloat16, (rows, w.F)),
+        yp=view(v.yp, rows * w.d, torch.float32, (rows, w.d)),
+    )
+    if s.route_flags & moe.ROUTE_EXPERT_CHOICE:
+        return dict(common,
+                    scores=view(v.scores, w.E * T, torch.float32, (w.E, T)).cpu(),
+                    emap=view(v.emap, T * w.E, torch.int32, (T, w.E)).cpu(),
+                    row_w=view(v.row_w, rows, torch.float32).cpu())
     res = dict(
         out=out, status=int(status.item()), n_seg=n_seg, rows=rows, ws=ws, x_dev=x,
         ids=view(v.topk_ids, T * k, torch.int32, (T, k)).cpu(),
@@ -181,3 +200,21 @@ def oracle_segments(case: Case, counts, capacity=None):
     else:
         segs = oracle.plain_segments(counts, capacity_rows(w) if capacity is None else capacity)
     return segs
+
+
+def expert_rows(pairs, wg, wu, wd, with_bound=False):
+    """{key: (h, y)} -- or (h, y, |h| . |W_d[e]|^T) with with_bound -- for (key, x_row64, expert)
+    pairs, evaluated in fp64 one expert's weights at a time."""
+    by_e = {}
+    for key, xrow, e in pairs:
+        by_e.setdefault(int(e), []).append((key, xrow))
+    out = {}
+    for e, items in by_e.items():
+        g64, u64, d64 = (oracle.f64(t[e].cpu()) for t in (wg, wu, wd))
+        xs = np.stack([x for _, x in items])
+        h = oracle.silu(xs @ g64.T) * (xs @ u64.T)
+        y = h @ d64.T
+        a = np.abs(h) @ np.abs(d64).T if with_bound else None
+        for i, (key, _) in enumerate(items):
+            out[key] = (h[i], y[i], a[i]) if with_bound else (h[i], y[i])
+    return out

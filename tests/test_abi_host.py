@@ -97,7 +97,11 @@ def test_workspace_sizes_grow_with_the_layer(lib):
     (dict(n_experts=300, top_k=2), 2), (dict(d_model=100), 2), (dict(d_ff=96), 2),
     (dict(n_experts=16, top_k=9), 2), (dict(T=1 << 29, top_k=2), 2),
     (dict(n_experts=256, n_groups=2, replica_slots=1000, T=64), 2),
-    (dict(route_flags=2), 1), (dict(route_flags=-1), 1),
+    (dict(route_flags=4), 1), (dict(route_flags=-1), 1),
+    # expert choice: needs a capacity, no groups, not with softmax-all
+    (dict(route_flags=2), 1), (dict(route_flags=3, capacity=8), 1),
+    (dict(route_flags=2, capacity=8, n_groups=2), 1),
+    (dict(route_flags=2, capacity=1 << 23, T=1 << 23, n_experts=256, top_k=1), 2),
 ])
 def test_shape_validation(lib, kw, code):
     s = _shape(**kw)
@@ -130,3 +134,29 @@ def test_misaligned_workspace_rejected(lib):
     rc = lib.moe_layer_fwd(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, None,
                            ctypes.c_void_p((1 << 20) + 64), need, None)
     assert rc == 3
+
+
+def test_expert_choice_layout_and_workspace(lib):
+    EC = moe.ROUTE_EXPERT_CHOICE
+    assert moe.moe_layout(_shape(route_flags=EC, capacity=10)) == (8, 80)
+    assert moe.moe_layout(_shape(route_flags=EC, capacity=1000)) == (8, 8 * 64)   # C' = min(C, T)
+    w = syn.EXPERT_CHOICE
+    C = -(-w.T * w.k // w.E)
+    s = moe.shape(w.T, w.d, w.E, w.k, w.F, capacity=C, route_flags=EC)
+    assert moe.moe_layout(s) == (w.E, w.T * w.k)
+    disp, layer = moe.moe_workspace_size(s)
+    assert disp == 0
+    rows = w.T * w.k
+    # Xp, Hp, Yp, the [E, T] scores and the [T, E] row map
+    assert layer >= rows * (2 * w.d + 2 * w.F + 4 * w.d) + 8 * w.T * w.E
+
+
+def test_expert_choice_calls_check_the_flag(lib):
+    s = _shape()                                     # top-k shape
+    ec = _shape(route_flags=moe.ROUTE_EXPERT_CHOICE, capacity=16)
+    fake = ctypes.c_void_p(1 << 20)                  # never dereferenced: the flag check comes first
+    assert lib.moe_route_scores(ctypes.byref(s), fake, fake, None, fake, None, None) == 1
+    assert lib.moe_expert_choose(ctypes.byref(s), *([fake] * 8), None) == 1
+    assert lib.moe_combine_expert_choice(ctypes.byref(s), fake, fake, fake, None, fake, None) == 1
+    assert lib.moe_dispatch(ctypes.byref(ec), fake, fake, 0, *([fake] * 9), 1 << 30, None) == 1
+    assert lib.moe_expert_choose(ctypes.byref(ec), None, *([fake] * 7), None) == 1   # null scores

@@ -13,27 +13,12 @@ import torch
 import oracle
 from mixture_experts_routing_02_b200 import synthetic as syn
 
-from gpu_cases import check_bf16_storage, check_close, check_layer_output, make_case, oracle_segments, run_layer, to_np
+from gpu_cases import (check_bf16_storage, check_close, check_layer_output, expert_rows, make_case, oracle_segments,
+                       run_layer, to_np)
 
 pytestmark = pytest.mark.gpu
 
 FULL = [syn.MIXTRAL_LIKE, syn.DEEPSEEK_LIKE, syn.SKEWED, syn.BALANCED]
-
-
-def _expert_rows(pairs, wg, wu, wd):
-    """{key: (h, y)} for (key, x_row64, expert) pairs, one expert's weights in fp64 at a time."""
-    by_e = {}
-    for key, xrow, e in pairs:
-        by_e.setdefault(int(e), []).append((key, xrow))
-    out = {}
-    for e, items in by_e.items():
-        g64, u64, d64 = (oracle.f64(t[e].cpu()) for t in (wg, wu, wd))
-        xs = np.stack([x for _, x in items])
-        h = oracle.silu(xs @ g64.T) * (xs @ u64.T)
-        y = h @ d64.T
-        for i, (key, _) in enumerate(items):
-            out[key] = (h[i], y[i])
-    return out
 
 
 @pytest.mark.parametrize("w", FULL, ids=[w.name for w in FULL])
@@ -76,7 +61,7 @@ def test_full_size_layer(cuda_ok, w):
         rows += sorted({a, b - 1, (a + b) // 2})
     x64 = oracle.f64(case.x)
     row_expert = {r: int(segs.expert[np.searchsorted(segs.offsets, r, side="right") - 1]) for r in rows}
-    ref_rows = _expert_rows([(r, x64[src[r] // w.k], row_expert[r]) for r in rows], case.wg, case.wu, case.wd)
+    ref_rows = expert_rows([(r, x64[src[r] // w.k], row_expert[r]) for r in rows], case.wg, case.wu, case.wd)
     rsel = torch.tensor(rows, device="cuda")
     check_bf16_storage(to_np(got["hp"][rsel]), np.stack([ref_rows[r][0] for r in rows]), "Hp (sampled rows)")
     check_close(to_np(got["yp"][rsel]), np.stack([ref_rows[r][1] for r in rows]), "Yp (sampled rows)")
@@ -84,7 +69,7 @@ def test_full_size_layer(cuda_ok, w):
     # layer output on sampled tokens, evaluated token by token (no dispatch)
     toks = sorted(set(rng.choice(w.T, size=12, replace=False).tolist()) | {0, w.T - 1})
     pairs = [((t, j), x64[t], ids[t, j]) for t in toks for j in range(w.k) if dest[t * w.k + j] >= 0]
-    ref_pairs = _expert_rows(pairs, case.wg, case.wu, case.wd)
+    ref_pairs = expert_rows(pairs, case.wg, case.wu, case.wd)
     ref_out = np.zeros((len(toks), w.d))
     for i, t in enumerate(toks):
         for j in range(w.k):
