@@ -252,6 +252,29 @@ moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* id
     const size_t need = permute_ws_bytes(v.T, v.k, v.E);
     if (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_WORKSPACE;
     const size_t scratch = permute_scratch_bytes(v.T, v.k, v.E);
+    PermuteArgs a{};
+    a.ids = ids; a.x = reinterpret_cast<const __nv_bfloat16*>(x); a.xp = reinterpret_cast<__nv_bfloat16*>(xp);
+    a.seg_expert = seg_expert; a.seg_offsets = seg_offsets; a.seg_first_rank = seg_first_rank;
+    a.dest = dest; a.src = src;
+    a.ticket = static_cast<uint32_t*>(ws);
+    a.sync = static_cast<uint32_t*>(ws) + 1;
+    a.tile_state = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 256);
+    a.status = status;
+    a.T = v.T; a.k = v.k; a.E = v.E; a.d = v.d; a.n_seg = v.n_seg;
+    a.tokens_per_tile = permute_tokens_per_tile(v.T, v.k);
+    a.rows = v.rows;
+    a.first_tile = first_tile;
+    a.n_tiles = permute_n_tiles(v.T, v.k);
+    if (!plan_ready && v.R == 0 && a.n_tiles > 0) {
+        // histogram, tables, ranks and row copies in one launch
+        a.capacity = v.C;
+        a.counts = counts; a.seg_expert_out = seg_expert; a.seg_offsets_out = seg_offsets;
+        a.seg_first_rank_out = seg_first_rank;
+        a.prefetch_x = static_cast<size_t>(v.T) * v.d * 2 <= (size_t(48) << 20);
+        if (static_cast<int64_t>(v.T) * v.k <= kCountMaxPairs && first_tile == 0)
+            return cuda_status(launch_dispatch_count(a, sm_count(), st));
+        return cuda_status(launch_dispatch_fused(a, sm_count(), st));
+    }
     if (!plan_ready) {
         // histogram partials + clearing of the look-back scratch in one launch, then the tables
         int32_t* partials = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + scratch);
@@ -262,18 +285,6 @@ moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* id
                              seg_first_rank, status, st);
         if (s != MOE_OK) return s;
     }
-    PermuteArgs a{};
-    a.ids = ids; a.x = reinterpret_cast<const __nv_bfloat16*>(x); a.xp = reinterpret_cast<__nv_bfloat16*>(xp);
-    a.seg_expert = seg_expert; a.seg_offsets = seg_offsets; a.seg_first_rank = seg_first_rank;
-    a.dest = dest; a.src = src;
-    a.ticket = static_cast<uint32_t*>(ws);
-    a.tile_state = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 256);
-    a.status = status;
-    a.T = v.T; a.k = v.k; a.E = v.E; a.d = v.d; a.n_seg = v.n_seg;
-    a.tokens_per_tile = permute_tokens_per_tile(v.T, v.k);
-    a.rows = v.rows;
-    a.first_tile = first_tile;
-    a.n_tiles = permute_n_tiles(v.T, v.k);
     return cuda_status(launch_permute(a, !plan_ready, sm_count(), st));
 }
 

@@ -31,6 +31,11 @@ constexpr uint32_t kFlagPrefix = 2u << 30;
 constexpr uint32_t kValueMask = (1u << 30) - 1;
 constexpr int kPermuteWarps = kPermuteThreads / 32;
 constexpr int kCopyUnroll = 8;
+constexpr int kLookbackWindow = 128;  // earlier tiles read per look-back round trip (when E allows)
+constexpr int kLookbackUnroll = 32;   // most look-back words one thread reads per round trip
+constexpr int kCountThreads = 1024;
+constexpr int kCountWarps = kCountThreads / 32;
+constexpr int kCountBatch = 8;  // expert ids per thread loaded together in the counting pass
 
 // Exclusive scan over the 256 threads of a block; *total receives the sum.
 __device__ __forceinline__ int block_exclusive_scan_256(int v, int* warp_sums, int* total) {
@@ -254,21 +259,150 @@ __global__ void __launch_bounds__(256) plan_kernel(int32_t* counts, const int32_
 
 // ------------------------------------------------------------------------------ stable rank + permute
 
+// Threads per expert in the look-back: a power of two, at most a warp, G * E <= kPermuteThreads.
+__device__ __forceinline__ int lookback_group(int E) {
+    int g = 32;
+    while (g > 1 && g * E > kPermuteThreads) g >>= 1;
+    return g;
+}
+
+struct TileSmem {
+    int wcnt[kPermuteWarps][kMaxExperts];  // per-warp counts of each expert in the tile
+    int h[kMaxExperts];                    // tile counts
+    int excl[kMaxExperts];                 // pairs of each expert in earlier tiles
+    int abort;
+};
+
+// Stable rank of the pairs of one tile.  Called by the whole CTA with sm.wcnt zeroed; ends
+// with a barrier.  *e = expert of this thread's pair (-1: none or out of range), *r = the
+// pair's rank among all pairs of that expert in q order.  A look-back wait that runs out
+// reports MOE_DEV_ERR_TIMEOUT, sets sm.abort and publishes nothing further for this tile.
+__device__ __forceinline__ void rank_tile(const PermuteArgs& a, int tile, TileSmem& sm, int* e_out, int* r_out) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = a.E, k = a.k;
+    const int t0 = tile * a.tokens_per_tile;
+    const int t1 = min(a.T, t0 + a.tokens_per_tile);
+    const int q0 = t0 * k;
+    const int nq = (t1 - t0) * k;
+
+    // 1. expert of this thread's pair and its rank among equal experts of the same warp
+    int e = -1;
+    if (tid < nq) {
+        e = __ldg(a.ids + q0 + tid);
+        if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) e = -1;
+    }
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int wrank = __popc(same & ((1u << lane) - 1u));
+    if (e >= 0 && wrank == 0) sm.wcnt[warp][e] = __popc(same);
+    __syncthreads();
+
+    // 2. tile histogram, published at once (tile 0: as its inclusive prefix)
+    if (tid < E) {
+        int h = 0;
+#pragma unroll
+        for (int w = 0; w < kPermuteWarps; ++w) h += sm.wcnt[w][tid];
+        sm.h[tid] = h;
+        st_relaxed_u32(a.tile_state + static_cast<size_t>(tile) * E + tid,
+                       (tile == 0 ? kFlagPrefix : kFlagAggregate) | static_cast<uint32_t>(h));
+        if (tile == 0) sm.excl[tid] = 0;
+    }
+    __syncthreads();
+    // 3. look back over a window of W = G * U earlier tiles per round trip: thread g of the
+    //    expert's group reads the U words of tiles hi - g*U - u (u < U), all loads in flight
+    //    together; the group adds the aggregates up to the nearest inclusive prefix and moves
+    //    the window back only when it holds no prefix.  Tiles tend to start together, so few
+    //    prefixes exist early; a wide window keeps the walk to a few round trips.  Every
+    //    decision is uniform inside a group.
+    const int G = lookback_group(E);
+    const int U = kLookbackWindow / G < kLookbackUnroll ? kLookbackWindow / G : kLookbackUnroll;
+    if (tile > 0 && tid < E * G) {
+        const int ge = tid / G, g = tid % G;
+        const int base = lane & ~(G - 1);
+        const unsigned gmask = (G == 32 ? 0xffffffffu : ((1u << G) - 1u)) << base;
+        int excl = 0;
+        int hi = tile - 1;
+        uint64_t t_start = 0;
+        uint32_t spins = 0;
+        bool gave_up = false;
+        while (hi >= 0) {
+            uint32_t w[kLookbackUnroll];
+#pragma unroll
+            for (int u = 0; u < kLookbackUnroll; ++u) {
+                const int j = hi - g * U - u;
+                w[u] = (u < U && j >= 0) ? ld_relaxed_u32(a.tile_state + static_cast<size_t>(j) * E + ge)
+                                         : kFlagPrefix;  // before tile 0: an inclusive prefix of 0
+            }
+            int first = kLookbackUnroll;  // nearest prefix among this thread's words
+#pragma unroll
+            for (int u = kLookbackUnroll - 1; u >= 0; --u)
+                if (u < U && (w[u] & ~kValueMask) == kFlagPrefix) first = u;
+            const unsigned has = __ballot_sync(gmask, first < kLookbackUnroll) & gmask;
+            const int gp = has ? __ffs(has >> base) - 1 : G;  // thread holding the nearest prefix
+            // words needed: all of threads g < gp, and u <= first of thread gp
+            const int need_u = g < gp ? U : (g == gp ? first + 1 : 0);
+            bool miss = false;
+            int v = 0;
+#pragma unroll
+            for (int u = 0; u < kLookbackUnroll; ++u) {
+                if (u < need_u) {
+                    if ((w[u] & ~kValueMask) == 0) miss = true;
+                    v += static_cast<int>(w[u] & kValueMask);
+                }
+            }
+            if (__ballot_sync(gmask, miss) & gmask) {
+                int out = 0;
+                if (g == 0 && (++spins & 63u) == 0) {
+                    const uint64_t now = globaltimer_ns();
+                    if (t_start == 0) t_start = now;
+                    else if (now - t_start > kWaitLimitNs) out = 1;
+                }
+                if (__shfl_sync(gmask, out, base)) {
+                    if (g == 0) {
+                        report(a.status, MOE_DEV_ERR_TIMEOUT);
+                        sm.abort = 1;
+                    }
+                    gave_up = true;
+                    break;
+                }
+                continue;
+            }
+            for (int o = G >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(gmask, v, o);
+            excl += v;
+            if (has) break;
+            hi -= G * U;
+        }
+        // a tile that gave up publishes no prefix, so the tiles after it give up too
+        if (g == 0) {
+            if (!gave_up)
+                st_relaxed_u32(a.tile_state + static_cast<size_t>(tile) * E + ge,
+                               kFlagPrefix | static_cast<uint32_t>(excl + sm.h[ge]));
+            sm.excl[ge] = excl;
+        }
+    }
+    __syncthreads();
+    int r = -1;
+    if (e >= 0) {
+        r = sm.excl[e] + wrank;
+        for (int w = 0; w < warp; ++w) r += sm.wcnt[w][e];
+    }
+    *e_out = e;
+    *r_out = r;
+}
+
 __global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs a) {
-    __shared__ int s_wcnt[kPermuteWarps][kMaxExperts];
+    __shared__ TileSmem sm;
     __shared__ int s_excl[kMaxExperts];
     __shared__ int s_cbeg[kMaxExperts + 1];
     __shared__ int s_cseg[kMaxSegments];
     __shared__ int warp_sums[8];
     __shared__ int s_tile;
-    __shared__ int s_abort;
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int E = a.E, k = a.k;
 
     // segments of each expert (CSR in shared memory); order inside an expert does not matter
     if (tid < E) s_excl[tid] = 0;
-    if (tid == 0) s_abort = 0;
+    if (tid == 0) sm.abort = 0;
     __syncthreads();
     for (int s = tid; s < a.n_seg; s += blockDim.x) {
         const int ex = __ldg(a.seg_expert + s);
@@ -292,80 +426,22 @@ __global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs
     }
     __syncthreads();
 
-    const unsigned lanemask_lt = (1u << lane) - 1u;
-
     for (;;) {
         if (tid == 0) s_tile = static_cast<int>(atomicAdd(a.ticket, 1u)) + a.first_tile;
-        for (int i = tid; i < kPermuteWarps * kMaxExperts; i += blockDim.x) (&s_wcnt[0][0])[i] = 0;
+        for (int i = tid; i < kPermuteWarps * kMaxExperts; i += blockDim.x) (&sm.wcnt[0][0])[i] = 0;
         __syncthreads();
         const int tile = s_tile;
-        if (tile >= a.n_tiles || s_abort) break;
+        if (tile >= a.n_tiles || sm.abort) break;
+        int e, r;
+        rank_tile(a, tile, sm, &e, &r);
+        if (sm.abort) break;
 
-        const int t0 = tile * a.tokens_per_tile;
-        const int t1 = min(a.T, t0 + a.tokens_per_tile);
-        const int q0 = t0 * k;
-        const int nq = (t1 - t0) * k;
-
-        // 1. expert of this thread's pair and its rank among equal experts of the same warp
-        int e = -1;
-        if (tid < nq) {
-            e = __ldg(a.ids + q0 + tid);
-            if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) e = -1;
-        }
-        const unsigned same = __match_any_sync(0xffffffffu, e);
-        const int wrank = __popc(same & lanemask_lt);
-        if (e >= 0 && wrank == 0) s_wcnt[warp][e] = __popc(same);
-        __syncthreads();
-
-        // 2. tile histogram, publish, look back, publish the inclusive prefix
-        if (tid < E) {
-            int h = 0;
-#pragma unroll
-            for (int w = 0; w < kPermuteWarps; ++w) h += s_wcnt[w][tid];
-            uint32_t* mine = a.tile_state + static_cast<size_t>(tile) * E + tid;
-            int excl = 0;
-            if (tile == 0) {
-                st_relaxed_u32(mine, kFlagPrefix | static_cast<uint32_t>(h));
-            } else {
-                st_relaxed_u32(mine, kFlagAggregate | static_cast<uint32_t>(h));
-                int j = tile - 1;
-                uint64_t t_start = 0;
-                uint32_t spins = 0;
-                bool gave_up = false;
-                while (j >= 0) {
-                    const uint32_t w = ld_relaxed_u32(a.tile_state + static_cast<size_t>(j) * E + tid);
-                    const uint32_t flag = w & ~kValueMask;
-                    if (flag == 0) {
-                        if ((++spins & 63u) == 0) {
-                            const uint64_t now = globaltimer_ns();
-                            if (t_start == 0) t_start = now;
-                            else if (now - t_start > kWaitLimitNs) {
-                                report(a.status, MOE_DEV_ERR_TIMEOUT);
-                                s_abort = 1;
-                                gave_up = true;
-                                break;
-                            }
-                        }
-                        continue;
-                    }
-                    excl += static_cast<int>(w & kValueMask);
-                    if (flag == kFlagPrefix) break;
-                    --j;
-                }
-                // a tile that gave up publishes no prefix, so the tiles after it give up too
-                if (!gave_up) st_relaxed_u32(mine, kFlagPrefix | static_cast<uint32_t>(excl + h));
-            }
-            s_excl[tid] = excl;
-        }
-        __syncthreads();
-        if (s_abort) break;
-
-        // 3. final slot of each pair
+        // 3. final slot of each pair: its expert's segment that holds rank r
+        const int q0 = tile * a.tokens_per_tile * k;
+        const int nq = (min(a.T, (tile + 1) * a.tokens_per_tile) - tile * a.tokens_per_tile) * k;
         if (tid < nq) {
             int dst = -1;
             if (e >= 0) {
-                int r = s_excl[e] + wrank;
-                for (int w = 0; w < warp; ++w) r += s_wcnt[w][e];
                 for (int p = s_cbeg[e]; p < s_cbeg[e + 1]; ++p) {
                     const int s = s_cseg[p];
                     const int fr = __ldg(a.seg_first_rank + s);
@@ -378,8 +454,272 @@ __global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs
             if (dst >= 0) a.src[dst] = q0 + tid;
         }
         __syncthreads();
+    }
+}
 
+// Copy the row of token t of X to its final slots dj[0..k) (one warp; 16-byte vectors, kCopyUnroll
+// in flight per lane).  Slots outside [0, rows) are skipped.
+__device__ __forceinline__ void copy_row(const __nv_bfloat16* __restrict__ x, int t, const int* dj, int k, int d,
+                                         int rows, __nv_bfloat16* __restrict__ xp, int lane) {
+    const int vec_per_row = d / 8;
+    const uint4* xs = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
+    for (int v = lane; v < vec_per_row; v += 32 * kCopyUnroll) {
+        uint4 val[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u)
+            if (v + 32 * u < vec_per_row) val[u] = __ldg(xs + v + 32 * u);
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            if (j < k && dj[j] >= 0 && dj[j] < rows) {
+                uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(dj[j]) * d);
+#pragma unroll
+                for (int u = 0; u < kCopyUnroll; ++u)
+                    if (v + 32 * u < vec_per_row) dst[v + 32 * u] = val[u];
+            }
+        }
+    }
+}
+
+// The whole dispatch of the plain (or capacity) layout in one launch, in two phases.
+//  1. Tiles from the ticket, as in rank_kernel: each pair's stable rank inside its expert,
+//     kept in dest for now.  The tile that holds the last ticket knows every expert's total
+//     (its inclusive prefix), so it writes counts and the segment tables and raises "ready".
+//  2. Every CTA (those that got no tile too) waits for "ready" and for all tiles to be
+//     ranked, then, one warp per token, turns ranks into final slots (capacity applied),
+//     writes dest and src, and copies the token's row to its slots.
+// A CTA only ever waits on tiles that running CTAs hold (tickets are taken in order), so no
+// CTA needs to be resident at the same time as another; every wait is bounded.  While
+// waiting, each warp prefetches the rows of X it will copy into L2, so the copy overlaps
+// the ranking.
+__global__ void __launch_bounds__(kPermuteThreads, 4) dispatch_fused_kernel(const PermuteArgs a) {
+    __shared__ TileSmem sm;
+    __shared__ int warp_sums[8];
+    __shared__ int s_tile;
+    __shared__ int s_off[kMaxExperts];
+    __shared__ int s_go;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = a.E, k = a.k;
+    const int warps_total = gridDim.x * kPermuteWarps;
+    const int my_warp = blockIdx.x * kPermuteWarps + warp;
+    if (tid == 0) sm.abort = 0;
+
+    // phase 1
+    for (;;) {
+        if (tid == 0) s_tile = static_cast<int>(atomicAdd(a.ticket, 1u)) + a.first_tile;
+        for (int i = tid; i < kPermuteWarps * kMaxExperts; i += blockDim.x) (&sm.wcnt[0][0])[i] = 0;
         __syncthreads();
+        const int tile = s_tile;
+        if (tile >= a.n_tiles || sm.abort) break;
+        int e, r;
+        rank_tile(a, tile, sm, &e, &r);
+        if (sm.abort) break;
+        const int q0 = tile * a.tokens_per_tile * k;
+        const int nq = (min(a.T, (tile + 1) * a.tokens_per_tile) - tile * a.tokens_per_tile) * k;
+        if (tid < nq) a.dest[q0 + tid] = r;  // rank for now (-1: no expert)
+        if (tile == a.n_tiles - 1) {
+            const int total_e = tid < E ? sm.excl[tid] + sm.h[tid] : 0;
+            const int v = (a.capacity > 0 && total_e > a.capacity) ? a.capacity : total_e;
+            int total;
+            const int off = block_exclusive_scan_256(tid < E ? v : 0, warp_sums, &total);
+            if (tid < E) {
+                a.counts[tid] = total_e;
+                a.seg_expert_out[tid] = tid;
+                a.seg_offsets_out[tid] = off;
+                a.seg_first_rank_out[tid] = 0;
+            }
+            if (tid == 0) a.seg_offsets_out[E] = total;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            red_release_add_u32(a.sync + 0, 1u);
+            if (tile == a.n_tiles - 1) st_release_u32(a.sync + 1, 1u);
+        }
+    }
+    if (sm.abort) {
+        if (tid == 0) st_relaxed_u32(a.sync + 2, 1u);
+        return;
+    }
+
+    // rows of X this warp copies in phase 2: into L2 while the last tiles are ranked
+    if (a.prefetch_x && lane == 0)
+        for (int t = my_warp; t < a.T; t += warps_total)
+            prefetch_l2_bulk(a.x + static_cast<size_t>(t) * a.d, static_cast<uint32_t>(a.d) * 2u);
+
+    // phase 2
+    if (tid == 0) {
+        int go = 1;
+        const uint64_t t0 = globaltimer_ns();
+        uint32_t spins = 0;
+        while (!(ld_acquire_u32(a.sync + 1) == 1u &&
+                 ld_acquire_u32(a.sync + 0) == static_cast<uint32_t>(a.n_tiles))) {
+            if (ld_relaxed_u32(a.sync + 2) != 0u) { go = 0; break; }
+            if ((++spins & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+                report(a.status, MOE_DEV_ERR_TIMEOUT);
+                st_relaxed_u32(a.sync + 2, 1u);
+                go = 0;
+                break;
+            }
+        }
+        s_go = go;
+    }
+    __syncthreads();
+    if (!s_go) return;
+    for (int e = tid; e < E; e += blockDim.x) s_off[e] = __ldcg(a.seg_offsets_out + e);
+    __syncthreads();
+
+    for (int t = my_warp; t < a.T; t += warps_total) {
+        int mine = -1;
+        if (lane < k) {
+            const int q = t * k + lane;
+            const int e = __ldg(a.ids + q);
+            const int r = __ldcg(a.dest + q);
+            if (static_cast<unsigned>(e) < static_cast<unsigned>(E) && r >= 0 &&
+                (a.capacity == 0 || r < a.capacity)) {
+                mine = s_off[e] + r;
+                if (mine >= a.rows) mine = -1;
+            }
+            a.dest[q] = mine;
+            if (mine >= 0) a.src[mine] = q;
+        }
+        int dj[kMaxTopK];
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) dj[j] = __shfl_sync(0xffffffffu, mine, j);
+        copy_row(a.x, t, dj, k, a.d, a.rows, a.xp, lane);
+    }
+}
+
+// Dispatch of the plain (or capacity) layout in one launch with no communication between CTAs,
+// for inputs of up to kCountMaxPairs pairs.  Each CTA owns a contiguous block of tokens and
+//  1. counts the expert ids of ALL pairs in shared memory (one shared atomic per id), split
+//     into the pairs before its block and the rest: the totals give the segment offsets and
+//     the first part is its block's exclusive prefix per expert, so neither a look-back nor
+//     a second launch is needed (the counting is repeated by every CTA; it reads T*k ids from
+//     L2, which is why it is limited to small T*k);
+//  2. ranks its own pairs in q order (match_any inside a warp, per-warp counts across warps),
+//     applies the capacity, writes dest and src (CTA 0 also writes counts and the tables);
+//  3. copies each of its tokens' rows to the token's slots, one warp per token.
+__global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const PermuteArgs a) {
+    __shared__ int s_pre[kMaxExperts];  // pairs of each expert before this CTA's block
+    __shared__ int s_tot[kMaxExperts];  // all pairs of each expert
+    __shared__ int s_off[kMaxExperts];  // segment offsets
+    __shared__ int s_run[kMaxExperts];  // pairs of each expert before the current chunk
+    __shared__ int s_wcnt[kCountWarps][kMaxExperts];
+    __shared__ int warp_sums[kCountWarps];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = a.E, k = a.k;
+    const unsigned lanemask_lt = (1u << lane) - 1u;
+    const int n = a.T * k;
+    const int tb = (a.T + gridDim.x - 1) / gridDim.x;
+    const int t_begin = min(a.T, static_cast<int>(blockIdx.x) * tb);
+    const int t_end = min(a.T, t_begin + tb);
+    const int q_begin = t_begin * k, q_end = t_end * k;
+
+    for (int i = tid; i < E; i += blockDim.x) { s_pre[i] = 0; s_tot[i] = 0; }
+    for (int i = tid; i < kCountWarps * kMaxExperts; i += blockDim.x) (&s_wcnt[0][0])[i] = 0;
+    __syncthreads();
+
+    // 1. counts of all pairs and of the pairs before this block (kCountBatch loads in flight)
+    for (int base = 0; base < n; base += blockDim.x * kCountBatch) {
+        int ev[kCountBatch];
+#pragma unroll
+        for (int u = 0; u < kCountBatch; ++u) {
+            const int i = base + u * blockDim.x + tid;
+            ev[u] = i < n ? __ldg(a.ids + i) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kCountBatch; ++u) {
+            const int i = base + u * blockDim.x + tid;
+            const int e = ev[u];
+            // one shared atomic per id: pairs before the block into s_pre, the rest into s_tot
+            if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(i < q_begin ? &s_pre[e] : &s_tot[e], 1);
+        }
+    }
+    __syncthreads();
+    for (int x = tid; x < E; x += blockDim.x) s_tot[x] += s_pre[x];
+    __syncthreads();
+
+    // 2a. segment offsets (capacity applied); CTA 0 publishes counts and the tables
+    {
+        const int tot = tid < E ? s_tot[tid] : 0;
+        const int v = (a.capacity > 0 && tot > a.capacity) ? a.capacity : tot;
+        // exclusive scan over the CTA (E <= 256 <= blockDim.x)
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += t;
+        }
+        if (lane == 31) warp_sums[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int w = warp_sums[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += t;
+            }
+            warp_sums[lane] = w;  // inclusive over warps
+        }
+        __syncthreads();
+        const int off = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+        if (tid < E) {
+            s_off[tid] = off;
+            s_run[tid] = s_pre[tid];
+            if (blockIdx.x == 0) {
+                a.counts[tid] = tot;
+                a.seg_expert_out[tid] = tid;
+                a.seg_offsets_out[tid] = off;
+                a.seg_first_rank_out[tid] = 0;
+            }
+        }
+        if (blockIdx.x == 0 && tid == 0) a.seg_offsets_out[E] = warp_sums[kCountWarps - 1];
+    }
+    __syncthreads();
+
+    // 2b. stable ranks of this block's pairs, in chunks of blockDim.x pairs
+    for (int q0 = q_begin; q0 < q_end; q0 += blockDim.x) {
+        const int q = q0 + tid;
+        int e = -1;
+        if (q < q_end) {
+            e = __ldg(a.ids + q);
+            if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) e = -1;
+        }
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int wrank = __popc(same & lanemask_lt);
+        if (e >= 0 && wrank == 0) s_wcnt[warp][e] = __popc(same);
+        __syncthreads();
+        if (q < q_end) {
+            int dst = -1;
+            if (e >= 0) {
+                int r = s_run[e] + wrank;
+                for (int w = 0; w < warp; ++w) r += s_wcnt[w][e];
+                if (a.capacity == 0 || r < a.capacity) {
+                    dst = s_off[e] + r;
+                    if (dst >= a.rows) dst = -1;
+                }
+            }
+            a.dest[q] = dst;
+            if (dst >= 0) a.src[dst] = q;
+        }
+        __syncthreads();
+        for (int x = tid; x < E; x += blockDim.x) {
+            int c = 0;
+            for (int w = 0; w < kCountWarps; ++w) { c += s_wcnt[w][x]; s_wcnt[w][x] = 0; }
+            s_run[x] += c;
+        }
+        __syncthreads();
+    }
+
+    // 3. rows of this block's tokens to their slots
+    for (int t = t_begin + warp; t < t_end; t += kCountWarps) {
+        const int mine = lane < k ? a.dest[static_cast<size_t>(t) * k + lane] : -1;
+        int dj[kMaxTopK];
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) dj[j] = __shfl_sync(0xffffffffu, mine, j);
+        copy_row(a.x, t, dj, k, a.d, a.rows, a.xp, lane);
     }
 }
 
@@ -392,28 +732,12 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* 
                                                            int rows, __nv_bfloat16* __restrict__ xp) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
-    const int vec_per_row = d / 8;
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
         const int mine = lane < k ? __ldg(dest + static_cast<size_t>(t) * k + lane) : -1;
         int dj[kMaxTopK];
 #pragma unroll
         for (int j = 0; j < kMaxTopK; ++j) dj[j] = __shfl_sync(0xffffffffu, mine, j);
-        const uint4* xs = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
-        for (int v = lane; v < vec_per_row; v += 32 * kCopyUnroll) {
-            uint4 val[kCopyUnroll];
-#pragma unroll
-            for (int u = 0; u < kCopyUnroll; ++u)
-                if (v + 32 * u < vec_per_row) val[u] = __ldg(xs + v + 32 * u);
-#pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j) {
-                if (j < k && dj[j] >= 0 && dj[j] < rows) {
-                    uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(dj[j]) * d);
-#pragma unroll
-                    for (int u = 0; u < kCopyUnroll; ++u)
-                        if (v + 32 * u < vec_per_row) dst[v + 32 * u] = val[u];
-                }
-            }
-        }
+        copy_row(x, t, dj, k, d, rows, xp, lane);
     }
 }
 
@@ -560,6 +884,25 @@ cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, c
     int sgrid = (a.T + 7) / 8;
     if (sgrid > 16 * num_sms) sgrid = 16 * num_sms;
     scatter_rows_kernel<<<sgrid, 256, 0, stream>>>(a.x, a.dest, a.T, a.k, a.d, a.rows, a.xp);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_fused(const PermuteArgs& a, int num_sms, cudaStream_t stream) {
+    cudaError_t err = cudaMemsetAsync(a.ticket, 0, permute_scratch_bytes(a.T, a.k, a.E), stream);
+    if (err != cudaSuccess) return err;
+    if (a.n_tiles == 0) return cudaSuccess;
+    int grid = (a.T + kPermuteWarps - 1) / kPermuteWarps;  // one warp per token in the copy phase
+    if (grid > 4 * num_sms) grid = 4 * num_sms;
+    if (grid < 1) grid = 1;
+    dispatch_fused_kernel<<<grid, kPermuteThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_t stream) {
+    if (a.T == 0) return cudaSuccess;
+    int grid = num_sms;
+    if (grid > a.T) grid = a.T;
+    dispatch_count_kernel<<<grid, kCountThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

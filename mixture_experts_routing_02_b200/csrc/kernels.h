@@ -72,6 +72,14 @@ struct PermuteArgs {
     int T, k, E, d, n_seg, tokens_per_tile, n_tiles;
     int rows;        // rows of xp: dest values outside [0, rows) are never written through
     int first_tile;  // 0; 1 only in moe_testing_dispatch_stalled (tile 0 is never taken)
+    // single-launch dispatch (no plan, tables not given): it writes the tables itself
+    int capacity;              // 0 = none
+    int32_t* counts;           // [E] out
+    int32_t* seg_expert_out;   // [E] out
+    int32_t* seg_offsets_out;  // [E + 1] out
+    int32_t* seg_first_rank_out;
+    uint32_t* sync;            // [3] zero on entry: tiles ranked, tables ready, abort
+    int prefetch_x;            // 1: prefetch the rows of X into L2 while the ranks are found
 };
 
 constexpr int kMaxHistogramPartials = 64;   // CTAs of the fused histogram (one partial count row each)
@@ -97,6 +105,12 @@ cudaError_t launch_plan(int32_t* counts, const int32_t* partials, int n_partials
                         cudaStream_t stream);
 // ws_cleared: the ticket and look-back words are already zero (cleared by the fused histogram)
 cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, cudaStream_t stream);
+// Histogram, segment tables, stable rank and row copies in one launch (plain or capacity layout):
+// with a look-back across tiles (any size), or with every CTA recounting all ids (up to
+// kCountMaxPairs pairs; no communication between CTAs, no workspace).
+cudaError_t launch_dispatch_fused(const PermuteArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_t stream);
+constexpr int kCountMaxPairs = 1 << 16;
 cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int route_flags, int32_t* ids,
                                      float* w, int num_sms, cudaStream_t stream);
 
