@@ -591,18 +591,21 @@ __global__ void __launch_bounds__(kPermuteThreads, 4) dispatch_fused_kernel(cons
 }
 
 // Dispatch of the plain (or capacity) layout in one launch with no communication between CTAs,
-// for inputs of up to kCountMaxPairs pairs.  Each CTA owns a contiguous block of tokens and
+// for inputs of up to kCountMaxPairs pairs.  The tokens form 2G blocks for G CTAs; CTA b owns
+// block b and block 2G-1-b (one from the front, one from the back: with a capacity, later
+// tokens lose more pairs, so the pairing evens out the rows each CTA copies).  Each CTA
 //  1. counts the expert ids of ALL pairs in shared memory (one shared atomic per id), split
-//     into the pairs before its block and the rest: the totals give the segment offsets and
-//     the first part is its block's exclusive prefix per expert, so neither a look-back nor
-//     a second launch is needed (the counting is repeated by every CTA; it reads T*k ids from
-//     L2, which is why it is limited to small T*k);
-//  2. ranks its own pairs in q order (match_any inside a warp, per-warp counts across warps),
-//     applies the capacity, writes dest and src (CTA 0 also writes counts and the tables);
+//     into the pairs before its first block, the pairs between its blocks and the rest: the
+//     totals give the segment offsets and the partial sums give each block's exclusive prefix
+//     per expert, so neither a look-back nor a second launch is needed (the counting is
+//     repeated by every CTA; it reads T*k ids from L2, which is why it is limited to small T*k);
+//  2. ranks the pairs of its blocks in q order (match_any inside a warp, per-warp counts across
+//     warps), applies the capacity, writes dest and src (CTA 0 also writes counts and tables);
 //  3. copies each of its tokens' rows to the token's slots, one warp per token.
 __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const PermuteArgs a) {
-    __shared__ int s_pre[kMaxExperts];  // pairs of each expert before this CTA's block
-    __shared__ int s_tot[kMaxExperts];  // all pairs of each expert
+    __shared__ int s_a[kMaxExperts];    // pairs of each expert before the first block
+    __shared__ int s_m[kMaxExperts];    // ... from the first block up to the second
+    __shared__ int s_tot[kMaxExperts];  // ... from the second block on; then: all pairs
     __shared__ int s_off[kMaxExperts];  // segment offsets
     __shared__ int s_run[kMaxExperts];  // pairs of each expert before the current chunk
     __shared__ int s_wcnt[kCountWarps][kMaxExperts];
@@ -612,16 +615,24 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
     const int E = a.E, k = a.k;
     const unsigned lanemask_lt = (1u << lane) - 1u;
     const int n = a.T * k;
-    const int tb = (a.T + gridDim.x - 1) / gridDim.x;
-    const int t_begin = min(a.T, static_cast<int>(blockIdx.x) * tb);
-    const int t_end = min(a.T, t_begin + tb);
-    const int q_begin = t_begin * k, q_end = t_end * k;
+    const int G = gridDim.x;
+    const int tb = (a.T + 2 * G - 1) / (2 * G);
+    int tb_[2], te_[2];
+    {
+        const int blk[2] = {static_cast<int>(blockIdx.x), 2 * G - 1 - static_cast<int>(blockIdx.x)};
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            tb_[r] = min(a.T, blk[r] * tb);
+            te_[r] = min(a.T, tb_[r] + tb);
+        }
+    }
+    const int q1 = tb_[0] * k, q2 = tb_[1] * k;  // q1 <= q2
 
-    for (int i = tid; i < E; i += blockDim.x) { s_pre[i] = 0; s_tot[i] = 0; }
+    for (int i = tid; i < E; i += blockDim.x) { s_a[i] = 0; s_m[i] = 0; s_tot[i] = 0; }
     for (int i = tid; i < kCountWarps * kMaxExperts; i += blockDim.x) (&s_wcnt[0][0])[i] = 0;
     __syncthreads();
 
-    // 1. counts of all pairs and of the pairs before this block (kCountBatch loads in flight)
+    // 1. counts of all pairs, split at the starts of the two blocks (kCountBatch loads in flight)
     for (int base = 0; base < n; base += blockDim.x * kCountBatch) {
         int ev[kCountBatch];
 #pragma unroll
@@ -633,17 +644,15 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
         for (int u = 0; u < kCountBatch; ++u) {
             const int i = base + u * blockDim.x + tid;
             const int e = ev[u];
-            // one shared atomic per id: pairs before the block into s_pre, the rest into s_tot
-            if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(i < q_begin ? &s_pre[e] : &s_tot[e], 1);
+            if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
+                atomicAdd(i < q1 ? &s_a[e] : (i < q2 ? &s_m[e] : &s_tot[e]), 1);
         }
     }
-    __syncthreads();
-    for (int x = tid; x < E; x += blockDim.x) s_tot[x] += s_pre[x];
     __syncthreads();
 
     // 2a. segment offsets (capacity applied); CTA 0 publishes counts and the tables
     {
-        const int tot = tid < E ? s_tot[tid] : 0;
+        const int tot = tid < E ? s_a[tid] + s_m[tid] + s_tot[tid] : 0;
         const int v = (a.capacity > 0 && tot > a.capacity) ? a.capacity : tot;
         // exclusive scan over the CTA (E <= 256 <= blockDim.x)
         int x = v;
@@ -667,7 +676,6 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
         const int off = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
         if (tid < E) {
             s_off[tid] = off;
-            s_run[tid] = s_pre[tid];
             if (blockIdx.x == 0) {
                 a.counts[tid] = tot;
                 a.seg_expert_out[tid] = tid;
@@ -677,49 +685,59 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
         }
         if (blockIdx.x == 0 && tid == 0) a.seg_offsets_out[E] = warp_sums[kCountWarps - 1];
     }
-    __syncthreads();
 
-    // 2b. stable ranks of this block's pairs, in chunks of blockDim.x pairs
-    for (int q0 = q_begin; q0 < q_end; q0 += blockDim.x) {
-        const int q = q0 + tid;
-        int e = -1;
-        if (q < q_end) {
-            e = __ldg(a.ids + q);
-            if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) e = -1;
-        }
-        const unsigned same = __match_any_sync(0xffffffffu, e);
-        const int wrank = __popc(same & lanemask_lt);
-        if (e >= 0 && wrank == 0) s_wcnt[warp][e] = __popc(same);
+    // 2b. stable ranks of the pairs of each block, in chunks of blockDim.x pairs
+#pragma unroll 1
+    for (int r = 0; r < 2; ++r) {
+        if (r == 1 && tb_[1] == tb_[0]) break;  // one block only (2G > T at the end)
+        for (int x = tid; x < E; x += blockDim.x) s_run[x] = r == 0 ? s_a[x] : s_a[x] + s_m[x];
         __syncthreads();
-        if (q < q_end) {
-            int dst = -1;
-            if (e >= 0) {
-                int r = s_run[e] + wrank;
-                for (int w = 0; w < warp; ++w) r += s_wcnt[w][e];
-                if (a.capacity == 0 || r < a.capacity) {
-                    dst = s_off[e] + r;
-                    if (dst >= a.rows) dst = -1;
-                }
+        const int qb = tb_[r] * k, qe = te_[r] * k;
+        for (int q0 = qb; q0 < qe; q0 += blockDim.x) {
+            const int q = q0 + tid;
+            int e = -1;
+            if (q < qe) {
+                e = __ldg(a.ids + q);
+                if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) e = -1;
             }
-            a.dest[q] = dst;
-            if (dst >= 0) a.src[dst] = q;
+            const unsigned same = __match_any_sync(0xffffffffu, e);
+            const int wrank = __popc(same & lanemask_lt);
+            if (e >= 0 && wrank == 0) s_wcnt[warp][e] = __popc(same);
+            __syncthreads();
+            if (q < qe) {
+                int dst = -1;
+                if (e >= 0) {
+                    int rk = s_run[e] + wrank;
+                    for (int w = 0; w < warp; ++w) rk += s_wcnt[w][e];
+                    if (a.capacity == 0 || rk < a.capacity) {
+                        dst = s_off[e] + rk;
+                        if (dst >= a.rows) dst = -1;
+                    }
+                }
+                a.dest[q] = dst;
+                if (dst >= 0) a.src[dst] = q;
+            }
+            __syncthreads();
+            for (int x = tid; x < E; x += blockDim.x) {
+                int c = 0;
+                for (int w = 0; w < kCountWarps; ++w) { c += s_wcnt[w][x]; s_wcnt[w][x] = 0; }
+                s_run[x] += c;
+            }
+            __syncthreads();
         }
-        __syncthreads();
-        for (int x = tid; x < E; x += blockDim.x) {
-            int c = 0;
-            for (int w = 0; w < kCountWarps; ++w) { c += s_wcnt[w][x]; s_wcnt[w][x] = 0; }
-            s_run[x] += c;
-        }
-        __syncthreads();
     }
 
-    // 3. rows of this block's tokens to their slots
-    for (int t = t_begin + warp; t < t_end; t += kCountWarps) {
-        const int mine = lane < k ? a.dest[static_cast<size_t>(t) * k + lane] : -1;
-        int dj[kMaxTopK];
+    // 3. rows of this CTA's tokens to their slots
+#pragma unroll 1
+    for (int r = 0; r < 2; ++r) {
+        if (r == 1 && tb_[1] == tb_[0]) break;
+        for (int t = tb_[r] + warp; t < te_[r]; t += kCountWarps) {
+            const int mine = lane < k ? a.dest[static_cast<size_t>(t) * k + lane] : -1;
+            int dj[kMaxTopK];
 #pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) dj[j] = __shfl_sync(0xffffffffu, mine, j);
-        copy_row(a.x, t, dj, k, a.d, a.rows, a.xp, lane);
+            for (int j = 0; j < kMaxTopK; ++j) dj[j] = __shfl_sync(0xffffffffu, mine, j);
+            copy_row(a.x, t, dj, k, a.d, a.rows, a.xp, lane);
+        }
     }
 }
 
