@@ -36,8 +36,6 @@ if ROOT not in sys.path:
 METRIC = "MoE layer fwd tokens/s; grouped-GEMM TFLOPS and permute GB/s vs roofline"
 FLUSH_BYTES = 256 << 20
 KERNELS = ("route", "dispatch", "gate_up", "down", "combine")
-LAUNCHES_PER_STEP = 7  # route, histogram, segments|plan, permute, gate_up, down, combine
-LAUNCHES_PER_STEP_EC = 6  # expert choice: route scores, select, gather, gate_up, down, combine
 
 
 def _peaks():
@@ -333,6 +331,12 @@ def run_ours(args, w):
         scores = view(v.scores, w.E * w.T, torch.float32)
         emap = view(v.emap, w.T * w.E, torch.int32)
         row_w = view(v.row_w, rows_alloc, torch.float32)
+    # the router projection's reduction is split over more CTAs when its row tiles are few
+    route_ws_bytes = moe.moe_route_workspace_size(s)
+    route_ws = torch.empty(max(route_ws_bytes, 256), dtype=torch.uint8, device=dev) if route_ws_bytes else None
+    launches = ((2 if route_ws_bytes else 1)                                   # route (+ partial sums)
+                + (2 if ec else (4 if w.n_groups else 1))                      # dispatch
+                + 3)                                                           # gate_up, down, combine
 
     Fs = args.shared_expert
     if Fs:
@@ -354,11 +358,11 @@ def run_ours(args, w):
             se1.record(side)
             shared_ms.append((se0, se1))
         if ec:
-            moe.moe_route_scores(s, x, w_r, bias, scores, status, stream)
+            moe.moe_route_scores_ws(s, x, w_r, bias, scores, status, route_ws, stream)
             ev[1].record(stream)
             moe.moe_expert_choose(s, scores, x, seg_e, seg_o, src, row_w, emap, xp, stream)
         else:
-            moe.moe_route(s, x, w_r, bias, None, ids, wts, status, stream)
+            moe.moe_route_ws(s, x, w_r, bias, None, ids, wts, status, route_ws, stream)
             ev[1].record(stream)
             moe.moe_dispatch(s, x, ids, 0, counts, seg_e, seg_o, seg_f, dest, src, xp, status, dws, stream)
         ev[2].record(stream)
@@ -507,7 +511,7 @@ def run_ours(args, w):
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init weights)", "config": _config(w, capacity),
-        "rows_dispatched": rows_used, "gpu_launches": (LAUNCHES_PER_STEP_EC if ec else LAUNCHES_PER_STEP) * args.steps,
+        "rows_dispatched": rows_used, "gpu_launches": launches * args.steps,
         "roofline": roof,
         "breakdown": {n: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in b.items()}
                       for n, b in breakdown.items()},
@@ -518,7 +522,7 @@ def run_ours(args, w):
     if shared_info:
         line["shared_expert"] = shared_info
         line["config"]["shared_expert_d_ff"] = Fs
-        line["gpu_launches"] = ((LAUNCHES_PER_STEP_EC if ec else LAUNCHES_PER_STEP) + 2) * args.steps
+        line["gpu_launches"] = (launches + 2) * args.steps
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         wg0, wu0, wd0 = wg[:1].cpu(), wu[:1].cpu(), wd[:1].cpu()
         cv, desc, _ = _oracle_sample(w, seed, 512, 32, wg0, wu0, wd0)

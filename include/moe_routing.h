@@ -377,6 +377,24 @@ MOE_API moe_status_t moe_testing_dispatch_stalled(const moe_shape_t *shape, cons
                                           moe_stream_t stream);
 
 /*
+ * The router projection on more CTAs.  Its ceil(T/128) row tiles can be fewer than the SMs;
+ * with a workspace the reduction over d is split into S parts (S chosen from T, d and the SM
+ * count; each part at least 256 columns of d), the parts' fp32 partial logits go to the
+ * workspace, and a second kernel sums them in a fixed order, adds the bias and routes.  The
+ * results equal those of moe_route / moe_route_scores up to fp32 rounding of the logits.
+ *   moe_route_workspace_size: bytes needed (0 when the split does not pay: then the calls
+ *                             below run the single-pass kernel and ignore ws)
+ *   ws: device, 256-byte aligned, at least that size; contents need no initialisation.
+ */
+MOE_API moe_status_t moe_route_workspace_size(const moe_shape_t *shape, size_t *bytes);
+MOE_API moe_status_t moe_route_ws(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *w_router,
+                          const float *bias, float *logits, int32_t *topk_ids, float *topk_w, int32_t *status,
+                          void *ws, size_t ws_bytes, moe_stream_t stream);
+MOE_API moe_status_t moe_route_scores_ws(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *w_router,
+                                 const float *bias, float *scores, int32_t *status, void *ws, size_t ws_bytes,
+                                 moe_stream_t stream);
+
+/*
  * Expert-choice routing (shape.route_flags = MOE_ROUTE_EXPERT_CHOICE; see
  * moe_shape_t).  Router scores, transposed so that each expert's column is
  * contiguous:

@@ -19,6 +19,7 @@ __all__ = [
     "moe_histogram", "moe_segments", "moe_plan_balanced", "moe_dispatch", "moe_dispatch_static", "moe_expert_gate_up",
     "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_combine_add", "moe_shared_expert", "moe_layer_fwd",
     "moe_route_scores", "moe_expert_choose", "moe_combine_expert_choice",
+    "moe_route_workspace_size", "moe_route_ws", "moe_route_scores_ws",
     "moe_layer_views",
     "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT", "ROUTE_SOFTMAX_ALL", "ROUTE_EXPERT_CHOICE",
 ]
@@ -74,6 +75,9 @@ SYMBOLS = {
     "moe_route_scores": [_S, _P, _P, _P, _P, _P, _P],
     "moe_expert_choose": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_combine_expert_choice": [_S, _P, _P, _P, _P, _P, _P],
+    "moe_route_workspace_size": [_S, _P],
+    "moe_route_ws": [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "moe_route_scores_ws": [_S, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
 }
 
 _lib = None
@@ -253,3 +257,25 @@ def moe_expert_choose(s, scores, x, seg_expert, seg_offsets, src, row_w, emap, x
 def moe_combine_expert_choice(s, yp, emap, row_w, base, out, stream=None):
     _check("moe_combine_expert_choice", load_library().moe_combine_expert_choice(
         ctypes.byref(s), _ptr(yp), _ptr(emap), _ptr(row_w), _ptr(base), _ptr(out), _stream(stream)))
+
+
+def moe_route_workspace_size(s) -> int:
+    n = ctypes.c_size_t()
+    _check("moe_route_workspace_size", load_library().moe_route_workspace_size(ctypes.byref(s), ctypes.byref(n)))
+    return n.value
+
+
+def _nbytes(ws):
+    return ws.numel() * ws.element_size() if ws is not None else 0
+
+
+def moe_route_ws(s, x, w_router, bias, logits, topk_ids, topk_w, status=None, ws=None, stream=None):
+    _check("moe_route_ws", load_library().moe_route_ws(
+        ctypes.byref(s), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logits), _ptr(topk_ids), _ptr(topk_w),
+        _ptr(status), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def moe_route_scores_ws(s, x, w_router, bias, scores, status=None, ws=None, stream=None):
+    _check("moe_route_scores_ws", load_library().moe_route_scores_ws(
+        ctypes.byref(s), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(scores), _ptr(status), _ptr(ws), _nbytes(ws),
+        _stream(stream)))

@@ -144,6 +144,60 @@ moe_status_t route_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_
     return cuda_status(launch_umma_gemm(kEpiRoute, ta, tb, tb, g, grid, st));
 }
 
+// The router projection has only ceil(T/128) row tiles.  When they are fewer than the SMs, its
+// reduction over d is cut into S parts (each at least 4 k-blocks of 64), the S*ceil(T/128) work
+// units write fp32 partial logits [S][T][ldp] to a workspace, and a warp-per-token kernel sums
+// the parts in order (so the result does not depend on timing), adds the bias and routes.
+constexpr int kMaxRouteSplits = 8;
+
+int route_splits(const Dims& v) {
+    const int m_tiles = (v.T + 127) / 128;
+    int s = sm_count() / std::max(1, m_tiles);
+    s = std::min(s, kMaxRouteSplits);
+    s = std::min(s, (v.d / 64) / 4);
+    return std::max(s, 1);
+}
+
+int route_ldp(const Dims& v) {
+    const int epad = std::max(16, (v.E + 15) / 16 * 16);
+    return (epad + 31) / 32 * 32;
+}
+
+size_t route_ws_bytes(const Dims& v) {
+    const int S = route_splits(v);
+    if (S < 2) return 0;
+    return align256(static_cast<size_t>(S) * v.T * route_ldp(v) * sizeof(float));
+}
+
+// Split router projection + routing; false when it does not apply (one part, or no workspace).
+bool route_split_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
+                      float* logits, int32_t* ids, float* w, float* scores, int32_t* status, void* ws,
+                      size_t ws_bytes, cudaStream_t st, moe_status_t* result) {
+    const size_t need = route_ws_bytes(v);
+    if (need == 0 || ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return false;
+    if (!have_encoder()) { *result = MOE_ERR_CUDA; return true; }
+    const int S = route_splits(v);
+    const int epad = std::max(16, (v.E + 15) / 16 * 16);
+    const int ldp = route_ldp(v);
+    CUtensorMap ta, tb;
+    if (!tmap_rows(&ta, x, v.T, v.d) || !tmap_experts(&tb, w_router, 1, v.E, v.d, epad)) {
+        *result = MOE_ERR_CUDA;
+        return true;
+    }
+    GemmArgs g{};
+    g.seg_offsets = nullptr; g.seg_expert = nullptr; g.n_seg = 1; g.M = v.T; g.K = v.d; g.N = v.E;
+    g.BN = epad; g.n_tiles_n = 1; g.mma_n = epad; g.stages = gemm_pick_stages(epad);
+    g.out = ws; g.ldo = ldp; g.status = status;
+    g.k_splits = S; g.split_stride = static_cast<size_t>(v.T) * ldp;
+    const int grid = std::min(sm_count(), (v.T + 127) / 128 * S);
+    moe_status_t r = cuda_status(launch_umma_gemm(kEpiStore, ta, tb, tb, g, grid, st));
+    if (r == MOE_OK)
+        r = cuda_status(launch_route_logits(static_cast<const float*>(ws), S, ldp, g.split_stride, bias, v.T, v.E, v.k,
+                                            v.flags & ~MOE_ROUTE_EXPERT_CHOICE, logits, ids, w, scores, sm_count(), st));
+    *result = r;
+    return true;
+}
+
 // Expert-choice scores: the router projection with the softmax over all E logits in the
 // epilogue, written expert-major ([E, T]).
 moe_status_t route_scores_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
@@ -313,7 +367,7 @@ void* static_scratch_address() {
 
 struct LayerLayout {
     size_t ids, w, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, dispatch_ws, xp, hp, yp, scores, emap,
-        row_w, total;
+        row_w, route_ws, total;
     size_t dispatch_ws_bytes;
 };
 
@@ -339,6 +393,7 @@ LayerLayout layer_layout(const Dims& v) {
     L.scores = o; o = align256(o + te * 4);
     L.emap = o; o = align256(o + te * 4);
     L.row_w = o; o = align256(o + (v.ec() ? static_cast<size_t>(v.rows) * 4 : 0));
+    L.route_ws = o; o = align256(o + route_ws_bytes(v));
     L.total = o;
     return L;
 }
@@ -383,6 +438,44 @@ moe_status_t moe_route(const moe_shape_t* shape, const moe_bf16_t* x, const moe_
     if (s != MOE_OK) return s;
     if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     return route_impl(v, x, w_router, bias, logits, topk_ids, topk_w, status, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_route_workspace_size(const moe_shape_t* shape, size_t* bytes) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (bytes) *bytes = route_ws_bytes(v);
+    return MOE_OK;
+}
+
+moe_status_t moe_route_ws(const moe_shape_t* shape, const moe_bf16_t* x, const moe_bf16_t* w_router,
+                          const float* bias, float* logits, int32_t* topk_ids, float* topk_w, int32_t* status,
+                          void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims v;
+    moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
+    if (!x || !w_router || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+    if (v.T == 0) return MOE_OK;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (route_split_impl(v, x, w_router, bias, logits, topk_ids, topk_w, nullptr, status, ws, ws_bytes, st, &s)) return s;
+    return route_impl(v, x, w_router, bias, logits, topk_ids, topk_w, status, st);
+}
+
+moe_status_t moe_route_scores_ws(const moe_shape_t* shape, const moe_bf16_t* x, const moe_bf16_t* w_router,
+                                 const float* bias, float* scores, int32_t* status, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream) {
+    Dims v;
+    moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!v.ec()) return MOE_ERR_INVALID_ARG;
+    if (!x || !w_router || !scores) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+    if (v.T == 0) return MOE_OK;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (route_split_impl(v, x, w_router, bias, nullptr, nullptr, nullptr, scores, status, ws, ws_bytes, st, &s)) return s;
+    return route_scores_impl(v, x, w_router, bias, scores, status, st);
 }
 
 moe_status_t moe_route_from_logits(const moe_shape_t* shape, const float* logits, int32_t* topk_ids, float* topk_w,
@@ -639,8 +732,12 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
     moe_layer_views_t w;
     moe_layer_views(shape, ws, &w);
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* route_ws = static_cast<uint8_t*>(ws) + L.route_ws;
+    const size_t route_ws_len = route_ws_bytes(v);
     if (v.ec()) {
-        s = route_scores_impl(v, x, w_router, bias, w.scores, status, st);
+        if (!route_split_impl(v, x, w_router, bias, nullptr, nullptr, nullptr, w.scores, status, route_ws,
+                              route_ws_len, st, &s))
+            s = route_scores_impl(v, x, w_router, bias, w.scores, status, st);
         if (s != MOE_OK) return s;
         s = choose_impl(v, w.scores, x, w.seg_expert, w.seg_offsets, w.src, w.row_w, w.emap, w.xp, st);
         if (s != MOE_OK) return s;
@@ -651,7 +748,9 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
         return cuda_status(launch_ec_combine(w.yp, w.emap, w.row_w, nullptr, v.T, v.E, v.d, v.rows, out, sm_count(),
                                              st));
     }
-    s = route_impl(v, x, w_router, bias, nullptr, w.topk_ids, w.topk_w, status, st);
+    if (!route_split_impl(v, x, w_router, bias, nullptr, w.topk_ids, w.topk_w, nullptr, status, route_ws,
+                          route_ws_len, st, &s))
+        s = route_impl(v, x, w_router, bias, nullptr, w.topk_ids, w.topk_w, status, st);
     if (s != MOE_OK) return s;
     s = dispatch_impl(v, x, w.topk_ids, 0, w.counts, w.seg_expert, w.seg_offsets, w.seg_first_rank, w.dest, w.src,
                       w.xp, status, w.dispatch_ws, w.dispatch_ws_bytes, st);

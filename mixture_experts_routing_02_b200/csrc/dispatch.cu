@@ -761,9 +761,17 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* 
 
 // ------------------------------------------------------------------------------ top-k from given logits
 
-__global__ void __launch_bounds__(256) route_from_logits_kernel(const float* __restrict__ logits, int T, int E,
-                                                                int k, int route_flags, int32_t* __restrict__ ids,
-                                                                float* __restrict__ w) {
+// Routing from fp32 logits, one warp per token (lanes over experts).  The logits of token t are
+// sum_s part[s * split_stride + t * ldp + e] over the n_split parts in order (+ bias[e]): one
+// part is the logits themselves (moe_route_from_logits); several are the partial sums of a
+// router projection whose reduction was split over more CTAs.  Writes the logits (optional),
+// then either the top-k ids and weights or, for expert-choice routing (scores_t non-null), the
+// softmax over all E experts stored expert-major.
+__global__ void __launch_bounds__(256) route_logits_kernel(const float* __restrict__ part, int n_split, int ldp,
+                                                           size_t split_stride, const float* __restrict__ bias, int T,
+                                                           int E, int k, int route_flags, float* __restrict__ logits,
+                                                           int32_t* __restrict__ ids, float* __restrict__ w,
+                                                           float* __restrict__ scores_t) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
@@ -772,8 +780,37 @@ __global__ void __launch_bounds__(256) route_from_logits_kernel(const float* __r
 #pragma unroll
         for (int u = 0; u < kMaxExperts / 32; ++u) {
             const int e = lane + 32 * u;
-            v[u] = e < E ? __ldg(logits + static_cast<size_t>(t) * E + e) : -INFINITY;
-            if (e >= E) taken |= 1u << u;
+            v[u] = -INFINITY;
+            if (e < E) {
+                const float* p = part + static_cast<size_t>(t) * ldp + e;
+                float acc = __ldg(p);
+                for (int sp = 1; sp < n_split; ++sp) acc += __ldg(p + sp * split_stride);
+                if (bias != nullptr) acc += __ldg(bias + e);
+                v[u] = acc;
+                if (logits != nullptr) logits[static_cast<size_t>(t) * E + e] = acc;
+            } else {
+                taken |= 1u << u;
+            }
+        }
+        if (scores_t != nullptr) {
+            float m = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < kMaxExperts / 32; ++u) m = fmaxf(m, v[u]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            float sum = 0.f;
+#pragma unroll
+            for (int u = 0; u < kMaxExperts / 32; ++u)
+                if (lane + 32 * u < E) sum += expf(v[u] - m);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            const float inv = 1.0f / sum;
+#pragma unroll
+            for (int u = 0; u < kMaxExperts / 32; ++u) {
+                const int e = lane + 32 * u;
+                if (e < E) scores_t[static_cast<size_t>(e) * T + t] = expf(v[u] - m) * inv;
+            }
+            continue;
         }
         float sv[kMaxTopK];
         int si[kMaxTopK];
@@ -926,10 +963,18 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
 
 cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int route_flags, int32_t* ids,
                                      float* w, int num_sms, cudaStream_t stream) {
+    return launch_route_logits(logits, 1, E, 0, nullptr, T, E, k, route_flags, nullptr, ids, w, nullptr, num_sms,
+                               stream);
+}
+
+cudaError_t launch_route_logits(const float* part, int n_split, int ldp, size_t split_stride, const float* bias, int T,
+                                int E, int k, int route_flags, float* logits, int32_t* ids, float* w, float* scores_t,
+                                int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     int grid = (T + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
-    route_from_logits_kernel<<<grid, 256, 0, stream>>>(logits, T, E, k, route_flags, ids, w);
+    route_logits_kernel<<<grid, 256, 0, stream>>>(part, n_split, ldp, split_stride, bias, T, E, k, route_flags, logits,
+                                                  ids, w, scores_t);
     return cudaGetLastError();
 }
 

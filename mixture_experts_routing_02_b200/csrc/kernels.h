@@ -37,6 +37,8 @@ struct GemmArgs {
     int k;
     int route_flags;  // MOE_ROUTE_SOFTMAX_ALL: weights from a softmax over all N logits
     float* scores_t;  // route only: non-null = write softmax scores [N, M] (expert-major) instead of top-k
+    int k_splits;          // plain fp32 epilogue only: > 1 cuts the reduction into this many parts
+    size_t split_stride;   // elements between the outputs of consecutive parts
     int32_t* status;
 };
 
@@ -113,6 +115,11 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
 constexpr int kCountMaxPairs = 1 << 16;
 cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int route_flags, int32_t* ids,
                                      float* w, int num_sms, cudaStream_t stream);
+// Routing from n_split partial logit slices (summed in order, + bias): top-k ids and weights, or
+// expert-choice scores (scores_t [E, T]) when scores_t is non-null; logits optional.
+cudaError_t launch_route_logits(const float* part, int n_split, int ldp, size_t split_stride, const float* bias, int T,
+                                int E, int k, int route_flags, float* logits, int32_t* ids, float* w, float* scores_t,
+                                int num_sms, cudaStream_t stream);
 
 // combine.cu
 cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,

@@ -101,7 +101,7 @@ __device__ __forceinline__ void build_tile_prefix(int* prefix, const GemmArgs& g
 // are row-contiguous (whole 128-byte lines per group of lanes), with rows >= row_end masked.
 template <int EPI>
 __device__ __forceinline__ void epilogue_rows(const GemmArgs& g, uint32_t t_row, int row_base, int row_end, int n0,
-                                              int lane, uint32_t* stg) {
+                                              int lane, uint32_t* stg, size_t out_off = 0) {
     if (EPI == kEpiSwiglu) {
         for (int cc = 0; cc < g.BN; cc += 32) {
             uint32_t gr[32], ur[32];
@@ -151,7 +151,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& g, uint32_t t_row,
                     const int grow = row_base + rl;
                     if (grow < row_end) {
                         const uint32_t* src = stg + rl * 33 + q * 4;
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(g.out) +
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(g.out) + out_off +
                                                               static_cast<size_t>(grow) * g.ldo + n0 + cc + q * 4);
                         *dst = make_uint4(src[0], src[1], src[2], src[3]);
                     }
@@ -162,7 +162,10 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& g, uint32_t t_row,
     }
 }
 
-template <int EPI>
+// SPLITK: the reduction is cut into g.k_splits equal parts, each a work unit of its own, and
+// part s of a tile is stored (plain fp32 epilogue) at out + s * split_stride; the caller sums
+// the parts.  Used for the router projection, whose T/128 row tiles are too few for the SMs.
+template <int EPI, bool SPLITK>
 __global__ void __launch_bounds__(kThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
@@ -209,7 +212,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     const uint32_t tmem_base = tmem_base_sh;
-    const int total = tile_prefix[g.n_seg] * g.n_tiles_n;
+    static_assert(!SPLITK || EPI == kEpiStore, "split reductions use the plain fp32 epilogue");
+    const int n_split = SPLITK ? g.k_splits : 1;
+    const int total = tile_prefix[g.n_seg] * g.n_tiles_n * n_split;
     const int nkb = g.K / kBK;
 
     if (warp == 0) {
@@ -220,9 +225,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tx = kABytes + (EPI == kEpiRoute ? static_cast<uint32_t>(g.N) * 128u : b_stage_bytes);
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g);
+                const int split = SPLITK ? tile % n_split : 0;
+                const TileCoord c = decode_tile(SPLITK ? tile / n_split : tile, tile_prefix, g.n_seg, g.n_tiles_n, g);
                 const int n0 = c.n * g.BN;
-                for (int kb = 0; kb < nkb; ++kb) {
+                const int kb0 = SPLITK ? split * nkb / n_split : 0;
+                const int kb1 = SPLITK ? (split + 1) * nkb / n_split : nkb;
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, g.status)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full_bar[stage], tx);
                     uint8_t* a_dst = sA + stage * kABytes;
@@ -259,7 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_sh, g.status)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kAccStride;
-                for (int kb = 0; kb < nkb; ++kb) {
+                const int split = SPLITK ? tile % n_split : 0;
+                const int kb0 = SPLITK ? split * nkb / n_split : 0;
+                const int kb1 = SPLITK ? (split + 1) * nkb / n_split : nkb;
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, &abort_sh, g.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * kABytes));
@@ -267,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                         // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4)
-                        umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
                     }
                     umma_commit(&empty_bar[stage]);
                     if (++stage == stages) { stage = 0; phase ^= 1u; }
@@ -289,7 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g);
+            const TileCoord c = decode_tile(SPLITK ? tile / n_split : tile, tile_prefix, g.n_seg, g.n_tiles_n, g);
+            const size_t out_off = SPLITK ? static_cast<size_t>(tile % n_split) * g.split_stride : 0;
             const bool got = mbar_wait(&tfull_bar[acc], acc_phase, &abort_sh, g.status);
             if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
@@ -301,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             if (EPI == kEpiSwiglu || EPI == kEpiStore) {
                 epilogue_rows<EPI>(g, t_row, c.row0 + quarter * 32, c.row_end, n0, lane,
-                                   epi_stage + (warp - 2) * kStageWords);
+                                   epi_stage + (warp - 2) * kStageWords, out_off);
             } else if (g.scores_t != nullptr) {
                 // expert choice: softmax over the E logits of this row, stored expert-major so
                 // that the 32 lanes (consecutive rows) of a warp write 128 contiguous bytes
@@ -599,10 +611,10 @@ int gemm_pick_stages(int mma_n) {
     return s;
 }
 
-template <int EPI>
+template <int EPI, bool SPLITK>
 static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmArgs& g,
                               int grid, cudaStream_t stream) {
-    auto kern = umma_gemm_kernel<EPI>;
+    auto kern = umma_gemm_kernel<EPI, SPLITK>;
     size_t smem = gemm_smem_bytes(g.stages, g.mma_n);
     if (smem < kGemmSmemMin) smem = kGemmSmemMin;  // keeps one CTA per SM (all TMEM columns are taken)
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -658,9 +670,11 @@ cudaError_t launch_umma_gemm_pair(int epi, const CUtensorMap& a, const CUtensorM
 cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                              const GemmArgs& g, int grid, cudaStream_t stream) {
     switch (epi) {
-        case kEpiRoute: return launch_one<kEpiRoute>(a, b0, b1, g, grid, stream);
-        case kEpiSwiglu: return launch_one<kEpiSwiglu>(a, b0, b1, g, grid, stream);
-        default: return launch_one<kEpiStore>(a, b0, b1, g, grid, stream);
+        case kEpiRoute: return launch_one<kEpiRoute, false>(a, b0, b1, g, grid, stream);
+        case kEpiSwiglu: return launch_one<kEpiSwiglu, false>(a, b0, b1, g, grid, stream);
+        default:
+            return g.k_splits > 1 ? launch_one<kEpiStore, true>(a, b0, b1, g, grid, stream)
+                                  : launch_one<kEpiStore, false>(a, b0, b1, g, grid, stream);
     }
 }
 

@@ -112,6 +112,53 @@ def test_route_logits_and_bias(E, flags):
     assert st.item() == 0
 
 
+@pytest.mark.parametrize("E,flags", [(8, 0), (60, 1), (256, 0)])
+def test_route_split_reduction(E, flags):
+    """moe_route_ws: the router projection's reduction split over more CTAs (partial logits in
+    the workspace, summed in order by a second kernel) gives the oracle's routing."""
+    w = syn.Workload("route-split", T=900, d=1024, E=E, k=min(6, E), F=64, zipf_s=1.2)
+    case = make_case(w, seed=3)
+    s = moe_shape(w)
+    s.route_flags = flags
+    n = moe.moe_route_workspace_size(s)
+    assert n > 0, "this shape should split the reduction"
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    logits = torch.empty(w.T, w.E, device="cuda")
+    ids = i32(w.T * w.k).view(w.T, w.k)
+    wt = torch.empty(w.T, w.k, device="cuda")
+    st = i32(1)
+    moe.moe_route_ws(s, dev(case.x), dev(case.w_r), dev(case.bias), logits, ids, wt, st, ws)
+    torch.cuda.synchronize()
+    l64, rid, rw = oracle.route(case.x, case.w_r, case.bias, w.k, softmax_all=bool(flags))
+    check_close(to_np(logits), l64, "logits", max_abs_of_rms=1e-4, mean_rel=1e-5)
+    assert (ids.cpu().numpy() == rid).all()
+    assert np.abs(wt.cpu().numpy() - rw).max() < 1e-4
+    assert st.item() == 0
+    # without a workspace the same call runs the single-pass kernel
+    ids2 = i32(w.T * w.k).view(w.T, w.k)
+    moe.moe_route_ws(s, dev(case.x), dev(case.w_r), dev(case.bias), None, ids2, wt, st, None)
+    torch.cuda.synchronize()
+    assert torch.equal(ids2, ids)
+
+
+def test_route_scores_split_reduction():
+    """moe_route_scores_ws (expert choice) with the split reduction against the oracle's scores."""
+    w = syn.Workload("ec-split", T=700, d=768, E=16, k=2, F=64, capacity_factor=1.0, expert_choice=True)
+    case = make_case(w, seed=4)
+    s = moe_shape(w)
+    n = moe.moe_route_workspace_size(s)
+    assert n > 0
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    scores = torch.empty(w.E, w.T, device="cuda")
+    st = i32(1)
+    moe.moe_route_scores_ws(s, dev(case.x), dev(case.w_r), dev(case.bias), scores, st, ws)
+    torch.cuda.synchronize()
+    ref = oracle.expert_scores(oracle.router_logits(case.x, case.w_r, case.bias))
+    got = scores.cpu().numpy().T
+    assert (np.abs(got - ref) <= 1e-4 * ref + 1e-9).all()
+    assert st.item() == 0
+
+
 @pytest.mark.parametrize("flags", [0, 1])
 def test_route_from_logits_ties_and_exact_decision(flags):
     T, E, k = 97, 37, 6
