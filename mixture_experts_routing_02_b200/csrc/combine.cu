@@ -87,7 +87,7 @@ cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w,
     else if (k <= 4)
         combine_kernel<4, 2><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
     else
-        combine_kernel<kMaxTopK, 1><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
+        combine_kernel<kMaxTopK, 2><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
     return cudaGetLastError();
 }
 

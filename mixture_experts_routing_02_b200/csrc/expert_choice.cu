@@ -21,6 +21,7 @@ namespace moe {
 namespace {
 
 constexpr int kSelectWarps = kSelectThreads / 32;
+constexpr int kSelectSmemKeys = 48 * 1024;  // 192 KB of keys: up to 49152 tokens per expert column
 static_assert(kSelectWarps == 32, "the warp-total scan below uses one lane per warp");
 
 // Order-preserving map of fp32 bits to uint32: larger float -> larger key.
@@ -57,6 +58,12 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
     return r;
 }
 
+// Inverse of order_key.
+__device__ __forceinline__ uint32_t key_bits(uint32_t k) { return (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k; }
+
+// SMEM: the expert's T keys are loaded once into dynamic shared memory (T <= kSelectSmemKeys)
+// and every pass reads them there; otherwise every pass reads the scores from global memory.
+template <bool SMEM>
 __global__ void __launch_bounds__(kSelectThreads, 1)
     ec_select_kernel(const float* __restrict__ scores_t, int T, int E, int cp, int32_t* __restrict__ seg_expert,
                      int32_t* __restrict__ seg_offsets, int32_t* __restrict__ src, float* __restrict__ row_w,
@@ -64,10 +71,16 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
     __shared__ uint32_t hist[2048];
     __shared__ uint32_t warp_sums[kSelectWarps + 1];
     __shared__ uint32_t sel[2];
+    extern __shared__ uint32_t skeys[];
     const int e = blockIdx.x;
     const int tid = threadIdx.x;
     if (tid == 0) { sel[0] = 0; sel[1] = 1; }
     const uint32_t* col = reinterpret_cast<const uint32_t*>(scores_t) + static_cast<size_t>(e) * T;
+    if (SMEM) {
+        for (int t = tid; t < T; t += kSelectThreads) skeys[t] = order_key(__ldg(col + t));
+        __syncthreads();
+    }
+    auto key_at = [&](int t) -> uint32_t { return SMEM ? skeys[t] : order_key(__ldg(col + t)); };
     if (tid == 0) {
         seg_expert[e] = e;
         seg_offsets[e] = e * cp;
@@ -83,7 +96,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
         for (int i = tid; i < nb; i += kSelectThreads) hist[i] = 0;
         __syncthreads();
         for (int t = tid; t < T; t += kSelectThreads) {
-            const uint32_t k = order_key(__ldg(col + t));
+            const uint32_t k = key_at(t);
             if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & static_cast<uint32_t>(nb - 1)], 1u);
         }
         __syncthreads();
@@ -124,8 +137,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
         uint32_t raw = 0;
         bool gt = false, eq = false;
         if (t < T) {
-            raw = __ldg(col + t);
-            const uint32_t k = order_key(raw);
+            const uint32_t k = key_at(t);
+            raw = key_bits(k);
             gt = k > prefix;
             eq = k == prefix;
         }
@@ -257,7 +270,20 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 cudaError_t launch_ec_select(const float* scores_t, int T, int E, int cp, int32_t* seg_expert, int32_t* seg_offsets,
                              int32_t* src, float* row_w, int32_t* emap, cudaStream_t stream) {
     if (T == 0 || E == 0) return cudaSuccess;
-    ec_select_kernel<<<E, kSelectThreads, 0, stream>>>(scores_t, T, E, cp, seg_expert, seg_offsets, src, row_w, emap);
+    if (T <= kSelectSmemKeys) {
+        const size_t smem = static_cast<size_t>(T) * sizeof(uint32_t);
+        if (smem > 48 * 1024) {
+            const cudaError_t err = cudaFuncSetAttribute(ec_select_kernel<true>,
+                                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                         static_cast<int>(kSelectSmemKeys * sizeof(uint32_t)));
+            if (err != cudaSuccess) return err;
+        }
+        ec_select_kernel<true><<<E, kSelectThreads, smem, stream>>>(scores_t, T, E, cp, seg_expert, seg_offsets, src,
+                                                                    row_w, emap);
+    } else {
+        ec_select_kernel<false><<<E, kSelectThreads, 0, stream>>>(scores_t, T, E, cp, seg_expert, seg_offsets, src,
+                                                                  row_w, emap);
+    }
     return cudaGetLastError();
 }
 

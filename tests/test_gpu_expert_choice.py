@@ -96,10 +96,13 @@ def test_expert_choice_layer_matches_oracle(cuda_ok, w):
         check_close(to_np(got["out"])[kept], out[kept], "out")
 
 
-def test_selection_with_many_equal_scores(cuda_ok):
+@pytest.mark.parametrize("T,E,C", [(3000, 5, 700), (50000, 3, 9000)])
+def test_selection_with_many_equal_scores(cuda_ok, T, E, C):
     """Scores on a coarse grid (many equal values at every threshold) and of both signs:
-    equal scores go to the lower token id; the whole selection is bit-exact."""
-    T, E, C, d = 3000, 5, 700, 64
+    equal scores go to the lower token id; the whole selection is bit-exact.  The larger case
+    has more tokens than the selection keeps in shared memory (it reads the scores from global
+    memory in every pass)."""
+    d = 64
     rng = np.random.default_rng(7)
     S = (rng.integers(-3, 6, size=(T, E)) / 8.0).astype(np.float32)
     x = torch.randn(T, d, generator=torch.Generator().manual_seed(8)).to(torch.bfloat16)
