@@ -35,6 +35,7 @@ if ROOT not in sys.path:
 
 METRIC = "MoE layer fwd tokens/s; grouped-GEMM TFLOPS and permute GB/s vs roofline"
 FLUSH_BYTES = 256 << 20
+E2E_MIN_STEPS = 64
 KERNELS = ("route", "dispatch", "gate_up", "down", "combine")
 
 
@@ -389,6 +390,10 @@ def run_ours(args, w):
     host_x = [x_host, x_cpu.clone().pin_memory()]
     host_out = [out_host, torch.empty_like(out_host).pin_memory()]
 
+    # the pipelined run's fill (first upload) and drain (last download) are paid once, so the
+    # end-to-end rate is taken over at least E2E_MIN_STEPS steps
+    e2e_steps = max(args.steps, E2E_MIN_STEPS)
+
     def e2e_run(n_steps):
         ev_in = [torch.cuda.Event() for _ in range(n_steps)]
         ev_cmp = [torch.cuda.Event() for _ in range(n_steps)]
@@ -451,7 +456,7 @@ def run_ours(args, w):
     # end to end through moe_layer_fwd with host buffers (pipelined steps; the weights, 2.8 GB and
     # more, stream through L2 every step, so no extra flush)
     barrier()
-    t0, t1 = e2e_run(args.steps)
+    t0, t1 = e2e_run(e2e_steps)
     barrier()
     e2e_ms = t0.elapsed_time(t1)
     if status.item() != 0:
@@ -515,7 +520,8 @@ def run_ours(args, w):
         "roofline": roof,
         "breakdown": {n: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in b.items()}
                       for n, b in breakdown.items()},
-        "e2e": {"value": job_throughput(T, args.steps, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
+        "e2e": {"value": job_throughput(T, e2e_steps, world, e2e_ms), "unit": "tokens/s", "steps": e2e_steps,
+                "h2d_bytes_per_step": T * d * 2,
                 "d2h_bytes_per_step": T * d * 4, "api": "moe_layer_fwd; per step X (bf16) copied in from pinned host memory and out (fp32) copied back; steps pipelined over copy-in / compute / copy-out streams with double-buffered device buffers"},
         "clocks": clocks.summary(),
     }

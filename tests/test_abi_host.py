@@ -160,3 +160,23 @@ def test_expert_choice_calls_check_the_flag(lib):
     assert lib.moe_combine_expert_choice(ctypes.byref(s), fake, fake, fake, None, fake, None) == 1
     assert lib.moe_dispatch(ctypes.byref(ec), fake, fake, 0, *([fake] * 9), 1 << 30, None) == 1
     assert lib.moe_expert_choose(ctypes.byref(ec), None, *([fake] * 7), None) == 1   # null scores
+
+
+def test_route_workspace_size(lib):
+    """The router's reduction is split only when its ceil(T/128) row tiles leave SMs idle and d
+    gives each part at least 4 k-blocks; a split needs S * T * 32*ceil(E/32) fp32 partials."""
+    assert moe.moe_route_workspace_size(_shape()) == 0                     # d = 128: too short to split
+    w = syn.MIXTRAL_LIKE
+    n = moe.moe_route_workspace_size(moe.shape(w.T, w.d, w.E, w.k, w.F))
+    assert n >= 2 * w.T * 32 * 4 and n % 256 == 0
+    b = syn.BALANCED                                                          # 256 row tiles: no split
+    assert moe.moe_route_workspace_size(moe.shape(b.T, b.d, b.E, b.k, b.F, n_groups=b.n_groups,
+                                                  replica_slots=b.replica_slots)) == 0
+
+
+def test_route_ws_checks_before_cuda(lib):
+    fake = ctypes.c_void_p(1 << 20)
+    ec = _shape(route_flags=moe.ROUTE_EXPERT_CHOICE, capacity=16)
+    assert lib.moe_route_ws(ctypes.byref(ec), fake, fake, None, None, fake, fake, None, None, 0, None) == 1
+    assert lib.moe_route_scores_ws(ctypes.byref(_shape()), fake, fake, None, fake, None, None, 0, None) == 1
+    assert lib.moe_route_ws(ctypes.byref(_shape()), None, fake, None, None, fake, fake, None, None, 0, None) == 1
