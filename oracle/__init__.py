@@ -11,4 +11,5 @@ from .moe_oracle import (  # noqa: F401
     plain_segments, route, router_logits, shared_expert, silu, token_output, topk_ids, topk_weights,
     topk_weights_softmax_all, ExpertChoice, expert_choice, expert_choice_forward, expert_scores,
     select_tokens, ec_margin_violations, enforce_ec_margin, combine_expert_choice, expert_choice_map,
+    Rerouted, candidate_order, reroute_overflow, reroute_positions, layer_forward_reroute,
 )

@@ -614,3 +614,104 @@ def enforce_ec_margin(x, w_router, bias, capacity: int, redraw, min_rel_gap: flo
         x[t] = row
         logits[t] = f64(row) @ w64.T + b64
         n += 1
+
+
+# ----------------------------------------------------------------------------
+# overflow re-routing   [MoE-impl] "로드 밸런싱 손실(load-balancing loss)과 용량(capacity)은
+# 별개": a pair over its expert's capacity may go to another candidate instead of being dropped
+# ----------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class Rerouted:
+    expert: np.ndarray   # [T*k] final expert of each pair (-1: dropped for good)
+    slot: np.ndarray     # [T*k] row of the pair inside its expert's segment
+    round: np.ndarray    # [T*k] round in which the pair was placed (0: its own top-k expert)
+    assigned: np.ndarray  # [E] rows of each expert (<= C)
+
+
+def candidate_order(logits32_row: np.ndarray) -> List[int]:
+    """A token's experts by logit, descending; equal logits: the lower id first."""
+    return sorted(range(len(logits32_row)), key=lambda e: (-float(logits32_row[e]), e))
+
+
+def reroute_overflow(ids: np.ndarray, logits64: np.ndarray, C: int) -> Rerouted:
+    """Round 0: each expert keeps its first C pairs in q = t*k + j order (the capacity rule).
+    Round r >= 1: every pair still unplaced proposes to its token's next candidate (in the
+    token's logit order below its top-k, compared in fp32) among the experts that had room when
+    the round began; a token's unplaced pairs take consecutive candidates in j order.  Each
+    expert accepts the round's proposals in q order while it has room.  A pair with no
+    candidate left is dropped.  Rows of a segment: round 0 pairs, then round 1, ... (q order
+    inside a round)."""
+    ids = i64(ids)
+    T, k = ids.shape
+    E = logits64.shape[1]
+    l32 = np.asarray(logits64, dtype=np.float64).astype(np.float32)
+    expert = np.full(T * k, -1, dtype=np.int64)
+    slot = np.full(T * k, -1, dtype=np.int64)
+    rnd = np.full(T * k, -1, dtype=np.int64)
+    assigned = np.zeros(E, dtype=np.int64)
+    pending = []
+    for q in range(T * k):
+        e = int(ids.ravel()[q])
+        if assigned[e] < C:
+            expert[q], slot[q], rnd[q] = e, assigned[e], 0
+            assigned[e] += 1
+        else:
+            pending.append(q)
+    order = {}      # token -> its candidates below the top-k, in logit order
+    cursor = {}     # token -> next position in that list
+    r = 0
+    while pending:
+        r += 1
+        open_ = assigned < C
+        if not open_.any():
+            break
+        proposals = []
+        for q in pending:
+            t = q // k
+            if t not in order:
+                held = set(int(e) for e in ids[t])
+                order[t] = [e for e in candidate_order(l32[t]) if e not in held]
+                cursor[t] = 0
+            lst = order[t]
+            while cursor[t] < len(lst) and not open_[lst[cursor[t]]]:
+                cursor[t] += 1
+            if cursor[t] < len(lst):
+                proposals.append((q, lst[cursor[t]]))
+                cursor[t] += 1
+        room = C - assigned
+        taken = np.zeros(E, dtype=np.int64)
+        still = []
+        for q, e in proposals:
+            if taken[e] < room[e]:
+                expert[q], slot[q], rnd[q] = e, assigned[e] + taken[e], r
+                taken[e] += 1
+            else:
+                still.append(q)
+        assigned += taken
+        pending = still
+    return Rerouted(expert, slot, rnd, assigned)
+
+
+def reroute_positions(rr: Rerouted):
+    """dest[q] and src[row] of the re-routed layout (one segment per expert)."""
+    segs = Segments(expert=np.arange(len(rr.assigned), dtype=np.int64), length=rr.assigned.copy(),
+                    first_rank=np.zeros(len(rr.assigned), dtype=np.int64))
+    off = segs.offsets
+    dest = np.where(rr.expert >= 0, off[np.maximum(rr.expert, 0)] + rr.slot, -1).astype(np.int64)
+    src = np.full(int(off[-1]), -1, dtype=np.int64)
+    for q in np.nonzero(dest >= 0)[0]:
+        src[dest[q]] = q
+    return segs, dest, src
+
+
+def layer_forward_reroute(x, w_router, bias, w_gate, w_up, w_down, k: int, capacity: int):
+    """The layer with overflow re-routing: a moved pair keeps its routing weight."""
+    T = x.shape[0]
+    logits, ids, w = route(x, w_router, bias, k)
+    rr = reroute_overflow(ids, logits, capacity)
+    segs, dest, src = reroute_positions(rr)
+    xp = permute_rows(x, src, k)
+    hp, yp = grouped_expert_ffn(xp, segs, w_gate, w_up, w_down)
+    out = combine(yp, dest, w, T, k)
+    return logits, ids, w, rr, segs, dest, src, xp, hp, yp, out

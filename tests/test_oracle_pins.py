@@ -201,6 +201,65 @@ def pin_expert_choice_layer_eager(seed=21):
     return bool(np.allclose(out, want, rtol=1e-11, atol=1e-13))
 
 
+def pin_reroute_worked_example():
+    """Hand-worked: C = 1, k = 1, E = 3; tokens 0-2 rank the experts 0 > 1 > 2, token 3 ranks
+    0 > 2 > 1; everyone picks expert 0.  Round 0: token 0 keeps expert 0.  Round 1 (experts 1, 2
+    open): tokens 1 and 2 propose 1, token 3 proposes 2; expert 1 takes token 1 (q order).
+    Round 2: no expert has room, token 2 is dropped."""
+    l = np.array([[3, 2, 1], [3, 2, 1], [3, 2, 1], [3, 1, 2]], dtype=np.float64)
+    rr = oracle.reroute_overflow(np.zeros((4, 1), dtype=np.int64), l, 1)
+    return (list(rr.expert) == [0, 1, -1, 2] and list(rr.slot) == [0, 0, -1, 0] and list(rr.round) == [0, 1, -1, 1]
+            and list(rr.assigned) == [1, 1, 1])
+
+
+def pin_reroute_without_overflow(seed=30):
+    """With room for every pair the re-routing is the plain top-k dispatch (library argsort ranks)."""
+    rng = np.random.default_rng(seed)
+    T, E, k = 50, 6, 2
+    logits = rng.normal(size=(T, E))
+    ids = oracle.topk_ids(logits, k)
+    rr = oracle.reroute_overflow(ids, logits, T * k)
+    flat = ids.ravel()
+    rank = np.empty(T * k, dtype=np.int64)
+    for e in range(E):
+        qs = np.nonzero(flat == e)[0]                 # ascending q: the stable order
+        rank[qs] = np.arange(len(qs))
+    return bool((rr.expert == flat).all() and (rr.slot == rank).all() and (rr.round == 0).all())
+
+
+def pin_reroute_invariants(seed=31):
+    """Random skewed cases: no expert over C; a token never holds an expert twice; a moved pair
+    sits at an expert below the token's top-k, and a token's moved pairs follow its logit order
+    (j order); a pair is dropped only when every expert its token does not hold is full; slots of
+    each expert are 0..assigned-1 with round-major, q-minor order."""
+    rng = np.random.default_rng(seed)
+    ok = True
+    for trial in range(6):
+        T, E, k = 40, 7, 2
+        logits = rng.normal(size=(T, E)) + np.linspace(2, 0, E)[None, :]   # skew toward low ids
+        ids = oracle.topk_ids(logits, k)
+        C = int(rng.integers(2, 9))
+        rr = oracle.reroute_overflow(ids, logits, C)
+        ok &= bool((rr.assigned <= C).all())
+        for t in range(T):
+            fin = [int(e) for e in rr.expert[t * k:(t + 1) * k] if e >= 0]
+            ok &= len(set(fin)) == len(fin)
+            order = [e for e in oracle.candidate_order(logits[t].astype(np.float32)) if e not in ids[t]]
+            moved = [int(rr.expert[t * k + j]) for j in range(k) if rr.round[t * k + j] > 0]
+            ok &= all(e in order for e in moved)
+            ok &= [order.index(e) for e in moved] == sorted(order.index(e) for e in moved)
+            if (rr.expert[t * k:(t + 1) * k] < 0).any():
+                others = [e for e in range(E) if e not in fin]
+                ok &= all(rr.assigned[e] == C for e in others)
+        for e in range(E):
+            qs = np.nonzero(rr.expert == e)[0]
+            ok &= sorted(rr.slot[qs].tolist()) == list(range(len(qs)))
+            keyed = sorted(qs.tolist(), key=lambda q: (rr.round[q], q))
+            ok &= [int(rr.slot[q]) for q in keyed] == list(range(len(qs)))
+        ok &= int((rr.expert >= 0).sum()) == int(rr.assigned.sum())
+    return bool(ok)
+
+
 def pin_silu_library():
     z = np.linspace(-30, 30, 2001)
     ref = torch.nn.functional.silu(torch.from_numpy(z)).numpy()
@@ -374,6 +433,18 @@ def test_expert_choice_capacity_above_tokens():
     assert all(list(p) == [0, 1, 2, 3, 4] for p in ec.picks)
 
 
+def test_reroute_worked_example():
+    assert pin_reroute_worked_example()
+
+
+def test_reroute_without_overflow_is_top_k():
+    assert pin_reroute_without_overflow()
+
+
+def test_reroute_invariants():
+    assert pin_reroute_invariants()
+
+
 def test_shared_expert_adds_a_dense_ffn():
     assert pin_shared_expert_additive()
 
@@ -478,6 +549,22 @@ def _mut_shared_transposed(x, w_gate_s, w_up_s, w_down_s):
     return om.expert_ffn(om.f64(x), w_up_s, w_gate_s, w_down_s)[1]   # gate and up swapped
 
 
+_orig_candidate_order = om.candidate_order
+
+
+def _mut_candidates_ascending(logits32_row):
+    return _orig_candidate_order(-np.asarray(logits32_row))   # worst candidate first
+
+
+_orig_reroute = om.reroute_overflow
+
+
+def _mut_reroute_keeps_full(ids, logits64, C):
+    rr = _orig_reroute(ids, logits64, C)
+    rr.assigned = np.minimum(rr.assigned + 1, C + 1)   # one row too many somewhere
+    return rr
+
+
 _orig_expert_choice = om.expert_choice
 
 
@@ -499,6 +586,8 @@ MUTATIONS = [
     ("expert_scores", lambda l: np.exp(l) / np.exp(l).sum(0, keepdims=True),   # softmax over tokens
      [pin_expert_choice_brute_force, pin_expert_choice_layer_eager]),
     ("expert_choice", _mut_ec_keeps_weakest, [pin_expert_choice_brute_force, pin_expert_choice_layer_eager]),
+    ("candidate_order", _mut_candidates_ascending, [pin_reroute_worked_example, pin_reroute_invariants]),
+    ("reroute_overflow", _mut_reroute_keeps_full, [pin_reroute_worked_example, pin_reroute_invariants]),
 ]
 
 
