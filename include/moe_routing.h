@@ -114,9 +114,26 @@ typedef enum {
  *                  rows_alloc = E * C'.  Takes moe_route_scores,
  *                  moe_expert_choose and moe_combine_expert_choice in place of
  *                  moe_route, moe_dispatch and moe_combine, which reject it.
+ *                  MOE_ROUTE_REROUTE: with a capacity, a pair over its expert's
+ *                  capacity goes to another candidate instead of being dropped
+ *                  ("Sparsely-Gated MoE 구현 관점에서 살펴보기", section "로드 밸런싱
+ *                  손실(load-balancing loss)과 용량(capacity)은 별개").  Round 0 is
+ *                  the capacity rule; in round r >= 1 every unplaced pair
+ *                  proposes to its token's next candidate in logit order (below
+ *                  its top-k; equal logits: lower id) among the experts that had
+ *                  room when the round began, a token's unplaced pairs taking
+ *                  consecutive candidates in j order; each expert accepts the
+ *                  round's proposals in q order while it has room; a pair with
+ *                  no candidate left is dropped.  A moved pair keeps its routing
+ *                  weight.  Segment e holds its rows round by round, q order
+ *                  inside a round.  Requires capacity >= 1, n_groups == 0 and
+ *                  T * k <= 65536; excludes MOE_ROUTE_EXPERT_CHOICE.  Takes
+ *                  moe_dispatch_reroute (which needs the router's fp32 logits) in
+ *                  place of moe_dispatch, which rejects it.
  */
 #define MOE_ROUTE_SOFTMAX_ALL 0x1
 #define MOE_ROUTE_EXPERT_CHOICE 0x2
+#define MOE_ROUTE_REROUTE 0x4
 
 typedef struct {
     int32_t T;
@@ -438,6 +455,22 @@ MOE_API moe_status_t moe_combine_expert_choice(const moe_shape_t *shape, const f
                                        const float *row_w, const float *base, float *out,
                                        moe_stream_t stream);
 
+/*
+ * Dispatch with overflow re-routing (shape.route_flags has MOE_ROUTE_REROUTE):
+ * as moe_dispatch (plan_ready = 0), plus
+ *   logits [T, E] fp32: the router logits that chose topk_ids (moe_route's
+ *          logits output); they order each token's further candidates
+ * counts receives the plain histogram of topk_ids; seg_offsets the rows each
+ * expert ends with (at most C).  ws: moe_workspace_size's dispatch_bytes for
+ * this shape (device, 256-byte aligned; no initialisation needed).  Two
+ * launches: the rounds (one CTA) and the row copies.
+ */
+MOE_API moe_status_t moe_dispatch_reroute(const moe_shape_t *shape, const moe_bf16_t *x, const int32_t *topk_ids,
+                                  const float *logits, int32_t *counts, int32_t *seg_expert,
+                                  int32_t *seg_offsets, int32_t *seg_first_rank, int32_t *dest, int32_t *src,
+                                  moe_bf16_t *xp, int32_t *status, void *ws, size_t ws_bytes,
+                                  moe_stream_t stream);
+
 /* Device addresses of the intermediates moe_layer_fwd keeps in its workspace. */
 typedef struct {
     int32_t *topk_ids;       /* [T, k] */
@@ -456,6 +489,7 @@ typedef struct {
     float *scores;           /* [E, T] expert-choice scores (NULL without the flag) */
     int32_t *emap;           /* [T, E] expert-choice row map (NULL without the flag) */
     float *row_w;            /* [rows_alloc] expert-choice row weights (NULL without the flag) */
+    float *logits;           /* [T, E] router logits (MOE_ROUTE_REROUTE only, else NULL) */
 } moe_layer_views_t;
 
 /* Fill *views with the addresses inside a layer workspace `ws`. Host only. */

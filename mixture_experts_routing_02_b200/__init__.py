@@ -19,9 +19,9 @@ __all__ = [
     "moe_histogram", "moe_segments", "moe_plan_balanced", "moe_dispatch", "moe_dispatch_static", "moe_expert_gate_up",
     "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_combine_add", "moe_shared_expert", "moe_layer_fwd",
     "moe_route_scores", "moe_expert_choose", "moe_combine_expert_choice",
-    "moe_route_workspace_size", "moe_route_ws", "moe_route_scores_ws",
+    "moe_route_workspace_size", "moe_route_ws", "moe_route_scores_ws", "moe_dispatch_reroute",
     "moe_layer_views",
-    "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT", "ROUTE_SOFTMAX_ALL", "ROUTE_EXPERT_CHOICE",
+    "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT", "ROUTE_SOFTMAX_ALL", "ROUTE_EXPERT_CHOICE", "ROUTE_REROUTE",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -44,7 +44,7 @@ class MoeLayerViews(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("topk_ids", "topk_w", "counts", "seg_expert", "seg_offsets", "seg_first_rank", "dest",
                  "src", "xp", "hp", "yp", "dispatch_ws")] + [("dispatch_ws_bytes", ctypes.c_size_t)] + \
-        [(n, ctypes.c_void_p) for n in ("scores", "emap", "row_w")]
+        [(n, ctypes.c_void_p) for n in ("scores", "emap", "row_w", "logits")]
 
 
 _P = ctypes.c_void_p
@@ -78,6 +78,7 @@ SYMBOLS = {
     "moe_route_workspace_size": [_S, _P],
     "moe_route_ws": [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_route_scores_ws": [_S, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "moe_dispatch_reroute": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
 }
 
 _lib = None
@@ -102,6 +103,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 ROUTE_SOFTMAX_ALL = 0x1
 ROUTE_EXPERT_CHOICE = 0x2
+ROUTE_REROUTE = 0x4
 
 
 def shape(T, d_model, n_experts, top_k, d_ff, capacity=0, n_groups=0, replica_slots=0, route_flags=0) -> MoeShape:
@@ -279,3 +281,10 @@ def moe_route_scores_ws(s, x, w_router, bias, scores, status=None, ws=None, stre
     _check("moe_route_scores_ws", load_library().moe_route_scores_ws(
         ctypes.byref(s), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(scores), _ptr(status), _ptr(ws), _nbytes(ws),
         _stream(stream)))
+
+
+def moe_dispatch_reroute(s, x, topk_ids, logits, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp,
+                         status=None, ws=None, stream=None):
+    _check("moe_dispatch_reroute", load_library().moe_dispatch_reroute(
+        ctypes.byref(s), _ptr(x), _ptr(topk_ids), _ptr(logits), _ptr(counts), _ptr(seg_expert), _ptr(seg_offsets),
+        _ptr(seg_first_rank), _ptr(dest), _ptr(src), _ptr(xp), _ptr(status), _ptr(ws), _nbytes(ws), _stream(stream)))

@@ -48,6 +48,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Dims {
     int T, d, E, k, F, C, R, B, S, flags;
     bool ec() const { return (flags & MOE_ROUTE_EXPERT_CHOICE) != 0; }
+    bool rr() const { return (flags & MOE_ROUTE_REROUTE) != 0; }
     int cp() const { return ec() ? std::min(C, T) : 0; }  // expert choice: rows per expert
     int n_seg;
     int rows;  // rows_alloc
@@ -58,9 +59,11 @@ moe_status_t check_shape(const moe_shape_t* s, Dims* out) {
     Dims v;
     v.T = s->T; v.d = s->d_model; v.E = s->n_experts; v.k = s->top_k; v.F = s->d_ff;
     v.C = s->capacity; v.R = s->n_groups; v.B = s->replica_slots; v.flags = s->route_flags;
-    if (v.flags & ~(MOE_ROUTE_SOFTMAX_ALL | MOE_ROUTE_EXPERT_CHOICE)) return MOE_ERR_INVALID_ARG;
+    if (v.flags & ~(MOE_ROUTE_SOFTMAX_ALL | MOE_ROUTE_EXPERT_CHOICE | MOE_ROUTE_REROUTE)) return MOE_ERR_INVALID_ARG;
     const bool ec = (v.flags & MOE_ROUTE_EXPERT_CHOICE) != 0;
     if (ec && ((v.flags & MOE_ROUTE_SOFTMAX_ALL) || s->capacity < 1 || s->n_groups != 0)) return MOE_ERR_INVALID_ARG;
+    const bool rr = (v.flags & MOE_ROUTE_REROUTE) != 0;
+    if (rr && (ec || s->capacity < 1 || s->n_groups != 0)) return MOE_ERR_INVALID_ARG;
     if (v.T < 0 || v.d < 1 || v.E < 1 || v.k < 1 || v.k > v.E || v.F < 1 || v.C < 0 || v.R < 0 || v.B < 0)
         return MOE_ERR_INVALID_ARG;
     if (v.R > 0 && (v.E % v.R != 0 || v.T % v.R != 0 || v.C > 0)) return MOE_ERR_INVALID_ARG;
@@ -72,6 +75,7 @@ moe_status_t check_shape(const moe_shape_t* s, Dims* out) {
     v.S = v.R > 0 ? v.T / v.R : v.T;
     int64_t rows = static_cast<int64_t>(v.T) * v.k;
     if (v.C > 0) rows = std::min<int64_t>(rows, static_cast<int64_t>(v.C) * v.E);
+    if (rr && static_cast<int64_t>(v.T) * v.k > kCountMaxPairs) return MOE_ERR_UNSUPPORTED;
     if (ec) {
         // segment e holds expert e's C' = min(C, T) chosen tokens
         rows = static_cast<int64_t>(std::min(v.C, v.T)) * v.E;
@@ -296,6 +300,23 @@ moe_status_t segments_or_plan(const Dims& v, int32_t* counts, const int32_t* par
         launch_segments(counts, partials, n_partials, v.E, v.C, seg_expert, seg_offsets, seg_first_rank, st));
 }
 
+moe_status_t reroute_impl(const Dims& v, const moe_bf16_t* x, const int32_t* ids, const float* logits,
+                          int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank,
+                          int32_t* dest, int32_t* src, moe_bf16_t* xp, void* ws, size_t ws_bytes, cudaStream_t st) {
+    if (!x || !ids || !logits || !counts || !seg_expert || !seg_offsets || !seg_first_rank || !dest || !src || !xp)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+    if (ws == nullptr || ws_bytes < reroute_ws_bytes(v.T, v.k) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return MOE_ERR_WORKSPACE;
+    RerouteArgs a{};
+    a.ids = ids; a.logits = logits;
+    a.T = v.T; a.k = v.k; a.E = v.E; a.capacity = v.C; a.rows = v.rows;
+    a.counts = counts; a.seg_expert = seg_expert; a.seg_offsets = seg_offsets; a.seg_first_rank = seg_first_rank;
+    a.dest = dest; a.src = src;
+    return cuda_status(launch_reroute(a, ws, reinterpret_cast<const __nv_bfloat16*>(x),
+                                      reinterpret_cast<__nv_bfloat16*>(xp), v.d, sm_count(), st));
+}
+
 moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* ids, int32_t plan_ready,
                            int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank,
                            int32_t* dest, int32_t* src, moe_bf16_t* xp, int32_t* status, void* ws,
@@ -367,7 +388,7 @@ void* static_scratch_address() {
 
 struct LayerLayout {
     size_t ids, w, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, dispatch_ws, xp, hp, yp, scores, emap,
-        row_w, route_ws, total;
+        row_w, route_ws, logits, total;
     size_t dispatch_ws_bytes;
 };
 
@@ -385,7 +406,7 @@ LayerLayout layer_layout(const Dims& v) {
     L.seg_first_rank = o; o = align256(o + static_cast<size_t>(v.n_seg) * 4);
     L.dest = o; o = align256(o + tk * 4);
     L.src = o; o = align256(o + static_cast<size_t>(v.rows) * 4);
-    L.dispatch_ws_bytes = v.ec() ? 0 : permute_ws_bytes(v.T, v.k, v.E);
+    L.dispatch_ws_bytes = v.ec() ? 0 : (v.rr() ? reroute_ws_bytes(v.T, v.k) : permute_ws_bytes(v.T, v.k, v.E));
     L.dispatch_ws = o; o = align256(o + L.dispatch_ws_bytes);
     L.xp = o; o = align256(o + static_cast<size_t>(v.rows) * v.d * 2);
     L.hp = o; o = align256(o + static_cast<size_t>(v.rows) * v.F * 2);
@@ -394,6 +415,7 @@ LayerLayout layer_layout(const Dims& v) {
     L.emap = o; o = align256(o + te * 4);
     L.row_w = o; o = align256(o + (v.ec() ? static_cast<size_t>(v.rows) * 4 : 0));
     L.route_ws = o; o = align256(o + route_ws_bytes(v));
+    L.logits = o; o = align256(o + (v.rr() ? static_cast<size_t>(v.T) * v.E * 4 : 0));
     L.total = o;
     return L;
 }
@@ -426,7 +448,8 @@ moe_status_t moe_workspace_size(const moe_shape_t* shape, size_t* dispatch_bytes
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
-    if (dispatch_bytes) *dispatch_bytes = v.ec() ? 0 : permute_ws_bytes(v.T, v.k, v.E);
+    if (dispatch_bytes)
+        *dispatch_bytes = v.ec() ? 0 : (v.rr() ? reroute_ws_bytes(v.T, v.k) : permute_ws_bytes(v.T, v.k, v.E));
     if (layer_bytes) *layer_bytes = layer_layout(v).total;
     return MOE_OK;
 }
@@ -504,6 +527,7 @@ moe_status_t moe_segments(const moe_shape_t* shape, const int32_t* counts, int32
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
+    if (v.rr()) return MOE_ERR_INVALID_ARG;  // re-routing has its own dispatch call
     if (v.R > 0 || !counts || !seg_expert || !seg_offsets || !seg_first_rank) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_segments(const_cast<int32_t*>(counts), nullptr, 0, v.E, v.C, seg_expert, seg_offsets,
                                        seg_first_rank, static_cast<cudaStream_t>(stream)));
@@ -515,6 +539,7 @@ moe_status_t moe_plan_balanced(const moe_shape_t* shape, const int32_t* counts, 
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
+    if (v.rr()) return MOE_ERR_INVALID_ARG;  // re-routing has its own dispatch call
     if (v.R == 0 || !counts || !seg_expert || !seg_offsets || !seg_first_rank) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_plan(const_cast<int32_t*>(counts), nullptr, 0, v.E, v.R, v.S, v.k, v.B, seg_expert,
                                    seg_offsets, seg_first_rank, status, static_cast<cudaStream_t>(stream)));
@@ -528,6 +553,7 @@ moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const i
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
+    if (v.rr()) return MOE_ERR_INVALID_ARG;  // re-routing has its own dispatch call
     return dispatch_impl(v, x, topk_ids, plan_ready, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp,
                          status, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
@@ -540,11 +566,25 @@ moe_status_t moe_dispatch_static(const moe_shape_t* shape, const moe_bf16_t* x, 
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
+    if (v.rr()) return MOE_ERR_INVALID_ARG;  // re-routing has its own dispatch call
     if (permute_ws_bytes(v.T, v.k, v.E) > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED;
     void* scratch = static_scratch_address();
     if (scratch == nullptr) return MOE_ERR_CUDA;
     return dispatch_impl(v, x, topk_ids, plan_ready, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp,
                          status, scratch, kStaticScratchBytes, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_dispatch_reroute(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_ids,
+                                  const float* logits, int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets,
+                                  int32_t* seg_first_rank, int32_t* dest, int32_t* src, moe_bf16_t* xp,
+                                  int32_t* status, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    (void)status;
+    if (!v.rr()) return MOE_ERR_INVALID_ARG;
+    return reroute_impl(v, x, topk_ids, logits, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp, ws,
+                        ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* xp, const int32_t* seg_expert,
@@ -598,6 +638,7 @@ moe_status_t moe_testing_dispatch_stalled(const moe_shape_t* shape, const moe_bf
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
+    if (v.rr()) return MOE_ERR_INVALID_ARG;  // re-routing has its own dispatch call
     if (permute_n_tiles(v.T, v.k) < 2) return MOE_ERR_INVALID_ARG;  // needs a tile that waits on tile 0
     return dispatch_impl(v, x, topk_ids, 0, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp, status,
                          ws, ws_bytes, static_cast<cudaStream_t>(stream), 1);
@@ -715,6 +756,7 @@ moe_status_t moe_layer_views(const moe_shape_t* shape, void* ws, moe_layer_views
     views->scores = v.ec() ? reinterpret_cast<float*>(b + L.scores) : nullptr;
     views->emap = v.ec() ? reinterpret_cast<int32_t*>(b + L.emap) : nullptr;
     views->row_w = v.ec() ? reinterpret_cast<float*>(b + L.row_w) : nullptr;
+    views->logits = v.rr() ? reinterpret_cast<float*>(b + L.logits) : nullptr;
     return MOE_OK;
 }
 
@@ -748,10 +790,20 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
         return cuda_status(launch_ec_combine(w.yp, w.emap, w.row_w, nullptr, v.T, v.E, v.d, v.rows, out, sm_count(),
                                              st));
     }
-    if (!route_split_impl(v, x, w_router, bias, nullptr, w.topk_ids, w.topk_w, nullptr, status, route_ws,
+    if (!route_split_impl(v, x, w_router, bias, w.logits, w.topk_ids, w.topk_w, nullptr, status, route_ws,
                           route_ws_len, st, &s))
-        s = route_impl(v, x, w_router, bias, nullptr, w.topk_ids, w.topk_w, status, st);
+        s = route_impl(v, x, w_router, bias, w.logits, w.topk_ids, w.topk_w, status, st);
     if (s != MOE_OK) return s;
+    if (v.rr()) {
+        s = reroute_impl(v, x, w.topk_ids, w.logits, w.counts, w.seg_expert, w.seg_offsets, w.seg_first_rank, w.dest,
+                         w.src, w.xp, w.dispatch_ws, w.dispatch_ws_bytes, st);
+        if (s != MOE_OK) return s;
+        s = gate_up_impl(v, w.xp, w.seg_expert, w.seg_offsets, w_gate, w_up, w.hp, status, st);
+        if (s != MOE_OK) return s;
+        s = down_impl(v, w.hp, w.seg_expert, w.seg_offsets, w_down, w.yp, status, st);
+        if (s != MOE_OK) return s;
+        return cuda_status(launch_combine(w.yp, w.dest, w.topk_w, nullptr, v.T, v.k, v.d, v.rows, out, sm_count(), st));
+    }
     s = dispatch_impl(v, x, w.topk_ids, 0, w.counts, w.seg_expert, w.seg_offsets, w.seg_first_rank, w.dest, w.src,
                       w.xp, status, w.dispatch_ws, w.dispatch_ws_bytes, st);
     if (s != MOE_OK) return s;

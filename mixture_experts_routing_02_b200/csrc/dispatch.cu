@@ -741,6 +741,212 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
     }
 }
 
+// ------------------------------------------------------------------------------ overflow re-routing
+
+// Exclusive scan over the 1024 threads of a block; *total = the sum.  warp_sums: 33 ints.
+__device__ __forceinline__ int block_exclusive_scan_1024(int v, int* warp_sums, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += t;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        const int w0 = warp_sums[lane];
+        int w = w0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += t;
+        }
+        __syncwarp();
+        warp_sums[lane] = w - w0;
+        if (lane == 31) warp_sums[32] = w;
+    }
+    __syncthreads();
+    const int r = warp_sums[warp] + x - v;
+    if (total != nullptr) *total = warp_sums[32];
+    __syncthreads();
+    return r;
+}
+
+// Capacity with re-routing of the overflow ("로드 밸런싱 손실 ... 용량(capacity)은 별개": a pair
+// over its expert's capacity may go to another candidate).  One CTA of kRerouteThreads threads:
+//  round 0  each expert keeps its first C pairs in q order (stable ranks: match_any inside a warp,
+//           per-warp counts across warps, running counts across chunks of the pair list);
+//  round r  every unplaced pair proposes to its token's next candidate in logit order (after the
+//           token's cursor, which starts at its k-th selected expert) among the experts that had
+//           room when the round began; a token's unplaced pairs take consecutive candidates in
+//           j order (one pass per multiplicity); each expert accepts the proposals in q order
+//           while it has room; a pair without a candidate is dropped.
+// Segment e holds expert e's rows: round 0 first, then round 1, ...; q order inside a round.
+// Writes counts (the plain histogram), the tables, dest and src; X rows are then copied by
+// scatter_rows_kernel.  At most E + 1 rounds: each round either places every proposal or
+// fills an expert.
+__global__ void __launch_bounds__(kRerouteThreads, 1) reroute_kernel(RerouteArgs a) {
+    __shared__ int s_wcnt[kRerouteThreads / 32][kMaxExperts];
+    __shared__ int s_run[kMaxExperts];      // round 0: pairs so far; round r: proposals so far
+    __shared__ int s_assigned[kMaxExperts];
+    __shared__ int s_room[kMaxExperts];
+    __shared__ int warp_sums[33];
+    __shared__ int s_n_pend, s_any_open;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kWarps = kRerouteThreads / 32;
+    const int E = a.E, k = a.k, C = a.capacity;
+    const int n = a.T * k;
+    const unsigned lanemask_lt = (1u << lane) - 1u;
+
+    for (int i = tid; i < kWarps * kMaxExperts; i += blockDim.x) (&s_wcnt[0][0])[i] = 0;
+    for (int e = tid; e < E; e += blockDim.x) s_run[e] = 0;
+    if (tid == 0) s_n_pend = 0;
+    __syncthreads();
+
+    // stable ranks of one chunk of entries whose experts are ex; returns the rank among equal
+    // experts so far (s_run) and adds the chunk's counts to s_run
+    auto chunk_rank = [&](int ex) -> int {
+        const unsigned same = __match_any_sync(0xffffffffu, ex);
+        const int wrank = __popc(same & lanemask_lt);
+        if (ex >= 0 && wrank == 0) s_wcnt[warp][ex] = __popc(same);
+        __syncthreads();
+        int r = -1;
+        if (ex >= 0) {
+            r = s_run[ex] + wrank;
+            for (int w = 0; w < warp; ++w) r += s_wcnt[w][ex];
+        }
+        __syncthreads();
+        for (int x = tid; x < E; x += blockDim.x) {
+            int c = 0;
+            for (int w = 0; w < kWarps; ++w) { c += s_wcnt[w][x]; s_wcnt[w][x] = 0; }
+            s_run[x] += c;
+        }
+        __syncthreads();
+        return r;
+    };
+
+    // round 0
+    for (int q0 = 0; q0 < n; q0 += blockDim.x) {
+        const int q = q0 + tid;
+        int e = -1;
+        if (q < n) {
+            e = __ldg(a.ids + q);
+            if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) e = -1;
+        }
+        const int r = chunk_rank(e);
+        const bool keep = e >= 0 && r < C;
+        if (q < n) {
+            a.fexp[q] = keep ? e : -1;
+            a.fslot[q] = keep ? r : -1;
+        }
+        int total;
+        const int pos = block_exclusive_scan_1024((q < n && e >= 0 && !keep) ? 1 : 0, warp_sums, &total);
+        if (q < n && e >= 0 && !keep) a.pend[s_n_pend + pos] = q;
+        __syncthreads();
+        if (tid == 0) s_n_pend += total;
+        __syncthreads();
+    }
+    for (int e = tid; e < E; e += blockDim.x) {
+        a.counts[e] = s_run[e];
+        s_assigned[e] = min(s_run[e], C);
+    }
+    // cursors: each token's k-th selected expert
+    for (int t = tid; t < a.T; t += blockDim.x) {
+        const int e = __ldg(a.ids + static_cast<size_t>(t) * k + (k - 1));
+        a.cur_i[t] = e;
+        a.cur_v[t] = (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? __ldg(a.logits + static_cast<size_t>(t) * E + e)
+                                                                           : INFINITY;
+    }
+    __syncthreads();
+
+    int* pend = a.pend;
+    int* next = a.pend2;
+    for (int round = 1; round <= E + 1 && s_n_pend > 0; ++round) {
+        const int np = s_n_pend;
+        if (tid == 0) s_any_open = 0;
+        __syncthreads();
+        for (int e = tid; e < E; e += blockDim.x) {
+            s_room[e] = C - s_assigned[e];
+            s_run[e] = 0;
+            if (s_room[e] > 0) s_any_open = 1;
+        }
+        __syncthreads();
+        if (!s_any_open) break;
+        // proposals, one pass per multiplicity (the m-th unplaced pair of its token)
+        for (int m = 0; m < k; ++m) {
+            for (int i = tid; i < np; i += blockDim.x) {
+                const int q = pend[i], t = q / k;
+                int mult = 0;
+                while (mult < i && pend[i - 1 - mult] / k == t) ++mult;
+                if (mult != m) continue;
+                const float cv = a.cur_v[t];
+                const int ci = a.cur_i[t];
+                float bv = -INFINITY;
+                int bi = -1;
+                const float* lt = a.logits + static_cast<size_t>(t) * E;
+                for (int e = 0; e < E; ++e) {
+                    if (s_room[e] <= 0) continue;
+                    const float v = __ldg(lt + e);
+                    const bool after = v < cv || (v == cv && e > ci);
+                    if (after && (bi < 0 || v > bv)) { bv = v; bi = e; }  // ascending e: ties keep the lower id
+                }
+                a.prop[i] = bi;
+                if (bi >= 0) { a.cur_v[t] = bv; a.cur_i[t] = bi; }
+            }
+            __syncthreads();
+        }
+        // acceptance in q order; the rest stays pending for the next round
+        if (tid == 0) s_n_pend = 0;
+        __syncthreads();
+        for (int i0 = 0; i0 < np; i0 += blockDim.x) {
+            const int i = i0 + tid;
+            const int e = i < np ? a.prop[i] : -1;
+            const int q = i < np ? pend[i] : -1;
+            const int r = chunk_rank(e);
+            const bool acc = e >= 0 && r < s_room[e];
+            if (acc) {
+                a.fexp[q] = e;
+                a.fslot[q] = s_assigned[e] + r;
+            }
+            int total;
+            const bool stay = e >= 0 && !acc;
+            const int pos = block_exclusive_scan_1024(stay ? 1 : 0, warp_sums, &total);
+            if (stay) next[s_n_pend + pos] = q;
+            __syncthreads();
+            if (tid == 0) s_n_pend += total;
+            __syncthreads();
+        }
+        for (int e = tid; e < E; e += blockDim.x) s_assigned[e] += min(s_run[e], s_room[e]);
+        __syncthreads();
+        int* tmp = pend; pend = next; next = tmp;
+    }
+
+    // tables and positions
+    int total;
+    const int v = tid < E ? s_assigned[tid] : 0;
+    const int off = block_exclusive_scan_1024(v, warp_sums, &total);
+    if (tid < E) {
+        s_room[tid] = off;
+        a.seg_expert[tid] = tid;
+        a.seg_offsets[tid] = off;
+        a.seg_first_rank[tid] = 0;
+    }
+    if (tid == 0) a.seg_offsets[E] = total;
+    __syncthreads();
+    for (int q = tid; q < n; q += blockDim.x) {
+        const int e = a.fexp[q];
+        int dst = -1;
+        if (e >= 0) {
+            dst = s_room[e] + a.fslot[q];
+            if (dst >= a.rows) dst = -1;
+        }
+        a.dest[q] = dst;
+        if (dst >= 0) a.src[dst] = q;
+    }
+}
+
 // ------------------------------------------------------------------------------ row scatter
 
 // One warp per token: read the token's row of X once (16-byte vectors, 8 in flight per lane)
@@ -958,6 +1164,35 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
     int grid = num_sms;
     if (grid > a.T) grid = a.T;
     dispatch_count_kernel<<<grid, kCountThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+size_t reroute_ws_bytes(int T, int k) {
+    auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
+    const size_t tk = static_cast<size_t>(T) * k;
+    return 256 + 5 * up(tk * sizeof(int32_t)) + 2 * up(static_cast<size_t>(T) * sizeof(int32_t));
+}
+
+cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16* x, __nv_bfloat16* xp, int d,
+                           int num_sms, cudaStream_t stream) {
+    if (a0.T == 0) return cudaSuccess;
+    RerouteArgs a = a0;
+    const size_t tk = static_cast<size_t>(a.T) * a.k;
+    uint8_t* p = static_cast<uint8_t*>(ws) + 256;
+    auto take = [&](size_t bytes) { uint8_t* r = p; p += (bytes + 255) & ~size_t(255); return r; };
+    a.pend = reinterpret_cast<int32_t*>(take(tk * 4));
+    a.pend2 = reinterpret_cast<int32_t*>(take(tk * 4));
+    a.prop = reinterpret_cast<int32_t*>(take(tk * 4));
+    a.fexp = reinterpret_cast<int32_t*>(take(tk * 4));
+    a.fslot = reinterpret_cast<int32_t*>(take(tk * 4));
+    a.cur_v = reinterpret_cast<float*>(take(static_cast<size_t>(a.T) * 4));
+    a.cur_i = reinterpret_cast<int32_t*>(take(static_cast<size_t>(a.T) * 4));
+    reroute_kernel<<<1, kRerouteThreads, 0, stream>>>(a);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    int sgrid = (a.T + 7) / 8;
+    if (sgrid > 16 * num_sms) sgrid = 16 * num_sms;
+    scatter_rows_kernel<<<sgrid, 256, 0, stream>>>(x, a.dest, a.T, a.k, d, a.rows, xp);
     return cudaGetLastError();
 }
 

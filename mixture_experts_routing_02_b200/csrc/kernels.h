@@ -113,6 +113,26 @@ cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, c
 cudaError_t launch_dispatch_fused(const PermuteArgs& a, int num_sms, cudaStream_t stream);
 cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_t stream);
 constexpr int kCountMaxPairs = 1 << 16;
+
+// Overflow re-routing (one CTA; T*k <= kCountMaxPairs), then the row copies.
+constexpr int kRerouteThreads = 1024;
+struct RerouteArgs {
+    const int32_t* ids;
+    const float* logits;  // [T, E] fp32: the candidate order of each token
+    int T, k, E, capacity, rows;
+    int32_t* counts;
+    int32_t* seg_expert;
+    int32_t* seg_offsets;
+    int32_t* seg_first_rank;
+    int32_t* dest;
+    int32_t* src;
+    // scratch, set by launch_reroute from the workspace
+    int32_t *pend, *pend2, *prop, *fexp, *fslot, *cur_i;
+    float* cur_v;
+};
+size_t reroute_ws_bytes(int T, int k);
+cudaError_t launch_reroute(const RerouteArgs& a, void* ws, const __nv_bfloat16* x, __nv_bfloat16* xp, int d,
+                           int num_sms, cudaStream_t stream);
 cudaError_t launch_route_from_logits(const float* logits, int T, int E, int k, int route_flags, int32_t* ids,
                                      float* w, int num_sms, cudaStream_t stream);
 // Routing from n_split partial logit slices (summed in order, + bias): top-k ids and weights, or

@@ -20,6 +20,7 @@ pages' own models and benchmarks are not available, so these stand in):
                   expert keeping C = T*k/E = 1024 tokens
 * expert-choice-e64  the skewed shape (Zipf(1.2) bias) with expert-choice
                   routing, C = 256 tokens per expert
+* skewed-reroute  the skewed layer with overflow re-routed to other candidates
 
 X ~ N(0, 1) and every weight ~ N(0, 0.02^2), drawn in fp32 and rounded to
 bf16.  Each tensor (and each expert of an expert tensor) has its own
@@ -50,6 +51,7 @@ class Workload:
     n_groups: int = 0              # R; 0 = no balanced plan
     replica_slots: int = 0         # B per group
     expert_choice: bool = False    # experts choose tokens; C = ceil(capacity_factor * T * k / E)
+    reroute: bool = False          # pairs over capacity go to their token's next open candidate
 
     @property
     def tokens_per_group(self) -> int:
@@ -74,6 +76,10 @@ EXPERT_CHOICE = Workload("expert-choice", T=4096, d=4096, E=8, k=2, F=14336, cap
 EXPERT_CHOICE_E64 = Workload("expert-choice-e64", T=8192, d=4096, E=64, k=2, F=1408, zipf_s=1.2,
                              capacity_factor=1.0, expert_choice=True)
 
+# The skewed layer with its overflow re-routed instead of dropped.
+SKEWED_REROUTE = Workload("skewed-reroute", T=8192, d=4096, E=64, k=2, F=1408, zipf_s=1.2, capacity_factor=1.25,
+                          reroute=True)
+
 # Reduced copies for profiling captures that must stay at a few GB on the device: the same
 # per-expert shapes and rows per expert as the full workloads, with fewer experts.
 DEEPSEEK_LIKE_E32 = Workload("deepseek-like-e32", T=512, d=7168, E=32, k=8, F=2048)
@@ -81,7 +87,7 @@ BALANCED_E32 = Workload("balanced-plan-e32", T=4096, d=7168, E=32, k=8, F=2048,
                         zipf_s=1.2, n_groups=2, replica_slots=16)
 
 WORKLOADS = {w.name: w for w in (TINY, MIXTRAL_LIKE, DEEPSEEK_LIKE, SKEWED, BALANCED, DEEPSEEK_LIKE_E32,
-                                 BALANCED_E32, EXPERT_CHOICE, EXPERT_CHOICE_E64)}
+                                 BALANCED_E32, EXPERT_CHOICE, EXPERT_CHOICE_E64, SKEWED_REROUTE)}
 
 
 def sub_seed(seed: int, tag: str, *idx: int) -> int:
@@ -180,7 +186,7 @@ def ceil_div(a: int, b: int) -> int:
 
 __all__ = [
     "Workload", "TINY", "MIXTRAL_LIKE", "DEEPSEEK_LIKE", "SKEWED", "BALANCED", "DEEPSEEK_LIKE_E32", "BALANCED_E32",
-    "EXPERT_CHOICE", "EXPERT_CHOICE_E64",
+    "EXPERT_CHOICE", "EXPERT_CHOICE_E64", "SKEWED_REROUTE",
     "WORKLOADS",
     "sub_seed", "zipf_bias", "router_inputs", "x_row_redraw", "expert_weights", "shared_expert_weights",
     "lognormal_topk_ids", "uniform_roundrobin_ids", "gib", "ceil_div",

@@ -122,8 +122,9 @@ def capacity_rows(w: syn.Workload) -> int:
 
 def moe_shape(w: syn.Workload, capacity: Optional[int] = None):
     C = capacity_rows(w) if capacity is None else capacity
+    flags = (moe.ROUTE_EXPERT_CHOICE if w.expert_choice else 0) | (moe.ROUTE_REROUTE if w.reroute else 0)
     return moe.shape(w.T, w.d, w.E, w.k, w.F, capacity=C, n_groups=w.n_groups, replica_slots=w.replica_slots,
-                     route_flags=moe.ROUTE_EXPERT_CHOICE if w.expert_choice else 0)
+                     route_flags=flags)
 
 
 @dataclasses.dataclass
@@ -143,6 +144,9 @@ def make_case(w: syn.Workload, seed: int = 0, weights_device="cpu", margin=True)
         redraw = lambda t, a: syn.x_row_redraw(w, seed, t, a)
         if w.expert_choice:
             oracle.enforce_ec_margin(x, w_r, bias, capacity_rows(w), redraw)
+        elif w.reroute:
+            # re-routed pairs go down each token's whole logit order: keep all of it 1e-3 apart
+            oracle.enforce_margin(x, w_r, bias, w.E - 1, redraw)
         else:
             oracle.enforce_margin(x, w_r, bias, w.k, redraw)
     wg, wu, wd = syn.expert_weights(w, seed, device=weights_device)
