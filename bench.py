@@ -163,7 +163,8 @@ def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: fl
 def _config(w, capacity):
     return {"workload": w.name, "T": w.T, "d_model": w.d, "n_experts": w.E, "top_k": w.k, "d_ff": w.F,
             "capacity": capacity, "n_groups": w.n_groups, "replica_slots": w.replica_slots,
-            "zipf_bias_s": w.zipf_s, "routing": "expert-choice" if w.expert_choice else "top-k",
+            "zipf_bias_s": w.zipf_s,
+            "routing": "expert-choice" if w.expert_choice else ("top-k, overflow re-routed" if w.reroute else "top-k"),
             "l2": "flushed between steps (256 MiB write outside the timed events)",
             "parallelism": "replicas (no exchange between GPUs)"}
 
@@ -180,6 +181,8 @@ def _oracle_sample(w, seed: int, n_route: int, n_ffn: int, wg, wu, wd):
     x, w_r, bias = syn.router_inputs(w.scaled(T=n_route), seed)
     if w.expert_choice:
         return _oracle_sample_ec(w, x, w_r, bias, n_route, n_ffn, wg, wu, wd)
+    if w.reroute:
+        return _oracle_sample_reroute(w, x, w_r, bias, n_route, n_ffn, wg, wu, wd)
     t0 = time.perf_counter()
     logits, ids, wts = oracle.route(x, w_r, bias, w.k)
     t1 = time.perf_counter()
@@ -199,6 +202,33 @@ def _oracle_sample(w, seed: int, n_route: int, n_ffn: int, wg, wu, wd):
             f"(gate/up/down, fp64) of {n_ffn} rows of one expert; per-token cost = per-token routing+dispatch"
             f"+combine + k x per-row FFN, extrapolated to tokens/s")
     return 1.0 / per_token, desc, t4 - t0
+
+
+def _oracle_sample_reroute(w, x, w_r, bias, n_route: int, n_ffn: int, wg, wu, wd):
+    """The re-routing layer's oracle on a sample: routing, capacity rounds and placement of
+    n_route tokens (C scaled to them), the FFN of n_ffn rows of one expert, the combine."""
+    import numpy as np
+    import oracle
+
+    C = _capacity(w.scaled(T=n_route))
+    t0 = time.perf_counter()
+    logits, ids, wts = oracle.route(x, w_r, bias, w.k)
+    rr = oracle.reroute_overflow(ids, logits, C)
+    segs, dest, src = oracle.reroute_positions(rr)
+    xp = oracle.permute_rows(x, src, w.k)
+    t1 = time.perf_counter()
+    _, y = oracle.expert_ffn(xp[:n_ffn], wg[0], wu[0], wd[0])
+    t2 = time.perf_counter()
+    yfull = np.zeros((xp.shape[0], w.d))
+    yfull[:n_ffn] = y
+    oracle.combine(yfull, dest, wts, n_route, w.k)
+    t3 = time.perf_counter()
+    rows_per_token = xp.shape[0] / n_route
+    per_token = (t1 - t0) / n_route + rows_per_token * (t2 - t1) / n_ffn + (t3 - t2) / n_route
+    desc = (f"routing, capacity re-routing rounds and dispatch of {n_route} tokens (C={C}) and combine; expert "
+            f"FFN (gate/up/down, fp64) of {n_ffn} rows of one expert; per-token cost = per-token routing+dispatch"
+            f"+combine + (rows per token = {rows_per_token:g}) x per-row FFN, extrapolated to tokens/s")
+    return 1.0 / per_token, desc, t3 - t0
 
 
 def _oracle_sample_ec(w, x, w_r, bias, n_route: int, n_ffn: int, wg, wu, wd):
@@ -292,8 +322,10 @@ def run_ours(args, w):
 
     capacity = _capacity(w)
     ec = w.expert_choice
+    rr = w.reroute
     s = moe.shape(w.T, w.d, w.E, w.k, w.F, capacity=capacity, n_groups=w.n_groups,
-                  replica_slots=w.replica_slots, route_flags=moe.ROUTE_EXPERT_CHOICE if ec else 0)
+                  replica_slots=w.replica_slots,
+                  route_flags=(moe.ROUTE_EXPERT_CHOICE if ec else 0) | (moe.ROUTE_REROUTE if rr else 0))
     n_seg, rows_alloc = moe.moe_layout(s)
     _, layer_bytes = moe.moe_workspace_size(s)
 
@@ -332,11 +364,12 @@ def run_ours(args, w):
         scores = view(v.scores, w.E * w.T, torch.float32)
         emap = view(v.emap, w.T * w.E, torch.int32)
         row_w = view(v.row_w, rows_alloc, torch.float32)
+    logits = view(v.logits, w.T * w.E, torch.float32) if rr else None
     # the router projection's reduction is split over more CTAs when its row tiles are few
     route_ws_bytes = moe.moe_route_workspace_size(s)
     route_ws = torch.empty(max(route_ws_bytes, 256), dtype=torch.uint8, device=dev) if route_ws_bytes else None
     launches = ((2 if route_ws_bytes else 1)                                   # route (+ partial sums)
-                + (2 if ec else (4 if w.n_groups else 1))                      # dispatch
+                + (2 if ec or rr else (4 if w.n_groups else 1))                # dispatch
                 + 3)                                                           # gate_up, down, combine
 
     Fs = args.shared_expert
@@ -363,9 +396,13 @@ def run_ours(args, w):
             ev[1].record(stream)
             moe.moe_expert_choose(s, scores, x, seg_e, seg_o, src, row_w, emap, xp, stream)
         else:
-            moe.moe_route_ws(s, x, w_r, bias, None, ids, wts, status, route_ws, stream)
+            moe.moe_route_ws(s, x, w_r, bias, logits, ids, wts, status, route_ws, stream)
             ev[1].record(stream)
-            moe.moe_dispatch(s, x, ids, 0, counts, seg_e, seg_o, seg_f, dest, src, xp, status, dws, stream)
+            if rr:
+                moe.moe_dispatch_reroute(s, x, ids, logits, counts, seg_e, seg_o, seg_f, dest, src, xp, status, dws,
+                                         stream)
+            else:
+                moe.moe_dispatch(s, x, ids, 0, counts, seg_e, seg_o, seg_f, dest, src, xp, status, dws, stream)
         ev[2].record(stream)
         moe.moe_expert_gate_up(s, xp, seg_e, seg_o, wg, wu, hp, status, stream)
         ev[3].record(stream)

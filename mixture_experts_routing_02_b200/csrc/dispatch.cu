@@ -743,197 +743,243 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
 
 // ------------------------------------------------------------------------------ overflow re-routing
 
-// Exclusive scan over the 1024 threads of a block; *total = the sum.  warp_sums: 33 ints.
-__device__ __forceinline__ int block_exclusive_scan_1024(int v, int* warp_sums, int* total) {
+// Stable ranks inside one CTA of kRerouteThreads threads, for a list of n entries whose keys
+// (experts, -1 = none) come from key(i): warp w owns the contiguous range [w*L, (w+1)*L) of the
+// list, counts its keys per expert (cnt[w][e]), the counts become exclusive prefixes across warps
+// (plus base[e]), and each warp walks its range again handing out ranks in list order.  Two
+// block barriers in all.  rank_out(i, e, r) receives every entry with a key; totals[e] (if not
+// null) the number of entries per expert.
+template <typename KeyF, typename OutF>
+__device__ __forceinline__ void warp_range_ranks(int n, int E, int (*cnt)[kMaxExperts], const int* base,
+                                                 int* totals, KeyF key, OutF rank_out) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += t;
+    constexpr int kWarps = kRerouteThreads / 32;
+    const unsigned lanemask_lt = (1u << lane) - 1u;
+    const int L = (n + kWarps - 1) / kWarps;
+    const int b0 = min(n, warp * L), b1 = min(n, b0 + L);
+    for (int e = lane; e < E; e += 32) cnt[warp][e] = 0;
+    __syncwarp();
+    for (int i0 = b0; i0 < b1; i0 += 32) {
+        const int i = i0 + lane;
+        const int e = i < b1 ? key(i) : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && (same & lanemask_lt) == 0) cnt[warp][e] += __popc(same);
+        __syncwarp();
     }
-    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = base ? base[e] : 0;
+        for (int w = 0; w < kWarps; ++w) {
+            const int c = cnt[w][e];
+            cnt[w][e] = run;
+            run += c;
+        }
+        if (totals) totals[e] = run - (base ? base[e] : 0);
+    }
+    __syncthreads();
+    for (int i0 = b0; i0 < b1; i0 += 32) {
+        const int i = i0 + lane;
+        const int e = i < b1 ? key(i) : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int r = e >= 0 ? cnt[warp][e] + __popc(same & lanemask_lt) : -1;
+        __syncwarp();
+        if (e >= 0 && (same & lanemask_lt) == 0) cnt[warp][e] += __popc(same);
+        __syncwarp();
+        if (e >= 0) rank_out(i, e, r);
+    }
+    __syncthreads();
+}
+
+// Order-preserving compaction inside one CTA: entries i < n with keep(i) are written, in order,
+// through put(position, i); returns the number kept.  Same warp ranges; two barriers.
+template <typename KeepF, typename PutF>
+__device__ __forceinline__ int warp_range_compact(int n, int* warp_cnt /*[33]*/, KeepF keep, PutF put) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int kWarps = kRerouteThreads / 32;
+    const int L = (n + kWarps - 1) / kWarps;
+    const int b0 = min(n, warp * L), b1 = min(n, b0 + L);
+    int c = 0;
+    for (int i0 = b0; i0 < b1; i0 += 32) {
+        const int i = i0 + lane;
+        c += __popc(__ballot_sync(0xffffffffu, i < b1 && keep(i)));
+    }
+    if (lane == 0) warp_cnt[warp] = c;
     __syncthreads();
     if (warp == 0) {
-        const int w0 = warp_sums[lane];
-        int w = w0;
+        const int v = warp_cnt[lane];
+        int x = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += t;
+            const int t = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += t;
         }
-        __syncwarp();
-        warp_sums[lane] = w - w0;
-        if (lane == 31) warp_sums[32] = w;
+        warp_cnt[lane] = x - v;
+        if (lane == 31) warp_cnt[32] = x;
     }
     __syncthreads();
-    const int r = warp_sums[warp] + x - v;
-    if (total != nullptr) *total = warp_sums[32];
+    int pos = warp_cnt[warp];
+    for (int i0 = b0; i0 < b1; i0 += 32) {
+        const int i = i0 + lane;
+        const bool k = i < b1 && keep(i);
+        const unsigned b = __ballot_sync(0xffffffffu, k);
+        if (k) put(pos + __popc(b & ((1u << lane) - 1u)), i);
+        pos += __popc(b);
+    }
+    const int total = warp_cnt[32];
     __syncthreads();
-    return r;
+    return total;
+}
+
+// Each token's experts in candidate order (logit descending, equal logits: the lower id), one
+// warp per token over the whole GPU: every lane ranks its U experts against all E by shuffles
+// and writes them to their positions.  A token's first k candidates are its top-k.
+template <int U>
+__global__ void __launch_bounds__(256) candidate_order_kernel(const float* __restrict__ logits, int T, int E,
+                                                              uint8_t* __restrict__ cand) {
+    const int lane = threadIdx.x & 31;
+    const int warps_total = gridDim.x * (blockDim.x >> 5);
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
+        const float* lt = logits + static_cast<size_t>(t) * E;
+        float v[U];
+        int rank[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            v[u] = (lane + 32 * u < E) ? __ldg(lt + lane + 32 * u) : -INFINITY;
+            rank[u] = 0;
+        }
+#pragma unroll
+        for (int u2 = 0; u2 < U; ++u2) {
+            for (int src = 0; src < 32; ++src) {
+                const float o = __shfl_sync(0xffffffffu, v[u2], src);
+                const int oe = 32 * u2 + src;
+                if (oe >= E) break;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int e = lane + 32 * u;
+                    rank[u] += (o > v[u] || (o == v[u] && oe < e)) ? 1 : 0;
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int e = lane + 32 * u;
+            if (e < E) cand[static_cast<size_t>(t) * E + rank[u]] = static_cast<uint8_t>(e);
+        }
+    }
 }
 
 // Capacity with re-routing of the overflow ("로드 밸런싱 손실 ... 용량(capacity)은 별개": a pair
 // over its expert's capacity may go to another candidate).  One CTA of kRerouteThreads threads:
-//  round 0  each expert keeps its first C pairs in q order (stable ranks: match_any inside a warp,
-//           per-warp counts across warps, running counts across chunks of the pair list);
-//  round r  every unplaced pair proposes to its token's next candidate in logit order (after the
-//           token's cursor, which starts at its k-th selected expert) among the experts that had
-//           room when the round began; a token's unplaced pairs take consecutive candidates in
-//           j order (one pass per multiplicity); each expert accepts the proposals in q order
-//           while it has room; a pair without a candidate is dropped.
+//  round 0  each expert keeps its first C pairs in q order (stable ranks over the pair list);
+//  round r  every unplaced pair proposes to its token's next candidate in logit order (the
+//           token's experts are sorted once; its cursor starts after its top-k) among the experts
+//           that had room when the round began; a token's unplaced pairs take consecutive
+//           candidates in j order (one pass per multiplicity); each expert accepts the proposals
+//           in q order while it has room; a pair without a candidate is dropped.
 // Segment e holds expert e's rows: round 0 first, then round 1, ...; q order inside a round.
 // Writes counts (the plain histogram), the tables, dest and src; X rows are then copied by
 // scatter_rows_kernel.  At most E + 1 rounds: each round either places every proposal or
-// fills an expert.
+// fills an expert (with a skewed router, about one expert fills per round).  The ranks and
+// compactions use warp-owned ranges of the lists (two block barriers per pass).
 __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_kernel(RerouteArgs a) {
-    __shared__ int s_wcnt[kRerouteThreads / 32][kMaxExperts];
-    __shared__ int s_run[kMaxExperts];      // round 0: pairs so far; round r: proposals so far
+    __shared__ int s_cnt[kRerouteThreads / 32][kMaxExperts];
+    __shared__ int s_tot[kMaxExperts];
     __shared__ int s_assigned[kMaxExperts];
     __shared__ int s_room[kMaxExperts];
-    __shared__ int warp_sums[33];
-    __shared__ int s_n_pend, s_any_open;
+    __shared__ int s_wc[33];
+    __shared__ int s_any_open;
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int kWarps = kRerouteThreads / 32;
+    const int tid = threadIdx.x;
     const int E = a.E, k = a.k, C = a.capacity;
     const int n = a.T * k;
-    const unsigned lanemask_lt = (1u << lane) - 1u;
 
-    for (int i = tid; i < kWarps * kMaxExperts; i += blockDim.x) (&s_wcnt[0][0])[i] = 0;
-    for (int e = tid; e < E; e += blockDim.x) s_run[e] = 0;
-    if (tid == 0) s_n_pend = 0;
-    __syncthreads();
-
-    // stable ranks of one chunk of entries whose experts are ex; returns the rank among equal
-    // experts so far (s_run) and adds the chunk's counts to s_run
-    auto chunk_rank = [&](int ex) -> int {
-        const unsigned same = __match_any_sync(0xffffffffu, ex);
-        const int wrank = __popc(same & lanemask_lt);
-        if (ex >= 0 && wrank == 0) s_wcnt[warp][ex] = __popc(same);
-        __syncthreads();
-        int r = -1;
-        if (ex >= 0) {
-            r = s_run[ex] + wrank;
-            for (int w = 0; w < warp; ++w) r += s_wcnt[w][ex];
-        }
-        __syncthreads();
-        for (int x = tid; x < E; x += blockDim.x) {
-            int c = 0;
-            for (int w = 0; w < kWarps; ++w) { c += s_wcnt[w][x]; s_wcnt[w][x] = 0; }
-            s_run[x] += c;
-        }
-        __syncthreads();
-        return r;
+    // round 0: stable ranks over all pairs; keep the first C of each expert
+    auto id_of = [&](int q) -> int {
+        const int e = __ldg(a.ids + q);
+        return static_cast<unsigned>(e) < static_cast<unsigned>(E) ? e : -1;
     };
-
-    // round 0
-    for (int q0 = 0; q0 < n; q0 += blockDim.x) {
-        const int q = q0 + tid;
-        int e = -1;
-        if (q < n) {
-            e = __ldg(a.ids + q);
-            if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) e = -1;
-        }
-        const int r = chunk_rank(e);
-        const bool keep = e >= 0 && r < C;
-        if (q < n) {
-            a.fexp[q] = keep ? e : -1;
-            a.fslot[q] = keep ? r : -1;
-        }
-        int total;
-        const int pos = block_exclusive_scan_1024((q < n && e >= 0 && !keep) ? 1 : 0, warp_sums, &total);
-        if (q < n && e >= 0 && !keep) a.pend[s_n_pend + pos] = q;
-        __syncthreads();
-        if (tid == 0) s_n_pend += total;
-        __syncthreads();
-    }
+    for (int q = tid; q < n; q += blockDim.x) { a.fexp[q] = -1; a.fslot[q] = -1; }
+    __syncthreads();
+    warp_range_ranks(n, E, s_cnt, nullptr, s_tot, id_of, [&](int q, int e, int r) {
+        if (r < C) { a.fexp[q] = e; a.fslot[q] = r; }
+    });
     for (int e = tid; e < E; e += blockDim.x) {
-        a.counts[e] = s_run[e];
-        s_assigned[e] = min(s_run[e], C);
+        a.counts[e] = s_tot[e];
+        s_assigned[e] = min(s_tot[e], C);
     }
-    // cursors: each token's k-th selected expert
-    for (int t = tid; t < a.T; t += blockDim.x) {
-        const int e = __ldg(a.ids + static_cast<size_t>(t) * k + (k - 1));
-        a.cur_i[t] = e;
-        a.cur_v[t] = (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? __ldg(a.logits + static_cast<size_t>(t) * E + e)
-                                                                           : INFINITY;
-    }
+    int n_pend = warp_range_compact(n, s_wc, [&](int q) { return id_of(q) >= 0 && a.fexp[q] < 0; },
+                                    [&](int pos, int q) { a.pend[pos] = q; });
+    for (int t = tid; t < a.T; t += blockDim.x) a.cur_pos[t] = k;  // a token's first k candidates are its top-k
     __syncthreads();
 
     int* pend = a.pend;
     int* next = a.pend2;
-    for (int round = 1; round <= E + 1 && s_n_pend > 0; ++round) {
-        const int np = s_n_pend;
+    for (int round = 1; round <= E + 1 && n_pend > 0; ++round) {
         if (tid == 0) s_any_open = 0;
         __syncthreads();
         for (int e = tid; e < E; e += blockDim.x) {
             s_room[e] = C - s_assigned[e];
-            s_run[e] = 0;
             if (s_room[e] > 0) s_any_open = 1;
         }
         __syncthreads();
         if (!s_any_open) break;
-        // proposals, one pass per multiplicity (the m-th unplaced pair of its token)
+        // proposals, one pass per multiplicity (the m-th unplaced pair of its token; pairs of a
+        // token are adjacent in the list, so the multiplicity is the distance to the first)
+        for (int i = tid; i < n_pend; i += blockDim.x) {
+            const int t = pend[i] / k;
+            int mult = 0;
+            while (mult < i && pend[i - 1 - mult] / k == t) ++mult;
+            next[i] = mult;  // next[] is free until the compaction below
+        }
+        __syncthreads();
         for (int m = 0; m < k; ++m) {
-            for (int i = tid; i < np; i += blockDim.x) {
-                const int q = pend[i], t = q / k;
-                int mult = 0;
-                while (mult < i && pend[i - 1 - mult] / k == t) ++mult;
-                if (mult != m) continue;
-                const float cv = a.cur_v[t];
-                const int ci = a.cur_i[t];
-                float bv = -INFINITY;
-                int bi = -1;
-                const float* lt = a.logits + static_cast<size_t>(t) * E;
-                for (int e = 0; e < E; ++e) {
-                    if (s_room[e] <= 0) continue;
-                    const float v = __ldg(lt + e);
-                    const bool after = v < cv || (v == cv && e > ci);
-                    if (after && (bi < 0 || v > bv)) { bv = v; bi = e; }  // ascending e: ties keep the lower id
-                }
-                a.prop[i] = bi;
-                if (bi >= 0) { a.cur_v[t] = bv; a.cur_i[t] = bi; }
+            for (int i = tid; i < n_pend; i += blockDim.x) {
+                if (next[i] != m) continue;
+                const int t = pend[i] / k;
+                // the next candidate with room (experts never reopen, so a skipped one stays skipped)
+                const uint8_t* ct = a.cand + static_cast<size_t>(t) * E;
+                int pos = a.cur_pos[t];
+                while (pos < E && s_room[ct[pos]] <= 0) ++pos;
+                a.prop[i] = pos < E ? ct[pos] : -1;
+                a.cur_pos[t] = pos < E ? pos + 1 : E;
             }
             __syncthreads();
         }
-        // acceptance in q order; the rest stays pending for the next round
-        if (tid == 0) s_n_pend = 0;
-        __syncthreads();
-        for (int i0 = 0; i0 < np; i0 += blockDim.x) {
-            const int i = i0 + tid;
-            const int e = i < np ? a.prop[i] : -1;
-            const int q = i < np ? pend[i] : -1;
-            const int r = chunk_rank(e);
-            const bool acc = e >= 0 && r < s_room[e];
-            if (acc) {
-                a.fexp[q] = e;
-                a.fslot[q] = s_assigned[e] + r;
-            }
-            int total;
-            const bool stay = e >= 0 && !acc;
-            const int pos = block_exclusive_scan_1024(stay ? 1 : 0, warp_sums, &total);
-            if (stay) next[s_n_pend + pos] = q;
-            __syncthreads();
-            if (tid == 0) s_n_pend += total;
-            __syncthreads();
-        }
-        for (int e = tid; e < E; e += blockDim.x) s_assigned[e] += min(s_run[e], s_room[e]);
-        __syncthreads();
+        // acceptance in q order, then the rejected stay pending
+        warp_range_ranks(n_pend, E, s_cnt, nullptr, s_tot, [&](int i) { return a.prop[i]; },
+                         [&](int i, int e, int r) {
+                             if (r < s_room[e]) { a.fexp[pend[i]] = e; a.fslot[pend[i]] = s_assigned[e] + r; }
+                         });
+        for (int e = tid; e < E; e += blockDim.x) s_assigned[e] += min(s_tot[e], s_room[e]);
+        n_pend = warp_range_compact(n_pend, s_wc, [&](int i) { return a.prop[i] >= 0 && a.fexp[pend[i]] < 0; },
+                                    [&](int pos, int i) { next[pos] = pend[i]; });
         int* tmp = pend; pend = next; next = tmp;
     }
 
     // tables and positions
-    int total;
-    const int v = tid < E ? s_assigned[tid] : 0;
-    const int off = block_exclusive_scan_1024(v, warp_sums, &total);
-    if (tid < E) {
-        s_room[tid] = off;
-        a.seg_expert[tid] = tid;
-        a.seg_offsets[tid] = off;
-        a.seg_first_rank[tid] = 0;
+    __syncthreads();
+    if (tid < 32) {
+        // exclusive scan of the experts' rows by one warp
+        int carry = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + tid;
+            const int v = e < E ? s_assigned[e] : 0;
+            int x = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, x, o);
+                if (tid >= o) x += t;
+            }
+            if (e < E) {
+                s_room[e] = carry + x - v;
+                a.seg_expert[e] = e;
+                a.seg_offsets[e] = carry + x - v;
+                a.seg_first_rank[e] = 0;
+            }
+            carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (tid == 0) a.seg_offsets[E] = carry;
     }
-    if (tid == 0) a.seg_offsets[E] = total;
     __syncthreads();
     for (int q = tid; q < n; q += blockDim.x) {
         const int e = a.fexp[q];
@@ -1170,7 +1216,8 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
 size_t reroute_ws_bytes(int T, int k) {
     auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
     const size_t tk = static_cast<size_t>(T) * k;
-    return 256 + 5 * up(tk * sizeof(int32_t)) + 2 * up(static_cast<size_t>(T) * sizeof(int32_t));
+    return 256 + 5 * up(tk * sizeof(int32_t)) + up(static_cast<size_t>(T) * sizeof(int32_t)) +
+           up(static_cast<size_t>(T) * kMaxExperts);
 }
 
 cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16* x, __nv_bfloat16* xp, int d,
@@ -1185,8 +1232,18 @@ cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16*
     a.prop = reinterpret_cast<int32_t*>(take(tk * 4));
     a.fexp = reinterpret_cast<int32_t*>(take(tk * 4));
     a.fslot = reinterpret_cast<int32_t*>(take(tk * 4));
-    a.cur_v = reinterpret_cast<float*>(take(static_cast<size_t>(a.T) * 4));
-    a.cur_i = reinterpret_cast<int32_t*>(take(static_cast<size_t>(a.T) * 4));
+    a.cur_pos = reinterpret_cast<int32_t*>(take(static_cast<size_t>(a.T) * 4));
+    a.cand = take(static_cast<size_t>(a.T) * a.E);
+    {
+        int grid = (a.T + 7) / 8;
+        if (grid > 8 * num_sms) grid = 8 * num_sms;
+        if (a.E <= 32) candidate_order_kernel<1><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, a.cand);
+        else if (a.E <= 64) candidate_order_kernel<2><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, a.cand);
+        else if (a.E <= 128) candidate_order_kernel<4><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, a.cand);
+        else candidate_order_kernel<8><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, a.cand);
+        const cudaError_t e0 = cudaGetLastError();
+        if (e0 != cudaSuccess) return e0;
+    }
     reroute_kernel<<<1, kRerouteThreads, 0, stream>>>(a);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;

@@ -127,8 +127,8 @@ struct RerouteArgs {
     int32_t* dest;
     int32_t* src;
     // scratch, set by launch_reroute from the workspace
-    int32_t *pend, *pend2, *prop, *fexp, *fslot, *cur_i;
-    float* cur_v;
+    int32_t *pend, *pend2, *prop, *fexp, *fslot, *cur_pos;
+    uint8_t* cand;  // [T, E] each token's experts in candidate order
 };
 size_t reroute_ws_bytes(int T, int k);
 cudaError_t launch_reroute(const RerouteArgs& a, void* ws, const __nv_bfloat16* x, __nv_bfloat16* xp, int d,
