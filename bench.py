@@ -60,16 +60,28 @@ def _traffic(kernel: str, workload: str):
     for e in entries:
         if e.get("kernel") != kernel or e.get("workload") != workload:
             continue
-        h = hashlib.sha256()
         try:
-            for fn in e["source_files"]:
-                with open(os.path.join(ROOT, fn), "rb") as f:
-                    h.update(f.read())
+            digest = source_digest(e["source_files"])
         except Exception:
             return None
-        if e.get("source_sha256") == h.hexdigest():
+        if e.get("source_sha256") == digest:
             return e.get("dram_bytes_per_launch")
     return None
+
+
+def source_digest(files) -> str:
+    """sha256 over the kernel's sources; "path#Name" hashes only `struct Name { ... };` of a header."""
+    h = hashlib.sha256()
+    for fn in files:
+        path, _, struct = fn.partition("#")
+        with open(os.path.join(ROOT, path), "rb") as f:
+            data = f.read()
+        if struct:
+            text = data.decode()
+            i = text.index(f"struct {struct} {{")
+            data = text[i:text.index("};", i) + 2].encode()
+        h.update(data)
+    return h.hexdigest()
 
 
 class ClockSampler:
