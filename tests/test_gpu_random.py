@@ -70,3 +70,77 @@ def test_random_layer_matches_oracle(cuda_ok, seed):
     check_output_elementwise(to_np(got["out"]), ref, case)
     dropped = (ref.dest.reshape(w.T, w.k) < 0).all(axis=1)
     assert (to_np(got["out"])[dropped] == 0).all()
+
+
+def _random_variant(seed, kind):
+    rng = np.random.default_rng(5000 + seed)
+    E = int(rng.choice([2, 3, 4, 6, 8, 12, 16]))
+    k = int(rng.integers(1, min(E, 4) + 1))
+    T = int(rng.integers(1, 500))
+    d = 64 * int(rng.integers(1, 5))
+    F = 64 * int(rng.integers(1, 5))
+    return syn.Workload(f"random-{kind}-{seed}", T=T, d=d, E=E, k=k, F=F, zipf_s=float(rng.choice([0.0, 1.0, 2.0])),
+                        capacity_factor=float(rng.uniform(0.2, 2.0)), expert_choice=(kind == "ec"),
+                        reroute=(kind == "reroute"))
+
+
+def _ec_bound(hp, ec, wd, T, d):
+    a = np.zeros((hp.shape[0], d))
+    off = ec.segs.offsets
+    for e in range(len(ec.picks)):
+        if off[e + 1] > off[e]:
+            a[off[e]:off[e + 1]] = np.abs(hp[off[e]:off[e + 1]]) @ np.abs(oracle.f64(wd[e])).T
+    return 2.0 ** -7 * oracle.combine_expert_choice(a, ec.src, np.abs(ec.row_w), T)
+
+
+def _elementwise(got, ref, bound, what):
+    err = np.abs(np.asarray(got, dtype=np.float64) - ref)
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    assert np.isfinite(got).all(), what
+    assert not (err > bound + 1e-7 * max(rms, 1e-30)).any(), f"{what}: elements above the bound"
+    denom = float(np.abs(ref).sum())
+    if denom > 0:
+        assert float(err.sum()) / denom <= 5e-3, what
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_expert_choice(cuda_ok, seed):
+    """Random shapes with expert-choice routing: the selection bit for bit, the rest in tolerance."""
+    w = _random_variant(seed, "ec")
+    case = make_case(w, seed=seed)
+    C = oracle.capacity_rows(w.capacity_factor, w.T, w.k, w.E)
+    logits, ec, xp, hp, yp, out = oracle.expert_choice_forward(case.x, case.w_r, case.bias, case.wg, case.wu,
+                                                                case.wd, C)
+    got = run_layer(case)
+    assert got["status"] == 0
+    assert (got["src"].numpy() == ec.src).all()
+    assert (got["emap"].numpy() == oracle.expert_choice_map(ec, w.T)).all()
+    assert (to_np(got["xp"]) == xp).all()
+    check_bf16_storage(to_np(got["hp"]), hp, "Hp")
+    _elementwise(to_np(got["out"]), out, _ec_bound(hp, ec, case.wd, w.T, w.d), "out")
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_reroute(cuda_ok, seed):
+    """Random shapes with overflow re-routing: the placement bit for bit, the rest in tolerance."""
+    w = _random_variant(seed, "reroute")
+    case = make_case(w, seed=seed)
+    C = oracle.capacity_rows(w.capacity_factor, w.T, w.k, w.E)
+    logits, ids, wts, rr, segs, dest, src, xp, hp, yp, out = oracle.layer_forward_reroute(
+        case.x, case.w_r, case.bias, case.wg, case.wu, case.wd, w.k, C)
+    got = run_layer(case)
+    assert got["status"] == 0
+    assert (got["ids"].numpy() == ids).all()
+    assert (got["seg_offsets"].numpy() == segs.offsets).all()
+    assert (got["dest"].numpy() == dest).all()
+    used = int(segs.offsets[-1])
+    assert (got["src"].numpy()[:used] == src).all()
+    assert (to_np(got["xp"][:used]) == xp).all()
+    check_bf16_storage(to_np(got["hp"][:used]), hp, "Hp")
+    a = np.zeros((used, w.d))
+    off = segs.offsets
+    for e in range(w.E):
+        if off[e + 1] > off[e]:
+            a[off[e]:off[e + 1]] = np.abs(hp[off[e]:off[e + 1]]) @ np.abs(oracle.f64(case.wd[e])).T
+    bound = 2.0 ** -7 * oracle.combine(a, dest, np.abs(wts), w.T, w.k)
+    _elementwise(to_np(got["out"]), out, bound, "out")
