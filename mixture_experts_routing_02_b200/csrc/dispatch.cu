@@ -1,24 +1,29 @@
-// Dispatch kernels: histogram, segment tables (plain or balanced plan), the stable
-// rank of every (token, k) pair inside its expert, and the scatter that writes each
-// token row straight into its k final expert-contiguous slots.
+// Dispatch kernels: expert counts, segment tables (plain, capacity, balanced plan or overflow
+// re-routing), the stable rank of every (token, k) pair inside its expert, and the copies that
+// write each token row straight into its k final expert-contiguous slots.
 //
-// The permutation is a counting sort on the expert id with one digit pass: the
-// global histogram is known beforehand (histogram_kernel), and the rank of a
-// pair inside its expert is (pairs of that expert in earlier tiles) + (earlier
-// pairs of the same tile).  The first term is an exclusive prefix over tiles,
-// found with a decoupled look-back (Merrill & Garland, "Single-pass Parallel
-// Prefix Scan with Decoupled Look-back", 2016): each tile publishes its own
-// per-expert counts at once and its inclusive prefix as soon as it knows it,
-// so a tile only waits for tiles already running.  Tiles are taken in order
-// from an atomic ticket, which guarantees that every tile a CTA waits for is
-// held by a CTA that is running.  Every wait is bounded.
+// The permutation is a counting sort on the expert id with one digit pass: the rank of a pair
+// inside its expert is (pairs of that expert before its block) + (earlier pairs of the same
+// block).  Three ways to get the first term:
+//   * dispatch_count_kernel (plain / capacity, up to kCountMaxPairs pairs): every CTA counts all
+//     ids itself, so no CTA waits for another and one launch does counts, tables, ranks and
+//     copies;
+//   * dispatch_fused_kernel (plain / capacity, any size) and rank_kernel (balanced plan, or
+//     tables given): an exclusive prefix over tiles found with a decoupled look-back (Merrill &
+//     Garland, "Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016): each tile
+//     publishes its own per-expert counts at once and its inclusive prefix as soon as it knows
+//     it, so a tile only waits for tiles already running.  Tiles are taken in order from an
+//     atomic ticket, which guarantees that every tile a CTA waits for is held by a CTA that is
+//     running;
+//   * reroute_kernel (overflow re-routing): one CTA ranks the pairs and then runs the rounds.
+// Every wait is bounded.
 //
 // Sources: "Sparsely-Gated MoE 구현 관점에서 살펴보기", section "순전파 과정 ..."
-// (permute tokens into expert order); "5.3 Expert Parallelism", section
-// "2. 디스패처 엔지니어링" (bincount per destination); the MoonEP page, sections
-// "이 기술은 무엇인가" (rows written to their final slot, no separate sort and
-// copy; static shapes, no host sync) and "설치 및 통합" (tokens_per_expert,
-// cu_seqlens).
+// (permute tokens into expert order) and "로드 밸런싱 손실(load-balancing loss)과 용량(capacity)은
+// 별개" (capacity; overflow dropped or sent to another candidate); "5.3 Expert Parallelism",
+// section "2. 디스패처 엔지니어링" (bincount per destination); the MoonEP page, sections
+// "이 기술은 무엇인가" (rows written to their final slot, no separate sort and copy; static
+// shapes, no host sync) and "설치 및 통합" (tokens_per_expert, cu_seqlens).
 #include "common.cuh"
 #include "kernels.h"
 
