@@ -239,11 +239,11 @@ MOE_API moe_status_t moe_plan_balanced(const moe_shape_t *shape, const int32_t *
 
 /*
  * Dispatch.  When plan_ready == 0 this computes counts
- * and the segment tables first (moe_histogram, then moe_plan_balanced if
+ * and the segment tables first (as moe_histogram, then moe_plan_balanced if
  * n_groups > 0 else moe_segments), writing them to the given buffers; when
- * plan_ready != 0 they are inputs from earlier calls.  Then, with a decoupled
- * look-back over tiles of (t, j) pairs, each pair gets its stable rank r
- * inside its expert and its final row
+ * plan_ready != 0 they are inputs from earlier calls.  Each pair gets its
+ * stable rank r inside its expert (pairs in q = t*k + j order) and its final
+ * row
  *   dest[t*k+j] = seg_offsets[s] + r - seg_first_rank[s]
  * for the segment s of that expert covering rank r (-1 if none: dropped), and
  * the token's row is copied straight to that slot ("MoonEP", section "이 기술은
@@ -254,6 +254,10 @@ MOE_API moe_status_t moe_plan_balanced(const moe_shape_t *shape, const int32_t *
  *   xp [rows_alloc, d] bf16 out (rows past seg_offsets[n_seg] untouched).
  *   ws, ws_bytes: at least moe_workspace_size()'s dispatch_bytes of device
  *   memory; its contents need not be initialised and are clobbered.
+ * Kernels: with plan_ready == 0 and no plan, one launch (T*k <= 65536: every
+ * CTA counts all ids itself; above: a memset and one launch with a decoupled
+ * look-back over tiles of pairs); with a plan or given tables, the histogram,
+ * the plan, the look-back ranks and the row copies as separate launches.
  */
 MOE_API moe_status_t moe_dispatch(const moe_shape_t *shape, const moe_bf16_t *x, const int32_t *topk_ids,
                           int32_t plan_ready, int32_t *counts, int32_t *seg_expert,
