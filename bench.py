@@ -381,7 +381,7 @@ def run_ours(args, w):
     route_ws_bytes = moe.moe_route_workspace_size(s)
     route_ws = torch.empty(max(route_ws_bytes, 256), dtype=torch.uint8, device=dev) if route_ws_bytes else None
     launches = ((2 if route_ws_bytes else 1)                                   # route (+ partial sums)
-                + (2 if ec or rr else (4 if w.n_groups else 1))                # dispatch
+                + (2 if ec or rr else (4 if w.n_groups and w.T * w.k > (1 << 20) else 1))  # dispatch
                 + 3)                                                           # gate_up, down, combine
 
     Fs = args.shared_expert

@@ -254,10 +254,11 @@ MOE_API moe_status_t moe_plan_balanced(const moe_shape_t *shape, const int32_t *
  *   xp [rows_alloc, d] bf16 out (rows past seg_offsets[n_seg] untouched).
  *   ws, ws_bytes: at least moe_workspace_size()'s dispatch_bytes of device
  *   memory; its contents need not be initialised and are clobbered.
- * Kernels: with plan_ready == 0 and no plan, one launch (T*k <= 65536: every
- * CTA counts all ids itself; above: a memset and one launch with a decoupled
- * look-back over tiles of pairs); with a plan or given tables, the histogram,
- * the plan, the look-back ranks and the row copies as separate launches.
+ * Kernels: with plan_ready == 0, one launch (no plan and T*k <= 65536, or a
+ * plan and T*k <= 2^20: every CTA counts all ids itself and computes the
+ * tables; no plan and larger: a memset and one launch with a decoupled
+ * look-back over tiles of pairs); otherwise the histogram, the plan, the
+ * look-back ranks and the row copies as separate launches.
  */
 MOE_API moe_status_t moe_dispatch(const moe_shape_t *shape, const moe_bf16_t *x, const int32_t *topk_ids,
                           int32_t plan_ready, int32_t *counts, int32_t *seg_expert,

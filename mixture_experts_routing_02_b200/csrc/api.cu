@@ -340,13 +340,16 @@ moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* id
     a.rows = v.rows;
     a.first_tile = first_tile;
     a.n_tiles = permute_n_tiles(v.T, v.k);
-    if (!plan_ready && v.R == 0 && a.n_tiles > 0) {
-        // histogram, tables, ranks and row copies in one launch
+    const int64_t pairs = static_cast<int64_t>(v.T) * v.k;
+    if (!plan_ready && a.n_tiles > 0 &&
+        (v.R == 0 || (pairs <= kCountMaxPairsPlan && first_tile == 0))) {
+        // counts, tables, ranks and row copies in one launch
         a.capacity = v.C;
         a.counts = counts; a.seg_expert_out = seg_expert; a.seg_offsets_out = seg_offsets;
         a.seg_first_rank_out = seg_first_rank;
         a.prefetch_x = static_cast<size_t>(v.T) * v.d * 2 <= (size_t(48) << 20);
-        if (static_cast<int64_t>(v.T) * v.k <= kCountMaxPairs && first_tile == 0)
+        a.R = v.R; a.S = v.S; a.B = v.B;
+        if (v.R > 0 || (pairs <= kCountMaxPairs && first_tile == 0))
             return cuda_status(launch_dispatch_count(a, sm_count(), st));
         return cuda_status(launch_dispatch_fused(a, sm_count(), st));
     }

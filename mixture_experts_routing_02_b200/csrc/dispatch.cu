@@ -5,9 +5,9 @@
 // The permutation is a counting sort on the expert id with one digit pass: the rank of a pair
 // inside its expert is (pairs of that expert before its block) + (earlier pairs of the same
 // block).  Three ways to get the first term:
-//   * dispatch_count_kernel (plain / capacity, up to kCountMaxPairs pairs): every CTA counts all
-//     ids itself, so no CTA waits for another and one launch does counts, tables, ranks and
-//     copies;
+//   * dispatch_count_kernel (plain / capacity up to kCountMaxPairs pairs, balanced plan up to
+//     kCountMaxPairsPlan): every CTA counts all ids itself (and computes the plan from the
+//     totals), so no CTA waits for another and one launch does counts, tables, ranks and copies;
 //   * dispatch_fused_kernel (plain / capacity, any size) and rank_kernel (balanced plan, or
 //     tables given): an exclusive prefix over tiles found with a decoupled look-back (Merrill &
 //     Garland, "Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016): each tile
@@ -147,119 +147,163 @@ __global__ void __launch_bounds__(256) segments_kernel(int32_t* counts, const in
 
 constexpr int kMaxGroups = 256;
 
-__global__ void __launch_bounds__(256) plan_kernel(int32_t* counts, const int32_t* partials, int n_partials, int E,
-                                                   int R, int S, int k, int B, int32_t* seg_expert,
-                                                   int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* status) {
-    __shared__ int c[kMaxExperts];
-    __shared__ int order[kMaxExperts];  // experts of each group by (count desc, id asc)
-    __shared__ int given[kMaxExperts];  // rows an expert hands to other groups
-    __shared__ int next_rank[kMaxExperts];
-    __shared__ int qe[kMaxExperts], qn[kMaxExperts];  // the donor queue
-    __shared__ int load[kMaxGroups];
-    __shared__ int n_slots[kMaxGroups];
-    __shared__ int slot_e[kMaxSegments], slot_n[kMaxSegments], slot_r[kMaxSegments];
-    __shared__ int seg_len[kMaxSegments];
-    __shared__ int warp_sums[8];
-    __shared__ int infeasible;
+// Exclusive scan over the threads of a block (any multiple of 32 up to 1024); *total = the sum.
+// warp_sums: 33 ints.  Ends with a barrier.
+__device__ __forceinline__ int block_exclusive_scan_any(int v, int* warp_sums, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += t;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        const int w0 = lane < nwarps ? warp_sums[lane] : 0;
+        int w = w0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += t;
+        }
+        __syncwarp();
+        if (lane < nwarps) warp_sums[lane] = w - w0;
+        if (lane == 31) warp_sums[32] = w;
+    }
+    __syncthreads();
+    const int r = warp_sums[warp] + x - v;
+    if (total != nullptr) *total = warp_sums[32];
+    __syncthreads();
+    return r;
+}
 
+// Shared memory of the balanced plan.
+struct PlanSmem {
+    int c[kMaxExperts];          // rows of each expert (filled by the caller)
+    int order[kMaxExperts];      // experts of each group by (count desc, id asc)
+    int given[kMaxExperts];      // rows an expert hands to other groups
+    int next_rank[kMaxExperts];
+    int qe[kMaxExperts], qn[kMaxExperts];  // the donor queue
+    int load[kMaxGroups];
+    int n_slots[kMaxGroups];
+    int slot_e[kMaxSegments], slot_n[kMaxSegments], slot_r[kMaxSegments];
+    int seg_len[kMaxSegments];
+    int warp_sums[33];
+    int infeasible;
+};
+
+// The greedy balanced plan from sm.c (written by the caller before a barrier) into the segment
+// tables (any memory).  Called by the whole block; the greedy itself runs on one thread.  An
+// infeasible plan (a group needs more than B replica slots) writes every segment empty and, if
+// report_status, sets MOE_DEV_ERR_PLAN.
+__device__ void compute_plan(PlanSmem& sm, int E, int R, int S, int k, int B, int* seg_expert, int* seg_offsets,
+                             int* seg_first_rank, int32_t* status, bool report_status) {
     const int tid = threadIdx.x;
     const int epg = E / R;
     const int per_group = epg + B;
     const int n_seg = R * per_group;
     const int cap = S * k;
 
-    for (int e = tid; e < E; e += blockDim.x) {
-        c[e] = expert_count(counts, partials, n_partials, E, e, counts);
-        given[e] = 0;
-    }
-    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) sm.given[e] = 0;
     for (int g = tid; g < R; g += blockDim.x) {
         int s = 0;
-        for (int e = g * epg; e < (g + 1) * epg; ++e) s += c[e];
-        load[g] = s;
+        for (int e = g * epg; e < (g + 1) * epg; ++e) s += sm.c[e];
+        sm.load[g] = s;
     }
     for (int e = tid; e < E; e += blockDim.x) {
         const int g = e / epg;
         int rank = 0;
-        for (int o = g * epg; o < (g + 1) * epg; ++o) rank += (c[o] > c[e]) || (c[o] == c[e] && o < e);
-        order[g * epg + rank] = e;
+        for (int o = g * epg; o < (g + 1) * epg; ++o) rank += (sm.c[o] > sm.c[e]) || (sm.c[o] == sm.c[e] && o < e);
+        sm.order[g * epg + rank] = e;
     }
     __syncthreads();
 
     if (tid == 0) {
         // the queue of excess rows, groups ascending, experts by (count desc, id asc)
         int nq = 0, total = 0;
-        for (int g = 0; g < R; ++g) total += load[g];
+        for (int g = 0; g < R; ++g) total += sm.load[g];
         int bad = (total != R * cap);
         for (int g = 0; g < R; ++g) {
-            int excess = load[g] - cap;
+            int excess = sm.load[g] - cap;
             for (int i = 0; i < epg && excess > 0; ++i) {
-                const int e = order[g * epg + i];
-                const int take = c[e] < excess ? c[e] : excess;
-                if (take > 0) { given[e] = take; qe[nq] = e; qn[nq] = take; ++nq; excess -= take; }
+                const int e = sm.order[g * epg + i];
+                const int take = sm.c[e] < excess ? sm.c[e] : excess;
+                if (take > 0) { sm.given[e] = take; sm.qe[nq] = e; sm.qn[nq] = take; ++nq; excess -= take; }
             }
         }
         // groups below the cap, ascending, take from the front of the queue
         int head = 0;
         for (int g = 0; g < R; ++g) {
-            int deficit = cap - load[g];
+            int deficit = cap - sm.load[g];
             int ns = 0;
             while (deficit > 0 && head < nq) {
-                const int take = qn[head] < deficit ? qn[head] : deficit;
-                if (ns < B) { slot_e[g * B + ns] = qe[head]; slot_n[g * B + ns] = take; }
+                const int take = sm.qn[head] < deficit ? sm.qn[head] : deficit;
+                if (ns < B) { sm.slot_e[g * B + ns] = sm.qe[head]; sm.slot_n[g * B + ns] = take; }
                 ++ns;
-                qn[head] -= take;
+                sm.qn[head] -= take;
                 deficit -= take;
-                if (qn[head] == 0) ++head;
+                if (sm.qn[head] == 0) ++head;
             }
             if (ns > B || deficit > 0) bad = 1;
-            n_slots[g] = ns < B ? ns : B;
+            sm.n_slots[g] = ns < B ? ns : B;
         }
         // within-expert rank at which each piece starts: after the home rows, in creation order
-        for (int e = 0; e < E; ++e) next_rank[e] = c[e] - given[e];
+        for (int e = 0; e < E; ++e) sm.next_rank[e] = sm.c[e] - sm.given[e];
         for (int g = 0; g < R; ++g)
-            for (int i = 0; i < n_slots[g]; ++i) {
+            for (int i = 0; i < sm.n_slots[g]; ++i) {
                 const int idx = g * B + i;
-                slot_r[idx] = next_rank[slot_e[idx]];
-                next_rank[slot_e[idx]] += slot_n[idx];
+                sm.slot_r[idx] = sm.next_rank[sm.slot_e[idx]];
+                sm.next_rank[sm.slot_e[idx]] += sm.slot_n[idx];
             }
-        infeasible = bad;
-        if (bad) report(status, MOE_DEV_ERR_PLAN);
+        sm.infeasible = bad;
+        if (bad && report_status) report(status, MOE_DEV_ERR_PLAN);
     }
     __syncthreads();
 
-    const bool bad = infeasible != 0;
+    const bool bad = sm.infeasible != 0;
     for (int s = tid; s < n_seg; s += blockDim.x) {
         const int g = s / per_group, i = s - g * per_group;
         int ex = -1, len = 0, fr = 0;
         if (!bad) {
             if (i < epg) {
                 ex = g * epg + i;
-                len = c[ex] - given[ex];
-            } else if (i - epg < n_slots[g]) {
+                len = sm.c[ex] - sm.given[ex];
+            } else if (i - epg < sm.n_slots[g]) {
                 const int idx = g * B + (i - epg);
-                ex = slot_e[idx];
-                len = slot_n[idx];
-                fr = slot_r[idx];
+                ex = sm.slot_e[idx];
+                len = sm.slot_n[idx];
+                fr = sm.slot_r[idx];
             }
         }
         seg_expert[s] = ex;
         seg_first_rank[s] = fr;
-        seg_len[s] = len;
+        sm.seg_len[s] = len;
     }
     __syncthreads();
     // offsets: exclusive scan of the lengths, each thread owning a contiguous chunk
     const int chunk = (n_seg + blockDim.x - 1) / blockDim.x;
     const int a = tid * chunk;
     int local = 0;
-    for (int s = a; s < a + chunk && s < n_seg; ++s) local += seg_len[s];
+    for (int s = a; s < a + chunk && s < n_seg; ++s) local += sm.seg_len[s];
     int total;
-    int run = block_exclusive_scan_256(local, warp_sums, &total);
+    int run = block_exclusive_scan_any(local, sm.warp_sums, &total);
     for (int s = a; s < a + chunk && s < n_seg; ++s) {
         seg_offsets[s] = run;
-        run += seg_len[s];
+        run += sm.seg_len[s];
     }
     if (tid == 0) seg_offsets[n_seg] = total;
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(256) plan_kernel(int32_t* counts, const int32_t* partials, int n_partials, int E,
+                                                   int R, int S, int k, int B, int32_t* seg_expert,
+                                                   int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* status) {
+    __shared__ PlanSmem sm;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) sm.c[e] = expert_count(counts, partials, n_partials, E, e, counts);
+    __syncthreads();
+    compute_plan(sm, E, R, S, k, B, seg_expert, seg_offsets, seg_first_rank, status, true);
 }
 
 // ------------------------------------------------------------------------------ stable rank + permute
@@ -607,7 +651,17 @@ __global__ void __launch_bounds__(kPermuteThreads, 4) dispatch_fused_kernel(cons
 //  2. ranks the pairs of its blocks in q order (match_any inside a warp, per-warp counts across
 //     warps), applies the capacity, writes dest and src (CTA 0 also writes counts and tables);
 //  3. copies each of its tokens' rows to the token's slots, one warp per token.
+// Dynamic shared memory of the count dispatch with a balanced plan: the plan, its segment tables
+// and each expert's segments (CSR by expert).
+struct CountPlanSmem {
+    PlanSmem plan;
+    int seg_e[kMaxSegments], seg_fr[kMaxSegments], seg_off[kMaxSegments + 1];
+    int cbeg[kMaxExperts + 1], cfill[kMaxExperts], cseg[kMaxSegments];
+};
+
+template <bool PLAN>
 __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const PermuteArgs a) {
+    extern __shared__ __align__(16) uint8_t count_dsmem[];
     __shared__ int s_a[kMaxExperts];    // pairs of each expert before the first block
     __shared__ int s_m[kMaxExperts];    // ... from the first block up to the second
     __shared__ int s_tot[kMaxExperts];  // ... from the second block on; then: all pairs
@@ -655,6 +709,55 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
     }
     __syncthreads();
 
+    CountPlanSmem& ps = *reinterpret_cast<CountPlanSmem*>(count_dsmem);
+    if (PLAN) {
+        // 2a. the balanced plan from the totals, computed by every CTA alike; CTA 0 publishes
+        // counts and the tables; each CTA keeps the segments of every expert (CSR)
+        for (int e = tid; e < E; e += blockDim.x) ps.plan.c[e] = s_a[e] + s_m[e] + s_tot[e];
+        __syncthreads();
+        compute_plan(ps.plan, E, a.R, a.S, k, a.B, ps.seg_e, ps.seg_off, ps.seg_fr, a.status, blockIdx.x == 0);
+        if (blockIdx.x == 0) {
+            for (int e = tid; e < E; e += blockDim.x) a.counts[e] = ps.plan.c[e];
+            for (int sg = tid; sg < a.n_seg; sg += blockDim.x) {
+                a.seg_expert_out[sg] = ps.seg_e[sg];
+                a.seg_offsets_out[sg] = ps.seg_off[sg];
+                a.seg_first_rank_out[sg] = ps.seg_fr[sg];
+            }
+            if (tid == 0) a.seg_offsets_out[a.n_seg] = ps.seg_off[a.n_seg];
+        }
+        for (int e = tid; e < E; e += blockDim.x) ps.cfill[e] = 0;
+        __syncthreads();
+        for (int sg = tid; sg < a.n_seg; sg += blockDim.x) {
+            const int ex = ps.seg_e[sg];
+            if (static_cast<unsigned>(ex) < static_cast<unsigned>(E) && ps.seg_off[sg + 1] > ps.seg_off[sg])
+                atomicAdd(&ps.cfill[ex], 1);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int carry = 0;
+            for (int e0 = 0; e0 < E; e0 += 32) {
+                const int e = e0 + lane;
+                const int v = e < E ? ps.cfill[e] : 0;
+                int x = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += t;
+                }
+                if (e < E) { ps.cbeg[e] = carry + x - v; ps.cfill[e] = carry + x - v; }
+                carry += __shfl_sync(0xffffffffu, x, 31);
+            }
+            if (lane == 0) ps.cbeg[E] = carry;
+        }
+        __syncthreads();
+        // segments in ascending index inside each expert (the order does not matter: ranges are disjoint)
+        for (int sg = tid; sg < a.n_seg; sg += blockDim.x) {
+            const int ex = ps.seg_e[sg];
+            if (static_cast<unsigned>(ex) < static_cast<unsigned>(E) && ps.seg_off[sg + 1] > ps.seg_off[sg])
+                ps.cseg[atomicAdd(&ps.cfill[ex], 1)] = sg;
+        }
+        __syncthreads();
+    } else {
     // 2a. segment offsets (capacity applied); CTA 0 publishes counts and the tables
     {
         const int tot = tid < E ? s_a[tid] + s_m[tid] + s_tot[tid] : 0;
@@ -690,6 +793,7 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
         }
         if (blockIdx.x == 0 && tid == 0) a.seg_offsets_out[E] = warp_sums[kCountWarps - 1];
     }
+    }
 
     // 2b. stable ranks of the pairs of each block, in chunks of blockDim.x pairs
 #pragma unroll 1
@@ -714,7 +818,15 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
                 if (e >= 0) {
                     int rk = s_run[e] + wrank;
                     for (int w = 0; w < warp; ++w) rk += s_wcnt[w][e];
-                    if (a.capacity == 0 || rk < a.capacity) {
+                    if (PLAN) {
+                        // the expert's segment holding rank rk (home rows, then replica pieces)
+                        for (int p = ps.cbeg[e]; p < ps.cbeg[e + 1]; ++p) {
+                            const int sg = ps.cseg[p];
+                            const int fr = ps.seg_fr[sg], off = ps.seg_off[sg], len = ps.seg_off[sg + 1] - off;
+                            if (rk >= fr && rk < fr + len) { dst = off + (rk - fr); break; }
+                        }
+                        if (dst >= a.rows) dst = -1;
+                    } else if (a.capacity == 0 || rk < a.capacity) {
                         dst = s_off[e] + rk;
                         if (dst >= a.rows) dst = -1;
                     }
@@ -1214,7 +1326,15 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
     if (a.T == 0) return cudaSuccess;
     int grid = num_sms;
     if (grid > a.T) grid = a.T;
-    dispatch_count_kernel<<<grid, kCountThreads, 0, stream>>>(a);
+    if (a.R > 0) {
+        const int smem = static_cast<int>(sizeof(CountPlanSmem));
+        const cudaError_t err = cudaFuncSetAttribute(dispatch_count_kernel<true>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (err != cudaSuccess) return err;
+        dispatch_count_kernel<true><<<grid, kCountThreads, smem, stream>>>(a);
+    } else {
+        dispatch_count_kernel<false><<<grid, kCountThreads, 0, stream>>>(a);
+    }
     return cudaGetLastError();
 }
 

@@ -82,6 +82,7 @@ struct PermuteArgs {
     int32_t* seg_first_rank_out;
     uint32_t* sync;            // [3] zero on entry: tiles ranked, tables ready, abort
     int prefetch_x;            // 1: prefetch the rows of X into L2 while the ranks are found
+    int R, S, B;               // balanced plan (count dispatch only): groups, tokens per group, slots
 };
 
 constexpr int kMaxHistogramPartials = 64;   // CTAs of the fused histogram (one partial count row each)
@@ -113,6 +114,7 @@ cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, c
 cudaError_t launch_dispatch_fused(const PermuteArgs& a, int num_sms, cudaStream_t stream);
 cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_t stream);
 constexpr int kCountMaxPairs = 1 << 16;
+constexpr int kCountMaxPairsPlan = 1 << 20;  // with a balanced plan the copies dwarf the recounting
 
 // Overflow re-routing (one CTA; T*k <= kCountMaxPairs), then the row copies.
 constexpr int kRerouteThreads = 1024;
