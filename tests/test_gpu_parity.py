@@ -222,6 +222,34 @@ def test_histogram_segments_and_plan_on_given_ids(sigma):
     assert (so2.cpu().numpy() == ref2.offsets).all() and (se2.cpu().numpy() == ref2.expert).all()
 
 
+def test_dispatch_large_balanced_plan():
+    """A balanced plan with more than 2^20 pairs takes the multi-launch path (histogram partials,
+    plan, look-back ranks, row copies): tables and positions bit for bit against the oracle."""
+    T, d, E, k, R, B = 140000, 64, 16, 8, 4, 4
+    ids = syn.lognormal_topk_ids(E, T, k, 1.0, seed=12).cuda()
+    s = moe.shape(T, d, E, k, 64, n_groups=R, replica_slots=B)
+    n_seg, rows = moe.moe_layout(s)
+    disp, _ = moe.moe_workspace_size(s)
+    x = torch.randn(T, d, generator=torch.Generator().manual_seed(13)).to(torch.bfloat16)
+    counts, se, so, sf, dest, src = i32(E), i32(n_seg), i32(n_seg + 1), i32(n_seg), i32(T * k), i32(rows)
+    xp = torch.zeros(rows, d, dtype=torch.bfloat16, device="cuda")
+    st = i32(1)
+    moe.moe_dispatch(s, x.cuda(), ids, 0, counts, se, so, sf, dest, src, xp, st,
+                     torch.empty(disp, dtype=torch.uint8, device="cuda"))
+    torch.cuda.synchronize()
+    ids_np = ids.view(T, k).cpu().numpy()
+    rc = oracle.histogram(ids_np, E)
+    segs, _ = oracle.balanced_plan(rc, R, T // R, k, B)
+    rdest, rsrc = oracle.dispatch_positions(ids_np, segs, E)
+    assert st.item() == 0
+    assert (counts.cpu().numpy() == rc).all()
+    assert (se.cpu().numpy() == segs.expert).all() and (so.cpu().numpy() == segs.offsets).all()
+    assert (sf.cpu().numpy() == segs.first_rank).all()
+    assert (dest.cpu().numpy() == rdest).all()
+    assert (src.cpu().numpy() == rsrc).all()
+    assert torch.equal(xp.cpu(), x[torch.from_numpy(rsrc // k)])
+
+
 def test_dispatch_with_given_plan_tables():
     """plan_ready = 1: the permutation alone, on counts and tables from the oracle."""
     E, R, S, k, B, d = 32, 4, 200, 4, 8, 128
