@@ -510,6 +510,11 @@ __global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs
 // in flight per lane).  Slots outside [0, rows) are skipped.
 __device__ __forceinline__ void copy_row(const __nv_bfloat16* __restrict__ x, int t, const int* dj, int k, int d,
                                          int rows, __nv_bfloat16* __restrict__ xp, int lane) {
+    // a token whose pairs were all dropped is not read at all (dj is the same in every lane)
+    bool any = false;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) any |= (j < k && dj[j] >= 0 && dj[j] < rows);
+    if (!any) return;
     const int vec_per_row = d / 8;
     const uint4* xs = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
     for (int v = lane; v < vec_per_row; v += 32 * kCopyUnroll) {
