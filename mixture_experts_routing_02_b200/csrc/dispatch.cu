@@ -849,11 +849,12 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
         }
     }
 
-    // 3. rows of this CTA's tokens to their slots
-#pragma unroll 1
-    for (int r = 0; r < 2; ++r) {
-        if (r == 1 && tb_[1] == tb_[0]) break;
-        for (int t = tb_[r] + warp; t < te_[r]; t += kCountWarps) {
+    // 3. rows of this CTA's tokens to their slots: both blocks form one list over all warps
+    {
+        const int n0 = te_[0] - tb_[0];
+        const int n1 = tb_[1] == tb_[0] ? 0 : te_[1] - tb_[1];
+        for (int i = warp; i < n0 + n1; i += kCountWarps) {
+            const int t = i < n0 ? tb_[0] + i : tb_[1] + (i - n0);
             const int mine = lane < k ? a.dest[static_cast<size_t>(t) * k + lane] : -1;
             int dj[kMaxTopK];
 #pragma unroll
