@@ -314,6 +314,8 @@ MOE_API moe_status_t moe_expert_gate_up(const moe_shape_t *shape, const moe_bf16
  * stored in fp32 (Yp is only read by the combine; keeping it in fp32 leaves
  * one rounding, the bf16 Hp operand, between the expert and the output).
  *   hp [rows_alloc, F] bf16; w_down [E, d, F] bf16; yp [rows_alloc, d] fp32 out.
+ * When segments average at least 192 rows and d_ff <= 4096, it runs on CTA pairs
+ * (tcgen05 cta_group::2, 256-row tiles); otherwise on single CTAs (128-row tiles).
  */
 MOE_API moe_status_t moe_expert_down(const moe_shape_t *shape, const moe_bf16_t *hp,
                              const int32_t *seg_expert, const int32_t *seg_offsets,
@@ -368,11 +370,13 @@ MOE_API moe_status_t moe_shared_expert(const moe_shape_t *shape, int32_t d_ff_sh
                                int32_t *status, moe_stream_t stream);
 
 /*
- * The whole layer: moe_route (logits not stored) -> moe_dispatch ->
+ * The whole layer: moe_route_ws (logits not stored) -> moe_dispatch ->
  * moe_expert_gate_up -> moe_expert_down -> moe_combine, all on `stream`.
- * With MOE_ROUTE_EXPERT_CHOICE: moe_route_scores -> moe_expert_choose ->
+ * With MOE_ROUTE_EXPERT_CHOICE: moe_route_scores_ws -> moe_expert_choose ->
  * moe_expert_gate_up -> moe_expert_down -> moe_combine_expert_choice; the
  * views topk_ids, topk_w, dest, seg_first_rank and dispatch_ws are then unused.
+ * With MOE_ROUTE_REROUTE the dispatch is moe_dispatch_reroute (the logits are
+ * then kept in the workspace).
  * out [T, d] fp32.  The intermediates live in `ws` (moe_workspace_size()'s
  * layer_bytes); their addresses are given by moe_layer_views.
  */
