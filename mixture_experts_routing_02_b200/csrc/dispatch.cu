@@ -655,7 +655,8 @@ __global__ void __launch_bounds__(kPermuteThreads, 4) dispatch_fused_kernel(cons
 //     repeated by every CTA; it reads T*k ids from L2, which is why it is limited to small T*k);
 //  2. ranks the pairs of its blocks in q order (match_any inside a warp, per-warp counts across
 //     warps), applies the capacity, writes dest and src (CTA 0 also writes counts and tables);
-//  3. copies each of its tokens' rows to the token's slots, one warp per token.
+//  3. copies each of its tokens' rows to the token's slots, one warp per token, the two blocks
+//     forming one list over all warps (a token whose pairs were all dropped is not read).
 // Dynamic shared memory of the count dispatch with a balanced plan: the plan, its segment tables
 // and each expert's segments (CSR by expert).
 struct CountPlanSmem {
