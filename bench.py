@@ -326,7 +326,9 @@ def run_ours(args, w):
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+        # every rank does the same set-up and steps, so the barriers are reached within seconds of
+        # each other; a rank that fails makes the others' next barrier end with an error in 2 min
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     moe.load_library()
     dev = torch.device("cuda", local)
