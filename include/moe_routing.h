@@ -501,6 +501,46 @@ typedef struct {
     float *logits;           /* [T, E] router logits (MOE_ROUTE_REROUTE only, else NULL) */
 } moe_layer_views_t;
 
+/*
+ * Routing statistics of one dispatch (top-k modes), for monitoring the routing
+ * distribution ("Expert를 똑같이 나눴는데도 GPU가 대기하는 이유", section "라우팅 분포와
+ * 학습 안정성": per-expert token counts, dropped tokens) and the balanced plan
+ * (MoonEP page, "실제 실험 결과": busiest group against the mean, migrated tokens,
+ * replica slots in use).  One small kernel; nothing returns to the host.
+ *   counts [E]: the raw per-expert counts the dispatch wrote (nullable: the
+ *   values that need them are then -1); seg_expert [n_seg], seg_offsets
+ *   [n_seg + 1]: its segment tables (e.g. the moe_layer_views of a layer run).
+ *   stats [MOE_STAT_COUNT] int32 out (device):
+ *     MOE_STAT_PAIRS             T * k
+ *     MOE_STAT_ROWS              rows placed (seg_offsets[n_seg])
+ *     MOE_STAT_DROPPED           pairs not placed (capacity, re-routing with no room)
+ *     MOE_STAT_MAX_EXPERT_LOAD   max over experts of counts[e]
+ *     MOE_STAT_ACTIVE_EXPERTS    experts with counts[e] > 0
+ *     MOE_STAT_MAX_SEGMENT_ROWS  rows of the longest segment (the longest GEMM)
+ *     MOE_STAT_MAX_GROUP_LOAD    with a plan: max over groups of the counts of its home
+ *                                experts (before the plan; the mean is T*k/R); else as
+ *                                MOE_STAT_MAX_EXPERT_LOAD
+ *     MOE_STAT_MAX_GROUP_ROWS    with a plan: max over groups of the rows it computes
+ *                                (S*k for a feasible plan); else as MOE_STAT_MAX_SEGMENT_ROWS
+ *     MOE_STAT_MIGRATED_ROWS     rows in replica segments (computed outside the home group)
+ *     MOE_STAT_REPLICAS_USED     replica segments holding rows
+ * MOE_ERR_INVALID_ARG for expert-choice shapes and null tables.
+ */
+#define MOE_STAT_PAIRS 0
+#define MOE_STAT_ROWS 1
+#define MOE_STAT_DROPPED 2
+#define MOE_STAT_MAX_EXPERT_LOAD 3
+#define MOE_STAT_ACTIVE_EXPERTS 4
+#define MOE_STAT_MAX_SEGMENT_ROWS 5
+#define MOE_STAT_MAX_GROUP_LOAD 6
+#define MOE_STAT_MAX_GROUP_ROWS 7
+#define MOE_STAT_MIGRATED_ROWS 8
+#define MOE_STAT_REPLICAS_USED 9
+#define MOE_STAT_COUNT 10
+MOE_API moe_status_t moe_routing_stats(const moe_shape_t *shape, const int32_t *counts,
+                               const int32_t *seg_expert, const int32_t *seg_offsets,
+                               int32_t *stats, moe_stream_t stream);
+
 /* Fill *views with the addresses inside a layer workspace `ws`. Host only. */
 MOE_API moe_status_t moe_layer_views(const moe_shape_t *shape, void *ws, moe_layer_views_t *views);
 

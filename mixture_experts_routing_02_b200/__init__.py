@@ -20,7 +20,7 @@ __all__ = [
     "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_combine_add", "moe_shared_expert", "moe_layer_fwd",
     "moe_route_scores", "moe_expert_choose", "moe_combine_expert_choice",
     "moe_route_workspace_size", "moe_route_ws", "moe_route_scores_ws", "moe_dispatch_reroute",
-    "moe_layer_views",
+    "moe_layer_views", "moe_routing_stats", "STAT_NAMES",
     "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT", "ROUTE_SOFTMAX_ALL", "ROUTE_EXPERT_CHOICE", "ROUTE_REROUTE",
 ]
 
@@ -79,7 +79,12 @@ SYMBOLS = {
     "moe_route_ws": [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_route_scores_ws": [_S, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_dispatch_reroute": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "moe_routing_stats": [_S, _P, _P, _P, _P, _P],
 }
+
+# order of the values moe_routing_stats writes (MOE_STAT_* in the header)
+STAT_NAMES = ("pairs", "rows", "dropped", "max_expert_load", "active_experts", "max_segment_rows",
+              "max_group_load", "max_group_rows", "migrated_rows", "replicas_used")
 
 _lib = None
 
@@ -288,3 +293,9 @@ def moe_dispatch_reroute(s, x, topk_ids, logits, counts, seg_expert, seg_offsets
     _check("moe_dispatch_reroute", load_library().moe_dispatch_reroute(
         ctypes.byref(s), _ptr(x), _ptr(topk_ids), _ptr(logits), _ptr(counts), _ptr(seg_expert), _ptr(seg_offsets),
         _ptr(seg_first_rank), _ptr(dest), _ptr(src), _ptr(xp), _ptr(status), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def moe_routing_stats(s, counts, seg_expert, seg_offsets, stats, stream=None):
+    """stats: int32 CUDA tensor of len(STAT_NAMES) values (see the header for their meaning)."""
+    _check("moe_routing_stats", load_library().moe_routing_stats(
+        ctypes.byref(s), _ptr(counts), _ptr(seg_expert), _ptr(seg_offsets), _ptr(stats), _stream(stream)))

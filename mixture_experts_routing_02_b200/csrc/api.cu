@@ -736,6 +736,17 @@ moe_status_t moe_combine_expert_choice(const moe_shape_t* shape, const float* yp
                                          static_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_routing_stats(const moe_shape_t* shape, const int32_t* counts, const int32_t* seg_expert,
+                               const int32_t* seg_offsets, int32_t* stats, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice keeps no per-pair counts
+    if (!seg_expert || !seg_offsets || !stats) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_routing_stats(counts, seg_expert, seg_offsets, v.E, v.n_seg, v.R, v.B, v.T * v.k,
+                                            stats, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_layer_views(const moe_shape_t* shape, void* ws, moe_layer_views_t* views) {
     Dims v;
     const moe_status_t s = check_shape(shape, &v);

@@ -156,4 +156,8 @@ cudaError_t launch_ec_gather(const __nv_bfloat16* x, const int32_t* src, int row
 cudaError_t launch_ec_combine(const float* yp, const int32_t* emap, const float* row_w, const float* base, int T,
                               int E, int d, int rows, float* out, int num_sms, cudaStream_t stream);
 
+// stats.cu: MOE_STAT_COUNT values from the counts (nullable) and segment tables of one dispatch
+cudaError_t launch_routing_stats(const int32_t* counts, const int32_t* seg_expert, const int32_t* seg_offsets,
+                                 int E, int n_seg, int R, int B, int pairs, int32_t* stats, cudaStream_t stream);
+
 }  // namespace moe

@@ -180,3 +180,22 @@ def test_route_ws_checks_before_cuda(lib):
     assert lib.moe_route_ws(ctypes.byref(ec), fake, fake, None, None, fake, fake, None, None, 0, None) == 1
     assert lib.moe_route_scores_ws(ctypes.byref(_shape()), fake, fake, None, fake, None, None, 0, None) == 1
     assert lib.moe_route_ws(ctypes.byref(_shape()), None, fake, None, None, fake, fake, None, None, 0, None) == 1
+
+
+def test_routing_stats_checks_before_cuda(lib):
+    fake = ctypes.c_void_p(1 << 20)                  # never dereferenced: the checks come first
+    ec = _shape(route_flags=moe.ROUTE_EXPERT_CHOICE, capacity=16)
+    assert lib.moe_routing_stats(ctypes.byref(ec), fake, fake, fake, fake, None) == 1
+    s = _shape()
+    assert lib.moe_routing_stats(ctypes.byref(s), fake, None, fake, fake, None) == 1
+    assert lib.moe_routing_stats(ctypes.byref(s), fake, fake, None, fake, None) == 1
+    assert lib.moe_routing_stats(ctypes.byref(s), fake, fake, fake, None, None) == 1
+
+
+def test_stat_names_follow_the_header():
+    """The binding's value names are the header's MOE_STAT_* indices, in order."""
+    with open(os.path.join(ROOT, "include", "moe_routing.h")) as f:
+        found = dict(re.findall(r"#define MOE_STAT_(\w+) (\d+)", f.read()))
+    count = int(found.pop("COUNT"))
+    assert count == len(moe.STAT_NAMES)
+    assert {n.lower(): int(i) for n, i in found.items()} == {n: i for i, n in enumerate(moe.STAT_NAMES)}
