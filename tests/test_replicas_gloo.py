@@ -61,3 +61,26 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch):
 
     from mixture_experts_routing_02_b200 import synthetic as syn
     assert bench.run_reference(A, syn.TINY) == 0      # returns at once, no work, no output
+
+
+def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
+    """--impl reference on rank 0: the oracle timed on a bounded sample, one JSON line with the
+    keys the driver reads (no GPU needed)."""
+    import json
+    monkeypatch.delenv("RANK", raising=False)
+    monkeypatch.setenv("WORLD_SIZE", "1")
+
+    class A:
+        steps, warmup, seed, gpus = 1, 0, 0, 1
+
+    from mixture_experts_routing_02_b200 import synthetic as syn
+    assert bench.run_reference(A, syn.TINY) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s"
+    assert d["higher_is_better"] is True and d["vs_baseline"] is None and d["steps"] == 1
+    assert d["config"]["workload"] == "tiny"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
