@@ -602,3 +602,59 @@ def test_planted_mistakes_are_caught(monkeypatch, name, mutant, pins):
         except Exception:
             results.append(False)
     assert not all(results), f"planted mistake in {name} went unnoticed"
+
+
+# --------------------------------------------------------------------------- randomised sweeps
+
+def test_plan_invariants_random_shapes():
+    """The plan's invariants over random group counts, group sizes, replica budgets and skews:
+    exact S*k rows per group, every pair placed once in a segment of its expert, the minimum
+    number of migrated rows; an infeasible budget raises, and the same counts with B = E (room
+    for any piece list) plan."""
+    rng = np.random.default_rng(123)
+    planned = infeasible = 0
+    for _ in range(60):
+        R = int(rng.integers(1, 7))
+        E = R * int(rng.integers(1, 6))
+        k = int(rng.integers(1, min(E, 4) + 1))
+        S = int(rng.integers(1, 40))
+        B = int(rng.integers(0, 4))
+        sigma = float(rng.choice([0.0, 0.5, 1.5, 4.0]))
+        ids = syn.lognormal_topk_ids(E, R * S, k, sigma, seed=int(rng.integers(1 << 30))).numpy()
+        try:
+            ok, _, _ = _plan_check(ids, E, R, S, k, B)
+            assert ok
+            planned += 1
+        except oracle.PlanInfeasible:
+            infeasible += 1
+            ok, _, _ = _plan_check(ids, E, R, S, k, E)
+            assert ok
+    assert planned > 10 and infeasible > 0
+
+
+def test_dispatch_invariants_random_shapes():
+    """Stable counting-sort placement over random shapes and capacities: dest is a bijection onto
+    the kept rows, each segment holds its expert's first min(count, C) pairs in q order (the
+    positions of numpy's stable argsort), and dropped pairs are exactly the excess."""
+    rng = np.random.default_rng(321)
+    for _ in range(80):
+        E = int(rng.integers(1, 40))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        T = int(rng.integers(1, 300))
+        ids = syn.lognormal_topk_ids(E, T, k, float(rng.choice([0.0, 1.0, 3.0])),
+                                     seed=int(rng.integers(1 << 30))).numpy()
+        counts = oracle.histogram(ids, E)
+        C = int(rng.integers(0, 2 * T * k // E + 2))
+        segs = oracle.plain_segments(counts, C)
+        dest, src = oracle.dispatch_positions(ids, segs, E)
+        flat = ids.ravel()
+        order = np.argsort(flat, kind="stable")           # q order inside each expert
+        starts = np.concatenate([[0], np.cumsum(counts)])
+        off = segs.offsets
+        for e in range(E):
+            qs = order[starts[e]:starts[e + 1]]
+            keep = len(qs) if C == 0 else min(len(qs), C)
+            assert (dest[qs[:keep]] == off[e] + np.arange(keep)).all()
+            assert (dest[qs[keep:]] == -1).all()
+            assert (src[off[e]:off[e + 1]] == qs[:keep]).all()
+        assert int((dest < 0).sum()) == (0 if C == 0 else int(np.maximum(counts - C, 0).sum()))
