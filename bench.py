@@ -488,14 +488,16 @@ def run_ours(args, w):
     active_experts = int((torch.bincount(seg_e[seg_o[1:] > seg_o[:-1]].long().clamp_min(0),
                                          minlength=w.E) > 0).sum().item())
 
-    # timed region: K steps, events between every call
+    # timed region: K steps, events between every call.  Clocks are sampled through both timed
+    # regions (these steps and the end-to-end run below), which also gives a short step loop
+    # enough samples.
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     barrier()
-    with ClockSampler(local) as clocks:
-        for i in range(args.steps):
-            flush.zero_()
-            step(events[i])
-        barrier()
+    clocks = ClockSampler(local).__enter__()
+    for i in range(args.steps):
+        flush.zero_()
+        step(events[i])
+    barrier()
     per_kernel = {k: [] for k in KERNELS}
     step_ms = []
     for ev in events:
@@ -509,6 +511,7 @@ def run_ours(args, w):
     barrier()
     t0, t1 = e2e_run(e2e_steps)
     barrier()
+    clocks.__exit__(None, None, None)
     e2e_ms = t0.elapsed_time(t1)
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()}")

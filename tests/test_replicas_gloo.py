@@ -84,3 +84,31 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_clock_sampler_with_a_fake_nvml(monkeypatch):
+    """The bench's clock sampler, run against a fake NVML on the CPU: it samples on its own thread
+    while the timed work runs, reports the median SM clock and the throttle reasons it saw, and
+    only reads the GPU's settings (the fake has no setter to call)."""
+    import sys
+    import time
+    import types
+
+    clocks = iter([1965, 1500, 1400, 1500] + [1450] * 10000)
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByPciBusId=lambda bus: "gpu0",
+        nvmlDeviceGetMaxClockInfo=lambda h, kind: 1965,
+        nvmlDeviceGetClockInfo=lambda h, kind: next(clocks),
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x4,      # sw_power_cap
+    )
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    props = types.SimpleNamespace(pci_domain_id=0, pci_bus_id=0x1B, pci_device_id=0)
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda dev: props)
+    s = bench.ClockSampler(0).__enter__()
+    time.sleep(0.1)
+    s.__exit__(None, None, None)
+    out = s.summary()
+    assert out["samples"] >= 5 and out["sm_max_mhz"] == 1965
+    assert out["sm_mhz"] == 1450 and out["reasons"] == ["sw_power_cap"]
