@@ -199,3 +199,34 @@ def test_stat_names_follow_the_header():
     count = int(found.pop("COUNT"))
     assert count == len(moe.STAT_NAMES)
     assert {n.lower(): int(i) for n, i in found.items()} == {n: i for i, n in enumerate(moe.STAT_NAMES)}
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(lib, tmp_path):
+    """include/moe_routing.h compiles as strict C99, and a C program linked against the library
+    calls its host-only entry points (no Python, no torch)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "moe_routing.h"\n'
+        "int main(void) {\n"
+        "    moe_shape_t s = {64, 128, 8, 2, 256, 0, 0, 0, 0};\n"
+        "    int32_t n_seg = 0, rows = 0;\n"
+        "    size_t disp = 0, layer = 0;\n"
+        "    if (moe_layout(&s, &n_seg, &rows) != MOE_OK) return 1;\n"
+        "    if (moe_workspace_size(&s, &disp, &layer) != MOE_OK) return 2;\n"
+        "    s.top_k = 9;\n"
+        "    if (moe_layout(&s, &n_seg, &rows) != MOE_ERR_INVALID_ARG) return 3;\n"
+        '    printf("%d %d %zu %zu %s\\n", (int)n_seg, (int)rows, disp, layer, moe_status_string(MOE_ERR_WORKSPACE));\n'
+        "    return 0;\n}\n")
+    pkg = os.path.dirname(moe.LIB_PATH)
+    exe = tmp_path / "abi"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", pkg, "-lmoe_b200", "-Wl,-rpath," + pkg], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    disp, layer = moe.moe_workspace_size(_shape())
+    assert out[:4] == ["8", "128", str(disp), str(layer)]
+    assert out[4] == "MOE_ERR_WORKSPACE:"
