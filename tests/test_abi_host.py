@@ -46,6 +46,13 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(moe.SYMBOLS) <= names | {"moe_status_string"}
 
 
+def test_every_declared_symbol_has_a_binding_of_the_same_name():
+    names = _declared_symbols()
+    assert names == set(moe.SYMBOLS)
+    for name in names:
+        assert callable(getattr(moe, name, None)), f"{name} has no Python binding"
+
+
 def test_status_strings(lib):
     for code in range(5):
         assert moe.moe_status_string(code).startswith("MOE_")
