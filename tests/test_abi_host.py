@@ -237,3 +237,9 @@ def test_header_is_plain_c_and_the_library_links_from_c(lib, tmp_path):
     disp, layer = moe.moe_workspace_size(_shape())
     assert out[:4] == ["8", "128", str(disp), str(layer)]
     assert out[4] == "MOE_ERR_WORKSPACE:"
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No fallback: without the built library every call raises instead of computing elsewhere."""
+    with pytest.raises(RuntimeError, match="not built"):
+        moe.load_library(str(tmp_path / "libmoe_b200.so"))
