@@ -1,10 +1,13 @@
 """Randomised GPU-vs-oracle checks over many small shapes and seeds (the property
 tests of the parity plan): every combination of capacity / balanced plan / bias /
 routing variant, ragged T, d and F, E from 1 to 64 and k from 1 to min(E, 8).
-Each case runs the whole layer through moe_layer_fwd and compares every output; the
-layer output is held to a per-element bound derived from its bf16 rounding
-(gpu_cases.check_output_elementwise) because random cases include very heavy-tailed
-outputs (deep capacity drops with unrenormalised weights)."""
+Each case runs the whole layer through moe_layer_fwd and compares every output.  The
+layer output is held to the stated tolerance (max-abs <= 2e-2 * RMS of the reference,
+mean relative error <= 5e-3, over the rows of tokens that keep a pair; fully dropped
+tokens exactly 0) and, in addition, to a per-element bound derived from its one bf16
+rounding (gpu_cases.check_output_elementwise).  A seed whose output misses the stated
+tolerance is listed in CONTRACT_MISSES with its measured error and reported as an
+expected failure, never as a pass."""
 import numpy as np
 import pytest
 
@@ -12,9 +15,25 @@ import oracle
 import mixture_experts_routing_02_b200 as moe
 from mixture_experts_routing_02_b200 import synthetic as syn
 
-from gpu_cases import check_bf16_storage, check_output_elementwise, make_case, run_layer, to_np
+from gpu_cases import check_bf16_storage, check_close, check_layer_output, check_output_elementwise, make_case, \
+    run_layer, to_np
 
 pytestmark = pytest.mark.gpu
+
+# Random layers whose output misses max-abs <= 2e-2 * RMS(reference).  The only rounding on the
+# path is the bf16 Hp operand of the down projection; these cases combine deep capacity drops with
+# weights that are not renormalised, so a few large outputs sit far above the RMS of the kept rows.
+# Simulating that one rounding on the CPU gives the value quoted for each.
+CONTRACT_MISSES = {
+    17: "E=64, k=8, capacity factor 0.38 (most pairs dropped), softmax over all E without "
+        "renormalisation: max-abs error 2.30e-2 x RMS in a CPU simulation of the bf16 Hp rounding",
+}
+
+
+def _seeds(n):
+    return [pytest.param(s, marks=pytest.mark.xfail(reason="measured miss of the stated tolerance: " +
+                                                    CONTRACT_MISSES[s], strict=False))
+            if s in CONTRACT_MISSES else s for s in range(n)]
 
 
 def _random_workload(seed):
@@ -39,7 +58,7 @@ def _random_workload(seed):
                         n_groups=R, replica_slots=int(rng.integers(1, 6)) if R else 0), int(rng.integers(0, 2))
 
 
-@pytest.mark.parametrize("seed", range(24))
+@pytest.mark.parametrize("seed", _seeds(24))
 def test_random_layer_matches_oracle(cuda_ok, seed):
     w, flags = _random_workload(seed)
     case = make_case(w, seed=seed)
@@ -68,8 +87,8 @@ def test_random_layer_matches_oracle(cuda_ok, seed):
     assert (to_np(got["xp"][:used]) == ref.xp).all()
     check_bf16_storage(to_np(got["hp"][:used]), ref.hp, "Hp")
     check_output_elementwise(to_np(got["out"]), ref, case)
-    dropped = (ref.dest.reshape(w.T, w.k) < 0).all(axis=1)
-    assert (to_np(got["out"])[dropped] == 0).all()
+    # the stated tolerance, last: a listed miss has passed every check above it
+    check_layer_output(to_np(got["out"]), ref.out, ref.dest, w.T, w.k)
 
 
 def _random_variant(seed, kind):
@@ -118,6 +137,10 @@ def test_random_expert_choice(cuda_ok, seed):
     assert (to_np(got["xp"]) == xp).all()
     check_bf16_storage(to_np(got["hp"]), hp, "Hp")
     _elementwise(to_np(got["out"]), out, _ec_bound(hp, ec, case.wd, w.T, w.d), "out")
+    kept = np.zeros(w.T, dtype=bool)
+    kept[ec.src] = True
+    assert (to_np(got["out"])[~kept] == 0).all()
+    check_close(to_np(got["out"])[kept], out[kept], "out")
 
 
 @pytest.mark.parametrize("seed", range(8))
@@ -144,3 +167,4 @@ def test_random_reroute(cuda_ok, seed):
             a[off[e]:off[e + 1]] = np.abs(hp[off[e]:off[e + 1]]) @ np.abs(oracle.f64(case.wd[e])).T
     bound = 2.0 ** -7 * oracle.combine(a, dest, np.abs(wts), w.T, w.k)
     _elementwise(to_np(got["out"]), out, bound, "out")
+    check_layer_output(to_np(got["out"]), out, dest, w.T, w.k)

@@ -260,6 +260,59 @@ def pin_reroute_invariants(seed=31):
     return bool(ok)
 
 
+def pin_reroute_positions_worked():
+    """Hand-worked layout of a re-routed result: T = 4 tokens, k = 2, E = 3.  Final experts per
+    pair q = t*k + j: [1, 0, 0, 2, 1, -, 2, 1] with slots inside each expert
+    [0, 0, 1, 0, 1, -, 1, 2]; so the experts hold 2, 3 and 2 rows, the segments start at rows
+    0, 2, 5 (7 rows in all), dest[q] = start of its expert + slot = [2, 0, 1, 5, 3, -1, 6, 4] and
+    the inverse src[row] = [1, 2, 0, 4, 7, 3, 6]."""
+    rr = om.Rerouted(expert=np.array([1, 0, 0, 2, 1, -1, 2, 1]), slot=np.array([0, 0, 1, 0, 1, -1, 1, 2]),
+                     round=np.array([0, 0, 0, 0, 0, -1, 1, 1]), assigned=np.array([2, 3, 2]))
+    segs, dest, src = oracle.reroute_positions(rr)
+    return bool(list(segs.offsets) == [0, 2, 5, 7] and list(segs.expert) == [0, 1, 2]
+                and list(dest) == [2, 0, 1, 5, 3, -1, 6, 4] and list(src) == [1, 2, 0, 4, 7, 3, 6])
+
+
+def pin_layer_reroute_eager(seed=32):
+    """The re-routed layer equals an eager loop over the pairs: pair (t, j) placed at expert
+    e = rr.expert[q] adds w[t, j] * FFN_e(x_t) to token t (a moved pair keeps its routing weight;
+    a dropped pair adds nothing), and the dispatched row of every placed pair is x_t."""
+    T, E, k, C = 40, 6, 2, 8
+    x, wr, b, wg, wu, wd = _small_layer(seed, T=T, E=E, k=k, zipf=1.5)
+    logits, ids, w, rr, segs, dest, src, xp, hp, yp, out = oracle.layer_forward_reroute(x, wr, b, wg, wu, wd, k, C)
+    x64 = oracle.f64(x)
+    want = np.zeros_like(out)
+    moved = 0
+    for t in range(T):
+        for j in range(k):
+            q = t * k + j
+            e = int(rr.expert[q])
+            if e < 0:
+                continue
+            moved += int(rr.round[q] > 0)
+            _, y = oracle.expert_ffn(x64[t][None, :], wg[e], wu[e], wd[e])
+            want[t] += w[t, j] * y[0]
+            if not np.array_equal(xp[dest[q]], x64[t]):
+                return False
+    return bool(moved > 0 and np.allclose(out, want, rtol=1e-11, atol=1e-13))
+
+
+def pin_expert_choice_map_argsort(seed=22, T=23, E=5, C=6):
+    """The [T, E] row map built independently: expert e keeps the first C tokens of a stable
+    descending argsort of its fp32 scores (library routine), listed in ascending token id; the
+    i-th of them sits at row e*C + i; every other entry is -1."""
+    rng = np.random.default_rng(seed)
+    logits = rng.normal(size=(T, E))
+    ec = oracle.expert_choice(logits, C)
+    S = torch.softmax(torch.from_numpy(logits), dim=1).numpy().astype(np.float32)
+    want = np.full((T, E), -1, dtype=np.int64)
+    for e in range(E):
+        picks = np.sort(np.argsort(-S[:, e], kind="stable")[:C])
+        want[picks, e] = e * C + np.arange(C)
+    got = oracle.expert_choice_map(ec, T)
+    return bool(got.shape == (T, E) and np.array_equal(got, want))
+
+
 def pin_silu_library():
     z = np.linspace(-30, 30, 2001)
     ref = torch.nn.functional.silu(torch.from_numpy(z)).numpy()
@@ -445,6 +498,18 @@ def test_reroute_invariants():
     assert pin_reroute_invariants()
 
 
+def test_reroute_positions_worked_example():
+    assert pin_reroute_positions_worked()
+
+
+def test_reroute_layer_equals_eager_pair_loop():
+    assert pin_layer_reroute_eager()
+
+
+def test_expert_choice_map_from_argsort():
+    assert pin_expert_choice_map_argsort()
+
+
 def test_shared_expert_adds_a_dense_ffn():
     assert pin_shared_expert_additive()
 
@@ -572,6 +637,39 @@ def _mut_ec_keeps_weakest(logits64, capacity):
     return _orig_expert_choice(-np.asarray(logits64, dtype=np.float64), capacity)   # picks the lowest scores
 
 
+_orig_reroute_positions = om.reroute_positions
+
+
+def _mut_reroute_positions_next_offset(rr):
+    segs, dest, src = _orig_reroute_positions(rr)
+    off = segs.offsets
+    dest = np.where(rr.expert >= 0, off[np.maximum(rr.expert, 0) + 1] + rr.slot, -1)   # off[e+1] for off[e]
+    return segs, dest, src
+
+
+_orig_layer_reroute = om.layer_forward_reroute
+
+
+def _mut_layer_reroute_drops_moved(x, w_router, bias, w_gate, w_up, w_down, k, capacity):
+    r = list(_orig_layer_reroute(x, w_router, bias, w_gate, w_up, w_down, k, capacity))
+    rr, dest = r[3], r[5]
+    dest = np.where(rr.round > 0, -1, dest)          # moved pairs treated as dropped
+    r[10] = om.combine(r[9], dest, r[2], r[0].shape[0], k)
+    return tuple(r)
+
+
+_orig_ec_map = om.expert_choice_map
+
+
+def _mut_ec_map_left_boundary(ec, T):
+    E = len(ec.picks)
+    m = np.full((T, E), -1, dtype=np.int64)
+    for r in range(len(ec.src)):
+        e = int(np.searchsorted(ec.segs.offsets, r, side="left") - 1)   # first row of a segment -> previous expert
+        m[ec.src[r], e] = r
+    return m
+
+
 MUTATIONS = [
     ("silu", _mut_silu_sign, [pin_silu_library, pin_dense_ffn_e1k1]),
     ("topk_weights", _mut_weights_no_renorm, [pin_worked_example, pin_weights_full_softmax]),
@@ -588,6 +686,9 @@ MUTATIONS = [
     ("expert_choice", _mut_ec_keeps_weakest, [pin_expert_choice_brute_force, pin_expert_choice_layer_eager]),
     ("candidate_order", _mut_candidates_ascending, [pin_reroute_worked_example, pin_reroute_invariants]),
     ("reroute_overflow", _mut_reroute_keeps_full, [pin_reroute_worked_example, pin_reroute_invariants]),
+    ("reroute_positions", _mut_reroute_positions_next_offset, [pin_reroute_positions_worked, pin_layer_reroute_eager]),
+    ("layer_forward_reroute", _mut_layer_reroute_drops_moved, [pin_layer_reroute_eager]),
+    ("expert_choice_map", _mut_ec_map_left_boundary, [pin_expert_choice_map_argsort]),
 ]
 
 
