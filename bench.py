@@ -35,6 +35,7 @@ if ROOT not in sys.path:
 
 METRIC = "MoE layer fwd tokens/s; grouped-GEMM TFLOPS and permute GB/s vs roofline"
 FLUSH_BYTES = 256 << 20
+NOMINAL_HBM_GBS = 8000.0     # B200 HBM3e, nominal (the measured copy bandwidth is the primary peak)
 E2E_MIN_STEPS = 64
 KERNELS = ("route", "dispatch", "gate_up", "down", "combine")
 
@@ -172,10 +173,10 @@ def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: fl
     return tokens_per_rank_step * steps * world / (max_ms / 1e3)
 
 
-def _config(w, capacity):
+def _config(w, capacity, out_dtype="bf16"):
     return {"workload": w.name, "T": w.T, "d_model": w.d, "n_experts": w.E, "top_k": w.k, "d_ff": w.F,
             "capacity": capacity, "n_groups": w.n_groups, "replica_slots": w.replica_slots,
-            "zipf_bias_s": w.zipf_s,
+            "zipf_bias_s": w.zipf_s, "out_dtype": out_dtype,
             "routing": "expert-choice" if w.expert_choice else ("top-k, overflow re-routed" if w.reroute else "top-k"),
             "l2": "flushed between steps (256 MiB write outside the timed events)",
             "parallelism": "replicas (no exchange between GPUs)"}
@@ -183,10 +184,21 @@ def _config(w, capacity):
 
 # ----------------------------------------------------------------------------- CPU oracle legs
 
-def _oracle_sample(w, seed: int, n_route: int, n_ffn: int, wg, wu, wd):
-    """Time the oracle on a bounded sample of the workload; returns (tokens/s, description)."""
+def _ffn_rows(xp, n_ffn: int, wg, wu, wd):
+    """The oracle's expert FFN on n_ffn dispatched rows spread evenly over the experts whose
+    weights were read back (wg/wu/wd hold experts 0..n_exp-1); returns (rows, y, seconds)."""
     import numpy as np
-    import torch
+    import oracle
+    n_exp = wg.shape[0]
+    per = max(1, n_ffn // n_exp)
+    t0 = time.perf_counter()
+    ys = [oracle.expert_ffn(xp[e * per:(e + 1) * per], wg[e], wu[e], wd[e])[1] for e in range(n_exp)]
+    return per * n_exp, np.concatenate(ys), time.perf_counter() - t0
+
+
+def _oracle_sample(w, seed: int, n_route: int, n_ffn: int, wg, wu, wd):
+    """Time the oracle on a bounded sample of the workload; returns (tokens/s, description, seconds)."""
+    import numpy as np
     import oracle
     from mixture_experts_routing_02_b200 import synthetic as syn
 
@@ -203,16 +215,16 @@ def _oracle_sample(w, seed: int, n_route: int, n_ffn: int, wg, wu, wd):
     dest, src = oracle.dispatch_positions(ids, segs, w.E)
     xp = oracle.permute_rows(x, src, w.k)
     t2 = time.perf_counter()
-    _, y = oracle.expert_ffn(xp[:n_ffn], wg[0], wu[0], wd[0])
+    n_rows, y, t_ffn = _ffn_rows(xp, n_ffn, wg, wu, wd)
     t3 = time.perf_counter()
     yfull = np.zeros((xp.shape[0], w.d))
-    yfull[:n_ffn] = y
+    yfull[:n_rows] = y
     oracle.combine(yfull, dest, wts, n_route, w.k)
     t4 = time.perf_counter()
-    per_token = (t1 - t0) / n_route + (t2 - t1) / n_route + w.k * (t3 - t2) / n_ffn + (t4 - t3) / n_route
+    per_token = (t1 - t0) / n_route + (t2 - t1) / n_route + w.k * t_ffn / n_rows + (t4 - t3) / n_route
     desc = (f"routing, histogram, segments, dispatch positions and combine of {n_route} tokens; expert FFN "
-            f"(gate/up/down, fp64) of {n_ffn} rows of one expert; per-token cost = per-token routing+dispatch"
-            f"+combine + k x per-row FFN, extrapolated to tokens/s")
+            f"(gate/up/down, fp64) of {n_rows} dispatched rows over {wg.shape[0]} experts; per-token cost = "
+            f"per-token routing+dispatch+combine + k x per-row FFN, extrapolated to tokens/s; one BLAS thread")
     return 1.0 / per_token, desc, t4 - t0
 
 
@@ -229,17 +241,18 @@ def _oracle_sample_reroute(w, x, w_r, bias, n_route: int, n_ffn: int, wg, wu, wd
     segs, dest, src = oracle.reroute_positions(rr)
     xp = oracle.permute_rows(x, src, w.k)
     t1 = time.perf_counter()
-    _, y = oracle.expert_ffn(xp[:n_ffn], wg[0], wu[0], wd[0])
+    n_rows, y, t_ffn = _ffn_rows(xp, n_ffn, wg, wu, wd)
     t2 = time.perf_counter()
     yfull = np.zeros((xp.shape[0], w.d))
-    yfull[:n_ffn] = y
+    yfull[:n_rows] = y
     oracle.combine(yfull, dest, wts, n_route, w.k)
     t3 = time.perf_counter()
     rows_per_token = xp.shape[0] / n_route
-    per_token = (t1 - t0) / n_route + rows_per_token * (t2 - t1) / n_ffn + (t3 - t2) / n_route
+    per_token = (t1 - t0) / n_route + rows_per_token * t_ffn / n_rows + (t3 - t2) / n_route
     desc = (f"routing, capacity re-routing rounds and dispatch of {n_route} tokens (C={C}) and combine; expert "
-            f"FFN (gate/up/down, fp64) of {n_ffn} rows of one expert; per-token cost = per-token routing+dispatch"
-            f"+combine + (rows per token = {rows_per_token:g}) x per-row FFN, extrapolated to tokens/s")
+            f"FFN (gate/up/down, fp64) of {n_rows} dispatched rows over {wg.shape[0]} experts; per-token cost = "
+            f"per-token routing+dispatch+combine + (rows per token = {rows_per_token:g}) x per-row FFN, "
+            f"extrapolated to tokens/s; one BLAS thread")
     return 1.0 / per_token, desc, t3 - t0
 
 
@@ -254,17 +267,18 @@ def _oracle_sample_ec(w, x, w_r, bias, n_route: int, n_ffn: int, wg, wu, wd):
     ec = oracle.expert_choice(oracle.router_logits(x, w_r, bias), C)
     xp = oracle.f64(x)[ec.src]
     t1 = time.perf_counter()
-    _, y = oracle.expert_ffn(xp[:n_ffn], wg[0], wu[0], wd[0])
+    n_rows, y, t_ffn = _ffn_rows(xp, n_ffn, wg, wu, wd)
     t2 = time.perf_counter()
     yfull = np.zeros((xp.shape[0], w.d))
-    yfull[:n_ffn] = y
+    yfull[:n_rows] = y
     oracle.combine_expert_choice(yfull, ec.src, ec.row_w, n_route)
     t3 = time.perf_counter()
     rows_per_token = len(ec.src) / n_route
-    per_token = (t1 - t0) / n_route + rows_per_token * (t2 - t1) / n_ffn + (t3 - t2) / n_route
+    per_token = (t1 - t0) / n_route + rows_per_token * t_ffn / n_rows + (t3 - t2) / n_route
     desc = (f"expert-choice scores, selection and dispatch of {n_route} tokens (C={C}) and combine; expert FFN "
-            f"(gate/up/down, fp64) of {n_ffn} rows of one expert; per-token cost = per-token routing+dispatch"
-            f"+combine + (rows per token = {rows_per_token:g}) x per-row FFN, extrapolated to tokens/s")
+            f"(gate/up/down, fp64) of {n_rows} dispatched rows over {wg.shape[0]} experts; per-token cost = "
+            f"per-token routing+dispatch+combine + (rows per token = {rows_per_token:g}) x per-row FFN, "
+            f"extrapolated to tokens/s; one BLAS thread")
     return 1.0 / per_token, desc, t3 - t0
 
 
@@ -277,6 +291,12 @@ def _threads_used():
         return os.cpu_count() or 1
 
 
+def _one_thread():
+    """Context in which the oracle's BLAS calls run on one thread (the single-threaded CPU baseline)."""
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=1, user_api="blas")
+
+
 def run_reference(args, w):
     world, rank, _ = _dist()
     if rank != 0:
@@ -284,23 +304,25 @@ def run_reference(args, w):
     capacity = _capacity(w)
     n_route, n_ffn = 256, 8
     from mixture_experts_routing_02_b200 import synthetic as syn
-    wg, wu, wd = syn.expert_weights(w, args.seed, experts=range(1))
-    for _ in range(args.warmup):
-        _oracle_sample(w, args.seed, n_route, n_ffn, wg, wu, wd)
+    wg, wu, wd = syn.expert_weights(w, args.seed, experts=range(2))
     vals, secs = [], []
     desc = ""
-    for _ in range(args.steps):
-        v, desc, s = _oracle_sample(w, args.seed, n_route, n_ffn, wg, wu, wd)
-        vals.append(v)
-        secs.append(s)
+    with _one_thread():
+        for _ in range(args.warmup):
+            _oracle_sample(w, args.seed, n_route, n_ffn, wg, wu, wd)
+        for _ in range(args.steps):
+            v, desc, s = _oracle_sample(w, args.seed, n_route, n_ffn, wg, wu, wd)
+            vals.append(v)
+            secs.append(s)
+        cores = _threads_used()
     value = statistics.mean(vals)
-    cores = _threads_used()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(secs),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded; random-init weights)", "config": _config(w, capacity),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "data": "synthetic (seeded; random-init weights)", "config": _config(w, capacity, args.out_dtype),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "host_cores": os.cpu_count(),
+                         "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -337,9 +359,13 @@ def run_ours(args, w):
     capacity = _capacity(w)
     ec = w.expert_choice
     rr = w.reroute
+    out_bf16 = args.out_dtype == "bf16"
+    out_torch = torch.bfloat16 if out_bf16 else torch.float32
+    out_bytes = 2 if out_bf16 else 4
     s = moe.shape(w.T, w.d, w.E, w.k, w.F, capacity=capacity, n_groups=w.n_groups,
                   replica_slots=w.replica_slots,
-                  route_flags=(moe.ROUTE_EXPERT_CHOICE if ec else 0) | (moe.ROUTE_REROUTE if rr else 0))
+                  route_flags=(moe.ROUTE_EXPERT_CHOICE if ec else 0) | (moe.ROUTE_REROUTE if rr else 0),
+                  out_dtype=moe.DTYPE_BF16 if out_bf16 else moe.DTYPE_F32)
     n_seg, rows_alloc = moe.moe_layout(s)
     _, layer_bytes = moe.moe_workspace_size(s)
 
@@ -351,8 +377,8 @@ def run_ours(args, w):
     bias = bias.to(dev) if bias is not None else None
     wg, wu, wd = syn.expert_weights(w, seed, device=dev)
     ws = torch.empty(layer_bytes, dtype=torch.uint8, device=dev)
-    out = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
-    out_host = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
+    out = torch.empty(w.T, w.d, dtype=out_torch, device=dev)
+    out_host = torch.empty(w.T, w.d, dtype=out_torch).pin_memory()
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     v = moe.moe_layer_views(s, ws)
@@ -387,6 +413,8 @@ def run_ours(args, w):
                 + 3)                                                           # gate_up, down, combine
 
     Fs = args.shared_expert
+    if Fs and out_bf16:
+        raise SystemExit("--shared-expert adds the shared expert's fp32 output in the combine: use --out-dtype f32")
     if Fs:
         gs, us, dsw = (t.to(dev) for t in syn.shared_expert_weights(w, Fs, seed))
         h_s = torch.empty(w.T, Fs, dtype=torch.bfloat16, device=dev)
@@ -542,9 +570,10 @@ def run_ours(args, w):
     breakdown["down"] = dict(ms=avg["down"], flops=2 * rows_used * d * F,
                              bytes=active_experts * d * F * 2 + rows_used * F * 2 + rows_used * d * 4)
     if ec:
-        breakdown["combine"] = dict(ms=avg["combine"], bytes=rows_used * d * 4 + T * d * 4 + T * E * 4 + rows_used * 4)
+        breakdown["combine"] = dict(ms=avg["combine"],
+                                    bytes=rows_used * d * 4 + T * d * out_bytes + T * E * 4 + rows_used * 4)
     else:
-        breakdown["combine"] = dict(ms=avg["combine"], bytes=rows_used * d * 4 + T * d * 4 + T * k * 8)
+        breakdown["combine"] = dict(ms=avg["combine"], bytes=rows_used * d * 4 + T * d * out_bytes + T * k * 8)
     for name, b in breakdown.items():
         sec = b["ms"] / 1e3
         if "flops" in b and name in ("gate_up", "down"):
@@ -552,6 +581,7 @@ def run_ours(args, w):
             b["frac_bf16_peak"] = b["tflops"] / bf16
         b["gbs"] = b["bytes"] / sec / 1e9
         b["frac_hbm_peak"] = b["gbs"] / hbm
+        b["frac_hbm_nominal"] = b["gbs"] / NOMINAL_HBM_GBS
     dom = max(breakdown, key=lambda n: breakdown[n]["ms"])
     db = breakdown[dom]
     if dom in ("gate_up", "down"):
@@ -563,20 +593,36 @@ def run_ours(args, w):
                 "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs"}
     traffic = _traffic(dom, w.name)
     roof["traffic"] = traffic
+    # The whole layer against its own roofline: the larger of the grouped-GEMM flops at the bf16
+    # peak and the layer's algorithmic bytes at the HBM peak (Hp, which a fused gate -> down
+    # pipeline need not store, is left out of the bytes).
+    gemm_flops = breakdown["gate_up"]["flops"] + breakdown["down"]["flops"]
+    hp_bytes = rows_used * F * 2
+    layer_bytes = sum(b["bytes"] for b in breakdown.values()) - 2 * hp_bytes
+    t_flop_ms = gemm_flops / (bf16 * 1e12) * 1e3
+    t_bytes_ms = layer_bytes / (hbm * 1e9) * 1e3
+    layer_roof = {"bound": "tensor" if t_flop_ms >= t_bytes_ms else "hbm", "gemm_flops": gemm_flops,
+                  "algorithmic_bytes": layer_bytes, "t_flop_ms": t_flop_ms, "t_bytes_ms": t_bytes_ms,
+                  "roofline_ms": max(t_flop_ms, t_bytes_ms), "peaks": f"{peak_kind} bf16_tflops {bf16}, hbm_gbs {hbm}"}
 
     value = job_throughput(T, args.steps, world, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded; random-init weights)", "config": _config(w, capacity),
+        "data": "synthetic (seeded; random-init weights)", "config": _config(w, capacity, args.out_dtype),
         "rows_dispatched": rows_used, "gpu_launches": launches * args.steps,
         "roofline": roof,
+        "layer_roofline": dict(layer_roof, ms_per_step=total_ms / args.steps,
+                               frac=layer_roof["roofline_ms"] / (total_ms / args.steps)),
         "breakdown": {n: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in b.items()}
                       for n, b in breakdown.items()},
         "e2e": {"value": job_throughput(T, e2e_steps, world, e2e_ms), "unit": "tokens/s", "steps": e2e_steps,
                 "h2d_bytes_per_step": T * d * 2,
-                "d2h_bytes_per_step": T * d * 4, "api": "moe_layer_fwd; per step X (bf16) copied in from pinned host memory and out (fp32) copied back; steps pipelined over copy-in / compute / copy-out streams with double-buffered device buffers"},
+                "d2h_bytes_per_step": T * d * out_bytes,
+                "api": f"moe_layer_fwd; per step X (bf16) copied in from pinned host memory and out "
+                       f"({args.out_dtype}) copied back; steps pipelined over copy-in / compute / copy-out streams "
+                       f"with double-buffered device buffers"},
         "clocks": clocks.summary(),
     }
     if shared_info:
@@ -584,10 +630,13 @@ def run_ours(args, w):
         line["config"]["shared_expert_d_ff"] = Fs
         line["gpu_launches"] = (launches + 2) * args.steps
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        wg0, wu0, wd0 = wg[:1].cpu(), wu[:1].cpu(), wd[:1].cpu()
-        cv, desc, _ = _oracle_sample(w, seed, 512, 32, wg0, wu0, wd0)
-        line["cpu_baseline"] = {"value": cv, "unit": "tokens/s", "cores": _threads_used(), "kind": "oracle",
-                                "sample": desc}
+        n_exp = min(4, w.E)
+        wg0, wu0, wd0 = wg[:n_exp].cpu(), wu[:n_exp].cpu(), wd[:n_exp].cpu()
+        with _one_thread():
+            cv, desc, _ = _oracle_sample(w, seed, 512, 64, wg0, wu0, wd0)
+            cores = _threads_used()
+        line["cpu_baseline"] = {"value": cv, "unit": "tokens/s", "cores": cores, "host_cores": os.cpu_count(),
+                                "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -607,7 +656,9 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shared-expert", type=int, default=0, metavar="F_S",
-                    help="add one shared expert of inner size F_S, overlapped on a second stream")
+                    help="add one shared expert of inner size F_S, overlapped on a second stream (needs --out-dtype f32)")
+    ap.add_argument("--out-dtype", choices=("bf16", "f32"), default="bf16",
+                    help="element type of the layer output (default bf16)")
     args = ap.parse_args()
     w = syn.WORKLOADS[args.workload]
     if args.impl == "reference":

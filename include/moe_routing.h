@@ -135,6 +135,18 @@ typedef enum {
 #define MOE_ROUTE_EXPERT_CHOICE 0x2
 #define MOE_ROUTE_REROUTE 0x4
 
+/*
+ *   out_dtype      element type of the layer output out [T, d] written by
+ *                  moe_combine, moe_combine_add, moe_combine_expert_choice and
+ *                  moe_layer_fwd: MOE_DTYPE_F32 (0, the value of a
+ *                  zero-initialised shape) stores the fp32 accumulator;
+ *                  MOE_DTYPE_BF16 rounds it once to bf16 (round to nearest
+ *                  even), half the bytes written and read back by the caller.
+ *                  Yp stays fp32 either way.
+ */
+#define MOE_DTYPE_F32 0
+#define MOE_DTYPE_BF16 1
+
 typedef struct {
     int32_t T;
     int32_t d_model;
@@ -145,6 +157,7 @@ typedef struct {
     int32_t n_groups;
     int32_t replica_slots;
     int32_t route_flags;
+    int32_t out_dtype;
 } moe_shape_t;
 
 /*
@@ -333,22 +346,24 @@ MOE_API moe_status_t moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *
  * ...", last step: un-permute and weight by the router; MoonEP page
  * "설치 및 통합": combine):
  *   out[t] = sum over j with dest[t*k+j] >= 0 of topk_w[t, j] * Yp[dest[t*k+j]]
- * accumulated in fp32 in ascending j and stored in fp32 (the layer output is
- * the combine's fp32 accumulator; rounding it to bf16 is left to the caller).
- * A token whose pairs were all dropped gets 0.
- *   yp [rows_alloc, d] fp32; dest [T*k]; topk_w [T, k]; out [T, d] fp32.
+ * accumulated in fp32 in ascending j and stored in shape->out_dtype: the fp32
+ * accumulator, or that value rounded once to bf16.  A token whose pairs were all
+ * dropped gets 0.
+ *   yp [rows_alloc, d] fp32; dest [T*k]; topk_w [T, k];
+ *   out [T, d] fp32 or bf16 (16-byte aligned).
  */
 MOE_API moe_status_t moe_combine(const moe_shape_t *shape, const float *yp, const int32_t *dest,
-                         const float *topk_w, float *out, moe_stream_t stream);
+                         const float *topk_w, void *out, moe_stream_t stream);
 
 /*
  * Combine with a base term: out[t] = base[t] + the combine above (base [T, d]
- * fp32, nullable: then identical to moe_combine).  With base = the shared
- * expert's output (moe_shared_expert) this finishes a layer with a shared
- * expert.  out may alias base.
+ * fp32, nullable: then identical to moe_combine), stored in shape->out_dtype.
+ * With base = the shared expert's output (moe_shared_expert) this finishes a
+ * layer with a shared expert.  out may alias base when out is fp32; with a bf16
+ * out an aliasing base is rejected (MOE_ERR_INVALID_ARG).
  */
 MOE_API moe_status_t moe_combine_add(const moe_shape_t *shape, const float *yp, const int32_t *dest,
-                             const float *topk_w, const float *base, float *out,
+                             const float *topk_w, const float *base, void *out,
                              moe_stream_t stream);
 
 /*
@@ -377,12 +392,13 @@ MOE_API moe_status_t moe_shared_expert(const moe_shape_t *shape, int32_t d_ff_sh
  * views topk_ids, topk_w, dest, seg_first_rank and dispatch_ws are then unused.
  * With MOE_ROUTE_REROUTE the dispatch is moe_dispatch_reroute (the logits are
  * then kept in the workspace).
- * out [T, d] fp32.  The intermediates live in `ws` (moe_workspace_size()'s
- * layer_bytes); their addresses are given by moe_layer_views.
+ * out [T, d] in shape->out_dtype (fp32, or bf16 as the pages' layer returns
+ * it).  The intermediates live in `ws` (moe_workspace_size()'s layer_bytes);
+ * their addresses are given by moe_layer_views.
  */
 MOE_API moe_status_t moe_layer_fwd(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *w_router,
                            const float *bias, const moe_bf16_t *w_gate, const moe_bf16_t *w_up,
-                           const moe_bf16_t *w_down, float *out, int32_t *status, void *ws,
+                           const moe_bf16_t *w_down, void *out, int32_t *status, void *ws,
                            size_t ws_bytes, moe_stream_t stream);
 
 /*
@@ -457,11 +473,12 @@ MOE_API moe_status_t moe_expert_choose(const moe_shape_t *shape, const float *sc
  * Expert-choice combine: out[t] = base[t] + sum over e ascending with
  * emap[t, e] >= 0 of row_w[r] * yp[r], r = emap[t, e], accumulated in fp32.
  *   yp [E * C', d] fp32;  emap [T, E] int32;  row_w [E * C'] fp32
- *   base [T, d] fp32 or NULL;  out [T, d] fp32 (may alias base)
+ *   base [T, d] fp32 or NULL;  out [T, d] in shape->out_dtype (an fp32 out may
+ *   alias base; a bf16 out may not)
  * Rows outside [0, E * C') contribute nothing.  Rejects shapes without the flag.
  */
 MOE_API moe_status_t moe_combine_expert_choice(const moe_shape_t *shape, const float *yp, const int32_t *emap,
-                                       const float *row_w, const float *base, float *out,
+                                       const float *row_w, const float *base, void *out,
                                        moe_stream_t stream);
 
 /*

@@ -22,6 +22,7 @@ __all__ = [
     "moe_route_workspace_size", "moe_route_ws", "moe_route_scores_ws", "moe_dispatch_reroute",
     "moe_layer_views", "moe_routing_stats", "STAT_NAMES",
     "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT", "ROUTE_SOFTMAX_ALL", "ROUTE_EXPERT_CHOICE", "ROUTE_REROUTE",
+    "DTYPE_F32", "DTYPE_BF16",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -37,7 +38,7 @@ class MoeError(RuntimeError):
 class MoeShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("T", "d_model", "n_experts", "top_k", "d_ff", "capacity", "n_groups", "replica_slots",
-                 "route_flags")]
+                 "route_flags", "out_dtype")]
 
 
 class MoeLayerViews(ctypes.Structure):
@@ -109,10 +110,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 ROUTE_SOFTMAX_ALL = 0x1
 ROUTE_EXPERT_CHOICE = 0x2
 ROUTE_REROUTE = 0x4
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
 
 
-def shape(T, d_model, n_experts, top_k, d_ff, capacity=0, n_groups=0, replica_slots=0, route_flags=0) -> MoeShape:
-    return MoeShape(T, d_model, n_experts, top_k, d_ff, capacity, n_groups, replica_slots, route_flags)
+def shape(T, d_model, n_experts, top_k, d_ff, capacity=0, n_groups=0, replica_slots=0, route_flags=0,
+          out_dtype=DTYPE_F32) -> MoeShape:
+    """out_dtype: DTYPE_F32 or DTYPE_BF16, the element type of the layer output `out`."""
+    return MoeShape(T, d_model, n_experts, top_k, d_ff, capacity, n_groups, replica_slots, route_flags, out_dtype)
 
 
 def _ptr(t) -> Optional[int]:

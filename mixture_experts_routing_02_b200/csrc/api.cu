@@ -47,6 +47,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Dims {
     int T, d, E, k, F, C, R, B, S, flags;
+    bool out_bf16;  // the layer output [T, d] is stored in bf16 (else fp32)
     bool ec() const { return (flags & MOE_ROUTE_EXPERT_CHOICE) != 0; }
     bool rr() const { return (flags & MOE_ROUTE_REROUTE) != 0; }
     int cp() const { return ec() ? std::min(C, T) : 0; }  // expert choice: rows per expert
@@ -59,6 +60,8 @@ moe_status_t check_shape(const moe_shape_t* s, Dims* out) {
     Dims v;
     v.T = s->T; v.d = s->d_model; v.E = s->n_experts; v.k = s->top_k; v.F = s->d_ff;
     v.C = s->capacity; v.R = s->n_groups; v.B = s->replica_slots; v.flags = s->route_flags;
+    if (s->out_dtype != MOE_DTYPE_F32 && s->out_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    v.out_bf16 = s->out_dtype == MOE_DTYPE_BF16;
     if (v.flags & ~(MOE_ROUTE_SOFTMAX_ALL | MOE_ROUTE_EXPERT_CHOICE | MOE_ROUTE_REROUTE)) return MOE_ERR_INVALID_ARG;
     const bool ec = (v.flags & MOE_ROUTE_EXPERT_CHOICE) != 0;
     if (ec && ((v.flags & MOE_ROUTE_SOFTMAX_ALL) || s->capacity < 1 || s->n_groups != 0)) return MOE_ERR_INVALID_ARG;
@@ -622,14 +625,14 @@ moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* xp, cons
 }
 
 moe_status_t moe_combine(const moe_shape_t* shape, const float* yp, const int32_t* dest, const float* topk_w,
-                         float* out, moe_stream_t stream) {
+                         void* out, moe_stream_t stream) {
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(yp) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_combine(yp, dest, topk_w, nullptr, v.T, v.k, v.d, v.rows, out, sm_count(),
+    return cuda_status(launch_combine(yp, dest, topk_w, nullptr, v.T, v.k, v.d, v.rows, out, v.out_bf16, sm_count(),
                                       static_cast<cudaStream_t>(stream)));
 }
 
@@ -648,14 +651,15 @@ moe_status_t moe_testing_dispatch_stalled(const moe_shape_t* shape, const moe_bf
 }
 
 moe_status_t moe_combine_add(const moe_shape_t* shape, const float* yp, const int32_t* dest, const float* topk_w,
-                             const float* base, float* out, moe_stream_t stream) {
+                             const float* base, void* out, moe_stream_t stream) {
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (v.ec()) return MOE_ERR_INVALID_ARG;  // expert choice has its own calls
     if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(yp) || !aligned16(out) || (base && !aligned16(base))) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_combine(yp, dest, topk_w, base, v.T, v.k, v.d, v.rows, out, sm_count(),
+    if (v.out_bf16 && base != nullptr && static_cast<const void*>(base) == out) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_combine(yp, dest, topk_w, base, v.T, v.k, v.d, v.rows, out, v.out_bf16, sm_count(),
                                       static_cast<cudaStream_t>(stream)));
 }
 
@@ -725,14 +729,15 @@ moe_status_t moe_expert_choose(const moe_shape_t* shape, const float* scores, co
 }
 
 moe_status_t moe_combine_expert_choice(const moe_shape_t* shape, const float* yp, const int32_t* emap,
-                                       const float* row_w, const float* base, float* out, moe_stream_t stream) {
+                                       const float* row_w, const float* base, void* out, moe_stream_t stream) {
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
     if (!v.ec()) return MOE_ERR_INVALID_ARG;
     if (!yp || !emap || !row_w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(yp) || !aligned16(out) || (base && !aligned16(base))) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_ec_combine(yp, emap, row_w, base, v.T, v.E, v.d, v.rows, out, sm_count(),
+    if (v.out_bf16 && base != nullptr && static_cast<const void*>(base) == out) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_ec_combine(yp, emap, row_w, base, v.T, v.E, v.d, v.rows, out, v.out_bf16, sm_count(),
                                          static_cast<cudaStream_t>(stream)));
 }
 
@@ -776,7 +781,7 @@ moe_status_t moe_layer_views(const moe_shape_t* shape, void* ws, moe_layer_views
 
 moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const moe_bf16_t* w_router,
                            const float* bias, const moe_bf16_t* w_gate, const moe_bf16_t* w_up,
-                           const moe_bf16_t* w_down, float* out, int32_t* status, void* ws, size_t ws_bytes,
+                           const moe_bf16_t* w_down, void* out, int32_t* status, void* ws, size_t ws_bytes,
                            moe_stream_t stream) {
     Dims v;
     moe_status_t s = check_shape(shape, &v);
@@ -801,8 +806,8 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
         if (s != MOE_OK) return s;
         s = down_impl(v, w.hp, w.seg_expert, w.seg_offsets, w_down, w.yp, status, st);
         if (s != MOE_OK) return s;
-        return cuda_status(launch_ec_combine(w.yp, w.emap, w.row_w, nullptr, v.T, v.E, v.d, v.rows, out, sm_count(),
-                                             st));
+        return cuda_status(launch_ec_combine(w.yp, w.emap, w.row_w, nullptr, v.T, v.E, v.d, v.rows, out, v.out_bf16,
+                                             sm_count(), st));
     }
     if (!route_split_impl(v, x, w_router, bias, w.logits, w.topk_ids, w.topk_w, nullptr, status, route_ws,
                           route_ws_len, st, &s))
@@ -816,7 +821,8 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
         if (s != MOE_OK) return s;
         s = down_impl(v, w.hp, w.seg_expert, w.seg_offsets, w_down, w.yp, status, st);
         if (s != MOE_OK) return s;
-        return cuda_status(launch_combine(w.yp, w.dest, w.topk_w, nullptr, v.T, v.k, v.d, v.rows, out, sm_count(), st));
+        return cuda_status(
+            launch_combine(w.yp, w.dest, w.topk_w, nullptr, v.T, v.k, v.d, v.rows, out, v.out_bf16, sm_count(), st));
     }
     s = dispatch_impl(v, x, w.topk_ids, 0, w.counts, w.seg_expert, w.seg_offsets, w.seg_first_rank, w.dest, w.src,
                       w.xp, status, w.dispatch_ws, w.dispatch_ws_bytes, st);
@@ -825,7 +831,8 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
     if (s != MOE_OK) return s;
     s = down_impl(v, w.hp, w.seg_expert, w.seg_offsets, w_down, w.yp, status, st);
     if (s != MOE_OK) return s;
-    return cuda_status(launch_combine(w.yp, w.dest, w.topk_w, nullptr, v.T, v.k, v.d, v.rows, out, sm_count(), st));
+    return cuda_status(
+        launch_combine(w.yp, w.dest, w.topk_w, nullptr, v.T, v.k, v.d, v.rows, out, v.out_bf16, sm_count(), st));
 }
 
 }  // extern "C"

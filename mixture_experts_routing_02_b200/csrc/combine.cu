@@ -1,6 +1,6 @@
 // Combine: out[t] = base[t] + sum_j w[t, j] * Yp[dest[t*k + j]] over the kept pairs,
-// accumulated in fp32 in ascending j; Yp, base (optional, e.g. the shared expert's
-// output) and out are fp32.
+// accumulated in fp32 in ascending j; Yp and base (optional, e.g. the shared expert's
+// output) are fp32; out is stored in fp32, or rounded once to bf16.
 //
 // Sources: "Sparsely-Gated MoE 구현 관점에서 살펴보기", section "순전파 과정 ..."
 // (un-permute the expert outputs and combine them with the router weights);
@@ -19,11 +19,11 @@ namespace moe {
 namespace {
 
 // KMAX: the largest k this instance handles (registers scale with KMAX * UNROLL);
-// UNROLL: row vectors per lane whose gathers are all in flight together.
-template <int KMAX, int UNROLL>
+// UNROLL: row vectors per lane whose gathers are all in flight together; OutT: float or bf16.
+template <int KMAX, int UNROLL, typename OutT>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ dest,
                                                       const float* __restrict__ w, const float* __restrict__ base,
-                                                      int T, int k, int d, int rows, float* __restrict__ out) {
+                                                      int T, int k, int d, int rows, OutT* __restrict__ out) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     const int vec_per_row = d / 4;  // float4 vectors
@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
             wr[j] = __shfl_sync(0xffffffffu, mine_w, j);
             if (j >= k || dr[j] >= rows) dr[j] = -1;  // dropped, or outside Yp: contributes nothing
         }
-        float4* orow = reinterpret_cast<float4*>(out + static_cast<size_t>(t) * d);
+        OutT* orow = out + static_cast<size_t>(t) * d;
         const float4* brow = base ? reinterpret_cast<const float4*>(base + static_cast<size_t>(t) * d) : nullptr;
         for (int v0 = lane; v0 < vec_per_row; v0 += 32 * UNROLL) {
             // all gathers of UNROLL vectors issued before any is used
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                         acc.w = fmaf(wr[j], val[u][j].w, acc.w);
                     }
                 }
-                orow[v] = acc;
+                store_out4(orow, v, acc);
             }
         }
     }
@@ -77,17 +77,26 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 }  // namespace
 
+template <typename OutT>
+static void launch_combine_t(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
+                             int d, int rows, OutT* out, int grid, cudaStream_t stream) {
+    if (k <= 2)
+        combine_kernel<2, 4, OutT><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
+    else if (k <= 4)
+        combine_kernel<4, 2, OutT><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
+    else
+        combine_kernel<kMaxTopK, 2, OutT><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
+}
+
 cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
-                           int d, int rows, float* out, int num_sms, cudaStream_t stream) {
+                           int d, int rows, void* out, bool out_bf16, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     int grid = (T + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
-    if (k <= 2)
-        combine_kernel<2, 4><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
-    else if (k <= 4)
-        combine_kernel<4, 2><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
+    if (out_bf16)
+        launch_combine_t(yp, dest, w, base, T, k, d, rows, static_cast<__nv_bfloat16*>(out), grid, stream);
     else
-        combine_kernel<kMaxTopK, 2><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
+        launch_combine_t(yp, dest, w, base, T, k, d, rows, static_cast<float*>(out), grid, stream);
     return cudaGetLastError();
 }
 

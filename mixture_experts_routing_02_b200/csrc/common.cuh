@@ -278,6 +278,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Store 4 consecutive output values at element 4*v of `row`: one 16-byte fp32 store, or one
+// 8-byte store of four values rounded to bf16 (round to nearest even).
+__device__ __forceinline__ void store_out4(float* row, int v, float4 a) { reinterpret_cast<float4*>(row)[v] = a; }
+__device__ __forceinline__ void store_out4(__nv_bfloat16* row, int v, float4 a) {
+    reinterpret_cast<uint2*>(row)[v] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 

@@ -10,7 +10,7 @@
 //     (segment e = expert e, C' rows) and the [T, E] map from (token, expert) to row.
 //   * ec_gather_kernel: Xp[r] = X[src[r]], one warp per row, 16-byte vectors.
 //   * ec_combine_kernel: out[t] = base[t] + sum of row_w[r] * Yp[r] over the rows r of
-//     token t in ascending expert order, one warp per token.
+//     token t in ascending expert order, one warp per token; out in fp32 or bf16.
 // The gather and the combine are HBM-bound; the selection reads the E x T scores four
 // times, from L2.
 #include "common.cuh"
@@ -195,9 +195,10 @@ __device__ __forceinline__ void fma4(float4& acc, float w, const float4& y) {
     acc.w = fmaf(w, y.w, acc.w);
 }
 
+template <typename OutT>
 __global__ void __launch_bounds__(kCombineWarps * 32)
     ec_combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ emap, const float* __restrict__ row_w,
-                      const float* __restrict__ base, int T, int E, int d, int rows, float* __restrict__ out) {
+                      const float* __restrict__ base, int T, int E, int d, int rows, OutT* __restrict__ out) {
     __shared__ int2 picks[kCombineWarps][kMaxExperts];  // (row, weight bits) of the current token
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int warps_total = gridDim.x * kCombineWarps;
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
             n += __popc(ball);
         }
         __syncwarp();
-        float4* orow = reinterpret_cast<float4*>(out + static_cast<size_t>(t) * d);
+        OutT* orow = out + static_cast<size_t>(t) * d;
         const float4* brow = base ? reinterpret_cast<const float4*>(base + static_cast<size_t>(t) * d) : nullptr;
         for (int v0 = lane; v0 < vec_per_row; v0 += 32 * kCombineUnroll) {
             float4 acc[kCombineUnroll];
@@ -259,7 +260,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
             }
 #pragma unroll
             for (int u = 0; u < kCombineUnroll; ++u)
-                if (v0 + 32 * u < vec_per_row) orow[v0 + 32 * u] = acc[u];
+                if (v0 + 32 * u < vec_per_row) store_out4(orow, v0 + 32 * u, acc[u]);
         }
         __syncwarp();
     }
@@ -297,11 +298,16 @@ cudaError_t launch_ec_gather(const __nv_bfloat16* x, const int32_t* src, int row
 }
 
 cudaError_t launch_ec_combine(const float* yp, const int32_t* emap, const float* row_w, const float* base, int T,
-                              int E, int d, int rows, float* out, int num_sms, cudaStream_t stream) {
+                              int E, int d, int rows, void* out, bool out_bf16, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     int grid = (T + kCombineWarps - 1) / kCombineWarps;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
-    ec_combine_kernel<<<grid, kCombineWarps * 32, 0, stream>>>(yp, emap, row_w, base, T, E, d, rows, out);
+    if (out_bf16)
+        ec_combine_kernel<__nv_bfloat16><<<grid, kCombineWarps * 32, 0, stream>>>(
+            yp, emap, row_w, base, T, E, d, rows, static_cast<__nv_bfloat16*>(out));
+    else
+        ec_combine_kernel<float><<<grid, kCombineWarps * 32, 0, stream>>>(yp, emap, row_w, base, T, E, d, rows,
+                                                                          static_cast<float*>(out));
     return cudaGetLastError();
 }
 

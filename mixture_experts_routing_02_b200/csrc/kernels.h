@@ -144,8 +144,9 @@ cudaError_t launch_route_logits(const float* part, int n_split, int ldp, size_t 
                                 int num_sms, cudaStream_t stream);
 
 // combine.cu
+// out: [T, d] fp32, or bf16 when out_bf16
 cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
-                           int d, int rows, float* out, int num_sms, cudaStream_t stream);
+                           int d, int rows, void* out, bool out_bf16, int num_sms, cudaStream_t stream);
 
 // expert_choice.cu
 constexpr int kSelectThreads = 1024;  // one CTA per expert
@@ -154,7 +155,7 @@ cudaError_t launch_ec_select(const float* scores_t, int T, int E, int cp, int32_
 cudaError_t launch_ec_gather(const __nv_bfloat16* x, const int32_t* src, int rows, int T, int d, __nv_bfloat16* xp,
                              int num_sms, cudaStream_t stream);
 cudaError_t launch_ec_combine(const float* yp, const int32_t* emap, const float* row_w, const float* base, int T,
-                              int E, int d, int rows, float* out, int num_sms, cudaStream_t stream);
+                              int E, int d, int rows, void* out, bool out_bf16, int num_sms, cudaStream_t stream);
 
 // stats.cu: MOE_STAT_COUNT values from the counts (nullable) and segment tables of one dispatch
 cudaError_t launch_routing_stats(const int32_t* counts, const int32_t* seg_expert, const int32_t* seg_offsets,

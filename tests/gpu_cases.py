@@ -167,16 +167,19 @@ def to_np(t):
     return t.detach().cpu().numpy()
 
 
-def run_layer(case: Case, capacity=None, stream=None, route_flags=0):
-    """moe_layer_fwd through the C ABI; returns the output and every intermediate (CPU)."""
+def run_layer(case: Case, capacity=None, stream=None, route_flags=0, out_dtype=moe.DTYPE_F32):
+    """moe_layer_fwd through the C ABI; returns the output (fp32 or bf16 on the device) and every
+    intermediate (CPU)."""
     w = case.w
     s = moe_shape(w, capacity)
     s.route_flags |= route_flags
+    s.out_dtype = out_dtype
     n_seg, rows = moe.moe_layout(s)
     _, layer_bytes = moe.moe_workspace_size(s)
     ws = torch.empty(layer_bytes, dtype=torch.uint8, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out = torch.full((w.T, w.d), float("nan"), dtype=torch.float32, device="cuda")
+    out = torch.full((w.T, w.d), float("nan"), device="cuda",
+                     dtype=torch.bfloat16 if out_dtype == moe.DTYPE_BF16 else torch.float32)
     x, w_r, bias = dev(case.x), dev(case.w_r), dev(case.bias)
     wg, wu, wd = dev(case.wg), dev(case.wu), dev(case.wd)
     moe.moe_layer_fwd(s, x, w_r, bias, wg, wu, wd, out, status, ws, stream=stream)

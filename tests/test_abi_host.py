@@ -220,7 +220,7 @@ def test_header_is_plain_c_and_the_library_links_from_c(lib, tmp_path):
     src.write_text(
         '#include <stdio.h>\n#include "moe_routing.h"\n'
         "int main(void) {\n"
-        "    moe_shape_t s = {64, 128, 8, 2, 256, 0, 0, 0, 0};\n"
+        "    moe_shape_t s = {64, 128, 8, 2, 256, 0, 0, 0, 0, MOE_DTYPE_BF16};\n"
         "    int32_t n_seg = 0, rows = 0;\n"
         "    size_t disp = 0, layer = 0;\n"
         "    if (moe_layout(&s, &n_seg, &rows) != MOE_OK) return 1;\n"
@@ -243,3 +243,10 @@ def test_missing_library_fails_loudly(tmp_path):
     """No fallback: without the built library every call raises instead of computing elsewhere."""
     with pytest.raises(RuntimeError, match="not built"):
         moe.load_library(str(tmp_path / "libmoe_b200.so"))
+
+
+def test_out_dtype_is_validated(lib):
+    """out_dtype takes MOE_DTYPE_F32 (0) or MOE_DTYPE_BF16 (1); anything else is rejected."""
+    for dt, want in ((moe.DTYPE_F32, 0), (moe.DTYPE_BF16, 0), (2, 1), (-1, 1)):
+        s = moe.shape(64, 128, 8, 2, 256, out_dtype=dt)
+        assert lib.moe_layout(ctypes.byref(s), None, None) == want

@@ -4,13 +4,15 @@ moe_layer_fwd (the launch configuration the benchmark times).
 Every index output (top-k ids, counts, segment tables, dest, src) is compared
 with the oracle in full, bit for bit; every permuted row is checked to be an
 exact copy of its token; floating-point outputs are compared on sampled rows
-and tokens that the oracle evaluates one by one in fp64.
+and tokens that the oracle evaluates one by one in fp64.  The layer output is
+stored in bf16, the type the layer returns in the benchmark.
 """
 import numpy as np
 import pytest
 import torch
 
 import oracle
+import mixture_experts_routing_02_b200 as moe
 from mixture_experts_routing_02_b200 import synthetic as syn
 
 from gpu_cases import (check_bf16_storage, check_close, check_layer_output, expert_rows, make_case, oracle_segments,
@@ -24,8 +26,8 @@ FULL = [syn.MIXTRAL_LIKE, syn.DEEPSEEK_LIKE, syn.SKEWED, syn.BALANCED]
 @pytest.mark.parametrize("w", FULL, ids=[w.name for w in FULL])
 def test_full_size_layer(cuda_ok, w):
     case = make_case(w, seed=0, weights_device="cuda")
-    got = run_layer(case)
-    assert got["status"] == 0
+    got = run_layer(case, out_dtype=moe.DTYPE_BF16)
+    assert got["status"] == 0 and got["out"].dtype == torch.bfloat16
 
     # routing of all T tokens
     logits, ids, wts = oracle.route(case.x, case.w_r, case.bias, w.k)
@@ -82,7 +84,6 @@ def test_full_size_layer(cuda_ok, w):
 
 def test_full_size_shared_expert(cuda_ok):
     """DeepSeek-like shape with one shared expert (F_s = 2048): sampled rows against the oracle."""
-    import mixture_experts_routing_02_b200 as moe
     w = syn.DEEPSEEK_LIKE
     Fs = 2048
     x, _, _ = syn.router_inputs(w, 0)

@@ -78,6 +78,55 @@ def test_layer_matches_oracle(w):
     check_layer_output(to_np(got["out"]), ref.out, ref.dest, w.T, w.k)
 
 
+BF16_OUT = ["tiny", "ragged", "capacity", "plan", "one-token", "count-largest", "lookback-capacity"]
+
+
+@pytest.mark.parametrize("name", BF16_OUT)
+def test_layer_bf16_output(name):
+    """out_dtype = bf16: the layer output is the fp32 combine rounded once to bf16 (round to nearest
+    even), bit for bit, and meets the stated tolerance against the fp64 oracle; fully dropped
+    tokens are exactly 0."""
+    w = next(x for x in SMALL if x.name == name)
+    case = make_case(w, seed=1)
+    ref = _oracle_layer(case)
+    f32 = run_layer(case)
+    b16 = run_layer(case, out_dtype=moe.DTYPE_BF16)
+    assert f32["status"] == 0 and b16["status"] == 0
+    assert b16["out"].dtype == torch.bfloat16
+    assert torch.equal(b16["out"], f32["out"].to(torch.bfloat16)), "bf16 output is not the rounded fp32 output"
+    check_layer_output(to_np(b16["out"]), ref.out, ref.dest, w.T, w.k, "bf16 out")
+
+
+def test_combine_add_and_expert_choice_bf16_output():
+    """moe_combine_add and moe_combine_expert_choice with a bf16 out: the fp32 results rounded once;
+    a bf16 out aliasing the fp32 base is rejected."""
+    w = syn.Workload("combine-bf16", T=257, d=192, E=6, k=3, F=64, zipf_s=1.0, capacity_factor=0.8)
+    s32 = moe_shape(w)
+    s16 = moe_shape(w)
+    s16.out_dtype = moe.DTYPE_BF16
+    n_seg, rows = moe.moe_layout(s32)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    yp = torch.randn(rows, w.d, device="cuda", generator=g)
+    base = torch.randn(w.T, w.d, device="cuda", generator=g)
+    wts = torch.rand(w.T, w.k, device="cuda", generator=g)
+    dest = torch.randint(-1, rows, (w.T * w.k,), device="cuda", dtype=torch.int32, generator=g)
+    o32 = torch.empty(w.T, w.d, device="cuda")
+    o16 = torch.empty(w.T, w.d, device="cuda", dtype=torch.bfloat16)
+    moe.moe_combine_add(s32, yp, dest, wts, base, o32)
+    moe.moe_combine_add(s16, yp, dest, wts, base, o16)
+    torch.cuda.synchronize()
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    with pytest.raises(moe.MoeError):
+        moe.moe_combine_add(s16, yp, dest, wts, base, base)
+
+    e = syn.Workload("ec-bf16", T=300, d=128, E=8, k=2, F=64, capacity_factor=1.0, expert_choice=True)
+    case = make_case(e, seed=4)
+    ref32 = run_layer(case)
+    got16 = run_layer(case, out_dtype=moe.DTYPE_BF16)
+    assert ref32["status"] == 0 and got16["status"] == 0
+    assert torch.equal(got16["out"], ref32["out"].to(torch.bfloat16))
+
+
 def test_layer_softmax_all_variant():
     """The whole layer with weights from a softmax over all experts (no renormalisation)."""
     w = syn.Workload("softmax-all", T=300, d=192, E=16, k=4, F=128, zipf_s=0.8)

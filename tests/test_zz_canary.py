@@ -62,7 +62,8 @@ def _run_topk(case, s):
         ids=((T, k), torch.int32), wts=((T, k), torch.float32), counts=((E,), torch.int32),
         seg_e=((n_seg,), torch.int32), seg_o=((n_seg + 1,), torch.int32), seg_f=((n_seg,), torch.int32),
         dest=((T * k,), torch.int32), src=((rows,), torch.int32), xp=((rows, d), torch.bfloat16),
-        hp=((rows, F), torch.bfloat16), yp=((rows, d), torch.float32), out=((T, d), torch.float32),
+        hp=((rows, F), torch.bfloat16), yp=((rows, d), torch.float32),
+        out=((T, d), torch.bfloat16 if s.out_dtype == moe.DTYPE_BF16 else torch.float32),
         logits=((T, E), torch.float32), route_ws=((max(route_ws_bytes, 1),), torch.uint8),
         dws=((max(disp_bytes, 1),), torch.uint8)))
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -117,6 +118,20 @@ def test_topk_calls_write_only_their_buffers(cuda_ok, w):
     ref = run_layer(case)
     assert ref["status"] == 0
     assert np.array_equal(to_np(g["out"].t), to_np(ref["out"])), "call-by-call output differs from moe_layer_fwd"
+
+
+def test_bf16_output_writes_only_its_buffer(cuda_ok):
+    """With out_dtype = bf16 the combine writes T * d * 2 bytes and nothing around them."""
+    w = CASES[0]
+    case = make_case(w, seed=33)
+    s = moe_shape(w)
+    s.out_dtype = moe.DTYPE_BF16
+    g, used, rr = _run_topk(case, s)
+    assert g["out"].t.dtype == torch.bfloat16
+    g["out"].check("out")
+    ref = run_layer(case, out_dtype=moe.DTYPE_BF16)
+    assert ref["status"] == 0
+    assert torch.equal(g["out"].t, ref["out"]), "call-by-call output differs from moe_layer_fwd"
 
 
 def test_expert_choice_calls_write_only_their_buffers(cuda_ok):
