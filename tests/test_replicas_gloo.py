@@ -57,7 +57,7 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
 
     class A:
-        steps, warmup, seed, gpus = 1, 0, 0, 2
+        steps, warmup, seed, gpus, out_dtype = 1, 0, 0, 2, "bf16"
 
     from mixture_experts_routing_02_b200 import synthetic as syn
     assert bench.run_reference(A, syn.TINY) == 0      # returns at once, no work, no output
@@ -71,7 +71,7 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "1")
 
     class A:
-        steps, warmup, seed, gpus = 1, 0, 0, 1
+        steps, warmup, seed, gpus, out_dtype = 1, 0, 0, 1, "bf16"
 
     from mixture_experts_routing_02_b200 import synthetic as syn
     assert bench.run_reference(A, syn.TINY) == 0
