@@ -419,6 +419,22 @@ MOE_API moe_status_t moe_testing_dispatch_stalled(const moe_shape_t *shape, cons
                                           moe_stream_t stream);
 
 /*
+ * Testing only: moe_expert_gate_up in which CTA 0 never issues the copy of its
+ * first pipeline stage, so the tensor-core issuer's wait on that stage can never
+ * end.  The wait gives up after its bound (about 2 s), sets MOE_DEV_ERR_TIMEOUT
+ * in *status and raises the CTA's abort flag; the copy issuer and the epilogue
+ * warps see it and stop, the copies already in flight are waited for (bounded),
+ * and the CTA frees its tensor memory before it exits.  The tiles of CTA 0 are
+ * not written; the other CTAs' tiles are.  It shows that the GEMM's abort path
+ * returns an error instead of hanging and leaves the context (and the SMs'
+ * tensor memory) usable.  Needs at least one row (rows_alloc > 0 and T > 0).
+ */
+MOE_API moe_status_t moe_testing_gemm_stalled(const moe_shape_t *shape, const moe_bf16_t *xp,
+                                      const int32_t *seg_expert, const int32_t *seg_offsets,
+                                      const moe_bf16_t *w_gate, const moe_bf16_t *w_up, moe_bf16_t *hp,
+                                      int32_t *status, moe_stream_t stream);
+
+/*
  * The router projection on more CTAs.  Its ceil(T/128) row tiles can be fewer than the SMs;
  * with a workspace the reduction over d is split into S parts (S chosen from T, d and the SM
  * count; each part at least 256 columns of d), the parts' fp32 partial logits go to the

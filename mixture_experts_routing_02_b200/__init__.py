@@ -66,6 +66,7 @@ SYMBOLS = {
     "moe_dispatch_static": [_S, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_testing_dispatch_stalled": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_expert_gate_up": [_S, _P, _P, _P, _P, _P, _P, _P, _P],
+    "moe_testing_gemm_stalled": [_S, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_expert_down": [_S, _P, _P, _P, _P, _P, _P, _P],
     "moe_expert_ffn": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_combine": [_S, _P, _P, _P, _P, _P],
@@ -211,6 +212,13 @@ def moe_testing_dispatch_stalled(s, x, topk_ids, counts, seg_expert, seg_offsets
 
 def moe_expert_gate_up(s, xp, seg_expert, seg_offsets, w_gate, w_up, hp, status=None, stream=None):
     _check("moe_expert_gate_up", load_library().moe_expert_gate_up(
+        ctypes.byref(s), _ptr(xp), _ptr(seg_expert), _ptr(seg_offsets), _ptr(w_gate), _ptr(w_up), _ptr(hp),
+        _ptr(status), _stream(stream)))
+
+
+def moe_testing_gemm_stalled(s, xp, seg_expert, seg_offsets, w_gate, w_up, hp, status, stream=None):
+    """Testing only: a gate/up GEMM whose first pipeline stage is never filled; its waits time out."""
+    _check("moe_testing_gemm_stalled", load_library().moe_testing_gemm_stalled(
         ctypes.byref(s), _ptr(xp), _ptr(seg_expert), _ptr(seg_offsets), _ptr(w_gate), _ptr(w_up), _ptr(hp),
         _ptr(status), _stream(stream)))
 

@@ -245,7 +245,7 @@ moe_status_t choose_impl(const Dims& v, const float* scores, const moe_bf16_t* x
 
 moe_status_t gate_up_impl(const Dims& v, const moe_bf16_t* xp, const int32_t* seg_expert, const int32_t* seg_offsets,
                           const moe_bf16_t* wg, const moe_bf16_t* wu, moe_bf16_t* hp, int32_t* status,
-                          cudaStream_t st) {
+                          cudaStream_t st, bool test_stall = false) {
     if (!xp || !seg_expert || !seg_offsets || !wg || !wu || !hp) return MOE_ERR_INVALID_ARG;
     if (!aligned16(xp) || !aligned16(wg) || !aligned16(wu) || !aligned16(hp)) return MOE_ERR_INVALID_ARG;
     if (v.T == 0 || v.rows == 0) return MOE_OK;
@@ -259,6 +259,7 @@ moe_status_t gate_up_impl(const Dims& v, const moe_bf16_t* xp, const int32_t* se
     g.seg_offsets = seg_offsets; g.seg_expert = seg_expert; g.n_seg = v.n_seg; g.M = v.rows; g.K = v.d; g.N = v.F;
     g.BN = bn; g.n_tiles_n = (v.F + bn - 1) / bn; g.mma_n = 2 * bn;
     g.out = hp; g.ldo = v.F; g.k = v.k; g.status = status;
+    g.test_skip_first_load = test_stall ? 1 : 0;
     g.stages = gemm_pick_stages(2 * bn);
     const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 128 + v.n_seg) * g.n_tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(sm_count(), max_tiles));
@@ -648,6 +649,17 @@ moe_status_t moe_testing_dispatch_stalled(const moe_shape_t* shape, const moe_bf
     if (permute_n_tiles(v.T, v.k) < 2) return MOE_ERR_INVALID_ARG;  // needs a tile that waits on tile 0
     return dispatch_impl(v, x, topk_ids, 0, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp, status,
                          ws, ws_bytes, static_cast<cudaStream_t>(stream), 1);
+}
+
+moe_status_t moe_testing_gemm_stalled(const moe_shape_t* shape, const moe_bf16_t* xp, const int32_t* seg_expert,
+                                      const int32_t* seg_offsets, const moe_bf16_t* w_gate, const moe_bf16_t* w_up,
+                                      moe_bf16_t* hp, int32_t* status, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (v.T == 0 || v.rows == 0) return MOE_ERR_INVALID_ARG;  // needs a tile whose wait can run out
+    return gate_up_impl(v, xp, seg_expert, seg_offsets, w_gate, w_up, hp, status, static_cast<cudaStream_t>(stream),
+                        true);
 }
 
 moe_status_t moe_combine_add(const moe_shape_t* shape, const float* yp, const int32_t* dest, const float* topk_w,

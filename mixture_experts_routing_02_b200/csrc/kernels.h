@@ -40,6 +40,7 @@ struct GemmArgs {
     int k_splits;          // plain fp32 epilogue only: > 1 cuts the reduction into this many parts
     size_t split_stride;   // elements between the outputs of consecutive parts
     int32_t* status;
+    int test_skip_first_load;  // testing only: CTA 0 never issues its first stage's copy (its waits time out)
 };
 
 size_t gemm_smem_bytes(int stages, int mma_n);

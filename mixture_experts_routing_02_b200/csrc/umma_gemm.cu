@@ -223,6 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0, issued = 0;
             uint32_t phase = 0;
             const uint32_t tx = kABytes + (EPI == kEpiRoute ? static_cast<uint32_t>(g.N) * 128u : b_stage_bytes);
+            // testing only (moe_testing_gemm_stalled): CTA 0's first stage is never filled, so the
+            // MMA warp's bounded wait on it runs out and every role takes the abort path
+            const bool skip_first = g.test_skip_first_load != 0 && blockIdx.x == 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
                 const int split = SPLITK ? tile % n_split : 0;
@@ -232,17 +235,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int kb1 = SPLITK ? (split + 1) * nkb / n_split : nkb;
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, g.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full_bar[stage], tx);
-                    uint8_t* a_dst = sA + stage * kABytes;
-                    uint8_t* b_dst = sB + stage * b_stage_bytes;
-                    tma_load_2d(a_dst, &tmA, kb * kBK, c.row0, &full_bar[stage]);
-                    if (EPI == kEpiRoute) {
-                        tma_load_2d(b_dst, &tmB0, kb * kBK, 0, &full_bar[stage]);
-                    } else if (EPI == kEpiSwiglu) {
-                        tma_load_3d(b_dst, &tmB0, kb * kBK, n0, c.expert, &full_bar[stage]);
-                        tma_load_3d(b_dst + g.BN * 128, &tmB1, kb * kBK, n0, c.expert, &full_bar[stage]);
-                    } else {
-                        tma_load_3d(b_dst, &tmB0, kb * kBK, n0, c.expert, &full_bar[stage]);
+                    if (!(skip_first && issued == 0)) {
+                        mbar_arrive_expect_tx(&full_bar[stage], tx);
+                        uint8_t* a_dst = sA + stage * kABytes;
+                        uint8_t* b_dst = sB + stage * b_stage_bytes;
+                        tma_load_2d(a_dst, &tmA, kb * kBK, c.row0, &full_bar[stage]);
+                        if (EPI == kEpiRoute) {
+                            tma_load_2d(b_dst, &tmB0, kb * kBK, 0, &full_bar[stage]);
+                        } else if (EPI == kEpiSwiglu) {
+                            tma_load_3d(b_dst, &tmB0, kb * kBK, n0, c.expert, &full_bar[stage]);
+                            tma_load_3d(b_dst + g.BN * 128, &tmB1, kb * kBK, n0, c.expert, &full_bar[stage]);
+                        } else {
+                            tma_load_3d(b_dst, &tmB0, kb * kBK, n0, c.expert, &full_bar[stage]);
+                        }
                     }
                     ++issued;
                     if (++stage == stages) { stage = 0; phase ^= 1u; }
@@ -251,8 +256,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) {
                 // give every copy still in flight a bounded chance to land before the CTA exits
                 const int first = issued > stages ? issued - stages : 0;
-                for (int i = first; i < issued; ++i)
+                for (int i = first; i < issued; ++i) {
+                    if (skip_first && i == 0) continue;  // never issued
                     mbar_wait(&full_bar[i % stages], static_cast<uint32_t>((i / stages) & 1), nullptr, nullptr);
+                }
             }
         }
         __syncwarp();

@@ -61,3 +61,35 @@ def test_stalled_dispatch_needs_two_tiles(cuda_ok):
                                          dummy, dummy, dummy, dummy, dummy,
                                          torch.zeros(20, 64, dtype=torch.bfloat16, device="cuda"), None,
                                          torch.zeros(1 << 16, dtype=torch.uint8, device="cuda"))
+
+
+def test_gemm_wait_that_cannot_end_times_out(cuda_ok):
+    """The grouped GEMM's abort path: CTA 0's first pipeline stage is never filled, so its tensor-core
+    issuer's wait runs out after ~2 s; the status reports the timeout, the CTA frees its tensor memory
+    and returns, and a normal gate/up projection right after (which allocates all tensor memory of
+    every SM it runs on) matches the oracle."""
+    from gpu_cases import check_bf16_storage, make_case
+    w = syn.Workload("stall", T=300, d=256, E=4, k=2, F=256, zipf_s=0.5)
+    case = make_case(w, seed=40)
+    ref = oracle.layer_forward(case.x, case.w_r, case.bias, case.wg, case.wu, case.wd, w.k)
+    s = moe.shape(w.T, w.d, w.E, w.k, w.F)
+    to_i32 = lambda a: torch.from_numpy(np.asarray(a, dtype=np.int32)).cuda()
+    xp = torch.from_numpy(ref.xp.astype(np.float32)).to(torch.bfloat16).cuda()
+    seg_e, seg_o = to_i32(ref.segs.expert), to_i32(ref.segs.offsets)
+    wg, wu = case.wg.cuda(), case.wu.cuda()
+    rows = xp.shape[0]
+    hp = torch.zeros(rows, w.F, dtype=torch.bfloat16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    moe.moe_testing_gemm_stalled(s, xp, seg_e, seg_o, wg, wu, hp, st)
+    torch.cuda.synchronize()
+    elapsed = time.time() - t0
+    assert st.item() & moe.DEV_ERR_TIMEOUT
+    assert 1.0 < elapsed < 60.0
+
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hp2 = torch.zeros(rows, w.F, dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_gate_up(s, xp, seg_e, seg_o, wg, wu, hp2, st2)
+    torch.cuda.synchronize()
+    assert st2.item() == 0
+    check_bf16_storage(hp2.float().cpu().numpy(), ref.hp, "Hp after the aborted GEMM")
