@@ -2,11 +2,13 @@
 """Benchmark of the single-GPU top-k MoE FFN layer forward (B200).
 
 One step = one whole layer forward over one batch of T tokens through the C
-ABI: moe_route -> moe_dispatch -> moe_expert_gate_up -> moe_expert_down ->
-moe_combine (the calls moe_layer_fwd makes), with CUDA events between the
-calls so every kernel's duration is measured inside the timed region.  The
-default workload is the Mixtral-like layer (T=4096, d=4096, E=8, top-2,
-F=14336), random-init weights and seeded synthetic inputs.
+ABI.  Two timed loops of K steps each: (1) moe_layer_fwd alone, with CUDA
+events only around each step -- `value` and `ms_per_step`; (2) the calls
+moe_layer_fwd makes, moe_route -> moe_dispatch -> moe_expert_gate_up ->
+moe_expert_down -> moe_combine, with CUDA events between the calls, so every
+kernel's duration is measured -- `breakdown` and `roofline`.  The default
+workload is the Mixtral-like layer (T=4096, d=4096, E=8, top-2, F=14336),
+random-init weights and seeded synthetic inputs, bf16 output.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -516,12 +518,23 @@ def run_ours(args, w):
     active_experts = int((torch.bincount(seg_e[seg_o[1:] > seg_o[:-1]].long().clamp_min(0),
                                          minlength=w.E) > 0).sum().item())
 
-    # timed region: K steps, events between every call.  Clocks are sampled through both timed
-    # regions (these steps and the end-to-end run below), which also gives a short step loop
-    # enough samples.
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    # timed regions.  Clocks are sampled through all of them (the layer loop, the call-by-call
+    # loop and the end-to-end run below), which also gives a short step loop enough samples.
+    # (1) the layer through moe_layer_fwd, events only around each step: its kernels may overlap
+    # their neighbours' launch and prologue (programmatic dependent launch)
+    layer_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
     barrier()
     clocks = ClockSampler(local).__enter__()
+    if not Fs:
+        for i in range(args.steps):
+            flush.zero_()
+            layer_ev[i][0].record(stream)
+            moe.moe_layer_fwd(s, x, w_r, bias, wg, wu, wd, out, status, ws, stream)
+            layer_ev[i][1].record(stream)
+        barrier()
+    # (2) call by call with events between the calls: each kernel's duration
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()
         step(events[i])
@@ -532,7 +545,9 @@ def run_ours(args, w):
         step_ms.append(ev[0].elapsed_time(ev[5]))
         for j, k in enumerate(KERNELS):
             per_kernel[k].append(ev[j].elapsed_time(ev[j + 1]))
-    total_ms = sum(step_ms)
+    calls_ms = sum(step_ms)
+    # with a shared expert the layer is the call sequence itself (moe_layer_fwd has no shared expert)
+    total_ms = calls_ms if Fs else sum(a.elapsed_time(b) for a, b in layer_ev)
 
     # end to end through moe_layer_fwd with host buffers (pipelined steps; the weights, 2.8 GB and
     # more, stream through L2 every step, so no extra flush)
@@ -544,7 +559,7 @@ def run_ours(args, w):
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()}")
 
-    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, world)
+    total_ms, e2e_ms, calls_ms = max_over_ranks([total_ms, e2e_ms, calls_ms], dev, world)
 
     shared_info = None
     if Fs:
@@ -611,7 +626,9 @@ def run_ours(args, w):
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init weights)", "config": _config(w, capacity, args.out_dtype),
-        "rows_dispatched": rows_used, "gpu_launches": launches * args.steps,
+        "rows_dispatched": rows_used,
+        "gpu_launches": launches * ((1 if Fs else 2) * args.steps + e2e_steps),
+        "ms_per_step_call_by_call": calls_ms / args.steps,
         "roofline": roof,
         "layer_roofline": dict(layer_roof, ms_per_step=total_ms / args.steps,
                                frac=layer_roof["roofline_ms"] / (total_ms / args.steps)),
@@ -628,7 +645,7 @@ def run_ours(args, w):
     if shared_info:
         line["shared_expert"] = shared_info
         line["config"]["shared_expert_d_ff"] = Fs
-        line["gpu_launches"] = (launches + 2) * args.steps
+        line["gpu_launches"] = (launches + 2) * args.steps + launches * e2e_steps
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_exp = min(4, w.E)
         wg0, wu0, wd0 = wg[:n_exp].cpu(), wu[:n_exp].cpu(), wd[:n_exp].cpu()
@@ -642,6 +659,115 @@ def run_ours(args, w):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+# ----------------------------------------------------------------------------- expert parallelism, one GPU
+
+EP_PHASES = ("route", "plan", "prefetch", "dispatch", "ffn", "combine")
+
+
+def run_ep_virtual(args, w):
+    """The balanced-plan layer as R expert-parallel ranks on one GPU (n_groups of the workload):
+    every rank's buffers are its own, the dispatch stores each row into its owner's final slot and
+    the combine reads the owners' outputs, the way R GPUs would run them -- with every "peer" in
+    local memory, so NVLink is not measured.  Same JSON line as the single-GPU arm."""
+    import torch
+
+    import mixture_experts_routing_02_b200 as moe
+    from mixture_experts_routing_02_b200 import ep
+    from mixture_experts_routing_02_b200 import synthetic as syn
+
+    world, rank, local = _dist()
+    if world > 1:
+        raise SystemExit("--ep-virtual runs on one GPU")
+    if not w.n_groups:
+        raise SystemExit("--ep-virtual needs a balanced-plan workload (n_groups > 0)")
+    torch.cuda.set_device(local)
+    moe.load_library()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    R, S = w.n_groups, w.tokens_per_group
+    out_bf16 = args.out_dtype == "bf16"
+    s = ep.ep_shape(R, S, w.d, w.E, w.k, w.F, w.replica_slots,
+                    out_dtype=moe.DTYPE_BF16 if out_bf16 else moe.DTYPE_F32)
+    x_cpu, w_r, bias = syn.router_inputs(w, args.seed)
+    x = x_cpu.to(dev)
+    w_r = w_r.to(dev)
+    bias = bias.to(dev) if bias is not None else None
+    wg, wu, wd = syn.expert_weights(w, args.seed, device=dev)
+    vr = ep.VirtualRanks(s, wg, wu, wd, device=dev)
+    del wg, wu, wd
+    torch.cuda.empty_cache()
+    xs = [x[r * S:(r + 1) * S] for r in range(R)]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        vr.forward(xs, w_r, bias, stream)
+    torch.cuda.synchronize()
+    if vr.status.item() != 0:
+        raise RuntimeError(f"device status {vr.status.item()} after warm-up")
+
+    steps = []
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local).__enter__()
+    for _ in range(args.steps):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True)]
+        ev[0].record(stream)
+
+        def mark(name, ev=ev):
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            ev.append(e)
+        vr.forward(xs, w_r, bias, stream, mark)
+        steps.append(ev)
+    torch.cuda.synchronize()
+    clocks.__exit__(None, None, None)
+    if vr.status.item() != 0:
+        raise RuntimeError(f"device status {vr.status.item()}")
+    total_ms = sum(ev[0].elapsed_time(ev[-1]) for ev in steps)
+    phase_ms = {p: statistics.mean(ev[i].elapsed_time(ev[i + 1]) for ev in steps) for i, p in enumerate(EP_PHASES)}
+
+    hbm, bf16, bf16_sus, peak_kind = _peaks()
+    T, d, k, F = w.T, w.d, w.k, w.F
+    rows = T * k
+    out_bytes = 2 if out_bf16 else 4
+    used_slots = sum(int(((b.seg_slot[w.E // R:] >= 0)).sum().item()) for b in vr.bufs)
+    breakdown = {
+        "dispatch": dict(ms=phase_ms["dispatch"], bytes=T * d * 2 + rows * d * 2 + rows * 4 * 3),
+        "prefetch": dict(ms=phase_ms["prefetch"], bytes=used_slots * 3 * F * d * 2 * 2,
+                         replica_slots_filled=used_slots),
+        "ffn": dict(ms=phase_ms["ffn"], flops=6 * rows * d * F),
+        "combine": dict(ms=phase_ms["combine"], bytes=rows * d * 4 + T * d * out_bytes + rows * 8),
+        "route": dict(ms=phase_ms["route"], bytes=T * d * 2 + T * k * 8),
+        "plan": dict(ms=phase_ms["plan"]),
+    }
+    for name, b in breakdown.items():
+        sec = b["ms"] / 1e3
+        if "bytes" in b:
+            b["gbs"] = b["bytes"] / sec / 1e9
+            b["frac_hbm_peak"] = b["gbs"] / hbm
+        if "flops" in b:
+            b["tflops"] = b["flops"] / sec / 1e12
+            b["frac_bf16_peak"] = b["tflops"] / bf16
+    db = breakdown["ffn"]
+    line = {
+        "metric": METRIC, "value": job_throughput(T, args.steps, 1, total_ms), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random-init weights)",
+        "config": dict(_config(w, 0, args.out_dtype),
+                       parallelism=f"expert parallel: {R} virtual ranks on one GPU (every peer buffer local)"),
+        "gpu_launches": vr.kernel_launches() * (args.warmup + args.steps),
+        "roofline": {"bound": "tensor", "achieved": db["tflops"], "peak": bf16, "unit": "TFLOP/s",
+                     "frac": db["tflops"] / bf16, "kernel": "ffn (R ranks' grouped GEMMs)",
+                     "peak_source": f"{peak_kind} bf16_tflops (burst); sustained {bf16_sus}", "traffic": None},
+        "breakdown": {n: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in b.items()}
+                      for n, b in breakdown.items()},
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -659,10 +785,14 @@ def main():
                     help="add one shared expert of inner size F_S, overlapped on a second stream (needs --out-dtype f32)")
     ap.add_argument("--out-dtype", choices=("bf16", "f32"), default="bf16",
                     help="element type of the layer output (default bf16)")
+    ap.add_argument("--ep-virtual", action="store_true",
+                    help="run a balanced-plan workload as expert-parallel ranks on one GPU")
     args = ap.parse_args()
     w = syn.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.ep_virtual:
+        return run_ep_virtual(args, w)
     return run_ours(args, w)
 
 

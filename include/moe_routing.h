@@ -574,6 +574,115 @@ MOE_API moe_status_t moe_routing_stats(const moe_shape_t *shape, const int32_t *
                                const int32_t *seg_expert, const int32_t *seg_offsets,
                                int32_t *stats, moe_stream_t stream);
 
+/*
+ * Expert parallelism across R ranks, one GPU each ("가장 바쁜 랭크가 속도를
+ * 정합니다: MoonEP의 계획 코드를 직접 돌려봤습니다", sections "이 기술은 무엇인가"
+ * and "설치 및 통합"; "5.3 Expert Parallelism", section "2. 디스패처 엔지니어링").
+ * The balanced plan's R groups are R ranks: rank g owns the E/R experts homed
+ * in group g (experts [g*E/R, (g+1)*E/R)) plus B replica weight slots, holds
+ * S = T/R tokens, and computes exactly S*k rows.  A step on rank g:
+ *   route its S tokens (moe_route / moe_route_ws with T = S) and count them
+ *   (moe_histogram); gather every rank's counts into counts_all [R, E] (a
+ *   collective of the caller's); moe_ep_plan; moe_ep_prefetch_weights;
+ *   moe_ep_dispatch; a barrier; moe_ep_expert_ffn; a barrier; moe_ep_combine.
+ * The layout equals the single-GPU balanced plan over the R*S tokens in rank
+ * order: rank g's dispatched rows are rows [g*S*k, (g+1)*S*k) of that layout.
+ * Peer buffers are passed as HOST arrays of device pointers, one per rank
+ * (entry r = rank r's buffer, a peer-mapped address on a multi-GPU node); the
+ * kernels touch them with plain loads and stores only and never wait for
+ * another rank, so the barriers are the caller's stream-ordered collectives.
+ * With fewer GPUs than ranks, one call can serve several source ranks (n_src >
+ * 1) whose buffers all live on the calling GPU.
+ *
+ * Shape of every moe_ep_* call: T = R*S (all ranks' tokens), n_groups = R
+ * (1 <= R <= MOE_EP_MAX_RANKS), replica_slots = B, capacity = 0, no expert
+ * choice or re-routing; S*k <= 2^20.  Per rank:
+ *   weights   w_gate, w_up [E/R + B, F, d], w_down [E/R + B, d, F]: slot i < E/R
+ *             holds home expert g*E/R + i, slot E/R + j replica slot j
+ *   rows      xp [S*k, d] bf16, src [S*k] int32, hp [S*k, F] bf16, yp [S*k, d] fp32
+ *   tables    seg_expert / seg_slot [E/R + B], seg_offsets [E/R + B + 1]
+ */
+#define MOE_EP_MAX_RANKS 16
+
+/*
+ * Per-rank sizes (host only; outputs nullable): *xp_bytes = S*k*d*2, the
+ * dispatch buffer a rank receives into; *replica_weight_bytes = B*3*d*F*2, the
+ * replica weight slots (the MoonEP page's "실제 실험 결과" memory table: 0.44 GiB
+ * and 0.33 GiB at S = 4096, d = 7168, k = 8, F = 2048, B = 4);
+ * *n_local_segments = E/R + B.
+ */
+MOE_API moe_status_t moe_ep_sizes(const moe_shape_t *shape, size_t *xp_bytes, size_t *replica_weight_bytes,
+                          int32_t *n_local_segments);
+
+/*
+ * The balanced plan over all ranks from counts_all [R, E] (row r = rank r's
+ * raw counts), identical on every rank, reduced to rank `rank`'s segments:
+ *   counts      [E] out (nullable): total pairs of each expert
+ *   seg_expert  [E/R + B] out: global expert of each local segment (-1 unused)
+ *   seg_slot    [E/R + B] out: local weight slot of each segment (its index),
+ *               -1 for a segment without rows
+ *   seg_offsets [E/R + B + 1] out: rows of each segment inside the rank's S*k
+ * An infeasible plan sets MOE_DEV_ERR_PLAN and writes empty segments.  One CTA.
+ */
+MOE_API moe_status_t moe_ep_plan(const moe_shape_t *shape, int32_t rank, const int32_t *counts_all,
+                         int32_t *counts, int32_t *seg_expert, int32_t *seg_slot, int32_t *seg_offsets,
+                         int32_t *status, moe_stream_t stream);
+
+/*
+ * Replica weights (MoonEP page, "설치 및 통합": prefetch_weight fills the
+ * slots [E, E+B) from the plan).  For each replica slot j of rank `rank` whose
+ * segment has rows, the gate, up and down matrices of its expert e are copied
+ * from slot e - h*E/R of e's home rank h into slot E/R + j of this rank.
+ *   seg_expert, seg_offsets: this rank's tables (moe_ep_plan)
+ *   w_gate, w_up, w_down: host arrays of R device pointers, each rank's
+ *   [E/R + B, ...] weight tensor (this rank's entry is written).
+ */
+MOE_API moe_status_t moe_ep_prefetch_weights(const moe_shape_t *shape, int32_t rank, const int32_t *seg_expert,
+                                     const int32_t *seg_offsets, moe_bf16_t *const *w_gate,
+                                     moe_bf16_t *const *w_up, moe_bf16_t *const *w_down,
+                                     moe_stream_t stream);
+
+/*
+ * Dispatch of the source ranks [src_rank, src_rank + n_src) (MoonEP page,
+ * "이 기술은 무엇인가": each row is written straight to its final slot on the
+ * receiving rank).  Pair (t, j) of rank r has global index q = r*S*k + t*k + j;
+ * its stable rank among all pairs of its expert (q order) selects the plan's
+ * segment that holds it, hence its owner g and row; then
+ *   dest_r[t*k + j] = g*S*k + row,  src_g[row] = q,  xp_g[row] = x_r[t].
+ *   x, topk_ids, dest: host arrays of n_src device pointers ([S, d] bf16,
+ *                      [S, k] int32, [S*k] int32 out)
+ *   counts_all: [R, E] as for moe_ep_plan
+ *   xp, src: host arrays of R device pointers (each owner's receive buffers)
+ * One launch; every CTA recomputes the plan from counts_all.  The kernel ends
+ * with a system-scope fence, so a collective that follows it on the stream
+ * also follows its stores to other GPUs.
+ */
+MOE_API moe_status_t moe_ep_dispatch(const moe_shape_t *shape, int32_t src_rank, int32_t n_src,
+                             const moe_bf16_t *const *x, const int32_t *const *topk_ids,
+                             const int32_t *counts_all, int32_t *const *dest, moe_bf16_t *const *xp,
+                             int32_t *const *src, int32_t *status, moe_stream_t stream);
+
+/*
+ * One rank's grouped GEMMs (moe_expert_gate_up then moe_expert_down) on its S*k
+ * rows, its E/R + B segments (seg_slot as the segment's weight slot) and its own
+ * weight slots.  All pointers are this rank's device memory.
+ */
+MOE_API moe_status_t moe_ep_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *xp, const int32_t *seg_slot,
+                               const int32_t *seg_offsets, const moe_bf16_t *w_gate, const moe_bf16_t *w_up,
+                               const moe_bf16_t *w_down, moe_bf16_t *hp, float *yp, int32_t *status,
+                               moe_stream_t stream);
+
+/*
+ * Combine of the source ranks [src_rank, src_rank + n_src): out_r[t] = sum over
+ * j of w_r[t, j] * yp_g[row], with (g, row) from dest_r[t*k + j] = g*S*k + row
+ * (fp32, ascending j), stored in shape->out_dtype.
+ *   yp: host array of R device pointers (each owner's [S*k, d] fp32)
+ *   dest, topk_w, out: host arrays of n_src device pointers
+ */
+MOE_API moe_status_t moe_ep_combine(const moe_shape_t *shape, int32_t src_rank, int32_t n_src,
+                            const float *const *yp, const int32_t *const *dest, const float *const *topk_w,
+                            void *const *out, moe_stream_t stream);
+
 /* Fill *views with the addresses inside a layer workspace `ws`. Host only. */
 MOE_API moe_status_t moe_layer_views(const moe_shape_t *shape, void *ws, moe_layer_views_t *views);
 

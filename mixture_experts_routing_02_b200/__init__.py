@@ -21,6 +21,8 @@ __all__ = [
     "moe_route_scores", "moe_expert_choose", "moe_combine_expert_choice",
     "moe_route_workspace_size", "moe_route_ws", "moe_route_scores_ws", "moe_dispatch_reroute",
     "moe_layer_views", "moe_routing_stats", "STAT_NAMES",
+    "EP_MAX_RANKS", "moe_ep_sizes", "moe_ep_plan", "moe_ep_prefetch_weights", "moe_ep_dispatch", "moe_ep_expert_ffn",
+    "moe_ep_combine",
     "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT", "ROUTE_SOFTMAX_ALL", "ROUTE_EXPERT_CHOICE", "ROUTE_REROUTE",
     "DTYPE_F32", "DTYPE_BF16",
 ]
@@ -82,6 +84,12 @@ SYMBOLS = {
     "moe_route_scores_ws": [_S, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_dispatch_reroute": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_routing_stats": [_S, _P, _P, _P, _P, _P],
+    "moe_ep_sizes": [_S, _P, _P, _P],
+    "moe_ep_plan": [_S, _I, _P, _P, _P, _P, _P, _P, _P],
+    "moe_ep_prefetch_weights": [_S, _I, _P, _P, _P, _P, _P, _P],
+    "moe_ep_dispatch": [_S, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P],
+    "moe_ep_expert_ffn": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "moe_ep_combine": [_S, _I, _I, _P, _P, _P, _P, _P],
 }
 
 # order of the values moe_routing_stats writes (MOE_STAT_* in the header)
@@ -312,3 +320,54 @@ def moe_routing_stats(s, counts, seg_expert, seg_offsets, stats, stream=None):
     """stats: int32 CUDA tensor of len(STAT_NAMES) values (see the header for their meaning)."""
     _check("moe_routing_stats", load_library().moe_routing_stats(
         ctypes.byref(s), _ptr(counts), _ptr(seg_expert), _ptr(seg_offsets), _ptr(stats), _stream(stream)))
+
+
+# ----------------------------------------------------------------------------- expert parallelism
+
+EP_MAX_RANKS = 16
+
+
+def _ptr_table(tensors):
+    """A host array of device pointers (entry i = tensors[i]'s address), as the moe_ep_* calls take."""
+    return (ctypes.c_void_p * len(tensors))(*[_ptr(t) for t in tensors])
+
+
+def moe_ep_sizes(s):
+    """(xp_bytes, replica_weight_bytes, n_local_segments) of one rank."""
+    a, b, n = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_int32()
+    _check("moe_ep_sizes", load_library().moe_ep_sizes(ctypes.byref(s), ctypes.byref(a), ctypes.byref(b),
+                                                        ctypes.byref(n)))
+    return a.value, b.value, n.value
+
+
+def moe_ep_plan(s, rank, counts_all, counts, seg_expert, seg_slot, seg_offsets, status=None, stream=None):
+    _check("moe_ep_plan", load_library().moe_ep_plan(
+        ctypes.byref(s), int(rank), _ptr(counts_all), _ptr(counts), _ptr(seg_expert), _ptr(seg_slot),
+        _ptr(seg_offsets), _ptr(status), _stream(stream)))
+
+
+def moe_ep_prefetch_weights(s, rank, seg_expert, seg_offsets, w_gate, w_up, w_down, stream=None):
+    """w_gate / w_up / w_down: lists of R tensors (every rank's weight slots; entry `rank` is written)."""
+    _check("moe_ep_prefetch_weights", load_library().moe_ep_prefetch_weights(
+        ctypes.byref(s), int(rank), _ptr(seg_expert), _ptr(seg_offsets), _ptr_table(w_gate), _ptr_table(w_up),
+        _ptr_table(w_down), _stream(stream)))
+
+
+def moe_ep_dispatch(s, src_rank, x, topk_ids, counts_all, dest, xp, src, status=None, stream=None):
+    """x / topk_ids / dest: lists of the n_src source ranks' tensors; xp / src: lists of R owners' buffers."""
+    _check("moe_ep_dispatch", load_library().moe_ep_dispatch(
+        ctypes.byref(s), int(src_rank), len(x), _ptr_table(x), _ptr_table(topk_ids), _ptr(counts_all),
+        _ptr_table(dest), _ptr_table(xp), _ptr_table(src), _ptr(status), _stream(stream)))
+
+
+def moe_ep_expert_ffn(s, xp, seg_slot, seg_offsets, w_gate, w_up, w_down, hp, yp, status=None, stream=None):
+    _check("moe_ep_expert_ffn", load_library().moe_ep_expert_ffn(
+        ctypes.byref(s), _ptr(xp), _ptr(seg_slot), _ptr(seg_offsets), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+        _ptr(hp), _ptr(yp), _ptr(status), _stream(stream)))
+
+
+def moe_ep_combine(s, src_rank, yp, dest, topk_w, out, stream=None):
+    """yp: list of R owners' Yp; dest / topk_w / out: lists of the n_src source ranks' tensors."""
+    _check("moe_ep_combine", load_library().moe_ep_combine(
+        ctypes.byref(s), int(src_rank), len(dest), _ptr_table(yp), _ptr_table(dest), _ptr_table(topk_w),
+        _ptr_table(out), _stream(stream)))

@@ -427,6 +427,26 @@ LayerLayout layer_layout(const Dims& v) {
     return L;
 }
 
+// Expert-parallel shapes: the balanced plan's R groups are R ranks of S = T / R tokens each.
+moe_status_t check_ep_shape(const moe_shape_t* shape, Dims* v) {
+    const moe_status_t s = check_shape(shape, v);
+    if (s != MOE_OK) return s;
+    if (v->R < 1 || v->ec() || v->rr()) return MOE_ERR_INVALID_ARG;
+    if (v->R > kEpMaxRanks) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+// The shape of one rank's grouped GEMMs: S*k rows in E/R + B segments over E/R + B weight slots.
+Dims ep_local_dims(const Dims& v) {
+    Dims l = v;
+    l.E = v.E / v.R + v.B;
+    l.n_seg = l.E;
+    l.T = v.S;
+    l.rows = v.S * v.k;
+    l.R = 0;
+    return l;
+}
+
 }  // namespace
 
 extern "C" {
@@ -845,6 +865,113 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
     if (s != MOE_OK) return s;
     return cuda_status(
         launch_combine(w.yp, w.dest, w.topk_w, nullptr, v.T, v.k, v.d, v.rows, out, v.out_bf16, sm_count(), st));
+}
+
+moe_status_t moe_ep_sizes(const moe_shape_t* shape, size_t* xp_bytes, size_t* replica_weight_bytes,
+                          int32_t* n_local_segments) {
+    Dims v;
+    const moe_status_t s = check_ep_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (xp_bytes) *xp_bytes = static_cast<size_t>(v.S) * v.k * v.d * 2;
+    if (replica_weight_bytes) *replica_weight_bytes = static_cast<size_t>(v.B) * 3 * v.d * v.F * 2;
+    if (n_local_segments) *n_local_segments = v.E / v.R + v.B;
+    return MOE_OK;
+}
+
+moe_status_t moe_ep_plan(const moe_shape_t* shape, int32_t rank, const int32_t* counts_all, int32_t* counts,
+                         int32_t* seg_expert, int32_t* seg_slot, int32_t* seg_offsets, int32_t* status,
+                         moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_ep_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (rank < 0 || rank >= v.R || !counts_all || !seg_expert || !seg_slot || !seg_offsets) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_ep_plan(counts_all, v.R, v.S, v.k, v.E, v.B, rank, counts, seg_expert, seg_slot,
+                                      seg_offsets, status, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_prefetch_weights(const moe_shape_t* shape, int32_t rank, const int32_t* seg_expert,
+                                     const int32_t* seg_offsets, moe_bf16_t* const* w_gate, moe_bf16_t* const* w_up,
+                                     moe_bf16_t* const* w_down, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_ep_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (rank < 0 || rank >= v.R || !seg_expert || !seg_offsets || !w_gate || !w_up || !w_down)
+        return MOE_ERR_INVALID_ARG;
+    EpPrefetchArgs a{};
+    moe_bf16_t* const* tabs[3] = {w_gate, w_up, w_down};
+    for (int m = 0; m < 3; ++m)
+        for (int r = 0; r < v.R; ++r) {
+            if (tabs[m][r] == nullptr || !aligned16(tabs[m][r])) return MOE_ERR_INVALID_ARG;
+            a.w[m][r] = reinterpret_cast<__nv_bfloat16*>(tabs[m][r]);
+        }
+    a.seg_expert = seg_expert; a.seg_offsets = seg_offsets;
+    a.R = v.R; a.E = v.E; a.B = v.B; a.F = v.F; a.d = v.d; a.rank = rank;
+    return cuda_status(launch_ep_prefetch(a, sm_count(), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_dispatch(const moe_shape_t* shape, int32_t src_rank, int32_t n_src, const moe_bf16_t* const* x,
+                             const int32_t* const* topk_ids, const int32_t* counts_all, int32_t* const* dest,
+                             moe_bf16_t* const* xp, int32_t* const* src, int32_t* status, moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_ep_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (v.S * static_cast<int64_t>(v.k) > kCountMaxPairsPlan) return MOE_ERR_UNSUPPORTED;
+    if (n_src < 1 || src_rank < 0 || src_rank + n_src > v.R) return MOE_ERR_INVALID_ARG;
+    if (!x || !topk_ids || !counts_all || !dest || !xp || !src) return MOE_ERR_INVALID_ARG;
+    EpDispatchArgs a{};
+    for (int i = 0; i < n_src; ++i) {
+        if (!x[i] || !topk_ids[i] || !dest[i] || !aligned16(x[i])) return MOE_ERR_INVALID_ARG;
+        a.x[i] = reinterpret_cast<const __nv_bfloat16*>(x[i]);
+        a.ids[i] = topk_ids[i];
+        a.dest[i] = dest[i];
+    }
+    for (int r = 0; r < v.R; ++r) {
+        if (!xp[r] || !src[r] || !aligned16(xp[r])) return MOE_ERR_INVALID_ARG;
+        a.xp[r] = reinterpret_cast<__nv_bfloat16*>(xp[r]);
+        a.src[r] = src[r];
+    }
+    a.counts_all = counts_all; a.status = status;
+    a.R = v.R; a.S = v.S; a.k = v.k; a.E = v.E; a.d = v.d; a.B = v.B; a.n_seg = v.n_seg;
+    a.src0 = src_rank; a.n_src = n_src;
+    return cuda_status(launch_ep_dispatch(a, sm_count(), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* xp, const int32_t* seg_slot,
+                               const int32_t* seg_offsets, const moe_bf16_t* w_gate, const moe_bf16_t* w_up,
+                               const moe_bf16_t* w_down, moe_bf16_t* hp, float* yp, int32_t* status,
+                               moe_stream_t stream) {
+    Dims v;
+    moe_status_t s = check_ep_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    const Dims l = ep_local_dims(v);
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = gate_up_impl(l, xp, seg_slot, seg_offsets, w_gate, w_up, hp, status, st);
+    if (s != MOE_OK) return s;
+    return down_impl(l, hp, seg_slot, seg_offsets, w_down, yp, status, st);
+}
+
+moe_status_t moe_ep_combine(const moe_shape_t* shape, int32_t src_rank, int32_t n_src, const float* const* yp,
+                            const int32_t* const* dest, const float* const* topk_w, void* const* out,
+                            moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_ep_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (n_src < 1 || src_rank < 0 || src_rank + n_src > v.R) return MOE_ERR_INVALID_ARG;
+    if (!yp || !dest || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+    EpCombineArgs a{};
+    for (int r = 0; r < v.R; ++r) {
+        if (!yp[r] || !aligned16(yp[r])) return MOE_ERR_INVALID_ARG;
+        a.yp[r] = yp[r];
+    }
+    for (int i = 0; i < n_src; ++i) {
+        if (!dest[i] || !topk_w[i] || !out[i] || !aligned16(out[i])) return MOE_ERR_INVALID_ARG;
+        a.dest[i] = dest[i];
+        a.w[i] = topk_w[i];
+        a.out[i] = out[i];
+    }
+    a.R = v.R; a.S = v.S; a.k = v.k; a.d = v.d; a.n_src = n_src;
+    (void)src_rank;  // the source rank only matters for the dispatch's global pair order
+    return cuda_status(launch_ep_combine(a, v.out_bf16, sm_count(), static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

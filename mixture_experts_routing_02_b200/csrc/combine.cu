@@ -24,6 +24,8 @@ template <int KMAX, int UNROLL, typename OutT>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ dest,
                                                       const float* __restrict__ w, const float* __restrict__ base,
                                                       int T, int k, int d, int rows, OutT* __restrict__ out) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     const int vec_per_row = d / 4;  // float4 vectors
@@ -78,14 +80,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 }  // namespace
 
 template <typename OutT>
-static void launch_combine_t(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
+static cudaError_t launch_combine_t(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
                              int d, int rows, OutT* out, int grid, cudaStream_t stream) {
-    if (k <= 2)
-        combine_kernel<2, 4, OutT><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
-    else if (k <= 4)
-        combine_kernel<4, 2, OutT><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
-    else
-        combine_kernel<kMaxTopK, 2, OutT><<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
+    auto kern = k <= 2 ? combine_kernel<2, 4, OutT> : (k <= 4 ? combine_kernel<4, 2, OutT> : combine_kernel<kMaxTopK, 2, OutT>);
+    return launch_pdl(kern, dim3(grid), dim3(256), 0, stream, yp, dest, w, base, T, k, d, rows, out);
 }
 
 cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
@@ -93,10 +91,10 @@ cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w,
     if (T == 0) return cudaSuccess;
     int grid = (T + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
-    if (out_bf16)
-        launch_combine_t(yp, dest, w, base, T, k, d, rows, static_cast<__nv_bfloat16*>(out), grid, stream);
-    else
-        launch_combine_t(yp, dest, w, base, T, k, d, rows, static_cast<float*>(out), grid, stream);
+    const cudaError_t err =
+        out_bf16 ? launch_combine_t(yp, dest, w, base, T, k, d, rows, static_cast<__nv_bfloat16*>(out), grid, stream)
+                 : launch_combine_t(yp, dest, w, base, T, k, d, rows, static_cast<float*>(out), grid, stream);
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 

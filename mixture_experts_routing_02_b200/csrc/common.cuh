@@ -12,6 +12,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moe_routing.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -271,6 +273,23 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t cluster_addr) {
 
 __device__ __forceinline__ void sleep_ns(uint32_t ns) { asm volatile("nanosleep.u32 %0;" ::"r"(ns)); }
 
+// ----------------------------------------------------------------------------- programmatic dependent launch
+//
+// The layer's kernels are launched with programmatic stream serialization, so a kernel may begin
+// (rasterise its CTAs and run a prologue that touches only its own shared / tensor memory) while
+// the previous kernel of the stream is still finishing.  griddep_wait() returns once every
+// earlier kernel of the stream has completed and its memory is visible; a kernel calls it before
+// its first access to global memory.  griddep_launch_dependents() lets the next kernel start
+// launching; a kernel calls it right after its wait, which keeps the chain transitive (a kernel
+// can only start after its predecessor has passed its own wait).  Both are no-ops for a kernel
+// launched without the attribute.
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------------- misc
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -320,5 +339,22 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 __host__ __device__ constexpr int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
+
+// Launch `kern` on `stream` with programmatic stream serialization (see griddep_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 }  // namespace moe

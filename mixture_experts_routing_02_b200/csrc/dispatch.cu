@@ -26,6 +26,7 @@
 // shapes, no host sync) and "설치 및 통합" (tokens_per_expert, cu_seqlens).
 #include "common.cuh"
 #include "kernels.h"
+#include "plan.cuh"
 
 namespace moe {
 
@@ -144,158 +145,6 @@ __global__ void __launch_bounds__(256) segments_kernel(int32_t* counts, const in
 }
 
 // ------------------------------------------------------------------------------ balanced plan
-
-constexpr int kMaxGroups = 256;
-
-// Exclusive scan over the threads of a block (any multiple of 32 up to 1024); *total = the sum.
-// warp_sums: 33 ints.  Ends with a barrier.
-__device__ __forceinline__ int block_exclusive_scan_any(int v, int* warp_sums, int* total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nwarps = blockDim.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += t;
-    }
-    if (lane == 31) warp_sums[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        const int w0 = lane < nwarps ? warp_sums[lane] : 0;
-        int w = w0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += t;
-        }
-        __syncwarp();
-        if (lane < nwarps) warp_sums[lane] = w - w0;
-        if (lane == 31) warp_sums[32] = w;
-    }
-    __syncthreads();
-    const int r = warp_sums[warp] + x - v;
-    if (total != nullptr) *total = warp_sums[32];
-    __syncthreads();
-    return r;
-}
-
-// Shared memory of the balanced plan.
-struct PlanSmem {
-    int c[kMaxExperts];          // rows of each expert (filled by the caller)
-    int order[kMaxExperts];      // experts of each group by (count desc, id asc)
-    int given[kMaxExperts];      // rows an expert hands to other groups
-    int next_rank[kMaxExperts];
-    int qe[kMaxExperts], qn[kMaxExperts];  // the donor queue
-    int load[kMaxGroups];
-    int n_slots[kMaxGroups];
-    int slot_e[kMaxSegments], slot_n[kMaxSegments], slot_r[kMaxSegments];
-    int seg_len[kMaxSegments];
-    int warp_sums[33];
-    int infeasible;
-};
-
-// The greedy balanced plan from sm.c (written by the caller before a barrier) into the segment
-// tables (any memory).  Called by the whole block; the greedy itself runs on one thread.  An
-// infeasible plan (a group needs more than B replica slots) writes every segment empty and, if
-// report_status, sets MOE_DEV_ERR_PLAN.
-__device__ void compute_plan(PlanSmem& sm, int E, int R, int S, int k, int B, int* seg_expert, int* seg_offsets,
-                             int* seg_first_rank, int32_t* status, bool report_status) {
-    const int tid = threadIdx.x;
-    const int epg = E / R;
-    const int per_group = epg + B;
-    const int n_seg = R * per_group;
-    const int cap = S * k;
-
-    for (int e = tid; e < E; e += blockDim.x) sm.given[e] = 0;
-    for (int g = tid; g < R; g += blockDim.x) {
-        int s = 0;
-        for (int e = g * epg; e < (g + 1) * epg; ++e) s += sm.c[e];
-        sm.load[g] = s;
-    }
-    for (int e = tid; e < E; e += blockDim.x) {
-        const int g = e / epg;
-        int rank = 0;
-        for (int o = g * epg; o < (g + 1) * epg; ++o) rank += (sm.c[o] > sm.c[e]) || (sm.c[o] == sm.c[e] && o < e);
-        sm.order[g * epg + rank] = e;
-    }
-    __syncthreads();
-
-    if (tid == 0) {
-        // the queue of excess rows, groups ascending, experts by (count desc, id asc)
-        int nq = 0, total = 0;
-        for (int g = 0; g < R; ++g) total += sm.load[g];
-        int bad = (total != R * cap);
-        for (int g = 0; g < R; ++g) {
-            int excess = sm.load[g] - cap;
-            for (int i = 0; i < epg && excess > 0; ++i) {
-                const int e = sm.order[g * epg + i];
-                const int take = sm.c[e] < excess ? sm.c[e] : excess;
-                if (take > 0) { sm.given[e] = take; sm.qe[nq] = e; sm.qn[nq] = take; ++nq; excess -= take; }
-            }
-        }
-        // groups below the cap, ascending, take from the front of the queue
-        int head = 0;
-        for (int g = 0; g < R; ++g) {
-            int deficit = cap - sm.load[g];
-            int ns = 0;
-            while (deficit > 0 && head < nq) {
-                const int take = sm.qn[head] < deficit ? sm.qn[head] : deficit;
-                if (ns < B) { sm.slot_e[g * B + ns] = sm.qe[head]; sm.slot_n[g * B + ns] = take; }
-                ++ns;
-                sm.qn[head] -= take;
-                deficit -= take;
-                if (sm.qn[head] == 0) ++head;
-            }
-            if (ns > B || deficit > 0) bad = 1;
-            sm.n_slots[g] = ns < B ? ns : B;
-        }
-        // within-expert rank at which each piece starts: after the home rows, in creation order
-        for (int e = 0; e < E; ++e) sm.next_rank[e] = sm.c[e] - sm.given[e];
-        for (int g = 0; g < R; ++g)
-            for (int i = 0; i < sm.n_slots[g]; ++i) {
-                const int idx = g * B + i;
-                sm.slot_r[idx] = sm.next_rank[sm.slot_e[idx]];
-                sm.next_rank[sm.slot_e[idx]] += sm.slot_n[idx];
-            }
-        sm.infeasible = bad;
-        if (bad && report_status) report(status, MOE_DEV_ERR_PLAN);
-    }
-    __syncthreads();
-
-    const bool bad = sm.infeasible != 0;
-    for (int s = tid; s < n_seg; s += blockDim.x) {
-        const int g = s / per_group, i = s - g * per_group;
-        int ex = -1, len = 0, fr = 0;
-        if (!bad) {
-            if (i < epg) {
-                ex = g * epg + i;
-                len = sm.c[ex] - sm.given[ex];
-            } else if (i - epg < sm.n_slots[g]) {
-                const int idx = g * B + (i - epg);
-                ex = sm.slot_e[idx];
-                len = sm.slot_n[idx];
-                fr = sm.slot_r[idx];
-            }
-        }
-        seg_expert[s] = ex;
-        seg_first_rank[s] = fr;
-        sm.seg_len[s] = len;
-    }
-    __syncthreads();
-    // offsets: exclusive scan of the lengths, each thread owning a contiguous chunk
-    const int chunk = (n_seg + blockDim.x - 1) / blockDim.x;
-    const int a = tid * chunk;
-    int local = 0;
-    for (int s = a; s < a + chunk && s < n_seg; ++s) local += sm.seg_len[s];
-    int total;
-    int run = block_exclusive_scan_any(local, sm.warp_sums, &total);
-    for (int s = a; s < a + chunk && s < n_seg; ++s) {
-        seg_offsets[s] = run;
-        run += sm.seg_len[s];
-    }
-    if (tid == 0) seg_offsets[n_seg] = total;
-    __syncthreads();
-}
 
 __global__ void __launch_bounds__(256) plan_kernel(int32_t* counts, const int32_t* partials, int n_partials, int E,
                                                    int R, int S, int k, int B, int32_t* seg_expert,
@@ -676,6 +525,8 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
     __shared__ int s_wcnt[kCountWarps][kMaxExperts];
     __shared__ int warp_sums[kCountWarps];
 
+    griddep_wait();
+    griddep_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = a.E, k = a.k;
     const unsigned lanemask_lt = (1u << lane) - 1u;
@@ -1148,6 +999,8 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const float* __restri
                                                            int E, int k, int route_flags, float* __restrict__ logits,
                                                            int32_t* __restrict__ ids, float* __restrict__ w,
                                                            float* __restrict__ scores_t) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
@@ -1338,9 +1191,11 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
         const cudaError_t err = cudaFuncSetAttribute(dispatch_count_kernel<true>,
                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err != cudaSuccess) return err;
-        dispatch_count_kernel<true><<<grid, kCountThreads, smem, stream>>>(a);
+        const cudaError_t e2 = launch_pdl(dispatch_count_kernel<true>, dim3(grid), dim3(kCountThreads), smem, stream, a);
+        if (e2 != cudaSuccess) return e2;
     } else {
-        dispatch_count_kernel<false><<<grid, kCountThreads, 0, stream>>>(a);
+        const cudaError_t e2 = launch_pdl(dispatch_count_kernel<false>, dim3(grid), dim3(kCountThreads), 0, stream, a);
+        if (e2 != cudaSuccess) return e2;
     }
     return cudaGetLastError();
 }
@@ -1397,8 +1252,9 @@ cudaError_t launch_route_logits(const float* part, int n_split, int ldp, size_t 
     if (T == 0) return cudaSuccess;
     int grid = (T + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
-    route_logits_kernel<<<grid, 256, 0, stream>>>(part, n_split, ldp, split_stride, bias, T, E, k, route_flags, logits,
-                                                  ids, w, scores_t);
+    const cudaError_t err = launch_pdl(route_logits_kernel, dim3(grid), dim3(256), 0, stream, part, n_split, ldp,
+                                       split_stride, bias, T, E, k, route_flags, logits, ids, w, scores_t);
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 

@@ -158,6 +158,39 @@ cudaError_t launch_ec_gather(const __nv_bfloat16* x, const int32_t* src, int row
 cudaError_t launch_ec_combine(const float* yp, const int32_t* emap, const float* row_w, const float* base, int T,
                               int E, int d, int rows, void* out, bool out_bf16, int num_sms, cudaStream_t stream);
 
+// ep.cu: expert parallelism over R ranks (pointer tables hold each rank's buffer; on one GPU the
+// "ranks" are local buffers)
+constexpr int kEpMaxRanks = 16;
+struct EpDispatchArgs {
+    const __nv_bfloat16* x[kEpMaxRanks];  // [n_src] source ranks' X [S, d]
+    const int32_t* ids[kEpMaxRanks];      // [n_src] [S * k]
+    int32_t* dest[kEpMaxRanks];           // [n_src] [S * k] out: owner * S*k + row
+    __nv_bfloat16* xp[kEpMaxRanks];       // [R] each owner's Xp [S*k, d]
+    int32_t* src[kEpMaxRanks];            // [R] each owner's src [S*k]: global pair index
+    const int32_t* counts_all;            // [R, E]
+    int32_t* status;
+    int R, S, k, E, d, B, n_seg, src0, n_src, ctas_per_src;
+};
+struct EpCombineArgs {
+    const float* yp[kEpMaxRanks];        // [R] each owner's Yp [S*k, d]
+    const int32_t* dest[kEpMaxRanks];    // [n_src]
+    const float* w[kEpMaxRanks];         // [n_src] router weights [S, k]
+    void* out[kEpMaxRanks];              // [n_src] [S, d] fp32 or bf16
+    int R, S, k, d, n_src;
+};
+struct EpPrefetchArgs {
+    __nv_bfloat16* w[3][kEpMaxRanks];  // gate, up, down: each rank's [E/R + B, F, d] (down: [.., d, F])
+    const int32_t* seg_expert;         // [E/R + B] of this rank (global expert ids)
+    const int32_t* seg_offsets;        // [E/R + B + 1]
+    int R, E, B, F, d, rank;
+};
+cudaError_t launch_ep_plan(const int32_t* counts_all, int R, int S, int k, int E, int B, int rank, int32_t* counts,
+                           int32_t* seg_expert, int32_t* seg_slot, int32_t* seg_offsets, int32_t* status,
+                           cudaStream_t stream);
+cudaError_t launch_ep_prefetch(const EpPrefetchArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_dispatch(const EpDispatchArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_combine(const EpCombineArgs& a, bool out_bf16, int num_sms, cudaStream_t stream);
+
 // stats.cu: MOE_STAT_COUNT values from the counts (nullable) and segment tables of one dispatch
 cudaError_t launch_routing_stats(const int32_t* counts, const int32_t* seg_expert, const int32_t* seg_offsets,
                                  int E, int n_seg, int R, int B, int pairs, int32_t* stats, cudaStream_t stream);

@@ -206,6 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (EPI == kEpiSwiglu) tma_prefetch_desc(&tmB1);
     }
     if (warp == 1) tmem_alloc(&tmem_base_sh, kTmemCols);
+    // everything above touched only this CTA's shared and tensor memory; the segment table and
+    // the operands may come from the previous kernel of the stream
+    griddep_wait();
+    griddep_launch_dependents();
     if (warp == 2) build_tile_prefix(tile_prefix, g, kBM, lane);
     tc_fence_before();
     __syncthreads();
@@ -492,6 +496,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(EPI == kEpiSwiglu && rank == 1 ? &tmB1 : &tmB0);
     }
     if (warp == 1) tmem_alloc_pair(&tmem_base_sh, kTmemCols);
+    griddep_wait();
+    griddep_launch_dependents();
     if (warp == 2) build_tile_prefix(tile_prefix, g, 2 * kBM, lane);
     tc_fence_before();
     __syncthreads();
@@ -626,7 +632,8 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     if (smem < kGemmSmemMin) smem = kGemmSmemMin;  // keeps one CTA per SM (all TMEM columns are taken)
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    kern<<<grid, kThreads, smem, stream>>>(a, b0, b1, g);
+    err = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, a, b0, b1, g);
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 
@@ -655,13 +662,15 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, cons
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see griddep_wait
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     err = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, g);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();

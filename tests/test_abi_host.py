@@ -250,3 +250,33 @@ def test_out_dtype_is_validated(lib):
     for dt, want in ((moe.DTYPE_F32, 0), (moe.DTYPE_BF16, 0), (2, 1), (-1, 1)):
         s = moe.shape(64, 128, 8, 2, 256, out_dtype=dt)
         assert lib.moe_layout(ctypes.byref(s), None, None) == want
+
+
+def test_ep_sizes_match_moonep_memory_table(lib):
+    """MoonEP page, "실제 실험 결과" (memory per rank at S = 4096, H = 7168, K = 8, H' = 2048): the
+    dispatch buffer S*K*H*2 bytes = 0.44 GiB and the replica weights of B = 4 slots, B*3*H*H'*2 bytes
+    = 0.33 GiB (both printed to two decimals)."""
+    R, S, d, E, k, F, B = 8, 4096, 7168, 256, 8, 2048, 4
+    s = moe.shape(R * S, d, E, k, F, n_groups=R, replica_slots=B)
+    xp_bytes, rep_bytes, n_loc = moe.moe_ep_sizes(s)
+    assert xp_bytes == S * k * d * 2 and round(xp_bytes / 2 ** 30, 2) == 0.44
+    assert rep_bytes == B * 3 * d * F * 2 and round(rep_bytes / 2 ** 30, 2) == 0.33
+    assert n_loc == E // R + B
+
+
+def test_ep_shapes_are_validated(lib):
+    """The moe_ep_* calls need a balanced-plan shape of 1..MOE_EP_MAX_RANKS ranks, without expert
+    choice or re-routing."""
+    n = ctypes.c_size_t()
+    ok = moe.shape(4 * 64, 128, 16, 2, 64, n_groups=4, replica_slots=2)
+    assert lib.moe_ep_sizes(ctypes.byref(ok), ctypes.byref(n), None, None) == 0
+    no_plan = moe.shape(256, 128, 16, 2, 64)
+    assert lib.moe_ep_sizes(ctypes.byref(no_plan), None, None, None) == 1
+    too_many = moe.shape(32 * 8, 64, 32, 2, 64, n_groups=32, replica_slots=1)
+    assert lib.moe_ep_sizes(ctypes.byref(too_many), None, None, None) == 2
+    ec = moe.shape(4 * 64, 128, 16, 2, 64, capacity=8, route_flags=moe.ROUTE_EXPERT_CHOICE)
+    assert lib.moe_ep_sizes(ctypes.byref(ec), None, None, None) == 1
+    # a rank outside [0, R) is rejected before anything is enqueued
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.moe_ep_plan(ctypes.byref(ok), 4, fake, None, fake, fake, fake, None, None) == 1
+    assert lib.moe_ep_plan(ctypes.byref(ok), -1, fake, None, fake, fake, fake, None, None) == 1
