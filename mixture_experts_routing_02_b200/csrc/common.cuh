@@ -340,21 +340,43 @@ __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 __host__ __device__ constexpr int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
 
-// Launch `kern` on `stream` with programmatic stream serialization (see griddep_wait).
+// Launch `kern` on `stream` with programmatic stream serialization (see griddep_wait), plus an
+// optional cluster shape.  Should the runtime refuse the attribute on this stream, the kernel is
+// launched again without it (the kernels' griddep_wait is then a no-op).
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                              Args&&... args) {
+inline cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                      unsigned cluster_x, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    cfg.numAttrs = n + 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (err != cudaSuccess) {
+        (void)cudaGetLastError();
+        cfg.numAttrs = n;
+        err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    }
+    return err;
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+    return launch_pdl_cluster(kern, grid, block, smem, stream, 1u, std::forward<Args>(args)...);
 }
 
 }  // namespace moe

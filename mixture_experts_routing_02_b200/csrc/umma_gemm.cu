@@ -657,21 +657,7 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, cons
     if (smem < kGemmSmemMin) smem = kGemmSmemMin;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * n_pairs, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see griddep_wait
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    err = cudaLaunchKernelEx(&cfg, kern, a, b0, b1, g);
+    err = launch_pdl_cluster(kern, dim3(2 * n_pairs), dim3(kThreads), smem, stream, 2u, a, b0, b1, g);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
