@@ -38,6 +38,7 @@ if ROOT not in sys.path:
 METRIC = "MoE layer fwd tokens/s; grouped-GEMM TFLOPS and permute GB/s vs roofline"
 FLUSH_BYTES = 256 << 20
 NOMINAL_HBM_GBS = 8000.0     # B200 HBM3e, nominal (the measured copy bandwidth is the primary peak)
+LONG_STEP_MS = 10.0          # steps this long are compared with the sustained (power-capped) bf16 peak
 E2E_MIN_STEPS = 64
 KERNELS = ("route", "dispatch", "gate_up", "down", "combine")
 
@@ -410,7 +411,7 @@ def run_ours(args, w):
     # the router projection's reduction is split over more CTAs when its row tiles are few
     route_ws_bytes = moe.moe_route_workspace_size(s)
     route_ws = torch.empty(max(route_ws_bytes, 256), dtype=torch.uint8, device=dev) if route_ws_bytes else None
-    launches = ((2 if route_ws_bytes else 1)                                   # route (+ partial sums)
+    launches = (1                                                              # route (routing fused)
                 + (2 if ec or rr else (4 if w.n_groups and w.T * w.k > (1 << 20) else 1))  # dispatch
                 + 3)                                                           # gate_up, down, combine
 
@@ -594,15 +595,22 @@ def run_ours(args, w):
         if "flops" in b and name in ("gate_up", "down"):
             b["tflops"] = b["flops"] / sec / 1e12
             b["frac_bf16_peak"] = b["tflops"] / bf16
+            if bf16_sus:
+                b["frac_bf16_sustained"] = b["tflops"] / bf16_sus
         b["gbs"] = b["bytes"] / sec / 1e9
         b["frac_hbm_peak"] = b["gbs"] / hbm
         b["frac_hbm_nominal"] = b["gbs"] / NOMINAL_HBM_GBS
     dom = max(breakdown, key=lambda n: breakdown[n]["ms"])
     db = breakdown[dom]
+    # a contraction inside a long step runs at the power-capped (sustained) rate; a short one at
+    # the burst rate: steps of 10 ms and more are compared with the sustained peak
+    long_step = (total_ms / args.steps) >= LONG_STEP_MS and bf16_sus > 0
+    gemm_peak = bf16_sus if long_step else bf16
     if dom in ("gate_up", "down"):
-        roof = {"bound": "tensor", "achieved": db["tflops"], "peak": bf16, "unit": "TFLOP/s",
-                "frac": db["tflops"] / bf16, "kernel": dom,
-                "peak_source": f"{peak_kind} bf16_tflops (burst); sustained {bf16_sus}"}
+        roof = {"bound": "tensor", "achieved": db["tflops"], "peak": gemm_peak, "unit": "TFLOP/s",
+                "frac": db["tflops"] / gemm_peak, "kernel": dom,
+                "peak_source": (f"{peak_kind} bf16_tflops_sustained (step >= {LONG_STEP_MS:g} ms); burst {bf16}"
+                                if long_step else f"{peak_kind} bf16_tflops (burst); sustained {bf16_sus}")}
     else:
         roof = {"bound": "hbm", "achieved": db["gbs"], "peak": hbm, "unit": "GB/s", "frac": db["gbs"] / hbm,
                 "kernel": dom, "peak_source": f"{peak_kind} hbm_gbs"}
@@ -614,11 +622,13 @@ def run_ours(args, w):
     gemm_flops = breakdown["gate_up"]["flops"] + breakdown["down"]["flops"]
     hp_bytes = rows_used * F * 2
     layer_bytes = sum(b["bytes"] for b in breakdown.values()) - 2 * hp_bytes
-    t_flop_ms = gemm_flops / (bf16 * 1e12) * 1e3
+    t_flop_ms = gemm_flops / (gemm_peak * 1e12) * 1e3
     t_bytes_ms = layer_bytes / (hbm * 1e9) * 1e3
     layer_roof = {"bound": "tensor" if t_flop_ms >= t_bytes_ms else "hbm", "gemm_flops": gemm_flops,
                   "algorithmic_bytes": layer_bytes, "t_flop_ms": t_flop_ms, "t_bytes_ms": t_bytes_ms,
-                  "roofline_ms": max(t_flop_ms, t_bytes_ms), "peaks": f"{peak_kind} bf16_tflops {bf16}, hbm_gbs {hbm}"}
+                  "roofline_ms": max(t_flop_ms, t_bytes_ms),
+                  "peaks": f"{peak_kind} bf16 {'sustained' if long_step else 'burst'} {gemm_peak} TFLOP/s, "
+                           f"hbm_gbs {hbm}"}
 
     value = job_throughput(T, args.steps, world, total_ms)
     line = {

@@ -683,6 +683,31 @@ MOE_API moe_status_t moe_ep_combine(const moe_shape_t *shape, int32_t src_rank, 
                             const float *const *yp, const int32_t *const *dest, const float *const *topk_w,
                             void *const *out, moe_stream_t stream);
 
+/*
+ * Routing results of a layer call, copied into the caller's own device buffers
+ * (every pointer nullable: NULL = not wanted).
+ */
+typedef struct {
+    int32_t *topk_ids;    /* [T, k] */
+    float *topk_w;        /* [T, k] */
+    int32_t *counts;      /* [E] raw per-expert counts */
+    int32_t *seg_offsets; /* [n_seg + 1] */
+    int32_t *dest;        /* [T * k] row of each pair, -1 = dropped */
+    int32_t *stats;       /* [MOE_STAT_COUNT], as moe_routing_stats writes them */
+} moe_aux_t;
+
+/*
+ * moe_layer_fwd, then the requested routing results copied out of the workspace
+ * (device-to-device copies on `stream`) and, with aux->stats, moe_routing_stats.
+ * aux may be NULL (then identical to moe_layer_fwd).  Expert-choice shapes have
+ * no per-pair results: requesting topk_ids, topk_w, dest, counts or stats for them
+ * is MOE_ERR_INVALID_ARG (seg_offsets is allowed).
+ */
+MOE_API moe_status_t moe_layer_fwd_aux(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *w_router,
+                               const float *bias, const moe_bf16_t *w_gate, const moe_bf16_t *w_up,
+                               const moe_bf16_t *w_down, void *out, const moe_aux_t *aux, int32_t *status,
+                               void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Fill *views with the addresses inside a layer workspace `ws`. Host only. */
 MOE_API moe_status_t moe_layer_views(const moe_shape_t *shape, void *ws, moe_layer_views_t *views);
 

@@ -20,7 +20,7 @@ __all__ = [
     "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_combine_add", "moe_shared_expert", "moe_layer_fwd",
     "moe_route_scores", "moe_expert_choose", "moe_combine_expert_choice",
     "moe_route_workspace_size", "moe_route_ws", "moe_route_scores_ws", "moe_dispatch_reroute",
-    "moe_layer_views", "moe_routing_stats", "STAT_NAMES",
+    "moe_layer_views", "moe_routing_stats", "STAT_NAMES", "MoeAux", "moe_layer_fwd_aux",
     "EP_MAX_RANKS", "moe_ep_sizes", "moe_ep_plan", "moe_ep_prefetch_weights", "moe_ep_dispatch", "moe_ep_expert_ffn",
     "moe_ep_combine",
     "DEV_ERR_PLAN", "DEV_ERR_TIMEOUT", "ROUTE_SOFTMAX_ALL", "ROUTE_EXPERT_CHOICE", "ROUTE_REROUTE",
@@ -41,6 +41,11 @@ class MoeShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("T", "d_model", "n_experts", "top_k", "d_ff", "capacity", "n_groups", "replica_slots",
                  "route_flags", "out_dtype")]
+
+
+class MoeAux(ctypes.Structure):
+    """moe_aux_t: device addresses (or None) that moe_layer_fwd_aux copies the routing results to."""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("topk_ids", "topk_w", "counts", "seg_offsets", "dest", "stats")]
 
 
 class MoeLayerViews(ctypes.Structure):
@@ -75,6 +80,7 @@ SYMBOLS = {
     "moe_combine_add": [_S, _P, _P, _P, _P, _P, _P],
     "moe_shared_expert": [_S, _I, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_layer_fwd": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "moe_layer_fwd_aux": [_S, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(MoeAux), _P, _P, ctypes.c_size_t, _P],
     "moe_layer_views": [_S, _P, ctypes.POINTER(MoeLayerViews)],
     "moe_route_scores": [_S, _P, _P, _P, _P, _P, _P],
     "moe_expert_choose": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P],
@@ -263,6 +269,15 @@ def moe_layer_fwd(s, x, w_router, bias, w_gate, w_up, w_down, out, status, ws, s
     _check("moe_layer_fwd", load_library().moe_layer_fwd(
         ctypes.byref(s), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(out),
         _ptr(status), _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def moe_layer_fwd_aux(s, x, w_router, bias, w_gate, w_up, w_down, out, status, ws, topk_ids=None, topk_w=None,
+                      counts=None, seg_offsets=None, dest=None, stats=None, stream=None):
+    """moe_layer_fwd plus the routing results copied into the given tensors (None = not wanted)."""
+    aux = MoeAux(_ptr(topk_ids), _ptr(topk_w), _ptr(counts), _ptr(seg_offsets), _ptr(dest), _ptr(stats))
+    _check("moe_layer_fwd_aux", load_library().moe_layer_fwd_aux(
+        ctypes.byref(s), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(out),
+        ctypes.byref(aux), _ptr(status), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def moe_layer_views(s, ws) -> MoeLayerViews:

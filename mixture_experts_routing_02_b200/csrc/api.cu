@@ -152,9 +152,10 @@ moe_status_t route_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_
 }
 
 // The router projection has only ceil(T/128) row tiles.  When they are fewer than the SMs, its
-// reduction over d is cut into S parts (each at least 4 k-blocks of 64), the S*ceil(T/128) work
-// units write fp32 partial logits [S][T][ldp] to a workspace, and a warp-per-token kernel sums
-// the parts in order (so the result does not depend on timing), adds the bias and routes.
+// reduction over d is cut into S parts (each at least 4 k-blocks of 64): S*ceil(T/128) CTAs in
+// clusters of S (one row tile per cluster) write fp32 partial logits [S][T][ldp] to a workspace,
+// and after a cluster barrier the cluster's CTAs sum the parts in order (so the result does not
+// depend on timing), add the bias and route -- one launch.
 constexpr int kMaxRouteSplits = 8;
 
 int route_splits(const Dims& v) {
@@ -196,12 +197,11 @@ bool route_split_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_ro
     g.BN = epad; g.n_tiles_n = 1; g.mma_n = epad; g.stages = gemm_pick_stages(epad);
     g.out = ws; g.ldo = ldp; g.status = status;
     g.k_splits = S; g.split_stride = static_cast<size_t>(v.T) * ldp;
-    const int grid = std::min(sm_count(), (v.T + 127) / 128 * S);
-    moe_status_t r = cuda_status(launch_umma_gemm(kEpiStore, ta, tb, tb, g, grid, st));
-    if (r == MOE_OK)
-        r = cuda_status(launch_route_logits(static_cast<const float*>(ws), S, ldp, g.split_stride, bias, v.T, v.E, v.k,
-                                            v.flags & ~MOE_ROUTE_EXPERT_CHOICE, logits, ids, w, scores, sm_count(), st));
-    *result = r;
+    // routing fused into the same launch: clusters of the S split CTAs of a row tile, one pass
+    g.bias = bias; g.logits = logits; g.topk_ids = ids; g.topk_w = w; g.scores_t = scores; g.k = v.k;
+    g.route_flags = v.flags & ~MOE_ROUTE_EXPERT_CHOICE;
+    const int grid = (v.T + 127) / 128 * S;  // <= the SM count (route_splits)
+    *result = cuda_status(launch_umma_gemm(kEpiRouteSplit, ta, tb, tb, g, grid, st));
     return true;
 }
 
@@ -865,6 +865,36 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
     if (s != MOE_OK) return s;
     return cuda_status(
         launch_combine(w.yp, w.dest, w.topk_w, nullptr, v.T, v.k, v.d, v.rows, out, v.out_bf16, sm_count(), st));
+}
+
+moe_status_t moe_layer_fwd_aux(const moe_shape_t* shape, const moe_bf16_t* x, const moe_bf16_t* w_router,
+                               const float* bias, const moe_bf16_t* w_gate, const moe_bf16_t* w_up,
+                               const moe_bf16_t* w_down, void* out, const moe_aux_t* aux, int32_t* status, void* ws,
+                               size_t ws_bytes, moe_stream_t stream) {
+    Dims v;
+    moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (aux && v.ec() && (aux->topk_ids || aux->topk_w || aux->dest || aux->counts || aux->stats))
+        return MOE_ERR_INVALID_ARG;  // expert choice keeps no per-pair results
+    s = moe_layer_fwd(shape, x, w_router, bias, w_gate, w_up, w_down, out, status, ws, ws_bytes, stream);
+    if (s != MOE_OK || aux == nullptr || v.T == 0) return s;
+    moe_layer_views_t w;
+    moe_layer_views(shape, ws, &w);
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t tk = static_cast<size_t>(v.T) * v.k;
+    auto copy = [&](void* dst, const void* src, size_t bytes) -> moe_status_t {
+        if (dst == nullptr || bytes == 0) return MOE_OK;
+        return cuda_status(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st));
+    };
+    if ((s = copy(aux->topk_ids, w.topk_ids, tk * 4)) != MOE_OK) return s;
+    if ((s = copy(aux->topk_w, w.topk_w, tk * 4)) != MOE_OK) return s;
+    if ((s = copy(aux->counts, w.counts, static_cast<size_t>(v.E) * 4)) != MOE_OK) return s;
+    if ((s = copy(aux->seg_offsets, w.seg_offsets, static_cast<size_t>(v.n_seg + 1) * 4)) != MOE_OK) return s;
+    if ((s = copy(aux->dest, w.dest, tk * 4)) != MOE_OK) return s;
+    if (aux->stats)
+        return cuda_status(launch_routing_stats(w.counts, w.seg_expert, w.seg_offsets, v.E, v.n_seg, v.R, v.B,
+                                                v.T * v.k, aux->stats, st));
+    return MOE_OK;
 }
 
 moe_status_t moe_ep_sizes(const moe_shape_t* shape, size_t* xp_bytes, size_t* replica_weight_bytes,

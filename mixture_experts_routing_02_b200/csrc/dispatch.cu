@@ -27,6 +27,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "plan.cuh"
+#include "route.cuh"
 
 namespace moe {
 
@@ -41,7 +42,8 @@ constexpr int kLookbackWindow = 128;  // earlier tiles read per look-back round 
 constexpr int kLookbackUnroll = 32;   // most look-back words one thread reads per round trip
 constexpr int kCountThreads = 1024;
 constexpr int kCountWarps = kCountThreads / 32;
-constexpr int kCountBatch = 8;  // expert ids per thread loaded together in the counting pass
+constexpr int kCountBatch = 8;   // expert ids per thread loaded together in the counting pass (scalar loads)
+constexpr int kCountBatch4 = 4;  // 16-byte loads (4 ids each) per thread in flight together
 
 // Exclusive scan over the 256 threads of a block; *total receives the sum.
 __device__ __forceinline__ int block_exclusive_scan_256(int v, int* warp_sums, int* total) {
@@ -548,8 +550,35 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
     for (int i = tid; i < kCountWarps * kMaxExperts; i += blockDim.x) (&s_wcnt[0][0])[i] = 0;
     __syncthreads();
 
-    // 1. counts of all pairs, split at the starts of the two blocks (kCountBatch loads in flight)
-    for (int base = 0; base < n; base += blockDim.x * kCountBatch) {
+    // 1. counts of all pairs, split at the starts of the two blocks: 16-byte loads of 4 ids,
+    // kCountBatch4 of them in flight per thread (scalar loads if the ids are not 16-byte aligned)
+    auto count_one = [&](int e, int i) {
+        if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
+            atomicAdd(i < q1 ? &s_a[e] : (i < q2 ? &s_m[e] : &s_tot[e]), 1);
+    };
+    int scalar_from = 0;
+    if ((reinterpret_cast<uintptr_t>(a.ids) & 15u) == 0) {
+        const int n4 = n >> 2;
+        const int4* ids4 = reinterpret_cast<const int4*>(a.ids);
+        for (int base = 0; base < n4; base += blockDim.x * kCountBatch4) {
+            int4 ev[kCountBatch4];
+#pragma unroll
+            for (int u = 0; u < kCountBatch4; ++u) {
+                const int i = base + u * blockDim.x + tid;
+                ev[u] = i < n4 ? __ldg(ids4 + i) : make_int4(-1, -1, -1, -1);
+            }
+#pragma unroll
+            for (int u = 0; u < kCountBatch4; ++u) {
+                const int i = 4 * (base + u * blockDim.x + tid);
+                count_one(ev[u].x, i);
+                count_one(ev[u].y, i + 1);
+                count_one(ev[u].z, i + 2);
+                count_one(ev[u].w, i + 3);
+            }
+        }
+        scalar_from = n4 << 2;
+    }
+    for (int base = scalar_from; base < n; base += blockDim.x * kCountBatch) {
         int ev[kCountBatch];
 #pragma unroll
         for (int u = 0; u < kCountBatch; ++u) {
@@ -557,12 +586,7 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
             ev[u] = i < n ? __ldg(a.ids + i) : -1;
         }
 #pragma unroll
-        for (int u = 0; u < kCountBatch; ++u) {
-            const int i = base + u * blockDim.x + tid;
-            const int e = ev[u];
-            if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
-                atomicAdd(i < q1 ? &s_a[e] : (i < q2 ? &s_m[e] : &s_tot[e]), 1);
-        }
+        for (int u = 0; u < kCountBatch; ++u) count_one(ev[u], base + u * blockDim.x + tid);
     }
     __syncthreads();
 
@@ -1003,94 +1027,8 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const float* __restri
     griddep_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
-    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
-        float v[kMaxExperts / 32];
-        unsigned taken = 0;
-#pragma unroll
-        for (int u = 0; u < kMaxExperts / 32; ++u) {
-            const int e = lane + 32 * u;
-            v[u] = -INFINITY;
-            if (e < E) {
-                const float* p = part + static_cast<size_t>(t) * ldp + e;
-                float acc = __ldg(p);
-                for (int sp = 1; sp < n_split; ++sp) acc += __ldg(p + sp * split_stride);
-                if (bias != nullptr) acc += __ldg(bias + e);
-                v[u] = acc;
-                if (logits != nullptr) logits[static_cast<size_t>(t) * E + e] = acc;
-            } else {
-                taken |= 1u << u;
-            }
-        }
-        if (scores_t != nullptr) {
-            float m = -INFINITY;
-#pragma unroll
-            for (int u = 0; u < kMaxExperts / 32; ++u) m = fmaxf(m, v[u]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            float sum = 0.f;
-#pragma unroll
-            for (int u = 0; u < kMaxExperts / 32; ++u)
-                if (lane + 32 * u < E) sum += expf(v[u] - m);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-            const float inv = 1.0f / sum;
-#pragma unroll
-            for (int u = 0; u < kMaxExperts / 32; ++u) {
-                const int e = lane + 32 * u;
-                if (e < E) scores_t[static_cast<size_t>(e) * T + t] = expf(v[u] - m) * inv;
-            }
-            continue;
-        }
-        float sv[kMaxTopK];
-        int si[kMaxTopK];
-#pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) {
-            sv[j] = 0.f;
-            si[j] = 0;
-            if (j < k) {
-                float bv = -INFINITY;
-                int bi = 0x7fffffff;
-#pragma unroll
-                for (int u = 0; u < kMaxExperts / 32; ++u) {
-                    const int e = lane + 32 * u;
-                    if (!((taken >> u) & 1u) && (v[u] > bv || (v[u] == bv && e < bi))) { bv = v[u]; bi = e; }
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-                }
-                if (bi < E && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-                sv[j] = bv;
-                si[j] = bi;
-            }
-        }
-        // denominator over all E logits (softmax-all mode), shifted by the largest (sv[0])
-        float all = 0.f;
-        if (route_flags & MOE_ROUTE_SOFTMAX_ALL) {
-#pragma unroll
-            for (int u = 0; u < kMaxExperts / 32; ++u)
-                if (lane + 32 * u < E) all += expf(v[u] - sv[0]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) all += __shfl_xor_sync(0xffffffffu, all, o);
-        }
-        if (lane == 0) {
-            float ex[kMaxTopK], sum = 0.f;
-#pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j) {
-                ex[j] = j < k ? expf(sv[j] - sv[0]) : 0.f;
-                sum += ex[j];
-            }
-            const float inv = 1.0f / ((route_flags & MOE_ROUTE_SOFTMAX_ALL) ? all : sum);
-#pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j)
-                if (j < k) {
-                    ids[static_cast<size_t>(t) * k + j] = si[j];
-                    w[static_cast<size_t>(t) * k + j] = ex[j] * inv;
-                }
-        }
-    }
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total)
+        route_token<false>(part, n_split, ldp, split_stride, bias, T, E, k, route_flags, logits, ids, w, scores_t, t, lane);
 }
 
 }  // namespace

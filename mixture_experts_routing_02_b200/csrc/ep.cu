@@ -428,7 +428,8 @@ cudaError_t launch_ep_prefetch(const EpPrefetchArgs& a, int num_sms, cudaStream_
 cudaError_t launch_ep_dispatch(const EpDispatchArgs& a0, int num_sms, cudaStream_t stream) {
     if (a0.S == 0 || a0.n_src == 0) return cudaSuccess;
     EpDispatchArgs a = a0;
-    int per = (num_sms + a.n_src - 1) / a.n_src;
+    // one CTA per SM (1024 threads, ~113 KB of shared memory), all in one wave
+    int per = num_sms / a.n_src;
     if (per > a.S) per = a.S;
     if (per < 1) per = 1;
     a.ctas_per_src = per;

@@ -484,3 +484,35 @@ def test_layer_fwd_captured_in_a_cuda_graph():
     torch.cuda.synchronize()
     assert torch.equal(graphed, eager)
     assert status.item() == 0
+
+
+@pytest.mark.parametrize("name", ["capacity", "plan"])
+def test_layer_fwd_aux_copies_the_routing_results(name):
+    """moe_layer_fwd_aux: the same output as moe_layer_fwd, and the routing results (ids, weights,
+    counts, segment offsets, dest, statistics) in the caller's buffers equal the oracle's."""
+    w = next(x for x in SMALL if x.name == name)
+    case = make_case(w, seed=1)
+    ref = _oracle_layer(case)
+    s = moe_shape(w)
+    s.out_dtype = moe.DTYPE_BF16
+    n_seg, rows = moe.moe_layout(s)
+    ws = torch.empty(moe.moe_workspace_size(s)[1], dtype=torch.uint8, device="cuda")
+    out = torch.empty(w.T, w.d, dtype=torch.bfloat16, device="cuda")
+    st = i32(1)
+    ids, wts = i32(w.T * w.k), torch.zeros(w.T * w.k, device="cuda")
+    counts, offs, dest, stats = i32(w.E), i32(n_seg + 1), i32(w.T * w.k), i32(len(moe.STAT_NAMES))
+    moe.moe_layer_fwd_aux(s, dev(case.x), dev(case.w_r), dev(case.bias), dev(case.wg), dev(case.wu), dev(case.wd),
+                          out, st, ws, topk_ids=ids, topk_w=wts, counts=counts, seg_offsets=offs, dest=dest,
+                          stats=stats)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    plain = run_layer(case, out_dtype=moe.DTYPE_BF16)
+    assert torch.equal(out, plain["out"])
+    assert (ids.cpu().numpy().reshape(w.T, w.k) == ref.ids).all()
+    assert np.abs(wts.cpu().numpy().reshape(w.T, w.k) - ref.weights).max() < 1e-4
+    assert (counts.cpu().numpy() == ref.counts).all()
+    assert (offs.cpu().numpy() == ref.segs.offsets).all()
+    assert (dest.cpu().numpy() == ref.dest).all()
+    got = dict(zip(moe.STAT_NAMES, stats.cpu().tolist()))
+    assert got["pairs"] == w.T * w.k and got["rows"] == int(ref.segs.offsets[-1])
+    assert got["dropped"] == int((ref.dest < 0).sum()) and got["max_expert_load"] == int(ref.counts.max())
