@@ -189,18 +189,19 @@ class EpRank:
             return t
 
         self.b = _RankBuffers(s, self.dev, allocate=symmetric)
-        epg = s.n_experts // self.R
         self.wg, self.wu, self.wd = _weight_slots_home(s, wg_home, wu_home, wd_home, symmetric)
         self.peers = [list(h.buffer_ptrs) for h in handles]   # xp, src, yp, wg, wu, wd: R addresses each
         self.counts = torch.zeros(s.n_experts, dtype=torch.int32, device=self.dev)
         self.counts_all = torch.zeros(self.R, s.n_experts, dtype=torch.int32, device=self.dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=self.dev)
         self._flag = torch.zeros(1, dtype=torch.int32, device=self.dev)
-        del epg
 
     def _barrier(self):
+        # stream-ordered on NCCL.  Two per step suffice: the next step's counts all-gather completes
+        # only once every rank has finished this step's combine, so the next dispatch (which writes
+        # the peers' Xp / src) and expert GEMMs (which write Yp) cannot overtake a peer's reads.
         import torch.distributed as dist
-        dist.all_reduce(self._flag, group=self.group)   # stream-ordered on NCCL
+        dist.all_reduce(self._flag, group=self.group)
 
     def forward(self, x, w_router, bias=None):
         import torch.distributed as dist

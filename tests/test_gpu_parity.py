@@ -163,8 +163,10 @@ def test_route_logits_and_bias(E, flags):
 
 @pytest.mark.parametrize("E,flags", [(8, 0), (60, 1), (256, 0)])
 def test_route_split_reduction(E, flags):
-    """moe_route_ws: the router projection's reduction split over more CTAs (partial logits in
-    the workspace, summed in order by a second kernel) gives the oracle's routing."""
+    """moe_route_ws: the router projection's reduction split over the CTAs of a cluster (partial
+    logits in the workspace, summed in order and routed by the cluster after a cluster barrier)
+    gives the oracle's routing, and exactly the routing of moe_route_from_logits on the logits it
+    wrote."""
     w = syn.Workload("route-split", T=900, d=1024, E=E, k=min(6, E), F=64, zipf_s=1.2)
     case = make_case(w, seed=3)
     s = moe_shape(w)
@@ -183,6 +185,11 @@ def test_route_split_reduction(E, flags):
     assert (ids.cpu().numpy() == rid).all()
     assert np.abs(wt.cpu().numpy() - rw).max() < 1e-4
     assert st.item() == 0
+    ids_l = i32(w.T * w.k).view(w.T, w.k)
+    wt_l = torch.empty(w.T, w.k, device="cuda")
+    moe.moe_route_from_logits(s, logits, ids_l, wt_l)
+    torch.cuda.synchronize()
+    assert torch.equal(ids_l, ids) and torch.equal(wt_l, wt), "fused routing differs from routing its logits"
     # without a workspace the same call runs the single-pass kernel
     ids2 = i32(w.T * w.k).view(w.T, w.k)
     moe.moe_route_ws(s, dev(case.x), dev(case.w_r), dev(case.bias), None, ids2, wt, st, None)
