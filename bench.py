@@ -411,7 +411,7 @@ def run_ours(args, w):
     # the router projection's reduction is split over more CTAs when its row tiles are few
     route_ws_bytes = moe.moe_route_workspace_size(s)
     route_ws = torch.empty(max(route_ws_bytes, 256), dtype=torch.uint8, device=dev) if route_ws_bytes else None
-    launches = (1                                                              # route (routing fused)
+    launches = ((2 if route_ws_bytes else 1)                                   # route (+ partial sums)
                 + (2 if ec or rr else (4 if w.n_groups and w.T * w.k > (1 << 20) else 1))  # dispatch
                 + 3)                                                           # gate_up, down, combine
 
@@ -793,12 +793,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shared-expert", type=int, default=0, metavar="F_S",
                     help="add one shared expert of inner size F_S, overlapped on a second stream (needs --out-dtype f32)")
-    ap.add_argument("--out-dtype", choices=("bf16", "f32"), default="bf16",
-                    help="element type of the layer output (default bf16)")
+    ap.add_argument("--out-dtype", choices=("auto", "bf16", "f32"), default="auto",
+                    help="element type of the layer output; auto (default): bf16 for the workloads whose "
+                         "bf16 output meets the stated tolerance at full size, fp32 otherwise")
     ap.add_argument("--ep-virtual", action="store_true",
                     help="run a balanced-plan workload as expert-parallel ranks on one GPU")
     args = ap.parse_args()
     w = syn.WORKLOADS[args.workload]
+    if args.out_dtype == "auto":
+        args.out_dtype = "bf16" if w.bf16_out else "f32"
     if args.impl == "reference":
         return run_reference(args, w)
     if args.ep_virtual:

@@ -152,10 +152,11 @@ moe_status_t route_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_
 }
 
 // The router projection has only ceil(T/128) row tiles.  When they are fewer than the SMs, its
-// reduction over d is cut into S parts (each at least 4 k-blocks of 64): S*ceil(T/128) CTAs in
-// clusters of S (one row tile per cluster) write fp32 partial logits [S][T][ldp] to a workspace,
-// and after a cluster barrier the cluster's CTAs sum the parts in order (so the result does not
-// depend on timing), add the bias and route -- one launch.
+// reduction over d is cut into S parts (each at least 4 k-blocks of 64), the S*ceil(T/128) work
+// units write fp32 partial logits [S][T][ldp] to a workspace, and a warp-per-token kernel sums
+// the parts in order (so the result does not depend on timing), adds the bias and routes.  (Routing
+// the rows inside the GEMM's clusters instead, after a cluster barrier, measured slower: it routes
+// with one warp per 8 tokens instead of one warp per token over the whole GPU.)
 constexpr int kMaxRouteSplits = 8;
 
 int route_splits(const Dims& v) {
@@ -197,11 +198,12 @@ bool route_split_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_ro
     g.BN = epad; g.n_tiles_n = 1; g.mma_n = epad; g.stages = gemm_pick_stages(epad);
     g.out = ws; g.ldo = ldp; g.status = status;
     g.k_splits = S; g.split_stride = static_cast<size_t>(v.T) * ldp;
-    // routing fused into the same launch: clusters of the S split CTAs of a row tile, one pass
-    g.bias = bias; g.logits = logits; g.topk_ids = ids; g.topk_w = w; g.scores_t = scores; g.k = v.k;
-    g.route_flags = v.flags & ~MOE_ROUTE_EXPERT_CHOICE;
-    const int grid = (v.T + 127) / 128 * S;  // <= the SM count (route_splits)
-    *result = cuda_status(launch_umma_gemm(kEpiRouteSplit, ta, tb, tb, g, grid, st));
+    const int grid = std::min(sm_count(), (v.T + 127) / 128 * S);
+    moe_status_t r = cuda_status(launch_umma_gemm(kEpiStore, ta, tb, tb, g, grid, st));
+    if (r == MOE_OK)
+        r = cuda_status(launch_route_logits(static_cast<const float*>(ws), S, ldp, g.split_stride, bias, v.T, v.E, v.k,
+                                            v.flags & ~MOE_ROUTE_EXPERT_CHOICE, logits, ids, w, scores, sm_count(), st));
+    *result = r;
     return true;
 }
 

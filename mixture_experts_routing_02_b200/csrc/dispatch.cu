@@ -1028,7 +1028,7 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const float* __restri
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total)
-        route_token<false>(part, n_split, ldp, split_stride, bias, T, E, k, route_flags, logits, ids, w, scores_t, t, lane);
+        route_token(part, n_split, ldp, split_stride, bias, T, E, k, route_flags, logits, ids, w, scores_t, t, lane);
 }
 
 }  // namespace

@@ -99,31 +99,42 @@ __global__ void __launch_bounds__(256) ep_plan_kernel(const int32_t* __restrict_
 
 // ------------------------------------------------------------------------------ replica weights
 
-// blockIdx.y = 3 * j + m: replica slot j of this rank, weight matrix m (gate, up, down).  A slot
-// whose segment is unused or empty is skipped; otherwise the expert's matrix is copied from its
-// home rank's slot into this rank's slot E/R + j (16-byte vectors, grid-stride over the matrix).
+// The copies of this rank's replica slots as one flat list of work items (slot j, matrix m, chunk c
+// of kPrefetchChunk 16-byte vectors), taken by the CTAs in turn; items of a slot whose segment is
+// unused or empty are skipped.  An item copies its chunk of expert e's matrix m from slot e - h*E/R
+// of e's home rank h into this rank's slot E/R + j.  So however few slots are in use, every CTA of
+// the grid streams their bytes.
+constexpr int kPrefetchChunk = 2048;  // 16-byte vectors per work item (32 KB)
+
 __global__ void __launch_bounds__(256) ep_prefetch_kernel(const __grid_constant__ EpPrefetchArgs a) {
-    const int j = blockIdx.y / 3, m = blockIdx.y - 3 * (blockIdx.y / 3);
     const int epg = a.E / a.R;
-    const int sg = epg + j;
-    const int e = __ldg(a.seg_expert + sg);
-    if (e < 0 || e >= a.E || __ldg(a.seg_offsets + sg + 1) <= __ldg(a.seg_offsets + sg)) return;
-    const int h = e / epg;
     const size_t mat = static_cast<size_t>(a.F) * a.d;  // elements of one expert's matrix
-    const uint4* src = reinterpret_cast<const uint4*>(a.w[m][h] + static_cast<size_t>(e - h * epg) * mat);
-    uint4* dst = reinterpret_cast<uint4*>(a.w[m][a.rank] + static_cast<size_t>(sg) * mat);
     const size_t nvec = mat / 8;
-    const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-    size_t v = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    for (; v + 3 * stride < nvec; v += 4 * stride) {
-        const uint4 a0 = __ldg(src + v), a1 = __ldg(src + v + stride);
-        const uint4 a2 = __ldg(src + v + 2 * stride), a3 = __ldg(src + v + 3 * stride);
-        dst[v] = a0;
-        dst[v + stride] = a1;
-        dst[v + 2 * stride] = a2;
-        dst[v + 3 * stride] = a3;
+    const int chunks = static_cast<int>((nvec + kPrefetchChunk - 1) / kPrefetchChunk);
+    const int64_t items = static_cast<int64_t>(a.B) * 3 * chunks;
+    for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+        const int c = static_cast<int>(it % chunks);
+        const int m = static_cast<int>((it / chunks) % 3);
+        const int j = static_cast<int>(it / (3 * static_cast<int64_t>(chunks)));
+        const int sg = epg + j;
+        const int e = __ldg(a.seg_expert + sg);
+        if (e < 0 || e >= a.E || __ldg(a.seg_offsets + sg + 1) <= __ldg(a.seg_offsets + sg)) continue;
+        const int h = e / epg;
+        const uint4* src = reinterpret_cast<const uint4*>(a.w[m][h] + static_cast<size_t>(e - h * epg) * mat);
+        uint4* dst = reinterpret_cast<uint4*>(a.w[m][a.rank] + static_cast<size_t>(sg) * mat);
+        const size_t v0 = static_cast<size_t>(c) * kPrefetchChunk;
+        const size_t v1 = v0 + kPrefetchChunk < nvec ? v0 + kPrefetchChunk : nvec;
+        size_t v = v0 + threadIdx.x;
+        for (; v + 3 * 256 < v1; v += 4 * 256) {
+            const uint4 a0 = __ldg(src + v), a1 = __ldg(src + v + 256);
+            const uint4 a2 = __ldg(src + v + 512), a3 = __ldg(src + v + 768);
+            dst[v] = a0;
+            dst[v + 256] = a1;
+            dst[v + 512] = a2;
+            dst[v + 768] = a3;
+        }
+        for (; v < v1; v += 256) dst[v] = __ldg(src + v);
     }
-    for (; v < nvec; v += stride) dst[v] = __ldg(src + v);
 }
 
 // ------------------------------------------------------------------------------ dispatch
@@ -418,10 +429,7 @@ cudaError_t launch_ep_plan(const int32_t* counts_all, int R, int S, int k, int E
 
 cudaError_t launch_ep_prefetch(const EpPrefetchArgs& a, int num_sms, cudaStream_t stream) {
     if (a.B == 0) return cudaSuccess;
-    // about two CTAs per SM over all (slot, matrix) pairs; each CTA streams its share of one matrix
-    int gx = (2 * num_sms + 3 * a.B - 1) / (3 * a.B);
-    if (gx < 1) gx = 1;
-    ep_prefetch_kernel<<<dim3(gx, 3 * a.B, 1), 256, 0, stream>>>(a);
+    ep_prefetch_kernel<<<4 * num_sms, 256, 0, stream>>>(a);  // four 256-thread CTAs per SM
     return cudaGetLastError();
 }
 

@@ -15,11 +15,7 @@ constexpr int kMaxSegments = 2048;
 constexpr size_t kGemmSmemBudget = 200 * 1024;  // operand stages of the GEMM
 constexpr size_t kGemmSmemMin = 120 * 1024;     // > half an SM's shared memory: one CTA per SM
 
-// kEpiRouteSplit: the router projection with its reduction split over the k_splits CTAs of a
-// cluster (one row tile per cluster): each CTA stores its fp32 partial tile, then, after a cluster
-// barrier, the cluster's CTAs route the tile's rows from the partials (top-k ids and weights, or
-// expert-choice scores).
-enum EpiKind : int { kEpiRoute = 0, kEpiSwiglu = 1, kEpiStore = 2, kEpiRouteSplit = 3 };
+enum EpiKind : int { kEpiRoute = 0, kEpiSwiglu = 1, kEpiStore = 2 };
 
 struct GemmArgs {
     const int32_t* seg_offsets;  // [n_seg+1] or nullptr: a single segment of M rows

@@ -2,8 +2,8 @@
 // partial slices (in slice order, so the result does not depend on timing) plus the bias; then
 // either the top-k ids in descending order (equal logits: the lower id) with their weights (softmax
 // over the selected logits, or over all E with MOE_ROUTE_SOFTMAX_ALL), or, for expert-choice
-// routing (scores_t non-null), the softmax over all E stored expert-major.  Shared by the routing
-// kernel and the router GEMM's fused epilogue.
+// routing (scores_t non-null), the softmax over all E stored expert-major.  Used by
+// route_logits_kernel, one warp per token.
 //
 // Sources: "Sparsely-Gated MoE 구현 관점에서 살펴보기", sections "Top-2 라우팅의 수치 예시" and
 // "pure Python으로 Top-k Router 확인하기"; "Expert를 똑같이 나눴는데도 GPU가 대기하는 이유", section
@@ -16,9 +16,6 @@
 namespace moe {
 namespace {
 
-// COHERENT: the partial slices were written by other CTAs of the same kernel, so they are read
-// through L2 (ld.global.cg) rather than the read-only path.
-template <bool COHERENT>
 __device__ __forceinline__ void route_token(const float* __restrict__ part, int n_split, int ldp, size_t split_stride,
                                             const float* __restrict__ bias, int T, int E, int k, int route_flags,
                                             float* __restrict__ logits, int32_t* __restrict__ ids,
@@ -31,8 +28,8 @@ __device__ __forceinline__ void route_token(const float* __restrict__ part, int 
         v[u] = -INFINITY;
         if (e < E) {
             const float* p = part + static_cast<size_t>(t) * ldp + e;
-            float acc = COHERENT ? __ldcg(p) : __ldg(p);
-            for (int sp = 1; sp < n_split; ++sp) acc += COHERENT ? __ldcg(p + sp * split_stride) : __ldg(p + sp * split_stride);
+            float acc = __ldg(p);
+            for (int sp = 1; sp < n_split; ++sp) acc += __ldg(p + sp * split_stride);
             if (bias != nullptr) acc += __ldg(bias + e);
             v[u] = acc;
             if (logits != nullptr) logits[static_cast<size_t>(t) * E + e] = acc;

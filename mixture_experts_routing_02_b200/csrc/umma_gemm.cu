@@ -31,7 +31,6 @@
 // one tile overlap the main loop of the next.
 #include "common.cuh"
 #include "kernels.h"
-#include "route.cuh"
 
 namespace moe {
 
@@ -217,8 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     const uint32_t tmem_base = tmem_base_sh;
-    static_assert(!SPLITK || EPI == kEpiStore || EPI == kEpiRouteSplit, "split reductions store fp32 partials");
-    static_assert(EPI != kEpiRouteSplit || SPLITK, "the fused split router needs the split reduction");
+    static_assert(!SPLITK || EPI == kEpiStore, "split reductions use the plain fp32 epilogue");
     const int n_split = SPLITK ? g.k_splits : 1;
     const int total = tile_prefix[g.n_seg] * g.n_tiles_n * n_split;
     const int nkb = g.K / kBK;
@@ -324,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool valid = row < c.row_end;
             const int n0 = c.n * g.BN;
 
-            if (EPI == kEpiSwiglu || EPI == kEpiStore || EPI == kEpiRouteSplit) {
+            if (EPI == kEpiSwiglu || EPI == kEpiStore) {
                 epilogue_rows<EPI>(g, t_row, c.row0 + quarter * 32, c.row_end, n0, lane,
                                    epi_stage + (warp - 2) * kStageWords, out_off);
             } else if (g.scores_t != nullptr) {
@@ -438,23 +436,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (EPI == kEpiRouteSplit) {
-        // One cluster = the n_split CTAs of one row tile, one pass (grid = row tiles x n_split).  The
-        // barrier's release / acquire makes every CTA's partial tile visible to the whole cluster;
-        // then CTA s of the cluster routes rows s, s + n_split, ... of the tile, one warp per row,
-        // summing the partials in split order (the same sums as the separate routing kernel).
-        cluster_sync_all();
-        if (warp >= 2 && total == static_cast<int>(gridDim.x)) {
-            const int split = static_cast<int>(blockIdx.x) % n_split;
-            const int row0 = (static_cast<int>(blockIdx.x) / n_split) * kBM;
-            for (int i = split + n_split * (warp - 2); i < kBM; i += 4 * n_split) {
-                const int row = row0 + i;
-                if (row < g.M)
-                    route_token<true>(static_cast<const float*>(g.out), n_split, g.ldo, g.split_stride, g.bias, g.M,
-                                      g.N, g.k, g.route_flags, g.logits, g.topk_ids, g.topk_w, g.scores_t, row, lane);
-            }
-        }
-    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
@@ -651,9 +632,7 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     if (smem < kGemmSmemMin) smem = kGemmSmemMin;  // keeps one CTA per SM (all TMEM columns are taken)
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    // the fused split router runs as clusters of its k_splits CTAs (one row tile each)
-    const unsigned cluster = EPI == kEpiRouteSplit ? static_cast<unsigned>(g.k_splits) : 1u;
-    err = launch_pdl_cluster(kern, dim3(grid), dim3(kThreads), smem, stream, cluster, a, b0, b1, g);
+    err = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, a, b0, b1, g);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
@@ -695,7 +674,6 @@ cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b
     switch (epi) {
         case kEpiRoute: return launch_one<kEpiRoute, false>(a, b0, b1, g, grid, stream);
         case kEpiSwiglu: return launch_one<kEpiSwiglu, false>(a, b0, b1, g, grid, stream);
-        case kEpiRouteSplit: return launch_one<kEpiRouteSplit, true>(a, b0, b1, g, grid, stream);
         default:
             return g.k_splits > 1 ? launch_one<kEpiStore, true>(a, b0, b1, g, grid, stream)
                                   : launch_one<kEpiStore, false>(a, b0, b1, g, grid, stream);

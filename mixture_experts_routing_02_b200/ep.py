@@ -157,9 +157,10 @@ class VirtualRanks:
         return [x.out for x in b]
 
     def kernel_launches(self) -> int:
-        """Kernels one forward launches (router with fused routing, histogram, plan, prefetch per rank;
-        one dispatch; gate/up + down per rank; one combine)."""
-        return self.R * (1 + 1 + 1 + 1 + 2) + 2
+        """Kernels one forward launches (route GEMM + routing, histogram, plan, prefetch per rank; one
+        dispatch; gate/up + down per rank; one combine)."""
+        route = 2 if self.bufs[0].route_ws is not None else 1
+        return self.R * (route + 1 + 1 + 1 + 2) + 2
 
 
 class EpRank:

@@ -52,6 +52,7 @@ class Workload:
     replica_slots: int = 0         # B per group
     expert_choice: bool = False    # experts choose tokens; C = ceil(capacity_factor * T * k / E)
     reroute: bool = False          # pairs over capacity go to their token's next open candidate
+    bf16_out: bool = False         # the full-size layer output meets the stated tolerance in bf16
 
     @property
     def tokens_per_group(self) -> int:
@@ -62,10 +63,10 @@ class Workload:
 
 
 TINY = Workload("tiny", T=64, d=128, E=8, k=2, F=256)
-MIXTRAL_LIKE = Workload("mixtral-like", T=4096, d=4096, E=8, k=2, F=14336)
-DEEPSEEK_LIKE = Workload("deepseek-like", T=4096, d=7168, E=256, k=8, F=2048)
+MIXTRAL_LIKE = Workload("mixtral-like", T=4096, d=4096, E=8, k=2, F=14336, bf16_out=True)
+DEEPSEEK_LIKE = Workload("deepseek-like", T=4096, d=7168, E=256, k=8, F=2048, bf16_out=True)
 SKEWED = Workload("skewed", T=8192, d=4096, E=64, k=2, F=1408,
-                  zipf_s=1.2, capacity_factor=1.25)
+                  zipf_s=1.2, capacity_factor=1.25, bf16_out=True)
 BALANCED = Workload("balanced-plan", T=32768, d=7168, E=256, k=8, F=2048,
                     zipf_s=1.2, n_groups=8, replica_slots=32)
 
