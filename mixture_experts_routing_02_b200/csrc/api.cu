@@ -347,6 +347,30 @@ moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* id
     a.first_tile = first_tile;
     a.n_tiles = permute_n_tiles(v.T, v.k);
     const int64_t pairs = static_cast<int64_t>(v.T) * v.k;
+    if (!plan_ready && a.n_tiles > 0 && v.R > 0 && v.R <= kEpMaxRanks && first_tile == 0 &&
+        static_cast<int64_t>(v.S) * v.k <= kCountMaxPairsPlan) {
+        // The balanced plan's R token groups run as R sources of the expert-parallel dispatch, all
+        // buffers local: each CTA counts only its own group's ids (the per-group counts come from
+        // one small launch), and the layout is the same.  Counts per group go to the partials area.
+        int32_t* counts_all = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + scratch);
+        moe_status_t s = cuda_status(launch_group_histogram(ids, v.R, v.S, v.k, v.E, counts_all, st));
+        if (s != MOE_OK) return s;
+        EpDispatchArgs e{};
+        const int cap = v.S * v.k;
+        for (int g = 0; g < v.R; ++g) {
+            e.x[g] = a.x + static_cast<size_t>(g) * v.S * v.d;
+            e.ids[g] = ids + static_cast<size_t>(g) * cap;
+            e.dest[g] = dest + static_cast<size_t>(g) * cap;
+            e.xp[g] = a.xp + static_cast<size_t>(g) * cap * v.d;
+            e.src[g] = src + static_cast<size_t>(g) * cap;
+        }
+        e.counts_all = counts_all; e.status = status;
+        e.R = v.R; e.S = v.S; e.k = v.k; e.E = v.E; e.d = v.d; e.B = v.B; e.n_seg = v.n_seg;
+        e.src0 = 0; e.n_src = v.R;
+        e.counts_out = counts; e.seg_expert_out = seg_expert; e.seg_offsets_out = seg_offsets;
+        e.seg_first_rank_out = seg_first_rank;
+        return cuda_status(launch_ep_dispatch(e, sm_count(), st));
+    }
     if (!plan_ready && a.n_tiles > 0 &&
         (v.R == 0 || (pairs <= kCountMaxPairsPlan && first_tile == 0))) {
         // counts, tables, ranks and row copies in one launch

@@ -12,6 +12,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <unordered_map>
 #include <utility>
 
 #include "../../include/moe_routing.h"
@@ -339,6 +341,29 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 __host__ __device__ constexpr int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) costs far more host time than a launch, so it is
+// made once per kernel, device and size: a size no larger than one already set is not set again.
+template <typename... KArgs>
+inline cudaError_t set_max_dynamic_smem(void (*kern)(KArgs...), int bytes) {
+    static std::mutex mu;
+    static std::unordered_map<uint64_t, int> done;  // (device, kernel address) -> bytes set
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    const uint64_t key = (static_cast<uint64_t>(dev) << 56) ^ reinterpret_cast<uint64_t>(kern);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        const auto it = done.find(key);
+        if (it != done.end() && it->second >= bytes) return cudaSuccess;
+    }
+    const cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (err == cudaSuccess) {
+        std::lock_guard<std::mutex> lock(mu);
+        int& v = done[key];
+        if (bytes > v) v = bytes;
+    }
+    return err;
+}
 
 // Launch `kern` on `stream` with programmatic stream serialization (see griddep_wait), plus an
 // optional cluster shape.  Should the runtime refuse the attribute on this stream, the kernel is

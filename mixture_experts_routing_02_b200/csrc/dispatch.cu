@@ -834,7 +834,7 @@ __device__ __forceinline__ int warp_range_compact(int n, int* warp_cnt /*[33]*/,
 // and writes them to their positions.  A token's first k candidates are its top-k.
 template <int U>
 __global__ void __launch_bounds__(256) candidate_order_kernel(const float* __restrict__ logits, int T, int E,
-                                                              uint8_t* __restrict__ cand) {
+                                                              int stride, uint8_t* __restrict__ cand) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
@@ -862,7 +862,7 @@ __global__ void __launch_bounds__(256) candidate_order_kernel(const float* __res
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int e = lane + 32 * u;
-            if (e < E) cand[static_cast<size_t>(t) * E + rank[u]] = static_cast<uint8_t>(e);
+            if (e < E) cand[static_cast<size_t>(t) * stride + rank[u]] = static_cast<uint8_t>(e);
         }
     }
 }
@@ -935,10 +935,21 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_kernel(RerouteArgs
             for (int i = tid; i < n_pend; i += blockDim.x) {
                 if (next[i] != m) continue;
                 const int t = pend[i] / k;
-                // the next candidate with room (experts never reopen, so a skipped one stays skipped)
-                const uint8_t* ct = a.cand + static_cast<size_t>(t) * E;
+                // the next candidate with room (experts never reopen, so a skipped one stays
+                // skipped); the token's list is read 16 candidates per load (rows 16-byte aligned)
+                const uint8_t* ct = a.cand + static_cast<size_t>(t) * a.cand_stride;
                 int pos = a.cur_pos[t];
-                while (pos < E && s_room[ct[pos]] <= 0) ++pos;
+                while (pos < E) {
+                    const int base = pos & ~15;
+                    const uint4 c4 = __ldcg(reinterpret_cast<const uint4*>(ct + base));
+                    const uint32_t words[4] = {c4.x, c4.y, c4.z, c4.w};
+                    bool found = false;
+                    for (; pos < base + 16 && pos < E; ++pos) {
+                        const int ex = (words[(pos - base) >> 2] >> (8 * ((pos - base) & 3))) & 0xffu;
+                        if (s_room[ex] > 0) { found = true; break; }
+                    }
+                    if (found) break;
+                }
                 a.prop[i] = pos < E ? ct[pos] : -1;
                 a.cur_pos[t] = pos < E ? pos + 1 : E;
             }
@@ -1126,8 +1137,7 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
     if (grid > a.T) grid = a.T;
     if (a.R > 0) {
         const int smem = static_cast<int>(sizeof(CountPlanSmem));
-        const cudaError_t err = cudaFuncSetAttribute(dispatch_count_kernel<true>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        const cudaError_t err = set_max_dynamic_smem(dispatch_count_kernel<true>, smem);
         if (err != cudaSuccess) return err;
         const cudaError_t e2 = launch_pdl(dispatch_count_kernel<true>, dim3(grid), dim3(kCountThreads), smem, stream, a);
         if (e2 != cudaSuccess) return e2;
@@ -1158,14 +1168,16 @@ cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16*
     a.fexp = reinterpret_cast<int32_t*>(take(tk * 4));
     a.fslot = reinterpret_cast<int32_t*>(take(tk * 4));
     a.cur_pos = reinterpret_cast<int32_t*>(take(static_cast<size_t>(a.T) * 4));
-    a.cand = take(static_cast<size_t>(a.T) * a.E);
+    a.cand_stride = (a.E + 15) & ~15;  // <= kMaxExperts bytes per token, as reroute_ws_bytes reserves
+    a.cand = take(static_cast<size_t>(a.T) * a.cand_stride);
     {
         int grid = (a.T + 7) / 8;
         if (grid > 8 * num_sms) grid = 8 * num_sms;
-        if (a.E <= 32) candidate_order_kernel<1><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, a.cand);
-        else if (a.E <= 64) candidate_order_kernel<2><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, a.cand);
-        else if (a.E <= 128) candidate_order_kernel<4><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, a.cand);
-        else candidate_order_kernel<8><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, a.cand);
+        const int st = a.cand_stride;
+        if (a.E <= 32) candidate_order_kernel<1><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, st, a.cand);
+        else if (a.E <= 64) candidate_order_kernel<2><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, st, a.cand);
+        else if (a.E <= 128) candidate_order_kernel<4><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, st, a.cand);
+        else candidate_order_kernel<8><<<grid, 256, 0, stream>>>(a.logits, a.T, a.E, st, a.cand);
         const cudaError_t e0 = cudaGetLastError();
         if (e0 != cudaSuccess) return e0;
     }

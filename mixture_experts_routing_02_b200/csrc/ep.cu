@@ -185,6 +185,8 @@ __global__ void __launch_bounds__(kEpThreads, 1) ep_dispatch_kernel(const __grid
     __shared__ int s_run[kMaxExperts];  // pairs of each expert before the current chunk
     __shared__ int s_wcnt[kEpWarps][kMaxExperts];
 
+    griddep_wait();
+    griddep_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int i_src = blockIdx.x / a.ctas_per_src;
     const int G = a.ctas_per_src;
@@ -232,6 +234,15 @@ __global__ void __launch_bounds__(kEpThreads, 1) ep_dispatch_kernel(const __grid
 
     // 2. the plan over all ranks (the first CTA of the launch reports an infeasible plan)
     compute_plan(ps.plan, E, a.R, a.S, k, a.B, ps.seg_e, ps.seg_off, ps.seg_fr, a.status, blockIdx.x == 0);
+    if (blockIdx.x == 0 && a.seg_offsets_out != nullptr) {
+        for (int e = tid; e < E; e += blockDim.x) a.counts_out[e] = ps.plan.c[e];
+        for (int sg = tid; sg < a.n_seg; sg += blockDim.x) {
+            a.seg_expert_out[sg] = ps.seg_e[sg];
+            a.seg_offsets_out[sg] = ps.seg_off[sg];
+            a.seg_first_rank_out[sg] = ps.seg_fr[sg];
+        }
+        if (tid == 0) a.seg_offsets_out[a.n_seg] = ps.seg_off[a.n_seg];
+    }
     for (int e = tid; e < E; e += blockDim.x) ps.cfill[e] = 0;
     __syncthreads();
     for (int sg = tid; sg < a.n_seg; sg += blockDim.x) {
@@ -340,6 +351,37 @@ __global__ void __launch_bounds__(kEpThreads, 1) ep_dispatch_kernel(const __grid
     __threadfence_system();
 }
 
+// Pairs of each expert in each token group: CTA g counts the S*k ids of group g in shared memory
+// (16-byte loads when aligned) and writes counts_all[g][0..E) -- no atomics in global memory, so
+// nothing needs clearing first.
+__global__ void __launch_bounds__(kEpThreads) group_histogram_kernel(const int32_t* __restrict__ ids, int S, int k,
+                                                                     int E, int32_t* __restrict__ counts_all) {
+    __shared__ int h[kMaxExperts];
+    griddep_wait();
+    griddep_launch_dependents();
+    const int g = blockIdx.x;
+    const int n = S * k;
+    const int32_t* gi = ids + static_cast<size_t>(g) * n;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    __syncthreads();
+    auto one = [&](int e) {
+        if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(&h[e], 1);
+    };
+    int from = 0;
+    if ((reinterpret_cast<uintptr_t>(gi) & 15u) == 0) {
+        const int n4 = n >> 2;
+        const int4* g4 = reinterpret_cast<const int4*>(gi);
+        for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+            const int4 v = __ldg(g4 + i);
+            one(v.x); one(v.y); one(v.z); one(v.w);
+        }
+        from = n4 << 2;
+    }
+    for (int i = from + threadIdx.x; i < n; i += blockDim.x) one(__ldg(gi + i));
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) counts_all[static_cast<size_t>(g) * E + e] = h[e];
+}
+
 // ------------------------------------------------------------------------------ combine
 
 // out_i[t] = sum over j with dest_i[t*k+j] >= 0 of w_i[t, j] * Yp_owner[row], accumulated in
@@ -420,7 +462,7 @@ cudaError_t launch_ep_plan(const int32_t* counts_all, int R, int S, int k, int E
                            int32_t* seg_expert, int32_t* seg_slot, int32_t* seg_offsets, int32_t* status,
                            cudaStream_t stream) {
     const int smem = static_cast<int>(sizeof(EpPlanSmem));
-    const cudaError_t err = cudaFuncSetAttribute(ep_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const cudaError_t err = set_max_dynamic_smem(ep_plan_kernel, smem);
     if (err != cudaSuccess) return err;
     ep_plan_kernel<<<1, 256, smem, stream>>>(counts_all, R, S, k, E, B, rank, counts, seg_expert, seg_slot,
                                              seg_offsets, status);
@@ -442,10 +484,19 @@ cudaError_t launch_ep_dispatch(const EpDispatchArgs& a0, int num_sms, cudaStream
     if (per < 1) per = 1;
     a.ctas_per_src = per;
     const int smem = static_cast<int>(sizeof(EpSmem));
-    const cudaError_t err =
-        cudaFuncSetAttribute(ep_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t err = set_max_dynamic_smem(ep_dispatch_kernel, smem);
     if (err != cudaSuccess) return err;
-    ep_dispatch_kernel<<<per * a.n_src, kEpThreads, smem, stream>>>(a);
+    err = launch_pdl(ep_dispatch_kernel, dim3(per * a.n_src), dim3(kEpThreads), static_cast<size_t>(smem), stream, a);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_group_histogram(const int32_t* ids, int R, int S, int k, int E, int32_t* counts_all,
+                                   cudaStream_t stream) {
+    if (R == 0) return cudaSuccess;
+    const cudaError_t err = launch_pdl(group_histogram_kernel, dim3(R), dim3(kEpThreads), 0, stream, ids, S, k, E,
+                                       counts_all);
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 

@@ -274,9 +274,7 @@ cudaError_t launch_ec_select(const float* scores_t, int T, int E, int cp, int32_
     if (T <= kSelectSmemKeys) {
         const size_t smem = static_cast<size_t>(T) * sizeof(uint32_t);
         if (smem > 48 * 1024) {
-            const cudaError_t err = cudaFuncSetAttribute(ec_select_kernel<true>,
-                                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                         static_cast<int>(kSelectSmemKeys * sizeof(uint32_t)));
+            const cudaError_t err = set_max_dynamic_smem(ec_select_kernel<true>, static_cast<int>(kSelectSmemKeys * sizeof(uint32_t)));
             if (err != cudaSuccess) return err;
         }
         ec_select_kernel<true><<<E, kSelectThreads, smem, stream>>>(scores_t, T, E, cp, seg_expert, seg_offsets, src,

@@ -131,7 +131,8 @@ struct RerouteArgs {
     int32_t* src;
     // scratch, set by launch_reroute from the workspace
     int32_t *pend, *pend2, *prop, *fexp, *fslot, *cur_pos;
-    uint8_t* cand;  // [T, E] each token's experts in candidate order
+    uint8_t* cand;   // [T, cand_stride] each token's experts in candidate order (first E bytes of a row)
+    int cand_stride; // E rounded up to 16: every row starts on a 16-byte boundary
 };
 size_t reroute_ws_bytes(int T, int k);
 cudaError_t launch_reroute(const RerouteArgs& a, void* ws, const __nv_bfloat16* x, __nv_bfloat16* xp, int d,
@@ -170,6 +171,12 @@ struct EpDispatchArgs {
     const int32_t* counts_all;            // [R, E]
     int32_t* status;
     int R, S, k, E, d, B, n_seg, src0, n_src, ctas_per_src;
+    // optional (nullable): the totals and the tables of all R groups, written by CTA 0 (the
+    // single-GPU balanced dispatch, where the R groups are token groups of one GPU)
+    int32_t* counts_out;          // [E]
+    int32_t* seg_expert_out;      // [n_seg]
+    int32_t* seg_offsets_out;     // [n_seg + 1]
+    int32_t* seg_first_rank_out;  // [n_seg]
 };
 struct EpCombineArgs {
     const float* yp[kEpMaxRanks];        // [R] each owner's Yp [S*k, d]
@@ -189,6 +196,9 @@ cudaError_t launch_ep_plan(const int32_t* counts_all, int R, int S, int k, int E
                            cudaStream_t stream);
 cudaError_t launch_ep_prefetch(const EpPrefetchArgs& a, int num_sms, cudaStream_t stream);
 cudaError_t launch_ep_dispatch(const EpDispatchArgs& a, int num_sms, cudaStream_t stream);
+// counts_all[g, e] = pairs of expert e among the S*k pairs of token group g (one CTA per group)
+cudaError_t launch_group_histogram(const int32_t* ids, int R, int S, int k, int E, int32_t* counts_all,
+                                   cudaStream_t stream);
 cudaError_t launch_ep_combine(const EpCombineArgs& a, bool out_bf16, int num_sms, cudaStream_t stream);
 
 // stats.cu: MOE_STAT_COUNT values from the counts (nullable) and segment tables of one dispatch

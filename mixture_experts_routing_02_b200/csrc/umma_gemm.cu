@@ -630,7 +630,7 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     auto kern = umma_gemm_kernel<EPI, SPLITK>;
     size_t smem = gemm_smem_bytes(g.stages, g.mma_n);
     if (smem < kGemmSmemMin) smem = kGemmSmemMin;  // keeps one CTA per SM (all TMEM columns are taken)
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t err = set_max_dynamic_smem(kern, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     err = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, a, b0, b1, g);
     if (err != cudaSuccess) return err;
@@ -655,7 +655,7 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, cons
     auto kern = umma_gemm_pair_kernel<EPI>;
     size_t smem = gemm_pair_smem_bytes(g.stages, g.mma_n);
     if (smem < kGemmSmemMin) smem = kGemmSmemMin;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t err = set_max_dynamic_smem(kern, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     err = launch_pdl_cluster(kern, dim3(2 * n_pairs), dim3(kThreads), smem, stream, 2u, a, b0, b1, g);
     if (err != cudaSuccess) return err;

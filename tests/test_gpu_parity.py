@@ -293,10 +293,13 @@ def test_histogram_segments_and_plan_on_given_ids(sigma):
     assert (so2.cpu().numpy() == ref2.offsets).all() and (se2.cpu().numpy() == ref2.expert).all()
 
 
-def test_dispatch_large_balanced_plan():
-    """A balanced plan with more than 2^20 pairs takes the multi-launch path (histogram partials,
-    plan, look-back ranks, row copies): tables and positions bit for bit against the oracle."""
-    T, d, E, k, R, B = 140000, 64, 16, 8, 4, 4
+@pytest.mark.parametrize("T,E,R", [(140000, 16, 4), (140032, 32, 32)], ids=["4-groups", "32-groups"])
+def test_dispatch_large_balanced_plan(T, E, R):
+    """A balanced plan with more than 2^20 pairs: with 4 groups the grouped dispatch (per-group
+    counts, then every CTA ranking its own group's pairs), with 32 groups the multi-launch path
+    (histogram partials, plan, look-back ranks, row copies): tables and positions bit for bit
+    against the oracle."""
+    d, k, B = 64, 8, 4
     ids = syn.lognormal_topk_ids(E, T, k, 1.0, seed=12).cuda()
     s = moe.shape(T, d, E, k, 64, n_groups=R, replica_slots=B)
     n_seg, rows = moe.moe_layout(s)

@@ -6,8 +6,9 @@ library instead of a caller-provided workspace.
 
 The array is read by every dispatch path that needs scratch: the single-launch
 look-back dispatch (more than 65536 pairs, no plan), a dispatch on given plan
-tables (plan_ready = 1), and a balanced plan of more than 2^20 pairs (histogram
-partials, plan, look-back ranks, row copies).  Each case first runs a call of a
+tables (plan_ready = 1), a balanced plan of up to 16 groups (per-group counts,
+then the grouped dispatch), and a balanced plan of more than 16 groups and more
+than 2^20 pairs (histogram partials, plan, look-back ranks, row copies).  Each case first runs a call of a
 different shape so that stale ticket and look-back words are left in the array,
 then calls moe_dispatch_static twice in a row; both results must equal
 moe_dispatch's (with its own workspace) and the oracle's bit for bit.
@@ -51,8 +52,10 @@ CASES = [
     dict(name="lookback-capacity", T=9000, d=64, E=32, k=8, R=0, B=0, C=2000, sigma=1.2, plan_ready=0),
     # tables given by the caller: look-back ranks and row copies after clearing the words
     dict(name="plan-given", T=800, d=128, E=32, k=4, R=4, B=8, C=0, sigma=2.0, plan_ready=1),
-    # a balanced plan of more than 2^20 pairs: histogram partials, plan, look-back ranks, row copies
-    dict(name="large-plan", T=140000, d=64, E=16, k=8, R=4, B=4, C=0, sigma=1.0, plan_ready=0),
+    # a balanced plan of up to 16 groups: per-group counts in the array, then the grouped dispatch
+    dict(name="plan-groups", T=1200, d=192, E=32, k=4, R=4, B=8, C=0, sigma=2.0, plan_ready=0),
+    # more than 16 groups and more than 2^20 pairs: histogram partials, plan, look-back ranks, copies
+    dict(name="large-plan", T=140032, d=64, E=32, k=8, R=32, B=4, C=0, sigma=1.0, plan_ready=0),
     # at most 65536 pairs and no plan: the count dispatch, which needs no scratch at all
     dict(name="count", T=999, d=128, E=16, k=2, R=0, B=0, C=90, sigma=1.0, plan_ready=0),
 ]
