@@ -353,7 +353,7 @@ moe_status_t dispatch_impl(const Dims& v, const moe_bf16_t* x, const int32_t* id
         // buffers local: each CTA counts only its own group's ids (the per-group counts come from
         // one small launch), and the layout is the same.  Counts per group go to the partials area.
         int32_t* counts_all = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + scratch);
-        moe_status_t s = cuda_status(launch_group_histogram(ids, v.R, v.S, v.k, v.E, counts_all, st));
+        moe_status_t s = cuda_status(launch_group_histogram(ids, v.R, v.S, v.k, v.E, counts_all, sm_count(), st));
         if (s != MOE_OK) return s;
         EpDispatchArgs e{};
         const int cap = v.S * v.k;

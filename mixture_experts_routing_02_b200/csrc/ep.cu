@@ -351,15 +351,14 @@ __global__ void __launch_bounds__(kEpThreads, 1) ep_dispatch_kernel(const __grid
     __threadfence_system();
 }
 
-// Pairs of each expert in each token group: CTA g counts the S*k ids of group g in shared memory
-// (16-byte loads when aligned) and writes counts_all[g][0..E) -- no atomics in global memory, so
-// nothing needs clearing first.
+// Pairs of each expert in each token group: the CTAs of group g (blockIdx.x / per_group) each
+// count a slice of the group's S*k ids in shared memory (16-byte loads when aligned) and add their
+// nonzero counts to counts_all[g][e], which the launcher clears first.
 __global__ void __launch_bounds__(kEpThreads) group_histogram_kernel(const int32_t* __restrict__ ids, int S, int k,
-                                                                     int E, int32_t* __restrict__ counts_all) {
+                                                                     int E, int per_group,
+                                                                     int32_t* __restrict__ counts_all) {
     __shared__ int h[kMaxExperts];
-    griddep_wait();
-    griddep_launch_dependents();
-    const int g = blockIdx.x;
+    const int g = blockIdx.x / per_group, c = blockIdx.x - g * per_group;
     const int n = S * k;
     const int32_t* gi = ids + static_cast<size_t>(g) * n;
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
@@ -371,15 +370,16 @@ __global__ void __launch_bounds__(kEpThreads) group_histogram_kernel(const int32
     if ((reinterpret_cast<uintptr_t>(gi) & 15u) == 0) {
         const int n4 = n >> 2;
         const int4* g4 = reinterpret_cast<const int4*>(gi);
-        for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+        for (int i = c * blockDim.x + threadIdx.x; i < n4; i += per_group * blockDim.x) {
             const int4 v = __ldg(g4 + i);
             one(v.x); one(v.y); one(v.z); one(v.w);
         }
         from = n4 << 2;
     }
-    for (int i = from + threadIdx.x; i < n; i += blockDim.x) one(__ldg(gi + i));
+    for (int i = from + c * blockDim.x + threadIdx.x; i < n; i += per_group * blockDim.x) one(__ldg(gi + i));
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) counts_all[static_cast<size_t>(g) * E + e] = h[e];
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        if (h[e] != 0) atomicAdd(counts_all + static_cast<size_t>(g) * E + e, h[e]);
 }
 
 // ------------------------------------------------------------------------------ combine
@@ -492,11 +492,15 @@ cudaError_t launch_ep_dispatch(const EpDispatchArgs& a0, int num_sms, cudaStream
 }
 
 cudaError_t launch_group_histogram(const int32_t* ids, int R, int S, int k, int E, int32_t* counts_all,
-                                   cudaStream_t stream) {
+                                   int num_sms, cudaStream_t stream) {
     if (R == 0) return cudaSuccess;
-    const cudaError_t err = launch_pdl(group_histogram_kernel, dim3(R), dim3(kEpThreads), 0, stream, ids, S, k, E,
-                                       counts_all);
+    cudaError_t err = cudaMemsetAsync(counts_all, 0, static_cast<size_t>(R) * E * sizeof(int32_t), stream);
     if (err != cudaSuccess) return err;
+    int per_group = num_sms / R;
+    const int per_needed = (S * k + 4 * kEpThreads - 1) / (4 * kEpThreads);  // ~4 ids per thread at least
+    if (per_group > per_needed) per_group = per_needed;
+    if (per_group < 1) per_group = 1;
+    group_histogram_kernel<<<R * per_group, kEpThreads, 0, stream>>>(ids, S, k, E, per_group, counts_all);
     return cudaGetLastError();
 }
 

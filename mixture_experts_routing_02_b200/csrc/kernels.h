@@ -196,9 +196,10 @@ cudaError_t launch_ep_plan(const int32_t* counts_all, int R, int S, int k, int E
                            cudaStream_t stream);
 cudaError_t launch_ep_prefetch(const EpPrefetchArgs& a, int num_sms, cudaStream_t stream);
 cudaError_t launch_ep_dispatch(const EpDispatchArgs& a, int num_sms, cudaStream_t stream);
-// counts_all[g, e] = pairs of expert e among the S*k pairs of token group g (one CTA per group)
+// counts_all[g, e] = pairs of expert e among the S*k pairs of token group g (cleared, then counted
+// by about num_sms CTAs)
 cudaError_t launch_group_histogram(const int32_t* ids, int R, int S, int k, int E, int32_t* counts_all,
-                                   cudaStream_t stream);
+                                   int num_sms, cudaStream_t stream);
 cudaError_t launch_ep_combine(const EpCombineArgs& a, bool out_bf16, int num_sms, cudaStream_t stream);
 
 // stats.cu: MOE_STAT_COUNT values from the counts (nullable) and segment tables of one dispatch
