@@ -313,6 +313,22 @@ def pin_expert_choice_map_argsort(seed=22, T=23, E=5, C=6):
     return bool(got.shape == (T, E) and np.array_equal(got, want))
 
 
+def pin_ec_margin_enforcement(seed=23, T=300, E=6, C=40, gap=5e-4):
+    """After enforce_ec_margin, every expert's C-th and (C+1)-th largest scores (library softmax over
+    the experts, library descending sort) are at least `gap` (relative) apart, and the inputs needed
+    redraws to get there."""
+    w = syn.Workload("ecm", T=T, d=64, E=E, k=1, F=64)
+    x, wr, b = syn.router_inputs(w, seed)
+
+    def worst(xx):
+        l = torch.nn.functional.linear(xx.double(), wr.double(), b.double() if b is not None else None)
+        srt = torch.sort(torch.softmax(l, dim=1), dim=0, descending=True).values
+        return float(((srt[C - 1] - srt[C]) / srt[C - 1]).min())
+    before = worst(x)
+    n = oracle.enforce_ec_margin(x, wr, b, C, lambda t, a: syn.x_row_redraw(w, seed, t, a), min_rel_gap=gap)
+    return bool(before < gap and n > 0 and worst(x) >= gap)
+
+
 def pin_silu_library():
     z = np.linspace(-30, 30, 2001)
     ref = torch.nn.functional.silu(torch.from_numpy(z)).numpy()
@@ -510,6 +526,10 @@ def test_expert_choice_map_from_argsort():
     assert pin_expert_choice_map_argsort()
 
 
+def test_expert_choice_margin_enforcement():
+    assert pin_ec_margin_enforcement()
+
+
 def test_shared_expert_adds_a_dense_ffn():
     assert pin_shared_expert_additive()
 
@@ -689,6 +709,8 @@ MUTATIONS = [
     ("reroute_positions", _mut_reroute_positions_next_offset, [pin_reroute_positions_worked, pin_layer_reroute_eager]),
     ("layer_forward_reroute", _mut_layer_reroute_drops_moved, [pin_layer_reroute_eager]),
     ("expert_choice_map", _mut_ec_map_left_boundary, [pin_expert_choice_map_argsort]),
+    ("ec_margin_violations", lambda S, capacity, min_rel_gap: np.zeros(np.asarray(S).shape[1], dtype=bool),
+     [pin_ec_margin_enforcement]),   # never asks for a redraw
 ]
 
 
