@@ -523,8 +523,7 @@ def run_ours(args, w):
 
     # timed regions.  Clocks are sampled through all of them (the layer loop, the call-by-call
     # loop and the end-to-end run below), which also gives a short step loop enough samples.
-    # (1) the layer through moe_layer_fwd, events only around each step: its kernels may overlap
-    # their neighbours' launch and prologue (programmatic dependent launch)
+    # (1) the layer through moe_layer_fwd, events only around each step
     layer_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(args.steps)]
     barrier()

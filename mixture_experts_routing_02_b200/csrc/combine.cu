@@ -24,8 +24,6 @@ template <int KMAX, int UNROLL, typename OutT>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ dest,
                                                       const float* __restrict__ w, const float* __restrict__ base,
                                                       int T, int k, int d, int rows, OutT* __restrict__ out) {
-    griddep_wait();
-    griddep_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     const int vec_per_row = d / 4;  // float4 vectors
@@ -82,8 +80,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 template <typename OutT>
 static cudaError_t launch_combine_t(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
                              int d, int rows, OutT* out, int grid, cudaStream_t stream) {
-    auto kern = k <= 2 ? combine_kernel<2, 4, OutT> : (k <= 4 ? combine_kernel<4, 2, OutT> : combine_kernel<kMaxTopK, 2, OutT>);
-    return launch_pdl(kern, dim3(grid), dim3(256), 0, stream, yp, dest, w, base, T, k, d, rows, out);
+    auto kern = k <= 2 ? combine_kernel<2, 4, OutT>
+                       : (k <= 4 ? combine_kernel<4, 2, OutT> : combine_kernel<kMaxTopK, 2, OutT>);
+    kern<<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,

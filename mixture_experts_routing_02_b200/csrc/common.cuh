@@ -275,23 +275,6 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t cluster_addr) {
 
 __device__ __forceinline__ void sleep_ns(uint32_t ns) { asm volatile("nanosleep.u32 %0;" ::"r"(ns)); }
 
-// ----------------------------------------------------------------------------- programmatic dependent launch
-//
-// The layer's kernels are launched with programmatic stream serialization, so a kernel may begin
-// (rasterise its CTAs and run a prologue that touches only its own shared / tensor memory) while
-// the previous kernel of the stream is still finishing.  griddep_wait() returns once every
-// earlier kernel of the stream has completed and its memory is visible; a kernel calls it before
-// its first access to global memory.  griddep_launch_dependents() lets the next kernel start
-// launching; a kernel calls it right after its wait, which keeps the chain transitive (a kernel
-// can only start after its predecessor has passed its own wait).  Both are no-ops for a kernel
-// launched without the attribute.
-
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
-__device__ __forceinline__ void griddep_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // ----------------------------------------------------------------------------- misc
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -365,43 +348,23 @@ inline cudaError_t set_max_dynamic_smem(void (*kern)(KArgs...), int bytes) {
     return err;
 }
 
-// Launch `kern` on `stream` with programmatic stream serialization (see griddep_wait), plus an
-// optional cluster shape.  Should the runtime refuse the attribute on this stream, the kernel is
-// launched again without it (the kernels' griddep_wait is then a no-op).
+// Launch `kern` on `stream` with a cluster shape of cluster_x CTAs (1: no cluster attribute).
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                                      unsigned cluster_x, Args&&... args) {
+inline cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             unsigned cluster_x, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    unsigned n = 0;
-    if (cluster_x > 1) {
-        attr[n].id = cudaLaunchAttributeClusterDimension;
-        attr[n].val.clusterDim.x = cluster_x;
-        attr[n].val.clusterDim.y = 1;
-        attr[n].val.clusterDim.z = 1;
-        ++n;
-    }
-    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster_x;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = n + 1;
-    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, args...);
-    if (err != cudaSuccess) {
-        (void)cudaGetLastError();
-        cfg.numAttrs = n;
-        err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-    }
-    return err;
-}
-
-template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                              Args&&... args) {
-    return launch_pdl_cluster(kern, grid, block, smem, stream, 1u, std::forward<Args>(args)...);
+    cfg.numAttrs = cluster_x > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace moe

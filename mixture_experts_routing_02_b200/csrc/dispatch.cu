@@ -527,8 +527,6 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
     __shared__ int s_wcnt[kCountWarps][kMaxExperts];
     __shared__ int warp_sums[kCountWarps];
 
-    griddep_wait();
-    griddep_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = a.E, k = a.k;
     const unsigned lanemask_lt = (1u << lane) - 1u;
@@ -1034,8 +1032,6 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const float* __restri
                                                            int E, int k, int route_flags, float* __restrict__ logits,
                                                            int32_t* __restrict__ ids, float* __restrict__ w,
                                                            float* __restrict__ scores_t) {
-    griddep_wait();
-    griddep_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total)
@@ -1139,11 +1135,9 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
         const int smem = static_cast<int>(sizeof(CountPlanSmem));
         const cudaError_t err = set_max_dynamic_smem(dispatch_count_kernel<true>, smem);
         if (err != cudaSuccess) return err;
-        const cudaError_t e2 = launch_pdl(dispatch_count_kernel<true>, dim3(grid), dim3(kCountThreads), smem, stream, a);
-        if (e2 != cudaSuccess) return e2;
+        dispatch_count_kernel<true><<<grid, kCountThreads, smem, stream>>>(a);
     } else {
-        const cudaError_t e2 = launch_pdl(dispatch_count_kernel<false>, dim3(grid), dim3(kCountThreads), 0, stream, a);
-        if (e2 != cudaSuccess) return e2;
+        dispatch_count_kernel<false><<<grid, kCountThreads, 0, stream>>>(a);
     }
     return cudaGetLastError();
 }
@@ -1202,9 +1196,8 @@ cudaError_t launch_route_logits(const float* part, int n_split, int ldp, size_t 
     if (T == 0) return cudaSuccess;
     int grid = (T + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
-    const cudaError_t err = launch_pdl(route_logits_kernel, dim3(grid), dim3(256), 0, stream, part, n_split, ldp,
-                                       split_stride, bias, T, E, k, route_flags, logits, ids, w, scores_t);
-    if (err != cudaSuccess) return err;
+    route_logits_kernel<<<grid, 256, 0, stream>>>(part, n_split, ldp, split_stride, bias, T, E, k, route_flags, logits,
+                                                  ids, w, scores_t);
     return cudaGetLastError();
 }
 

@@ -185,8 +185,6 @@ __global__ void __launch_bounds__(kEpThreads, 1) ep_dispatch_kernel(const __grid
     __shared__ int s_run[kMaxExperts];  // pairs of each expert before the current chunk
     __shared__ int s_wcnt[kEpWarps][kMaxExperts];
 
-    griddep_wait();
-    griddep_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int i_src = blockIdx.x / a.ctas_per_src;
     const int G = a.ctas_per_src;
@@ -486,8 +484,7 @@ cudaError_t launch_ep_dispatch(const EpDispatchArgs& a0, int num_sms, cudaStream
     const int smem = static_cast<int>(sizeof(EpSmem));
     cudaError_t err = set_max_dynamic_smem(ep_dispatch_kernel, smem);
     if (err != cudaSuccess) return err;
-    err = launch_pdl(ep_dispatch_kernel, dim3(per * a.n_src), dim3(kEpThreads), static_cast<size_t>(smem), stream, a);
-    if (err != cudaSuccess) return err;
+    ep_dispatch_kernel<<<per * a.n_src, kEpThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 

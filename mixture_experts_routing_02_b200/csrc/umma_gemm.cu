@@ -206,10 +206,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (EPI == kEpiSwiglu) tma_prefetch_desc(&tmB1);
     }
     if (warp == 1) tmem_alloc(&tmem_base_sh, kTmemCols);
-    // everything above touched only this CTA's shared and tensor memory; the segment table and
-    // the operands may come from the previous kernel of the stream
-    griddep_wait();
-    griddep_launch_dependents();
     if (warp == 2) build_tile_prefix(tile_prefix, g, kBM, lane);
     tc_fence_before();
     __syncthreads();
@@ -496,8 +492,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(EPI == kEpiSwiglu && rank == 1 ? &tmB1 : &tmB0);
     }
     if (warp == 1) tmem_alloc_pair(&tmem_base_sh, kTmemCols);
-    griddep_wait();
-    griddep_launch_dependents();
     if (warp == 2) build_tile_prefix(tile_prefix, g, 2 * kBM, lane);
     tc_fence_before();
     __syncthreads();
@@ -632,8 +626,7 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     if (smem < kGemmSmemMin) smem = kGemmSmemMin;  // keeps one CTA per SM (all TMEM columns are taken)
     cudaError_t err = set_max_dynamic_smem(kern, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    err = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, a, b0, b1, g);
-    if (err != cudaSuccess) return err;
+    kern<<<grid, kThreads, smem, stream>>>(a, b0, b1, g);
     return cudaGetLastError();
 }
 
@@ -657,7 +650,7 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, cons
     if (smem < kGemmSmemMin) smem = kGemmSmemMin;
     cudaError_t err = set_max_dynamic_smem(kern, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    err = launch_pdl_cluster(kern, dim3(2 * n_pairs), dim3(kThreads), smem, stream, 2u, a, b0, b1, g);
+    err = launch_ex(kern, dim3(2 * n_pairs), dim3(kThreads), smem, stream, 2u, a, b0, b1, g);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
