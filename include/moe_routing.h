@@ -504,8 +504,10 @@ MOE_API moe_status_t moe_combine_expert_choice(const moe_shape_t *shape, const f
  *          logits output); they order each token's further candidates
  * counts receives the plain histogram of topk_ids; seg_offsets the rows each
  * expert ends with (at most C).  ws: moe_workspace_size's dispatch_bytes for
- * this shape (device, 256-byte aligned; no initialisation needed).  Two
- * launches: the rounds (one CTA) and the row copies.
+ * this shape (device, 256-byte aligned; no initialisation needed).  Launches:
+ * each token's candidate order, the rounds (a cooperative grid of up to one CTA
+ * per SM exchanging per-expert counts through a bounded grid barrier; a wait
+ * that runs out sets MOE_DEV_ERR_TIMEOUT in *status) and the row copies.
  */
 MOE_API moe_status_t moe_dispatch_reroute(const moe_shape_t *shape, const moe_bf16_t *x, const int32_t *topk_ids,
                                   const float *logits, int32_t *counts, int32_t *seg_expert,

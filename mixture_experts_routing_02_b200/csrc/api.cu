@@ -308,7 +308,8 @@ moe_status_t segments_or_plan(const Dims& v, int32_t* counts, const int32_t* par
 
 moe_status_t reroute_impl(const Dims& v, const moe_bf16_t* x, const int32_t* ids, const float* logits,
                           int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank,
-                          int32_t* dest, int32_t* src, moe_bf16_t* xp, void* ws, size_t ws_bytes, cudaStream_t st) {
+                          int32_t* dest, int32_t* src, moe_bf16_t* xp, int32_t* status, void* ws, size_t ws_bytes,
+                          cudaStream_t st) {
     if (!x || !ids || !logits || !counts || !seg_expert || !seg_offsets || !seg_first_rank || !dest || !src || !xp)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
@@ -318,7 +319,7 @@ moe_status_t reroute_impl(const Dims& v, const moe_bf16_t* x, const int32_t* ids
     a.ids = ids; a.logits = logits;
     a.T = v.T; a.k = v.k; a.E = v.E; a.capacity = v.C; a.rows = v.rows;
     a.counts = counts; a.seg_expert = seg_expert; a.seg_offsets = seg_offsets; a.seg_first_rank = seg_first_rank;
-    a.dest = dest; a.src = src;
+    a.dest = dest; a.src = src; a.status = status;
     return cuda_status(launch_reroute(a, ws, reinterpret_cast<const __nv_bfloat16*>(x),
                                       reinterpret_cast<__nv_bfloat16*>(xp), v.d, sm_count(), st));
 }
@@ -634,10 +635,9 @@ moe_status_t moe_dispatch_reroute(const moe_shape_t* shape, const moe_bf16_t* x,
     Dims v;
     const moe_status_t s = check_shape(shape, &v);
     if (s != MOE_OK) return s;
-    (void)status;
     if (!v.rr()) return MOE_ERR_INVALID_ARG;
-    return reroute_impl(v, x, topk_ids, logits, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp, ws,
-                        ws_bytes, static_cast<cudaStream_t>(stream));
+    return reroute_impl(v, x, topk_ids, logits, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp, status,
+                        ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* xp, const int32_t* seg_expert,
@@ -873,7 +873,7 @@ moe_status_t moe_layer_fwd(const moe_shape_t* shape, const moe_bf16_t* x, const 
     if (s != MOE_OK) return s;
     if (v.rr()) {
         s = reroute_impl(v, x, w.topk_ids, w.logits, w.counts, w.seg_expert, w.seg_offsets, w.seg_first_rank, w.dest,
-                         w.src, w.xp, w.dispatch_ws, w.dispatch_ws_bytes, st);
+                         w.src, w.xp, status, w.dispatch_ws, w.dispatch_ws_bytes, st);
         if (s != MOE_OK) return s;
         s = gate_up_impl(v, w.xp, w.seg_expert, w.seg_offsets, w_gate, w_up, w.hp, status, st);
         if (s != MOE_OK) return s;

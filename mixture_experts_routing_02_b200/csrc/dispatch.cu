@@ -15,7 +15,8 @@
 //     it, so a tile only waits for tiles already running.  Tiles are taken in order from an
 //     atomic ticket, which guarantees that every tile a CTA waits for is held by a CTA that is
 //     running;
-//   * reroute_kernel (overflow re-routing): one CTA ranks the pairs and then runs the rounds.
+//   * reroute_grid_kernel (overflow re-routing): a cooperative grid runs the capacity rounds, the
+//     CTAs exchanging per-expert counts through a bounded grid barrier.
 // Every wait is bounded.
 //
 // Sources: "Sparsely-Gated MoE 구현 관점에서 살펴보기", section "순전파 과정 ..."
@@ -866,80 +867,171 @@ __global__ void __launch_bounds__(256) candidate_order_kernel(const float* __res
 }
 
 // Capacity with re-routing of the overflow ("로드 밸런싱 손실 ... 용량(capacity)은 별개": a pair
-// over its expert's capacity may go to another candidate).  One CTA of kRerouteThreads threads:
+// over its expert's capacity may go to another candidate):
 //  round 0  each expert keeps its first C pairs in q order (stable ranks over the pair list);
 //  round r  every unplaced pair proposes to its token's next candidate in logit order (the
 //           token's experts are sorted once; its cursor starts after its top-k) among the experts
 //           that had room when the round began; a token's unplaced pairs take consecutive
-//           candidates in j order (one pass per multiplicity); each expert accepts the proposals
-//           in q order while it has room; a pair without a candidate is dropped.
+//           candidates in j order; each expert accepts the proposals in q order while it has room;
+//           a pair without a candidate is dropped.
 // Segment e holds expert e's rows: round 0 first, then round 1, ...; q order inside a round.
 // Writes counts (the plain histogram), the tables, dest and src; X rows are then copied by
-// scatter_rows_kernel.  At most E + 1 rounds: each round either places every proposal or
-// fills an expert (with a skewed router, about one expert fills per round).  The ranks and
-// compactions use warp-owned ranges of the lists (two block barriers per pass).
-__global__ void __launch_bounds__(kRerouteThreads, 1) reroute_kernel(RerouteArgs a) {
+// scatter_rows_kernel.  At most E + 1 rounds: each round either places every proposal or fills
+// an expert (with a skewed router, about one expert fills per round).
+
+// Bounded grid-wide barrier of a cooperative launch: bar[0] counts the CTAs that arrived, bar[1]
+// is the generation.  Thread 0 of each CTA arrives; the last one clears the count and advances the
+// generation; the others wait for it (bounded: a wait that runs out reports MOE_DEV_ERR_TIMEOUT and
+// sets *abort, and an aborted CTA no longer arrives, so the others run out too and every CTA ends).
+// The fences before the arrival and after the wait order each CTA's global writes before the
+// other CTAs' reads that follow the barrier.
+__device__ __forceinline__ bool grid_barrier(uint32_t* bar, int32_t* status, volatile int* abort) {
+    __syncthreads();
+    if (threadIdx.x == 0 && !*abort) {
+        const uint32_t gen = ld_acquire_u32(bar + 1);
+        __threadfence();
+        if (atomicAdd(bar, 1u) == gridDim.x - 1) {
+            st_relaxed_u32(bar, 0u);
+            __threadfence();
+            st_release_u32(bar + 1, gen + 1u);
+        } else {
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_u32(bar + 1) == gen) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    report(status, MOE_DEV_ERR_TIMEOUT);
+                    *abort = 1;
+                    break;
+                }
+                sleep_ns(64);
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    return *abort == 0;
+}
+
+// The rounds above over the whole GPU: a cooperative launch of G CTAs (one
+// per SM at most), every CTA computing the same decisions from the same exchanged counts.  Each
+// pass over a list splits it into G contiguous slices (the pending list at token boundaries, so
+// that one thread walks all of a token's unplaced pairs in j order); a CTA counts its slice's keys
+// per expert, the counts of all CTAs are exchanged through a grid barrier, and each CTA takes the
+// counts of the CTAs before it as the base of its stable ranks -- the same ranks, in q order, as
+// one CTA over the whole list.  Three barriers per round (proposal counts, kept counts, the new
+// list).  Data other CTAs wrote is read through L2 (ld.global.cg).
+__global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(RerouteArgs a) {
     __shared__ int s_cnt[kRerouteThreads / 32][kMaxExperts];
-    __shared__ int s_tot[kMaxExperts];
+    __shared__ int s_loc[kMaxExperts];       // this CTA's counts, then: all CTAs' totals
+    __shared__ int s_base[kMaxExperts];      // counts of the CTAs before this one
     __shared__ int s_assigned[kMaxExperts];
     __shared__ int s_room[kMaxExperts];
     __shared__ int s_wc[33];
-    __shared__ int s_any_open;
+    __shared__ int s_lo, s_hi, s_any_open;
+    __shared__ volatile int s_abort;
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, G = gridDim.x, cta = blockIdx.x;
     const int E = a.E, k = a.k, C = a.capacity;
     const int n = a.T * k;
+    if (tid == 0) s_abort = 0;
+    int xbuf = 0;
 
-    // round 0: stable ranks over all pairs; keep the first C of each expert
+    // counts s_loc[0..len) of every CTA exchanged: s_base = sum over the CTAs before this one,
+    // s_loc = sum over all CTAs.  Two buffers in turn: a CTA overwrites a buffer only after the
+    // barrier of the next exchange, which every CTA passes only after reading it.
+    auto exchange = [&](int len) -> bool {
+        int32_t* buf = a.xchg + static_cast<size_t>(xbuf) * kRerouteMaxCtas * kMaxExperts;
+        xbuf ^= 1;
+        for (int x = tid; x < len; x += blockDim.x) __stcg(buf + static_cast<size_t>(cta) * kMaxExperts + x, s_loc[x]);
+        if (!grid_barrier(a.bar, a.status, &s_abort)) return false;
+        for (int x = tid; x < len; x += blockDim.x) {
+            int before = 0, all = 0;
+            for (int c = 0; c < G; ++c) {
+                const int v = __ldcg(buf + static_cast<size_t>(c) * kMaxExperts + x);
+                all += v;
+                if (c < cta) before += v;
+            }
+            s_base[x] = before;
+            s_loc[x] = all;
+        }
+        __syncthreads();
+        return true;
+    };
     auto id_of = [&](int q) -> int {
         const int e = __ldg(a.ids + q);
         return static_cast<unsigned>(e) < static_cast<unsigned>(E) ? e : -1;
     };
-    for (int q = tid; q < n; q += blockDim.x) { a.fexp[q] = -1; a.fslot[q] = -1; }
+
+    // ---- round 0: stable ranks over all pairs (contiguous slices); keep the first C of each expert
+    const int L0 = (n + G - 1) / G;
+    const int b0 = min(n, cta * L0), e0 = min(n, b0 + L0);
+    for (int q = b0 + tid; q < e0; q += blockDim.x) { __stcg(a.fexp + q, -1); __stcg(a.fslot + q, -1); }
+    for (int t = cta * blockDim.x + tid; t < a.T; t += G * blockDim.x) __stcg(a.cur_pos + t, k);
+    for (int x = tid; x < E; x += blockDim.x) s_loc[x] = 0;
     __syncthreads();
-    warp_range_ranks(n, E, s_cnt, nullptr, s_tot, id_of, [&](int q, int e, int r) {
-        if (r < C) { a.fexp[q] = e; a.fslot[q] = r; }
-    });
-    for (int e = tid; e < E; e += blockDim.x) {
-        a.counts[e] = s_tot[e];
-        s_assigned[e] = min(s_tot[e], C);
+    for (int q = b0 + tid; q < e0; q += blockDim.x) {
+        const int e = id_of(q);
+        if (e >= 0) atomicAdd(&s_loc[e], 1);
     }
-    int n_pend = warp_range_compact(n, s_wc, [&](int q) { return id_of(q) >= 0 && a.fexp[q] < 0; },
-                                    [&](int pos, int q) { a.pend[pos] = q; });
-    for (int t = tid; t < a.T; t += blockDim.x) a.cur_pos[t] = k;  // a token's first k candidates are its top-k
     __syncthreads();
+    if (!exchange(E)) return;
+    if (cta == 0)
+        for (int x = tid; x < E; x += blockDim.x) a.counts[x] = s_loc[x];
+    for (int x = tid; x < E; x += blockDim.x) s_assigned[x] = min(s_loc[x], C);
+    warp_range_ranks(e0 - b0, E, s_cnt, s_base, nullptr, [&](int i) { return id_of(b0 + i); },
+                     [&](int i, int e, int r) {
+                         if (r < C) { __stcg(a.fexp + b0 + i, e); __stcg(a.fslot + b0 + i, r); }
+                     });
+    // the pending list: pairs over capacity, in q order
+    auto over = [&](int q) { return id_of(q) >= 0 && __ldcg(a.fexp + q) < 0; };
+    {
+        int c = 0;
+        for (int q = b0 + tid; q < e0; q += blockDim.x) c += over(q) ? 1 : 0;
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if (tid == 0) s_loc[0] = 0;
+        __syncthreads();
+        if ((tid & 31) == 0) atomicAdd(&s_loc[0], c);
+        __syncthreads();
+    }
+    if (!exchange(1)) return;
+    int n_pend = s_loc[0];
+    const int out0 = s_base[0];
+    warp_range_compact(e0 - b0, s_wc, [&](int i) { return over(b0 + i); },
+                       [&](int pos, int i) { __stcg(a.pend + out0 + pos, b0 + i); });
+    if (!grid_barrier(a.bar, a.status, &s_abort)) return;
 
     int* pend = a.pend;
     int* next = a.pend2;
     for (int round = 1; round <= E + 1 && n_pend > 0; ++round) {
         if (tid == 0) s_any_open = 0;
         __syncthreads();
-        for (int e = tid; e < E; e += blockDim.x) {
-            s_room[e] = C - s_assigned[e];
-            if (s_room[e] > 0) s_any_open = 1;
+        for (int x = tid; x < E; x += blockDim.x) {
+            s_room[x] = C - s_assigned[x];
+            if (s_room[x] > 0) s_any_open = 1;
+        }
+        // this CTA's slice of the pending list, both ends moved up to a token boundary
+        if (tid == 0) {
+            const int L = (n_pend + G - 1) / G;
+            auto aligned = [&](int i) {
+                i = min(i, n_pend);
+                while (i > 0 && i < n_pend && __ldcg(pend + i) / k == __ldcg(pend + i - 1) / k) ++i;
+                return i;
+            };
+            s_lo = aligned(cta * L);
+            s_hi = cta == G - 1 ? n_pend : aligned((cta + 1) * L);
         }
         __syncthreads();
-        if (!s_any_open) break;
-        // proposals, one pass per multiplicity (the m-th unplaced pair of its token; pairs of a
-        // token are adjacent in the list, so the multiplicity is the distance to the first)
-        for (int i = tid; i < n_pend; i += blockDim.x) {
-            const int t = pend[i] / k;
-            int mult = 0;
-            while (mult < i && pend[i - 1 - mult] / k == t) ++mult;
-            next[i] = mult;  // next[] is free until the compaction below
-        }
-        __syncthreads();
-        for (int m = 0; m < k; ++m) {
-            for (int i = tid; i < n_pend; i += blockDim.x) {
-                if (next[i] != m) continue;
-                const int t = pend[i] / k;
-                // the next candidate with room (experts never reopen, so a skipped one stays
-                // skipped); the token's list is read 16 candidates per load (rows 16-byte aligned)
-                const uint8_t* ct = a.cand + static_cast<size_t>(t) * a.cand_stride;
-                int pos = a.cur_pos[t];
+        if (!s_any_open) break;  // the same on every CTA
+        const int lo = s_lo, hi = s_hi;
+        // proposals: the thread at a token's first pending pair walks that token's pairs in j order
+        for (int i = lo + tid; i < hi; i += blockDim.x) {
+            const int t = __ldcg(pend + i) / k;
+            if (i > lo && __ldcg(pend + i - 1) / k == t) continue;
+            const uint8_t* ct = a.cand + static_cast<size_t>(t) * a.cand_stride;
+            int pos = __ldcg(a.cur_pos + t);
+            for (int j = i; j < hi && __ldcg(pend + j) / k == t; ++j) {
                 while (pos < E) {
                     const int base = pos & ~15;
-                    const uint4 c4 = __ldcg(reinterpret_cast<const uint4*>(ct + base));
+                    const uint4 c4 = __ldg(reinterpret_cast<const uint4*>(ct + base));
                     const uint32_t words[4] = {c4.x, c4.y, c4.z, c4.w};
                     bool found = false;
                     for (; pos < base + 16 && pos < E; ++pos) {
@@ -948,29 +1040,56 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_kernel(RerouteArgs
                     }
                     if (found) break;
                 }
-                a.prop[i] = pos < E ? ct[pos] : -1;
-                a.cur_pos[t] = pos < E ? pos + 1 : E;
+                __stcg(a.prop + j, pos < E ? static_cast<int>(ct[pos]) : -1);
+                pos = pos < E ? pos + 1 : E;
             }
+            __stcg(a.cur_pos + t, pos);
+        }
+        __syncthreads();
+        // acceptance in q order: ranks of the proposals over all CTAs
+        for (int x = tid; x < E; x += blockDim.x) s_loc[x] = 0;
+        __syncthreads();
+        for (int i = lo + tid; i < hi; i += blockDim.x) {
+            const int e = __ldcg(a.prop + i);
+            if (e >= 0) atomicAdd(&s_loc[e], 1);
+        }
+        __syncthreads();
+        if (!exchange(E)) return;
+        warp_range_ranks(hi - lo, E, s_cnt, s_base, nullptr, [&](int i) { return __ldcg(a.prop + lo + i); },
+                         [&](int i, int e, int r) {
+                             if (r < s_room[e]) {
+                                 const int q = __ldcg(pend + lo + i);
+                                 __stcg(a.fexp + q, e);
+                                 __stcg(a.fslot + q, s_assigned[e] + r);
+                             }
+                         });
+        for (int x = tid; x < E; x += blockDim.x) s_assigned[x] += min(s_loc[x], s_room[x]);
+        // still pending: a proposal that was not accepted (a pair without a candidate is dropped)
+        auto stays = [&](int i) { return __ldcg(a.prop + i) >= 0 && __ldcg(a.fexp + __ldcg(pend + i)) < 0; };
+        {
+            int c = 0;
+            for (int i = lo + tid; i < hi; i += blockDim.x) c += stays(i) ? 1 : 0;
+            for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+            if (tid == 0) s_loc[0] = 0;
+            __syncthreads();
+            if ((tid & 31) == 0) atomicAdd(&s_loc[0], c);
             __syncthreads();
         }
-        // acceptance in q order, then the rejected stay pending
-        warp_range_ranks(n_pend, E, s_cnt, nullptr, s_tot, [&](int i) { return a.prop[i]; },
-                         [&](int i, int e, int r) {
-                             if (r < s_room[e]) { a.fexp[pend[i]] = e; a.fslot[pend[i]] = s_assigned[e] + r; }
-                         });
-        for (int e = tid; e < E; e += blockDim.x) s_assigned[e] += min(s_tot[e], s_room[e]);
-        n_pend = warp_range_compact(n_pend, s_wc, [&](int i) { return a.prop[i] >= 0 && a.fexp[pend[i]] < 0; },
-                                    [&](int pos, int i) { next[pos] = pend[i]; });
+        if (!exchange(1)) return;
+        n_pend = s_loc[0];
+        const int out = s_base[0];
+        warp_range_compact(hi - lo, s_wc, [&](int i) { return stays(lo + i); },
+                           [&](int pos, int i) { __stcg(next + out + pos, __ldcg(pend + lo + i)); });
+        if (!grid_barrier(a.bar, a.status, &s_abort)) return;
         int* tmp = pend; pend = next; next = tmp;
     }
 
-    // tables and positions
+    // tables (CTA 0) and positions (all CTAs): segment e starts at the exclusive scan of the rows
     __syncthreads();
     if (tid < 32) {
-        // exclusive scan of the experts' rows by one warp
         int carry = 0;
-        for (int e0 = 0; e0 < E; e0 += 32) {
-            const int e = e0 + tid;
+        for (int e0_ = 0; e0_ < E; e0_ += 32) {
+            const int e = e0_ + tid;
             const int v = e < E ? s_assigned[e] : 0;
             int x = v;
 #pragma unroll
@@ -980,20 +1099,22 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_kernel(RerouteArgs
             }
             if (e < E) {
                 s_room[e] = carry + x - v;
-                a.seg_expert[e] = e;
-                a.seg_offsets[e] = carry + x - v;
-                a.seg_first_rank[e] = 0;
+                if (cta == 0) {
+                    a.seg_expert[e] = e;
+                    a.seg_offsets[e] = carry + x - v;
+                    a.seg_first_rank[e] = 0;
+                }
             }
             carry += __shfl_sync(0xffffffffu, x, 31);
         }
-        if (tid == 0) a.seg_offsets[E] = carry;
+        if (tid == 0 && cta == 0) a.seg_offsets[E] = carry;
     }
     __syncthreads();
-    for (int q = tid; q < n; q += blockDim.x) {
-        const int e = a.fexp[q];
+    for (int q = b0 + tid; q < e0; q += blockDim.x) {
+        const int e = __ldcg(a.fexp + q);
         int dst = -1;
         if (e >= 0) {
-            dst = s_room[e] + a.fslot[q];
+            dst = s_room[e] + __ldcg(a.fslot + q);
             if (dst >= a.rows) dst = -1;
         }
         a.dest[q] = dst;
@@ -1146,7 +1267,8 @@ size_t reroute_ws_bytes(int T, int k) {
     auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
     const size_t tk = static_cast<size_t>(T) * k;
     return 256 + 5 * up(tk * sizeof(int32_t)) + up(static_cast<size_t>(T) * sizeof(int32_t)) +
-           up(static_cast<size_t>(T) * kMaxExperts);
+           up(static_cast<size_t>(T) * kMaxExperts) +
+           up(size_t(2) * kRerouteMaxCtas * kMaxExperts * sizeof(int32_t));
 }
 
 cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16* x, __nv_bfloat16* xp, int d,
@@ -1175,8 +1297,22 @@ cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16*
         const cudaError_t e0 = cudaGetLastError();
         if (e0 != cudaSuccess) return e0;
     }
-    reroute_kernel<<<1, kRerouteThreads, 0, stream>>>(a);
-    cudaError_t err = cudaGetLastError();
+    a.xchg = reinterpret_cast<int32_t*>(take(size_t(2) * kRerouteMaxCtas * kMaxExperts * sizeof(int32_t)));
+    a.bar = static_cast<uint32_t*>(ws);  // the first 8 bytes of the workspace header
+    // the rounds over about one CTA per SM (fewer for few pairs), co-resident by a cooperative launch
+    int per_sm = 0;
+    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reroute_grid_kernel, kRerouteThreads, 0);
+    if (err != cudaSuccess) return err;
+    int G = (static_cast<int>(tk) + kRerouteThreads - 1) / kRerouteThreads;
+    const int resident = num_sms * (per_sm > 1 ? per_sm : 1);
+    if (G > resident) G = resident;
+    if (G > kRerouteMaxCtas) G = kRerouteMaxCtas;
+    if (G < 1) G = 1;
+    err = cudaMemsetAsync(a.bar, 0, 2 * sizeof(uint32_t), stream);
+    if (err != cudaSuccess) return err;
+    void* kargs[] = {&a};
+    err = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(reroute_grid_kernel), dim3(G),
+                                      dim3(kRerouteThreads), kargs, 0, stream);
     if (err != cudaSuccess) return err;
     int sgrid = (a.T + 7) / 8;
     if (sgrid > 16 * num_sms) sgrid = 16 * num_sms;

@@ -117,7 +117,8 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
 constexpr int kCountMaxPairs = 1 << 16;
 constexpr int kCountMaxPairsPlan = 1 << 20;  // with a balanced plan the copies dwarf the recounting
 
-// Overflow re-routing (one CTA; T*k <= kCountMaxPairs), then the row copies.
+// Overflow re-routing (the capacity rounds on a cooperative grid; T*k <= kCountMaxPairs), then the
+// row copies.
 constexpr int kRerouteThreads = 1024;
 struct RerouteArgs {
     const int32_t* ids;
@@ -133,7 +134,11 @@ struct RerouteArgs {
     int32_t *pend, *pend2, *prop, *fexp, *fslot, *cur_pos;
     uint8_t* cand;   // [T, cand_stride] each token's experts in candidate order (first E bytes of a row)
     int cand_stride; // E rounded up to 16: every row starts on a 16-byte boundary
+    uint32_t* bar;   // [2] grid barrier (arrivals, generation); arrivals zero on entry
+    int32_t* xchg;   // [2][kRerouteMaxCtas][kMaxExperts] per-CTA counts, two buffers used in turn
+    int32_t* status; // MOE_DEV_ERR_TIMEOUT if a grid barrier wait runs out (nullable)
 };
+constexpr int kRerouteMaxCtas = 256;  // CTAs of the grid-wide rounds (one per SM at most)
 size_t reroute_ws_bytes(int T, int k);
 cudaError_t launch_reroute(const RerouteArgs& a, void* ws, const __nv_bfloat16* x, __nv_bfloat16* xp, int d,
                            int num_sms, cudaStream_t stream);
