@@ -911,14 +911,15 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* bar, int32_t* status, vol
     return *abort == 0;
 }
 
-// The rounds above over the whole GPU: a cooperative launch of G CTAs (one
-// per SM at most), every CTA computing the same decisions from the same exchanged counts.  Each
-// pass over a list splits it into G contiguous slices (the pending list at token boundaries, so
-// that one thread walks all of a token's unplaced pairs in j order); a CTA counts its slice's keys
-// per expert, the counts of all CTAs are exchanged through a grid barrier, and each CTA takes the
-// counts of the CTAs before it as the base of its stable ranks -- the same ranks, in q order, as
-// one CTA over the whole list.  Three barriers per round (proposal counts, kept counts, the new
-// list).  Data other CTAs wrote is read through L2 (ld.global.cg).
+// The rounds above over the whole GPU: a cooperative launch of G CTAs (one per SM at most), every
+// CTA taking the same decisions from the same exchanged counts.  CTA c owns a fixed slice of whole
+// tokens (pairs [c*L, (c+1)*L), L a multiple of k); its unplaced pairs stay in its own slice from
+// round to round, so CTA order is q order, one thread walks a token's unplaced pairs in j order,
+// and a round needs one exchange: the CTAs' per-expert counts of their proposals (round 0: of their
+// pairs), through a bounded grid barrier.  From the exchanged [G, E] counts each CTA takes the
+// counts of the CTAs before it as the base of its stable ranks (the same q-ordered ranks as one CTA
+// over the whole list) and the totals, from which every CTA derives the experts' new row counts and
+// the number of pairs still unplaced.  Data other CTAs wrote is read through L2 (ld.global.cg).
 __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(RerouteArgs a) {
     __shared__ int s_cnt[kRerouteThreads / 32][kMaxExperts];
     __shared__ int s_loc[kMaxExperts];       // this CTA's counts, then: all CTAs' totals
@@ -926,24 +927,26 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
     __shared__ int s_assigned[kMaxExperts];
     __shared__ int s_room[kMaxExperts];
     __shared__ int s_wc[33];
-    __shared__ int s_lo, s_hi, s_any_open;
+    __shared__ int s_n_local, s_any_open;
     __shared__ volatile int s_abort;
 
     const int tid = threadIdx.x, G = gridDim.x, cta = blockIdx.x;
     const int E = a.E, k = a.k, C = a.capacity;
     const int n = a.T * k;
+    const int tokens_per_cta = (a.T + G - 1) / G;
+    const int b0 = min(n, cta * tokens_per_cta * k), e0 = min(n, b0 + tokens_per_cta * k);
     if (tid == 0) s_abort = 0;
     int xbuf = 0;
 
-    // counts s_loc[0..len) of every CTA exchanged: s_base = sum over the CTAs before this one,
-    // s_loc = sum over all CTAs.  Two buffers in turn: a CTA overwrites a buffer only after the
-    // barrier of the next exchange, which every CTA passes only after reading it.
-    auto exchange = [&](int len) -> bool {
+    // this CTA's counts s_loc[0..E) exchanged with every CTA's: s_base = the sum over the CTAs before
+    // this one, s_loc = the sum over all.  Two buffers in turn: a CTA writes a buffer again only after
+    // the barrier of the next exchange, which every CTA passes only after reading it.
+    auto exchange = [&]() -> bool {
         int32_t* buf = a.xchg + static_cast<size_t>(xbuf) * kRerouteMaxCtas * kMaxExperts;
         xbuf ^= 1;
-        for (int x = tid; x < len; x += blockDim.x) __stcg(buf + static_cast<size_t>(cta) * kMaxExperts + x, s_loc[x]);
+        for (int x = tid; x < E; x += blockDim.x) __stcg(buf + static_cast<size_t>(cta) * kMaxExperts + x, s_loc[x]);
         if (!grid_barrier(a.bar, a.status, &s_abort)) return false;
-        for (int x = tid; x < len; x += blockDim.x) {
+        for (int x = tid; x < E; x += blockDim.x) {
             int before = 0, all = 0;
             for (int c = 0; c < G; ++c) {
                 const int v = __ldcg(buf + static_cast<size_t>(c) * kMaxExperts + x);
@@ -960,47 +963,44 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
         const int e = __ldg(a.ids + q);
         return static_cast<unsigned>(e) < static_cast<unsigned>(E) ? e : -1;
     };
+    // pairs of expert e over capacity (room) among those ranked: a block-wide sum over the experts
+    auto sum_over = [&](auto per_expert) -> int {
+        if (tid == 0) s_n_local = 0;
+        __syncthreads();
+        int v = 0;
+        for (int x = tid; x < E; x += blockDim.x) v += per_expert(x);
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if ((tid & 31) == 0 && v) atomicAdd(&s_n_local, v);
+        __syncthreads();
+        return s_n_local;
+    };
 
-    // ---- round 0: stable ranks over all pairs (contiguous slices); keep the first C of each expert
-    const int L0 = (n + G - 1) / G;
-    const int b0 = min(n, cta * L0), e0 = min(n, b0 + L0);
-    for (int q = b0 + tid; q < e0; q += blockDim.x) { __stcg(a.fexp + q, -1); __stcg(a.fslot + q, -1); }
-    for (int t = cta * blockDim.x + tid; t < a.T; t += G * blockDim.x) __stcg(a.cur_pos + t, k);
+    // ---- round 0: stable ranks of the slice's pairs; keep the first C of each expert
+    for (int t = b0 / k + tid; t < e0 / k; t += blockDim.x) __stcg(a.cur_pos + t, k);
     for (int x = tid; x < E; x += blockDim.x) s_loc[x] = 0;
     __syncthreads();
     for (int q = b0 + tid; q < e0; q += blockDim.x) {
+        __stcg(a.fexp + q, -1);
+        __stcg(a.fslot + q, -1);
         const int e = id_of(q);
         if (e >= 0) atomicAdd(&s_loc[e], 1);
     }
     __syncthreads();
-    if (!exchange(E)) return;
+    if (!exchange()) return;
     if (cta == 0)
         for (int x = tid; x < E; x += blockDim.x) a.counts[x] = s_loc[x];
-    for (int x = tid; x < E; x += blockDim.x) s_assigned[x] = min(s_loc[x], C);
     warp_range_ranks(e0 - b0, E, s_cnt, s_base, nullptr, [&](int i) { return id_of(b0 + i); },
                      [&](int i, int e, int r) {
                          if (r < C) { __stcg(a.fexp + b0 + i, e); __stcg(a.fslot + b0 + i, r); }
                      });
-    // the pending list: pairs over capacity, in q order
-    auto over = [&](int q) { return id_of(q) >= 0 && __ldcg(a.fexp + q) < 0; };
-    {
-        int c = 0;
-        for (int q = b0 + tid; q < e0; q += blockDim.x) c += over(q) ? 1 : 0;
-        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-        if (tid == 0) s_loc[0] = 0;
-        __syncthreads();
-        if ((tid & 31) == 0) atomicAdd(&s_loc[0], c);
-        __syncthreads();
-    }
-    if (!exchange(1)) return;
-    int n_pend = s_loc[0];
-    const int out0 = s_base[0];
-    warp_range_compact(e0 - b0, s_wc, [&](int i) { return over(b0 + i); },
-                       [&](int pos, int i) { __stcg(a.pend + out0 + pos, b0 + i); });
-    if (!grid_barrier(a.bar, a.status, &s_abort)) return;
-
+    for (int x = tid; x < E; x += blockDim.x) s_assigned[x] = min(s_loc[x], C);
+    int n_pend = sum_over([&](int x) { return max(0, s_loc[x] - C); });
+    // this CTA's unplaced pairs, in q order, in its own slice of the list
     int* pend = a.pend;
     int* next = a.pend2;
+    int n_local = warp_range_compact(e0 - b0, s_wc, [&](int i) { return id_of(b0 + i) >= 0 && __ldcg(a.fexp + b0 + i) < 0; },
+                                     [&](int pos, int i) { __stcg(pend + b0 + pos, b0 + i); });
+
     for (int round = 1; round <= E + 1 && n_pend > 0; ++round) {
         if (tid == 0) s_any_open = 0;
         __syncthreads();
@@ -1008,27 +1008,15 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
             s_room[x] = C - s_assigned[x];
             if (s_room[x] > 0) s_any_open = 1;
         }
-        // this CTA's slice of the pending list, both ends moved up to a token boundary
-        if (tid == 0) {
-            const int L = (n_pend + G - 1) / G;
-            auto aligned = [&](int i) {
-                i = min(i, n_pend);
-                while (i > 0 && i < n_pend && __ldcg(pend + i) / k == __ldcg(pend + i - 1) / k) ++i;
-                return i;
-            };
-            s_lo = aligned(cta * L);
-            s_hi = cta == G - 1 ? n_pend : aligned((cta + 1) * L);
-        }
         __syncthreads();
         if (!s_any_open) break;  // the same on every CTA
-        const int lo = s_lo, hi = s_hi;
-        // proposals: the thread at a token's first pending pair walks that token's pairs in j order
-        for (int i = lo + tid; i < hi; i += blockDim.x) {
-            const int t = __ldcg(pend + i) / k;
-            if (i > lo && __ldcg(pend + i - 1) / k == t) continue;
+        // proposals: the thread at a token's first unplaced pair walks that token's pairs in j order
+        for (int i = tid; i < n_local; i += blockDim.x) {
+            const int t = __ldcg(pend + b0 + i) / k;
+            if (i > 0 && __ldcg(pend + b0 + i - 1) / k == t) continue;
             const uint8_t* ct = a.cand + static_cast<size_t>(t) * a.cand_stride;
             int pos = __ldcg(a.cur_pos + t);
-            for (int j = i; j < hi && __ldcg(pend + j) / k == t; ++j) {
+            for (int j = i; j < n_local && __ldcg(pend + b0 + j) / k == t; ++j) {
                 while (pos < E) {
                     const int base = pos & ~15;
                     const uint4 c4 = __ldg(reinterpret_cast<const uint4*>(ct + base));
@@ -1040,7 +1028,7 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
                     }
                     if (found) break;
                 }
-                __stcg(a.prop + j, pos < E ? static_cast<int>(ct[pos]) : -1);
+                __stcg(a.prop + b0 + j, pos < E ? static_cast<int>(ct[pos]) : -1);
                 pos = pos < E ? pos + 1 : E;
             }
             __stcg(a.cur_pos + t, pos);
@@ -1049,47 +1037,38 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
         // acceptance in q order: ranks of the proposals over all CTAs
         for (int x = tid; x < E; x += blockDim.x) s_loc[x] = 0;
         __syncthreads();
-        for (int i = lo + tid; i < hi; i += blockDim.x) {
-            const int e = __ldcg(a.prop + i);
+        for (int i = tid; i < n_local; i += blockDim.x) {
+            const int e = __ldcg(a.prop + b0 + i);
             if (e >= 0) atomicAdd(&s_loc[e], 1);
         }
         __syncthreads();
-        if (!exchange(E)) return;
-        warp_range_ranks(hi - lo, E, s_cnt, s_base, nullptr, [&](int i) { return __ldcg(a.prop + lo + i); },
+        if (!exchange()) return;
+        warp_range_ranks(n_local, E, s_cnt, s_base, nullptr, [&](int i) { return __ldcg(a.prop + b0 + i); },
                          [&](int i, int e, int r) {
                              if (r < s_room[e]) {
-                                 const int q = __ldcg(pend + lo + i);
+                                 const int q = __ldcg(pend + b0 + i);
                                  __stcg(a.fexp + q, e);
                                  __stcg(a.fslot + q, s_assigned[e] + r);
                              }
                          });
+        n_pend = sum_over([&](int x) { return max(0, s_loc[x] - s_room[x]); });  // rejected stay unplaced
         for (int x = tid; x < E; x += blockDim.x) s_assigned[x] += min(s_loc[x], s_room[x]);
-        // still pending: a proposal that was not accepted (a pair without a candidate is dropped)
-        auto stays = [&](int i) { return __ldcg(a.prop + i) >= 0 && __ldcg(a.fexp + __ldcg(pend + i)) < 0; };
-        {
-            int c = 0;
-            for (int i = lo + tid; i < hi; i += blockDim.x) c += stays(i) ? 1 : 0;
-            for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-            if (tid == 0) s_loc[0] = 0;
-            __syncthreads();
-            if ((tid & 31) == 0) atomicAdd(&s_loc[0], c);
-            __syncthreads();
-        }
-        if (!exchange(1)) return;
-        n_pend = s_loc[0];
-        const int out = s_base[0];
-        warp_range_compact(hi - lo, s_wc, [&](int i) { return stays(lo + i); },
-                           [&](int pos, int i) { __stcg(next + out + pos, __ldcg(pend + lo + i)); });
-        if (!grid_barrier(a.bar, a.status, &s_abort)) return;
+        // still unplaced: a proposal that was not accepted (a pair without a candidate is dropped)
+        n_local = warp_range_compact(n_local, s_wc,
+                                     [&](int i) {
+                                         return __ldcg(a.prop + b0 + i) >= 0 &&
+                                                __ldcg(a.fexp + __ldcg(pend + b0 + i)) < 0;
+                                     },
+                                     [&](int pos, int i) { __stcg(next + b0 + pos, __ldcg(pend + b0 + i)); });
         int* tmp = pend; pend = next; next = tmp;
     }
 
-    // tables (CTA 0) and positions (all CTAs): segment e starts at the exclusive scan of the rows
+    // tables (CTA 0) and the positions of this CTA's pairs: segment e starts at the scan of the rows
     __syncthreads();
     if (tid < 32) {
         int carry = 0;
-        for (int e0_ = 0; e0_ < E; e0_ += 32) {
-            const int e = e0_ + tid;
+        for (int x0 = 0; x0 < E; x0 += 32) {
+            const int e = x0 + tid;
             const int v = e < E ? s_assigned[e] : 0;
             int x = v;
 #pragma unroll
@@ -1304,6 +1283,7 @@ cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16*
     cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reroute_grid_kernel, kRerouteThreads, 0);
     if (err != cudaSuccess) return err;
     int G = (static_cast<int>(tk) + kRerouteThreads - 1) / kRerouteThreads;
+    if (G > a.T) G = a.T;  // every CTA owns whole tokens
     const int resident = num_sms * (per_sm > 1 ? per_sm : 1);
     if (G > resident) G = resident;
     if (G > kRerouteMaxCtas) G = kRerouteMaxCtas;
