@@ -7,9 +7,9 @@
 // the MoonEP page, section "설치 및 통합" (combine returns the tokens in their
 // original order).
 //
-// One warp per token: each lane owns 16-byte vectors (4 floats) of the row,
-// issues the k gathers of a vector before using any of them, and writes the
-// result with one 16-byte store.  The kernel is HBM-bound: it reads k rows and
+// One warp per token: each lane owns 32-byte vectors (8 floats) of the row (16-byte
+// vectors where the buffers are only 16-byte aligned), issues the k gathers of a vector
+// before using any of them, and writes the result with one store.  The kernel is HBM-bound: it reads k rows and
 // writes one row per token.
 #include "common.cuh"
 #include "kernels.h"
@@ -18,15 +18,59 @@ namespace moe {
 
 namespace {
 
-// KMAX: the largest k this instance handles (registers scale with KMAX * UNROLL);
+// VW floats of a row moved by one instruction: 4 (16-byte vectors) or 8 (32-byte vectors, when
+// Yp, base and an fp32 out are 32-byte aligned: half the memory instructions).
+template <int VW>
+struct FVec {
+    float f[VW];
+};
+
+template <int VW>
+__device__ __forceinline__ FVec<VW> ld_fvec(const float* p) {
+    FVec<VW> r;
+    if constexpr (VW == 8) {
+        const Vec32 v = ld_nc_v8(p);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r.f[i] = __uint_as_float(v.w[i]);
+    } else {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+        r.f[0] = v.x; r.f[1] = v.y; r.f[2] = v.z; r.f[3] = v.w;
+    }
+    return r;
+}
+
+template <int VW>
+__device__ __forceinline__ void st_fvec(float* p, const FVec<VW>& a) {
+    if constexpr (VW == 8) {
+        Vec32 v;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v.w[i] = __float_as_uint(a.f[i]);
+        st_v8(p, v);
+    } else {
+        *reinterpret_cast<float4*>(p) = make_float4(a.f[0], a.f[1], a.f[2], a.f[3]);
+    }
+}
+
+// rounded once to bf16 (round to nearest even): 16- or 8-byte stores
+template <int VW>
+__device__ __forceinline__ void st_fvec(__nv_bfloat16* p, const FVec<VW>& a) {
+    if constexpr (VW == 8) {
+        *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(a.f[0], a.f[1]), pack_bf16x2(a.f[2], a.f[3]),
+                                                  pack_bf16x2(a.f[4], a.f[5]), pack_bf16x2(a.f[6], a.f[7]));
+    } else {
+        *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(a.f[0], a.f[1]), pack_bf16x2(a.f[2], a.f[3]));
+    }
+}
+
+// KMAX: the largest k this instance handles (registers scale with KMAX * UNROLL * VW);
 // UNROLL: row vectors per lane whose gathers are all in flight together; OutT: float or bf16.
-template <int KMAX, int UNROLL, typename OutT>
+template <int KMAX, int UNROLL, int VW, typename OutT>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ dest,
                                                       const float* __restrict__ w, const float* __restrict__ base,
                                                       int T, int k, int d, int rows, OutT* __restrict__ out) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
-    const int vec_per_row = d / 4;  // float4 vectors
+    const int vec_per_row = d / VW;
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
         int mine_d = -1;
         float mine_w = 0.f;
@@ -43,33 +87,37 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
             if (j >= k || dr[j] >= rows) dr[j] = -1;  // dropped, or outside Yp: contributes nothing
         }
         OutT* orow = out + static_cast<size_t>(t) * d;
-        const float4* brow = base ? reinterpret_cast<const float4*>(base + static_cast<size_t>(t) * d) : nullptr;
+        const float* brow = base ? base + static_cast<size_t>(t) * d : nullptr;
         for (int v0 = lane; v0 < vec_per_row; v0 += 32 * UNROLL) {
             // all gathers of UNROLL vectors issued before any is used
-            float4 val[UNROLL][KMAX];
+            FVec<VW> val[UNROLL][KMAX];
 #pragma unroll
             for (int u = 0; u < UNROLL; ++u) {
                 const int v = v0 + 32 * u;
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j)
                     if (dr[j] >= 0 && v < vec_per_row)
-                        val[u][j] = __ldg(reinterpret_cast<const float4*>(yp + static_cast<size_t>(dr[j]) * d) + v);
+                        val[u][j] = ld_fvec<VW>(yp + static_cast<size_t>(dr[j]) * d + static_cast<size_t>(v) * VW);
             }
 #pragma unroll
             for (int u = 0; u < UNROLL; ++u) {
                 const int v = v0 + 32 * u;
                 if (v >= vec_per_row) break;
-                float4 acc = brow ? __ldg(brow + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+                FVec<VW> acc;
+                if (brow) {
+                    acc = ld_fvec<VW>(brow + static_cast<size_t>(v) * VW);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < VW; ++i) acc.f[i] = 0.f;
+                }
 #pragma unroll
                 for (int j = 0; j < KMAX; ++j) {
                     if (dr[j] >= 0) {
-                        acc.x = fmaf(wr[j], val[u][j].x, acc.x);
-                        acc.y = fmaf(wr[j], val[u][j].y, acc.y);
-                        acc.z = fmaf(wr[j], val[u][j].z, acc.z);
-                        acc.w = fmaf(wr[j], val[u][j].w, acc.w);
+#pragma unroll
+                        for (int i = 0; i < VW; ++i) acc.f[i] = fmaf(wr[j], val[u][j].f[i], acc.f[i]);
                     }
                 }
-                store_out4(orow, v, acc);
+                st_fvec<VW>(orow + static_cast<size_t>(v) * VW, acc);
             }
         }
     }
@@ -80,8 +128,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 template <typename OutT>
 static cudaError_t launch_combine_t(const float* yp, const int32_t* dest, const float* w, const float* base, int T, int k,
                              int d, int rows, OutT* out, int grid, cudaStream_t stream) {
-    auto kern = k <= 2 ? combine_kernel<2, 4, OutT>
-                       : (k <= 4 ? combine_kernel<4, 2, OutT> : combine_kernel<kMaxTopK, 2, OutT>);
+    // 32-byte vectors need Yp, base and an fp32 out 32-byte aligned (a bf16 out gets 16-byte stores)
+    const uintptr_t al = reinterpret_cast<uintptr_t>(yp) | reinterpret_cast<uintptr_t>(base) |
+                         (sizeof(OutT) == 4 ? reinterpret_cast<uintptr_t>(out) : 0);
+    auto kern = (al & 31u) == 0
+                    ? (k <= 2 ? combine_kernel<2, 2, 8, OutT>
+                              : (k <= 4 ? combine_kernel<4, 1, 8, OutT> : combine_kernel<kMaxTopK, 1, 8, OutT>))
+                    : (k <= 2 ? combine_kernel<2, 4, 4, OutT>
+                              : (k <= 4 ? combine_kernel<4, 2, 4, OutT> : combine_kernel<kMaxTopK, 2, 4, OutT>));
     kern<<<grid, 256, 0, stream>>>(yp, dest, w, base, T, k, d, rows, out);
     return cudaGetLastError();
 }

@@ -358,15 +358,10 @@ __global__ void __launch_bounds__(kPermuteThreads) rank_kernel(const PermuteArgs
     }
 }
 
-// Copy the row of token t of X to its final slots dj[0..k) (one warp; 16-byte vectors, kCopyUnroll
-// in flight per lane).  Slots outside [0, rows) are skipped.
-__device__ __forceinline__ void copy_row(const __nv_bfloat16* __restrict__ x, int t, const int* dj, int k, int d,
+// Copy the row of token t of X to its final slots dj[0..k) with 16-byte vectors, kCopyUnroll in
+// flight per lane (one warp; for X or Xp not 32-byte aligned).
+__device__ __forceinline__ void copy_row_v4(const __nv_bfloat16* __restrict__ x, int t, const int* dj, int k, int d,
                                          int rows, __nv_bfloat16* __restrict__ xp, int lane) {
-    // a token whose pairs were all dropped is not read at all (dj is the same in every lane)
-    bool any = false;
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) any |= (j < k && dj[j] >= 0 && dj[j] < rows);
-    if (!any) return;
     const int vec_per_row = d / 8;
     const uint4* xs = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
     for (int v = lane; v < vec_per_row; v += 32 * kCopyUnroll) {
@@ -386,6 +381,42 @@ __device__ __forceinline__ void copy_row(const __nv_bfloat16* __restrict__ x, in
     }
 }
 
+// Copy the row of token t of X to its final slots dj[0..k) (one warp).  Slots outside [0, rows)
+// are skipped.  V8 (X and Xp 32-byte aligned; rows are multiples of 128 bytes): each lane moves
+// 32-byte vectors, kCopyUnroll / 2 in flight, half the memory instructions of 16-byte vectors.
+// The kernels that copy rows are instantiated for both and launched by the alignment.
+template <bool V8>
+__device__ __forceinline__ void copy_row(const __nv_bfloat16* __restrict__ x, int t, const int* dj, int k, int d,
+                                         int rows, __nv_bfloat16* __restrict__ xp, int lane) {
+    // a token whose pairs were all dropped is not read at all (dj is the same in every lane)
+    bool any = false;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) any |= (j < k && dj[j] >= 0 && dj[j] < rows);
+    if (!any) return;
+    if (!V8) {
+        copy_row_v4(x, t, dj, k, d, rows, xp, lane);
+        return;
+    }
+    constexpr int U = kCopyUnroll / 2;
+    const int vec_per_row = d / 16;
+    const uint8_t* xs = reinterpret_cast<const uint8_t*>(x + static_cast<size_t>(t) * d);
+    for (int v = lane; v < vec_per_row; v += 32 * U) {
+        Vec32 val[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (v + 32 * u < vec_per_row) val[u] = ld_nc_v8(xs + static_cast<size_t>(v + 32 * u) * 32);
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            if (j < k && dj[j] >= 0 && dj[j] < rows) {
+                uint8_t* dst = reinterpret_cast<uint8_t*>(xp + static_cast<size_t>(dj[j]) * d);
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (v + 32 * u < vec_per_row) st_v8(dst + static_cast<size_t>(v + 32 * u) * 32, val[u]);
+            }
+        }
+    }
+}
+
 // The whole dispatch of the plain (or capacity) layout in one launch, in two phases.
 //  1. Tiles from the ticket, as in rank_kernel: each pair's stable rank inside its expert,
 //     kept in dest for now.  The tile that holds the last ticket knows every expert's total
@@ -397,6 +428,7 @@ __device__ __forceinline__ void copy_row(const __nv_bfloat16* __restrict__ x, in
 // CTA needs to be resident at the same time as another; every wait is bounded.  While
 // waiting, each warp prefetches the rows of X it will copy into L2, so the copy overlaps
 // the ranking.
+template <bool V8>
 __global__ void __launch_bounds__(kPermuteThreads, 4) dispatch_fused_kernel(const PermuteArgs a) {
     __shared__ TileSmem sm;
     __shared__ int warp_sums[8];
@@ -492,7 +524,7 @@ __global__ void __launch_bounds__(kPermuteThreads, 4) dispatch_fused_kernel(cons
         int dj[kMaxTopK];
 #pragma unroll
         for (int j = 0; j < kMaxTopK; ++j) dj[j] = __shfl_sync(0xffffffffu, mine, j);
-        copy_row(a.x, t, dj, k, a.d, a.rows, a.xp, lane);
+        copy_row<V8>(a.x, t, dj, k, a.d, a.rows, a.xp, lane);
     }
 }
 
@@ -517,7 +549,7 @@ struct CountPlanSmem {
     int cbeg[kMaxExperts + 1], cfill[kMaxExperts], cseg[kMaxSegments];
 };
 
-template <bool PLAN>
+template <bool PLAN, bool V8>
 __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const PermuteArgs a) {
     extern __shared__ __align__(16) uint8_t count_dsmem[];
     __shared__ int s_a[kMaxExperts];    // pairs of each expert before the first block
@@ -734,7 +766,7 @@ __global__ void __launch_bounds__(kCountThreads, 1) dispatch_count_kernel(const 
             int dj[kMaxTopK];
 #pragma unroll
             for (int j = 0; j < kMaxTopK; ++j) dj[j] = __shfl_sync(0xffffffffu, mine, j);
-            copy_row(a.x, t, dj, k, a.d, a.rows, a.xp, lane);
+            copy_row<V8>(a.x, t, dj, k, a.d, a.rows, a.xp, lane);
         }
     }
 }
@@ -1105,6 +1137,7 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
 
 // One warp per token: read the token's row of X once (16-byte vectors, 8 in flight per lane)
 // and write it to each of its k final slots.  Pure streaming: no shared memory, no barriers.
+template <bool V8>
 __global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* __restrict__ x,
                                                            const int32_t* __restrict__ dest, int T, int k, int d,
                                                            int rows, __nv_bfloat16* __restrict__ xp) {
@@ -1115,7 +1148,7 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* 
         int dj[kMaxTopK];
 #pragma unroll
         for (int j = 0; j < kMaxTopK; ++j) dj[j] = __shfl_sync(0xffffffffu, mine, j);
-        copy_row(x, t, dj, k, d, rows, xp, lane);
+        copy_row<V8>(x, t, dj, k, d, rows, xp, lane);
     }
 }
 
@@ -1200,6 +1233,11 @@ cudaError_t launch_plan(int32_t* counts, const int32_t* partials, int n_partials
     return cudaGetLastError();
 }
 
+// rows move in 32-byte vectors when X and Xp allow it
+static bool rows_v8(const void* x, const void* xp) {
+    return ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(xp)) & 31u) == 0;
+}
+
 cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, cudaStream_t stream) {
     if (!ws_cleared) {
         cudaError_t err = cudaMemsetAsync(a.ticket, 0, permute_scratch_bytes(a.T, a.k, a.E), stream);
@@ -1212,7 +1250,8 @@ cudaError_t launch_permute(const PermuteArgs& a, bool ws_cleared, int num_sms, c
     if (err != cudaSuccess) return err;
     int sgrid = (a.T + 7) / 8;
     if (sgrid > 16 * num_sms) sgrid = 16 * num_sms;
-    scatter_rows_kernel<<<sgrid, 256, 0, stream>>>(a.x, a.dest, a.T, a.k, a.d, a.rows, a.xp);
+    if (rows_v8(a.x, a.xp)) scatter_rows_kernel<true><<<sgrid, 256, 0, stream>>>(a.x, a.dest, a.T, a.k, a.d, a.rows, a.xp);
+    else scatter_rows_kernel<false><<<sgrid, 256, 0, stream>>>(a.x, a.dest, a.T, a.k, a.d, a.rows, a.xp);
     return cudaGetLastError();
 }
 
@@ -1223,7 +1262,8 @@ cudaError_t launch_dispatch_fused(const PermuteArgs& a, int num_sms, cudaStream_
     int grid = (a.T + kPermuteWarps - 1) / kPermuteWarps;  // one warp per token in the copy phase
     if (grid > 4 * num_sms) grid = 4 * num_sms;
     if (grid < 1) grid = 1;
-    dispatch_fused_kernel<<<grid, kPermuteThreads, 0, stream>>>(a);
+    if (rows_v8(a.x, a.xp)) dispatch_fused_kernel<true><<<grid, kPermuteThreads, 0, stream>>>(a);
+    else dispatch_fused_kernel<false><<<grid, kPermuteThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -1231,13 +1271,16 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
     if (a.T == 0) return cudaSuccess;
     int grid = num_sms;
     if (grid > a.T) grid = a.T;
+    const bool v8 = rows_v8(a.x, a.xp);
     if (a.R > 0) {
         const int smem = static_cast<int>(sizeof(CountPlanSmem));
-        const cudaError_t err = set_max_dynamic_smem(dispatch_count_kernel<true>, smem);
+        auto kern = v8 ? dispatch_count_kernel<true, true> : dispatch_count_kernel<true, false>;
+        const cudaError_t err = set_max_dynamic_smem(kern, smem);
         if (err != cudaSuccess) return err;
-        dispatch_count_kernel<true><<<grid, kCountThreads, smem, stream>>>(a);
+        kern<<<grid, kCountThreads, smem, stream>>>(a);
     } else {
-        dispatch_count_kernel<false><<<grid, kCountThreads, 0, stream>>>(a);
+        auto kern = v8 ? dispatch_count_kernel<false, true> : dispatch_count_kernel<false, false>;
+        kern<<<grid, kCountThreads, 0, stream>>>(a);
     }
     return cudaGetLastError();
 }
@@ -1296,7 +1339,8 @@ cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16*
     if (err != cudaSuccess) return err;
     int sgrid = (a.T + 7) / 8;
     if (sgrid > 16 * num_sms) sgrid = 16 * num_sms;
-    scatter_rows_kernel<<<sgrid, 256, 0, stream>>>(x, a.dest, a.T, a.k, d, a.rows, xp);
+    if (rows_v8(x, xp)) scatter_rows_kernel<true><<<sgrid, 256, 0, stream>>>(x, a.dest, a.T, a.k, d, a.rows, xp);
+    else scatter_rows_kernel<false><<<sgrid, 256, 0, stream>>>(x, a.dest, a.T, a.k, d, a.rows, xp);
     return cudaGetLastError();
 }
 
