@@ -13,6 +13,7 @@
 // writes one row per token.
 #include "common.cuh"
 #include "kernels.h"
+#include "vec.cuh"
 
 namespace moe {
 

@@ -289,31 +289,6 @@ __device__ __forceinline__ void store_out4(__nv_bfloat16* row, int v, float4 a) 
     reinterpret_cast<uint2*>(row)[v] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
 }
 
-// 32-byte vectors (sm_100 and later): one instruction moves 8 words.  Addresses 32-byte aligned.
-struct Vec32 {
-    uint32_t w[8];
-};
-
-// read-only (non-coherent) path, for data no kernel writes while it runs
-__device__ __forceinline__ Vec32 ld_nc_v8(const void* p) {
-    Vec32 v;
-    asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]),
-                   "=r"(v.w[7])
-                 : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ void st_v8(void* p, const Vec32& v) {
-    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]),
-                 "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]), "r"(v.w[7])
-                 : "memory");
-}
-
-__device__ __forceinline__ bool aligned32(const void* a, const void* b) {
-    return ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 31u) == 0;
-}
-
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 

@@ -27,6 +27,7 @@
 // shapes, no host sync) and "설치 및 통합" (tokens_per_expert, cu_seqlens).
 #include "common.cuh"
 #include "kernels.h"
+#include "vec.cuh"
 #include "plan.cuh"
 #include "route.cuh"
 
