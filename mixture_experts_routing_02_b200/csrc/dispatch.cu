@@ -946,21 +946,34 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* bar, int32_t* status, vol
 
 // The rounds above over the whole GPU: a cooperative launch of G CTAs (one per SM at most), every
 // CTA taking the same decisions from the same exchanged counts.  CTA c owns a fixed slice of whole
-// tokens (pairs [c*L, (c+1)*L), L a multiple of k); its unplaced pairs stay in its own slice from
-// round to round, so CTA order is q order, one thread walks a token's unplaced pairs in j order,
-// and a round needs one exchange: the CTAs' per-expert counts of their proposals (round 0: of their
-// pairs), through a bounded grid barrier.  From the exchanged [G, E] counts each CTA takes the
-// counts of the CTAs before it as the base of its stable ranks (the same q-ordered ranks as one CTA
-// over the whole list) and the totals, from which every CTA derives the experts' new row counts and
-// the number of pairs still unplaced.  Data other CTAs wrote is read through L2 (ld.global.cg).
+// tokens (pairs [c*L, (c+1)*L), L a multiple of k, at most kRerouteSliceMax pairs) and keeps all of
+// the slice's state in shared memory: its unplaced pairs in q order, their proposals, each pair's
+// final expert and rank, each token's candidate cursor.  CTA order is q order and one thread walks
+// a token's unplaced pairs in j order, so a round needs one exchange through global memory: the
+// CTAs' per-expert counts of their proposals (round 0: of their pairs), through a bounded grid
+// barrier.  From the exchanged [G, E] counts each CTA takes the counts of the CTAs before it as the
+// base of its stable ranks (the same q-ordered ranks as one CTA over the whole list) and the
+// totals, from which every CTA derives the experts' new row counts and the number of pairs still
+// unplaced.  Exchanged counts are read through L2 (ld.global.cg).
+constexpr int kRerouteSliceMax = kRerouteThreads + kMaxTopK;
+
+size_t reroute_smem_bytes() { return size_t(6) * kRerouteSliceMax * sizeof(int); }
+
 __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(RerouteArgs a) {
+    extern __shared__ __align__(16) int rr_dsmem[];
+    int* s_pend = rr_dsmem;                     // unplaced pairs (offsets in the slice), q order
+    int* s_next = s_pend + kRerouteSliceMax;    // the same after a round
+    int* s_prop = s_next + kRerouteSliceMax;    // each unplaced pair's proposal (-1: no candidate left)
+    int* s_fexp = s_prop + kRerouteSliceMax;    // each pair's final expert (-1: none yet)
+    int* s_fslot = s_fexp + kRerouteSliceMax;   // and its rank in that expert's rows
+    int* s_cur = s_fslot + kRerouteSliceMax;    // each token's next candidate position
     __shared__ int s_cnt[kRerouteThreads / 32][kMaxExperts];
     __shared__ int s_loc[kMaxExperts];       // this CTA's counts, then: all CTAs' totals
     __shared__ int s_base[kMaxExperts];      // counts of the CTAs before this one
     __shared__ int s_assigned[kMaxExperts];
     __shared__ int s_room[kMaxExperts];
     __shared__ int s_wc[33];
-    __shared__ int s_n_local, s_any_open;
+    __shared__ int s_sum, s_any_open;
     __shared__ volatile int s_abort;
 
     const int tid = threadIdx.x, G = gridDim.x, cta = blockIdx.x;
@@ -968,6 +981,7 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
     const int n = a.T * k;
     const int tokens_per_cta = (a.T + G - 1) / G;
     const int b0 = min(n, cta * tokens_per_cta * k), e0 = min(n, b0 + tokens_per_cta * k);
+    const int nl = e0 - b0;  // <= kRerouteSliceMax (checked by the launcher)
     if (tid == 0) s_abort = 0;
     int xbuf = 0;
 
@@ -992,47 +1006,46 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
         __syncthreads();
         return true;
     };
-    auto id_of = [&](int q) -> int {
-        const int e = __ldg(a.ids + q);
+    auto id_of = [&](int i) -> int {  // expert of pair b0 + i (-1: outside [0, E))
+        const int e = __ldg(a.ids + b0 + i);
         return static_cast<unsigned>(e) < static_cast<unsigned>(E) ? e : -1;
     };
-    // pairs of expert e over capacity (room) among those ranked: a block-wide sum over the experts
+    // a block-wide sum over the experts of per_expert(e)
     auto sum_over = [&](auto per_expert) -> int {
-        if (tid == 0) s_n_local = 0;
+        if (tid == 0) s_sum = 0;
         __syncthreads();
         int v = 0;
         for (int x = tid; x < E; x += blockDim.x) v += per_expert(x);
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if ((tid & 31) == 0 && v) atomicAdd(&s_n_local, v);
+        if ((tid & 31) == 0 && v) atomicAdd(&s_sum, v);
         __syncthreads();
-        return s_n_local;
+        return s_sum;
     };
 
     // ---- round 0: stable ranks of the slice's pairs; keep the first C of each expert
-    for (int t = b0 / k + tid; t < e0 / k; t += blockDim.x) __stcg(a.cur_pos + t, k);
+    for (int t = tid; t < nl / k; t += blockDim.x) s_cur[t] = k;
     for (int x = tid; x < E; x += blockDim.x) s_loc[x] = 0;
     __syncthreads();
-    for (int q = b0 + tid; q < e0; q += blockDim.x) {
-        __stcg(a.fexp + q, -1);
-        __stcg(a.fslot + q, -1);
-        const int e = id_of(q);
+    for (int i = tid; i < nl; i += blockDim.x) {
+        s_fexp[i] = -1;
+        s_fslot[i] = -1;
+        const int e = id_of(i);
         if (e >= 0) atomicAdd(&s_loc[e], 1);
     }
     __syncthreads();
     if (!exchange()) return;
     if (cta == 0)
         for (int x = tid; x < E; x += blockDim.x) a.counts[x] = s_loc[x];
-    warp_range_ranks(e0 - b0, E, s_cnt, s_base, nullptr, [&](int i) { return id_of(b0 + i); },
+    warp_range_ranks(nl, E, s_cnt, s_base, nullptr, [&](int i) { return id_of(i); },
                      [&](int i, int e, int r) {
-                         if (r < C) { __stcg(a.fexp + b0 + i, e); __stcg(a.fslot + b0 + i, r); }
+                         if (r < C) { s_fexp[i] = e; s_fslot[i] = r; }
                      });
     for (int x = tid; x < E; x += blockDim.x) s_assigned[x] = min(s_loc[x], C);
-    int n_pend = sum_over([&](int x) { return max(0, s_loc[x] - C); });
-    // this CTA's unplaced pairs, in q order, in its own slice of the list
-    int* pend = a.pend;
-    int* next = a.pend2;
-    int n_local = warp_range_compact(e0 - b0, s_wc, [&](int i) { return id_of(b0 + i) >= 0 && __ldcg(a.fexp + b0 + i) < 0; },
-                                     [&](int pos, int i) { __stcg(pend + b0 + pos, b0 + i); });
+    int n_pend = sum_over([&](int x) { return max(0, s_loc[x] - C); });  // over all CTAs
+    int* pend = s_pend;
+    int* next = s_next;
+    int n_local = warp_range_compact(nl, s_wc, [&](int i) { return id_of(i) >= 0 && s_fexp[i] < 0; },
+                                     [&](int pos, int i) { pend[pos] = i; });
 
     for (int round = 1; round <= E + 1 && n_pend > 0; ++round) {
         if (tid == 0) s_any_open = 0;
@@ -1045,11 +1058,11 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
         if (!s_any_open) break;  // the same on every CTA
         // proposals: the thread at a token's first unplaced pair walks that token's pairs in j order
         for (int i = tid; i < n_local; i += blockDim.x) {
-            const int t = __ldcg(pend + b0 + i) / k;
-            if (i > 0 && __ldcg(pend + b0 + i - 1) / k == t) continue;
-            const uint8_t* ct = a.cand + static_cast<size_t>(t) * a.cand_stride;
-            int pos = __ldcg(a.cur_pos + t);
-            for (int j = i; j < n_local && __ldcg(pend + b0 + j) / k == t; ++j) {
+            const int tl = pend[i] / k;  // token within the slice (b0 is a multiple of k)
+            if (i > 0 && pend[i - 1] / k == tl) continue;
+            const uint8_t* ct = a.cand + static_cast<size_t>(b0 / k + tl) * a.cand_stride;
+            int pos = s_cur[tl];
+            for (int j = i; j < n_local && pend[j] / k == tl; ++j) {
                 while (pos < E) {
                     const int base = pos & ~15;
                     const uint4 c4 = __ldg(reinterpret_cast<const uint4*>(ct + base));
@@ -1061,38 +1074,32 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
                     }
                     if (found) break;
                 }
-                __stcg(a.prop + b0 + j, pos < E ? static_cast<int>(ct[pos]) : -1);
+                s_prop[j] = pos < E ? static_cast<int>(ct[pos]) : -1;
                 pos = pos < E ? pos + 1 : E;
             }
-            __stcg(a.cur_pos + t, pos);
+            s_cur[tl] = pos;
         }
-        __syncthreads();
         // acceptance in q order: ranks of the proposals over all CTAs
         for (int x = tid; x < E; x += blockDim.x) s_loc[x] = 0;
         __syncthreads();
         for (int i = tid; i < n_local; i += blockDim.x) {
-            const int e = __ldcg(a.prop + b0 + i);
+            const int e = s_prop[i];
             if (e >= 0) atomicAdd(&s_loc[e], 1);
         }
         __syncthreads();
         if (!exchange()) return;
-        warp_range_ranks(n_local, E, s_cnt, s_base, nullptr, [&](int i) { return __ldcg(a.prop + b0 + i); },
+        warp_range_ranks(n_local, E, s_cnt, s_base, nullptr, [&](int i) { return s_prop[i]; },
                          [&](int i, int e, int r) {
                              if (r < s_room[e]) {
-                                 const int q = __ldcg(pend + b0 + i);
-                                 __stcg(a.fexp + q, e);
-                                 __stcg(a.fslot + q, s_assigned[e] + r);
+                                 s_fexp[pend[i]] = e;
+                                 s_fslot[pend[i]] = s_assigned[e] + r;
                              }
                          });
         n_pend = sum_over([&](int x) { return max(0, s_loc[x] - s_room[x]); });  // rejected stay unplaced
         for (int x = tid; x < E; x += blockDim.x) s_assigned[x] += min(s_loc[x], s_room[x]);
         // still unplaced: a proposal that was not accepted (a pair without a candidate is dropped)
-        n_local = warp_range_compact(n_local, s_wc,
-                                     [&](int i) {
-                                         return __ldcg(a.prop + b0 + i) >= 0 &&
-                                                __ldcg(a.fexp + __ldcg(pend + b0 + i)) < 0;
-                                     },
-                                     [&](int pos, int i) { __stcg(next + b0 + pos, __ldcg(pend + b0 + i)); });
+        n_local = warp_range_compact(n_local, s_wc, [&](int i) { return s_prop[i] >= 0 && s_fexp[pend[i]] < 0; },
+                                     [&](int pos, int i) { next[pos] = pend[i]; });
         int* tmp = pend; pend = next; next = tmp;
     }
 
@@ -1122,15 +1129,15 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
         if (tid == 0 && cta == 0) a.seg_offsets[E] = carry;
     }
     __syncthreads();
-    for (int q = b0 + tid; q < e0; q += blockDim.x) {
-        const int e = __ldcg(a.fexp + q);
+    for (int i = tid; i < nl; i += blockDim.x) {
+        const int e = s_fexp[i];
         int dst = -1;
         if (e >= 0) {
-            dst = s_room[e] + __ldcg(a.fslot + q);
+            dst = s_room[e] + s_fslot[i];
             if (dst >= a.rows) dst = -1;
         }
-        a.dest[q] = dst;
-        if (dst >= 0) a.src[dst] = q;
+        a.dest[b0 + i] = dst;
+        if (dst >= 0) a.src[dst] = b0 + i;
     }
 }
 
@@ -1289,9 +1296,8 @@ cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_
 size_t reroute_ws_bytes(int T, int k) {
     auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
     const size_t tk = static_cast<size_t>(T) * k;
-    return 256 + 5 * up(tk * sizeof(int32_t)) + up(static_cast<size_t>(T) * sizeof(int32_t)) +
-           up(static_cast<size_t>(T) * kMaxExperts) +
-           up(size_t(2) * kRerouteMaxCtas * kMaxExperts * sizeof(int32_t));
+    (void)tk;
+    return 256 + up(static_cast<size_t>(T) * kMaxExperts) + up(size_t(2) * kRerouteMaxCtas * kMaxExperts * sizeof(int32_t));
 }
 
 cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16* x, __nv_bfloat16* xp, int d,
@@ -1301,12 +1307,6 @@ cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16*
     const size_t tk = static_cast<size_t>(a.T) * a.k;
     uint8_t* p = static_cast<uint8_t*>(ws) + 256;
     auto take = [&](size_t bytes) { uint8_t* r = p; p += (bytes + 255) & ~size_t(255); return r; };
-    a.pend = reinterpret_cast<int32_t*>(take(tk * 4));
-    a.pend2 = reinterpret_cast<int32_t*>(take(tk * 4));
-    a.prop = reinterpret_cast<int32_t*>(take(tk * 4));
-    a.fexp = reinterpret_cast<int32_t*>(take(tk * 4));
-    a.fslot = reinterpret_cast<int32_t*>(take(tk * 4));
-    a.cur_pos = reinterpret_cast<int32_t*>(take(static_cast<size_t>(a.T) * 4));
     a.cand_stride = (a.E + 15) & ~15;  // <= kMaxExperts bytes per token, as reroute_ws_bytes reserves
     a.cand = take(static_cast<size_t>(a.T) * a.cand_stride);
     {
@@ -1323,8 +1323,11 @@ cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16*
     a.xchg = reinterpret_cast<int32_t*>(take(size_t(2) * kRerouteMaxCtas * kMaxExperts * sizeof(int32_t)));
     a.bar = static_cast<uint32_t*>(ws);  // the first 8 bytes of the workspace header
     // the rounds over about one CTA per SM (fewer for few pairs), co-resident by a cooperative launch
+    const int smem = static_cast<int>(reroute_smem_bytes());
+    cudaError_t err = set_max_dynamic_smem(reroute_grid_kernel, smem);
+    if (err != cudaSuccess) return err;
     int per_sm = 0;
-    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reroute_grid_kernel, kRerouteThreads, 0);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reroute_grid_kernel, kRerouteThreads, smem);
     if (err != cudaSuccess) return err;
     int G = (static_cast<int>(tk) + kRerouteThreads - 1) / kRerouteThreads;
     if (G > a.T) G = a.T;  // every CTA owns whole tokens
@@ -1332,11 +1335,14 @@ cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16*
     if (G > resident) G = resident;
     if (G > kRerouteMaxCtas) G = kRerouteMaxCtas;
     if (G < 1) G = 1;
+    // every CTA's slice fits its shared memory (with T*k <= kCountMaxPairs, G is never capped
+    // below T*k / kRerouteThreads, so a slice holds at most kRerouteThreads + k pairs)
+    if (static_cast<int64_t>((a.T + G - 1) / G) * a.k > kRerouteSliceMax) return cudaErrorInvalidValue;
     err = cudaMemsetAsync(a.bar, 0, 2 * sizeof(uint32_t), stream);
     if (err != cudaSuccess) return err;
     void* kargs[] = {&a};
     err = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(reroute_grid_kernel), dim3(G),
-                                      dim3(kRerouteThreads), kargs, 0, stream);
+                                      dim3(kRerouteThreads), kargs, static_cast<size_t>(smem), stream);
     if (err != cudaSuccess) return err;
     int sgrid = (a.T + 7) / 8;
     if (sgrid > 16 * num_sms) sgrid = 16 * num_sms;

@@ -131,7 +131,6 @@ struct RerouteArgs {
     int32_t* dest;
     int32_t* src;
     // scratch, set by launch_reroute from the workspace
-    int32_t *pend, *pend2, *prop, *fexp, *fslot, *cur_pos;
     uint8_t* cand;   // [T, cand_stride] each token's experts in candidate order (first E bytes of a row)
     int cand_stride; // E rounded up to 16: every row starts on a 16-byte boundary
     uint32_t* bar;   // [2] grid barrier (arrivals, generation); arrivals zero on entry
