@@ -995,10 +995,16 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
         if (!grid_barrier(a.bar, a.status, &s_abort)) return false;
         for (int x = tid; x < E; x += blockDim.x) {
             int before = 0, all = 0;
-            for (int c = 0; c < G; ++c) {
-                const int v = __ldcg(buf + static_cast<size_t>(c) * kMaxExperts + x);
-                all += v;
-                if (c < cta) before += v;
+            for (int c0 = 0; c0 < G; c0 += 16) {  // 16 CTAs' counts in flight together
+                int v[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    v[u] = c0 + u < G ? __ldcg(buf + static_cast<size_t>(c0 + u) * kMaxExperts + x) : 0;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    all += v[u];
+                    if (c0 + u < cta) before += v[u];
+                }
             }
             s_base[x] = before;
             s_loc[x] = all;
