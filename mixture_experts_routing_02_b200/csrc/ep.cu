@@ -31,6 +31,7 @@
 // then the tokens).
 #include "common.cuh"
 #include "kernels.h"
+#include "vec.cuh"
 #include "plan.cuh"
 
 namespace moe {
@@ -99,41 +100,83 @@ __global__ void __launch_bounds__(256) ep_plan_kernel(const int32_t* __restrict_
 
 // ------------------------------------------------------------------------------ replica weights
 
-// The copies of this rank's replica slots as one flat list of work items (slot j, matrix m, chunk c
-// of kPrefetchChunk 16-byte vectors), taken by the CTAs in turn; items of a slot whose segment is
-// unused or empty are skipped.  An item copies its chunk of expert e's matrix m from slot e - h*E/R
-// of e's home rank h into this rank's slot E/R + j.  So however few slots are in use, every CTA of
-// the grid streams their bytes.
-constexpr int kPrefetchChunk = 2048;  // 16-byte vectors per work item (32 KB)
+// The copies of this rank's replica slots as one flat list of work items (used slot u, matrix m,
+// chunk c of kPrefetchChunkBytes), taken by the CTAs in turn.  Each CTA first lists the slots in
+// use (a segment with rows) and their experts in shared memory, so an item starts its copy with no
+// dependent load.  An item copies its chunk of expert e's matrix m from slot e - h*E/R of e's home
+// rank h into this rank's slot E/R + j.  So however few slots are in use, every CTA of the grid
+// streams their bytes: 32-byte vectors (16-byte ones when a weight buffer is not 32-byte aligned),
+// four per thread in flight.
+constexpr int kPrefetchChunkBytes = 32768;
 
+template <bool V8>
 __global__ void __launch_bounds__(256) ep_prefetch_kernel(const __grid_constant__ EpPrefetchArgs a) {
+    __shared__ int s_slot[kMaxSegments];    // replica slots in use, in slot order
+    __shared__ int s_expert[kMaxSegments];  // and their experts
+    __shared__ int s_n;
     const int epg = a.E / a.R;
+    if (threadIdx.x < 32) {
+        int n = 0;
+        for (int j0 = 0; j0 < a.B; j0 += 32) {
+            const int j = j0 + static_cast<int>(threadIdx.x);
+            int e = -1;
+            if (j < a.B) {
+                const int sg = epg + j;
+                e = __ldg(a.seg_expert + sg);
+                if (e >= a.E || __ldg(a.seg_offsets + sg + 1) <= __ldg(a.seg_offsets + sg)) e = -1;
+            }
+            const unsigned b = __ballot_sync(0xffffffffu, e >= 0);
+            if (e >= 0) {
+                const int pos = n + __popc(b & ((1u << threadIdx.x) - 1u));
+                s_slot[pos] = j;
+                s_expert[pos] = e;
+            }
+            n += __popc(b);
+        }
+        if (threadIdx.x == 0) s_n = n;
+    }
+    __syncthreads();
+    constexpr int VB = V8 ? 32 : 16;                    // bytes per vector
+    constexpr int kChunk = kPrefetchChunkBytes / VB;    // vectors per work item
     const size_t mat = static_cast<size_t>(a.F) * a.d;  // elements of one expert's matrix
-    const size_t nvec = mat / 8;
-    const int chunks = static_cast<int>((nvec + kPrefetchChunk - 1) / kPrefetchChunk);
-    const int64_t items = static_cast<int64_t>(a.B) * 3 * chunks;
+    const size_t nvec = mat * 2 / VB;                   // F*d is a multiple of 4096
+    const int chunks = static_cast<int>((nvec + kChunk - 1) / kChunk);
+    const int64_t items = static_cast<int64_t>(s_n) * 3 * chunks;
     for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
         const int c = static_cast<int>(it % chunks);
         const int m = static_cast<int>((it / chunks) % 3);
-        const int j = static_cast<int>(it / (3 * static_cast<int64_t>(chunks)));
-        const int sg = epg + j;
-        const int e = __ldg(a.seg_expert + sg);
-        if (e < 0 || e >= a.E || __ldg(a.seg_offsets + sg + 1) <= __ldg(a.seg_offsets + sg)) continue;
+        const int u = static_cast<int>(it / (3 * static_cast<int64_t>(chunks)));
+        const int sg = epg + s_slot[u];
+        const int e = s_expert[u];
         const int h = e / epg;
-        const uint4* src = reinterpret_cast<const uint4*>(a.w[m][h] + static_cast<size_t>(e - h * epg) * mat);
-        uint4* dst = reinterpret_cast<uint4*>(a.w[m][a.rank] + static_cast<size_t>(sg) * mat);
-        const size_t v0 = static_cast<size_t>(c) * kPrefetchChunk;
-        const size_t v1 = v0 + kPrefetchChunk < nvec ? v0 + kPrefetchChunk : nvec;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.w[m][h] + static_cast<size_t>(e - h * epg) * mat);
+        uint8_t* dst = reinterpret_cast<uint8_t*>(a.w[m][a.rank] + static_cast<size_t>(sg) * mat);
+        const size_t v0 = static_cast<size_t>(c) * kChunk;
+        const size_t v1 = v0 + kChunk < nvec ? v0 + kChunk : nvec;
         size_t v = v0 + threadIdx.x;
-        for (; v + 3 * 256 < v1; v += 4 * 256) {
-            const uint4 a0 = __ldg(src + v), a1 = __ldg(src + v + 256);
-            const uint4 a2 = __ldg(src + v + 512), a3 = __ldg(src + v + 768);
-            dst[v] = a0;
-            dst[v + 256] = a1;
-            dst[v + 512] = a2;
-            dst[v + 768] = a3;
+        if constexpr (V8) {
+            for (; v + 3 * 256 < v1; v += 4 * 256) {
+                const Vec32 a0 = ld_nc_v8(src + v * 32), a1 = ld_nc_v8(src + (v + 256) * 32);
+                const Vec32 a2 = ld_nc_v8(src + (v + 512) * 32), a3 = ld_nc_v8(src + (v + 768) * 32);
+                st_v8(dst + v * 32, a0);
+                st_v8(dst + (v + 256) * 32, a1);
+                st_v8(dst + (v + 512) * 32, a2);
+                st_v8(dst + (v + 768) * 32, a3);
+            }
+            for (; v < v1; v += 256) st_v8(dst + v * 32, ld_nc_v8(src + v * 32));
+        } else {
+            const uint4* s4 = reinterpret_cast<const uint4*>(src);
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+            for (; v + 3 * 256 < v1; v += 4 * 256) {
+                const uint4 a0 = __ldg(s4 + v), a1 = __ldg(s4 + v + 256);
+                const uint4 a2 = __ldg(s4 + v + 512), a3 = __ldg(s4 + v + 768);
+                d4[v] = a0;
+                d4[v + 256] = a1;
+                d4[v + 512] = a2;
+                d4[v + 768] = a3;
+            }
+            for (; v < v1; v += 256) d4[v] = __ldg(s4 + v);
         }
-        for (; v < v1; v += 256) dst[v] = __ldg(src + v);
     }
 }
 
@@ -469,7 +512,12 @@ cudaError_t launch_ep_plan(const int32_t* counts_all, int R, int S, int k, int E
 
 cudaError_t launch_ep_prefetch(const EpPrefetchArgs& a, int num_sms, cudaStream_t stream) {
     if (a.B == 0) return cudaSuccess;
-    ep_prefetch_kernel<<<4 * num_sms, 256, 0, stream>>>(a);  // four 256-thread CTAs per SM
+    bool v8 = true;
+    for (int m = 0; m < 3; ++m)
+        for (int r = 0; r < a.R; ++r) v8 = v8 && (reinterpret_cast<uintptr_t>(a.w[m][r]) & 31u) == 0;
+    // four 256-thread CTAs per SM
+    if (v8) ep_prefetch_kernel<true><<<4 * num_sms, 256, 0, stream>>>(a);
+    else ep_prefetch_kernel<false><<<4 * num_sms, 256, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
