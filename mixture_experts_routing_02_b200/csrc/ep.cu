@@ -182,28 +182,51 @@ __global__ void __launch_bounds__(256) ep_prefetch_kernel(const __grid_constant_
 
 // ------------------------------------------------------------------------------ dispatch
 
-// Copy token row xs (d bf16) to the k destinations dst[0..k) (null: none), one warp, 16-byte
-// vectors, kEpCopyUnroll in flight per lane.
+// Copy token row xs (d bf16) to the k destinations dst[0..k) (null: none), one warp: V8 (every
+// row 32-byte aligned) 32-byte vectors, kEpCopyUnroll / 2 in flight per lane, else 16-byte
+// vectors, kEpCopyUnroll in flight.
+template <bool V8>
 __device__ __forceinline__ void ep_copy_row(const __nv_bfloat16* __restrict__ xs, __nv_bfloat16* const* dst, int k,
                                             int d, int lane) {
     bool any = false;
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) any |= (j < k && dst[j] != nullptr);
     if (!any) return;
-    const int vec_per_row = d / 8;
-    const uint4* s = reinterpret_cast<const uint4*>(xs);
-    for (int v = lane; v < vec_per_row; v += 32 * kEpCopyUnroll) {
-        uint4 val[kEpCopyUnroll];
+    if constexpr (V8) {
+        constexpr int U = kEpCopyUnroll / 2;
+        const int vec_per_row = d / 16;
+        const uint8_t* s = reinterpret_cast<const uint8_t*>(xs);
+        for (int v = lane; v < vec_per_row; v += 32 * U) {
+            Vec32 val[U];
 #pragma unroll
-        for (int u = 0; u < kEpCopyUnroll; ++u)
-            if (v + 32 * u < vec_per_row) val[u] = __ldg(s + v + 32 * u);
+            for (int u = 0; u < U; ++u)
+                if (v + 32 * u < vec_per_row) val[u] = ld_nc_v8(s + static_cast<size_t>(v + 32 * u) * 32);
 #pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) {
-            if (j < k && dst[j] != nullptr) {
-                uint4* o = reinterpret_cast<uint4*>(dst[j]);
+            for (int j = 0; j < kMaxTopK; ++j) {
+                if (j < k && dst[j] != nullptr) {
+                    uint8_t* o = reinterpret_cast<uint8_t*>(dst[j]);
 #pragma unroll
-                for (int u = 0; u < kEpCopyUnroll; ++u)
-                    if (v + 32 * u < vec_per_row) o[v + 32 * u] = val[u];
+                    for (int u = 0; u < U; ++u)
+                        if (v + 32 * u < vec_per_row) st_v8(o + static_cast<size_t>(v + 32 * u) * 32, val[u]);
+                }
+            }
+        }
+    } else {
+        const int vec_per_row = d / 8;
+        const uint4* s = reinterpret_cast<const uint4*>(xs);
+        for (int v = lane; v < vec_per_row; v += 32 * kEpCopyUnroll) {
+            uint4 val[kEpCopyUnroll];
+#pragma unroll
+            for (int u = 0; u < kEpCopyUnroll; ++u)
+                if (v + 32 * u < vec_per_row) val[u] = __ldg(s + v + 32 * u);
+#pragma unroll
+            for (int j = 0; j < kMaxTopK; ++j) {
+                if (j < k && dst[j] != nullptr) {
+                    uint4* o = reinterpret_cast<uint4*>(dst[j]);
+#pragma unroll
+                    for (int u = 0; u < kEpCopyUnroll; ++u)
+                        if (v + 32 * u < vec_per_row) o[v + 32 * u] = val[u];
+                }
             }
         }
     }
@@ -219,6 +242,7 @@ __device__ __forceinline__ void ep_copy_row(const __nv_bfloat16* __restrict__ xs
 //     owner and row there; writes dest (owner * S*k + row) and the owner's src (global pair
 //     index, a peer store);
 //  4. stores each token's row into its k slots on their owners (peer stores).
+template <bool V8>
 __global__ void __launch_bounds__(kEpThreads, 1) ep_dispatch_kernel(const __grid_constant__ EpDispatchArgs a) {
     extern __shared__ __align__(16) uint8_t ep_dsmem[];
     EpSmem& ps = *reinterpret_cast<EpSmem*>(ep_dsmem);
@@ -384,7 +408,7 @@ __global__ void __launch_bounds__(kEpThreads, 1) ep_dispatch_kernel(const __grid
             for (int j = 0; j < kMaxTopK; ++j)
                 dj[j] = reinterpret_cast<__nv_bfloat16*>(
                     __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(mine), j));
-            ep_copy_row(x + static_cast<size_t>(t) * a.d, dj, k, a.d, lane);
+            ep_copy_row<V8>(x + static_cast<size_t>(t) * a.d, dj, k, a.d, lane);
         }
     }
     // the stores above may go to other GPUs: make them visible system-wide before the kernel ends,
@@ -529,10 +553,15 @@ cudaError_t launch_ep_dispatch(const EpDispatchArgs& a0, int num_sms, cudaStream
     if (per > a.S) per = a.S;
     if (per < 1) per = 1;
     a.ctas_per_src = per;
+    // 32-byte row copies when every source's X and every owner's Xp is 32-byte aligned
+    uintptr_t al = 0;
+    for (int i = 0; i < a.n_src; ++i) al |= reinterpret_cast<uintptr_t>(a.x[i]);
+    for (int r = 0; r < a.R; ++r) al |= reinterpret_cast<uintptr_t>(a.xp[r]);
+    auto kern = (al & 31u) == 0 ? ep_dispatch_kernel<true> : ep_dispatch_kernel<false>;
     const int smem = static_cast<int>(sizeof(EpSmem));
-    cudaError_t err = set_max_dynamic_smem(ep_dispatch_kernel, smem);
+    cudaError_t err = set_max_dynamic_smem(kern, smem);
     if (err != cudaSuccess) return err;
-    ep_dispatch_kernel<<<per * a.n_src, kEpThreads, smem, stream>>>(a);
+    kern<<<per * a.n_src, kEpThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 

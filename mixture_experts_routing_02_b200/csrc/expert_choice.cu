@@ -8,13 +8,15 @@
 //     number of kept tokens before it, from one block-wide scan per 1024 tokens.  Equal
 //     scores at the threshold go to the lower token ids.  It also writes the segment table
 //     (segment e = expert e, C' rows) and the [T, E] map from (token, expert) to row.
-//   * ec_gather_kernel: Xp[r] = X[src[r]], one warp per row, 16-byte vectors.
+//   * ec_gather_kernel: Xp[r] = X[src[r]], one warp per row, 32-byte vectors (16-byte ones for
+//     buffers that are only 16-byte aligned).
 //   * ec_combine_kernel: out[t] = base[t] + sum of row_w[r] * Yp[r] over the rows r of
-//     token t in ascending expert order, one warp per token; out in fp32 or bf16.
+//     token t in ascending expert order, one warp per (token, column part); out in fp32 or bf16.
 // The gather and the combine are HBM-bound; the selection reads the E x T scores four
 // times, from L2.
 #include "common.cuh"
 #include "kernels.h"
+#include "vec.cuh"
 
 namespace moe {
 
@@ -162,49 +164,112 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
 
 constexpr int kGatherUnroll = 8;
 
+// V8 (X and Xp 32-byte aligned): 32-byte vectors, kGatherUnroll / 2 in flight per lane; else
+// 16-byte vectors, kGatherUnroll in flight.
+template <bool V8>
 __global__ void __launch_bounds__(256) ec_gather_kernel(const __nv_bfloat16* __restrict__ x,
                                                         const int32_t* __restrict__ src, int rows, int T, int d,
                                                         __nv_bfloat16* __restrict__ xp) {
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
-    const int vec_per_row = d / 8;
     for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps_total) {
         const int t = __ldg(src + r);
         if (t < 0 || t >= T) continue;
-        const uint4* xs = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
-        uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(r) * d);
-        for (int v = lane; v < vec_per_row; v += 32 * kGatherUnroll) {
-            uint4 val[kGatherUnroll];
+        if constexpr (V8) {
+            constexpr int U = kGatherUnroll / 2;
+            const int vec_per_row = d / 16;
+            const uint8_t* xs = reinterpret_cast<const uint8_t*>(x + static_cast<size_t>(t) * d);
+            uint8_t* dst = reinterpret_cast<uint8_t*>(xp + static_cast<size_t>(r) * d);
+            for (int v = lane; v < vec_per_row; v += 32 * U) {
+                Vec32 val[U];
 #pragma unroll
-            for (int u = 0; u < kGatherUnroll; ++u)
-                if (v + 32 * u < vec_per_row) val[u] = __ldg(xs + v + 32 * u);
+                for (int u = 0; u < U; ++u)
+                    if (v + 32 * u < vec_per_row) val[u] = ld_nc_v8(xs + static_cast<size_t>(v + 32 * u) * 32);
 #pragma unroll
-            for (int u = 0; u < kGatherUnroll; ++u)
-                if (v + 32 * u < vec_per_row) dst[v + 32 * u] = val[u];
+                for (int u = 0; u < U; ++u)
+                    if (v + 32 * u < vec_per_row) st_v8(dst + static_cast<size_t>(v + 32 * u) * 32, val[u]);
+            }
+        } else {
+            const int vec_per_row = d / 8;
+            const uint4* xs = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
+            uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(r) * d);
+            for (int v = lane; v < vec_per_row; v += 32 * kGatherUnroll) {
+                uint4 val[kGatherUnroll];
+#pragma unroll
+                for (int u = 0; u < kGatherUnroll; ++u)
+                    if (v + 32 * u < vec_per_row) val[u] = __ldg(xs + v + 32 * u);
+#pragma unroll
+                for (int u = 0; u < kGatherUnroll; ++u)
+                    if (v + 32 * u < vec_per_row) dst[v + 32 * u] = val[u];
+            }
         }
     }
 }
 
 constexpr int kCombineWarps = 8;
-constexpr int kCombineUnroll = 4;
+constexpr int kCombineUnroll = 2;   // row vectors per lane whose gathers are in flight together
+constexpr int kCombineMaxParts = 4; // column parts per token (work items: token x part)
 
-__device__ __forceinline__ void fma4(float4& acc, float w, const float4& y) {
-    acc.x = fmaf(w, y.x, acc.x);
-    acc.y = fmaf(w, y.y, acc.y);
-    acc.z = fmaf(w, y.z, acc.z);
-    acc.w = fmaf(w, y.w, acc.w);
+// VW floats per vector: 8 (32-byte loads and stores; Yp, base and an fp32 out 32-byte aligned) or 4.
+template <int VW>
+struct EcVec {
+    float f[VW];
+};
+
+template <int VW>
+__device__ __forceinline__ EcVec<VW> ec_ld(const float* p) {
+    EcVec<VW> r;
+    if constexpr (VW == 8) {
+        const Vec32 v = ld_nc_v8(p);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r.f[i] = __uint_as_float(v.w[i]);
+    } else {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+        r.f[0] = v.x; r.f[1] = v.y; r.f[2] = v.z; r.f[3] = v.w;
+    }
+    return r;
 }
 
-template <typename OutT>
+template <int VW>
+__device__ __forceinline__ void ec_st(float* p, const EcVec<VW>& a) {
+    if constexpr (VW == 8) {
+        Vec32 v;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v.w[i] = __float_as_uint(a.f[i]);
+        st_v8(p, v);
+    } else {
+        *reinterpret_cast<float4*>(p) = make_float4(a.f[0], a.f[1], a.f[2], a.f[3]);
+    }
+}
+
+template <int VW>
+__device__ __forceinline__ void ec_st(__nv_bfloat16* p, const EcVec<VW>& a) {
+    if constexpr (VW == 8) {
+        *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(a.f[0], a.f[1]), pack_bf16x2(a.f[2], a.f[3]),
+                                                  pack_bf16x2(a.f[4], a.f[5]), pack_bf16x2(a.f[6], a.f[7]));
+    } else {
+        *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(a.f[0], a.f[1]), pack_bf16x2(a.f[2], a.f[3]));
+    }
+}
+
+// One warp per work item (token t, column part p of `parts`): the token's (row, weight) pairs
+// in ascending expert order go to shared memory, then the part's vectors are accumulated two
+// rows at a time with all their gathers in flight.  Cutting each row into parts gives the warps
+// several small items each, so the last wave is short.
+template <int VW, typename OutT>
 __global__ void __launch_bounds__(kCombineWarps * 32)
     ec_combine_kernel(const float* __restrict__ yp, const int32_t* __restrict__ emap, const float* __restrict__ row_w,
-                      const float* __restrict__ base, int T, int E, int d, int rows, OutT* __restrict__ out) {
+                      const float* __restrict__ base, int T, int E, int d, int rows, int parts,
+                      OutT* __restrict__ out) {
     __shared__ int2 picks[kCombineWarps][kMaxExperts];  // (row, weight bits) of the current token
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int warps_total = gridDim.x * kCombineWarps;
-    const int vec_per_row = d / 4;
+    const int vec_per_row = d / VW;
+    const int vec_per_part = (vec_per_row + parts - 1) / parts;
     int2* my = picks[warp];
-    for (int t = blockIdx.x * kCombineWarps + warp; t < T; t += warps_total) {
+    const int64_t items = static_cast<int64_t>(T) * parts;
+    for (int64_t item = static_cast<int64_t>(blockIdx.x) * kCombineWarps + warp; item < items; item += warps_total) {
+        const int t = static_cast<int>(item / parts), part = static_cast<int>(item % parts);
         int n = 0;
         for (int c = 0; c < E; c += 32) {
             const int e = c + lane;
@@ -219,32 +284,41 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
         }
         __syncwarp();
         OutT* orow = out + static_cast<size_t>(t) * d;
-        const float4* brow = base ? reinterpret_cast<const float4*>(base + static_cast<size_t>(t) * d) : nullptr;
-        for (int v0 = lane; v0 < vec_per_row; v0 += 32 * kCombineUnroll) {
-            float4 acc[kCombineUnroll];
+        const float* brow = base ? base + static_cast<size_t>(t) * d : nullptr;
+        const int vb = part * vec_per_part;
+        const int ve = min(vec_per_row, vb + vec_per_part);
+        for (int v0 = vb + lane; v0 < ve; v0 += 32 * kCombineUnroll) {
+            EcVec<VW> acc[kCombineUnroll];
 #pragma unroll
             for (int u = 0; u < kCombineUnroll; ++u) {
                 const int v = v0 + 32 * u;
-                acc[u] = (brow && v < vec_per_row) ? __ldg(brow + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+                if (brow && v < ve) {
+                    acc[u] = ec_ld<VW>(brow + static_cast<size_t>(v) * VW);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < VW; ++i) acc[u].f[i] = 0.f;
+                }
             }
             int p = 0;
             // two rows at a time: all 2 x kCombineUnroll gathers in flight before any is used
             for (; p + 1 < n; p += 2) {
                 const int2 a = my[p], b = my[p + 1];
-                float4 ya[kCombineUnroll], yb[kCombineUnroll];
+                EcVec<VW> ya[kCombineUnroll], yb[kCombineUnroll];
 #pragma unroll
                 for (int u = 0; u < kCombineUnroll; ++u) {
                     const int v = v0 + 32 * u;
-                    if (v < vec_per_row) {
-                        ya[u] = __ldg(reinterpret_cast<const float4*>(yp + static_cast<size_t>(a.x) * d) + v);
-                        yb[u] = __ldg(reinterpret_cast<const float4*>(yp + static_cast<size_t>(b.x) * d) + v);
+                    if (v < ve) {
+                        ya[u] = ec_ld<VW>(yp + static_cast<size_t>(a.x) * d + static_cast<size_t>(v) * VW);
+                        yb[u] = ec_ld<VW>(yp + static_cast<size_t>(b.x) * d + static_cast<size_t>(v) * VW);
                     }
                 }
 #pragma unroll
                 for (int u = 0; u < kCombineUnroll; ++u) {
-                    if (v0 + 32 * u < vec_per_row) {
-                        fma4(acc[u], __int_as_float(a.y), ya[u]);
-                        fma4(acc[u], __int_as_float(b.y), yb[u]);
+                    if (v0 + 32 * u < ve) {
+#pragma unroll
+                        for (int i = 0; i < VW; ++i) acc[u].f[i] = fmaf(__int_as_float(a.y), ya[u].f[i], acc[u].f[i]);
+#pragma unroll
+                        for (int i = 0; i < VW; ++i) acc[u].f[i] = fmaf(__int_as_float(b.y), yb[u].f[i], acc[u].f[i]);
                     }
                 }
             }
@@ -253,14 +327,16 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 #pragma unroll
                 for (int u = 0; u < kCombineUnroll; ++u) {
                     const int v = v0 + 32 * u;
-                    if (v < vec_per_row)
-                        fma4(acc[u], __int_as_float(a.y),
-                             __ldg(reinterpret_cast<const float4*>(yp + static_cast<size_t>(a.x) * d) + v));
+                    if (v < ve) {
+                        const EcVec<VW> y = ec_ld<VW>(yp + static_cast<size_t>(a.x) * d + static_cast<size_t>(v) * VW);
+#pragma unroll
+                        for (int i = 0; i < VW; ++i) acc[u].f[i] = fmaf(__int_as_float(a.y), y.f[i], acc[u].f[i]);
+                    }
                 }
             }
 #pragma unroll
             for (int u = 0; u < kCombineUnroll; ++u)
-                if (v0 + 32 * u < vec_per_row) store_out4(orow, v0 + 32 * u, acc[u]);
+                if (v0 + 32 * u < ve) ec_st<VW>(orow + static_cast<size_t>(v0 + 32 * u) * VW, acc[u]);
         }
         __syncwarp();
     }
@@ -291,21 +367,38 @@ cudaError_t launch_ec_gather(const __nv_bfloat16* x, const int32_t* src, int row
     if (rows == 0) return cudaSuccess;
     int grid = (rows + 7) / 8;
     if (grid > 8 * num_sms) grid = 8 * num_sms;
-    ec_gather_kernel<<<grid, 256, 0, stream>>>(x, src, rows, T, d, xp);
+    if (((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(xp)) & 31u) == 0)
+        ec_gather_kernel<true><<<grid, 256, 0, stream>>>(x, src, rows, T, d, xp);
+    else
+        ec_gather_kernel<false><<<grid, 256, 0, stream>>>(x, src, rows, T, d, xp);
     return cudaGetLastError();
 }
 
 cudaError_t launch_ec_combine(const float* yp, const int32_t* emap, const float* row_w, const float* base, int T,
                               int E, int d, int rows, void* out, bool out_bf16, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    int grid = (T + kCombineWarps - 1) / kCombineWarps;
+    // 32-byte vectors need Yp, base and an fp32 out 32-byte aligned (a bf16 out gets 16-byte stores)
+    const uintptr_t al = reinterpret_cast<uintptr_t>(yp) | reinterpret_cast<uintptr_t>(base) |
+                         (out_bf16 ? 0 : reinterpret_cast<uintptr_t>(out));
+    const bool v8 = (al & 31u) == 0;
+    // parts of at least one full pass of the warp (32 lanes x kCombineUnroll vectors)
+    const int vw = v8 ? 8 : 4;
+    int parts = d / (32 * kCombineUnroll * vw);
+    if (parts > kCombineMaxParts) parts = kCombineMaxParts;
+    if (parts < 1) parts = 1;
+    const int64_t items = static_cast<int64_t>(T) * parts;
+    int grid = static_cast<int>((items + kCombineWarps - 1) / kCombineWarps);
     if (grid > 8 * num_sms) grid = 8 * num_sms;
-    if (out_bf16)
-        ec_combine_kernel<__nv_bfloat16><<<grid, kCombineWarps * 32, 0, stream>>>(
-            yp, emap, row_w, base, T, E, d, rows, static_cast<__nv_bfloat16*>(out));
-    else
-        ec_combine_kernel<float><<<grid, kCombineWarps * 32, 0, stream>>>(yp, emap, row_w, base, T, E, d, rows,
-                                                                          static_cast<float*>(out));
+    const dim3 block(kCombineWarps * 32);
+    if (out_bf16) {
+        auto* o = static_cast<__nv_bfloat16*>(out);
+        if (v8) ec_combine_kernel<8, __nv_bfloat16><<<grid, block, 0, stream>>>(yp, emap, row_w, base, T, E, d, rows, parts, o);
+        else ec_combine_kernel<4, __nv_bfloat16><<<grid, block, 0, stream>>>(yp, emap, row_w, base, T, E, d, rows, parts, o);
+    } else {
+        auto* o = static_cast<float*>(out);
+        if (v8) ec_combine_kernel<8, float><<<grid, block, 0, stream>>>(yp, emap, row_w, base, T, E, d, rows, parts, o);
+        else ec_combine_kernel<4, float><<<grid, block, 0, stream>>>(yp, emap, row_w, base, T, E, d, rows, parts, o);
+    }
     return cudaGetLastError();
 }
 

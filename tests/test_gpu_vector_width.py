@@ -1,6 +1,7 @@
 """Row copies and gathers move 32-byte vectors when their buffers are 32-byte aligned and 16-byte
 vectors otherwise: each copying kernel (count, look-back and scatter dispatch, re-routing's row
-copies, combine, replica-weight prefetch) is built for both widths and launched by the alignment.
+copies, combine, expert-choice gather and combine, replica-weight prefetch, expert-parallel
+dispatch) is built for both widths and launched by the alignment.
 The other GPU tests allocate through torch (256-byte aligned) and so run the 32-byte kernels; here
 the same calls run on buffers that start 16 bytes past a 32-byte boundary, against the oracle
 (placement bit for bit, the combine to fp32 accumulation order)."""
@@ -32,11 +33,13 @@ def buf(shape, dtype, misalign: bool):
 
 DISPATCH = [
     # (name, T, d, E, k, capacity, R, B): the count kernel, with a capacity, the look-back kernel
-    # (T*k > 65536), the count kernel with a plan of more than 16 groups, and the multi-launch
-    # plan path (more than 2^20 pairs, more than 16 groups: rank + scatter kernels)
+    # (T*k > 65536), the grouped (expert-parallel) dispatch of a plan of at most 16 groups, the
+    # count kernel with a plan of more than 16 groups, and the multi-launch plan path (more than
+    # 2^20 pairs, more than 16 groups: rank + scatter kernels)
     ("count", 300, 192, 6, 2, 0, 0, 0),
     ("capacity", 500, 128, 16, 2, 40, 0, 0),
     ("lookback", 9000, 64, 64, 8, 0, 0, 0),
+    ("plan-8-groups", 4096, 128, 64, 4, 0, 8, 8),
     ("plan-32-groups", 2048, 64, 64, 4, 0, 32, 8),
     ("plan-multi-launch", 140032, 64, 32, 8, 0, 32, 4),
 ]
@@ -164,3 +167,50 @@ def test_replica_prefetch_vector_widths(cuda_ok, misalign):
         assert torch.equal(ws[m][0][:2], before[m][0][:2]), m         # home slots untouched
         assert torch.equal(ws[m][0][3:], before[m][0][3:]), m         # unused slots untouched
         assert torch.equal(ws[m][1], before[m][1]), m                 # the home rank is only read
+
+
+@pytest.mark.parametrize("misalign", [True, False], ids=["16-byte", "32-byte"])
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16", "f32+base"])
+def test_expert_choice_gather_and_combine_vector_widths(cuda_ok, misalign, out_dtype):
+    """Expert choice on given scores: the selection's row gather (X -> Xp) and the combine over
+    each token's rows (in column parts), on shifted or aligned buffers."""
+    T, E, C, d = 900, 6, 200, 320
+    rng = np.random.default_rng(28)
+    S = rng.random((T, E)).astype(np.float32)
+    s = moe.shape(T, d, E, 1, 64, capacity=C, route_flags=moe.ROUTE_EXPERT_CHOICE)
+    n_seg, rows = moe.moe_layout(s)
+    x = buf((T, d), torch.bfloat16, misalign)
+    x.copy_(torch.randn(T, d, generator=torch.Generator().manual_seed(29)).to(torch.bfloat16))
+    xp = buf((rows, d), torch.bfloat16, misalign)
+    se, so, src, emap = i32(E), i32(E + 1), i32(rows), i32(T * E)
+    row_w = torch.zeros(rows, dtype=torch.float32, device="cuda")
+    moe.moe_expert_choose(s, torch.from_numpy(np.ascontiguousarray(S.T)).cuda(), x, se, so, src, row_w, emap, xp)
+    torch.cuda.synchronize()
+    ec = oracle.select_tokens(S, C)
+    assert (src.cpu().numpy() == ec.src).all()
+    assert (emap.view(T, E).cpu().numpy() == oracle.expert_choice_map(ec, T)).all()
+    assert torch.equal(xp.cpu(), x.cpu()[torch.from_numpy(ec.src)])
+
+    yp_h = torch.randn(rows, d, generator=torch.Generator().manual_seed(30))
+    base_h = torch.randn(T, d, generator=torch.Generator().manual_seed(31)) if out_dtype == "f32+base" else None
+    ref = oracle.combine_expert_choice(oracle.f64(yp_h), ec.src, ec.row_w.astype(np.float32), T)
+    if base_h is not None:
+        ref = ref + oracle.f64(base_h)
+    yp = buf((rows, d), torch.float32, misalign)
+    yp.copy_(yp_h)
+    bf16 = out_dtype == "bf16"
+    if bf16:
+        s.out_dtype = moe.DTYPE_BF16
+    out = buf((T, d), torch.bfloat16 if bf16 else torch.float32, misalign)
+    base = None
+    if base_h is not None:
+        base = buf((T, d), torch.float32, misalign)
+        base.copy_(base_h)
+    moe.moe_combine_expert_choice(s, yp, emap, row_w, base, out)
+    torch.cuda.synchronize()
+    got = to_np(out)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    if bf16:
+        assert (np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6 * rms).all()
+    else:
+        check_close(got, ref, "out", max_abs_of_rms=1e-5, mean_rel=1e-6)
