@@ -327,8 +327,7 @@ MOE_API moe_status_t moe_expert_gate_up(const moe_shape_t *shape, const moe_bf16
  * stored in fp32 (Yp is only read by the combine; keeping it in fp32 leaves
  * one rounding, the bf16 Hp operand, between the expert and the output).
  *   hp [rows_alloc, F] bf16; w_down [E, d, F] bf16; yp [rows_alloc, d] fp32 out.
- * When segments average at least 192 rows and d_ff <= 4096, it runs on CTA pairs
- * (tcgen05 cta_group::2, 256-row tiles); otherwise on single CTAs (128-row tiles).
+ * Tiles of 128 rows x 256 columns, one CTA each.
  */
 MOE_API moe_status_t moe_expert_down(const moe_shape_t *shape, const moe_bf16_t *hp,
                              const int32_t *seg_expert, const int32_t *seg_offsets,

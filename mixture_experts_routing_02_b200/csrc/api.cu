@@ -115,16 +115,6 @@ bool tmap_experts(CUtensorMap* m, const void* p, int E, int N, int K, int box_n)
 
 inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// The down projection runs on CTA pairs (256-row tiles) when segments are long enough on average
-// that the second 128 rows of a tile are mostly real rows and its reduction (F) is short, so the
-// fp32 epilogue is a large share of each tile; measured on B200 the pair kernel is then ~8 % faster.
-// Everything else (and the gate/up projection always) runs on single CTAs with 128-row tiles,
-// which measured as fast or faster: the contraction is power-limited, not operand-bandwidth-limited.
-bool use_pairs_for_down(const Dims& v) {
-    return v.n_seg > 0 && v.F <= kPairMaxReduction &&
-           static_cast<int64_t>(v.rows) >= static_cast<int64_t>(kPairMinRowsPerSegment) * v.n_seg;
-}
-
 // ------------------------------------------------------------------------------ implementations
 
 moe_status_t route_impl(const Dims& v, const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
@@ -275,21 +265,12 @@ moe_status_t down_impl(const Dims& v, const moe_bf16_t* hp, const int32_t* seg_e
     if (v.T == 0 || v.rows == 0) return MOE_OK;
     if (!have_encoder()) return MOE_ERR_CUDA;
     const int bn = v.d >= 256 ? 256 : v.d;
-    const bool pairs = use_pairs_for_down(v);
     CUtensorMap ta, tb;
-    // a CTA of a pair loads half of the B tile's rows
-    if (!tmap_rows(&ta, hp, v.rows, v.F) || !tmap_experts(&tb, wd, v.E, v.d, v.F, pairs ? bn / 2 : bn))
-        return MOE_ERR_CUDA;
+    if (!tmap_rows(&ta, hp, v.rows, v.F) || !tmap_experts(&tb, wd, v.E, v.d, v.F, bn)) return MOE_ERR_CUDA;
     GemmArgs g{};
     g.seg_offsets = seg_offsets; g.seg_expert = seg_expert; g.n_seg = v.n_seg; g.M = v.rows; g.K = v.F; g.N = v.d;
     g.BN = bn; g.n_tiles_n = (v.d + bn - 1) / bn; g.mma_n = bn;
     g.out = yp; g.ldo = v.d; g.k = v.k; g.status = status;
-    if (pairs) {
-        g.stages = gemm_pair_pick_stages(bn);
-        const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 256 + v.n_seg) * g.n_tiles_n;
-        const int n_pairs = static_cast<int>(std::min<int64_t>(sm_count() / 2, max_tiles));
-        return cuda_status(launch_umma_gemm_pair(kEpiStore, ta, tb, tb, g, n_pairs, st));
-    }
     g.stages = gemm_pick_stages(bn);
     const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 128 + v.n_seg) * g.n_tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(sm_count(), max_tiles));

@@ -47,14 +47,6 @@ size_t gemm_smem_bytes(int stages, int mma_n);
 int gemm_pick_stages(int mma_n);
 cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                              const GemmArgs& g, int grid, cudaStream_t stream);
-// CTA-pair version (plain fp32 epilogue, i.e. the down projection): 256-row tiles; B tiles of
-// mma_n/2 rows per CTA.
-size_t gemm_pair_smem_bytes(int stages, int mma_n);
-int gemm_pair_pick_stages(int mma_n);
-cudaError_t launch_umma_gemm_pair(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                                  const GemmArgs& g, int n_pairs, cudaStream_t stream);
-constexpr int kPairMinRowsPerSegment = 192;  // average rows per segment from which pairs pay off
-constexpr int kPairMaxReduction = 4096;      // the down projection uses pairs up to this d_ff
 
 // dispatch.cu
 constexpr int kPermuteThreads = 256;

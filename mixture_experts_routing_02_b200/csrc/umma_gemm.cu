@@ -439,171 +439,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 
-// ------------------------------------------------------------------------------------------
-// The same contraction on a CTA pair (cluster of 2, tcgen05 cta_group::2): a 256-row tile whose
-// rows [0,128) live in CTA 0 and [128,256) in CTA 1.  Each CTA loads its own 128 rows of A and
-// its half of the B tile (SwiGLU: CTA 0 the gate rows, CTA 1 the up rows; plain: the two halves
-// of the output columns), so every SM moves half the B bytes of the single-CTA kernel and a stage
-// is 32 KB (6 stages).  The leader (rank 0) expects the bytes of both CTAs' loads on its full
-// barrier and issues M=256 MMAs; its commits arrive on the barriers of both CTAs; the epilogue
-// warps of both CTAs read their own tensor memory and release the accumulator buffer on the
-// leader's barrier.
-template <int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
-    umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                          const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
-    __shared__ __align__(8) uint64_t full_bar[kMaxStages];
-    __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
-    __shared__ __align__(8) uint64_t tfull_bar[2];
-    __shared__ __align__(8) uint64_t tempty_bar[2];
-    __shared__ __align__(8) uint64_t drain_bar;
-    __shared__ uint32_t tmem_base_sh;
-    __shared__ int abort_sh;
-    __shared__ int tile_prefix[kMaxSegments + 1];
-    extern __shared__ uint8_t dsmem[];
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();
-    const int pair = blockIdx.x >> 1;
-    const int n_pairs = gridDim.x >> 1;
-    const int stages = g.stages;
-    const int b_half_rows = g.mma_n / 2;
-    const uint32_t b_half_bytes = static_cast<uint32_t>(b_half_rows) * 128u;
-
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + stages * kABytes;
-    uint32_t* epi_stage = reinterpret_cast<uint32_t*>(sB + stages * b_half_bytes);
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < stages; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull_bar[b], 1);
-            mbar_init(&tempty_bar[b], 8);  // 4 epilogue warps of each CTA (used in the leader)
-        }
-        mbar_init(&drain_bar, 1);
-        abort_sh = 0;
-        mbar_fence_init();
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(EPI == kEpiSwiglu && rank == 1 ? &tmB1 : &tmB0);
-    }
-    if (warp == 1) tmem_alloc_pair(&tmem_base_sh, kTmemCols);
-    if (warp == 2) build_tile_prefix(tile_prefix, g, 2 * kBM, lane);
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrive
-    tc_fence_after();
-
-    const uint32_t tmem_base = tmem_base_sh;
-    const int total = tile_prefix[g.n_seg] * g.n_tiles_n;
-    const int nkb = g.K / kBK;
-
-    if (warp == 0) {
-        // ------------------------------------------------------------------ TMA producer (both CTAs)
-        if (lane == 0) {
-            int stage = 0, issued = 0;
-            uint32_t phase = 0;
-            const uint32_t tx = 2u * (kABytes + b_half_bytes);
-            const CUtensorMap* tb = (EPI == kEpiSwiglu && rank == 1) ? &tmB1 : &tmB0;
-            bool ok = true;
-            for (int tile = pair; ok && tile < total; tile += n_pairs) {
-                const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g, 2 * kBM);
-                const int n0 = c.n * g.BN;
-                const int b_row = (EPI == kEpiSwiglu) ? n0 : n0 + static_cast<int>(rank) * b_half_rows;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, g.status)) { ok = false; break; }
-                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], tx);
-                    const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
-                    tma_load_2d_pair(sA + stage * kABytes, &tmA, kb * kBK, c.row0 + static_cast<int>(rank) * kBM, fb);
-                    tma_load_3d_pair(sB + stage * b_half_bytes, tb, kb * kBK, b_row, c.expert, fb);
-                    ++issued;
-                    if (++stage == stages) { stage = 0; phase ^= 1u; }
-                }
-            }
-            if (!ok) {
-                // let copies in flight land before the CTA pair exits (bounded)
-                if (rank == 0) {
-                    const int first = issued > stages ? issued - stages : 0;
-                    for (int i = first; i < issued; ++i)
-                        mbar_wait(&full_bar[i % stages], static_cast<uint32_t>((i / stages) & 1), nullptr, nullptr);
-                } else {
-                    for (int i = 0; i < 1000; ++i) sleep_ns(1000);
-                }
-            }
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer (leader only)
-        if (lane == 0 && rank == 0) {
-            int stage = 0, acc = 0;
-            uint32_t phase = 0, acc_phase = 0;
-            const uint32_t idesc = umma_idesc_bf16(2 * kBM, g.mma_n);
-            bool ok = true;
-            for (int tile = pair; ok && tile < total; tile += n_pairs) {
-                if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_sh, g.status)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kAccStride;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&full_bar[stage], phase, &abort_sh, g.status)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * kABytes));
-                    const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * b_half_bytes));
-#pragma unroll
-                    for (int kk = 0; kk < kBK / kUmmaK; ++kk)
-                        umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-                    const uint32_t eb = smem_u32(&empty_bar[stage]);
-                    umma_commit_pair(eb);
-                    umma_commit_pair(mapa_shared(eb, 1));
-                    if (++stage == stages) { stage = 0; phase ^= 1u; }
-                }
-                if (!ok) break;
-                const uint32_t fb = smem_u32(&tfull_bar[acc]);
-                umma_commit_pair(fb);
-                umma_commit_pair(mapa_shared(fb, 1));
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1u;
-            }
-            umma_commit_pair(smem_u32(&drain_bar));
-            mbar_wait(&drain_bar, 0, nullptr, nullptr);
-        }
-        __syncwarp();
-    } else {
-        // ------------------------------------------------------------------ epilogue (both CTAs)
-        const int quarter = warp & 3;
-        int acc = 0;
-        uint32_t acc_phase = 0;
-        const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
-        const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty_bar[1]), 0);
-        for (int tile = pair; tile < total; tile += n_pairs) {
-            const TileCoord c = decode_tile(tile, tile_prefix, g.n_seg, g.n_tiles_n, g, 2 * kBM);
-            const bool got = mbar_wait(&tfull_bar[acc], acc_phase, &abort_sh, g.status);
-            if (!__all_sync(0xffffffffu, got)) break;
-            tc_fence_after();
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                   static_cast<uint32_t>(acc) * kAccStride;
-            epilogue_rows<EPI>(g, t_row, c.row0 + static_cast<int>(rank) * kBM + quarter * 32, c.row_end,
-                               c.n * g.BN, lane, epi_stage + (warp - 2) * kStageWords);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
-            acc ^= 1;
-            if (acc == 0) acc_phase ^= 1u;
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync_all();  // no CTA leaves while its pair may still read its shared or tensor memory
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc_pair(tmem_base, kTmemCols);
-    }
-}
-
 }  // namespace
 
 size_t gemm_smem_bytes(int stages, int mma_n) {
@@ -628,38 +463,6 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const
     if (err != cudaSuccess) return err;
     kern<<<grid, kThreads, smem, stream>>>(a, b0, b1, g);
     return cudaGetLastError();
-}
-
-size_t gemm_pair_smem_bytes(int stages, int mma_n) {
-    return 1024 + static_cast<size_t>(stages) * (kABytes + static_cast<size_t>(mma_n / 2) * 128u) +
-           4 * kStageWords * sizeof(uint32_t);
-}
-
-int gemm_pair_pick_stages(int mma_n) {
-    const size_t per = kABytes + static_cast<size_t>(mma_n / 2) * 128u;
-    int s = static_cast<int>((kGemmSmemBudget - 1024) / per);
-    if (s > kMaxStages) s = kMaxStages;
-    return s;
-}
-
-template <int EPI>
-static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmArgs& g,
-                               int n_pairs, cudaStream_t stream) {
-    auto kern = umma_gemm_pair_kernel<EPI>;
-    size_t smem = gemm_pair_smem_bytes(g.stages, g.mma_n);
-    if (smem < kGemmSmemMin) smem = kGemmSmemMin;
-    cudaError_t err = set_max_dynamic_smem(kern, static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    err = launch_ex(kern, dim3(2 * n_pairs), dim3(kThreads), smem, stream, 2u, a, b0, b1, g);
-    if (err != cudaSuccess) return err;
-    return cudaGetLastError();
-}
-
-cudaError_t launch_umma_gemm_pair(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                                  const GemmArgs& g, int n_pairs, cudaStream_t stream) {
-    // only the plain (down-projection) epilogue runs on pairs; see use_pairs_for_down in api.cu
-    if (epi == kEpiStore) return launch_pair<kEpiStore>(a, b0, b1, g, n_pairs, stream);
-    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_umma_gemm(int epi, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,

@@ -93,7 +93,7 @@ CASES = [
     syn.Workload("plan", T=512, d=128, E=16, k=4, F=128, zipf_s=1.2, n_groups=4, replica_slots=8),
     # more than 65536 pairs: the look-back dispatch
     syn.Workload("lookback", T=9000, d=64, E=64, k=8, F=64, zipf_s=0.5),
-    # long segments, d_ff <= 4096: the down projection on CTA pairs
+    # long segments: several row tiles per expert
     syn.Workload("pairs", T=700, d=192, E=3, k=2, F=320, zipf_s=1.0),
     # overflow re-routing
     syn.Workload("reroute", T=600, d=128, E=8, k=2, F=128, zipf_s=1.2, capacity_factor=1.0, reroute=True),
