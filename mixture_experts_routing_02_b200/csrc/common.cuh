@@ -14,7 +14,6 @@
 
 #include <mutex>
 #include <unordered_map>
-#include <utility>
 
 #include "../../include/moe_routing.h"
 
@@ -211,9 +210,6 @@ __device__ __forceinline__ void store_out4(__nv_bfloat16* row, int v, float4 a) 
     reinterpret_cast<uint2*>(row)[v] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -242,10 +238,6 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
-
-__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
-
-__host__ __device__ constexpr int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
 
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) costs far more host time than a launch, so it is
 // made once per kernel, device and size: a size no larger than one already set is not set again.
