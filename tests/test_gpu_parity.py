@@ -479,10 +479,23 @@ def test_shared_expert_overlapped_on_a_second_stream():
     assert torch.equal(y1, y2)
 
 
-def test_layer_fwd_captured_in_a_cuda_graph():
+GRAPHED = [
+    SMALL[1],  # ragged top-k, single-pass router
+    syn.Workload("split-router", T=600, d=1024, E=16, k=2, F=128, zipf_s=0.8),  # router split over CTAs
+    syn.Workload("plan", T=512, d=128, E=16, k=4, F=128, zipf_s=1.2, n_groups=4, replica_slots=8),
+    syn.Workload("lookback", T=9000, d=64, E=64, k=8, F=64, zipf_s=0.5),  # memset + look-back dispatch
+    syn.Workload("reroute", T=300, d=128, E=8, k=2, F=192, zipf_s=1.2, capacity_factor=0.9, reroute=True),
+    syn.Workload("expert-choice", T=700, d=128, E=8, k=2, F=192, zipf_s=1.0, capacity_factor=1.0,
+                 expert_choice=True),
+]
+
+
+@pytest.mark.parametrize("w", GRAPHED, ids=[w.name for w in GRAPHED])
+def test_layer_fwd_captured_in_a_cuda_graph(w):
     """The whole layer allocates nothing and never synchronises, so it can be captured into a
-    CUDA graph and replayed; replays read the same device buffers and match eager calls."""
-    w = SMALL[1]  # ragged
+    CUDA graph and replayed; replays read the same device buffers and match eager calls.  Every
+    dispatch mode: the count kernel, the balanced plan, the look-back (with its memset), the
+    re-routing rounds (a cooperative launch) and expert choice."""
     case = make_case(w, seed=14)
     s = moe_shape(w)
     _, layer_bytes = moe.moe_workspace_size(s)
