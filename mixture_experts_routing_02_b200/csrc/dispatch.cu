@@ -1174,6 +1174,7 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const __nv_bfloat16* 
 // router projection whose reduction was split over more CTAs.  Writes the logits (optional),
 // then either the top-k ids and weights or, for expert-choice routing (scores_t non-null), the
 // softmax over all E experts stored expert-major.
+template <int U, int KMAX>
 __global__ void __launch_bounds__(256) route_logits_kernel(const float* __restrict__ part, int n_split, int ldp,
                                                            size_t split_stride, const float* __restrict__ bias, int T,
                                                            int E, int k, int route_flags, float* __restrict__ logits,
@@ -1182,7 +1183,8 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const float* __restri
     const int lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (blockDim.x >> 5);
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total)
-        route_token(part, n_split, ldp, split_stride, bias, T, E, k, route_flags, logits, ids, w, scores_t, t, lane);
+        route_token<U, KMAX>(part, n_split, ldp, split_stride, bias, T, E, k, route_flags, logits, ids, w, scores_t, t,
+                             lane);
 }
 
 }  // namespace
@@ -1367,10 +1369,21 @@ cudaError_t launch_route_logits(const float* part, int n_split, int ldp, size_t 
                                 int E, int k, int route_flags, float* logits, int32_t* ids, float* w, float* scores_t,
                                 int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
+    // one warp per token, grid-stride; at most four 256-thread CTAs per SM, so one wave
     int grid = (T + 7) / 8;
-    if (grid > 8 * num_sms) grid = 8 * num_sms;
-    route_logits_kernel<<<grid, 256, 0, stream>>>(part, n_split, ldp, split_stride, bias, T, E, k, route_flags, logits,
-                                                  ids, w, scores_t);
+    if (grid > 4 * num_sms) grid = 4 * num_sms;
+    using Kern = void (*)(const float*, int, int, size_t, const float*, int, int, int, int, float*, int32_t*, float*,
+                          float*);
+    // the loops bounded by E rounded up to 32, 64, 128 or 256 experts and by k rounded up to 2, 4 or 8
+    static const Kern table[4][3] = {
+        {route_logits_kernel<1, 2>, route_logits_kernel<1, 4>, route_logits_kernel<1, 8>},
+        {route_logits_kernel<2, 2>, route_logits_kernel<2, 4>, route_logits_kernel<2, 8>},
+        {route_logits_kernel<4, 2>, route_logits_kernel<4, 4>, route_logits_kernel<4, 8>},
+        {route_logits_kernel<8, 2>, route_logits_kernel<8, 4>, route_logits_kernel<8, 8>}};
+    const int ui = E <= 32 ? 0 : (E <= 64 ? 1 : (E <= 128 ? 2 : 3));
+    const int ki = k <= 2 ? 0 : (k <= 4 ? 1 : 2);
+    table[ui][ki]<<<grid, 256, 0, stream>>>(part, n_split, ldp, split_stride, bias, T, E, k, route_flags, logits, ids,
+                                            w, scores_t);
     return cudaGetLastError();
 }
 

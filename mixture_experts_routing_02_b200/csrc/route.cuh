@@ -16,14 +16,17 @@
 namespace moe {
 namespace {
 
+// U: experts per lane (E <= 32U); KMAX: the largest k.  Both bound the unrolled loops only: the
+// arithmetic and its order do not depend on them.
+template <int U, int KMAX>
 __device__ __forceinline__ void route_token(const float* __restrict__ part, int n_split, int ldp, size_t split_stride,
                                             const float* __restrict__ bias, int T, int E, int k, int route_flags,
                                             float* __restrict__ logits, int32_t* __restrict__ ids,
                                             float* __restrict__ w, float* __restrict__ scores_t, int t, int lane) {
-    float v[kMaxExperts / 32];
+    float v[U];
     unsigned taken = 0;
 #pragma unroll
-    for (int u = 0; u < kMaxExperts / 32; ++u) {
+    for (int u = 0; u < U; ++u) {
         const int e = lane + 32 * u;
         v[u] = -INFINITY;
         if (e < E) {
@@ -40,34 +43,34 @@ __device__ __forceinline__ void route_token(const float* __restrict__ part, int 
     if (scores_t != nullptr) {
         float m = -INFINITY;
 #pragma unroll
-        for (int u = 0; u < kMaxExperts / 32; ++u) m = fmaxf(m, v[u]);
+        for (int u = 0; u < U; ++u) m = fmaxf(m, v[u]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         float sum = 0.f;
 #pragma unroll
-        for (int u = 0; u < kMaxExperts / 32; ++u)
+        for (int u = 0; u < U; ++u)
             if (lane + 32 * u < E) sum += expf(v[u] - m);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         const float inv = 1.0f / sum;
 #pragma unroll
-        for (int u = 0; u < kMaxExperts / 32; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int e = lane + 32 * u;
             if (e < E) scores_t[static_cast<size_t>(e) * T + t] = expf(v[u] - m) * inv;
         }
         return;
     }
-    float sv[kMaxTopK];
-    int si[kMaxTopK];
+    float sv[KMAX];
+    int si[KMAX];
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
         sv[j] = 0.f;
         si[j] = 0;
         if (j < k) {
             float bv = -INFINITY;
             int bi = 0x7fffffff;
 #pragma unroll
-            for (int u = 0; u < kMaxExperts / 32; ++u) {
+            for (int u = 0; u < U; ++u) {
                 const int e = lane + 32 * u;
                 if (!((taken >> u) & 1u) && (v[u] > bv || (v[u] == bv && e < bi))) { bv = v[u]; bi = e; }
             }
@@ -86,21 +89,21 @@ __device__ __forceinline__ void route_token(const float* __restrict__ part, int 
     float all = 0.f;
     if (route_flags & MOE_ROUTE_SOFTMAX_ALL) {
 #pragma unroll
-        for (int u = 0; u < kMaxExperts / 32; ++u)
+        for (int u = 0; u < U; ++u)
             if (lane + 32 * u < E) all += expf(v[u] - sv[0]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) all += __shfl_xor_sync(0xffffffffu, all, o);
     }
     if (lane == 0) {
-        float ex[kMaxTopK], sum = 0.f;
+        float ex[KMAX], sum = 0.f;
 #pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) {
+        for (int j = 0; j < KMAX; ++j) {
             ex[j] = j < k ? expf(sv[j] - sv[0]) : 0.f;
             sum += ex[j];
         }
         const float inv = 1.0f / ((route_flags & MOE_ROUTE_SOFTMAX_ALL) ? all : sum);
 #pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j)
+        for (int j = 0; j < KMAX; ++j)
             if (j < k) {
                 ids[static_cast<size_t>(t) * k + j] = si[j];
                 w[static_cast<size_t>(t) * k + j] = ex[j] * inv;
