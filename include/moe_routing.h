@@ -127,7 +127,7 @@ typedef enum {
  *                  no candidate left is dropped.  A moved pair keeps its routing
  *                  weight.  Segment e holds its rows round by round, q order
  *                  inside a round.  Requires capacity >= 1, n_groups == 0 and
- *                  T * k <= 65536; excludes MOE_ROUTE_EXPERT_CHOICE.  Takes
+ *                  T * k <= 524288 (2^19); excludes MOE_ROUTE_EXPERT_CHOICE.  Takes
  *                  moe_dispatch_reroute (which needs the router's fp32 logits) in
  *                  place of moe_dispatch, which rejects it.
  */

@@ -78,7 +78,7 @@ moe_status_t check_shape(const moe_shape_t* s, Dims* out) {
     v.S = v.R > 0 ? v.T / v.R : v.T;
     int64_t rows = static_cast<int64_t>(v.T) * v.k;
     if (v.C > 0) rows = std::min<int64_t>(rows, static_cast<int64_t>(v.C) * v.E);
-    if (rr && static_cast<int64_t>(v.T) * v.k > kCountMaxPairs) return MOE_ERR_UNSUPPORTED;
+    if (rr && static_cast<int64_t>(v.T) * v.k > kRerouteMaxPairs) return MOE_ERR_UNSUPPORTED;
     if (ec) {
         // segment e holds expert e's C' = min(C, T) chosen tokens
         rows = static_cast<int64_t>(std::min(v.C, v.T)) * v.E;

@@ -955,7 +955,7 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* bar, int32_t* status, vol
 // base of its stable ranks (the same q-ordered ranks as one CTA over the whole list) and the
 // totals, from which every CTA derives the experts' new row counts and the number of pairs still
 // unplaced.  Exchanged counts are read through L2 (ld.global.cg).
-constexpr int kRerouteSliceMax = kRerouteThreads + kMaxTopK;
+constexpr int kRerouteSliceMax = 4096 + kMaxTopK;  // pairs of one CTA's slice (shared memory: 6 ints each)
 
 size_t reroute_smem_bytes() { return size_t(6) * kRerouteSliceMax * sizeof(int); }
 
@@ -1343,8 +1343,8 @@ cudaError_t launch_reroute(const RerouteArgs& a0, void* ws, const __nv_bfloat16*
     if (G > resident) G = resident;
     if (G > kRerouteMaxCtas) G = kRerouteMaxCtas;
     if (G < 1) G = 1;
-    // every CTA's slice fits its shared memory (with T*k <= kCountMaxPairs, G is never capped
-    // below T*k / kRerouteThreads, so a slice holds at most kRerouteThreads + k pairs)
+    // every CTA's slice fits its shared memory (with T*k <= kRerouteMaxPairs and one CTA on each of
+    // at least 128 SMs, a slice holds at most 4096 + k pairs)
     if (static_cast<int64_t>((a.T + G - 1) / G) * a.k > kRerouteSliceMax) return cudaErrorInvalidValue;
     err = cudaMemsetAsync(a.bar, 0, 2 * sizeof(uint32_t), stream);
     if (err != cudaSuccess) return err;

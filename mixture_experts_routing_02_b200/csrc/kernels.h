@@ -108,8 +108,9 @@ cudaError_t launch_dispatch_fused(const PermuteArgs& a, int num_sms, cudaStream_
 cudaError_t launch_dispatch_count(const PermuteArgs& a, int num_sms, cudaStream_t stream);
 constexpr int kCountMaxPairs = 1 << 16;
 constexpr int kCountMaxPairsPlan = 1 << 20;  // with a balanced plan the copies dwarf the recounting
+constexpr int kRerouteMaxPairs = 1 << 19;    // re-routing: one CTA per SM holds 4096 pairs at most
 
-// Overflow re-routing (the capacity rounds on a cooperative grid; T*k <= kCountMaxPairs), then the
+// Overflow re-routing (the capacity rounds on a cooperative grid; T*k <= kRerouteMaxPairs), then the
 // row copies.
 constexpr int kRerouteThreads = 1024;
 struct RerouteArgs {

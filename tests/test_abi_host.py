@@ -109,6 +109,9 @@ def test_workspace_sizes_grow_with_the_layer(lib):
     (dict(route_flags=2), 1), (dict(route_flags=3, capacity=8), 1),
     (dict(route_flags=2, capacity=8, n_groups=2), 1),
     (dict(route_flags=2, capacity=1 << 23, T=1 << 23, n_experts=256, top_k=1), 2),
+    # re-routing: up to 2^19 (t, j) pairs (each of up to 128 CTAs keeps 4096 in shared memory)
+    (dict(route_flags=4, capacity=64, T=1 << 18, top_k=2), 0),
+    (dict(route_flags=4, capacity=64, T=(1 << 18) + 1, top_k=2), 2),
 ])
 def test_shape_validation(lib, kw, code):
     s = _shape(**kw)

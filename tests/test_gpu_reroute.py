@@ -122,6 +122,28 @@ def test_reroute_dispatch_full_skewed_size(cuda_ok):
     assert torch.equal(xp[:used].cpu(), x[torch.from_numpy(rsrc // w.k)])
 
 
+@pytest.mark.parametrize("T,E,k", [(40000, 32, 2), (65536, 16, 8)], ids=["80k-pairs", "2^19-pairs"])
+def test_reroute_dispatch_beyond_64k_pairs(cuda_ok, T, E, k):
+    """More pairs than one 1024-pair slice per SM: each CTA of the grid keeps several thousand pairs
+    in shared memory (the largest case is the 2^19-pair limit).  Zipf(1.2)-skewed fp32 logits, a
+    capacity of the average load: the whole placement bit for bit."""
+    C = T * k // E
+    rng = np.random.default_rng(T + k)
+    l = (rng.normal(scale=1.28, size=(T, E)) - 1.2 * np.log(np.arange(1, E + 1))[None, :]).astype(np.float32)
+    x, ids, counts, so, dest, src, xp = _dispatch(T, 64, E, k, C, l, seed=3)
+    l64 = l.astype(np.float64)
+    rid = oracle.topk_ids(l64, k)
+    assert (ids == rid).all()
+    rr = oracle.reroute_overflow(rid, l64, C)
+    segs, rdest, rsrc = oracle.reroute_positions(rr)
+    assert (rr.round > 0).any()
+    assert (so == segs.offsets).all()
+    assert (dest == rdest).all()
+    used = int(segs.offsets[-1])
+    assert (src[:used] == rsrc).all()
+    assert torch.equal(xp[:used].cpu(), x[torch.from_numpy(rsrc // k)])
+
+
 def test_dispatch_rejects_the_reroute_flag(cuda_ok):
     s = moe.shape(64, 128, 8, 2, 128, capacity=16, route_flags=moe.ROUTE_REROUTE)
     dummy = torch.zeros(1 << 16, dtype=torch.int32, device="cuda")
