@@ -418,6 +418,21 @@ MOE_API moe_status_t moe_testing_dispatch_stalled(const moe_shape_t *shape, cons
                                           moe_stream_t stream);
 
 /*
+ * Testing only: moe_dispatch_reroute in which CTA 0 of the re-routing rounds'
+ * cooperative grid never arrives at the first grid barrier, so every other CTA's
+ * wait there can never end.  Each wait gives up after its bound (about 2 s), sets
+ * MOE_DEV_ERR_TIMEOUT in *status and its CTA returns; counts, the tables, dest,
+ * src and xp are then incomplete (values outside [0, rows_alloc) are never written
+ * through).  It shows that the grid barrier returns an error instead of hanging and
+ * leaves the context usable.  Needs MOE_ROUTE_REROUTE and T * k > 1024 (two CTAs).
+ */
+MOE_API moe_status_t moe_testing_reroute_stalled(const moe_shape_t *shape, const moe_bf16_t *x,
+                                         const int32_t *topk_ids, const float *logits, int32_t *counts,
+                                         int32_t *seg_expert, int32_t *seg_offsets, int32_t *seg_first_rank,
+                                         int32_t *dest, int32_t *src, moe_bf16_t *xp, int32_t *status,
+                                         void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Testing only: moe_expert_gate_up in which CTA 0 never issues the copy of its
  * first pipeline stage, so the tensor-core issuer's wait on that stage can never
  * end.  The wait gives up after its bound (about 2 s), sets MOE_DEV_ERR_TIMEOUT

@@ -74,6 +74,7 @@ SYMBOLS = {
     "moe_testing_dispatch_stalled": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_expert_gate_up": [_S, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_testing_gemm_stalled": [_S, _P, _P, _P, _P, _P, _P, _P, _P],
+    "moe_testing_reroute_stalled": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_expert_down": [_S, _P, _P, _P, _P, _P, _P, _P],
     "moe_expert_ffn": [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "moe_combine": [_S, _P, _P, _P, _P, _P],
@@ -228,6 +229,14 @@ def moe_expert_gate_up(s, xp, seg_expert, seg_offsets, w_gate, w_up, hp, status=
     _check("moe_expert_gate_up", load_library().moe_expert_gate_up(
         ctypes.byref(s), _ptr(xp), _ptr(seg_expert), _ptr(seg_offsets), _ptr(w_gate), _ptr(w_up), _ptr(hp),
         _ptr(status), _stream(stream)))
+
+
+def moe_testing_reroute_stalled(s, x, topk_ids, logits, counts, seg_expert, seg_offsets, seg_first_rank, dest, src,
+                                xp, status, ws, stream=None):
+    """Testing only: the re-routing dispatch with CTA 0 never arriving at the first grid barrier."""
+    _check("moe_testing_reroute_stalled", load_library().moe_testing_reroute_stalled(
+        ctypes.byref(s), _ptr(x), _ptr(topk_ids), _ptr(logits), _ptr(counts), _ptr(seg_expert), _ptr(seg_offsets),
+        _ptr(seg_first_rank), _ptr(dest), _ptr(src), _ptr(xp), _ptr(status), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def moe_testing_gemm_stalled(s, xp, seg_expert, seg_offsets, w_gate, w_up, hp, status, stream=None):

@@ -290,7 +290,7 @@ moe_status_t segments_or_plan(const Dims& v, int32_t* counts, const int32_t* par
 moe_status_t reroute_impl(const Dims& v, const moe_bf16_t* x, const int32_t* ids, const float* logits,
                           int32_t* counts, int32_t* seg_expert, int32_t* seg_offsets, int32_t* seg_first_rank,
                           int32_t* dest, int32_t* src, moe_bf16_t* xp, int32_t* status, void* ws, size_t ws_bytes,
-                          cudaStream_t st) {
+                          cudaStream_t st, bool test_stall = false) {
     if (!x || !ids || !logits || !counts || !seg_expert || !seg_offsets || !seg_first_rank || !dest || !src || !xp)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
@@ -301,6 +301,7 @@ moe_status_t reroute_impl(const Dims& v, const moe_bf16_t* x, const int32_t* ids
     a.T = v.T; a.k = v.k; a.E = v.E; a.capacity = v.C; a.rows = v.rows;
     a.counts = counts; a.seg_expert = seg_expert; a.seg_offsets = seg_offsets; a.seg_first_rank = seg_first_rank;
     a.dest = dest; a.src = src; a.status = status;
+    a.test_skip_arrival = test_stall ? 1 : 0;
     return cuda_status(launch_reroute(a, ws, reinterpret_cast<const __nv_bfloat16*>(x),
                                       reinterpret_cast<__nv_bfloat16*>(xp), v.d, sm_count(), st));
 }
@@ -676,6 +677,20 @@ moe_status_t moe_testing_dispatch_stalled(const moe_shape_t* shape, const moe_bf
     if (permute_n_tiles(v.T, v.k) < 2) return MOE_ERR_INVALID_ARG;  // needs a tile that waits on tile 0
     return dispatch_impl(v, x, topk_ids, 0, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp, status,
                          ws, ws_bytes, static_cast<cudaStream_t>(stream), 1);
+}
+
+moe_status_t moe_testing_reroute_stalled(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_ids,
+                                         const float* logits, int32_t* counts, int32_t* seg_expert,
+                                         int32_t* seg_offsets, int32_t* seg_first_rank, int32_t* dest, int32_t* src,
+                                         moe_bf16_t* xp, int32_t* status, void* ws, size_t ws_bytes,
+                                         moe_stream_t stream) {
+    Dims v;
+    const moe_status_t s = check_shape(shape, &v);
+    if (s != MOE_OK) return s;
+    if (!v.rr()) return MOE_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(v.T) * v.k <= kRerouteThreads || v.T < 2) return MOE_ERR_INVALID_ARG;  // needs 2+ CTAs
+    return reroute_impl(v, x, topk_ids, logits, counts, seg_expert, seg_offsets, seg_first_rank, dest, src, xp, status,
+                        ws, ws_bytes, static_cast<cudaStream_t>(stream), true);
 }
 
 moe_status_t moe_testing_gemm_stalled(const moe_shape_t* shape, const moe_bf16_t* xp, const int32_t* seg_expert,

@@ -982,7 +982,9 @@ __global__ void __launch_bounds__(kRerouteThreads, 1) reroute_grid_kernel(Rerout
     const int tokens_per_cta = (a.T + G - 1) / G;
     const int b0 = min(n, cta * tokens_per_cta * k), e0 = min(n, b0 + tokens_per_cta * k);
     const int nl = e0 - b0;  // <= kRerouteSliceMax (checked by the launcher)
-    if (tid == 0) s_abort = 0;
+    // testing only (moe_testing_reroute_stalled): CTA 0 starts aborted, so it never arrives at the
+    // first grid barrier and every other CTA's bounded wait there runs out
+    if (tid == 0) s_abort = (a.test_skip_arrival != 0 && cta == 0) ? 1 : 0;
     int xbuf = 0;
 
     // this CTA's counts s_loc[0..E) exchanged with every CTA's: s_base = the sum over the CTAs before

@@ -129,6 +129,7 @@ struct RerouteArgs {
     uint32_t* bar;   // [2] grid barrier (arrivals, generation); arrivals zero on entry
     int32_t* xchg;   // [2][kRerouteMaxCtas][kMaxExperts] per-CTA counts, two buffers used in turn
     int32_t* status; // MOE_DEV_ERR_TIMEOUT if a grid barrier wait runs out (nullable)
+    int test_skip_arrival;  // testing only: CTA 0 never arrives at the first grid barrier
 };
 constexpr int kRerouteMaxCtas = 256;  // CTAs of the grid-wide rounds (one per SM at most)
 size_t reroute_ws_bytes(int T, int k);

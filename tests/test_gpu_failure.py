@@ -93,3 +93,47 @@ def test_gemm_wait_that_cannot_end_times_out(cuda_ok):
     torch.cuda.synchronize()
     assert st2.item() == 0
     check_bf16_storage(hp2.float().cpu().numpy(), ref.hp, "Hp after the aborted GEMM")
+
+
+def test_reroute_grid_barrier_that_cannot_end_times_out(cuda_ok):
+    """The re-routing rounds' grid barrier: CTA 0 never arrives at the first one, so the other CTAs'
+    bounded waits run out after ~2 s; the status reports the timeout and every CTA returns (the
+    cooperative launch ends), and a normal re-routing dispatch right after gives the oracle's
+    placement."""
+    T, d, E, k, C = 1500, 64, 8, 2, 300   # 3000 pairs: three CTAs
+    rng = np.random.default_rng(41)
+    l = (rng.normal(size=(T, E)) - 1.2 * np.log(np.arange(1, E + 1))[None, :]).astype(np.float32)
+    s = moe.shape(T, d, E, k, 64, capacity=C, route_flags=moe.ROUTE_REROUTE)
+    n_seg, rows = moe.moe_layout(s)
+    disp, _ = moe.moe_workspace_size(s)
+    lg = torch.from_numpy(l).cuda()
+    ids = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    wts = torch.empty(T * k, dtype=torch.float32, device="cuda")
+    moe.moe_route_from_logits(s, lg, ids, wts)
+    x = torch.randn(T, d, generator=torch.Generator().manual_seed(42)).to(torch.bfloat16).cuda()
+    z = lambda n: torch.full((max(n, 1),), -1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(disp, dtype=torch.uint8, device="cuda")
+
+    counts, se, so, sf, dest, src = z(E), z(n_seg), z(n_seg + 1), z(n_seg), z(T * k), z(rows)
+    xp = torch.zeros(rows, d, dtype=torch.bfloat16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    moe.moe_testing_reroute_stalled(s, x, ids, lg, counts, se, so, sf, dest, src, xp, st, ws)
+    torch.cuda.synchronize()
+    elapsed = time.time() - t0
+    assert st.item() & moe.DEV_ERR_TIMEOUT
+    assert 1.0 < elapsed < 60.0
+
+    counts, se, so, sf, dest, src = z(E), z(n_seg), z(n_seg + 1), z(n_seg), z(T * k), z(rows)
+    xp = torch.zeros(rows, d, dtype=torch.bfloat16, device="cuda")
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.moe_dispatch_reroute(s, x, ids, lg, counts, se, so, sf, dest, src, xp, st2, ws)
+    torch.cuda.synchronize()
+    assert st2.item() == 0
+    l64 = l.astype(np.float64)
+    rr = oracle.reroute_overflow(oracle.topk_ids(l64, k), l64, C)
+    segs, rdest, rsrc = oracle.reroute_positions(rr)
+    assert (dest.cpu().numpy() == rdest).all()
+    used = int(segs.offsets[-1])
+    assert (src.cpu().numpy()[:used] == rsrc).all()
+    assert torch.equal(xp[:used].cpu(), x.cpu()[torch.from_numpy(rsrc // k)])
