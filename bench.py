@@ -411,8 +411,18 @@ def run_ours(args, w):
     # the router projection's reduction is split over more CTAs when its row tiles are few
     route_ws_bytes = moe.moe_route_workspace_size(s)
     route_ws = torch.empty(max(route_ws_bytes, 256), dtype=torch.uint8, device=dev) if route_ws_bytes else None
+    if rr:
+        dispatch_launches = 3        # candidate order, re-routing rounds, row copies
+    elif ec:
+        dispatch_launches = 2        # selection, row gather
+    elif w.n_groups and w.n_groups <= moe.EP_MAX_RANKS and (w.T // w.n_groups) * w.k <= (1 << 20):
+        dispatch_launches = 2        # per-group counts, grouped dispatch
+    elif w.n_groups and w.T * w.k > (1 << 20):
+        dispatch_launches = 4        # histogram partials, plan, ranks, row copies
+    else:
+        dispatch_launches = 1        # counts, tables, ranks and copies in one launch
     launches = ((2 if route_ws_bytes else 1)                                   # route (+ partial sums)
-                + (2 if ec or rr else (4 if w.n_groups and w.T * w.k > (1 << 20) else 1))  # dispatch
+                + dispatch_launches
                 + 3)                                                           # gate_up, down, combine
 
     Fs = args.shared_expert
