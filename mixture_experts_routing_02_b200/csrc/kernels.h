@@ -14,6 +14,8 @@ constexpr int kMaxTopK = 8;
 constexpr int kMaxSegments = 2048;
 constexpr size_t kGemmSmemBudget = 200 * 1024;  // operand stages of the GEMM
 constexpr size_t kGemmSmemMin = 120 * 1024;     // > half an SM's shared memory: one CTA per SM
+constexpr int kSwapTailRows = 32;                // down projection: largest segment tail computed
+                                                 // with swapped operands
 
 enum EpiKind : int { kEpiRoute = 0, kEpiSwiglu = 1, kEpiStore = 2 };
 
@@ -41,6 +43,8 @@ struct GemmArgs {
     size_t split_stride;   // elements between the outputs of consecutive parts
     int32_t* status;
     int test_skip_first_load;  // testing only: CTA 0 never issues its first stage's copy (its waits time out)
+    int swap_tail;  // plain epilogue with 256-row B stages: a segment's last row tile holding at most
+                    // this many rows is computed with the operands swapped (0: never)
 };
 
 size_t gemm_smem_bytes(int stages, int mma_n);

@@ -162,6 +162,42 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& g, uint32_t t_row,
     }
 }
 
+// A segment's last row tile holds r = row_end - row0 rows (1..128), and a 128-row MMA spends the
+// same time on its 128 - r padding rows as on real ones.  In the down projection (256-row weight
+// tiles, plain fp32 epilogue) a last tile with r <= g.swap_tail rows is computed with the operands
+// swapped: the 256 weight rows of the B stage become two 128-row A operands, the tile's rows the
+// N = ceil16(r) operand, and the accumulators hold [output column][row] at column offsets 0 and
+// 128 of the buffer.  Measured on B200 (same box, each kernel alone): segments of 128 + 16 and
+// 128 + 32 rows over 256 experts (d = 7168, d_ff = 2048) ran the down projection in 1.73 / 1.82 ms
+// instead of 2.18 / 2.16 ms; tails of 64 or 96 rows gained nothing (2.11 vs 2.03 ms, 1.95 vs
+// 1.92 ms), and the gate/up projection, whose swapped tiles issue four MMAs per 64-column stage
+// with two weight matrices, got slower at every tail size (3.82-4.53 vs 3.41-3.43 ms).  Returns
+// N, or 0 for a tile computed the usual way.
+__device__ __forceinline__ int swapped_cols(const TileCoord& c, const GemmArgs& g) {
+    const int r = c.row_end - c.row0;
+    return (g.swap_tail > 0 && r <= g.swap_tail) ? (r + 15) & ~15 : 0;
+}
+
+// Epilogue of a swapped down-projection tile: TMEM lane = output column (f for the accumulator at
+// column offset 0, f + 128 for the one at 128), TMEM column = the tile's row.  Each store
+// instruction writes one row's 32 consecutive fp32 columns (128 contiguous bytes per warp).
+__device__ __forceinline__ void epilogue_swapped(const GemmArgs& g, uint32_t t_row, int row0, int r, int nt, int f) {
+    float* out = static_cast<float*>(g.out);
+    for (int h = 0; h < 2; ++h) {
+        const int fh = f + 128 * h;
+        for (int cc = 0; cc < nt; cc += 32) {
+            uint32_t v[32];
+            tmem_ld32(t_row + 128 * h + cc, v);
+            tmem_ld_wait();
+            if (fh < g.N) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (cc + i < r) out[static_cast<size_t>(row0 + cc + i) * g.ldo + fh] = __uint_as_float(v[i]);
+            }
+        }
+    }
+}
+
 // SPLITK: the reduction is cut into g.k_splits equal parts, each a work unit of its own, and
 // part s of a tile is stored (plain fp32 epilogue) at out + s * split_stride; the caller sums
 // the parts.  Used for the router projection, whose T/128 row tiles are too few for the SMs.
@@ -177,6 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
     __shared__ int tile_prefix[kMaxSegments + 1];
+    // swapped width of each tile, by the CTA's tile sequence number mod 16: written by the producer
+    // before the tile's first stage is armed, read by the MMA issuer after that stage's full barrier
+    // (the producer runs at most `stages` <= 8 stages, hence tiles, ahead)
+    __shared__ int tile_swap[16];
     extern __shared__ uint8_t dsmem[];
 
     const int warp = threadIdx.x >> 5;
@@ -227,10 +267,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // MMA warp's bounded wait on it runs out and every role takes the abort path
             const bool skip_first = g.test_skip_first_load != 0 && blockIdx.x == 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            int seq = 0;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++seq) {
                 const int split = SPLITK ? tile % n_split : 0;
                 const TileCoord c = decode_tile(SPLITK ? tile / n_split : tile, tile_prefix, g.n_seg, g.n_tiles_n, g);
                 const int n0 = c.n * g.BN;
+                if (EPI == kEpiStore && !SPLITK) tile_swap[seq & 15] = swapped_cols(c, g);
                 const int kb0 = SPLITK ? split * nkb / n_split : 0;
                 const int kb1 = SPLITK ? (split + 1) * nkb / n_split : nkb;
                 for (int kb = kb0; kb < kb1; ++kb) {
@@ -270,25 +312,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0, acc_phase = 0;
             const uint32_t idesc = umma_idesc_bf16(kBM, g.mma_n);
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            int seq = 0;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++seq) {
                 if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_sh, g.status)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kAccStride;
                 const int split = SPLITK ? tile % n_split : 0;
                 const int kb0 = SPLITK ? split * nkb / n_split : 0;
                 const int kb1 = SPLITK ? (split + 1) * nkb / n_split : nkb;
-                for (int kb = kb0; kb < kb1; ++kb) {
+                int nt = 0;
+                if (EPI == kEpiStore && !SPLITK) {
+                    // the tile's swapped width, published by the producer before it armed the tile's
+                    // first stage (the usual loop below waits on that stage again at no cost)
                     if (!mbar_wait(&full_bar[stage], phase, &abort_sh, g.status)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * kABytes));
-                    const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * b_stage_bytes));
+                    nt = tile_swap[seq & 15];
+                }
+                if (nt > 0) {
+                    // swapped: weight rows [0,128) and [128,256) of the B stage against the tile's rows
+                    const uint32_t idesc_sw = umma_idesc_bf16(kBM, nt);
+                    for (int kb = kb0; kb < kb1; ++kb) {
+                        if (!mbar_wait(&full_bar[stage], phase, &abort_sh, g.status)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * kABytes));
+                        const uint64_t wdesc0 = umma_desc_sw128(smem_u32(sB + stage * b_stage_bytes));
+                        const uint64_t wdesc1 = umma_desc_sw128(smem_u32(sB + stage * b_stage_bytes + 128 * 128));
 #pragma unroll
-                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-                        // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4)
-                        umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                            const uint32_t accum = (kb != kb0 || kk != 0) ? 1u : 0u;
+                            umma_bf16(d_tmem, wdesc0 + 2 * kk, adesc + 2 * kk, idesc_sw, accum);
+                            umma_bf16(d_tmem + 128, wdesc1 + 2 * kk, adesc + 2 * kk, idesc_sw, accum);
+                        }
+                        umma_commit(&empty_bar[stage]);
+                        if (++stage == stages) { stage = 0; phase ^= 1u; }
                     }
-                    umma_commit(&empty_bar[stage]);
-                    if (++stage == stages) { stage = 0; phase ^= 1u; }
+                } else {
+                    for (int kb = kb0; kb < kb1; ++kb) {
+                        if (!mbar_wait(&full_bar[stage], phase, &abort_sh, g.status)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * kABytes));
+                        const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * b_stage_bytes));
+#pragma unroll
+                        for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                            // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4)
+                            umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+                        }
+                        umma_commit(&empty_bar[stage]);
+                        if (++stage == stages) { stage = 0; phase ^= 1u; }
+                    }
                 }
                 if (!ok) break;
                 umma_commit(&tfull_bar[acc]);
@@ -319,8 +389,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n0 = c.n * g.BN;
 
             if (EPI == kEpiSwiglu || EPI == kEpiStore) {
-                epilogue_rows<EPI>(g, t_row, c.row0 + quarter * 32, c.row_end, n0, lane,
-                                   epi_stage + (warp - 2) * kStageWords, out_off);
+                const int nt = (EPI == kEpiStore && !SPLITK) ? swapped_cols(c, g) : 0;
+                if (nt > 0)
+                    epilogue_swapped(g, t_row, c.row0, c.row_end - c.row0, nt, n0 + r_in_tile);
+                else
+                    epilogue_rows<EPI>(g, t_row, c.row0 + quarter * 32, c.row_end, n0, lane,
+                                       epi_stage + (warp - 2) * kStageWords, out_off);
             } else if (g.scores_t != nullptr) {
                 // expert choice: softmax over the E logits of this row, stored expert-major so
                 // that the 32 lanes (consecutive rows) of a warp write 128 contiguous bytes
