@@ -29,10 +29,10 @@ SMALL = [
     syn.Workload("multi-tile", T=1000, d=512, E=4, k=2, F=512, zipf_s=0.5),
     syn.Workload("wide-router", T=260, d=128, E=256, k=6, F=64),
     # long segments: several 128-row tiles per expert, ragged tails
-    syn.Workload("pair-ragged", T=700, d=192, E=3, k=2, F=320, zipf_s=1.0),
-    syn.Workload("pair-plan", T=2048, d=128, E=8, k=2, F=128, zipf_s=1.2, n_groups=2, replica_slots=4),
-    syn.Workload("pair-capacity", T=1500, d=256, E=4, k=2, F=192, zipf_s=1.2, capacity_factor=1.0),
-    syn.Workload("pair-small", T=600, d=64, E=2, k=1, F=64),
+    syn.Workload("long-ragged", T=700, d=192, E=3, k=2, F=320, zipf_s=1.0),
+    syn.Workload("long-plan", T=2048, d=128, E=8, k=2, F=128, zipf_s=1.2, n_groups=2, replica_slots=4),
+    syn.Workload("long-capacity", T=1500, d=256, E=4, k=2, F=192, zipf_s=1.2, capacity_factor=1.0),
+    syn.Workload("long-small", T=600, d=64, E=2, k=1, F=64),
     # dispatch paths by size: T*k = 65536 is the largest for the single-pass count kernel; above
     # it the look-back kernel runs (with and without a capacity)
     syn.Workload("count-largest", T=8192, d=64, E=16, k=8, F=64, zipf_s=0.7),
