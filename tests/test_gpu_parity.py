@@ -454,6 +454,25 @@ def test_shared_expert_and_combine_add():
     assert torch.equal(out2, got["out"])
 
 
+@pytest.mark.parametrize("T", [270, 128, 97])
+def test_shared_expert_row_tails(T):
+    """The shared expert's down projection over T rows whose last 128-row tile holds 14, 128 or 97
+    rows (14 takes the swapped-operand tail of the down projection; d = 512 gives it full 256-column
+    weight tiles)."""
+    w = syn.Workload("shared-tail", T=T, d=512, E=4, k=2, F=128)
+    case = make_case(w, seed=12)
+    Fs = 320
+    sh = syn.shared_expert_weights(w, Fs, 12)
+    s = moe_shape(w)
+    h_s = torch.empty(w.T, Fs, dtype=torch.bfloat16, device="cuda")
+    y_s = torch.empty(w.T, w.d, dtype=torch.float32, device="cuda")
+    st = i32(1)
+    moe.moe_shared_expert(s, Fs, dev(case.x), *(dev(t) for t in sh), h_s, y_s, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    check_close(to_np(y_s), oracle.shared_expert(case.x, *sh), "shared expert")
+
+
 def test_shared_expert_overlapped_on_a_second_stream():
     """Run on a side stream while the routed path runs; joined by an event, the result is bit-identical."""
     w, case, Fs, sh = _shared_case(seed=11)
