@@ -28,7 +28,10 @@
 //               fused math, a shared-memory transpose, then row-contiguous 16-byte
 //               stores of the valid rows
 // Two accumulator buffers (columns [0,256) and [256,512)) let the epilogue of
-// one tile overlap the main loop of the next.
+// one tile overlap the main loop of the next.  In the down projection a
+// segment's last tile of at most 32 rows swaps the operand roles (see
+// swapped_cols): the warps keep their jobs, the MMA warp issues two narrow
+// MMAs per K step and the epilogue stores columns instead of rows.
 #include "common.cuh"
 #include "kernels.h"
 
