@@ -327,9 +327,10 @@ MOE_API moe_status_t moe_expert_gate_up(const moe_shape_t *shape, const moe_bf16
  * stored in fp32 (Yp is only read by the combine; keeping it in fp32 leaves
  * one rounding, the bf16 Hp operand, between the expert and the output).
  *   hp [rows_alloc, F] bf16; w_down [E, d, F] bf16; yp [rows_alloc, d] fp32 out.
- * Tiles of 128 rows x 256 columns, one CTA each; a segment's last tile of at
- * most 32 rows is computed with the weight tile as the 128-row MMA operand and
- * its rows as the narrow one (same results within fp32 accumulation order).
+ * Tiles of 128 rows x 256 columns, one CTA each; with d_ff <= 4096 a segment's
+ * last tile of at most 32 rows is computed with the weight tile as the 128-row
+ * MMA operand and its rows as the narrow one (same results within fp32
+ * accumulation order).
  */
 MOE_API moe_status_t moe_expert_down(const moe_shape_t *shape, const moe_bf16_t *hp,
                              const int32_t *seg_expert, const int32_t *seg_offsets,

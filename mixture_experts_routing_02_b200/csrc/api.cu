@@ -271,7 +271,7 @@ moe_status_t down_impl(const Dims& v, const moe_bf16_t* hp, const int32_t* seg_e
     g.seg_offsets = seg_offsets; g.seg_expert = seg_expert; g.n_seg = v.n_seg; g.M = v.rows; g.K = v.F; g.N = v.d;
     g.BN = bn; g.n_tiles_n = (v.d + bn - 1) / bn; g.mma_n = bn;
     g.out = yp; g.ldo = v.d; g.k = v.k; g.status = status;
-    g.swap_tail = bn == 256 ? kSwapTailRows : 0;
+    g.swap_tail = (bn == 256 && v.F <= kSwapTailMaxK) ? kSwapTailRows : 0;
     g.stages = gemm_pick_stages(bn);
     const int64_t max_tiles = (static_cast<int64_t>(v.rows) / 128 + v.n_seg) * g.n_tiles_n;
     const int grid = static_cast<int>(std::min<int64_t>(sm_count(), max_tiles));
@@ -757,7 +757,8 @@ moe_status_t moe_shared_expert(const moe_shape_t* shape, int32_t d_ff_shared, co
         GemmArgs g{};
         g.seg_offsets = nullptr; g.seg_expert = nullptr; g.n_seg = 1; g.M = v.T; g.K = Fs; g.N = v.d;
         g.BN = bn; g.n_tiles_n = (v.d + bn - 1) / bn; g.mma_n = bn; g.stages = gemm_pick_stages(bn);
-        g.out = y_s; g.ldo = v.d; g.status = status; g.swap_tail = bn == 256 ? kSwapTailRows : 0;
+        g.out = y_s; g.ldo = v.d; g.status = status;
+        g.swap_tail = (bn == 256 && Fs <= kSwapTailMaxK) ? kSwapTailRows : 0;
         const int64_t tiles = static_cast<int64_t>((v.T + 127) / 128) * g.n_tiles_n;
         const int grid = static_cast<int>(std::min<int64_t>(sm_count(), tiles));
         return cuda_status(launch_umma_gemm(kEpiStore, ta, tb, tb, g, grid, st));

@@ -16,6 +16,7 @@ constexpr size_t kGemmSmemBudget = 200 * 1024;  // operand stages of the GEMM
 constexpr size_t kGemmSmemMin = 120 * 1024;     // > half an SM's shared memory: one CTA per SM
 constexpr int kSwapTailRows = 32;                // down projection: largest segment tail computed
                                                  // with swapped operands
+constexpr int kSwapTailMaxK = 4096;              // ... when its reduction (d_ff) is at most this long
 
 enum EpiKind : int { kEpiRoute = 0, kEpiSwiglu = 1, kEpiStore = 2 };
 

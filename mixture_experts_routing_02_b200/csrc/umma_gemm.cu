@@ -28,9 +28,9 @@
 //               fused math, a shared-memory transpose, then row-contiguous 16-byte
 //               stores of the valid rows
 // Two accumulator buffers (columns [0,256) and [256,512)) let the epilogue of
-// one tile overlap the main loop of the next.  In the down projection a
-// segment's last tile of at most 32 rows swaps the operand roles (see
-// swapped_cols): the warps keep their jobs, the MMA warp issues two narrow
+// one tile overlap the main loop of the next.  In the down projection with
+// d_ff <= 4096 a segment's last tile of at most 32 rows swaps the operand roles
+// (see swapped_cols): the warps keep their jobs, the MMA warp issues two narrow
 // MMAs per K step and the epilogue stores columns instead of rows.
 #include "common.cuh"
 #include "kernels.h"
@@ -174,7 +174,9 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& g, uint32_t t_row,
 // 128 + 32 rows over 256 experts (d = 7168, d_ff = 2048) ran the down projection in 1.73 / 1.82 ms
 // instead of 2.18 / 2.16 ms; tails of 64 or 96 rows gained nothing (2.11 vs 2.03 ms, 1.95 vs
 // 1.92 ms), and the gate/up projection, whose swapped tiles issue four MMAs per 64-column stage
-// with two weight matrices, got slower at every tail size (3.82-4.53 vs 3.41-3.43 ms).  Returns
+// with two weight matrices, got slower at every tail size (3.82-4.53 vs 3.41-3.43 ms).  With a long
+// reduction the swapped tile gains nothing either: on Mixtral-like segments (d_ff = 14336) the down
+// projection took 1.4-1.7 % longer with it, so the host turns it on only for d_ff <= 4096.  Returns
 // N, or 0 for a tile computed the usual way.
 __device__ __forceinline__ int swapped_cols(const TileCoord& c, const GemmArgs& g) {
     const int r = c.row_end - c.row0;
