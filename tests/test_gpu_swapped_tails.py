@@ -1,10 +1,11 @@
 """The grouped expert GEMMs on segments whose last row tile is short.
 
-A segment's last 128-row tile with at most 96 rows is computed with the operands swapped (the
-weight tile as the 128-row operand, the tile's rows as the narrow one).  These cases put every
-kind of tail next to each other -- 1, 15, 16, 17, 33, 64, 95, 96 rows (swapped), 97, 127, 128 rows
-(not), whole tiles followed by a short tail, an empty segment -- with output widths that end on a
-partial column tile, and compare Hp and Yp with the oracle's expert FFN ("5.3 Expert
+In the down projection with d_ff <= 4096, a segment's last 128-row tile with at most 32 rows is
+computed with the operands swapped (the weight tile as the 128-row operand, the tile's rows as the
+narrow one).  These cases put every kind of tail next to each other -- 1, 15, 16, 17 rows
+(swapped), 33, 64, 95, 96, 97, 127, 128 rows (not), whole tiles followed by a short tail, an empty
+segment -- with output widths that end on a partial column tile and d_ff on both sides of 4096,
+and compare Hp and Yp with the oracle's expert FFN ("5.3 Expert
 Parallelism", section "3. 고도화된 최적화: 오버래핑(Overlapping) 및 GroupGEMM": one grouped GEMM
 over every expert's rows)."""
 from types import SimpleNamespace
@@ -34,7 +35,8 @@ SEGMENTS = {
 }
 
 
-@pytest.mark.parametrize("d,F", [(512, 384), (384, 320), (256, 128)])
+# d_ff = 4096 is the longest reduction that takes the swapped tails, 4160 the shortest that does not
+@pytest.mark.parametrize("d,F", [(512, 384), (384, 320), (256, 128), (256, 4096), (256, 4160)])
 @pytest.mark.parametrize("layout", sorted(SEGMENTS))
 def test_expert_ffn_with_short_segment_tails(layout, d, F):
     lengths = SEGMENTS[layout]
