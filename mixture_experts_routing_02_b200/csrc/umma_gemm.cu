@@ -316,6 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             const uint32_t idesc = umma_idesc_bf16(kBM, g.mma_n);
+            // stage s's descriptors are stage 0's plus s stages (the address field counts 16-byte units)
+            const uint64_t adesc_0 = umma_desc_sw128(smem_u32(sA));
+            const uint64_t bdesc_0 = umma_desc_sw128(smem_u32(sB));
             bool ok = true;
             int seq = 0;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++seq) {
@@ -343,9 +346,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kb = kb0; kb < kb1; ++kb) {
                         if (!mbar_wait(&full_bar[stage], phase, &abort_sh, g.status)) { ok = false; break; }
                         tc_fence_after();
-                        const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * kABytes));
-                        const uint64_t wdesc0 = umma_desc_sw128(smem_u32(sB + stage * b_stage_bytes));
-                        const uint64_t wdesc1 = umma_desc_sw128(smem_u32(sB + stage * b_stage_bytes + 128 * 128));
+                        const uint64_t adesc = adesc_0 + static_cast<uint64_t>(stage) * (kABytes >> 4);
+                        const uint64_t wdesc0 = bdesc_0 + static_cast<uint64_t>(stage) * (b_stage_bytes >> 4);
+                        const uint64_t wdesc1 = wdesc0 + ((128u * 128u) >> 4);  // weight rows [128, 256)
 #pragma unroll
                         for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                             const uint32_t accum = (kb != kb0 || kk != 0) ? 1u : 0u;
@@ -359,8 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kb = kb0; kb < kb1; ++kb) {
                         if (!mbar_wait(&full_bar[stage], phase, &abort_sh, g.status)) { ok = false; break; }
                         tc_fence_after();
-                        const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * kABytes));
-                        const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * b_stage_bytes));
+                        const uint64_t adesc = adesc_0 + static_cast<uint64_t>(stage) * (kABytes >> 4);
+                        const uint64_t bdesc = bdesc_0 + static_cast<uint64_t>(stage) * (b_stage_bytes >> 4);
 #pragma unroll
                         for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                             // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4)
